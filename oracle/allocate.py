@@ -1,0 +1,130 @@
+"""Budgeted per-expert precision: the exact solution of PagedWeight's allocation problem.
+
+PagedWeight, "Quality-Aware Quantization": choose b_e to minimise
+sum_e p_e * L(b_e) subject to sum_e b_e * W_e <= B, where p_e is the expert's
+average routing probability and W_e its number of weight elements. The bit
+widths available are {3, 4, 8} (PagedWeight, "Code Illustration", bit_options).
+
+Readings taken where the page is open (each listed in the design doc):
+* L(b) is the mean squared error of a uniform symmetric quantizer whose step
+  is proportional to 1/q_b, q_b = 2^(b-1) - 1, so L(b) = 1 / q_b^2 (the page
+  says "e.g., mean squared error"; the allocator receives no weights, so the
+  loss is expert-independent up to p_e).
+* B counts bits of codes only (scales and page slack are not counted), as in
+  the page's constraint.
+* The problem is solved exactly (dynamic program), not by the page's
+  simplified proportional illustration.
+
+Dynamic program (units of g = gcd(W_e)): R = floor((B - 3*sum W) / g) budget
+units may be spent on upgrades; upgrading expert e from 3 to 4 bits costs
+W_e/g units, from 3 to 8 bits 5*W_e/g. D_e[r] is the least objective over the
+first e experts that spend exactly r units. Options are tried in the order
+3, 4, 8 and replace the incumbent only when strictly smaller (ties keep the
+lower width). The answer is argmin_r D_E[r] (ties: smallest r), then a
+backtrack. Costs are p_e * L(b) (one float64 multiply) added to D_{e-1}
+(one float64 add), with no fused multiply-add.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+BIT_OPTIONS = (3, 4, 8)
+
+
+class Infeasible(ValueError):
+    """B < 3 * sum_e W_e: even all-3-bit experts exceed the budget."""
+
+
+class StateCapExceeded(ValueError):
+    """The budget, in units of gcd(W_e), needs more DP states than the cap allows."""
+
+
+def q_levels(b: int) -> int:
+    """q_b = 2^(b-1) - 1, the largest code magnitude at b bits."""
+    return (1 << (b - 1)) - 1
+
+
+def loss(b: int) -> float:
+    """L(b) = 1 / q_b^2 in float64."""
+    q = q_levels(b)
+    return 1.0 / float(q * q)
+
+
+def allocate_bits(p, W, B: int, state_cap: int = 1 << 22) -> np.ndarray:
+    """b_e in {3,4,8} minimising sum p_e L(b_e) under sum b_e W_e <= B.
+
+    p: float64[E] importances; W: int[E] weight elements (> 0); B: budget in bits.
+    Returns uint8[E]. Raises Infeasible or StateCapExceeded.
+    """
+    p = np.asarray(p, dtype=np.float64)
+    W = [int(w) for w in W]
+    E = len(W)
+    if E == 0 or len(p) != E or any(w <= 0 for w in W):
+        raise ValueError("need E > 0 experts with W_e > 0 and one p_e each")
+    B = int(B)
+    sum_w = sum(W)
+    if B < 3 * sum_w:
+        raise Infeasible(f"B={B} < 3*sum(W)={3 * sum_w}")
+    if B >= 8 * sum_w:
+        return np.full(E, 8, dtype=np.uint8)
+    g = 0
+    for w in W:
+        g = math.gcd(g, w)
+    up = [{3: 0, 4: w // g, 8: 5 * w // g} for w in W]
+    R = (B - 3 * sum_w) // g
+    R = min(R, sum(u[8] for u in up))
+    if R + 1 > state_cap:
+        raise StateCapExceeded(f"{R + 1} states > cap {state_cap}")
+
+    L = {b: loss(b) for b in BIT_OPTIONS}
+    inf = math.inf
+    D = [0.0] + [inf] * R
+    choice = np.zeros((E, R + 1), dtype=np.uint8)
+    for e in range(E):
+        Dn = [inf] * (R + 1)
+        for r in range(R + 1):
+            best = inf
+            best_b = 0
+            for b in BIT_OPTIONS:
+                rp = r - up[e][b]
+                if rp < 0:
+                    continue
+                prev = D[rp]
+                if prev == inf:
+                    continue
+                cost = p[e] * L[b]          # float64 multiply
+                cand = prev + cost          # float64 add
+                if cand < best:
+                    best = cand
+                    best_b = b
+            Dn[r] = best
+            choice[e, r] = best_b
+        D = Dn
+
+    r_best = 0
+    for r in range(1, R + 1):
+        if D[r] < D[r_best]:
+            r_best = r
+    bits = np.zeros(E, dtype=np.uint8)
+    r = r_best
+    for e in range(E - 1, -1, -1):
+        b = int(choice[e, r])
+        assert b in BIT_OPTIONS
+        bits[e] = b
+        r -= up[e][b]
+    assert r == 0
+    return bits
+
+
+def objective(p, bits) -> float:
+    """sum_e p_e L(b_e), accumulated in ascending e with float64 multiply then add."""
+    total = 0.0
+    for pe, b in zip(np.asarray(p, dtype=np.float64), bits):
+        total = total + pe * loss(int(b))
+    return total
+
+
+def budget_used(W, bits) -> int:
+    return sum(int(w) * int(b) for w, b in zip(W, bits))

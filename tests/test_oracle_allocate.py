@@ -1,0 +1,131 @@
+"""Pins for oracle.allocate (PagedWeight, "Quality-Aware Quantization").
+
+The dynamic program is checked against exhaustive search over all 3^E width
+assignments (a different algorithm that evaluates the page's objective and
+constraint directly), against the special cases the constraint fixes, and
+against the exchange property of the optimum for equal-size experts.
+"""
+import itertools
+import math
+
+import numpy as np
+import pytest
+
+from oracle import allocate as A
+
+
+def brute_force(p, W, B):
+    """Exhaustive min of sum p_e L(b_e) over {3,4,8}^E with sum b_e W_e <= B.
+
+    The objective is accumulated in ascending e (same float64 order as the DP),
+    so the optimal value compares exactly. Returns (best value, all optimal
+    assignments)."""
+    Ls = {b: 1.0 / float(((1 << (b - 1)) - 1) ** 2) for b in (3, 4, 8)}
+    best, arg = math.inf, []
+    for bits in itertools.product((3, 4, 8), repeat=len(W)):
+        if sum(b * w for b, w in zip(bits, W)) > B:
+            continue
+        v = 0.0
+        for pe, b in zip(p, bits):
+            v = v + pe * Ls[b]
+        if v < best:
+            best, arg = v, [bits]
+        elif v == best:
+            arg.append(bits)
+    return best, arg
+
+
+def test_loss_values():
+    # L(b) = 1/q_b^2, q_b = 2^(b-1)-1: q = 3, 7, 127
+    assert A.q_levels(3) == 3 and A.q_levels(4) == 7 and A.q_levels(8) == 127
+    assert A.loss(3) == 1.0 / 9.0
+    assert A.loss(4) == 1.0 / 49.0
+    assert A.loss(8) == 1.0 / 16129.0
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_dp_matches_brute_force_equal_W(seed):
+    rng = np.random.default_rng(seed)
+    E = int(rng.integers(1, 9))
+    p = rng.dirichlet(np.full(E, 0.7))
+    W = [393216] * E
+    sw = sum(W)
+    B = int(rng.integers(3 * sw, 8 * sw + 1))
+    bits = A.allocate_bits(p, W, B)
+    best, args = brute_force(p, W, B)
+    assert A.objective(p, bits) == best
+    assert tuple(int(b) for b in bits) in args
+    assert A.budget_used(W, bits) <= B
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_dp_matches_brute_force_unequal_W(seed):
+    rng = np.random.default_rng(100 + seed)
+    E = int(rng.integers(1, 8))
+    p = rng.dirichlet(np.full(E, 1.0))
+    W = [int(x) * 64 for x in rng.integers(1, 40, size=E)]
+    sw = sum(W)
+    B = int(rng.integers(3 * sw, 8 * sw + 1))
+    bits = A.allocate_bits(p, W, B)
+    best, args = brute_force(p, W, B)
+    assert A.objective(p, bits) == best
+    assert tuple(int(b) for b in bits) in args
+
+
+def test_tiny_layer_budget_brute_force():
+    # 8 experts of 3*256*512 weights at 4.5 bits average: 3^8 = 6561 assignments
+    rng = np.random.default_rng(7)
+    p = rng.dirichlet(np.ones(8))
+    W = [3 * 256 * 512] * 8
+    B = int(math.floor(4.5 * sum(W)))
+    bits = A.allocate_bits(p, W, B)
+    best, args = brute_force(p, W, B)
+    assert A.objective(p, bits) == best and tuple(int(b) for b in bits) in args
+    assert len(set(int(b) for b in bits)) >= 2  # a mixed allocation
+
+
+def test_special_cases():
+    p = np.array([0.5, 0.3, 0.2])
+    W = [100, 200, 300]
+    sw = sum(W)
+    assert list(A.allocate_bits(p, W, 3 * sw)) == [3, 3, 3]
+    assert list(A.allocate_bits(p, W, 8 * sw)) == [8, 8, 8]
+    assert list(A.allocate_bits(p, W, 10 * sw)) == [8, 8, 8]
+    with pytest.raises(A.Infeasible):
+        A.allocate_bits(p, W, 3 * sw - 1)
+
+
+def test_single_expert_takes_widest_that_fits():
+    W = [1000]
+    assert list(A.allocate_bits([1.0], W, 3999)) == [3]
+    assert list(A.allocate_bits([1.0], W, 4000)) == [4]
+    assert list(A.allocate_bits([1.0], W, 7999)) == [4]
+    assert list(A.allocate_bits([1.0], W, 8000)) == [8]
+
+
+def test_zero_importance_gets_lowest_width():
+    # an expert with p_e = 0 gains nothing from bits: ties keep 3 bits
+    bits = A.allocate_bits([0.0, 1.0], [10, 10], 8 * 20 - 1)
+    assert list(bits) == [3, 8]
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_exchange_property_equal_W(seed):
+    # for equal W_e, swapping widths between i and j keeps the budget; an optimum
+    # therefore never gives the more important expert fewer bits
+    rng = np.random.default_rng(200 + seed)
+    E = 64
+    p = rng.dirichlet(np.full(E, 0.5))
+    W = [4718592] * E
+    B = int(math.floor(3.5 * sum(W)))
+    bits = A.allocate_bits(p, W, B)
+    assert A.budget_used(W, bits) <= B
+    for i in range(E):
+        for j in range(E):
+            if p[i] > p[j]:
+                assert bits[i] >= bits[j]
+
+
+def test_state_cap():
+    with pytest.raises(A.StateCapExceeded):
+        A.allocate_bits([0.5, 0.5], [1, 2], 3 * 3 + 10, state_cap=4)
