@@ -1,0 +1,252 @@
+/*
+ * mpe.h -- mixed-precision MoE experts served from paged 3/4/8-bit weights.
+ *
+ * C ABI of libmpe.so. Plain pointers and sizes only; every array argument
+ * states whether it lives in host or device memory. All device work runs in
+ * the library's CUDA kernels (sm_100a) on the context's stream.
+ *
+ * The operations follow the PagedWeight method ("PagedWeight: Efficient MoE
+ * LLM Serving with Dynamic Quality-Aware Weight Quantization", llmdb.app
+ * summary page):
+ *   - allocate precision per expert under a weight budget B
+ *     ("Quality-Aware Quantization": min sum_e p_e L(b_e) s.t. sum_e b_e W_e <= B);
+ *   - quantize each expert with one absmax scale and store it in pages of its
+ *     bit width, reached through a page table keyed by expert ID
+ *     ("Implementation Details": Q(w) = round(w/s) s, s = max|w|/(2^(b-1)-1);
+ *     memory management via a page table; "Dynamic Paging": pages of 8/4/3 bits);
+ *   - run the routed expert FFN straight from those pages, dequantizing on the
+ *     fly ("Dynamic Paging": the router picks experts, their pages are fetched
+ *     and dequantized on the fly);
+ *   - re-quantize when the budget changes with KV-cache occupancy ("Implementation
+ *     Details": the scheduler adjusts page sizes with KV-cache occupancy).
+ *
+ * Error behaviour: every int-returning call returns MPE_OK (0) or a negative
+ * MPE_ERR_* code; a human-readable message is kept per context (mpe_last_error)
+ * or per thread for calls without a context. No call exits, throws or traps.
+ * Device-side faults that kernels detect (an out-of-range expert id, NaN/Inf
+ * in a master, a bounded wait that ran out) set bits of a sticky status word
+ * read by mpe_get_status; kernels skip the offending work instead of faulting.
+ *
+ * Thread safety: a context may be used by one host thread at a time.
+ */
+#ifndef MPE_H
+#define MPE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- return codes ------------------------------------------------------ */
+#define MPE_OK               0
+#define MPE_ERR_INVALID     -1  /* bad argument: null pointer, size or alignment      */
+#define MPE_ERR_INFEASIBLE  -2  /* B < 3 * sum_e W_e                                  */
+#define MPE_ERR_STATE_CAP   -3  /* budget needs more allocation states than the cap   */
+#define MPE_ERR_POOL        -4  /* page pool exhausted; nothing was changed           */
+#define MPE_ERR_CUDA        -5  /* a CUDA runtime call failed (message has details)   */
+#define MPE_ERR_ORDER       -6  /* call out of order, e.g. moe_ffn before quantize    */
+#define MPE_ERR_DEVICE      -7  /* a kernel reported a problem: see mpe_get_status    */
+
+/* ---- sticky device status bits (mpe_get_status) ------------------------ */
+#define MPE_STATUS_BAD_EXPERT_ID   0x1u  /* an id outside [0, E): that slot was dropped */
+#define MPE_STATUS_NONFINITE       0x2u  /* a master holds NaN/Inf: expert not encoded  */
+#define MPE_STATUS_WAIT_TIMEOUT    0x4u  /* a bounded device wait gave up               */
+#define MPE_STATUS_ALLOC_INFEASIBLE 0x8u /* allocator kernel: B < 3 * sum W             */
+#define MPE_STATUS_ALLOC_STATE_CAP 0x10u /* allocator kernel: too many states           */
+
+/* ---- limits ------------------------------------------------------------- */
+#define MPE_MAX_EXPERTS        1024  /* E                                               */
+#define MPE_ALLOC_STATE_CAP    65536 /* allocator DP states (budget units + 1)          */
+#define MPE_DEFAULT_PAGE_BYTES 65536
+
+/* ---- forward-pass path selection --------------------------------------- */
+#define MPE_PATH_AUTO    0   /* decode kernels for small token counts, prefill above */
+#define MPE_PATH_DECODE  1   /* force the grouped GEMV (mma.sync) path              */
+#define MPE_PATH_PREFILL 2   /* force the tcgen05 grouped GEMM path                  */
+
+/*
+ * Layer shape and resources. E experts, each a SwiGLU FFN with gate W1 [F x H],
+ * up W3 [F x H] and down W2 [H x F] (row = output feature, K contiguous).
+ * H and F must be multiples of 128.
+ */
+typedef struct mpe_config {
+    int32_t  E;            /* experts, 1 .. MPE_MAX_EXPERTS                                 */
+    int32_t  H;            /* hidden size, multiple of 128                                  */
+    int32_t  F;            /* expert FFN size, multiple of 128                              */
+    uint32_t page_bytes;   /* physical page size; 0 = 65536; multiple of 4096, >= 4096      */
+    uint32_t pool_pages;   /* pages in the pool; 0 = enough for every expert at 8 bits      */
+    int32_t  device;       /* CUDA device ordinal; -1 = the current device                  */
+    int32_t  path;         /* MPE_PATH_*                                                    */
+    int32_t  reserved;
+    void*    stream;       /* cudaStream_t for all work; NULL = the legacy default stream   */
+} mpe_config;
+
+/* One page-table entry: expert e's pages are page_idx[first .. first+n_pages). */
+typedef struct mpe_pte {
+    uint8_t  bits;         /* 3, 4 or 8; 0 = not quantized yet   */
+    uint8_t  pad[3];
+    float    scale;        /* s_e = RN_f32(max|w| / (2^(b-1)-1)) */
+    uint32_t first;        /* index into the page-index array    */
+    uint32_t n_pages;      /* pages held by the expert           */
+} mpe_pte;
+
+typedef struct mpe_ctx mpe_ctx;
+
+/*
+ * mpe_create -- make a context: device page pool, page table, caches and
+ * scratch, all owned by the library. *out receives the context (host pointer).
+ * Returns MPE_ERR_INVALID for a bad shape, MPE_ERR_CUDA if allocation fails.
+ */
+int mpe_create(mpe_ctx** out, const mpe_config* cfg);
+
+/* mpe_destroy -- synchronise the context's stream and free everything it owns. */
+void mpe_destroy(mpe_ctx* ctx);
+
+/* mpe_set_stream -- run later work on `stream` (a cudaStream_t; NULL = default). */
+int mpe_set_stream(mpe_ctx* ctx, void* stream);
+
+/* mpe_set_path -- choose the forward-pass path (MPE_PATH_*). */
+int mpe_set_path(mpe_ctx* ctx, int32_t path);
+
+/*
+ * mpe_allocate_bits -- PagedWeight's allocation problem
+ * ("Quality-Aware Quantization"): choose b_e in {3,4,8} minimising
+ * sum_e p_e L(b_e) subject to sum_e b_e W_e <= B_bits, L(b) = 1/(2^(b-1)-1)^2,
+ * solved exactly by a dynamic program in one device kernel on the current
+ * device. Ties keep the lower width and the lower budget.
+ *   p        host, float64[E], importances
+ *   W        host, uint64[E], weight elements per expert (> 0)
+ *   E        1 .. MPE_MAX_EXPERTS
+ *   B_bits   budget in bits of codes
+ *   bits_out host, uint8[E], receives b_e
+ * Synchronous. MPE_ERR_INFEASIBLE if B_bits < 3 sum W; MPE_ERR_STATE_CAP if
+ * (B_bits - 3 sum W) / gcd(W) + 1 exceeds MPE_ALLOC_STATE_CAP.
+ */
+int mpe_allocate_bits(const double* p, const uint64_t* W, int32_t E, uint64_t B_bits,
+                      uint8_t* bits_out);
+
+/*
+ * mpe_quantize_experts -- quantize every expert at the given widths
+ * ("Implementation Details", quantization scheme): per-expert absmax m_e
+ * (cached: the master must not change while the context lives), scale
+ * s_e = RN_f32(m_e / (2^(b-1)-1)), codes k = round-half-even(w / s_e) clamped
+ * to +-(2^(b-1)-1), stored offset-binary in chunks of 16 rows x 128 codes,
+ * placed in the pool's pages (lowest free page first, experts ascending) and
+ * recorded in the page table.
+ *   master_f16 host array of E device pointers; expert e's fp16 master is
+ *              W1 [F x H] | W3 [F x H] | W2 [H x F], row-major, contiguous,
+ *              16-byte aligned. Borrowed: it must outlive the context
+ *              (mpe_repage re-reads it).
+ *   bits       host, uint8[E], each 3, 4 or 8.
+ * Asynchronous on the context stream (the page table is uploaded from
+ * context-owned host memory). A NaN/Inf master sets MPE_STATUS_NONFINITE.
+ * MPE_ERR_POOL if the pool is too small (nothing changes).
+ */
+int mpe_quantize_experts(mpe_ctx* ctx, const void* const* master_f16, const uint8_t* bits);
+
+/*
+ * mpe_repage -- budget change with KV-cache occupancy ("Implementation
+ * Details"; 0to1log digest: lower precision as the KV cache grows, raise it
+ * as it shrinks): re-run mpe_allocate_bits with B_bits and importances p
+ * (host float64[E]), release the pages of experts whose width changed, give
+ * them new pages and re-encode only those experts from the fp16 master with
+ * the cached absmax. *n_changed_out (host, may be NULL) receives the count.
+ * Synchronises once (the new widths decide the page moves); the encode is
+ * asynchronous. MPE_ERR_POOL leaves widths, pages and codes unchanged.
+ */
+int mpe_repage(mpe_ctx* ctx, uint64_t B_bits, const double* p, int32_t* n_changed_out);
+
+/*
+ * mpe_moe_ffn -- the routed expert SwiGLU FFN run from the pages ("Dynamic
+ * Paging"): bucket the T*k (token, slot) assignments by expert, then for each
+ * expert with tokens, stream its pages through the page table, unpack and
+ * dequantize in registers, and compute g = s W1 x, v = s W3 x,
+ * h = silu(g) v (rounded to bf16), y = s W2 h with fp32 accumulation;
+ * out[t] = bf16(sum_j w[t,j] y_{t,j}), summed in fp32.
+ *   x    device, bf16 [T x H], 16-byte aligned rows
+ *   T    tokens (>= 0)
+ *   ids  device, int32 [T x k]; ids outside [0,E) are dropped and set
+ *        MPE_STATUS_BAD_EXPERT_ID
+ *   w    device, float32 [T x k] top-k weights
+ *   k    1 .. 32
+ *   out  device, bf16 [T x H]
+ * Asynchronous on the context stream; scratch grows on demand (that call
+ * synchronises).
+ */
+int mpe_moe_ffn(mpe_ctx* ctx, const void* x, int32_t T, const int32_t* ids, const float* w,
+                int32_t k, void* out);
+
+/*
+ * mpe_moe_ffn_host -- mpe_moe_ffn with HOST buffers (preferably pinned):
+ * copies x, ids and w to context-owned device staging, runs the layer and
+ * copies out back, then synchronises. Same shapes as mpe_moe_ffn.
+ */
+int mpe_moe_ffn_host(mpe_ctx* ctx, const void* x_host, int32_t T, const int32_t* ids_host,
+                     const float* w_host, int32_t k, void* out_host);
+
+/*
+ * mpe_route -- the bucketing step alone (for inspection): perm = the
+ * assignments a = t*k + j sorted stably by expert id, offsets[E+1] = exclusive
+ * prefix sums of the per-expert counts, inv[a] = position of a in perm (-1 for
+ * dropped ids). Device pointers: ids int32 [T*k], perm int32 [T*k],
+ * offsets int32 [E+1], inv int32 [T*k]. Asynchronous.
+ */
+int mpe_route(mpe_ctx* ctx, const int32_t* ids, int32_t T, int32_t k, int32_t* perm,
+              int32_t* offsets, int32_t* inv);
+
+/*
+ * mpe_get_page_table -- copy the page table to host: pte_host mpe_pte[E] and
+ * page_idx_host uint32[cap] (the compact page-index array; its length is the
+ * sum of n_pages). Either pointer may be NULL. Synchronous.
+ * MPE_ERR_INVALID if cap is smaller than the array.
+ */
+int mpe_get_page_table(mpe_ctx* ctx, mpe_pte* pte_host, uint32_t* page_idx_host, size_t cap);
+
+/*
+ * mpe_expert_stream_bytes -- bytes of expert e's chunk stream at its current
+ * width (b * W_e / 8); 0 if not quantized.
+ */
+size_t mpe_expert_stream_bytes(mpe_ctx* ctx, int32_t e);
+
+/*
+ * mpe_read_expert_packed -- gather expert e's chunk stream (W1, W3, W2 chunks
+ * in stream order) out of its pages into host_dst (bytes >= the stream size).
+ * Synchronous.
+ */
+int mpe_read_expert_packed(mpe_ctx* ctx, int32_t e, void* host_dst, size_t bytes);
+
+/*
+ * mpe_get_scales -- host float32[E] scales and float32[E] absmax values
+ * (either may be NULL). Synchronous.
+ */
+int mpe_get_scales(mpe_ctx* ctx, float* scale_host, float* absmax_host);
+
+/* mpe_get_bits -- host uint8[E] current widths (0 = not quantized). */
+int mpe_get_bits(mpe_ctx* ctx, uint8_t* bits_host);
+
+/*
+ * mpe_get_status -- synchronise the stream and return the sticky device
+ * status word (MPE_STATUS_* bits) in *status_out; clear it if `clear` != 0.
+ */
+int mpe_get_status(mpe_ctx* ctx, uint32_t* status_out, int32_t clear);
+
+/* mpe_last_error -- message for the context's last failure ("" if none). */
+const char* mpe_last_error(mpe_ctx* ctx);
+
+/* mpe_last_error_global -- message for the calling thread's last failure of a
+ * context-free call (mpe_allocate_bits, mpe_create). */
+const char* mpe_last_error_global(void);
+
+/* mpe_kernel_launches -- how many kernels this context has launched so far. */
+uint64_t mpe_kernel_launches(mpe_ctx* ctx);
+
+/* mpe_version -- library version, e.g. 100 for 0.1.0. */
+int32_t mpe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MPE_H */

@@ -1,0 +1,599 @@
+// C ABI of libmpe: context, page allocator, page table and the call sequence
+// of each entry point (see include/mpe.h for the contract of every call).
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <numeric>
+
+#include "internal.h"
+
+namespace mpe {
+void route_set_smem_limits();
+void decode_set_smem_limits();
+}  // namespace mpe
+
+using namespace mpe;
+
+namespace {
+
+thread_local std::string g_err;
+
+int fail_global(int code, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return code;
+}
+
+int fail(mpe_ctx* c, int code, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    if (c) c->err = buf;
+    g_err = buf;
+    return code;
+}
+
+#define CK(call)                                                                           \
+    do {                                                                                   \
+        cudaError_t e_ = (call);                                                           \
+        if (e_ != cudaSuccess)                                                             \
+            return fail(c, MPE_ERR_CUDA, "%s failed: %s", #call, cudaGetErrorString(e_)); \
+    } while (0)
+
+#define CKLAUNCH()                                                                         \
+    do {                                                                                   \
+        cudaError_t e_ = cudaGetLastError();                                               \
+        if (e_ != cudaSuccess)                                                             \
+            return fail(c, MPE_ERR_CUDA, "kernel launch failed: %s", cudaGetErrorString(e_)); \
+    } while (0)
+
+// Make the context's device current for the duration of a call.
+struct DeviceGuard {
+    int prev = -1;
+    explicit DeviceGuard(int dev) {
+        cudaGetDevice(&prev);
+        if (prev != dev) cudaSetDevice(dev);
+    }
+    ~DeviceGuard() {
+        int cur = -1;
+        cudaGetDevice(&cur);
+        if (prev >= 0 && cur != prev) cudaSetDevice(prev);
+    }
+};
+
+int pages_needed(int b, int H, int F, uint32_t page_bytes) {
+    const int nc = 3 * chunks_w1(H, F);
+    const int cpp = chunks_per_page(b, page_bytes);
+    return (nc + cpp - 1) / cpp;
+}
+
+bool valid_bits(int b) { return b == 3 || b == 4 || b == 8; }
+
+// Lowest-index-first page moves for the experts whose width changes.
+// Transactional: on shortage, returns false and leaves `a` untouched.
+bool plan_pages(const mpe_ctx* c, const std::vector<uint8_t>& new_bits, HostAllocator& a,
+                std::vector<int>& changed) {
+    HostAllocator n = c->alloc;
+    changed.clear();
+    for (int e = 0; e < c->E; ++e)
+        if (new_bits[e] != c->bits[e]) changed.push_back(e);
+    for (int e : changed) {
+        for (uint32_t p : n.pages[e]) n.free[p] = 1;
+        n.pages[e].clear();
+    }
+    uint32_t cursor = 0;
+    for (int e : changed) {
+        const int need = pages_needed(new_bits[e], c->H, c->F, c->page_bytes);
+        for (int i = 0; i < need; ++i) {
+            while (cursor < c->pool_pages && !n.free[cursor]) ++cursor;
+            if (cursor >= c->pool_pages) return false;
+            n.free[cursor] = 0;
+            n.pages[e].push_back(cursor);
+        }
+    }
+    a = std::move(n);
+    return true;
+}
+
+// Rebuild the host page table from the allocator and upload it (async, from
+// pinned staging that is reused only after the previous upload finished).
+int upload_table(mpe_ctx* c) {
+    c->pidx.clear();
+    for (int e = 0; e < c->E; ++e) {
+        Pte& p = c->pte[e];
+        p.bits = c->bits[e];
+        p.first = (uint32_t)c->pidx.size();
+        p.n_pages = (uint32_t)c->alloc.pages[e].size();
+        c->pidx.insert(c->pidx.end(), c->alloc.pages[e].begin(), c->alloc.pages[e].end());
+    }
+    CK(cudaEventSynchronize(c->upload_done));
+    std::memcpy(c->h_pte_pinned, c->pte.data(), sizeof(Pte) * c->E);
+    if (!c->pidx.empty())
+        std::memcpy(c->h_pidx_pinned, c->pidx.data(), sizeof(uint32_t) * c->pidx.size());
+    CK(cudaMemcpyAsync(c->d_pte, c->h_pte_pinned, sizeof(Pte) * c->E, cudaMemcpyHostToDevice,
+                       c->stream));
+    if (!c->pidx.empty())
+        CK(cudaMemcpyAsync(c->d_pidx, c->h_pidx_pinned, sizeof(uint32_t) * c->pidx.size(),
+                           cudaMemcpyHostToDevice, c->stream));
+    CK(cudaEventRecord(c->upload_done, c->stream));
+    return MPE_OK;
+}
+
+int upload_list(mpe_ctx* c, const std::vector<int>& list) {
+    // the list staging is shared with the previous call: wait for its upload
+    CK(cudaEventSynchronize(c->upload_done));
+    for (size_t i = 0; i < list.size(); ++i) c->h_list_pinned[i] = list[i];
+    CK(cudaMemcpyAsync(c->d_list, c->h_list_pinned, sizeof(int32_t) * list.size(),
+                       cudaMemcpyHostToDevice, c->stream));
+    CK(cudaEventRecord(c->upload_done, c->stream));
+    return MPE_OK;
+}
+
+template <typename T>
+int dev_alloc(mpe_ctx* c, T** p, size_t n) {
+    *p = nullptr;
+    if (n == 0) n = 1;
+    CK(cudaMalloc(reinterpret_cast<void**>(p), n * sizeof(T)));
+    return MPE_OK;
+}
+
+void free_scratch(Scratch& s) {
+    cudaFree(s.perm); cudaFree(s.inv); cudaFree(s.offsets); cudaFree(s.wg); cudaFree(s.n_wg);
+    cudaFree(s.hist); cudaFree(s.h); cudaFree(s.y);
+    cudaFree(s.x_stage); cudaFree(s.ids_stage); cudaFree(s.w_stage); cudaFree(s.out_stage);
+    s = Scratch{};
+}
+
+int wg_capacity(int E, size_t Tk, int group) {
+    return (int)(std::min<size_t>((size_t)E, Tk) + Tk / group + 1);
+}
+
+int ensure_scratch(mpe_ctx* c, size_t Tk) {
+    Scratch& s = c->s;
+    if (Tk <= s.cap_assign && s.perm) return MPE_OK;
+    CK(cudaStreamSynchronize(c->stream));
+    const size_t stage_tokens = s.stage_tokens;
+    void* xs = s.x_stage; int32_t* is = s.ids_stage; float* ws = s.w_stage; void* os = s.out_stage;
+    s.x_stage = nullptr; s.ids_stage = nullptr; s.w_stage = nullptr; s.out_stage = nullptr;
+    free_scratch(s);
+    s.stage_tokens = stage_tokens; s.x_stage = xs; s.ids_stage = is; s.w_stage = ws; s.out_stage = os;
+    size_t cap = 1024;
+    while (cap < Tk) cap *= 2;
+    const int E = c->E;
+    int r;
+    if ((r = dev_alloc(c, &s.perm, cap))) return r;
+    if ((r = dev_alloc(c, &s.inv, cap))) return r;
+    if ((r = dev_alloc(c, &s.offsets, E + 1))) return r;
+    if ((r = dev_alloc(c, &s.wg, 3 * (size_t)wg_capacity(E, cap, 1)))) return r;
+    if ((r = dev_alloc(c, &s.n_wg, 1))) return r;
+    s.hist_cap = ((cap + 1023) / 1024) * E;
+    if ((r = dev_alloc(c, &s.hist, s.hist_cap))) return r;
+    if ((r = dev_alloc(c, &s.h, cap * c->F))) return r;
+    if ((r = dev_alloc(c, &s.y, cap * c->H))) return r;
+    s.cap_assign = cap;
+    return MPE_OK;
+}
+
+int ensure_stage(mpe_ctx* c, int T, int k) {
+    Scratch& s = c->s;
+    if ((size_t)T <= s.stage_tokens && s.x_stage && (size_t)T * k <= s.cap_assign) return MPE_OK;
+    CK(cudaStreamSynchronize(c->stream));
+    cudaFree(s.x_stage); cudaFree(s.ids_stage); cudaFree(s.w_stage); cudaFree(s.out_stage);
+    size_t cap = 64;
+    while (cap < (size_t)T) cap *= 2;
+    int r;
+    if ((r = dev_alloc(c, reinterpret_cast<__nv_bfloat16**>(&s.x_stage), cap * c->H))) return r;
+    if ((r = dev_alloc(c, reinterpret_cast<__nv_bfloat16**>(&s.out_stage), cap * c->H))) return r;
+    if ((r = dev_alloc(c, &s.ids_stage, cap * 32))) return r;
+    if ((r = dev_alloc(c, &s.w_stage, cap * 32))) return r;
+    s.stage_tokens = cap;
+    return MPE_OK;
+}
+
+// Run the allocator kernel on the context's stream and fetch the widths.
+int run_allocate(mpe_ctx* c, const double* p, uint64_t B, std::vector<uint8_t>& out) {
+    const int E = c->E;
+    for (int e = 0; e < E; ++e)
+        if (!(p[e] >= 0.0) || !std::isfinite(p[e]))
+            return fail(c, MPE_ERR_INVALID, "importance p[%d] must be finite and >= 0", e);
+    std::vector<uint64_t> W(E, (uint64_t)3 * c->H * c->F);
+    const uint64_t sum_w = W[0] * E;
+    if (B < 3 * sum_w) return fail(c, MPE_ERR_INFEASIBLE, "budget %llu < 3 * sum W = %llu",
+                                   (unsigned long long)B, (unsigned long long)(3 * sum_w));
+    const uint64_t g = W[0];
+    uint64_t R = B >= 8 * sum_w ? 0 : (B - 3 * sum_w) / g;
+    R = std::min<uint64_t>(R, 5 * (sum_w / g));
+    if (R + 1 > MPE_ALLOC_STATE_CAP) return fail(c, MPE_ERR_STATE_CAP, "too many states");
+    const size_t need = (size_t)E * (R + 1);
+    if (need > c->choice_cap) {
+        cudaFree(c->d_choice);
+        CK(cudaMalloc(&c->d_choice, need));
+        c->choice_cap = need;
+    }
+    CK(cudaMemcpyAsync(c->d_p, p, sizeof(double) * E, cudaMemcpyHostToDevice, c->stream));
+    CK(cudaMemcpyAsync(c->d_W, W.data(), sizeof(uint64_t) * E, cudaMemcpyHostToDevice,
+                       c->stream));
+    launch_allocate(c->stream, c->d_p, c->d_W, E, B, c->d_bits_out, c->d_alloc_status,
+                    c->d_choice, c->d_D, MPE_ALLOC_STATE_CAP);
+    c->launches++;
+    CKLAUNCH();
+    int32_t st = -1;
+    out.assign(E, 0);
+    CK(cudaMemcpyAsync(&st, c->d_alloc_status, sizeof(int32_t), cudaMemcpyDeviceToHost,
+                       c->stream));
+    CK(cudaMemcpyAsync(out.data(), c->d_bits_out, E, cudaMemcpyDeviceToHost, c->stream));
+    CK(cudaStreamSynchronize(c->stream));
+    if (st == 1) return fail(c, MPE_ERR_INFEASIBLE, "budget below 3 bits per weight");
+    if (st == 3) return fail(c, MPE_ERR_STATE_CAP, "too many allocation states");
+    return MPE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t mpe_version(void) { return 100; }
+
+const char* mpe_last_error_global(void) { return g_err.c_str(); }
+
+const char* mpe_last_error(mpe_ctx* c) { return c ? c->err.c_str() : g_err.c_str(); }
+
+uint64_t mpe_kernel_launches(mpe_ctx* c) { return c ? c->launches : 0; }
+
+int mpe_create(mpe_ctx** out, const mpe_config* cfg) {
+    if (!out || !cfg) return fail_global(MPE_ERR_INVALID, "null argument");
+    *out = nullptr;
+    if (cfg->E < 1 || cfg->E > MPE_MAX_EXPERTS)
+        return fail_global(MPE_ERR_INVALID, "E=%d out of range", cfg->E);
+    if (cfg->H <= 0 || cfg->F <= 0 || cfg->H % 128 || cfg->F % 128)
+        return fail_global(MPE_ERR_INVALID, "H and F must be positive multiples of 128");
+    const uint32_t pb = cfg->page_bytes ? cfg->page_bytes : MPE_DEFAULT_PAGE_BYTES;
+    if (pb < 4096 || pb % 4096)
+        return fail_global(MPE_ERR_INVALID, "page_bytes must be a multiple of 4096");
+    if (cfg->path < MPE_PATH_AUTO || cfg->path > MPE_PATH_PREFILL)
+        return fail_global(MPE_ERR_INVALID, "bad path");
+    int dev = cfg->device;
+    if (dev < 0 && cudaGetDevice(&dev) != cudaSuccess)
+        return fail_global(MPE_ERR_CUDA, "no CUDA device");
+    auto* c = new mpe_ctx();
+    c->device = dev;
+    DeviceGuard guard(dev);
+    c->E = cfg->E;
+    c->H = cfg->H;
+    c->F = cfg->F;
+    c->page_bytes = pb;
+    c->path = cfg->path;
+    c->stream = reinterpret_cast<cudaStream_t>(cfg->stream);
+    c->pool_pages = cfg->pool_pages ? cfg->pool_pages
+                                    : (uint32_t)(c->E * pages_needed(8, c->H, c->F, pb));
+    auto bail = [&](int r) {
+        mpe_destroy(c);
+        return r;
+    };
+    int r;
+    if (cudaMalloc(&c->pool, (size_t)c->pool_pages * pb) != cudaSuccess) {
+        cudaGetLastError();
+        delete c;
+        return fail_global(MPE_ERR_CUDA, "pool allocation of %zu bytes failed",
+                           (size_t)c->pool_pages * pb);
+    }
+    if ((r = dev_alloc(c, &c->d_pte, c->E))) return bail(r);
+    if ((r = dev_alloc(c, &c->d_pidx, c->pool_pages))) return bail(r);
+    if ((r = dev_alloc(c, &c->d_absmax, c->E))) return bail(r);
+    if ((r = dev_alloc(c, &c->d_status, 1))) return bail(r);
+    if ((r = dev_alloc(c, &c->d_masters, c->E))) return bail(r);
+    if ((r = dev_alloc(c, &c->d_list, c->E))) return bail(r);
+    if ((r = dev_alloc(c, &c->d_p, c->E))) return bail(r);
+    if ((r = dev_alloc(c, &c->d_W, c->E))) return bail(r);
+    if ((r = dev_alloc(c, &c->d_bits_out, c->E))) return bail(r);
+    if ((r = dev_alloc(c, &c->d_alloc_status, 1))) return bail(r);
+    if ((r = dev_alloc(c, &c->d_D, 2 * (size_t)MPE_ALLOC_STATE_CAP))) return bail(r);
+    if (cudaMallocHost(&c->h_pte_pinned, sizeof(Pte) * c->E) != cudaSuccess ||
+        cudaMallocHost(&c->h_pidx_pinned, sizeof(uint32_t) * c->pool_pages) != cudaSuccess ||
+        cudaMallocHost(&c->h_list_pinned, sizeof(int32_t) * c->E) != cudaSuccess ||
+        cudaMallocHost(&c->h_masters_pinned, sizeof(void*) * c->E) != cudaSuccess ||
+        cudaEventCreateWithFlags(&c->upload_done, cudaEventDisableTiming) != cudaSuccess)
+        return bail(fail_global(MPE_ERR_CUDA, "host staging allocation failed"));
+    if (cudaMemset(c->d_pte, 0, sizeof(Pte) * c->E) != cudaSuccess ||
+        cudaMemset(c->d_status, 0, sizeof(uint32_t)) != cudaSuccess ||
+        cudaEventRecord(c->upload_done, c->stream) != cudaSuccess)
+        return bail(fail_global(MPE_ERR_CUDA, "initialisation failed"));
+    c->bits.assign(c->E, 0);
+    c->pte.assign(c->E, Pte{});
+    c->masters.assign(c->E, nullptr);
+    c->alloc.free.assign(c->pool_pages, 1);
+    c->alloc.pages.assign(c->E, {});
+    route_set_smem_limits();
+    decode_set_smem_limits();
+    if (cudaGetLastError() != cudaSuccess)
+        return bail(fail_global(MPE_ERR_CUDA, "kernel attribute setup failed"));
+    *out = c;
+    return MPE_OK;
+}
+
+void mpe_destroy(mpe_ctx* c) {
+    if (!c) return;
+    {
+        DeviceGuard guard(c->device);
+        cudaStreamSynchronize(c->stream);
+        free_scratch(c->s);
+        cudaFree(c->pool); cudaFree(c->d_pte); cudaFree(c->d_pidx); cudaFree(c->d_absmax);
+        cudaFree(c->d_status); cudaFree(c->d_masters); cudaFree(c->d_list); cudaFree(c->d_p);
+        cudaFree(c->d_W); cudaFree(c->d_bits_out); cudaFree(c->d_alloc_status);
+        cudaFree(c->d_choice); cudaFree(c->d_D); cudaFree(c->d_gather);
+        cudaFreeHost(c->h_pte_pinned); cudaFreeHost(c->h_pidx_pinned);
+        cudaFreeHost(c->h_list_pinned); cudaFreeHost(c->h_masters_pinned);
+        if (c->upload_done) cudaEventDestroy(c->upload_done);
+        cudaGetLastError();
+    }
+    delete c;
+}
+
+int mpe_set_stream(mpe_ctx* c, void* stream) {
+    if (!c) return fail_global(MPE_ERR_INVALID, "null context");
+    c->stream = reinterpret_cast<cudaStream_t>(stream);
+    return MPE_OK;
+}
+
+int mpe_set_path(mpe_ctx* c, int32_t path) {
+    if (!c) return fail_global(MPE_ERR_INVALID, "null context");
+    if (path < MPE_PATH_AUTO || path > MPE_PATH_PREFILL) return fail(c, MPE_ERR_INVALID, "bad path");
+    c->path = path;
+    return MPE_OK;
+}
+
+int mpe_allocate_bits(const double* p, const uint64_t* W, int32_t E, uint64_t B_bits,
+                      uint8_t* bits_out) {
+    if (!p || !W || !bits_out) return fail_global(MPE_ERR_INVALID, "null argument");
+    if (E < 1 || E > MPE_MAX_EXPERTS) return fail_global(MPE_ERR_INVALID, "E out of range");
+    uint64_t sum_w = 0, g = 0;
+    for (int e = 0; e < E; ++e) {
+        if (W[e] == 0) return fail_global(MPE_ERR_INVALID, "W[%d] = 0", e);
+        if (!(p[e] >= 0.0) || !std::isfinite(p[e]))
+            return fail_global(MPE_ERR_INVALID, "p[%d] must be finite and >= 0", e);
+        sum_w += W[e];
+        g = std::gcd(g, W[e]);
+    }
+    if (B_bits < 3 * sum_w) return fail_global(MPE_ERR_INFEASIBLE, "budget below 3 bits per weight");
+    uint64_t R = B_bits >= 8 * sum_w ? 0 : (B_bits - 3 * sum_w) / g;
+    R = std::min<uint64_t>(R, 5 * (sum_w / g));
+    if (R + 1 > MPE_ALLOC_STATE_CAP) return fail_global(MPE_ERR_STATE_CAP, "too many states");
+    double* dp = nullptr; uint64_t* dW = nullptr; uint8_t* db = nullptr; int32_t* ds = nullptr;
+    uint8_t* dch = nullptr; double* dD = nullptr;
+    int rc = MPE_OK;
+    int32_t st = -1;
+    auto ok = [](cudaError_t e) { return e == cudaSuccess; };
+    if (!ok(cudaMalloc(&dp, sizeof(double) * E)) || !ok(cudaMalloc(&dW, sizeof(uint64_t) * E)) ||
+        !ok(cudaMalloc(&db, E)) || !ok(cudaMalloc(&ds, sizeof(int32_t))) ||
+        !ok(cudaMalloc(&dch, (size_t)E * (R + 1))) ||
+        !ok(cudaMalloc(&dD, 2 * sizeof(double) * (R + 1))) ||
+        !ok(cudaMemcpy(dp, p, sizeof(double) * E, cudaMemcpyHostToDevice)) ||
+        !ok(cudaMemcpy(dW, W, sizeof(uint64_t) * E, cudaMemcpyHostToDevice))) {
+        rc = fail_global(MPE_ERR_CUDA, "allocate_bits: %s", cudaGetErrorString(cudaGetLastError()));
+    } else {
+        launch_allocate(nullptr, dp, dW, E, B_bits, db, ds, dch, dD, MPE_ALLOC_STATE_CAP);
+        if (!ok(cudaGetLastError()) || !ok(cudaMemcpy(&st, ds, sizeof(int32_t), cudaMemcpyDeviceToHost)) ||
+            !ok(cudaMemcpy(bits_out, db, E, cudaMemcpyDeviceToHost)))
+            rc = fail_global(MPE_ERR_CUDA, "allocate_bits kernel: %s",
+                             cudaGetErrorString(cudaGetLastError()));
+        else if (st == 1)
+            rc = fail_global(MPE_ERR_INFEASIBLE, "budget below 3 bits per weight");
+        else if (st == 3)
+            rc = fail_global(MPE_ERR_STATE_CAP, "too many allocation states");
+    }
+    cudaFree(dp); cudaFree(dW); cudaFree(db); cudaFree(ds); cudaFree(dch); cudaFree(dD);
+    return rc;
+}
+
+int mpe_quantize_experts(mpe_ctx* c, const void* const* master_f16, const uint8_t* bits) {
+    if (!c) return fail_global(MPE_ERR_INVALID, "null context");
+    if (!master_f16 || !bits) return fail(c, MPE_ERR_INVALID, "null argument");
+    for (int e = 0; e < c->E; ++e) {
+        if (!valid_bits(bits[e])) return fail(c, MPE_ERR_INVALID, "bits[%d]=%d not 3/4/8", e, bits[e]);
+        if (!master_f16[e] || (reinterpret_cast<uintptr_t>(master_f16[e]) & 15))
+            return fail(c, MPE_ERR_INVALID, "master[%d] null or not 16-byte aligned", e);
+    }
+    DeviceGuard guard(c->device);
+    std::vector<uint8_t> nb(bits, bits + c->E);
+    HostAllocator na;
+    std::vector<int> changed;
+    if (!plan_pages(c, nb, na, changed)) return fail(c, MPE_ERR_POOL, "page pool exhausted");
+    c->alloc = std::move(na);
+    c->bits = nb;
+    int r;
+    if ((r = upload_table(c))) return r;
+    // master pointers and the all-experts list
+    CK(cudaEventSynchronize(c->upload_done));
+    for (int e = 0; e < c->E; ++e) {
+        c->masters[e] = master_f16[e];
+        c->h_masters_pinned[e] = master_f16[e];
+    }
+    CK(cudaMemcpyAsync(c->d_masters, c->h_masters_pinned, sizeof(void*) * c->E,
+                       cudaMemcpyHostToDevice, c->stream));
+    std::vector<int> all(c->E);
+    std::iota(all.begin(), all.end(), 0);
+    if ((r = upload_list(c, all))) return r;
+    CK(cudaMemsetAsync(c->d_absmax, 0, sizeof(uint32_t) * c->E, c->stream));
+    launch_absmax(c, c->d_list, c->E);
+    launch_scales(c);
+    launch_encode(c, c->d_list, c->E);
+    CKLAUNCH();
+    c->absmax_valid = true;
+    return MPE_OK;
+}
+
+int mpe_repage(mpe_ctx* c, uint64_t B_bits, const double* p, int32_t* n_changed_out) {
+    if (!c) return fail_global(MPE_ERR_INVALID, "null context");
+    if (!p) return fail(c, MPE_ERR_INVALID, "null importances");
+    if (!c->absmax_valid) return fail(c, MPE_ERR_ORDER, "repage before quantize_experts");
+    DeviceGuard guard(c->device);
+    std::vector<uint8_t> nb;
+    int r;
+    if ((r = run_allocate(c, p, B_bits, nb))) return r;
+    HostAllocator na;
+    std::vector<int> changed;
+    if (!plan_pages(c, nb, na, changed)) return fail(c, MPE_ERR_POOL, "page pool exhausted");
+    c->alloc = std::move(na);
+    c->bits = nb;
+    if ((r = upload_table(c))) return r;
+    launch_scales(c);
+    if (!changed.empty()) {
+        if ((r = upload_list(c, changed))) return r;
+        launch_encode(c, c->d_list, (int)changed.size());
+    }
+    CKLAUNCH();
+    if (n_changed_out) *n_changed_out = (int32_t)changed.size();
+    return MPE_OK;
+}
+
+static int moe_ffn_device(mpe_ctx* c, const void* x, int32_t T, const int32_t* ids,
+                          const float* w, int32_t k, void* out) {
+    const size_t Tk = (size_t)T * k;
+    int r;
+    if ((r = ensure_scratch(c, Tk))) return r;
+    launch_route(c, ids, (int)Tk, k, c->s.perm, c->s.offsets, c->s.inv, kDecodeGroup);
+    const int bound = wg_capacity(c->E, Tk, kDecodeGroup);
+    launch_decode_gateup(c, reinterpret_cast<const __nv_bfloat16*>(x), k, bound);
+    launch_decode_down(c, w, bound);
+    launch_combine(c, ids, T, k, reinterpret_cast<__nv_bfloat16*>(out));
+    CKLAUNCH();
+    return MPE_OK;
+}
+
+int mpe_moe_ffn(mpe_ctx* c, const void* x, int32_t T, const int32_t* ids, const float* w,
+                int32_t k, void* out) {
+    if (!c) return fail_global(MPE_ERR_INVALID, "null context");
+    if (T < 0 || k < 1 || k > 32) return fail(c, MPE_ERR_INVALID, "bad T=%d or k=%d", T, k);
+    if (T == 0) return MPE_OK;
+    if (!x || !ids || !w || !out) return fail(c, MPE_ERR_INVALID, "null argument");
+    if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(out)) & 15)
+        return fail(c, MPE_ERR_INVALID, "x and out must be 16-byte aligned");
+    if (!c->absmax_valid) return fail(c, MPE_ERR_ORDER, "moe_ffn before quantize_experts");
+    DeviceGuard guard(c->device);
+    return moe_ffn_device(c, x, T, ids, w, k, out);
+}
+
+int mpe_moe_ffn_host(mpe_ctx* c, const void* x_host, int32_t T, const int32_t* ids_host,
+                     const float* w_host, int32_t k, void* out_host) {
+    if (!c) return fail_global(MPE_ERR_INVALID, "null context");
+    if (T < 0 || k < 1 || k > 32) return fail(c, MPE_ERR_INVALID, "bad T=%d or k=%d", T, k);
+    if (T == 0) return MPE_OK;
+    if (!x_host || !ids_host || !w_host || !out_host) return fail(c, MPE_ERR_INVALID, "null argument");
+    if (!c->absmax_valid) return fail(c, MPE_ERR_ORDER, "moe_ffn before quantize_experts");
+    DeviceGuard guard(c->device);
+    int r;
+    if ((r = ensure_scratch(c, (size_t)T * k))) return r;
+    if ((r = ensure_stage(c, T, k))) return r;
+    Scratch& s = c->s;
+    const size_t xb = (size_t)T * c->H * 2;
+    CK(cudaMemcpyAsync(s.x_stage, x_host, xb, cudaMemcpyHostToDevice, c->stream));
+    CK(cudaMemcpyAsync(s.ids_stage, ids_host, (size_t)T * k * 4, cudaMemcpyHostToDevice, c->stream));
+    CK(cudaMemcpyAsync(s.w_stage, w_host, (size_t)T * k * 4, cudaMemcpyHostToDevice, c->stream));
+    if ((r = moe_ffn_device(c, s.x_stage, T, s.ids_stage, s.w_stage, k, s.out_stage))) return r;
+    CK(cudaMemcpyAsync(out_host, s.out_stage, xb, cudaMemcpyDeviceToHost, c->stream));
+    CK(cudaStreamSynchronize(c->stream));
+    return MPE_OK;
+}
+
+int mpe_route(mpe_ctx* c, const int32_t* ids, int32_t T, int32_t k, int32_t* perm,
+              int32_t* offsets, int32_t* inv) {
+    if (!c) return fail_global(MPE_ERR_INVALID, "null context");
+    if (T < 0 || k < 1 || k > 32) return fail(c, MPE_ERR_INVALID, "bad T or k");
+    if (!ids || !perm || !offsets || !inv) return fail(c, MPE_ERR_INVALID, "null argument");
+    DeviceGuard guard(c->device);
+    const size_t Tk = (size_t)T * k;
+    int r;
+    if ((r = ensure_scratch(c, Tk))) return r;
+    if (Tk == 0) {
+        CK(cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (c->E + 1), c->stream));
+        return MPE_OK;
+    }
+    launch_route(c, ids, (int)Tk, k, perm, offsets, inv, kDecodeGroup);
+    CKLAUNCH();
+    return MPE_OK;
+}
+
+int mpe_get_page_table(mpe_ctx* c, mpe_pte* pte_host, uint32_t* page_idx_host, size_t cap) {
+    if (!c) return fail_global(MPE_ERR_INVALID, "null context");
+    DeviceGuard guard(c->device);
+    CK(cudaStreamSynchronize(c->stream));
+    if (pte_host) CK(cudaMemcpy(pte_host, c->d_pte, sizeof(Pte) * c->E, cudaMemcpyDeviceToHost));
+    if (page_idx_host) {
+        if (cap < c->pidx.size()) return fail(c, MPE_ERR_INVALID, "cap %zu < %zu", cap, c->pidx.size());
+        if (!c->pidx.empty())
+            CK(cudaMemcpy(page_idx_host, c->d_pidx, sizeof(uint32_t) * c->pidx.size(),
+                          cudaMemcpyDeviceToHost));
+    }
+    return MPE_OK;
+}
+
+size_t mpe_expert_stream_bytes(mpe_ctx* c, int32_t e) {
+    if (!c || e < 0 || e >= c->E || !valid_bits(c->bits[e])) return 0;
+    return (size_t)3 * chunks_w1(c->H, c->F) * chunk_bytes(c->bits[e]);
+}
+
+int mpe_read_expert_packed(mpe_ctx* c, int32_t e, void* host_dst, size_t bytes) {
+    if (!c) return fail_global(MPE_ERR_INVALID, "null context");
+    if (e < 0 || e >= c->E || !host_dst) return fail(c, MPE_ERR_INVALID, "bad expert or buffer");
+    const size_t n = mpe_expert_stream_bytes(c, e);
+    if (n == 0) return fail(c, MPE_ERR_ORDER, "expert %d not quantized", e);
+    if (bytes < n) return fail(c, MPE_ERR_INVALID, "buffer %zu < stream %zu", bytes, n);
+    DeviceGuard guard(c->device);
+    if (n > c->gather_cap) {
+        CK(cudaStreamSynchronize(c->stream));
+        cudaFree(c->d_gather);
+        c->d_gather = nullptr;
+        CK(cudaMalloc(&c->d_gather, n));
+        c->gather_cap = n;
+    }
+    launch_gather_stream(c, e, c->d_gather);
+    CKLAUNCH();
+    CK(cudaMemcpyAsync(host_dst, c->d_gather, n, cudaMemcpyDeviceToHost, c->stream));
+    CK(cudaStreamSynchronize(c->stream));
+    return MPE_OK;
+}
+
+int mpe_get_scales(mpe_ctx* c, float* scale_host, float* absmax_host) {
+    if (!c) return fail_global(MPE_ERR_INVALID, "null context");
+    DeviceGuard guard(c->device);
+    CK(cudaStreamSynchronize(c->stream));
+    if (scale_host) {
+        std::vector<Pte> p(c->E);
+        CK(cudaMemcpy(p.data(), c->d_pte, sizeof(Pte) * c->E, cudaMemcpyDeviceToHost));
+        for (int e = 0; e < c->E; ++e) scale_host[e] = p[e].scale;
+    }
+    if (absmax_host) {
+        std::vector<uint32_t> m(c->E);
+        CK(cudaMemcpy(m.data(), c->d_absmax, sizeof(uint32_t) * c->E, cudaMemcpyDeviceToHost));
+        for (int e = 0; e < c->E; ++e) {
+            const __half h = __ushort_as_half((unsigned short)(m[e] & 0xFFFF));
+            absmax_host[e] = __half2float(h);
+        }
+    }
+    return MPE_OK;
+}
+
+int mpe_get_bits(mpe_ctx* c, uint8_t* bits_host) {
+    if (!c || !bits_host) return fail_global(MPE_ERR_INVALID, "null argument");
+    std::memcpy(bits_host, c->bits.data(), c->E);
+    return MPE_OK;
+}
+
+int mpe_get_status(mpe_ctx* c, uint32_t* status_out, int32_t clear) {
+    if (!c || !status_out) return fail_global(MPE_ERR_INVALID, "null argument");
+    DeviceGuard guard(c->device);
+    CK(cudaStreamSynchronize(c->stream));
+    CK(cudaMemcpy(status_out, c->d_status, sizeof(uint32_t), cudaMemcpyDeviceToHost));
+    if (clear) CK(cudaMemset(c->d_status, 0, sizeof(uint32_t)));
+    return MPE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,216 @@
+// Device-side building blocks shared by the mpe kernels (sm_100a).
+//
+// Packed format (the library's own definition of PagedWeight's "pages of
+// varying bit-widths"): a matrix [R x K] is cut into chunks of 16 rows x 128
+// codes; chunk (tau, j) holds the 16 blocks of rows 16 tau .. 16 tau + 15 at
+// block column j, 16 b bytes per block, rows in order. A block is four
+// quarters of 32 codes (4 b bytes each). Inside a quarter the 32 offset-binary
+// codes c'_0..c'_31 are b little-endian words:
+//   b = 8: word w holds c'_{4w+i} at bit 16(i&1) + 8(i>>1), i < 4
+//   b = 4: word w holds c'_{8w+i} at bit 16(i&1) + 4(i>>1), i < 8
+//   b = 3: word v holds c'_{10v+i} at bit 16(i&1) + 3(i>>1), i < 10; bit n of
+//          c'_30 / c'_31 is bit 15 / 31 of word n (n < 3)
+// so each pair (c'_{2m}, c'_{2m+1}) sits in matching positions of the two
+// 16-bit halves of a word and unpacks to one bf16x2 register.
+// An expert stream is the chunks of W1 (gate [F x H]), W3 (up [F x H]) and W2
+// (down [H x F]); chunk c of an expert lives in page pidx[first + c / cpp] at
+// byte (c % cpp) * 256 b, cpp = page_bytes / (256 b).
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "mpe.h"
+
+namespace mpe {
+
+constexpr int kRowsPerChunk = 16;
+constexpr int kCodesPerBlock = 128;
+
+__host__ __device__ constexpr int chunk_bytes(int b) { return 256 * b; }
+__host__ __device__ constexpr int block_bytes(int b) { return 16 * b; }
+__host__ __device__ inline int chunks_per_page(int b, uint32_t page_bytes) {
+    return (int)(page_bytes / (uint32_t)(256 * b));
+}
+__host__ __device__ constexpr int q_levels(int b) { return (1 << (b - 1)) - 1; }
+
+// Device copy of one page-table entry (same layout as mpe_pte).
+struct Pte {
+    uint8_t bits;
+    uint8_t pad[3];
+    float scale;
+    uint32_t first;
+    uint32_t n_pages;
+};
+static_assert(sizeof(Pte) == sizeof(mpe_pte), "pte layout");
+
+// What every kernel needs to reach an expert's pages.
+struct PagedExperts {
+    uint8_t* pool;
+    const Pte* pte;
+    const uint32_t* pidx;
+    uint32_t page_bytes;
+    int E, H, F;
+};
+
+__device__ __forceinline__ void set_status(uint32_t* status, uint32_t bit) {
+    atomicOr(status, bit);
+}
+
+// chunk index offsets of the three matrices inside an expert stream
+__host__ __device__ inline int chunks_w1(int H, int F) { return (F / 16) * (H / 128); }
+
+// Address of chunk c of an expert.
+__device__ __forceinline__ const uint8_t* chunk_addr(const PagedExperts& P, const Pte& pte,
+                                                     int b, int c) {
+    const int cpp = chunks_per_page(b, P.page_bytes);
+    const uint32_t page = P.pidx[pte.first + (uint32_t)(c / cpp)];
+    return P.pool + (size_t)page * P.page_bytes + (size_t)(c % cpp) * chunk_bytes(b);
+}
+
+// ---------------------------------------------------------------------------
+// timers and bounded waits
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Upper bound on any single device-side wait: far above a healthy wait (a few
+// microseconds), far below anything that looks like a hang.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+                 : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+// 1-D bulk copy global -> shared (no multicast), completing on an mbarrier.
+// dst, src 16-byte aligned; bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
+                                         uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+            "r"(smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait for phase `parity` of an mbarrier, giving up after kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (global_ns() - t0 > kWaitLimitNs) return false;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// tensor-core fragment (legacy warp-level mma, bf16 inputs, fp32 accumulate)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1,
+                                               uint32_t a2, uint32_t a3, uint32_t b0,
+                                               uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// ---------------------------------------------------------------------------
+// bf16x2 helpers for the unpack: OR-ing a small unsigned field into the
+// mantissa of bf16 128.0 (0x4300) gives the exact value 128 + field; one
+// bf16x2 subtract / fma then yields the signed code k, exactly.
+// ---------------------------------------------------------------------------
+constexpr uint32_t kMagic = 0x43004300u;  // bf16x2 (128, 128)
+
+__device__ __forceinline__ uint32_t bf2_sub(uint32_t a, uint32_t c) {
+    __nv_bfloat162 r = __hsub2(*reinterpret_cast<__nv_bfloat162*>(&a),
+                               *reinterpret_cast<__nv_bfloat162*>(&c));
+    return *reinterpret_cast<uint32_t*>(&r);
+}
+
+__device__ __forceinline__ uint32_t bf2_fma(uint32_t a, uint32_t m, uint32_t c) {
+    __nv_bfloat162 r = __hfma2(*reinterpret_cast<__nv_bfloat162*>(&a),
+                               *reinterpret_cast<__nv_bfloat162*>(&m),
+                               *reinterpret_cast<__nv_bfloat162*>(&c));
+    return *reinterpret_cast<uint32_t*>(&r);
+}
+
+// bf16 bit patterns used by the unpack
+constexpr uint32_t kBf2_132 = 0x43044304u;  // 128 + 4  (3-bit offset)
+constexpr uint32_t kBf2_136 = 0x43084308u;  // 128 + 8  (4-bit offset)
+constexpr uint32_t kBf2_eighth = 0x3E003E00u;  // 0.125
+constexpr uint32_t kBf2_m20 = 0xC1A0C1A0u;  // -20 = -(128/8 + 4)
+
+// Signed codes of pair m (0..15) of one quarter as bf16x2, from the quarter's
+// raw words w[] (b words for b = 3, 4; for b = 8 the thread holds the two
+// 16-byte halves of a 32-code range, see decode.cu).
+template <int B>
+__device__ __forceinline__ uint32_t unpack_pair(const uint32_t* w, int m);
+
+template <>
+__device__ __forceinline__ uint32_t unpack_pair<4>(const uint32_t* w, int m) {
+    const uint32_t v = w[m >> 2] >> (4 * (m & 3));
+    return bf2_sub((v & 0x000F000Fu) | kMagic, kBf2_136);
+}
+
+template <>
+__device__ __forceinline__ uint32_t unpack_pair<8>(const uint32_t* w, int m) {
+    const uint32_t v = w[m >> 1] >> (8 * (m & 1));
+    const uint32_t lo = (v & 0x007F007Fu) | kMagic;   // 128 + (u & 127)
+    const uint32_t hi = (~v & 0x00800080u) | kMagic;  // 256 - 128 * bit7(u)
+    return bf2_sub(lo, hi);                            // u - 128 = k
+}
+
+template <>
+__device__ __forceinline__ uint32_t unpack_pair<3>(const uint32_t* w, int m) {
+    if (m == 15) {
+        const uint32_t t = ((w[0] >> 15) & 0x00010001u) | ((w[1] >> 14) & 0x00020002u) |
+                           ((w[2] >> 13) & 0x00040004u) | kMagic;
+        return bf2_sub(t, kBf2_132);
+    }
+    const int v = m / 5, f = m % 5;
+    const uint32_t x = w[v] >> (f < 2 ? 0 : (f < 4 ? 6 : 12));
+    if (f == 1 || f == 3) {
+        return bf2_fma((x & 0x00380038u) | kMagic, kBf2_eighth, kBf2_m20);  // (128+8u)/8 - 20
+    }
+    return bf2_sub((x & 0x00070007u) | kMagic, kBf2_132);  // 128 + u - 132
+}
+
+}  // namespace mpe

@@ -1,0 +1,113 @@
+// Host-side context of libmpe and the launch wrappers each kernel file exports.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <string>
+#include <vector>
+
+#include "common.cuh"
+#include "mpe.h"
+
+namespace mpe {
+
+// Tokens per work group of the decode kernels (two 8-token mma n-tiles).
+constexpr int kDecodeGroup = 16;
+
+struct Scratch {
+    size_t cap_assign = 0;   // T*k capacity
+    int32_t* perm = nullptr;
+    int32_t* inv = nullptr;
+    int32_t* offsets = nullptr;  // E+1
+    int32_t* wg = nullptr;       // work groups: 3 ints each
+    int32_t* n_wg = nullptr;
+    int32_t* hist = nullptr;     // per-chunk histograms (large-T route)
+    size_t hist_cap = 0;
+    __nv_bfloat16* h = nullptr;  // [cap_assign x F]
+    float* y = nullptr;          // [cap_assign x H]
+    // staging for the host-buffer entry point
+    size_t stage_tokens = 0;
+    void* x_stage = nullptr;
+    int32_t* ids_stage = nullptr;
+    float* w_stage = nullptr;
+    void* out_stage = nullptr;
+};
+
+struct HostAllocator {
+    std::vector<uint8_t> free;             // 1 = free page
+    std::vector<std::vector<uint32_t>> pages;
+};
+
+}  // namespace mpe
+
+struct mpe_ctx {
+    int device = 0;
+    int E = 0, H = 0, F = 0;
+    uint32_t page_bytes = MPE_DEFAULT_PAGE_BYTES;
+    uint32_t pool_pages = 0;
+    int path = MPE_PATH_AUTO;
+    cudaStream_t stream = nullptr;
+    std::string err;
+    uint64_t launches = 0;
+
+    // device state
+    uint8_t* pool = nullptr;
+    mpe::Pte* d_pte = nullptr;
+    uint32_t* d_pidx = nullptr;
+    uint32_t* d_absmax = nullptr;     // fp16 bits of max|w| per expert
+    uint32_t* d_status = nullptr;
+    const void** d_masters = nullptr; // E device pointers
+    int32_t* d_list = nullptr;        // expert list for encode
+    double* d_p = nullptr;            // allocator inputs
+    uint64_t* d_W = nullptr;
+    uint8_t* d_bits_out = nullptr;
+    int32_t* d_alloc_status = nullptr;
+    uint8_t* d_choice = nullptr;
+    size_t choice_cap = 0;
+    double* d_D = nullptr;            // two DP rows
+    uint8_t* d_gather = nullptr;      // expert stream gather buffer
+    size_t gather_cap = 0;
+
+    // host mirrors
+    std::vector<const void*> masters;
+    std::vector<uint8_t> bits;
+    std::vector<mpe::Pte> pte;
+    std::vector<uint32_t> pidx;
+    mpe::Pte* h_pte_pinned = nullptr;       // upload staging (pinned)
+    uint32_t* h_pidx_pinned = nullptr;
+    int32_t* h_list_pinned = nullptr;
+    const void** h_masters_pinned = nullptr;
+    cudaEvent_t upload_done = nullptr;
+    bool absmax_valid = false;
+    mpe::HostAllocator alloc;
+    mpe::Scratch s;
+};
+
+namespace mpe {
+
+PagedExperts paged(const mpe_ctx* c);
+
+// quantize.cu
+void launch_absmax(mpe_ctx* c, const int32_t* d_list, int n_list);
+void launch_scales(mpe_ctx* c);
+void launch_encode(mpe_ctx* c, const int32_t* d_list, int n_list);
+void launch_gather_stream(mpe_ctx* c, int e, uint8_t* dst);
+
+// allocate.cu
+void launch_allocate(cudaStream_t st, const double* p, const uint64_t* W, int E, uint64_t B,
+                     uint8_t* bits_out, int32_t* status, uint8_t* choice, double* D,
+                     int state_cap);
+
+// route.cu
+void launch_route(mpe_ctx* c, const int32_t* ids, int Tk, int k, int32_t* perm,
+                  int32_t* offsets, int32_t* inv, int group);
+
+// decode.cu
+void launch_decode_gateup(mpe_ctx* c, const __nv_bfloat16* x, int k, int wg_bound);
+void launch_decode_down(mpe_ctx* c, const float* topk_w, int wg_bound);
+
+// combine.cu
+void launch_combine(mpe_ctx* c, const int32_t* ids, int T, int k, __nv_bfloat16* out);
+
+}  // namespace mpe

@@ -1,0 +1,260 @@
+// Per-expert absmax quantizer and packer.
+//
+// PagedWeight, "Implementation Details", quantization scheme:
+//   Q(w) = round(w / s) * s,  s = max|w| / (2^(b-1) - 1),  one s per expert.
+// Here: m_e = max |w| over the expert's fp16 master (exact integer max of the
+// magnitude bits), s_e = RN_f32(m_e / q_b), k = round-half-even of the exact
+// quotient w / s_e, clamped to [-q_b, q_b], stored offset-binary in the packed
+// chunk format (common.cuh) inside the expert's pages.
+#include "internal.h"
+
+namespace mpe {
+namespace {
+
+constexpr int kAbsmaxThreads = 256;
+constexpr int kAbsmaxUnroll = 4;
+constexpr int64_t kAbsmaxSegVec = 8192;  // 16-byte vectors (65536 weights) per CTA
+
+// Integer max of (h & 0x7FFF) over a segment of one expert. The magnitude bits
+// of an fp16 order exactly like |w|, so the max is exact and order-free; a
+// value >= 0x7C00 means the master holds an Inf or a NaN.
+__global__ void __launch_bounds__(kAbsmaxThreads)
+k_absmax(const void* const* masters, const int32_t* list, int64_t n_vec, uint32_t* absmax) {
+    const int e = list[blockIdx.y];
+    const uint4* src = reinterpret_cast<const uint4*>(masters[e]);
+    const int64_t beg = (int64_t)blockIdx.x * kAbsmaxSegVec;
+    const int64_t end = min(beg + kAbsmaxSegVec, n_vec);
+    uint32_t m = 0;
+    for (int64_t i = beg + threadIdx.x; i < end; i += kAbsmaxThreads * kAbsmaxUnroll) {
+        uint4 v[kAbsmaxUnroll];
+#pragma unroll
+        for (int u = 0; u < kAbsmaxUnroll; ++u) {
+            const int64_t idx = i + (int64_t)u * kAbsmaxThreads;
+            v[u] = idx < end ? __ldcs(src + idx) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < kAbsmaxUnroll; ++u) {
+            m = __vmaxu2(m, v[u].x & 0x7FFF7FFFu);
+            m = __vmaxu2(m, v[u].y & 0x7FFF7FFFu);
+            m = __vmaxu2(m, v[u].z & 0x7FFF7FFFu);
+            m = __vmaxu2(m, v[u].w & 0x7FFF7FFFu);
+        }
+    }
+    m = max(m & 0xFFFFu, m >> 16);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+    __shared__ uint32_t red[kAbsmaxThreads / 32];
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t r = red[0];
+        for (int w = 1; w < kAbsmaxThreads / 32; ++w) r = max(r, red[w]);
+        atomicMax(absmax + e, r);
+    }
+}
+
+// s_e = RN_f32(m_e / q_b); a non-finite master gets a NaN scale and a status bit.
+__global__ void k_scales(Pte* pte, const uint32_t* absmax, int E, uint32_t* status) {
+    const int e = blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= E) return;
+    const int b = pte[e].bits;
+    if (b != 3 && b != 4 && b != 8) return;
+    const uint32_t m = absmax[e];
+    if (m >= 0x7C00u) {
+        pte[e].scale = __int_as_float(0x7FC00000);
+        set_status(status, MPE_STATUS_NONFINITE);
+        return;
+    }
+    const float mf = __half2float(__ushort_as_half((unsigned short)m));
+    pte[e].scale = (m == 0) ? 0.0f : __fdiv_rn(mf, (float)q_levels(b));
+}
+
+// k = round-half-even(w / s), exactly, clamped; returns offset-binary u = k + 2^(b-1).
+// r = w * (1/s) is within ~2^-16 of the exact quotient (|w/s| < 2^8), so
+// rounding r agrees with rounding the exact quotient unless r lies within
+// that distance of a half-integer; there the sign of the single-rounded
+// fma (k -+ 1/2) s - w decides exactly.
+__device__ __forceinline__ uint32_t encode_one(float w, float s, float inv_s, float qf, int off) {
+    const float r = __fmul_rn(w, inv_s);
+    const float kr = __fsub_rn(__fadd_rn(r, 12582912.0f), 12582912.0f);  // RNE to integer
+    float kf = kr;
+    const float d = __fsub_rn(r, kr);
+    if (fabsf(d) > 0.4990234375f) {
+        const float lo = __fmaf_rn(__fsub_rn(kf, 0.5f), s, -w);  // (k - 1/2) s - w
+        const float hi = __fmaf_rn(__fadd_rn(kf, 0.5f), s, -w);  // (k + 1/2) s - w
+        const bool odd = (((int)kf) & 1) != 0;
+        if (lo > 0.0f) {
+            kf = __fsub_rn(kf, 1.0f);
+        } else if (hi < 0.0f) {
+            kf = __fadd_rn(kf, 1.0f);
+        } else if (lo == 0.0f) {
+            if (odd) kf = __fsub_rn(kf, 1.0f);
+        } else if (hi == 0.0f) {
+            if (odd) kf = __fadd_rn(kf, 1.0f);
+        }
+    }
+    kf = fminf(fmaxf(kf, -qf), qf);
+    return (uint32_t)((int)kf + off);
+}
+
+__device__ __forceinline__ void load32_half(const __half* src, float (&f)[32]) {
+    const uint4* p = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint4 v = __ldcs(p + i);
+        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const __half2 h2 = *reinterpret_cast<const __half2*>(&wv[j]);
+            const float2 ff = __half22float2(h2);
+            f[8 * i + 2 * j] = ff.x;
+            f[8 * i + 2 * j + 1] = ff.y;
+        }
+    }
+}
+
+// Encode one quarter (32 consecutive weights of a row) and store its b words.
+template <int B>
+__device__ __forceinline__ void encode_quarter(const __half* src, float s, float inv_s,
+                                               uint8_t* dst) {
+    constexpr float qf = (float)q_levels(B);
+    constexpr int off = 1 << (B - 1);
+    float f[32];
+    load32_half(src, f);
+    uint32_t u[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) u[i] = encode_one(f[i], s, inv_s, qf, off);
+    if constexpr (B == 8) {
+        uint32_t wv[8];
+#pragma unroll
+        for (int w = 0; w < 8; ++w)
+            wv[w] = u[4 * w] | (u[4 * w + 1] << 16) | (u[4 * w + 2] << 8) | (u[4 * w + 3] << 24);
+        reinterpret_cast<uint4*>(dst)[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+        reinterpret_cast<uint4*>(dst)[1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
+    } else if constexpr (B == 4) {
+        uint32_t wv[4];
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            uint32_t x = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) x |= u[8 * w + i] << (16 * (i & 1) + 4 * (i >> 1));
+            wv[w] = x;
+        }
+        reinterpret_cast<uint4*>(dst)[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+    } else {
+        uint32_t* d32 = reinterpret_cast<uint32_t*>(dst);
+#pragma unroll
+        for (int v = 0; v < 3; ++v) {
+            uint32_t x = 0;
+#pragma unroll
+            for (int i = 0; i < 10; ++i) x |= u[10 * v + i] << (16 * (i & 1) + 3 * (i >> 1));
+            x |= ((u[30] >> v) & 1u) << 15;
+            x |= ((u[31] >> v) & 1u) << 31;
+            d32[v] = x;
+        }
+    }
+}
+
+// One warp per chunk (16 rows x 128 codes). Lane l encodes quarter (l & 3) of
+// rows (l >> 2) and (l >> 2) + 8; quarter index in the chunk is l and l + 32,
+// so the lanes' stores cover the chunk contiguously.
+__global__ void __launch_bounds__(256)
+k_encode(PagedExperts P, const void* const* masters, const int32_t* list) {
+    const int e = list[blockIdx.y];
+    const Pte pte = P.pte[e];
+    const int b = pte.bits;
+    const float s = pte.scale;
+    if (!(s >= 0.0f)) return;  // non-finite master: left unencoded, status already set
+    const int H = P.H, F = P.F;
+    const int nc1 = chunks_w1(H, F);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int c = blockIdx.x * 8 + warp;
+    if (c >= 3 * nc1) return;
+    int K, cc;
+    size_t moff;
+    if (c < nc1) {
+        K = H; cc = c; moff = 0;
+    } else if (c < 2 * nc1) {
+        K = H; cc = c - nc1; moff = (size_t)F * H;
+    } else {
+        K = F; cc = c - 2 * nc1; moff = 2 * (size_t)F * H;
+    }
+    const int nj = K / kCodesPerBlock;
+    const int tau = cc / nj, j = cc - tau * nj;
+    const int rho = lane >> 2, q = lane & 3;
+    const __half* base = reinterpret_cast<const __half*>(masters[e]) + moff;
+    const __half* r0 = base + (size_t)(tau * 16 + rho) * K + 128 * j + 32 * q;
+    const __half* r8 = r0 + (size_t)8 * K;
+    uint8_t* dst = const_cast<uint8_t*>(chunk_addr(P, pte, b, c));
+    const float inv_s = s > 0.0f ? __frcp_rn(s) : 0.0f;
+    switch (b) {
+        case 3:
+            encode_quarter<3>(r0, s, inv_s, dst + 12 * lane);
+            encode_quarter<3>(r8, s, inv_s, dst + 12 * (lane + 32));
+            break;
+        case 4:
+            encode_quarter<4>(r0, s, inv_s, dst + 16 * lane);
+            encode_quarter<4>(r8, s, inv_s, dst + 16 * (lane + 32));
+            break;
+        case 8:
+            encode_quarter<8>(r0, s, inv_s, dst + 32 * lane);
+            encode_quarter<8>(r8, s, inv_s, dst + 32 * (lane + 32));
+            break;
+        default:
+            break;
+    }
+}
+
+// Copy expert e's chunk stream out of its pages, in stream order.
+__global__ void k_gather_stream(PagedExperts P, int e, uint8_t* dst) {
+    const Pte pte = P.pte[e];
+    const int b = pte.bits;
+    if (b != 3 && b != 4 && b != 8) return;
+    const int nc = 3 * chunks_w1(P.H, P.F);
+    const int cb = chunk_bytes(b);
+    for (int c = blockIdx.x; c < nc; c += gridDim.x) {
+        const uint4* src = reinterpret_cast<const uint4*>(chunk_addr(P, pte, b, c));
+        uint4* d = reinterpret_cast<uint4*>(dst + (size_t)c * cb);
+        for (int i = threadIdx.x; i < cb / 16; i += blockDim.x) d[i] = src[i];
+    }
+}
+
+}  // namespace
+
+PagedExperts paged(const mpe_ctx* c) {
+    PagedExperts P;
+    P.pool = c->pool;
+    P.pte = c->d_pte;
+    P.pidx = c->d_pidx;
+    P.page_bytes = c->page_bytes;
+    P.E = c->E;
+    P.H = c->H;
+    P.F = c->F;
+    return P;
+}
+
+void launch_absmax(mpe_ctx* c, const int32_t* d_list, int n_list) {
+    const int64_t n_vec = (int64_t)3 * c->H * c->F / 8;
+    dim3 grid((unsigned)((n_vec + kAbsmaxSegVec - 1) / kAbsmaxSegVec), (unsigned)n_list);
+    k_absmax<<<grid, kAbsmaxThreads, 0, c->stream>>>(c->d_masters, d_list, n_vec, c->d_absmax);
+    c->launches++;
+}
+
+void launch_scales(mpe_ctx* c) {
+    k_scales<<<(c->E + 127) / 128, 128, 0, c->stream>>>(c->d_pte, c->d_absmax, c->E, c->d_status);
+    c->launches++;
+}
+
+void launch_encode(mpe_ctx* c, const int32_t* d_list, int n_list) {
+    const int nc = 3 * chunks_w1(c->H, c->F);
+    dim3 grid((unsigned)((nc + 7) / 8), (unsigned)n_list);
+    k_encode<<<grid, 256, 0, c->stream>>>(paged(c), c->d_masters, d_list);
+    c->launches++;
+}
+
+void launch_gather_stream(mpe_ctx* c, int e, uint8_t* dst) {
+    k_gather_stream<<<148, 128, 0, c->stream>>>(paged(c), e, dst);
+    c->launches++;
+}
+
+}  // namespace mpe

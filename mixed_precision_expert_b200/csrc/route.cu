@@ -1,0 +1,206 @@
+// Token-to-expert bucketing for the forward pass.
+//
+// PagedWeight, "Dynamic Paging": the router decides which experts a pass
+// needs; their pages serve all of their tokens at once. Assignment a = t*k + j
+// (token t's j-th routed expert ids[a]):
+//   perm    = the assignments ordered by expert id, stable in a;
+//   offsets = exclusive prefix sums of the per-expert counts (E+1 entries);
+//   inv[a]  = position of a in perm, -1 for ids outside [0, E) (dropped, with
+//             MPE_STATUS_BAD_EXPERT_ID set);
+// plus the decode work groups: each expert's tokens cut into runs of at most
+// `group` positions, listed as (expert, first position, count).
+//
+// Stable ranks come from warp matching: inside a warp, lanes holding the same
+// id rank by lane; across warps, by the per-warp counts of earlier warps;
+// across 1024-assignment chunks, by the per-chunk histograms.
+#include "internal.h"
+
+namespace mpe {
+namespace {
+
+constexpr int kChunk = 1024;
+
+// Exclusive block scan of one uint64 per thread over 1024 threads.
+__device__ uint64_t block_exclusive_scan(uint64_t v, uint64_t* s_warp, uint64_t* total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint64_t x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint64_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) s_warp[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        uint64_t w = s_warp[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint64_t y = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += y;
+        }
+        s_warp[lane] = w;  // inclusive over warps
+    }
+    __syncthreads();
+    const uint64_t before = (warp > 0 ? s_warp[warp - 1] : 0) + x - v;
+    *total = s_warp[31];
+    __syncthreads();
+    return before;
+}
+
+// Offsets and work groups from per-expert counts (thread e holds count[e]).
+__device__ void offsets_and_groups(int E, int cnt, int group, int32_t* offsets, int32_t* wg,
+                                   int32_t* n_wg, int32_t* s_off) {
+    __shared__ uint64_t s_warp[32];
+    const int e = threadIdx.x;
+    const int ng = (e < E) ? (cnt + group - 1) / group : 0;
+    const uint64_t packed = ((uint64_t)(e < E ? cnt : 0) << 32) | (uint64_t)ng;
+    uint64_t total;
+    const uint64_t ex = block_exclusive_scan(packed, s_warp, &total);
+    const int off = (int)(ex >> 32), goff = (int)(ex & 0xFFFFFFFFu);
+    if (e < E) {
+        offsets[e] = off;
+        s_off[e] = off;
+        for (int i = 0; i < ng; ++i) {
+            wg[3 * (goff + i) + 0] = e;
+            wg[3 * (goff + i) + 1] = off + i * group;
+            wg[3 * (goff + i) + 2] = min(group, cnt - i * group);
+        }
+    }
+    if (e == 0) {
+        offsets[E] = (int)(total >> 32);
+        *n_wg = (int)(total & 0xFFFFFFFFu);
+    }
+}
+
+// Stable scatter of one chunk: base[e] = first position of this chunk's
+// assignments with id e.
+__device__ void scatter_chunk(const int32_t* ids, int a0, int n, int E, const int32_t* base,
+                              uint16_t* wcnt, int32_t* perm, int32_t* inv, uint32_t* status) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int a = a0 + threadIdx.x;
+    int e = -1;
+    bool valid = false;
+    if (threadIdx.x < n) {
+        e = ids[a];
+        valid = (e >= 0 && e < E);
+        if (!valid) set_status(status, MPE_STATUS_BAD_EXPERT_ID);
+    }
+    const int key = valid ? e : -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, key);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    if (valid && rank == 0) wcnt[warp * E + e] = (uint16_t)__popc(peers);
+    __syncthreads();
+    if (valid) {
+        int pre = 0;
+        for (int w = 0; w < warp; ++w) pre += wcnt[w * E + e];
+        const int pos = base[e] + pre + rank;
+        perm[pos] = a;
+        inv[a] = pos;
+    } else if (threadIdx.x < n) {
+        inv[a] = -1;
+    }
+}
+
+// T*k <= 1024: everything in one CTA.
+__global__ void __launch_bounds__(kChunk)
+k_route_small(const int32_t* ids, int Tk, int E, int group, int32_t* perm, int32_t* offsets,
+              int32_t* inv, int32_t* wg, int32_t* n_wg, uint32_t* status) {
+    extern __shared__ __align__(16) uint8_t sm[];
+    int32_t* s_cnt = reinterpret_cast<int32_t*>(sm);       // [E]
+    int32_t* s_off = s_cnt + MPE_MAX_EXPERTS;               // [E]
+    uint16_t* wcnt = reinterpret_cast<uint16_t*>(s_off + MPE_MAX_EXPERTS);  // [32][E]
+    for (int i = threadIdx.x; i < 32 * E; i += kChunk) wcnt[i] = 0;
+    for (int i = threadIdx.x; i < E; i += kChunk) s_cnt[i] = 0;
+    __syncthreads();
+    if (threadIdx.x < Tk) {
+        const int e = ids[threadIdx.x];
+        if (e >= 0 && e < E) atomicAdd(&s_cnt[e], 1);
+    }
+    __syncthreads();
+    const int cnt = threadIdx.x < E ? s_cnt[threadIdx.x] : 0;
+    offsets_and_groups(E, cnt, group, offsets, wg, n_wg, s_off);
+    __syncthreads();
+    scatter_chunk(ids, 0, Tk, E, s_off, wcnt, perm, inv, status);
+}
+
+// T*k > 1024, step 1: per-chunk histograms hist[c][e].
+__global__ void __launch_bounds__(kChunk)
+k_route_hist(const int32_t* ids, int Tk, int E, int32_t* hist) {
+    __shared__ int32_t s_cnt[MPE_MAX_EXPERTS];
+    for (int i = threadIdx.x; i < E; i += kChunk) s_cnt[i] = 0;
+    __syncthreads();
+    const int a = blockIdx.x * kChunk + threadIdx.x;
+    if (a < Tk) {
+        const int e = ids[a];
+        if (e >= 0 && e < E) atomicAdd(&s_cnt[e], 1);
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < E; i += kChunk) hist[(size_t)blockIdx.x * E + i] = s_cnt[i];
+}
+
+// Step 2 (one CTA): hist[c][e] <- first position of chunk c's id-e assignments.
+__global__ void __launch_bounds__(kChunk)
+k_route_scan(int32_t* hist, int n_chunks, int E, int group, int32_t* offsets, int32_t* wg,
+             int32_t* n_wg) {
+    __shared__ int32_t s_off[MPE_MAX_EXPERTS];
+    const int e = threadIdx.x;
+    int run = 0;
+    if (e < E) {
+        for (int c = 0; c < n_chunks; ++c) {
+            const int h = hist[(size_t)c * E + e];
+            hist[(size_t)c * E + e] = run;
+            run += h;
+        }
+    }
+    offsets_and_groups(E, run, group, offsets, wg, n_wg, s_off);
+    __syncthreads();
+    if (e < E) {
+        const int off = s_off[e];
+        for (int c = 0; c < n_chunks; ++c) hist[(size_t)c * E + e] += off;
+    }
+}
+
+// Step 3: stable scatter of each chunk.
+__global__ void __launch_bounds__(kChunk)
+k_route_scatter(const int32_t* ids, int Tk, int E, const int32_t* hist, int32_t* perm,
+                int32_t* inv, uint32_t* status) {
+    extern __shared__ __align__(16) uint8_t sm[];
+    uint16_t* wcnt = reinterpret_cast<uint16_t*>(sm);  // [32][E]
+    for (int i = threadIdx.x; i < 32 * E; i += kChunk) wcnt[i] = 0;
+    __syncthreads();
+    const int a0 = blockIdx.x * kChunk;
+    scatter_chunk(ids, a0, min(kChunk, Tk - a0), E, hist + (size_t)blockIdx.x * E, wcnt, perm,
+                  inv, status);
+}
+
+}  // namespace
+
+void launch_route(mpe_ctx* c, const int32_t* ids, int Tk, int k, int32_t* perm,
+                  int32_t* offsets, int32_t* inv, int group) {
+    (void)k;
+    const int E = c->E;
+    if (Tk <= kChunk) {
+        const size_t sm = 2 * MPE_MAX_EXPERTS * sizeof(int32_t) + 32 * E * sizeof(uint16_t);
+        k_route_small<<<1, kChunk, sm, c->stream>>>(ids, Tk, E, group, perm, offsets, inv,
+                                                    c->s.wg, c->s.n_wg, c->d_status);
+        c->launches++;
+        return;
+    }
+    const int nch = (Tk + kChunk - 1) / kChunk;
+    k_route_hist<<<nch, kChunk, 0, c->stream>>>(ids, Tk, E, c->s.hist);
+    k_route_scan<<<1, kChunk, 0, c->stream>>>(c->s.hist, nch, E, group, offsets, c->s.wg,
+                                              c->s.n_wg);
+    const size_t sm = 32 * E * sizeof(uint16_t);
+    k_route_scatter<<<nch, kChunk, sm, c->stream>>>(ids, Tk, E, c->s.hist, perm, inv,
+                                                    c->d_status);
+    c->launches += 3;
+}
+
+void route_set_smem_limits() {
+    const int maxsm = 2 * MPE_MAX_EXPERTS * 4 + 32 * MPE_MAX_EXPERTS * 2;
+    cudaFuncSetAttribute(k_route_small, cudaFuncAttributeMaxDynamicSharedMemorySize, maxsm);
+    cudaFuncSetAttribute(k_route_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         32 * MPE_MAX_EXPERTS * 2);
+}
+
+}  // namespace mpe

@@ -1,0 +1,52 @@
+"""The C ABI library builds, loads without a GPU and exports every symbol that
+include/mpe.h declares; the binding's error path works without a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from mixed_precision_expert_b200.build import build
+    build()
+    import mixed_precision_expert_b200 as mpe
+    return mpe.lib()
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "mpe.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mpe_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_binding_exports():
+    import mixed_precision_expert_b200 as mpe
+    assert declared_symbols() == sorted(mpe.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+        assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def test_version_and_argument_errors_without_gpu(lib):
+    import mixed_precision_expert_b200 as mpe
+    assert lib.mpe_version() == 100
+    # invalid arguments are rejected before any device work
+    assert lib.mpe_create(None, None) == -1
+    cfg = mpe.Config(0, 256, 512, 0, 0, 0, 0, 0, None)
+    h = ctypes.c_void_p()
+    assert lib.mpe_create(ctypes.byref(h), ctypes.byref(cfg)) == -1
+    assert b"E=0" in lib.mpe_last_error_global()
+    cfg = mpe.Config(8, 200, 512, 0, 0, 0, 0, 0, None)
+    assert lib.mpe_create(ctypes.byref(h), ctypes.byref(cfg)) == -1
+    with pytest.raises(mpe.MpeError):
+        mpe.allocate_bits([0.5, 0.5], [10, 0], 100)      # W_e = 0
+    with pytest.raises(mpe.MpeError) as ei:
+        mpe.allocate_bits([0.5, 0.5], [10, 10], 59)      # below 3 bits per weight
+    assert ei.value.code == -2

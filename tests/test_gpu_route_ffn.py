@@ -1,0 +1,149 @@
+"""GPU parity for token bucketing (bit-exact) and for the routed SwiGLU expert
+FFN run from the pages (rel-Frobenius <= 5e-3, max-abs <= 2e-2 * max|oracle|)
+against the float64 dequantize-then-multiply oracle (PagedWeight, "Dynamic
+Paging")."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import route as orr
+
+from _helpers import OracleExpert, check_ffn, oracle_moe
+
+pytestmark = pytest.mark.gpu
+
+mpe = pytest.importorskip("mixed_precision_expert_b200")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from mixed_precision_expert_b200.build import build
+    build()
+    assert torch.cuda.is_available()
+
+
+@pytest.mark.parametrize("T,k,E,seed", [(1, 1, 8, 0), (64, 2, 8, 1), (64, 8, 128, 2),
+                                        (128, 8, 256, 3), (100, 7, 33, 4), (1000, 8, 128, 5),
+                                        (8192, 8, 128, 6), (3000, 3, 1024, 7)])
+def test_route_parity(T, k, E, seed):
+    rng = np.random.default_rng(seed)
+    ids = rng.integers(0, E, size=(T, k)).astype(np.int32)
+    if seed % 2:
+        ids[rng.integers(0, T, 3), rng.integers(0, k, 3)] = rng.choice([-5, E, E + 7], 3)
+    ctx = mpe.Context(E, 128, 128)
+    perm, offs, inv = ctx.route(torch.from_numpy(ids).cuda())
+    rp, ro, ri = orr.route(ids, E)
+    assert np.array_equal(offs.cpu().numpy(), ro)
+    n = int(ro[-1])
+    assert np.array_equal(perm.cpu().numpy()[:n], rp)
+    assert np.array_equal(inv.cpu().numpy(), ri)
+    bad = bool((ids < 0).any() or (ids >= E).any())
+    assert bool(ctx.status(clear=True) & mpe.STATUS_BAD_EXPERT_ID) == bad
+
+
+def _layer(wl, bits=None, device="cuda", path=0):
+    if bits is None:
+        bits = mpe.allocate_bits(synth.importance(wl), [wl.W_e] * wl.E, wl.budget_bits)
+    masters = [synth.expert_weights(wl, e, device=device) for e in range(wl.E)]
+    ctx = mpe.Context(wl.E, wl.H, wl.F, path=path)
+    ctx.quantize_experts(masters, bits)
+    ox = [OracleExpert(m.cpu().numpy(), wl.H, wl.F, int(b)) for m, b in zip(masters, bits)]
+    mats = {}
+
+    def mats_of(e):
+        if e not in mats:
+            mats[e] = ox[e].mats()
+        return mats[e]
+
+    return ctx, masters, mats_of
+
+
+def _run(ctx, x, ids, w):
+    out = ctx.moe_ffn(x.cuda(), torch.from_numpy(ids).cuda(), torch.from_numpy(w).cuda())
+    torch.cuda.synchronize()
+    return out.double().cpu().numpy()
+
+
+def test_ffn_tiny_layer():
+    wl = synth.WORKLOADS[1]
+    ctx, _, mats_of = _layer(wl)
+    ids, w = synth.routing(wl)
+    x = synth.activations(wl)
+    got = _run(ctx, x, ids, w)
+    check_ffn(got, oracle_moe(x, ids, w, mats_of, wl.E))
+    assert ctx.status() == 0
+
+
+@pytest.mark.parametrize("bits", [(3,) * 4, (4,) * 4, (8,) * 4, (3, 4, 8, 3)])
+def test_ffn_each_width(bits):
+    wl = synth.scaled(synth.WORKLOADS[1], E=4, H=384, F=256, T=19, k=2)
+    ctx, _, mats_of = _layer(wl, np.array(bits, np.uint8))
+    ids, w = synth.routing(wl)
+    x = synth.activations(wl)
+    check_ffn(_run(ctx, x, ids, w), oracle_moe(x, ids, w, mats_of, wl.E))
+
+
+def test_ffn_edge_token_counts():
+    wl = synth.scaled(synth.WORKLOADS[1], E=6, H=256, F=384, T=40, k=3)
+    ctx, _, mats_of = _layer(wl, np.array([3, 4, 8, 4, 3, 8], np.uint8))
+    x = synth.activations(wl)
+    rng = np.random.default_rng(3)
+    cases = []
+    # a single token
+    cases.append((x[:1], np.array([[2, 0, 5]], np.int32)))
+    # every token on expert 1 (more than one 16-token work group), expert 4 unused
+    ids = np.stack([np.ones(40, np.int32), rng.integers(0, 4, 40).astype(np.int32),
+                    np.full(40, 5, np.int32)], 1)
+    cases.append((x, ids))
+    # 17 tokens: a ragged last n-tile and work group
+    ids = rng.integers(0, 6, size=(17, 3)).astype(np.int32)
+    cases.append((x[:17], ids))
+    for xi, ids in cases:
+        w = rng.random(ids.shape).astype(np.float32)
+        check_ffn(_run(ctx, xi.contiguous(), ids, w), oracle_moe(xi, ids, w, mats_of, wl.E))
+
+
+def test_ffn_invalid_ids_are_dropped():
+    wl = synth.scaled(synth.WORKLOADS[1], E=4, H=128, F=256, T=5, k=2)
+    ctx, _, mats_of = _layer(wl, np.array([4, 4, 8, 3], np.uint8))
+    x = synth.activations(wl)
+    ids = np.array([[0, 9], [1, -1], [2, 3], [4, 0], [3, 3]], np.int32)
+    w = np.full(ids.shape, 0.5, np.float32)
+    got = _run(ctx, x, ids, w)
+    assert ctx.status(clear=True) & mpe.STATUS_BAD_EXPERT_ID
+    check_ffn(got, oracle_moe(x, ids, w, mats_of, wl.E))
+
+
+def test_ffn_zero_tokens_is_a_no_op():
+    wl = synth.scaled(synth.WORKLOADS[1], E=2, H=128, F=128)
+    ctx, _, _ = _layer(wl, np.array([4, 4], np.uint8))
+    out = ctx.moe_ffn(torch.empty(0, 128, dtype=torch.bfloat16, device="cuda"),
+                      torch.empty(0, 2, dtype=torch.int32, device="cuda"),
+                      torch.empty(0, 2, dtype=torch.float32, device="cuda"))
+    assert out.shape == (0, 128)
+
+
+def test_ffn_host_buffers_match_device_call():
+    wl = synth.WORKLOADS[1]
+    ctx, _, _ = _layer(wl)
+    ids, w = synth.routing(wl)
+    x = synth.activations(wl)
+    dev = _run(ctx, x, ids, w)
+    xh = x.pin_memory()
+    idh = torch.from_numpy(ids).pin_memory()
+    wh = torch.from_numpy(w).pin_memory()
+    oh = torch.empty(x.shape, dtype=torch.bfloat16).pin_memory()
+    ctx.moe_ffn_host(xh, idh, wh, oh)
+    assert np.array_equal(oh.double().numpy(), dev)
+
+
+def test_ffn_finegrained_decode_full_size():
+    # 128 experts, hidden 2048, ffn 768, 64 tokens top-8 (Zipf-skewed), 3.5 bits average
+    wl = synth.WORKLOADS[3]
+    ctx, _, mats_of = _layer(wl)
+    ids, w = synth.routing(wl)
+    x = synth.activations(wl)
+    got = _run(ctx, x, ids, w)
+    toks = np.arange(0, wl.T, 4)
+    check_ffn(got[toks], oracle_moe(x, ids, w, mats_of, wl.E, tokens=toks))
