@@ -1,0 +1,449 @@
+"""Benchmark: MoE-layer tokens/s and packed-weight HBM GB/s against the roofline.
+
+Default workload: the Mixtral-shaped decode layer (8 experts, hidden 4096, SwiGLU
+ffn 14336, fp16 master ~N(0, 0.02) with 0.1% outliers at 10 sigma, 4.5 bits per
+weight on average, 16 bf16 tokens per step, top-2). One step = one pass of the
+forward path over one fresh batch (route, page-table gather + unpack/dequant
+fused into the gate/up and down contractions, SwiGLU, top-k combine) with the
+quantized pages resident; the quantize pass that produced them is timed
+separately and reported under "quantize".
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 2]
+    python bench.py --impl reference ...   # the float64 CPU oracle arm
+
+With N > 1 (torchrun), every rank runs an independent replica of the layer on
+its own GPU (the path needs no collective); value = tokens of all ranks / the
+slowest rank's device time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "MoE-layer tokens/s & packed-weight HBM GB/s vs roofline (mixed 3/4/8-bit)"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["mpe", "reference"], default="mpe")
+    ap.add_argument("--workload", type=int, default=2, choices=[1, 2, 3, 5])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (replicas: barriers and a max over ranks only)
+# ---------------------------------------------------------------------------
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+
+    def init(self, backend: str):
+        if self.world > 1:
+            import datetime
+
+            import torch.distributed as dist
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg:
+            self.pg.barrier()
+
+    def max(self, v: float) -> float:
+        if not self.pg:
+            return v
+        import torch
+        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines: list[str] = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict | None:
+        if not self.proc:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# shared helpers
+# ---------------------------------------------------------------------------
+def measured_peaks() -> tuple[float, str]:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "mixed_precision_expert_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str) -> float | None:
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel sources."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    ent = rec.get(f"{kernel}:{workload}")
+    if not ent or ent.get("source_hash") != kernel_source_hash():
+        return None
+    return float(ent["dram_bytes_per_launch"])
+
+
+def workload_config(wl, bits=None):
+    cfg = {"workload": wl.name, "E": wl.E, "H": wl.H, "F": wl.F, "tokens_per_step": wl.T,
+           "top_k": wl.k, "avg_bits_budget": wl.avg_bits, "page_bytes": 65536,
+           "parallelism": "replicas"}
+    if bits is not None:
+        cfg["bits_hist"] = {str(b): int((np.asarray(bits) == b).sum()) for b in (3, 4, 8)}
+    return cfg
+
+
+def cores_used() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+class OracleSample:
+    """Bounded sample of the oracle's forward work: one token through one expert,
+    in slices of rows of F (SwiGLU separates over F, so the slices of all F rows
+    sum to the expert's output). Input generation and the oracle's quantization
+    of the expert (the resident pages) happen once, untimed; each slice
+    dequantizes its rows and runs the float64 SwiGLU."""
+
+    def __init__(self, wl, e: int = 0, token: int = 0):
+        import synth
+        from oracle import allocate as oa
+        from oracle import quantize as oq
+        self.wl = wl
+        bits = oa.allocate_bits(synth.importance(wl), [wl.W_e] * wl.E, wl.budget_bits)
+        master = synth.expert_weights(wl, e).numpy()
+        self.m, self.s, k = oq.quantize_expert(master, int(bits[e]))
+        H, F = wl.H, wl.F
+        self.k1 = k[:F * H].reshape(F, H)
+        self.k3 = k[F * H:2 * F * H].reshape(F, H)
+        self.k2 = k[2 * F * H:].reshape(H, F)
+        self.x = synth.activations(wl, T=token + 1)[token:token + 1].double().numpy()
+
+    def run(self, n_slices: int, slice_rows: int):
+        """(seconds, tokens of layer work done)."""
+        from oracle import ffn as of
+        from oracle import quantize as oq
+        F = self.wl.F
+        t0 = time.perf_counter()
+        y = np.zeros((1, self.wl.H))
+        for i in range(n_slices):
+            f0 = (i * slice_rows) % F
+            sl = slice(f0, f0 + slice_rows)
+            y += of.expert_ffn(self.x, oq.dequantize(self.k1[sl], self.s),
+                               oq.dequantize(self.k3[sl], self.s),
+                               oq.dequantize(self.k2[:, sl], self.s))
+        return time.perf_counter() - t0, n_slices * slice_rows / F / self.wl.k
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the float64 oracle on the host cores
+# ---------------------------------------------------------------------------
+def run_reference(args, dist: Dist):
+    import synth
+    if dist.rank != 0:
+        return
+    wl = synth.WORKLOADS[args.workload]
+    slice_rows = 128
+    sample = OracleSample(wl)
+    # warm-up and timed steps: each step = one 128-row F-slice of one token-slot
+    sample.run(max(1, args.warmup), slice_rows)
+    dt, frac = sample.run(args.steps, slice_rows)
+    value = frac / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(wl),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores_used(),
+                         "kind": "oracle",
+                         "sample": f"each step: one {slice_rows}-row slice of ffn for one token "
+                                   f"through one expert (dequantize + SwiGLU, float64); "
+                                   f"{args.steps} steps = {frac:.4f} tokens of layer work"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# the library arm
+# ---------------------------------------------------------------------------
+def run_mpe(args, dist: Dist):
+    import torch
+
+    from mixed_precision_expert_b200.build import build
+    if dist.rank == 0:
+        build()
+    dist.barrier()
+    import mixed_precision_expert_b200 as mpe
+    import synth
+
+    dev = dist.local_rank
+    torch.cuda.set_device(dev)
+    wl = synth.WORKLOADS[args.workload]
+    E, H, F, T, k = wl.E, wl.H, wl.F, wl.T, wl.k
+
+    # resident state: fp16 masters -> bit allocation -> quantized pages
+    masters = []
+    for e in range(E):
+        t = torch.empty(wl.W_e, dtype=torch.float16, device="cuda")
+        synth.fill_expert_weights(wl, e, t)
+        masters.append(t)
+    p = synth.importance(wl)
+    bits = mpe.allocate_bits(p, [wl.W_e] * E, wl.budget_bits)
+    ctx = mpe.Context(E, H, F)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    q_ms = []
+    for _ in range(3):
+        torch.cuda.synchronize()
+        ev0.record()
+        ctx.quantize_experts(masters, bits)
+        ev1.record()
+        torch.cuda.synchronize()
+        q_ms.append(ev0.elapsed_time(ev1))
+    q_bytes = 4 * wl.sum_W + sum(int(b) * wl.W_e // 8 for b in bits)  # absmax + encode passes
+    if ctx.status() != 0:
+        raise RuntimeError(f"device status {ctx.status():#x} after quantize")
+
+    # per-step batches, resident in HBM (distinct seeds, cycled)
+    nb = min(64, args.steps + args.warmup)
+    batches = []
+    for i in range(nb):
+        seed = 7_000_000 + 1000 * dist.rank + i
+        ids, w = synth.routing(wl, seed=seed)
+        x = synth.activations(wl, seed=seed, device="cuda")
+        batches.append((x, torch.from_numpy(ids).cuda(), torch.from_numpy(w).cuda(), ids))
+    out = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
+
+    def gateup_bytes(ids_np):
+        act = np.unique(ids_np)
+        wbytes = sum(int(bits[e]) * 2 * F * H // 8 for e in act)
+        return wbytes + T * H * 2 + T * k * F * 2
+
+    def layer_bytes(ids_np):
+        act = np.unique(ids_np)
+        return sum(int(bits[e]) * wl.W_e // 8 for e in act) + 2 * T * H * 2
+
+    for i in range(args.warmup):
+        x, idt, wt, _ = batches[i % nb]
+        ctx.moe_ffn(x, idt, wt, out)
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(dev)
+    clocks.start()
+    time.sleep(0.3)  # let the sampler attach before the timed region
+    ctx.profile(True)
+    launches0 = ctx.kernel_launches()
+    dist.barrier()
+    torch.cuda.synchronize()
+    ev0.record()
+    for i in range(args.steps):
+        x, idt, wt, _ = batches[i % nb]
+        ctx.moe_ffn(x, idt, wt, out)
+    ev1.record()
+    torch.cuda.synchronize()
+    dist.barrier()
+    ms_local = ev0.elapsed_time(ev1)
+    launches = ctx.kernel_launches() - launches0
+    prof = ctx.profile_read(reset=True)
+    ctx.profile(False)
+    clk = clocks.stop()
+    ms = dist.max(ms_local)
+    if ctx.status() != 0:
+        raise RuntimeError(f"device status {ctx.status():#x} after the timed region")
+
+    tokens = T * args.steps * dist.world
+    value = tokens / (ms / 1e3)
+    alg_gu = np.mean([gateup_bytes(batches[i % nb][3]) for i in range(args.steps)])
+    alg_layer = np.mean([layer_bytes(batches[i % nb][3]) for i in range(args.steps)])
+    gu_ms, gu_n = prof["gate_up"]
+    peak, peak_kind = measured_peaks()
+    achieved = alg_gu / (gu_ms / gu_n / 1e3) / 1e9
+    roofline = {"bound": "hbm", "kernel": "decode gate/up (k_decode<true>)",
+                "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                "peak_source": peak_kind,
+                "traffic": recorded_traffic("k_decode_gateup", wl.name),
+                "algorithmic_bytes_per_launch": alg_gu,
+                "avg_launch_us": gu_ms / gu_n * 1e3}
+    layer_gbs = alg_layer / (ms_local / args.steps / 1e3) / 1e9
+    kernel_share = {kname: round(v[0] / max(sum(x[0] for x in prof.values()), 1e-9), 4)
+                    for kname, v in prof.items() if v[1]}
+
+    # end to end through the C ABI with host buffers (pinned), copies in the timed region
+    e2e = None
+    hb = []
+    for i in range(min(nb, 16)):
+        x, idt, wt, ids_np = batches[i]
+        hb.append((x.cpu().pin_memory(), torch.from_numpy(ids_np).pin_memory(),
+                   wt.cpu().pin_memory(), torch.empty(T, H, dtype=torch.bfloat16).pin_memory()))
+    n_e2e = max(10, min(args.steps, 500))
+    for i in range(5):
+        xh, ih, wh, oh = hb[i % len(hb)]
+        ctx.moe_ffn_host(xh, ih, wh, oh)
+    dist.barrier()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for i in range(n_e2e):
+        xh, ih, wh, oh = hb[i % len(hb)]
+        ctx.moe_ffn_host(xh, ih, wh, oh)
+    e2e_s = dist.max(time.perf_counter() - t0)
+    h2d = T * H * 2 + T * k * 4 + T * k * 4
+    d2h = T * H * 2
+    e2e = {"value": T * n_e2e * dist.world / e2e_s, "unit": "tokens/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e}
+
+    cpu = None
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        slice_rows = 128
+        n_slices = max(1, F // slice_rows)
+        dt, frac = OracleSample(wl).run(n_slices, slice_rows)
+        cpu = {"value": frac / dt, "unit": "tokens/s", "cores": cores_used(), "kind": "oracle",
+               "sample": f"one token through one expert (all {F} ffn rows in {n_slices} slices; "
+                         f"dequantize + SwiGLU in float64) = {frac:.3f} tokens of layer work"}
+
+    qms = float(np.median(q_ms))
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": dist.world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {**workload_config(wl, bits),
+                   "l2": f"no flush: packed weights of the active experts "
+                         f"({alg_layer / 1e6:.0f} MB per step) exceed the 126 MB L2"},
+        "packed_weight_gbs": layer_gbs,
+        "packed_weight_frac_of_peak": layer_gbs / peak,
+        "roofline": roofline,
+        "kernel_time_share": kernel_share,
+        "quantize": {"ms": qms, "GB/s": q_bytes / (qms / 1e3) / 1e9,
+                     "frac": q_bytes / (qms / 1e3) / 1e9 / peak,
+                     "bytes": q_bytes, "passes": "absmax read + encode read/write"},
+        "gpu_launches": launches,
+        "clocks": clk,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+    }
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+    ctx.close()
+
+
+def main():
+    args = parse_args()
+    dist = Dist()
+    if args.impl == "reference":
+        run_reference(args, dist)
+        return
+    import torch
+    torch.cuda.set_device(dist.local_rank)
+    dist.init("nccl")
+    try:
+        run_mpe(args, dist)
+    finally:
+        dist.close()
+
+
+if __name__ == "__main__":
+    main()

@@ -239,6 +239,23 @@ const char* mpe_last_error(mpe_ctx* ctx);
  * context-free call (mpe_allocate_bits, mpe_create). */
 const char* mpe_last_error_global(void);
 
+/*
+ * mpe_profile_enable -- when enable != 0, mpe_moe_ffn records a CUDA event
+ * pair around each of its kernels (on the context stream) so their device
+ * times can be read back; 0 stops recording. Recording costs one event
+ * record per kernel boundary.
+ */
+int mpe_profile_enable(mpe_ctx* ctx, int32_t enable);
+
+/*
+ * mpe_profile_read -- synchronise and sum the recorded kernel times per slot
+ * (0 route, 1 gate/up, 2 SwiGLU reduce, 3 down, 4 combine): ms_host
+ * double[n_slots] milliseconds, launches_host int64[n_slots] counts (either
+ * may be NULL). reset != 0 clears the records.
+ */
+int mpe_profile_read(mpe_ctx* ctx, double* ms_host, int64_t* launches_host, int32_t n_slots,
+                     int32_t reset);
+
 /* mpe_kernel_launches -- how many kernels this context has launched so far. */
 uint64_t mpe_kernel_launches(mpe_ctx* ctx);
 

@@ -39,8 +39,10 @@ EXPORTS = [
     "mpe_quantize_experts", "mpe_repage", "mpe_moe_ffn", "mpe_moe_ffn_host", "mpe_route",
     "mpe_get_page_table", "mpe_expert_stream_bytes", "mpe_read_expert_packed",
     "mpe_get_scales", "mpe_get_bits", "mpe_get_status", "mpe_last_error",
-    "mpe_last_error_global", "mpe_kernel_launches", "mpe_version",
+    "mpe_last_error_global", "mpe_kernel_launches", "mpe_version", "mpe_profile_enable",
+    "mpe_profile_read",
 ]
+PROFILE_SLOTS = ["route", "gate_up", "swiglu_reduce", "down", "combine"]
 
 
 class MpeError(RuntimeError):
@@ -100,6 +102,8 @@ def lib() -> ctypes.CDLL:
         "mpe_last_error_global": (ctypes.c_char_p, []),
         "mpe_kernel_launches": (u64, [vp]),
         "mpe_version": (i32, []),
+        "mpe_profile_enable": (i32, [vp, i32]),
+        "mpe_profile_read": (i32, [vp, vp, vp, i32, i32]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -250,3 +254,16 @@ class Context:
 
     def kernel_launches(self) -> int:
         return int(lib().mpe_kernel_launches(self._h))
+
+    def profile(self, enable: bool):
+        """Record CUDA events around each forward-pass kernel (device times)."""
+        _check(lib().mpe_profile_enable(self._h, 1 if enable else 0), self._h)
+
+    def profile_read(self, reset: bool = True) -> dict:
+        """{slot: (total ms, launches)} for the recorded kernels."""
+        n = len(PROFILE_SLOTS)
+        ms = np.zeros(n, dtype=np.float64)
+        cnt = np.zeros(n, dtype=np.int64)
+        _check(lib().mpe_profile_read(self._h, _ptr(ms), _ptr(cnt), n, 1 if reset else 0),
+               self._h)
+        return {name: (float(ms[i]), int(cnt[i])) for i, name in enumerate(PROFILE_SLOTS)}

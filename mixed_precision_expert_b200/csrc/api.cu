@@ -147,7 +147,7 @@ int dev_alloc(mpe_ctx* c, T** p, size_t n) {
 
 void free_scratch(Scratch& s) {
     cudaFree(s.perm); cudaFree(s.inv); cudaFree(s.offsets); cudaFree(s.wg); cudaFree(s.n_wg);
-    cudaFree(s.hist); cudaFree(s.h); cudaFree(s.y);
+    cudaFree(s.hist); cudaFree(s.h); cudaFree(s.y); cudaFree(s.part); cudaFree(s.task_ctr);
     cudaFree(s.x_stage); cudaFree(s.ids_stage); cudaFree(s.w_stage); cudaFree(s.out_stage);
     s = Scratch{};
 }
@@ -173,12 +173,15 @@ int ensure_scratch(mpe_ctx* c, size_t Tk) {
     if ((r = dev_alloc(c, &s.inv, cap))) return r;
     if ((r = dev_alloc(c, &s.offsets, E + 1))) return r;
     if ((r = dev_alloc(c, &s.wg, 3 * (size_t)wg_capacity(E, cap, 1)))) return r;
-    if ((r = dev_alloc(c, &s.n_wg, 1))) return r;
+    if ((r = dev_alloc(c, &s.n_wg, 4))) return r;
     s.hist_cap = ((cap + 1023) / 1024) * E;
     if ((r = dev_alloc(c, &s.hist, s.hist_cap))) return r;
     if ((r = dev_alloc(c, &s.h, cap * c->F))) return r;
-    if ((r = dev_alloc(c, &s.y, cap * c->H))) return r;
+    s.y_cap = cap * c->H;
+    if ((r = dev_alloc(c, &s.y, s.y_cap))) return r;
     s.cap_assign = cap;
+    if ((r = dev_alloc(c, &s.task_ctr, 6))) return r;
+    CK(cudaMemset(s.task_ctr, 0, 6 * sizeof(int32_t)));
     return MPE_OK;
 }
 
@@ -332,6 +335,11 @@ void mpe_destroy(mpe_ctx* c) {
         cudaFreeHost(c->h_pte_pinned); cudaFreeHost(c->h_pidx_pinned);
         cudaFreeHost(c->h_list_pinned); cudaFreeHost(c->h_masters_pinned);
         if (c->upload_done) cudaEventDestroy(c->upload_done);
+        for (const ProfileRecord& r : c->prof) {
+            cudaEventDestroy(r.start);
+            cudaEventDestroy(r.stop);
+        }
+        for (cudaEvent_t e : c->event_pool) cudaEventDestroy(e);
         cudaGetLastError();
     }
     delete c;
@@ -454,16 +462,81 @@ int mpe_repage(mpe_ctx* c, uint64_t B_bits, const double* p, int32_t* n_changed_
     return MPE_OK;
 }
 
+static cudaEvent_t take_event(mpe_ctx* c) {
+    if (!c->event_pool.empty()) {
+        cudaEvent_t e = c->event_pool.back();
+        c->event_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+}
+
+// Brackets one kernel launch with an event pair when tracing is on.
+struct KernelSpan {
+    mpe_ctx* c;
+    ProfileRecord r{};
+    KernelSpan(mpe_ctx* ctx, int slot) : c(ctx) {
+        if (!c->profiling) return;
+        r.slot = slot;
+        r.start = take_event(c);
+        r.stop = take_event(c);
+        cudaEventRecord(r.start, c->stream);
+    }
+    ~KernelSpan() {
+        if (!c->profiling || !r.start) return;
+        cudaEventRecord(r.stop, c->stream);
+        c->prof.push_back(r);
+    }
+};
+
 static int moe_ffn_device(mpe_ctx* c, const void* x, int32_t T, const int32_t* ids,
                           const float* w, int32_t k, void* out) {
     const size_t Tk = (size_t)T * k;
     int r;
     if ((r = ensure_scratch(c, Tk))) return r;
-    launch_route(c, ids, (int)Tk, k, c->s.perm, c->s.offsets, c->s.inv, kDecodeGroup);
-    const int bound = wg_capacity(c->E, Tk, kDecodeGroup);
-    launch_decode_gateup(c, reinterpret_cast<const __nv_bfloat16*>(x), k, bound);
-    launch_decode_down(c, w, bound);
-    launch_combine(c, ids, T, k, reinterpret_cast<__nv_bfloat16*>(out));
+    {
+        KernelSpan sp(c, 0);
+        launch_route(c, ids, (int)Tk, k, c->s.perm, c->s.offsets, c->s.inv, kDecodeGroup);
+    }
+    DecodePlan pl;
+    decode_plan(c, Tk, pl);
+    const size_t need_part = pl.p_gu > 1 ? (size_t)pl.p_gu * 2 * Tk * c->F : 0;
+    if (need_part > c->s.part_cap) {
+        CK(cudaStreamSynchronize(c->stream));
+        cudaFree(c->s.part);
+        c->s.part = nullptr;
+        c->s.part_cap = 0;
+        if ((r = dev_alloc(c, &c->s.part, need_part))) return r;
+        c->s.part_cap = need_part;
+    }
+    const size_t need_y = (size_t)pl.p_dn * Tk * c->H;
+    if (need_y > c->s.y_cap) {
+        CK(cudaStreamSynchronize(c->stream));
+        cudaFree(c->s.y);
+        c->s.y = nullptr;
+        c->s.y_cap = 0;
+        if ((r = dev_alloc(c, &c->s.y, need_y))) return r;
+        c->s.y_cap = need_y;
+    }
+    {
+        KernelSpan sp(c, 1);
+        launch_decode_gateup(c, reinterpret_cast<const __nv_bfloat16*>(x), k, Tk, pl.p_gu,
+                             pl.kb_gu, pl.claim);
+    }
+    if (pl.p_gu > 1) {
+        KernelSpan sp(c, 2);
+        launch_swiglu_reduce(c, Tk, pl.p_gu);
+    }
+    {
+        KernelSpan sp(c, 3);
+        launch_decode_down(c, w, Tk, pl.p_dn, pl.kb_dn, pl.claim);
+    }
+    {
+        KernelSpan sp(c, 4);
+        launch_combine(c, ids, T, k, pl.p_dn, reinterpret_cast<__nv_bfloat16*>(out));
+    }
     CKLAUNCH();
     return MPE_OK;
 }
@@ -584,6 +657,40 @@ int mpe_get_scales(mpe_ctx* c, float* scale_host, float* absmax_host) {
 int mpe_get_bits(mpe_ctx* c, uint8_t* bits_host) {
     if (!c || !bits_host) return fail_global(MPE_ERR_INVALID, "null argument");
     std::memcpy(bits_host, c->bits.data(), c->E);
+    return MPE_OK;
+}
+
+int mpe_profile_enable(mpe_ctx* c, int32_t enable) {
+    if (!c) return fail_global(MPE_ERR_INVALID, "null context");
+    c->profiling = enable != 0;
+    return MPE_OK;
+}
+
+int mpe_profile_read(mpe_ctx* c, double* ms_host, int64_t* launches_host, int32_t n_slots,
+                     int32_t reset) {
+    if (!c) return fail_global(MPE_ERR_INVALID, "null context");
+    if (n_slots < 0) return fail(c, MPE_ERR_INVALID, "n_slots < 0");
+    DeviceGuard guard(c->device);
+    CK(cudaStreamSynchronize(c->stream));
+    std::vector<double> ms(kProfileSlots, 0.0);
+    std::vector<int64_t> cnt(kProfileSlots, 0);
+    for (const ProfileRecord& r : c->prof) {
+        float t = 0.0f;
+        CK(cudaEventElapsedTime(&t, r.start, r.stop));
+        ms[r.slot] += t;
+        cnt[r.slot] += 1;
+    }
+    for (int i = 0; i < n_slots; ++i) {
+        if (ms_host) ms_host[i] = i < kProfileSlots ? ms[i] : 0.0;
+        if (launches_host) launches_host[i] = i < kProfileSlots ? cnt[i] : 0;
+    }
+    if (reset) {
+        for (const ProfileRecord& r : c->prof) {
+            c->event_pool.push_back(r.start);
+            c->event_pool.push_back(r.stop);
+        }
+        c->prof.clear();
+    }
     return MPE_OK;
 }
 

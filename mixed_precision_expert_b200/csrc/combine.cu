@@ -1,13 +1,38 @@
-// Top-k weighted combine: out[t] = bf16( sum_j y[t*k + j] ), the slots summed in
-// order j = 0..k-1 in fp32 (the down kernel already applied w[t, j]); slots with
-// an id outside [0, E) contribute nothing. Deterministic: no atomics.
+// Top-k weighted combine: out[t] = bf16( sum_j sum_p y[p][t*k + j] ), summed in
+// fp32 with slots j = 0..k-1 outermost and K parts p = 0..P-1 inside (the down
+// kernel already applied w[t, j] and the scale); slots with an id outside
+// [0, E) contribute nothing. Deterministic: no atomics.
+//
+// SwiGLU reduce (gate/up split over K): h[pos][f] = bf16( silu(g) v ) with
+// g = sum_p gv[p][pos][0][f], v = sum_p gv[p][pos][1][f] (already scaled).
+#include <algorithm>
+
 #include "internal.h"
 
 namespace mpe {
 namespace {
 
 __global__ void __launch_bounds__(256)
-k_combine(const float* y, const int32_t* ids, int T, int k, int H, int E, __nv_bfloat16* out) {
+k_swiglu_reduce(const float* gv, const int32_t* offsets, int E, int F, int parts,
+                size_t part_stride, __nv_bfloat16* h) {
+    const int n_pos = offsets[E];
+    const size_t total = (size_t)n_pos * F;
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+         i += (size_t)gridDim.x * blockDim.x) {
+        const size_t pos = i / F, f = i - pos * F;
+        float g = 0.0f, v = 0.0f;
+        for (int p = 0; p < parts; ++p) {
+            const float* src = gv + (size_t)p * part_stride + pos * 2 * F + f;
+            g += src[0];
+            v += src[F];
+        }
+        h[pos * F + f] = __float2bfloat16_rn(g / (1.0f + __expf(-g)) * v);
+    }
+}
+
+__global__ void __launch_bounds__(256)
+k_combine(const float* y, const int32_t* ids, int T, int k, int H, int E, int parts,
+          size_t part_stride, __nv_bfloat16* out) {
     const int t = blockIdx.x;
     const int n4 = H / 4;
     for (int i = blockIdx.y * blockDim.x + threadIdx.x; i < n4; i += gridDim.y * blockDim.x) {
@@ -15,11 +40,14 @@ k_combine(const float* y, const int32_t* ids, int T, int k, int H, int E, __nv_b
         for (int j = 0; j < k; ++j) {
             const int e = ids[t * k + j];
             if (e < 0 || e >= E) continue;
-            const float4 v = reinterpret_cast<const float4*>(y + (size_t)(t * k + j) * H)[i];
-            acc.x += v.x;
-            acc.y += v.y;
-            acc.z += v.z;
-            acc.w += v.w;
+            for (int p = 0; p < parts; ++p) {
+                const float4 v = reinterpret_cast<const float4*>(y + (size_t)p * part_stride +
+                                                                 (size_t)(t * k + j) * H)[i];
+                acc.x += v.x;
+                acc.y += v.y;
+                acc.z += v.z;
+                acc.w += v.w;
+            }
         }
         __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
         __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
@@ -32,10 +60,20 @@ k_combine(const float* y, const int32_t* ids, int T, int k, int H, int E, __nv_b
 
 }  // namespace
 
-void launch_combine(mpe_ctx* c, const int32_t* ids, int T, int k, __nv_bfloat16* out) {
+void launch_swiglu_reduce(mpe_ctx* c, size_t Tk, int parts) {
+    const size_t total = Tk * c->F;
+    const int grid = (int)std::min<size_t>((total + 255) / 256, 148 * 8);
+    k_swiglu_reduce<<<grid, 256, 0, c->stream>>>(c->s.part, c->s.offsets, c->E, c->F, parts,
+                                                 (size_t)2 * Tk * c->F, c->s.h);
+    c->launches++;
+}
+
+void launch_combine(mpe_ctx* c, const int32_t* ids, int T, int k, int parts,
+                    __nv_bfloat16* out) {
     const int n4 = c->H / 4;
     dim3 grid((unsigned)T, (unsigned)((n4 + 255) / 256));
-    k_combine<<<grid, 256, 0, c->stream>>>(c->s.y, ids, T, k, c->H, c->E, out);
+    k_combine<<<grid, 256, 0, c->stream>>>(c->s.y, ids, T, k, c->H, c->E, parts,
+                                           (size_t)T * k * c->H, out);
     c->launches++;
 }
 

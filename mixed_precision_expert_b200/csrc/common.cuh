@@ -117,16 +117,24 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
         : "memory");
 }
 
+// One potentially-blocking test of an mbarrier phase: the hardware suspends
+// the thread until the phase completes or the suspend hint (ns) runs out, so
+// waiting warps do not spin on the issue slots.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(1000000u)
         : "memory");
     return ok != 0;
+}
+
+// Plain arrive (no transaction bytes).
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 // Wait for phase `parity` of an mbarrier, giving up after kWaitLimitNs.
@@ -145,7 +153,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1,
                                                uint32_t a2, uint32_t a3, uint32_t b0,
                                                uint32_t b1) {
-    asm volatile(
+    asm(
         "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
         "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
@@ -159,17 +167,36 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint3
 // ---------------------------------------------------------------------------
 constexpr uint32_t kMagic = 0x43004300u;  // bf16x2 (128, 128)
 
+// d = (a & mask) | magic, one lop3 (truth table 0xEA = (A & B) | C)
+__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t mask, uint32_t magic) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(mask), "r"(magic));
+    return d;
+}
+
+// d = (~a & mask) | magic, one lop3 (truth table 0xAE = (~A & B) | C)
+__device__ __forceinline__ uint32_t andnot_or(uint32_t a, uint32_t mask, uint32_t magic) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xAE;" : "=r"(d) : "r"(a), "r"(mask), "r"(magic));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t shr(uint32_t a, uint32_t n) {
+    uint32_t d;
+    asm("shr.b32 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(n));
+    return d;
+}
+
 __device__ __forceinline__ uint32_t bf2_sub(uint32_t a, uint32_t c) {
-    __nv_bfloat162 r = __hsub2(*reinterpret_cast<__nv_bfloat162*>(&a),
-                               *reinterpret_cast<__nv_bfloat162*>(&c));
-    return *reinterpret_cast<uint32_t*>(&r);
+    uint32_t d;
+    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(c));
+    return d;
 }
 
 __device__ __forceinline__ uint32_t bf2_fma(uint32_t a, uint32_t m, uint32_t c) {
-    __nv_bfloat162 r = __hfma2(*reinterpret_cast<__nv_bfloat162*>(&a),
-                               *reinterpret_cast<__nv_bfloat162*>(&m),
-                               *reinterpret_cast<__nv_bfloat162*>(&c));
-    return *reinterpret_cast<uint32_t*>(&r);
+    uint32_t d;
+    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(m), "r"(c));
+    return d;
 }
 
 // bf16 bit patterns used by the unpack
@@ -186,31 +213,33 @@ __device__ __forceinline__ uint32_t unpack_pair(const uint32_t* w, int m);
 
 template <>
 __device__ __forceinline__ uint32_t unpack_pair<4>(const uint32_t* w, int m) {
-    const uint32_t v = w[m >> 2] >> (4 * (m & 3));
-    return bf2_sub((v & 0x000F000Fu) | kMagic, kBf2_136);
+    const uint32_t v = (m & 3) ? shr(w[m >> 2], 4 * (m & 3)) : w[m >> 2];
+    return bf2_sub(and_or(v, 0x000F000Fu, kMagic), kBf2_136);
 }
 
 template <>
 __device__ __forceinline__ uint32_t unpack_pair<8>(const uint32_t* w, int m) {
-    const uint32_t v = w[m >> 1] >> (8 * (m & 1));
-    const uint32_t lo = (v & 0x007F007Fu) | kMagic;   // 128 + (u & 127)
-    const uint32_t hi = (~v & 0x00800080u) | kMagic;  // 256 - 128 * bit7(u)
-    return bf2_sub(lo, hi);                            // u - 128 = k
+    const uint32_t v = (m & 1) ? shr(w[m >> 1], 8) : w[m >> 1];
+    const uint32_t lo = and_or(v, 0x007F007Fu, kMagic);   // 128 + (u & 127)
+    const uint32_t hi = andnot_or(v, 0x00800080u, kMagic);  // 256 - 128 * bit7(u)
+    return bf2_sub(lo, hi);                                // u - 128 = k
 }
 
 template <>
 __device__ __forceinline__ uint32_t unpack_pair<3>(const uint32_t* w, int m) {
     if (m == 15) {
-        const uint32_t t = ((w[0] >> 15) & 0x00010001u) | ((w[1] >> 14) & 0x00020002u) |
-                           ((w[2] >> 13) & 0x00040004u) | kMagic;
+        uint32_t t = and_or(shr(w[0], 15), 0x00010001u, kMagic);
+        t = and_or(shr(w[1], 14), 0x00020002u, t);
+        t = and_or(shr(w[2], 13), 0x00040004u, t);
         return bf2_sub(t, kBf2_132);
     }
     const int v = m / 5, f = m % 5;
-    const uint32_t x = w[v] >> (f < 2 ? 0 : (f < 4 ? 6 : 12));
+    const int sh = f < 2 ? 0 : (f < 4 ? 6 : 12);
+    const uint32_t x = sh ? shr(w[v], sh) : w[v];
     if (f == 1 || f == 3) {
-        return bf2_fma((x & 0x00380038u) | kMagic, kBf2_eighth, kBf2_m20);  // (128+8u)/8 - 20
+        return bf2_fma(and_or(x, 0x00380038u, kMagic), kBf2_eighth, kBf2_m20);  // (128+8u)/8 - 20
     }
-    return bf2_sub((x & 0x00070007u) | kMagic, kBf2_132);  // 128 + u - 132
+    return bf2_sub(and_or(x, 0x00070007u, kMagic), kBf2_132);  // 128 + u - 132
 }
 
 }  // namespace mpe

@@ -21,17 +21,28 @@ struct Scratch {
     int32_t* inv = nullptr;
     int32_t* offsets = nullptr;  // E+1
     int32_t* wg = nullptr;       // work groups: 3 ints each
-    int32_t* n_wg = nullptr;
+    int32_t* n_wg = nullptr;     // {total, 8-bit, 4-bit, 3-bit} work groups
     int32_t* hist = nullptr;     // per-chunk histograms (large-T route)
     size_t hist_cap = 0;
     __nv_bfloat16* h = nullptr;  // [cap_assign x F]
-    float* y = nullptr;          // [cap_assign x H]
+    float* y = nullptr;          // [P][T*k][H] down outputs (P K-part slices)
+    float* part = nullptr;       // gate/up split-K partials [P][T*k][2][F]
+    size_t part_cap = 0;         // floats
+    size_t y_cap = 0;            // floats in y (P slices of T*k x H)
+    int32_t* task_ctr = nullptr; // 6 task counters (3 classes x 2 kernels), zeroed by route
     // staging for the host-buffer entry point
     size_t stage_tokens = 0;
     void* x_stage = nullptr;
     int32_t* ids_stage = nullptr;
     float* w_stage = nullptr;
     void* out_stage = nullptr;
+};
+
+// CUDA-event records around the forward-pass kernels (optional tracing).
+constexpr int kProfileSlots = 5;  // route, gate/up, swiglu reduce, down, combine
+struct ProfileRecord {
+    int slot;
+    cudaEvent_t start, stop;
 };
 
 struct HostAllocator {
@@ -82,6 +93,11 @@ struct mpe_ctx {
     bool absmax_valid = false;
     mpe::HostAllocator alloc;
     mpe::Scratch s;
+
+    // tracing
+    bool profiling = false;
+    std::vector<mpe::ProfileRecord> prof;
+    std::vector<cudaEvent_t> event_pool;
 };
 
 namespace mpe {
@@ -102,12 +118,21 @@ void launch_allocate(cudaStream_t st, const double* p, const uint64_t* W, int E,
 // route.cu
 void launch_route(mpe_ctx* c, const int32_t* ids, int Tk, int k, int32_t* perm,
                   int32_t* offsets, int32_t* inv, int group);
+// zero-on-route counters: the route kernel clears task_ctr[0..1]
 
 // decode.cu
-void launch_decode_gateup(mpe_ctx* c, const __nv_bfloat16* x, int k, int wg_bound);
-void launch_decode_down(mpe_ctx* c, const float* topk_w, int wg_bound);
+struct DecodePlan {
+    int p_gu = 1, kb_gu = 1, p_dn = 1, kb_dn = 1, claim = 1;
+};
+void decode_plan(mpe_ctx* c, size_t Tk, DecodePlan& pl);
+void launch_decode_gateup(mpe_ctx* c, const __nv_bfloat16* x, int k, size_t Tk, int parts,
+                          int kb, int claim);
+void launch_decode_down(mpe_ctx* c, const float* topk_w, size_t Tk, int parts, int kb,
+                        int claim);
 
 // combine.cu
-void launch_combine(mpe_ctx* c, const int32_t* ids, int T, int k, __nv_bfloat16* out);
+void launch_swiglu_reduce(mpe_ctx* c, size_t Tk, int parts);
+void launch_combine(mpe_ctx* c, const int32_t* ids, int T, int k, int parts,
+                    __nv_bfloat16* out);
 
 }  // namespace mpe

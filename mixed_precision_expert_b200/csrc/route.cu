@@ -48,27 +48,47 @@ __device__ uint64_t block_exclusive_scan(uint64_t v, uint64_t* s_warp, uint64_t*
 }
 
 // Offsets and work groups from per-expert counts (thread e holds count[e]).
-__device__ void offsets_and_groups(int E, int cnt, int group, int32_t* offsets, int32_t* wg,
-                                   int32_t* n_wg, int32_t* s_off) {
+// Work groups are listed by width class of their expert -- 8-bit, then 4-bit,
+// then 3-bit -- so each decode loop runs one specialised code path;
+// n_wg = {total, class 8, class 4, class 3}.
+__device__ void offsets_and_groups(int E, int cnt, int group, const Pte* pte, int32_t* offsets,
+                                   int32_t* wg, int32_t* n_wg, int32_t* s_off) {
     __shared__ uint64_t s_warp[32];
     const int e = threadIdx.x;
-    const int ng = (e < E) ? (cnt + group - 1) / group : 0;
-    const uint64_t packed = ((uint64_t)(e < E ? cnt : 0) << 32) | (uint64_t)ng;
+    const int c = (e < E) ? cnt : 0;
     uint64_t total;
-    const uint64_t ex = block_exclusive_scan(packed, s_warp, &total);
-    const int off = (int)(ex >> 32), goff = (int)(ex & 0xFFFFFFFFu);
+    const int off = (int)block_exclusive_scan((uint64_t)c, s_warp, &total);
+    const int n_assign = (int)total;
+    int cls = -1;
+    if (e < E) {
+        const int b = pte[e].bits;
+        cls = b == 8 ? 0 : (b == 4 ? 1 : (b == 3 ? 2 : -1));
+    }
+    const int ng = (cls >= 0) ? (c + group - 1) / group : 0;
+    const uint64_t packed = cls < 0 ? 0ull : ((uint64_t)ng << (21 * cls));
+    uint64_t gtot;
+    const uint64_t gex = block_exclusive_scan(packed, s_warp, &gtot);
+    const int t8 = (int)(gtot & 0x1FFFFF), t4 = (int)((gtot >> 21) & 0x1FFFFF),
+              t3 = (int)((gtot >> 42) & 0x1FFFFF);
     if (e < E) {
         offsets[e] = off;
         s_off[e] = off;
-        for (int i = 0; i < ng; ++i) {
-            wg[3 * (goff + i) + 0] = e;
-            wg[3 * (goff + i) + 1] = off + i * group;
-            wg[3 * (goff + i) + 2] = min(group, cnt - i * group);
+        if (cls >= 0) {
+            const int start = cls == 0 ? 0 : (cls == 1 ? t8 : t8 + t4);
+            const int goff = start + (int)((gex >> (21 * cls)) & 0x1FFFFF);
+            for (int i = 0; i < ng; ++i) {
+                wg[3 * (goff + i) + 0] = e;
+                wg[3 * (goff + i) + 1] = off + i * group;
+                wg[3 * (goff + i) + 2] = min(group, c - i * group);
+            }
         }
     }
     if (e == 0) {
-        offsets[E] = (int)(total >> 32);
-        *n_wg = (int)(total & 0xFFFFFFFFu);
+        offsets[E] = n_assign;
+        n_wg[0] = t8 + t4 + t3;
+        n_wg[1] = t8;
+        n_wg[2] = t4;
+        n_wg[3] = t3;
     }
 }
 
@@ -103,8 +123,10 @@ __device__ void scatter_chunk(const int32_t* ids, int a0, int n, int E, const in
 
 // T*k <= 1024: everything in one CTA.
 __global__ void __launch_bounds__(kChunk)
-k_route_small(const int32_t* ids, int Tk, int E, int group, int32_t* perm, int32_t* offsets,
-              int32_t* inv, int32_t* wg, int32_t* n_wg, uint32_t* status) {
+k_route_small(const int32_t* ids, int Tk, int E, int group, const Pte* pte, int32_t* perm,
+              int32_t* offsets, int32_t* inv, int32_t* wg, int32_t* n_wg, uint32_t* status,
+              int32_t* zero6) {
+    if (threadIdx.x < 6 && zero6) zero6[threadIdx.x] = 0;
     extern __shared__ __align__(16) uint8_t sm[];
     int32_t* s_cnt = reinterpret_cast<int32_t*>(sm);       // [E]
     int32_t* s_off = s_cnt + MPE_MAX_EXPERTS;               // [E]
@@ -118,7 +140,7 @@ k_route_small(const int32_t* ids, int Tk, int E, int group, int32_t* perm, int32
     }
     __syncthreads();
     const int cnt = threadIdx.x < E ? s_cnt[threadIdx.x] : 0;
-    offsets_and_groups(E, cnt, group, offsets, wg, n_wg, s_off);
+    offsets_and_groups(E, cnt, group, pte, offsets, wg, n_wg, s_off);
     __syncthreads();
     scatter_chunk(ids, 0, Tk, E, s_off, wcnt, perm, inv, status);
 }
@@ -140,8 +162,9 @@ k_route_hist(const int32_t* ids, int Tk, int E, int32_t* hist) {
 
 // Step 2 (one CTA): hist[c][e] <- first position of chunk c's id-e assignments.
 __global__ void __launch_bounds__(kChunk)
-k_route_scan(int32_t* hist, int n_chunks, int E, int group, int32_t* offsets, int32_t* wg,
-             int32_t* n_wg) {
+k_route_scan(int32_t* hist, int n_chunks, int E, int group, const Pte* pte, int32_t* offsets,
+             int32_t* wg, int32_t* n_wg, int32_t* zero6) {
+    if (threadIdx.x < 6 && zero6) zero6[threadIdx.x] = 0;
     __shared__ int32_t s_off[MPE_MAX_EXPERTS];
     const int e = threadIdx.x;
     int run = 0;
@@ -152,7 +175,7 @@ k_route_scan(int32_t* hist, int n_chunks, int E, int group, int32_t* offsets, in
             run += h;
         }
     }
-    offsets_and_groups(E, run, group, offsets, wg, n_wg, s_off);
+    offsets_and_groups(E, run, group, pte, offsets, wg, n_wg, s_off);
     __syncthreads();
     if (e < E) {
         const int off = s_off[e];
@@ -181,15 +204,16 @@ void launch_route(mpe_ctx* c, const int32_t* ids, int Tk, int k, int32_t* perm,
     const int E = c->E;
     if (Tk <= kChunk) {
         const size_t sm = 2 * MPE_MAX_EXPERTS * sizeof(int32_t) + 32 * E * sizeof(uint16_t);
-        k_route_small<<<1, kChunk, sm, c->stream>>>(ids, Tk, E, group, perm, offsets, inv,
-                                                    c->s.wg, c->s.n_wg, c->d_status);
+        k_route_small<<<1, kChunk, sm, c->stream>>>(ids, Tk, E, group, c->d_pte, perm, offsets,
+                                                    inv, c->s.wg, c->s.n_wg, c->d_status,
+                                                    c->s.task_ctr);
         c->launches++;
         return;
     }
     const int nch = (Tk + kChunk - 1) / kChunk;
     k_route_hist<<<nch, kChunk, 0, c->stream>>>(ids, Tk, E, c->s.hist);
-    k_route_scan<<<1, kChunk, 0, c->stream>>>(c->s.hist, nch, E, group, offsets, c->s.wg,
-                                              c->s.n_wg);
+    k_route_scan<<<1, kChunk, 0, c->stream>>>(c->s.hist, nch, E, group, c->d_pte, offsets,
+                                              c->s.wg, c->s.n_wg, c->s.task_ctr);
     const size_t sm = 32 * E * sizeof(uint16_t);
     k_route_scatter<<<nch, kChunk, sm, c->stream>>>(ids, Tk, E, c->s.hist, perm, inv,
                                                     c->d_status);

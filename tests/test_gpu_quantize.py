@@ -99,7 +99,7 @@ def test_quantize_small_pages_every_width(page_bytes):
     bits = np.array([3, 4, 8, 8, 3, 4], np.uint8)
     masters = [synth.expert_weights(wl, e, device="cuda") for e in range(wl.E)]
     cpu = [m.cpu().numpy() for m in masters]
-    pool = 200
+    pool = 400  # 274 pages at 4 KiB: 29 + 36 + 72 + 72 + 29 + 36
     ctx = mpe.Context(wl.E, wl.H, wl.F, page_bytes=page_bytes, pool_pages=pool)
     ctx.quantize_experts(masters, bits)
     alloc = op.PageAllocator(pool, wl.E, wl.H, wl.F, page_bytes=page_bytes)

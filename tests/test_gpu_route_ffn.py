@@ -62,6 +62,8 @@ def _layer(wl, bits=None, device="cuda", path=0):
 def _run(ctx, x, ids, w):
     out = ctx.moe_ffn(x.cuda(), torch.from_numpy(ids).cuda(), torch.from_numpy(w).cuda())
     torch.cuda.synchronize()
+    # no bounded device wait may have run out (that would mean a lost stage)
+    assert not (ctx.status() & mpe.STATUS_WAIT_TIMEOUT)
     return out.double().cpu().numpy()
 
 
