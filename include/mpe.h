@@ -197,6 +197,32 @@ int mpe_route(mpe_ctx* ctx, const int32_t* ids, int32_t T, int32_t k, int32_t* p
               int32_t* offsets, int32_t* inv);
 
 /*
+ * mpe_route_noalloc -- the same bucketing as mpe_route (perm, offsets, inv;
+ * identical results) for callers that cannot allocate device memory when they
+ * route: a serving engine that fixes its GPU memory plan up front, or code
+ * running while another component owns the allocator. It needs no context and
+ * allocates nothing (no cudaMalloc, cudaFree or allocating library routine);
+ * its working memory is one file-scope device array that every GPU loading the
+ * library keeps until the process exits. The pages have no counterpart for
+ * this call: it is an engineering variant of mpe_route.
+ *   ids      device, int32 [T*k]; ids outside [0,E) are dropped (inv = -1)
+ *   T, k     tokens and slots per token, 1 <= k <= 32; T*k <= 65536
+ *   E        experts, 1 .. MPE_MAX_EXPERTS
+ *   perm     device, int32 [T*k]; offsets device, int32 [E+1];
+ *   inv      device, int32 [T*k]
+ *   stream   cudaStream_t (NULL = the legacy default stream)
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture. All calls on a device share the array: calls that overlap on the
+ * GPU (different streams, no ordering between them) race and must not be
+ * issued. Asynchronous. With T*k = 0 only offsets is written (all zero) and
+ * ids, perm, inv may be NULL. MPE_ERR_INVALID (message in
+ * mpe_last_error_global) for a null pointer, a bad E/T/k or T*k above 65536.
+ */
+int mpe_route_noalloc(const int32_t* ids, int32_t T, int32_t k, int32_t E, int32_t* perm,
+                      int32_t* offsets, int32_t* inv, void* stream);
+
+/*
  * mpe_get_page_table -- copy the page table to host: pte_host mpe_pte[E] and
  * page_idx_host uint32[cap] (the compact page-index array; its length is the
  * sum of n_pages). Either pointer may be NULL. Synchronous.

@@ -40,7 +40,7 @@ EXPORTS = [
     "mpe_get_page_table", "mpe_expert_stream_bytes", "mpe_read_expert_packed",
     "mpe_get_scales", "mpe_get_bits", "mpe_get_status", "mpe_last_error",
     "mpe_last_error_global", "mpe_kernel_launches", "mpe_version", "mpe_profile_enable",
-    "mpe_profile_read",
+    "mpe_profile_read", "mpe_route_noalloc",
 ]
 PROFILE_SLOTS = ["route", "gate_up", "swiglu_reduce", "down", "combine"]
 
@@ -104,6 +104,7 @@ def lib() -> ctypes.CDLL:
         "mpe_version": (i32, []),
         "mpe_profile_enable": (i32, [vp, i32]),
         "mpe_profile_read": (i32, [vp, vp, vp, i32, i32]),
+        "mpe_route_noalloc": (i32, [vp, i32, i32, i32, vp, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -142,6 +143,14 @@ def allocate_bits(p, W, B: int) -> np.ndarray:
     out = np.zeros(len(p), dtype=np.uint8)
     _check(lib().mpe_allocate_bits(_ptr(p), _ptr(W), len(p), int(B), _ptr(out)))
     return out
+
+
+def route_noalloc(ids, E: int, perm, offsets, inv):
+    """Bucketing into caller-provided device buffers without any device
+    allocation (mpe_route_noalloc); runs on the current stream."""
+    T, k = ids.shape
+    _check(lib().mpe_route_noalloc(_ptr(ids), T, k, E, _ptr(perm), _ptr(offsets), _ptr(inv),
+                                   _stream()))
 
 
 class Context:

@@ -241,6 +241,11 @@ int run_allocate(mpe_ctx* c, const double* p, uint64_t B, std::vector<uint8_t>& 
 
 }  // namespace
 
+namespace mpe {
+// Records a message for mpe_last_error_global (context-free calls in other files).
+int report_global_error(int code, const char* msg) { return fail_global(code, "%s", msg); }
+}  // namespace mpe
+
 extern "C" {
 
 int32_t mpe_version(void) { return 100; }

@@ -13,6 +13,9 @@
 // Stable ranks come from warp matching: inside a warp, lanes holding the same
 // id rank by lane; across warps, by the per-warp counts of earlier warps;
 // across 1024-assignment chunks, by the per-chunk histograms.
+#include <cstdio>
+#include <mutex>
+
 #include "internal.h"
 
 namespace mpe {
@@ -228,3 +231,116 @@ void route_set_smem_limits() {
 }
 
 }  // namespace mpe
+
+// ---------------------------------------------------------------------------
+// No-allocation variant of the bucketing step (mpe_route_noalloc).
+//
+// Some callers cannot allocate device memory at the point where they route
+// tokens: a serving engine that hands the GPU a fixed memory plan up front, or
+// code recorded while another component owns the allocator. For them the
+// multi-chunk histograms live in one file-scope device array instead of
+// context scratch. The array holds up to kNoAllocMaxAssign assignments
+// (64 chunks of 1024) for up to MPE_MAX_EXPERTS experts; every GPU that loads
+// the library keeps it until the process exits.
+// ---------------------------------------------------------------------------
+namespace mpe {
+int report_global_error(int code, const char* msg);
+
+namespace {
+
+constexpr int kNoAllocMaxAssign = 65536;
+constexpr int kNoAllocChunks = kNoAllocMaxAssign / kChunk;
+constexpr size_t kNaHistBytes = sizeof(int32_t) * (size_t)kNoAllocChunks * MPE_MAX_EXPERTS;
+constexpr size_t kNaWgBytes =
+    sizeof(int32_t) * 3 * ((size_t)MPE_MAX_EXPERTS + kNoAllocMaxAssign / kDecodeGroup + 1);
+constexpr size_t kNaSmallBytes = 256;  // work-group counts and a status word
+constexpr size_t kNaPteBytes = sizeof(Pte) * MPE_MAX_EXPERTS;
+constexpr size_t kNaBytes = kNaHistBytes + kNaWgBytes + kNaSmallBytes + kNaPteBytes;
+
+// Shared by every call on a device; the histograms are fully rewritten by each
+// call before they are read, and the page-table region is never written (all
+// widths 0, so no decode work groups are formed).
+static __device__ __align__(256) unsigned char g_route_scratch[kNaBytes];
+
+std::mutex g_noalloc_mu;
+constexpr int kMaxDevices = 64;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of the array on the current device (host code may only use
+// the symbol through cudaGetSymbolAddress); set up once per device.
+int noalloc_scratch(unsigned char** out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return report_global_error(MPE_ERR_CUDA, "mpe_route_noalloc: no usable device");
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_addr[dev]) {
+        void* p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_route_scratch);
+        if (e != cudaSuccess) {
+            char buf[256];
+            snprintf(buf, sizeof(buf), "mpe_route_noalloc: cudaGetSymbolAddress failed: %s",
+                     cudaGetErrorString(e));
+            return report_global_error(MPE_ERR_CUDA, buf);
+        }
+        route_set_smem_limits();
+        if (cudaGetLastError() != cudaSuccess)
+            return report_global_error(MPE_ERR_CUDA, "mpe_route_noalloc: kernel setup failed");
+        g_noalloc_addr[dev] = p;
+    }
+    *out = static_cast<unsigned char*>(g_noalloc_addr[dev]);
+    return MPE_OK;
+}
+
+}  // namespace
+}  // namespace mpe
+
+extern "C" int mpe_route_noalloc(const int32_t* ids, int32_t T, int32_t k, int32_t E,
+                                 int32_t* perm, int32_t* offsets, int32_t* inv, void* stream) {
+    using namespace mpe;
+    if (E < 1 || E > MPE_MAX_EXPERTS || T < 0 || k < 1 || k > 32)
+        return report_global_error(MPE_ERR_INVALID, "mpe_route_noalloc: bad E, T or k");
+    const long long Tk = (long long)T * k;
+    if (!offsets || (Tk > 0 && (!ids || !perm || !inv)))
+        return report_global_error(MPE_ERR_INVALID, "mpe_route_noalloc: null pointer");
+    if (Tk > kNoAllocMaxAssign) {
+        char buf[160];
+        snprintf(buf, sizeof(buf),
+                 "mpe_route_noalloc: T*k = %lld exceeds the no-allocation maximum of %d",
+                 Tk, kNoAllocMaxAssign);
+        return report_global_error(MPE_ERR_INVALID, buf);
+    }
+    unsigned char* base = nullptr;
+    int rc = noalloc_scratch(&base);
+    if (rc != MPE_OK) return rc;
+    int32_t* hist = reinterpret_cast<int32_t*>(base);
+    int32_t* wg = reinterpret_cast<int32_t*>(base + kNaHistBytes);
+    int32_t* n_wg = reinterpret_cast<int32_t*>(base + kNaHistBytes + kNaWgBytes);
+    uint32_t* status = reinterpret_cast<uint32_t*>(n_wg + 8);
+    const Pte* pte = reinterpret_cast<const Pte*>(base + kNaHistBytes + kNaWgBytes + kNaSmallBytes);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int n = (int)Tk;
+    if (n == 0) {
+        if (cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), st) != cudaSuccess)
+            return report_global_error(MPE_ERR_CUDA, "mpe_route_noalloc: memset failed");
+        return MPE_OK;
+    }
+    if (n <= kChunk) {
+        const size_t sm = 2 * MPE_MAX_EXPERTS * sizeof(int32_t) + 32 * E * sizeof(uint16_t);
+        k_route_small<<<1, kChunk, sm, st>>>(ids, n, E, kDecodeGroup, pte, perm, offsets, inv, wg,
+                                             n_wg, status, nullptr);
+    } else {
+        const int nch = (n + kChunk - 1) / kChunk;
+        k_route_hist<<<nch, kChunk, 0, st>>>(ids, n, E, hist);
+        k_route_scan<<<1, kChunk, 0, st>>>(hist, nch, E, kDecodeGroup, pte, offsets, wg, n_wg,
+                                           nullptr);
+        k_route_scatter<<<nch, kChunk, 32 * E * sizeof(uint16_t), st>>>(ids, n, E, hist, perm,
+                                                                         inv, status);
+    }
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        char buf[200];
+        snprintf(buf, sizeof(buf), "mpe_route_noalloc: launch failed: %s", cudaGetErrorString(e));
+        return report_global_error(MPE_ERR_CUDA, buf);
+    }
+    return MPE_OK;
+}
