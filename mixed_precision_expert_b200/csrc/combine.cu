@@ -30,32 +30,33 @@ k_swiglu_reduce(const float* gv, const int32_t* offsets, int E, int F, int parts
     }
 }
 
-__global__ void __launch_bounds__(256)
+// One thread per 4 columns of one token; a CTA covers 256 x 4 columns of one
+// token row (grid: tokens x column blocks).
+__global__ void __launch_bounds__(128)
 k_combine(const float* y, const int32_t* ids, int T, int k, int H, int E, int parts,
           size_t part_stride, __nv_bfloat16* out) {
     const int t = blockIdx.x;
-    const int n4 = H / 4;
-    for (int i = blockIdx.y * blockDim.x + threadIdx.x; i < n4; i += gridDim.y * blockDim.x) {
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int j = 0; j < k; ++j) {
-            const int e = ids[t * k + j];
-            if (e < 0 || e >= E) continue;
-            for (int p = 0; p < parts; ++p) {
-                const float4 v = reinterpret_cast<const float4*>(y + (size_t)p * part_stride +
-                                                                 (size_t)(t * k + j) * H)[i];
-                acc.x += v.x;
-                acc.y += v.y;
-                acc.z += v.z;
-                acc.w += v.w;
-            }
+    const int i = blockIdx.y * blockDim.x + threadIdx.x;  // float4 column index
+    if (i >= H / 4) return;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < k; ++j) {
+        const int e = ids[t * k + j];
+        if (e < 0 || e >= E) continue;
+        for (int p = 0; p < parts; ++p) {
+            const float4 v = reinterpret_cast<const float4*>(y + (size_t)p * part_stride +
+                                                             (size_t)(t * k + j) * H)[i];
+            acc.x += v.x;
+            acc.y += v.y;
+            acc.z += v.z;
+            acc.w += v.w;
         }
-        __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
-        __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
-        uint2 pk;
-        pk.x = *reinterpret_cast<uint32_t*>(&lo);
-        pk.y = *reinterpret_cast<uint32_t*>(&hi);
-        reinterpret_cast<uint2*>(out + (size_t)t * H)[i] = pk;
     }
+    __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+    __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+    uint2 pk;
+    pk.x = *reinterpret_cast<uint32_t*>(&lo);
+    pk.y = *reinterpret_cast<uint32_t*>(&hi);
+    reinterpret_cast<uint2*>(out + (size_t)t * H)[i] = pk;
 }
 
 }  // namespace
@@ -71,8 +72,8 @@ void launch_swiglu_reduce(mpe_ctx* c, size_t Tk, int parts) {
 void launch_combine(mpe_ctx* c, const int32_t* ids, int T, int k, int parts,
                     __nv_bfloat16* out) {
     const int n4 = c->H / 4;
-    dim3 grid((unsigned)T, (unsigned)((n4 + 255) / 256));
-    k_combine<<<grid, 256, 0, c->stream>>>(c->s.y, ids, T, k, c->H, c->E, parts,
+    dim3 grid((unsigned)T, (unsigned)((n4 + 127) / 128));
+    k_combine<<<grid, 128, 0, c->stream>>>(c->s.y, ids, T, k, c->H, c->E, parts,
                                            (size_t)T * k * c->H, out);
     c->launches++;
 }

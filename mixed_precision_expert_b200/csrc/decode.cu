@@ -7,18 +7,21 @@
 //   gate/up:  g = s_e (K1 x), v = s_e (K3 x), h = silu(g) v   (h stored bf16)
 //   down:     y_a = w_a s_e (K2 h_a)                          (y stored fp32)
 //
-// Work is cut into tasks (work group of <= 16 tokens of one expert, 16-row
-// output tile, K part); a persistent grid of warps claims tasks from a global
-// counter. Every warp streams its tasks' chunks (16 rows x 128 codes each)
-// through its own 3-stage shared-memory ring, filled by 1-D bulk copies
-// (cp.async.bulk, no multicast) that complete on mbarriers, and keeps the
-// ring full across task boundaries. Lanes unpack codes to exact bf16 integers
-// in registers (common.cuh) and feed mma.sync m16n8k16: weights are the
-// 16-row A operand, up to two 8-token n-tiles of activations are B, and the
-// per-expert scale multiplies the fp32 accumulator at the end. A task whose K
-// range is split in P parts writes fp32 partials; the last part to finish
-// (arrival counter per tile) sums the P partials in part order -- the result
-// does not depend on arrival order -- and applies the epilogue.
+// Warp-specialised persistent kernel. A CTA has 8 consumer warps and 1
+// producer warp and works on one task at a time: a work group (<= 16 tokens of
+// one expert) x 8 consecutive 16-row output tiles (one per consumer warp) x a
+// K part. The producer warp claims tasks from a per-width-class counter and,
+// for each block column j of the task, fills one slot of the CTA's
+// shared-memory ring with the 8 tiles' chunks (one 1-D bulk copy per tile and
+// matrix, issued by 8-16 producer lanes in parallel, no multicast; a full
+// mbarrier counts the bytes) and prefetches the block's activation lines into
+// L1. Consumer warps wait on the slot's full barrier, copy their chunk's words
+// to registers, release the slot on its empty barrier (8 arrivals) and only
+// then unpack (common.cuh) and multiply with mma.sync m16n8k16 -- weights are
+// the 16-row A operand, one or two 8-token n-tiles of activations are B, fp32
+// accumulate, the per-expert scale applied once at the end. A task whose K
+// range is split in P parts writes a scaled partial to its own slice; a later
+// pass sums the slices in part order (deterministic, no atomics).
 //
 // k-permutation: inside a 128-code block, thread t (= lane & 3) owns 16 code
 // pairs; mma step c (0..7) uses its pairs 2c and 2c+1 as the logical k-pairs
@@ -33,25 +36,25 @@
 namespace mpe {
 namespace {
 
-constexpr int kWarps = 4;
-constexpr int kStages = 3;
-constexpr int kStageBytes = 2048;  // per matrix per stage
+constexpr int kConsumers = 8;                    // consumer warps per CTA (one tile each)
+constexpr int kThreads = (kConsumers + 1) * 32;  // + the producer warp
+constexpr int kRingBytes = 96 * 1024;            // shared-memory ring per CTA
+constexpr int kMaxSlots = 16;
 constexpr int kMaxTiles = kDecodeGroup / 8;
 
-template <int B>
+template <int B, int NM>
 struct Geo {
-    static constexpr int CB = 256 * B;                           // chunk bytes
-    static constexpr int J = (2048 / CB) > 0 ? (2048 / CB) : 1;  // chunks per stage
-    static constexpr int WORDS = (B == 8) ? 8 : B;               // raw words per row
+    static constexpr int CB = 256 * B;                   // chunk bytes
+    static constexpr int TILE = NM * CB;                 // one warp's share of a slot
+    static constexpr int SLOT = kConsumers * TILE;       // one block column of 8 tiles
+    static constexpr int S = (kRingBytes / SLOT) < kMaxSlots ? (kRingBytes / SLOT) : kMaxSlots;
+    static constexpr int WORDS = (B == 8) ? 8 : B;       // raw words per row
+    static_assert(S >= 3, "ring geometry");
 };
 
-__host__ __device__ inline int stage_chunks(int b) { return b == 8 ? 1 : 2; }
-
-struct StageDesc {
-    int task;  // -1: no more work
-    int j0;
-    int nch;
-    int pad;
+struct SlotDesc {
+    int task;  // -1: no more tasks of this class
+    int j;     // block column held by the slot
 };
 
 struct Args {
@@ -69,35 +72,20 @@ struct Args {
     int32_t* task_ctr;         // claimed-task counters (one per class), zero at launch
     int parts;                 // P
     int kb;                    // blocks per part
-    int claim;                 // tasks claimed per atomic
     uint32_t* status;
 };
 
-__host__ __device__ constexpr size_t ring_bytes(int nm) { return (size_t)kWarps * kStages * nm * kStageBytes; }
-__host__ __device__ constexpr size_t smem_bytes(int nm);
-
-struct Task {
-    int gi, tau, p, e, pos0, ntok, bits, j_lo, j_hi;
-    float scale;
-};
-
-struct ProducerState {
-    int task, tau, j, j_hi, claim_left, done;
-    Pte pte;
-};
-
-__host__ __device__ constexpr size_t smem_bytes(int nm) {
-    return ring_bytes(nm) + kWarps * kStages * (sizeof(uint64_t) + sizeof(StageDesc)) +
-           kWarps * sizeof(ProducerState);
+__host__ __device__ constexpr size_t smem_bytes() {
+    return (size_t)kRingBytes + kMaxSlots * (2 * sizeof(uint64_t) + sizeof(SlotDesc));
 }
 
-// Task order: tile fastest, then K part, then work group, so tasks claimed
-// close together read the same activation K-range (L1 hits) and sweep one
+// CTA task order: tile group fastest, then K part, then work group, so tasks
+// claimed close together read the same activation K-range and sweep one
 // expert's pages.
-__device__ __forceinline__ void split_task(int task, int n_tiles, int parts, int& gi, int& tau,
+__device__ __forceinline__ void split_task(int task, int n_tq, int parts, int& gi, int& tq,
                                            int& p) {
-    tau = task % n_tiles;
-    const int u = task / n_tiles;
+    tq = task % n_tq;
+    const int u = task / n_tq;
     p = u % parts;
     gi = u / parts;
 }
@@ -105,7 +93,7 @@ __device__ __forceinline__ void split_task(int task, int n_tiles, int parts, int
 // Raw words of this thread's share of one row's block (chunk row `r`).
 template <int B>
 __device__ __forceinline__ void load_row_words(const uint8_t* chunk, int r, int t, int g,
-                                               uint32_t (&w)[Geo<B>::WORDS]) {
+                                               uint32_t (&w)[Geo<B, 1>::WORDS]) {
     const uint8_t* blk = chunk + r * block_bytes(B);
     if constexpr (B == 4) {
         const uint4 v = *reinterpret_cast<const uint4*>(blk + 16 * t);
@@ -142,47 +130,36 @@ __device__ __forceinline__ void load_act_half(const __nv_bfloat16* row, int j, i
     xb[4] = v1.x; xb[5] = v1.y; xb[6] = v1.z; xb[7] = v1.w;
 }
 
-// One stage: nch blocks (j0 ..) of NM matrices for the current task, with NT
-// 8-token n-tiles (compile-time, so no per-mma guards). Each block is done in
-// two halves (mma steps 0-3, then 4-7) to bound the live registers: the
-// second half's activations load while the first computes.
+// Unpack and multiply one block (128 codes of 16 rows, NM matrices) with NT
+// 8-token n-tiles of activations.
 template <int B, int NM, int NT>
-__device__ __forceinline__ void consume(const uint8_t* stage, int j0, int nch,
-                                        const __nv_bfloat16* const (&arow)[kMaxTiles], int g,
-                                        int t, float (&acc)[kMaxTiles][NM][4]) {
-    using G = Geo<B>;
-    for (int jj = 0; jj < nch; ++jj) {
-        const int j = j0 + jj;
-        uint32_t xa[NT][8], xz[NT][8];
+__device__ __forceinline__ void block_mma(const uint32_t (&wr)[NM][2][Geo<B, 1>::WORDS],
+                                          const uint32_t (&xa)[kMaxTiles][8],
+                                          const uint32_t (&xz)[kMaxTiles][8],
+                                          float (&acc)[kMaxTiles][NM][4]) {
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) load_act_half(arow[nt], j, t, B == 8, 0, xa[nt]);
-        uint32_t wr[NM][2][G::WORDS];
+    for (int c = 0; c < 8; ++c) {
 #pragma unroll
         for (int m = 0; m < NM; ++m) {
-            const uint8_t* chunk = stage + (size_t)m * kStageBytes + jj * G::CB;
-            load_row_words<B>(chunk, g, t, g, wr[m][0]);
-            load_row_words<B>(chunk, g + 8, t, g, wr[m][1]);
-        }
+            const uint32_t a0 = unpack_pair<B>(wr[m][0], 2 * c);
+            const uint32_t a1 = unpack_pair<B>(wr[m][1], 2 * c);
+            const uint32_t a2 = unpack_pair<B>(wr[m][0], 2 * c + 1);
+            const uint32_t a3 = unpack_pair<B>(wr[m][1], 2 * c + 1);
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) load_act_half(arow[nt], j, t, B == 8, 1, xz[nt]);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-#pragma unroll
-            for (int m = 0; m < NM; ++m) {
-                const uint32_t a0 = unpack_pair<B>(wr[m][0], 2 * c);
-                const uint32_t a1 = unpack_pair<B>(wr[m][1], 2 * c);
-                const uint32_t a2 = unpack_pair<B>(wr[m][0], 2 * c + 1);
-                const uint32_t a3 = unpack_pair<B>(wr[m][1], 2 * c + 1);
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    const uint32_t b0 = c < 4 ? xa[nt][2 * c] : xz[nt][2 * c - 8];
-                    const uint32_t b1 = c < 4 ? xa[nt][2 * c + 1] : xz[nt][2 * c - 7];
-                    mma_bf16_16816(acc[nt][m], a0, a1, a2, a3, b0, b1);
-                }
+            for (int nt = 0; nt < NT; ++nt) {
+                const uint32_t b0 = c < 4 ? xa[nt][2 * c] : xz[nt][2 * c - 8];
+                const uint32_t b1 = c < 4 ? xa[nt][2 * c + 1] : xz[nt][2 * c - 7];
+                mma_bf16_16816(acc[nt][m], a0, a1, a2, a3, b0, b1);
             }
         }
     }
 }
+
+struct Task {
+    int gi, tau, p, pos0, ntok, j_hi;
+    float scale;
+    bool valid;  // this warp's tile exists
+};
 
 // Finish a task. One K part (P = 1): gate/up applies SwiGLU and stores h
 // (bf16); down stores y_a = w_a s_e acc (fp32). Several parts: the task's
@@ -192,6 +169,7 @@ __device__ __forceinline__ void consume(const uint8_t* stage, int j0, int nch,
 template <bool GATEUP>
 __device__ __forceinline__ void finish(const Args& a, const Task& T,
                                        float (&acc)[kMaxTiles][GATEUP ? 2 : 1][4], int lane) {
+    if (!T.valid) return;
     const int g = lane >> 2, t = lane & 3;
     const int F = a.P.F, H = a.P.H;
 #pragma unroll
@@ -221,121 +199,164 @@ __device__ __forceinline__ void finish(const Args& a, const Task& T,
         }
 }
 
-// Per-warp shared-memory layout: ring, mbarriers, stage descriptors, producer state.
-struct WarpSmem {
+struct CtaSmem {
     uint8_t* ring;
-    uint64_t* bars;
-    StageDesc* descs;
-    ProducerState* ps;
+    uint64_t* full;   // per slot: 1 producer arrival + transaction bytes
+    uint64_t* empty;  // per slot: one arrival per consumer warp
+    SlotDesc* descs;
 };
 
-// All tasks of one width class, as a persistent per-warp pipeline. `seq`
-// counts the stages this warp has used so far (it sets the mbarrier phases)
-// and carries over from one class to the next.
+// Producer warp: all tasks of one width class. Lane l < 8*NM owns the copy
+// stream of tile l / NM, matrix l % NM (a page cursor in registers); lane 0
+// claims tasks, arms the full barriers and writes the slot descriptors; every
+// lane prefetches one activation line. `ep`/`used` track the empty barriers'
+// phases per slot across classes.
 template <int B, bool GATEUP>
-__device__ __forceinline__ bool run_class(const Args& a, const WarpSmem& w, int group0,
-                                          int n_groups, int32_t* ctr, int& seq) {
-    using G = Geo<B>;
+__device__ __forceinline__ bool produce_class(const Args& a, const CtaSmem& sm, int group0,
+                                              int n_groups, int32_t* ctr, uint32_t& ep,
+                                              uint32_t& used) {
     constexpr int NM = GATEUP ? 2 : 1;
+    using G = Geo<B, NM>;
+    constexpr int S = G::S;
     const PagedExperts& P = a.P;
     const int H = P.H, F = P.F;
     const int K = GATEUP ? H : F;
     const int R = GATEUP ? F : H;
     const int nj = K / kCodesPerBlock, n_tiles = R / 16;
+    const int n_tq = (n_tiles + kConsumers - 1) / kConsumers;
     const int nc1 = chunks_w1(H, F);
     const int lane = threadIdx.x & 31;
-    const int g = lane >> 2, t = lane & 3;
-    const int n_tasks = n_groups * n_tiles * a.parts;
+    const int n_tasks = n_groups * n_tq * a.parts;
     if (n_tasks == 0) return true;
+    const int cpp = chunks_per_page(B, P.page_bytes);
+    const int my_w = lane / NM, my_m = lane % NM;
+    const bool copier = lane < kConsumers * NM;
 
-    // ---- producer (lane 0) ----
-    auto issue = [&](int s) {
-        ProducerState& ps = *w.ps;
-        if (ps.done) return;
-        if (ps.task < 0 || ps.j >= ps.j_hi) {
-            // next task: the rest of the claimed batch, else claim a new batch
-            int nt;
-            if (ps.claim_left > 0) {
-                nt = ps.task + 1;
-                --ps.claim_left;
-            } else {
-                nt = atomicAdd(ctr, a.claim);
-                ps.claim_left = a.claim - 1;
+    int s = 0;
+    int task = -1, j = 0, j_hi = 0;
+    uint32_t first = 0;
+    int pslot = 0, poff = 0;           // this lane's page cursor
+    bool my_tile = false;
+    const __nv_bfloat16* pre_row = nullptr;  // this lane's activation row to prefetch
+    int pre_half = 0;
+    int active = 0;                    // tiles present in the current task
+    for (;;) {
+        // slot s must have been released by all consumers since its last fill
+        if ((used >> s) & 1u) {
+            if (!mbar_wait_bounded(&sm.empty[s], (ep >> s) & 1u)) {
+                if (lane == 0) set_status(a.status, MPE_STATUS_WAIT_TIMEOUT);
+                return false;
             }
+            ep ^= 1u << s;
+        }
+        used |= 1u << s;
+        if (task < 0 || j >= j_hi) {
+            int nt = 0;
+            if (lane == 0) nt = atomicAdd(ctr, 1);
+            nt = __shfl_sync(0xffffffffu, nt, 0);
             if (nt >= n_tasks) {
-                w.descs[s] = StageDesc{-1, 0, 0, 0};
-                mbar_arrive(&w.bars[s]);
-                ps.done = 1;
-                return;
+                if (lane == 0) {
+                    sm.descs[s] = SlotDesc{-1, 0};
+                    mbar_arrive(&sm.full[s]);
+                }
+                __syncwarp();
+                return true;
             }
-            int gi, p;
-            split_task(nt, n_tiles, a.parts, gi, ps.tau, p);
-            ps.task = nt;
-            ps.pte = P.pte[a.wg[3 * (group0 + gi)]];
-            ps.j = p * a.kb;
-            ps.j_hi = min(nj, ps.j + a.kb);
-        }
-        const int nch = min(G::J, ps.j_hi - ps.j);
-        w.descs[s] = StageDesc{ps.task, ps.j, nch, 0};
-        mbar_arrive_expect_tx(&w.bars[s], (uint32_t)(nch * G::CB * NM));
-        const int cpp = chunks_per_page(B, P.page_bytes);
-#pragma unroll
-        for (int m = 0; m < NM; ++m) {
-            const int cbase = (GATEUP ? m * nc1 : 2 * nc1) + ps.tau * nj;
-            uint8_t* dst = w.ring + (size_t)(s * NM + m) * kStageBytes;
-            int done = 0;
-            while (done < nch) {
-                const int c = cbase + ps.j + done;
-                const int n = min(nch - done, cpp - c % cpp);
-                bulk_g2s(dst + done * G::CB, chunk_addr(P, ps.pte, B, c), (uint32_t)(n * G::CB),
-                         &w.bars[s]);
-                done += n;
+            int gi, tq, p;
+            split_task(nt, n_tq, a.parts, gi, tq, p);
+            task = nt;
+            gi += group0;
+            const int e = a.wg[3 * gi];
+            const int pos0 = a.wg[3 * gi + 1], ntok = a.wg[3 * gi + 2];
+            first = P.pte[e].first;
+            j = p * a.kb;
+            j_hi = min(nj, j + a.kb);
+            active = min(kConsumers, n_tiles - tq * kConsumers);
+            const int tau = tq * kConsumers + my_w;
+            my_tile = copier && my_w < active;
+            if (my_tile) {
+                const int c = (GATEUP ? my_m * nc1 : 2 * nc1) + tau * nj + j;
+                pslot = c / cpp;
+                poff = c - pslot * cpp;
+            }
+            pre_row = nullptr;
+            pre_half = lane & 1;
+            if ((lane >> 1) < ntok) {
+                const int pos = pos0 + (lane >> 1);
+                pre_row = a.act + (size_t)(GATEUP ? (a.perm[pos] / a.k) : pos) * K;
             }
         }
-        ps.j += nch;
-    };
-
-    // prime the ring: stages seq .. seq + kStages - 1
-    if (lane == 0) {
-        *w.ps = ProducerState{-1, 0, 0, 0, 0, 0, Pte{}};
-        fence_proxy_async_smem();
-        for (int r = 0; r < kStages; ++r) issue((seq + r) % kStages);
+        if (lane == 0) {
+            sm.descs[s] = SlotDesc{task, j};
+            mbar_arrive_expect_tx(&sm.full[s], (uint32_t)(active * G::TILE));
+        }
+        __syncwarp();
+        if (my_tile) {
+            const uint8_t* src = P.pool + (size_t)P.pidx[first + pslot] * P.page_bytes +
+                                 (size_t)poff * G::CB;
+            bulk_g2s(sm.ring + (size_t)s * G::SLOT + (size_t)lane * G::CB, src, (uint32_t)G::CB,
+                     &sm.full[s]);
+            if (++poff == cpp) {
+                ++pslot;
+                poff = 0;
+            }
+        }
+        if (pre_row) prefetch_l1(pre_row + 128 * j + 64 * pre_half);
+        ++j;
+        s = (s + 1 == S) ? 0 : s + 1;
     }
-    __syncwarp();
+}
 
-    // ---- consumer (all lanes) ----
+// Consumer warp w: all tasks of one width class, tile w of each task.
+template <int B, bool GATEUP>
+__device__ __forceinline__ bool consume_class(const Args& a, const CtaSmem& sm, int group0,
+                                              int n_groups, uint32_t& fp, int w) {
+    constexpr int NM = GATEUP ? 2 : 1;
+    using G = Geo<B, NM>;
+    constexpr int S = G::S;
+    const PagedExperts& P = a.P;
+    const int H = P.H, F = P.F;
+    const int K = GATEUP ? H : F;
+    const int R = GATEUP ? F : H;
+    const int nj = K / kCodesPerBlock, n_tiles = R / 16;
+    const int n_tq = (n_tiles + kConsumers - 1) / kConsumers;
+    const int lane = threadIdx.x & 31;
+    const int g = lane >> 2, t = lane & 3;
+    if (n_groups * n_tq * a.parts == 0) return true;
+
     int cur = -1;
     Task T{};
     const __nv_bfloat16* arow[kMaxTiles] = {nullptr, nullptr};
     int ntiles = 0;
     float acc[kMaxTiles][NM][4];
-    for (;; ++seq) {
-        const int s = seq % kStages;
-        if (!mbar_wait_bounded(&w.bars[s], (uint32_t)((seq / kStages) & 1))) {
+    uint32_t xa[kMaxTiles][8], xz[kMaxTiles][8];
+    for (int s = 0;; s = (s + 1 == S) ? 0 : s + 1) {
+        const uint32_t par = (fp >> s) & 1u;
+        fp ^= 1u << s;
+        if (!mbar_wait_bounded(&sm.full[s], par)) {
             if (lane == 0) set_status(a.status, MPE_STATUS_WAIT_TIMEOUT);
-            // let copies already issued land before shared memory goes away
-            for (int r = seq + 1; r < seq + kStages; ++r)
-                mbar_wait_bounded(&w.bars[r % kStages], (uint32_t)((r / kStages) & 1));
             return false;
         }
-        const StageDesc d = w.descs[s];
-        if (d.task < 0) {  // terminator: no more tasks of this class for this warp
-            if (cur >= 0) finish<GATEUP>(a, T, acc, lane);
-            ++seq;          // the terminator used this stage
-            break;
+        const SlotDesc d = sm.descs[s];
+        if (d.task < 0) {  // terminator
+            finish<GATEUP>(a, T, acc, lane);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.empty[s]);
+            return true;
         }
         if (d.task != cur) {
             if (cur >= 0) finish<GATEUP>(a, T, acc, lane);
             cur = d.task;
-            split_task(cur, n_tiles, a.parts, T.gi, T.tau, T.p);
+            int tq;
+            split_task(cur, n_tq, a.parts, T.gi, tq, T.p);
             T.gi += group0;
-            T.e = a.wg[3 * T.gi];
+            T.tau = tq * kConsumers + w;
+            T.valid = T.tau < n_tiles;
+            const int e = a.wg[3 * T.gi];
             T.pos0 = a.wg[3 * T.gi + 1];
             T.ntok = a.wg[3 * T.gi + 2];
-            T.bits = B;
-            T.scale = P.pte[T.e].scale;
-            T.j_lo = T.p * a.kb;
-            T.j_hi = min(nj, T.j_lo + a.kb);
+            T.scale = P.pte[e].scale;
+            T.j_hi = min(nj, T.p * a.kb + a.kb);
             ntiles = (T.ntok + 7) / 8;
 #pragma unroll
             for (int nt = 0; nt < kMaxTiles; ++nt) {
@@ -352,44 +373,62 @@ __device__ __forceinline__ bool run_class(const Args& a, const WarpSmem& w, int 
                     for (int q = 0; q < 4; ++q) acc[nt][m][q] = 0.0f;
             }
         }
-        const uint8_t* stage = w.ring + (size_t)s * NM * kStageBytes;
-        if (ntiles == 1)
-            consume<B, NM, 1>(stage, d.j0, d.nch, arow, g, t, acc);
-        else
-            consume<B, NM, kMaxTiles>(stage, d.j0, d.nch, arow, g, t, acc);
+        const int j = d.j;
+        uint32_t wr[NM][2][G::WORDS];
+        if (T.valid) {
+            const uint8_t* tile = sm.ring + (size_t)s * G::SLOT + (size_t)w * G::TILE;
+#pragma unroll
+            for (int m = 0; m < NM; ++m) {
+                load_row_words<B>(tile + m * G::CB, g, t, g, wr[m][0]);
+                load_row_words<B>(tile + m * G::CB, g + 8, t, g, wr[m][1]);
+            }
+        }
         __syncwarp();
-        if (lane == 0) {
-            fence_proxy_async_smem();
-            issue(s);
+        if (lane == 0) mbar_arrive(&sm.empty[s]);  // words are in registers: release the slot
+        if (!T.valid) continue;
+        load_act_half(arow[0], j, t, B == 8, 0, xa[0]);
+        load_act_half(arow[0], j, t, B == 8, 1, xz[0]);
+        if (ntiles > 1) {
+            load_act_half(arow[1], j, t, B == 8, 0, xa[1]);
+            load_act_half(arow[1], j, t, B == 8, 1, xz[1]);
+            block_mma<B, NM, kMaxTiles>(wr, xa, xz, acc);
+        } else {
+            block_mma<B, NM, 1>(wr, xa, xz, acc);
         }
     }
-    return true;
 }
 
 template <bool GATEUP>
-__global__ void __launch_bounds__(kWarps * 32, 4) k_decode(Args a) {
+__global__ void __launch_bounds__(kThreads, 2) k_decode(Args a) {
     extern __shared__ __align__(128) uint8_t smem[];
-    constexpr int NM = GATEUP ? 2 : 1;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    WarpSmem w;
-    w.ring = smem + (size_t)warp * kStages * NM * kStageBytes;
-    w.bars = reinterpret_cast<uint64_t*>(smem + ring_bytes(NM)) + warp * kStages;
-    w.descs =
-        reinterpret_cast<StageDesc*>(smem + ring_bytes(NM) + kWarps * kStages * sizeof(uint64_t)) +
-        warp * kStages;
-    w.ps = reinterpret_cast<ProducerState*>(smem + ring_bytes(NM) +
-                                            kWarps * kStages * (sizeof(uint64_t) + sizeof(StageDesc))) +
-           warp;
-    if (lane == 0) {
-        for (int s = 0; s < kStages; ++s) mbar_init(&w.bars[s], 1);
+    CtaSmem sm;
+    sm.ring = smem;
+    sm.full = reinterpret_cast<uint64_t*>(smem + kRingBytes);
+    sm.empty = sm.full + kMaxSlots;
+    sm.descs = reinterpret_cast<SlotDesc*>(sm.empty + kMaxSlots);
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kMaxSlots; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], kConsumers);
+        }
         fence_mbar_init();
+        fence_proxy_async_smem();
     }
-    __syncwarp();
+    __syncthreads();
     const int n8 = a.n_wg_class[0], n4 = a.n_wg_class[1], n3 = a.n_wg_class[2];
-    int seq = 0;
-    if (!run_class<8, GATEUP>(a, w, 0, n8, a.task_ctr + 0, seq)) return;
-    if (!run_class<4, GATEUP>(a, w, n8, n4, a.task_ctr + 1, seq)) return;
-    run_class<3, GATEUP>(a, w, n8 + n4, n3, a.task_ctr + 2, seq);
+    if (warp == kConsumers) {
+        uint32_t ep = 0, used = 0;
+        (void)lane;
+        if (!produce_class<8, GATEUP>(a, sm, 0, n8, a.task_ctr + 0, ep, used)) return;
+        if (!produce_class<4, GATEUP>(a, sm, n8, n4, a.task_ctr + 1, ep, used)) return;
+        produce_class<3, GATEUP>(a, sm, n8 + n4, n3, a.task_ctr + 2, ep, used);
+    } else {
+        uint32_t fp = 0;
+        if (!consume_class<8, GATEUP>(a, sm, 0, n8, fp, warp)) return;
+        if (!consume_class<4, GATEUP>(a, sm, n8, n4, fp, warp)) return;
+        consume_class<3, GATEUP>(a, sm, n8 + n4, n3, fp, warp);
+    }
 }
 
 int g_num_sms = 0;
@@ -398,18 +437,18 @@ int g_num_sms = 0;
 
 void decode_set_smem_limits() {
     cudaFuncSetAttribute(k_decode<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)smem_bytes(2));
+                         (int)smem_bytes());
     cudaFuncSetAttribute(k_decode<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)smem_bytes(1));
+                         (int)smem_bytes());
 }
 
-// K parts per task: enough tasks that every warp of the persistent grid gets
-// about `per_warp` of them, at least 4 blocks per part.
-int decode_parts(int est_groups, int n_tiles, int nj, int total_warps, int per_warp) {
-    const long target = (long)per_warp * total_warps;
+// K parts per task: enough CTA tasks that every CTA of the persistent grid gets
+// about `per_cta` of them, at least 4 blocks per part.
+int decode_parts(int est_groups, int n_tq, int nj, int total_ctas, int per_cta) {
+    const long target = (long)per_cta * total_ctas;
     int P = 1;
     const int pmax = max(1, nj / 4);
-    while (P < pmax && (long)est_groups * n_tiles * P < target) ++P;
+    while (P < pmax && (long)est_groups * n_tq * P < target) ++P;
     return P;
 }
 
@@ -420,15 +459,15 @@ static int env_int(const char* name, int dflt) {
 
 void decode_plan(mpe_ctx* c, size_t Tk, DecodePlan& pl) {
     if (!g_num_sms) cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, c->device);
-    const int warps = g_num_sms * 4 * kWarps;
+    const int ctas = g_num_sms * 2;
     const int groups = (int)std::min<size_t>((size_t)c->E, Tk);
-    const int per_warp = env_int("MPE_DECODE_TASKS_PER_WARP", 4);
-    pl.claim = std::max(1, env_int("MPE_DECODE_CLAIM", 1));
+    const int per_cta = env_int("MPE_DECODE_TASKS_PER_CTA", 8);
+    pl.claim = 1;
     const int nj_gu = c->H / kCodesPerBlock, nj_dn = c->F / kCodesPerBlock;
-    int p = decode_parts(groups, c->F / 16, nj_gu, warps, per_warp);
+    int p = decode_parts(groups, (c->F / 16 + kConsumers - 1) / kConsumers, nj_gu, ctas, per_cta);
     pl.kb_gu = (nj_gu + p - 1) / p;
     pl.p_gu = (nj_gu + pl.kb_gu - 1) / pl.kb_gu;
-    p = decode_parts(groups, c->H / 16, nj_dn, warps, per_warp);
+    p = decode_parts(groups, (c->H / 16 + kConsumers - 1) / kConsumers, nj_dn, ctas, per_cta);
     pl.kb_dn = (nj_dn + p - 1) / p;
     pl.p_dn = (nj_dn + pl.kb_dn - 1) / pl.kb_dn;
 }
@@ -436,12 +475,13 @@ void decode_plan(mpe_ctx* c, size_t Tk, DecodePlan& pl) {
 static int persistent_grid(mpe_ctx* c, const void* fn, size_t smem) {
     if (!g_num_sms) cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, c->device);
     int per_sm = 0;
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kWarps * 32, smem);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, smem);
     return g_num_sms * std::max(1, per_sm);
 }
 
 void launch_decode_gateup(mpe_ctx* c, const __nv_bfloat16* x, int k, size_t Tk, int parts,
                           int kb, int claim) {
+    (void)claim;
     Args a{};
     a.P = paged(c);
     a.wg = c->s.wg;
@@ -452,18 +492,18 @@ void launch_decode_gateup(mpe_ctx* c, const __nv_bfloat16* x, int k, size_t Tk, 
     a.h_out = c->s.h;
     a.part = c->s.part;
     a.part_stride = (size_t)2 * Tk * c->F;
-    a.claim = claim;
     a.task_ctr = c->s.task_ctr;
     a.parts = parts;
     a.kb = kb;
     a.status = c->d_status;
-    const int grid = persistent_grid(c, (const void*)k_decode<true>, smem_bytes(2));
-    k_decode<true><<<grid, kWarps * 32, smem_bytes(2), c->stream>>>(a);
+    const int grid = persistent_grid(c, (const void*)k_decode<true>, smem_bytes());
+    k_decode<true><<<grid, kThreads, smem_bytes(), c->stream>>>(a);
     c->launches++;
 }
 
 void launch_decode_down(mpe_ctx* c, const float* topk_w, size_t Tk, int parts, int kb,
                         int claim) {
+    (void)claim;
     Args a{};
     a.P = paged(c);
     a.wg = c->s.wg;
@@ -475,13 +515,12 @@ void launch_decode_down(mpe_ctx* c, const float* topk_w, size_t Tk, int parts, i
     a.topk_w = topk_w;
     a.part = c->s.part;
     a.part_stride = (size_t)Tk * c->H;
-    a.claim = claim;
     a.task_ctr = c->s.task_ctr + 3;
     a.parts = parts;
     a.kb = kb;
     a.status = c->d_status;
-    const int grid = persistent_grid(c, (const void*)k_decode<false>, smem_bytes(1));
-    k_decode<false><<<grid, kWarps * 32, smem_bytes(1), c->stream>>>(a);
+    const int grid = persistent_grid(c, (const void*)k_decode<false>, smem_bytes());
+    k_decode<false><<<grid, kThreads, smem_bytes(), c->stream>>>(a);
     c->launches++;
 }
 
