@@ -172,6 +172,10 @@ int mpe_repage(mpe_ctx* ctx, uint64_t B_bits, const double* p, int32_t* n_change
  *   w    device, float32 [T x k] top-k weights
  *   k    1 .. 32
  *   out  device, bf16 [T x H]
+ * Two contraction paths compute the same values: a streaming one (packed
+ * pages read once per 16-token work group, warp-level MMA) and a tensor-core
+ * one (tcgen05 MMA over 128-token groups, weights dequantized into shared
+ * memory). MPE_PATH_AUTO takes the tensor-core path when T*k >= 32 E.
  * Asynchronous on the context stream; scratch grows on demand (that call
  * synchronises).
  */
@@ -275,7 +279,9 @@ int mpe_profile_enable(mpe_ctx* ctx, int32_t enable);
 
 /*
  * mpe_profile_read -- synchronise and sum the recorded kernel times per slot
- * (0 route, 1 gate/up, 2 SwiGLU reduce, 3 down, 4 combine): ms_host
+ * (0 route, 1 gate/up, 2 SwiGLU reduce, 3 down, 4 combine -- the streaming
+ * path; 5 gate/up, 6 down -- the tensor-core path; route and combine are
+ * shared): ms_host
  * double[n_slots] milliseconds, launches_host int64[n_slots] counts (either
  * may be NULL). reset != 0 clears the records.
  */

@@ -42,7 +42,8 @@ EXPORTS = [
     "mpe_last_error_global", "mpe_kernel_launches", "mpe_version", "mpe_profile_enable",
     "mpe_profile_read", "mpe_route_noalloc",
 ]
-PROFILE_SLOTS = ["route", "gate_up", "swiglu_reduce", "down", "combine"]
+PROFILE_SLOTS = ["route", "gate_up", "swiglu_reduce", "down", "combine", "tc_gate_up",
+                 "tc_down"]
 
 
 class MpeError(RuntimeError):

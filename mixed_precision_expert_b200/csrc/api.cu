@@ -321,6 +321,7 @@ int mpe_create(mpe_ctx** out, const mpe_config* cfg) {
     c->alloc.pages.assign(c->E, {});
     route_set_smem_limits();
     decode_set_smem_limits();
+    prefill_set_smem_limits();
     if (cudaGetLastError() != cudaSuccess)
         return bail(fail_global(MPE_ERR_CUDA, "kernel attribute setup failed"));
     *out = c;
@@ -496,11 +497,56 @@ struct KernelSpan {
     }
 };
 
+// Average assignments per expert from which MPE_PATH_AUTO takes the tensor-core
+// (prefill) path: below it most experts see fewer tokens than half an MMA tile
+// and the streaming decode kernels move fewer bytes per token.
+constexpr size_t kPrefillMinAvg = 32;
+
+static bool use_prefill(const mpe_ctx* c, size_t Tk) {
+    if (c->path == MPE_PATH_PREFILL) return true;
+    if (c->path == MPE_PATH_DECODE) return false;
+    return Tk >= kPrefillMinAvg * (size_t)c->E;
+}
+
+static int grow_y(mpe_ctx* c, size_t need_y) {
+    if (need_y <= c->s.y_cap) return MPE_OK;
+    CK(cudaStreamSynchronize(c->stream));
+    cudaFree(c->s.y);
+    c->s.y = nullptr;
+    c->s.y_cap = 0;
+    int r;
+    if ((r = dev_alloc(c, &c->s.y, need_y))) return r;
+    c->s.y_cap = need_y;
+    return MPE_OK;
+}
+
 static int moe_ffn_device(mpe_ctx* c, const void* x, int32_t T, const int32_t* ids,
                           const float* w, int32_t k, void* out) {
     const size_t Tk = (size_t)T * k;
     int r;
     if ((r = ensure_scratch(c, Tk))) return r;
+    const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
+    if (use_prefill(c, Tk)) {
+        if ((r = grow_y(c, Tk * c->H))) return r;
+        {
+            KernelSpan sp(c, 0);
+            launch_route(c, ids, (int)Tk, k, c->s.perm, c->s.offsets, c->s.inv, kPrefillGroup);
+        }
+        {
+            KernelSpan sp(c, 5);
+            launch_prefill_gateup(c, xb, k);
+        }
+        {
+            KernelSpan sp(c, 6);
+            launch_prefill_down(c, w);
+        }
+        {
+            KernelSpan sp(c, 4);
+            launch_combine(c, ids, T, k, 1, reinterpret_cast<__nv_bfloat16*>(out));
+        }
+        CKLAUNCH();
+        return MPE_OK;
+    }
     {
         KernelSpan sp(c, 0);
         launch_route(c, ids, (int)Tk, k, c->s.perm, c->s.offsets, c->s.inv, kDecodeGroup);
@@ -516,19 +562,10 @@ static int moe_ffn_device(mpe_ctx* c, const void* x, int32_t T, const int32_t* i
         if ((r = dev_alloc(c, &c->s.part, need_part))) return r;
         c->s.part_cap = need_part;
     }
-    const size_t need_y = (size_t)pl.p_dn * Tk * c->H;
-    if (need_y > c->s.y_cap) {
-        CK(cudaStreamSynchronize(c->stream));
-        cudaFree(c->s.y);
-        c->s.y = nullptr;
-        c->s.y_cap = 0;
-        if ((r = dev_alloc(c, &c->s.y, need_y))) return r;
-        c->s.y_cap = need_y;
-    }
+    if ((r = grow_y(c, (size_t)pl.p_dn * Tk * c->H))) return r;
     {
         KernelSpan sp(c, 1);
-        launch_decode_gateup(c, reinterpret_cast<const __nv_bfloat16*>(x), k, Tk, pl.p_gu,
-                             pl.kb_gu, pl.claim);
+        launch_decode_gateup(c, xb, k, Tk, pl.p_gu, pl.kb_gu, pl.claim);
     }
     if (pl.p_gu > 1) {
         KernelSpan sp(c, 2);

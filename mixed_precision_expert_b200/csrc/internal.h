@@ -39,7 +39,8 @@ struct Scratch {
 };
 
 // CUDA-event records around the forward-pass kernels (optional tracing).
-constexpr int kProfileSlots = 5;  // route, gate/up, swiglu reduce, down, combine
+// route, gate/up, swiglu reduce, down, combine, tensor-core gate/up, tensor-core down
+constexpr int kProfileSlots = 7;
 struct ProfileRecord {
     int slot;
     cudaEvent_t start, stop;
@@ -129,6 +130,12 @@ void launch_decode_gateup(mpe_ctx* c, const __nv_bfloat16* x, int k, size_t Tk, 
                           int kb, int claim);
 void launch_decode_down(mpe_ctx* c, const float* topk_w, size_t Tk, int parts, int kb,
                         int claim);
+
+// prefill.cu (tcgen05 grouped GEMM; work groups of up to kPrefillGroup positions)
+constexpr int kPrefillGroup = 128;
+void prefill_set_smem_limits();
+void launch_prefill_gateup(mpe_ctx* c, const __nv_bfloat16* x, int k);
+void launch_prefill_down(mpe_ctx* c, const float* topk_w);
 
 // combine.cu
 void launch_swiglu_reduce(mpe_ctx* c, size_t Tk, int parts);
