@@ -132,7 +132,7 @@ void launch_decode_down(mpe_ctx* c, const float* topk_w, size_t Tk, int parts, i
                         int claim);
 
 // prefill.cu (tcgen05 grouped GEMM; work groups of up to kPrefillGroup positions)
-constexpr int kPrefillGroup = 128;
+constexpr int kPrefillGroup = 96;
 void prefill_set_smem_limits();
 void launch_prefill_gateup(mpe_ctx* c, const __nv_bfloat16* x, int k);
 void launch_prefill_down(mpe_ctx* c, const float* topk_w);
