@@ -148,6 +148,7 @@ int dev_alloc(mpe_ctx* c, T** p, size_t n) {
 void free_scratch(Scratch& s) {
     cudaFree(s.perm); cudaFree(s.inv); cudaFree(s.offsets); cudaFree(s.wg); cudaFree(s.n_wg);
     cudaFree(s.hist); cudaFree(s.h); cudaFree(s.y); cudaFree(s.part); cudaFree(s.task_ctr);
+    cudaFree(s.xp);
     cudaFree(s.x_stage); cudaFree(s.ids_stage); cudaFree(s.w_stage); cudaFree(s.out_stage);
     s = Scratch{};
 }
@@ -520,6 +521,18 @@ static int grow_y(mpe_ctx* c, size_t need_y) {
     return MPE_OK;
 }
 
+static int grow_xp(mpe_ctx* c, size_t need) {
+    if (need <= c->s.xp_cap) return MPE_OK;
+    CK(cudaStreamSynchronize(c->stream));
+    cudaFree(c->s.xp);
+    c->s.xp = nullptr;
+    c->s.xp_cap = 0;
+    int r;
+    if ((r = dev_alloc(c, &c->s.xp, need))) return r;
+    c->s.xp_cap = need;
+    return MPE_OK;
+}
+
 static int moe_ffn_device(mpe_ctx* c, const void* x, int32_t T, const int32_t* ids,
                           const float* w, int32_t k, void* out) {
     const size_t Tk = (size_t)T * k;
@@ -528,21 +541,23 @@ static int moe_ffn_device(mpe_ctx* c, const void* x, int32_t T, const int32_t* i
     const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
     if (use_prefill(c, Tk)) {
         if ((r = grow_y(c, Tk * c->H))) return r;
+        if ((r = grow_xp(c, Tk * c->H))) return r;
         {
             KernelSpan sp(c, 0);
             launch_route(c, ids, (int)Tk, k, c->s.perm, c->s.offsets, c->s.inv, kPrefillGroup);
         }
         {
             KernelSpan sp(c, 5);
-            launch_prefill_gateup(c, xb, k);
+            launch_permute_tokens(c, xb, k);
+            if ((r = launch_prefill_gateup(c, Tk))) return r;
         }
         {
             KernelSpan sp(c, 6);
-            launch_prefill_down(c, w);
+            if ((r = launch_prefill_down(c, Tk))) return r;
         }
         {
             KernelSpan sp(c, 4);
-            launch_combine(c, ids, T, k, 1, reinterpret_cast<__nv_bfloat16*>(out));
+            launch_combine_by_position(c, w, T, k, reinterpret_cast<__nv_bfloat16*>(out));
         }
         CKLAUNCH();
         return MPE_OK;

@@ -59,6 +59,34 @@ k_combine(const float* y, const int32_t* ids, int T, int k, int H, int E, int pa
     reinterpret_cast<uint2*>(out + (size_t)t * H)[i] = pk;
 }
 
+// Tensor-core path: y[pos] = s * (W2 h_pos) is stored by route position, so
+// out[t] = bf16( sum_j w[t, j] * y[inv[t k + j]] ) in slot order; dropped slots
+// (inv < 0) add nothing.
+__global__ void __launch_bounds__(128)
+k_combine_by_position(const float* y, const int32_t* inv, const float* w, int T, int k, int H,
+                      __nv_bfloat16* out) {
+    const int t = blockIdx.x;
+    const int i = blockIdx.y * blockDim.x + threadIdx.x;  // float4 column index
+    if (i >= H / 4) return;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < k; ++j) {
+        const int pos = inv[t * k + j];
+        if (pos < 0) continue;
+        const float wj = w[t * k + j];
+        const float4 v = reinterpret_cast<const float4*>(y + (size_t)pos * H)[i];
+        acc.x = fmaf(wj, v.x, acc.x);
+        acc.y = fmaf(wj, v.y, acc.y);
+        acc.z = fmaf(wj, v.z, acc.z);
+        acc.w = fmaf(wj, v.w, acc.w);
+    }
+    __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+    __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+    uint2 pk;
+    pk.x = *reinterpret_cast<uint32_t*>(&lo);
+    pk.y = *reinterpret_cast<uint32_t*>(&hi);
+    reinterpret_cast<uint2*>(out + (size_t)t * H)[i] = pk;
+}
+
 }  // namespace
 
 void launch_swiglu_reduce(mpe_ctx* c, size_t Tk, int parts) {
@@ -75,6 +103,13 @@ void launch_combine(mpe_ctx* c, const int32_t* ids, int T, int k, int parts,
     dim3 grid((unsigned)T, (unsigned)((n4 + 127) / 128));
     k_combine<<<grid, 128, 0, c->stream>>>(c->s.y, ids, T, k, c->H, c->E, parts,
                                            (size_t)T * k * c->H, out);
+    c->launches++;
+}
+
+void launch_combine_by_position(mpe_ctx* c, const float* w, int T, int k, __nv_bfloat16* out) {
+    const int n4 = c->H / 4;
+    dim3 grid((unsigned)T, (unsigned)((n4 + 127) / 128));
+    k_combine_by_position<<<grid, 128, 0, c->stream>>>(c->s.y, c->s.inv, w, T, k, c->H, out);
     c->launches++;
 }
 

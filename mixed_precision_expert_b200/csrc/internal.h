@@ -30,6 +30,8 @@ struct Scratch {
     size_t part_cap = 0;         // floats
     size_t y_cap = 0;            // floats in y (P slices of T*k x H)
     int32_t* task_ctr = nullptr; // 6 task counters (3 classes x 2 kernels), zeroed by route
+    __nv_bfloat16* xp = nullptr; // routed tokens in route-position order [xp_cap x H] (tensor-core path)
+    size_t xp_cap = 0;           // elements
     // staging for the host-buffer entry point
     size_t stage_tokens = 0;
     void* x_stage = nullptr;
@@ -132,14 +134,18 @@ void launch_decode_down(mpe_ctx* c, const float* topk_w, size_t Tk, int parts, i
                         int claim);
 
 // prefill.cu (tcgen05 grouped GEMM; work groups of up to kPrefillGroup positions)
-constexpr int kPrefillGroup = 96;
+constexpr int kPrefillGroup = 208;
 void prefill_set_smem_limits();
-void launch_prefill_gateup(mpe_ctx* c, const __nv_bfloat16* x, int k);
-void launch_prefill_down(mpe_ctx* c, const float* topk_w);
+// xp[pos] = x[perm[pos] / k] for the routed positions
+void launch_permute_tokens(mpe_ctx* c, const __nv_bfloat16* x, int k);
+int launch_prefill_gateup(mpe_ctx* c, size_t Tk);
+int launch_prefill_down(mpe_ctx* c, size_t Tk);
 
 // combine.cu
 void launch_swiglu_reduce(mpe_ctx* c, size_t Tk, int parts);
 void launch_combine(mpe_ctx* c, const int32_t* ids, int T, int k, int parts,
                     __nv_bfloat16* out);
+// y stored by route position (tensor-core path); weights applied here
+void launch_combine_by_position(mpe_ctx* c, const float* w, int T, int k, __nv_bfloat16* out);
 
 }  // namespace mpe

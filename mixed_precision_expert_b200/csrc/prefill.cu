@@ -4,62 +4,68 @@
 // the fly and multiplied with the tokens; at prefill sizes (hundreds of tokens
 // per expert) this is a dense grouped GEMM per expert, computed transposed so
 // that the dequantized weights never touch shared memory:
-//   gate/up: G^T = K1 X^T, V^T = K3 X^T (features x tokens),
-//            h = silu(s G) (s V) -> bf16, h[pos][f]
-//   down:    Y^T = K2 h^T, y[a][o] = w_a s Y[a][o] (fp32, summed by the combine)
+//   gate/up: [G; V]^T = [K1; K3] X^T with the rows of K1 and K3 interleaved
+//            (feature f's gate row, then its up row), h = silu(s G) (s V) -> bf16
+//   down:    Y^T = K2 h^T, y[pos][o] = s Y[pos][o] (fp32, by route position; the
+//            combine applies the top-k weights and sums each token's slots)
 // The MMA's A operand (128 weight rows x K) lives in TENSOR MEMORY, written by
 // the producer warps straight from the registers they unpacked it into; the B
-// operand (the tile's tokens, K-major, SWIZZLE_128B) is gathered into shared
-// memory; fp32 accumulators live in tensor memory.
+// operand (the tile's tokens, K-major, SWIZZLE_128B) arrives in shared memory
+// by one TMA tile copy per stage: the routed tokens are first written in route
+// position order (a tile's tokens are then consecutive rows), because gathering
+// scattered 128-byte rows reaches only a fraction of the L2 bandwidth that
+// contiguous boxes do; fp32 accumulators live in tensor memory.
 //
-// Persistent warp-specialised kernel, one CTA per SM, 15 warps:
-//   warps 0-7   dequant producers: warp w owns weight matrix w / 4 of the tile
-//               (gate/up: W1, W3 rows of 128 features; down: two 128-row tiles
-//               of W2) and tensor-memory lanes 32 (w % 4) ..; each thread owns
-//               one weight row. Per K-step of 32 codes (one quarter block) it
-//               unpacks 16 bf16 pairs and stores them with one tcgen05.st. The
-//               packed words come from a register ring filled one load unit
-//               (4 K-steps; 2 for 8-bit) ahead, statically named so no load is
-//               waited on before its K-step.
-//   warps 8-11  epilogue: tcgen05.ld of their 32 accumulator lanes, expert scale
-//               and SwiGLU (gate/up) or top-k weight (down), global stores.
-//   warps 12-13 token loaders: cp.async gather of the tile's token rows (128
-//               bytes = 64 K per stage) into a 6-stage swizzled ring.
-//   warp 14     MMA issuer (one thread): tcgen05.mma.cta_group::1.kind::f16,
-//               A from tensor memory, B from shared memory, M = 128,
-//               N = the tile's tokens rounded up to 16 (<= 96), K = 16.
-// Tensor memory (512 columns): two accumulator buffers of 2 x 96 columns (the
-// epilogue of one tile overlaps the MMAs of the next) and a 4-stage ring of A
-// operands (2 matrices x 16 columns per K-step). Work: tiles of <= 96 positions
-// of one expert (route work groups) x 128 output features (gate/up) or
-// 256 (down); CTA b takes tiles b, b + grid, ... Every wait is bounded.
+// A tcgen05.mma of M = 128, K = 16 costs a fixed ~118 cycles up to N ~ 208 and
+// about N / 1.85 cycles beyond, so a tile carries up to kNT = 208 tokens (N
+// rounds the group up to 16): two accumulator buffers of 208 columns (the
+// epilogue of one tile overlaps the MMAs of the next) and a 3-stage ring of A
+// operands of K = 64 fill the 512 tensor-memory columns.
+//
+// Persistent warp-specialised kernel, one CTA per SM, 14 warps:
+//   warps 0-7   dequant producers: warp w owns tensor-memory lanes 32 (w % 4) ..
+//               and half w / 4 of every 128-code block (one A stage); each
+//               thread owns one A row and per stage unpacks 32 bf16 pairs into
+//               two tcgen05.st. The packed words of the next block are loaded a
+//               whole block ahead into statically named registers.
+//   warps 8-11  epilogue: tcgen05.ld of their 32 accumulator lanes; gate/up
+//               pairs lanes 2i (gate) and 2i+1 (up) with one shuffle per two
+//               tokens and stores h; down scales and stores y rows.
+//   warp 12     token loader (one thread): per stage (64 K of the tile's rows)
+//               it arms the stage's barrier with the byte count and issues one
+//               TMA tile copy of kNT rows, which completes on the barrier.
+//   warp 13     MMA issuer (one thread): tcgen05.mma.cta_group::1.kind::f16,
+//               A from tensor memory, B from shared memory, M = 128, four MMAs
+//               per stage.
+// Work: tiles of <= kNT positions of one expert (route work groups) x 64
+// features (gate/up) or 128 outputs (down); CTA b takes tiles b, b + grid, ...
+// Every wait is bounded.
+#include <cuda.h>
+
+#include <cstdio>
+#include <mutex>
+
 #include "internal.h"
 
 namespace mpe {
 namespace {
 
-constexpr int kNT = kPrefillGroup;  // tokens per tile (MMA N at most)
-constexpr int kNM = 2;              // A matrices per tile
-constexpr int kAStages = 4;         // tensor-memory A ring (K = 32 each)
-constexpr int kTStages = 6;         // shared-memory token ring (K = 64 each)
-constexpr int kTLag = 3;            // cp.async groups in flight per loader thread
+constexpr int kNT = kPrefillGroup;            // tokens per tile (MMA N at most)
+constexpr int kACol0 = 2 * kNT;               // A ring after the two accumulators
+constexpr int kAStageCols = 32;               // K = 64 per stage: 32 bf16x2 columns
+constexpr int kAStages = (512 - kACol0) / kAStageCols;
+constexpr int kTStages = 7;                   // shared-memory token ring (K = 64 each)
 constexpr int kTStageBytes = kNT * 128;
-constexpr int kDCols = kNM * kNT;             // one accumulator buffer
-constexpr int kACol0 = 2 * kDCols;            // A ring after the two buffers
-constexpr int kAStageCols = kNM * 16;         // 16 bf16x2 columns per matrix
-static_assert(kACol0 + kAStages * kAStageCols == 512, "tensor memory plan");
+static_assert(kAStages >= 3 && kACol0 + kAStages * kAStageCols <= 512, "tensor memory plan");
 static_assert(kNT % 16 == 0 && kNT <= 256, "MMA N");
 static_assert(kTStageBytes % 1024 == 0, "swizzle atoms");
-static_assert(kTStages > kTLag, "token ring");
 
 constexpr int kProdWarps = 8;
-constexpr int kLoadWarp0 = 12;
-constexpr int kLoadWarps = 2;
-constexpr int kMmaWarp = 14;
+constexpr int kEpiWarp0 = 8;  // warps 8-11: warp % 4 covers all four TMEM lane quarters
+constexpr int kLoadWarp = 12;
+constexpr int kMmaWarp = 13;
+static_assert(kEpiWarp0 % 4 == 0 && kEpiWarp0 + 4 == kLoadWarp, "epilogue warps");
 constexpr int kPThreads = 32 * (kMmaWarp + 1);
-constexpr int kLoadThreads = 32 * kLoadWarps;
-constexpr int kRowsPerLoader = kNT * 8 / kLoadThreads;  // 16-byte chunks per thread per stage
-static_assert(kNT * 8 % kLoadThreads == 0 && kLoadThreads % 8 == 0, "loader split");
 
 constexpr size_t kSmem = 1024 + (size_t)kTStages * kTStageBytes + 1024;
 
@@ -67,12 +73,8 @@ struct PArgs {
     PagedExperts P;
     const int32_t* wg;     // work groups (expert, first position, count), <= kNT positions
     const int32_t* n_wg;   // total groups
-    const int32_t* perm;
-    int k;
-    const __nv_bfloat16* act;  // gate/up: x [T x H] by token; down: h [Tk x F] by position
     __nv_bfloat16* h_out;      // gate/up: h [Tk x F] by position
-    float* y_out;              // down: y [Tk x H] by assignment
-    const float* topk_w;       // down: [Tk]
+    float* y_out;              // down: y [Tk x H] by route position
     uint32_t* status;
 };
 
@@ -141,16 +143,16 @@ __device__ __forceinline__ void tmem_wait_st() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-    asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+// A box of kNT rows x 64 bf16 columns at (column x, row y) of the tensor map's
+// matrix into shared memory, SWIZZLE_128B; rows past the matrix read as zero.
+// Completes on bar.
+__device__ __forceinline__ void tma_tile(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                         uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
 }
 
 struct Tile {
@@ -185,165 +187,147 @@ struct Ring {
 // ---------------------------------------------------------------------------
 // dequant producers
 // ---------------------------------------------------------------------------
-// Load unit: U K-steps of 32 codes of one row (b = 3, 4: a whole 128-code
-// block, 48 / 64 bytes; b = 8: half a block, 64 bytes); kRing units in flight.
+// Packed words of half a 128-code block of one row: 2 quarters of B words
+// (b = 3: 24 bytes at 8-byte alignment; b = 4, 8: 32 / 64 bytes, 16-aligned).
 template <int B>
-struct Unit {
-    static constexpr int U = (B == 8) ? 2 : 4;
-    static constexpr int W = U * B;  // 32-bit words
-};
-constexpr int kRing = 2;
-
-template <int B>
-__device__ __forceinline__ void load_unit(const uint8_t* src, uint32_t (&w)[Unit<B>::W]) {
-    const uint4* p = reinterpret_cast<const uint4*>(src);
+__device__ __forceinline__ void load_half(const uint8_t* src, uint32_t (&w)[2 * B]) {
+    if constexpr (B == 3) {
+        const uint2* p = reinterpret_cast<const uint2*>(src);
 #pragma unroll
-    for (int i = 0; i < Unit<B>::W / 4; ++i) {
-        const uint4 v = __ldg(p + i);
-        w[4 * i] = v.x;
-        w[4 * i + 1] = v.y;
-        w[4 * i + 2] = v.z;
-        w[4 * i + 3] = v.w;
+        for (int i = 0; i < 3; ++i) {
+            const uint2 v = __ldg(p + i);
+            w[2 * i] = v.x;
+            w[2 * i + 1] = v.y;
+        }
+    } else {
+        const uint4* p = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+        for (int i = 0; i < B / 2; ++i) {
+            const uint4 v = __ldg(p + i);
+            w[4 * i] = v.x;
+            w[4 * i + 1] = v.y;
+            w[4 * i + 2] = v.z;
+            w[4 * i + 3] = v.w;
+        }
     }
 }
 
-// One producer warp: all K-steps of one tile for its matrix.
+// One producer warp, one tile: half `hp` of every block column j, i.e. the
+// A stage of K = 64 that is the tile's K-step 2 j + hp; `g0` is the tile's first
+// global K-step (even), which fixes the A stage and its reuse parity.
 template <int B, bool GATEUP>
-__device__ __forceinline__ bool produce_tile(const PArgs& a, const Tile& T, int m, int lq,
+__device__ __forceinline__ bool produce_tile(const PArgs& a, const Tile& T, int hp, int lq,
                                              int lane, uint32_t tbase, uint64_t* a_full,
-                                             uint64_t* a_empty, Ring& ar) {
-    using UT = Unit<B>;
-    constexpr int kUnitsPerChunk = 4 / UT::U;
+                                             uint64_t* a_empty, uint32_t g0) {
     const PagedExperts& P = a.P;
     const int H = P.H, F = P.F;
     const int K = GATEUP ? H : F;
-    const int nunits = K / 32 / UT::U;
     const int nj = K / kCodesPerBlock;
     const int nc1 = chunks_w1(H, F);
     const int cpp = chunks_per_page(B, P.page_bytes);
-    // this warp's matrix: gate/up W1 (m = 0) or W3 (m = 1) rows nt*128 ..;
-    // down: W2 rows (2 nt + m) * 128 .. (inactive past H)
-    const int mt = GATEUP ? T.nt : 2 * T.nt + m;
-    const bool active = GATEUP || mt * 128 < H;
-    const int row = mt * 128 + lq * 32 + lane;  // weight row within its matrix
-    int pslot = 0, poff = 0;
-    if (active) {
-        const int c = (GATEUP ? m * nc1 : 2 * nc1) + (row >> 4) * nj;
-        pslot = c / cpp;
-        poff = c - pslot * cpp;
+    // this thread's A row: gate/up feature nt*64 + 16 lq + lane/2 of W1 (even
+    // lanes) or W3 (odd lanes); down: output nt*128 + 32 lq + lane of W2
+    int c, rr;
+    if (GATEUP) {
+        const int f = T.nt * 64 + lq * 16 + (lane >> 1);
+        c = (lane & 1) * nc1 + (f >> 4) * nj;
+        rr = f & 15;
+    } else {
+        const int o = T.nt * 128 + lq * 32 + lane;
+        c = 2 * nc1 + (o >> 4) * nj;
+        rr = o & 15;
     }
-    const int rho_off = (row & 15) * block_bytes(B);
-    int lu = 0;  // next unit to load
-    auto load_next = [&](uint32_t (&w)[UT::W]) {
-        if (lu < nunits && active) {
-            if (lu > 0 && (lu % kUnitsPerChunk) == 0) {  // next block column: next chunk
+    int pslot = c / cpp;
+    int poff = c - pslot * cpp;
+    const int off = rr * block_bytes(B) + hp * 8 * B;
+    auto src = [&]() {
+        return P.pool + (size_t)P.pidx[T.first + pslot] * P.page_bytes +
+               (size_t)poff * chunk_bytes(B) + off;
+    };
+    uint32_t ring[2][2 * B];
+    load_half<B>(src(), ring[0]);
+    const uint32_t lane_base = (uint32_t)(lq * 32) << 16;
+    for (int j0 = 0; j0 < nj; j0 += 2) {
+#pragma unroll
+        for (int ui = 0; ui < 2; ++ui) {
+            const int j = j0 + ui;
+            if (j >= nj) break;
+            if (j + 1 < nj) {
                 if (++poff == cpp) {
                     ++pslot;
                     poff = 0;
                 }
+                load_half<B>(src(), ring[ui ^ 1]);
             }
-            load_unit<B>(P.pool + (size_t)P.pidx[T.first + pslot] * P.page_bytes +
-                             (size_t)poff * chunk_bytes(B) + rho_off +
-                             (lu % kUnitsPerChunk) * UT::W * 4,
-                         w);
-        }
-        ++lu;
-    };
-    uint32_t ring[kRing][UT::W];
-#pragma unroll
-    for (int i = 0; i < kRing - 1; ++i) load_next(ring[i]);
-    const uint32_t lane_base = (uint32_t)(lq * 32) << 16;
-    for (int u0 = 0; u0 < nunits; u0 += kRing) {
-#pragma unroll
-        for (int ui = 0; ui < kRing; ++ui) {
-            if (u0 + ui >= nunits) break;
-            load_next(ring[(ui + kRing - 1) % kRing]);
-#pragma unroll
-            for (int q = 0; q < UT::U; ++q) {
-                const int s = ar.s;
-                if ((ar.used >> s) & 1u) {
-                    if (!mbar_wait_bounded(&a_empty[s], (ar.phase >> s) & 1u)) return false;
-                    ar.phase ^= 1u << s;
-                    tc_fence_after();
-                }
-                ar.used |= 1u << s;
-                if (active) {
-                    uint32_t v[16];
-#pragma unroll
-                    for (int p = 0; p < 16; ++p) v[p] = unpack_pair<B>(&ring[ui][q * B], p);
-                    tmem_st16(tbase + lane_base + (uint32_t)(kACol0 + s * kAStageCols + m * 16), v);
-                    tmem_wait_st();
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&a_full[s]);
-                ar.advance<kAStages>();
+            const uint32_t g = g0 + 2 * j + hp;
+            const uint32_t m = g / kAStages;
+            const int s = (int)(g - m * kAStages);
+            if (m > 0) {
+                if (!mbar_wait_bounded(&a_empty[s], (m - 1) & 1u)) return false;
+                tc_fence_after();
             }
-        }
-    }
-    return true;
-}
-
-// ---------------------------------------------------------------------------
-// token loaders: thread lt copies 16-byte chunk (lt & 7) of rows (lt >> 3) + 8 i
-// ---------------------------------------------------------------------------
-struct LoadState {
-    Ring r;
-    int pub = 0;    // oldest issued stage not yet published
-    int npend = 0;  // issued stages not yet published
-};
-
-template <bool GATEUP>
-__device__ __forceinline__ bool load_tile_tokens(const PArgs& a, const Tile& T, int lt,
-                                                 uint8_t* tring, uint64_t* t_full,
-                                                 uint64_t* t_empty, LoadState& ls) {
-    const int K = GATEUP ? a.P.H : a.P.F;
-    const int nts = K / 64;
-    const int c = lt & 7;
-    const int r0 = lt >> 3;
-    // rows past the group are not loaded: the MMA columns they feed are never stored
-    int src_row[kRowsPerLoader];  // activation row of each of this thread's tile rows, or -1
+            const uint32_t dst = tbase + lane_base + (uint32_t)(kACol0 + s * kAStageCols);
 #pragma unroll
-    for (int i = 0; i < kRowsPerLoader; ++i) {
-        const int r = r0 + (kLoadThreads / 8) * i;
-        src_row[i] = -1;
-        if (r < T.ntok) {
-            const int pos = T.pos0 + r;
-            src_row[i] = GATEUP ? (a.perm[pos] / a.k) : pos;
-        }
-    }
-    const __nv_bfloat16* act = a.act + 8 * c;
-    const int lane = lt & 31;
-    for (int j = 0; j < nts; ++j) {
-        const int s = ls.r.s;
-        if ((ls.r.used >> s) & 1u) {
-            if (!mbar_wait_bounded(&t_empty[s], (ls.r.phase >> s) & 1u)) return false;
-            ls.r.phase ^= 1u << s;
-        }
-        ls.r.used |= 1u << s;
-        uint8_t* st = tring + (size_t)s * kTStageBytes;
+            for (int q = 0; q < 2; ++q) {
+                uint32_t v[16];
 #pragma unroll
-        for (int i = 0; i < kRowsPerLoader; ++i) {
-            const int r = r0 + (kLoadThreads / 8) * i;
-            if (src_row[i] >= 0)
-                cp_async16(st + r * 128 + ((c ^ (r & 7)) << 4), act + (size_t)src_row[i] * K + 64 * j);
-        }
-        cp_async_commit();
-        ls.r.advance<kTStages>();
-        if (++ls.npend > kTLag) {
-            cp_async_wait<kTLag>();
-            fence_proxy_async_smem();
+                for (int p = 0; p < 16; ++p) v[p] = unpack_pair<B>(&ring[ui][q * B], p);
+                tmem_st16(dst + 16 * q, v);
+            }
+            tmem_wait_st();
+            tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&t_full[ls.pub]);
-            ls.pub = (ls.pub + 1 == kTStages) ? 0 : ls.pub + 1;
-            --ls.npend;
+            if (lane == 0) mbar_arrive(&a_full[s]);
         }
     }
     return true;
 }
 
+// ---------------------------------------------------------------------------
+// token loader (one thread): stage j of a tile holds columns 64 j .. 64 j + 63 of
+// rows pos0 .. pos0 + kNT - 1 of the position-ordered activations. Rows past
+// the group belong to other groups (or read as zero past the matrix): the MMA
+// columns they feed are never stored.
+// ---------------------------------------------------------------------------
 template <bool GATEUP>
-__global__ void __launch_bounds__(kPThreads, 1) k_prefill(PArgs a) {
+__device__ __forceinline__ bool load_tile_tokens(const PArgs& a, const CUtensorMap* map,
+                                                 const Tile& T, uint8_t* tring, uint64_t* t_full,
+                                                 uint64_t* t_empty, Ring& tr, uint32_t& issued) {
+    const int nts = (GATEUP ? a.P.H : a.P.F) / 64;
+    for (int j = 0; j < nts; ++j) {
+        const int s = tr.s;
+        if ((tr.used >> s) & 1u) {
+            if (!mbar_wait_bounded(&t_empty[s], (tr.phase >> s) & 1u)) return false;
+            tr.phase ^= 1u << s;
+        }
+        tr.used |= 1u << s;
+        mbar_arrive_expect_tx(&t_full[s], (uint32_t)kTStageBytes);
+        tma_tile(smem_u32(tring + (size_t)s * kTStageBytes), map, 64 * j, T.pos0, &t_full[s]);
+        issued ^= 1u << s;  // parity of the number of fills of slot s
+        tr.advance<kTStages>();
+    }
+    return true;
+}
+
+// xp[pos] = x[perm[pos] / k] for pos < offsets[E]: one warp per row, 16-byte
+// chunks (H a multiple of 128).
+__global__ void __launch_bounds__(256)
+k_permute_rows(const __nv_bfloat16* x, const int32_t* perm, const int32_t* n_valid, int k,
+               int H, __nv_bfloat16* xp) {
+    const int n = *n_valid;
+    const int lane = threadIdx.x & 31;
+    const int chunks = H / 8;
+    for (int pos = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; pos < n;
+         pos += (gridDim.x * blockDim.x) >> 5) {
+        const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)(perm[pos] / k) * H);
+        uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)pos * H);
+        for (int i = lane; i < chunks; i += 32) dst[i] = __ldg(src + i);
+    }
+}
+
+template <bool GATEUP>
+__global__ void __launch_bounds__(kPThreads, 1)
+k_prefill(const __grid_constant__ CUtensorMap tmap, PArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* tring = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -358,8 +342,8 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill(PArgs a) {
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int H = a.P.H, F = a.P.F;
-    const int n_nt = GATEUP ? F / 128 : (H / 128 + 1) / 2;
-    const int nk = (GATEUP ? H : F) / 32;
+    const int n_nt = GATEUP ? F / 64 : H / 128;
+    const int nk = (GATEUP ? H : F) / 64;  // K-steps (A stages, token stages) per tile, even
     const int n_tasks = (*a.n_wg) * n_nt;
 
     if (warp == 0) {
@@ -370,11 +354,11 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill(PArgs a) {
     }
     if (threadIdx.x == 32) {
         for (int i = 0; i < kAStages; ++i) {
-            mbar_init(&a_full[i], kProdWarps);
+            mbar_init(&a_full[i], 4);  // the four warps of the half that owns the K-step
             mbar_init(&a_empty[i], 1);
         }
         for (int i = 0; i < kTStages; ++i) {
-            mbar_init(&t_full[i], kLoadWarps);
+            mbar_init(&t_full[i], 1);  // the loader's arrive + the copies' bytes
             mbar_init(&t_empty[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
@@ -392,38 +376,39 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill(PArgs a) {
 
     if (warp < kProdWarps) {
         // ---------------- dequant producers ----------------
-        const int m = warp >> 2, lq = warp & 3;
-        Ring ar;
-        for (int task = blockIdx.x; task < n_tasks && ok; task += gridDim.x) {
+        const int hp = warp >> 2, lq = warp & 3;
+        uint32_t g0 = 0;
+        for (int task = blockIdx.x; task < n_tasks && ok; task += gridDim.x, g0 += nk) {
             const Tile T = load_tile(a, task, n_nt);
             switch (T.bits) {
-                case 3: ok = produce_tile<3, GATEUP>(a, T, m, lq, lane, tbase, a_full, a_empty, ar); break;
-                case 4: ok = produce_tile<4, GATEUP>(a, T, m, lq, lane, tbase, a_full, a_empty, ar); break;
-                default: ok = produce_tile<8, GATEUP>(a, T, m, lq, lane, tbase, a_full, a_empty, ar); break;
+                case 3: ok = produce_tile<3, GATEUP>(a, T, hp, lq, lane, tbase, a_full, a_empty, g0); break;
+                case 4: ok = produce_tile<4, GATEUP>(a, T, hp, lq, lane, tbase, a_full, a_empty, g0); break;
+                default: ok = produce_tile<8, GATEUP>(a, T, hp, lq, lane, tbase, a_full, a_empty, g0); break;
             }
         }
-    } else if (warp >= kLoadWarp0 && warp < kLoadWarp0 + kLoadWarps) {
-        // ---------------- token loaders ----------------
-        const int lt = threadIdx.x - 32 * kLoadWarp0;
-        LoadState ls;
-        for (int task = blockIdx.x; task < n_tasks && ok; task += gridDim.x) {
-            const Tile T = load_tile(a, task, n_nt);
-            ok = load_tile_tokens<GATEUP>(a, T, lt, tring, t_full, t_empty, ls);
-        }
-        cp_async_wait<0>();
-        if (ok) {
-            fence_proxy_async_smem();
-            __syncwarp();
-            for (; ls.npend > 0; --ls.npend) {
-                if (lane == 0) mbar_arrive(&t_full[ls.pub]);
-                ls.pub = (ls.pub + 1 == kTStages) ? 0 : ls.pub + 1;
+    } else if (warp == kLoadWarp) {
+        // ---------------- token loader ----------------
+        Ring tr;
+        uint32_t issued = 0;
+        if (lane == 0)
+            for (int task = blockIdx.x; task < n_tasks && ok; task += gridDim.x) {
+                const Tile T = load_tile(a, task, n_nt);
+                ok = load_tile_tokens<GATEUP>(a, &tmap, T, tring, t_full, t_empty, tr, issued);
             }
-        }
+        // the copies of every slot's last fill have landed before shared memory is
+        // released (already true unless a wait above gave up)
+        if (lane == 0)
+            for (int s = 0; s < kTStages; ++s)
+                if (((tr.used >> s) & 1u) && !mbar_wait_bounded(&t_full[s], ((issued >> s) & 1u) ^ 1u))
+                    ok = false;
+        __syncwarp();
     } else if (warp == kMmaWarp) {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
-            Ring ar, tr, dr;
-            uint32_t a_ph = 0, t_ph = 0;
+            Ring tr, dr;
+            uint32_t t_ph = 0, g = 0;
+            // descriptor of token stage 0; stage ts adds ts * kTStageBytes / 16
+            const uint64_t desc0 = umma_desc(smem_u32(tring));
             for (int task = blockIdx.x; task < n_tasks && ok; task += gridDim.x) {
                 const Tile T = load_tile(a, task, n_nt);
                 const int b = dr.s;
@@ -433,36 +418,24 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill(PArgs a) {
                 }
                 dr.used |= 1u << b;
                 tc_fence_after();
-                const int nmma = (T.ntok + 15) & ~15;
-                const uint32_t idesc = umma_idesc(128, nmma);
-                const bool act1 = GATEUP || (2 * T.nt + 1) * 128 < H;
-                const uint32_t dcol = tbase + (uint32_t)(b * kDCols);
-                for (int kk = 0; kk < nk; ++kk) {
+                const uint32_t idesc = umma_idesc(128, (T.ntok + 15) & ~15);
+                const uint32_t dcol = tbase + (uint32_t)(b * kNT);
+                for (int kk = 0; kk < nk; ++kk, ++g) {
                     const int ts = tr.s;
-                    if ((kk & 1) == 0) {
-                        if (!mbar_wait_bounded(&t_full[ts], (t_ph >> ts) & 1u)) { ok = false; break; }
-                        t_ph ^= 1u << ts;
-                    }
-                    const int as = ar.s;
-                    if (!mbar_wait_bounded(&a_full[as], (a_ph >> as) & 1u)) { ok = false; break; }
-                    a_ph ^= 1u << as;
+                    if (!mbar_wait_bounded(&t_full[ts], (t_ph >> ts) & 1u)) { ok = false; break; }
+                    t_ph ^= 1u << ts;
+                    const uint32_t m = g / kAStages;
+                    const int s = (int)(g - m * kAStages);
+                    if (!mbar_wait_bounded(&a_full[s], m & 1u)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t tsm = smem_u32(tring + (size_t)ts * kTStageBytes) + (kk & 1) * 64;
+                    const uint64_t bd = desc0 + (uint64_t)(ts * (kTStageBytes >> 4));
+                    const uint32_t acol = tbase + (uint32_t)(kACol0 + s * kAStageCols);
 #pragma unroll
-                    for (int mm = 0; mm < kNM; ++mm) {
-                        if (mm == 1 && !act1) break;
-#pragma unroll
-                        for (int k16 = 0; k16 < 2; ++k16)
-                            umma_ts(dcol + mm * kNT,
-                                    tbase + (uint32_t)(kACol0 + as * kAStageCols + mm * 16 + k16 * 8),
-                                    umma_desc(tsm + k16 * 32), idesc, (kk | k16) ? 1u : 0u);
-                    }
-                    umma_commit(&a_empty[as]);
-                    ar.advance<kAStages>();
-                    if (kk & 1) {
-                        umma_commit(&t_empty[ts]);
-                        tr.advance<kTStages>();
-                    }
+                    for (int k16 = 0; k16 < 4; ++k16)
+                        umma_ts(dcol, acol + 8 * k16, bd + 2 * k16, idesc, (kk | k16) ? 1u : 0u);
+                    umma_commit(&a_empty[s]);
+                    umma_commit(&t_empty[ts]);
+                    tr.advance<kTStages>();
                 }
                 if (!ok) break;
                 umma_commit(&d_full[b]);
@@ -476,6 +449,7 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill(PArgs a) {
     } else {
         // ---------------- epilogue (warps 8-11: TMEM lanes 32 (warp % 4) ..) ----------------
         const int lq = warp & 3;
+        const bool odd = lane & 1;
         Ring dr;
         for (int task = blockIdx.x; task < n_tasks && ok; task += gridDim.x) {
             const Tile T = load_tile(a, task, n_nt);
@@ -483,62 +457,38 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill(PArgs a) {
             if (!mbar_wait_bounded(&d_full[b], (dr.phase >> b) & 1u)) { ok = false; break; }
             dr.phase ^= 1u << b;
             tc_fence_after();
-            const uint32_t tl = tbase + ((uint32_t)(lq * 32) << 16) + (uint32_t)(b * kDCols);
+            const uint32_t tl = tbase + ((uint32_t)(lq * 32) << 16) + (uint32_t)(b * kNT);
             if (GATEUP) {
-                const int f = T.nt * 128 + lq * 32 + lane;  // this lane's feature
-                const bool odd = lane & 1;
+                // even lane: gate of feature f, odd lane: up of f; per 16 tokens the
+                // even lane finishes tokens 0-7 and the odd lane tokens 8-15
+                const int f = T.nt * 64 + lq * 16 + (lane >> 1);
 #pragma unroll 1
                 for (int c0 = 0; c0 < T.ntok; c0 += 16) {
-                    uint32_t g[16], v[16];
-                    tmem_ld16(tl + c0, g);
-                    tmem_ld16(tl + kNT + c0, v);
+                    uint32_t d[16];
+                    tmem_ld16(tl + c0, d);
                     tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
-                        uint32_t hb[2];
-#pragma unroll
-                        for (int u = 0; u < 2; ++u) {
-                            const float gg = T.scale * __uint_as_float(g[2 * i + u]);
-                            const float vv = T.scale * __uint_as_float(v[2 * i + u]);
-                            hb[u] = __bfloat16_as_ushort(
-                                __float2bfloat16_rn(__fdividef(gg, 1.0f + __expf(-gg)) * vv));
-                        }
-                        // lanes 2l, 2l+1 swap halves so each stores a (f even, f odd)
-                        // pair: the even lane for token t, the odd lane for t + 1
-                        const uint32_t recv = __shfl_xor_sync(0xffffffffu, odd ? hb[0] : hb[1], 1);
-                        const int t = c0 + 2 * i + (odd ? 1 : 0);
-                        const uint32_t lo = odd ? recv : hb[0];
-                        const uint32_t hi = odd ? hb[1] : recv;
+                        const uint32_t recv = __shfl_xor_sync(0xffffffffu, odd ? d[i] : d[8 + i], 1);
+                        const float gg = T.scale * __uint_as_float(odd ? recv : d[i]);
+                        const float vv = T.scale * __uint_as_float(odd ? d[8 + i] : recv);
+                        const int t = c0 + i + (odd ? 8 : 0);
                         if (t < T.ntok)
-                            *reinterpret_cast<uint32_t*>(a.h_out + (size_t)(T.pos0 + t) * F + (f & ~1)) =
-                                lo | (hi << 16);
+                            a.h_out[(size_t)(T.pos0 + t) * F + f] =
+                                __float2bfloat16_rn(__fdividef(gg, 1.0f + __expf(-gg)) * vv);
                     }
                 }
             } else {
+                const int o = T.nt * 128 + lq * 32 + lane;  // output feature
+                float* dst = a.y_out + (size_t)T.pos0 * H + o;
 #pragma unroll 1
-                for (int mm = 0; mm < kNM; ++mm) {
-                    if ((2 * T.nt + mm) * 128 >= H) break;
-                    const int o = (2 * T.nt + mm) * 128 + lq * 32 + lane;  // output feature
-#pragma unroll 1
-                    for (int c0 = 0; c0 < T.ntok; c0 += 16) {
-                        uint32_t y[16];
-                        tmem_ld16(tl + mm * kNT + c0, y);
-                        // assignment and weight of tokens c0 .. c0 + 15 (lanes 0..15)
-                        int asg = 0;
-                        float wt = 0.0f;
-                        if (lane < 16 && c0 + lane < T.ntok) {
-                            asg = a.perm[T.pos0 + c0 + lane];
-                            wt = a.topk_w[asg];
-                        }
-                        tmem_wait_ld();
+                for (int c0 = 0; c0 < T.ntok; c0 += 16) {
+                    uint32_t y[16];
+                    tmem_ld16(tl + c0, y);
+                    tmem_wait_ld();
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const int ai = __shfl_sync(0xffffffffu, asg, i);
-                            const float wi = __shfl_sync(0xffffffffu, wt, i);
-                            if (c0 + i < T.ntok)
-                                a.y_out[(size_t)ai * H + o] = wi * (T.scale * __uint_as_float(y[i]));
-                        }
-                    }
+                    for (int i = 0; i < 16; ++i)
+                        if (c0 + i < T.ntok) dst[(size_t)(c0 + i) * H] = T.scale * __uint_as_float(y[i]);
                 }
             }
             tc_fence_before();
@@ -563,6 +513,52 @@ int sm_count(int device) {
     return n > 0 ? n : 1;
 }
 
+typedef CUresult (*TensorMapEncodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                         const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                         const cuuint32_t*, CUtensorMapInterleave,
+                                         CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                         CUtensorMapFloatOOBfill);
+
+// The driver's tensor-map encoder, looked up once through the runtime.
+TensorMapEncodeTiled encoder() {
+    static TensorMapEncodeTiled fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<TensorMapEncodeTiled>(p);
+    });
+    return fn;
+}
+
+int encode_fail(mpe_ctx* c, const char* what, int code) {
+    char buf[128];
+    snprintf(buf, sizeof(buf), "%s (%d)", what, code);
+    c->err = buf;
+    return MPE_ERR_CUDA;
+}
+
+// Row-major bf16 [rows x cols] in global memory, read as boxes of kNT rows x 64
+// columns (128-byte row pieces) with the 128-byte swizzle the MMA's B descriptor
+// expects. base 16-byte aligned, cols a multiple of 64.
+int encode_rows(mpe_ctx* c, CUtensorMap* map, const void* base, size_t rows, int cols) {
+    TensorMapEncodeTiled enc = encoder();
+    if (!enc) return encode_fail(c, "cuTensorMapEncodeTiled is not available", 0);
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)kNT};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return encode_fail(c, "tensor map encode failed", (int)r);
+    return MPE_OK;
+}
+
 }  // namespace
 
 void prefill_set_smem_limits() {
@@ -570,33 +566,40 @@ void prefill_set_smem_limits() {
     cudaFuncSetAttribute(k_prefill<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
 }
 
-void launch_prefill_gateup(mpe_ctx* c, const __nv_bfloat16* x, int k) {
-    PArgs a{};
-    a.P = paged(c);
-    a.wg = c->s.wg;
-    a.n_wg = c->s.n_wg;
-    a.perm = c->s.perm;
-    a.k = k;
-    a.act = x;
-    a.h_out = c->s.h;
-    a.status = c->d_status;
-    k_prefill<true><<<sm_count(c->device), kPThreads, kSmem, c->stream>>>(a);
+void launch_permute_tokens(mpe_ctx* c, const __nv_bfloat16* x, int k) {
+    k_permute_rows<<<sm_count(c->device) * 8, 256, 0, c->stream>>>(
+        x, c->s.perm, c->s.offsets + c->E, k, c->H, c->s.xp);
     c->launches++;
 }
 
-void launch_prefill_down(mpe_ctx* c, const float* topk_w) {
+int launch_prefill_gateup(mpe_ctx* c, size_t Tk) {
+    alignas(64) CUtensorMap map;
+    int r;
+    if ((r = encode_rows(c, &map, c->s.xp, Tk, c->H))) return r;
     PArgs a{};
     a.P = paged(c);
     a.wg = c->s.wg;
     a.n_wg = c->s.n_wg;
-    a.perm = c->s.perm;
-    a.k = 1;
-    a.act = c->s.h;
-    a.y_out = c->s.y;
-    a.topk_w = topk_w;
+    a.h_out = c->s.h;
     a.status = c->d_status;
-    k_prefill<false><<<sm_count(c->device), kPThreads, kSmem, c->stream>>>(a);
+    k_prefill<true><<<sm_count(c->device), kPThreads, kSmem, c->stream>>>(map, a);
     c->launches++;
+    return MPE_OK;
+}
+
+int launch_prefill_down(mpe_ctx* c, size_t Tk) {
+    alignas(64) CUtensorMap map;
+    int r;
+    if ((r = encode_rows(c, &map, c->s.h, Tk, c->F))) return r;
+    PArgs a{};
+    a.P = paged(c);
+    a.wg = c->s.wg;
+    a.n_wg = c->s.n_wg;
+    a.y_out = c->s.y;
+    a.status = c->d_status;
+    k_prefill<false><<<sm_count(c->device), kPThreads, kSmem, c->stream>>>(map, a);
+    c->launches++;
+    return MPE_OK;
 }
 
 }  // namespace mpe
