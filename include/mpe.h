@@ -280,8 +280,8 @@ int mpe_profile_enable(mpe_ctx* ctx, int32_t enable);
 /*
  * mpe_profile_read -- synchronise and sum the recorded kernel times per slot
  * (0 route, 1 gate/up, 2 SwiGLU reduce, 3 down, 4 combine -- the streaming
- * path; 5 gate/up, 6 down -- the tensor-core path; route and combine are
- * shared): ms_host
+ * path; 5 gate/up, 6 down, 7 token permute -- the tensor-core path; route
+ * and combine are shared): ms_host
  * double[n_slots] milliseconds, launches_host int64[n_slots] counts (either
  * may be NULL). reset != 0 clears the records.
  */

@@ -43,7 +43,7 @@ EXPORTS = [
     "mpe_profile_read", "mpe_route_noalloc",
 ]
 PROFILE_SLOTS = ["route", "gate_up", "swiglu_reduce", "down", "combine", "tc_gate_up",
-                 "tc_down"]
+                 "tc_down", "tc_permute"]
 
 
 class MpeError(RuntimeError):

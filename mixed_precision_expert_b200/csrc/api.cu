@@ -547,8 +547,11 @@ static int moe_ffn_device(mpe_ctx* c, const void* x, int32_t T, const int32_t* i
             launch_route(c, ids, (int)Tk, k, c->s.perm, c->s.offsets, c->s.inv, kPrefillGroup);
         }
         {
-            KernelSpan sp(c, 5);
+            KernelSpan sp(c, 7);
             launch_permute_tokens(c, xb, k);
+        }
+        {
+            KernelSpan sp(c, 5);
             if ((r = launch_prefill_gateup(c, Tk))) return r;
         }
         {

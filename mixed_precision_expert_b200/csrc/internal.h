@@ -41,8 +41,9 @@ struct Scratch {
 };
 
 // CUDA-event records around the forward-pass kernels (optional tracing).
-// route, gate/up, swiglu reduce, down, combine, tensor-core gate/up, tensor-core down
-constexpr int kProfileSlots = 7;
+// route, gate/up, swiglu reduce, down, combine, tensor-core gate/up, tensor-core
+// down, token permute (tensor-core path)
+constexpr int kProfileSlots = 8;
 struct ProfileRecord {
     int slot;
     cudaEvent_t start, stop;
