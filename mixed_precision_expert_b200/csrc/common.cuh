@@ -155,6 +155,11 @@ __device__ __forceinline__ void prefetch_l1(const void* p) {
     asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
 }
 
+// Bring a global line into L2 ahead of use.
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // Wait for phase `parity` of an mbarrier, giving up after kWaitLimitNs.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -163,6 +168,14 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
         if (mbar_try_wait(bar, parity)) return true;
         if (global_ns() - t0 > kWaitLimitNs) return false;
     }
+}
+
+// Latency-critical wait (an MMA issuer): a non-blocking test first, which costs
+// far less than the potentially suspending try_wait when the phase is already
+// complete; then the bounded wait.
+__device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity) {
+    if (mbar_test(bar, parity)) return true;
+    return mbar_wait_bounded(bar, parity);
 }
 
 // ---------------------------------------------------------------------------

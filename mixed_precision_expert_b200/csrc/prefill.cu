@@ -217,7 +217,7 @@ __device__ __forceinline__ void load_half(const uint8_t* src, uint32_t (&w)[2 * 
 // global K-step (even), which fixes the A stage and its reuse parity.
 template <int B, bool GATEUP>
 __device__ __forceinline__ bool produce_tile(const PArgs& a, const Tile& T, int hp, int lq,
-                                             int lane, uint32_t tbase, uint64_t* a_full,
+                                             int lane, uint32_t tbase, uint64_t* full,
                                              uint64_t* a_empty, uint32_t g0) {
     const PagedExperts& P = a.P;
     const int H = P.H, F = P.F;
@@ -244,6 +244,19 @@ __device__ __forceinline__ bool produce_tile(const PArgs& a, const Tile& T, int 
         return P.pool + (size_t)P.pidx[T.first + pslot] * P.page_bytes +
                (size_t)poff * chunk_bytes(B) + off;
     };
+    // a second cursor kPrefetch block columns ahead pulls this row's packed words
+    // into L2 (no registers held), so the register loads one block ahead hit L2
+    constexpr int kPrefetch = 4;
+    int fslot = (c + kPrefetch) / cpp;
+    int foff = (c + kPrefetch) - fslot * cpp;
+    const int fmax = c + nj;  // the row's chunks end here
+    int fchunk = c + kPrefetch;
+    for (int i = 1; i < kPrefetch && i < nj; ++i) {
+        const int ci = c + i;
+        const int si = ci / cpp;
+        prefetch_l2(P.pool + (size_t)P.pidx[T.first + si] * P.page_bytes +
+                    (size_t)(ci - si * cpp) * chunk_bytes(B) + off);
+    }
     uint32_t ring[2][2 * B];
     load_half<B>(src(), ring[0]);
     const uint32_t lane_base = (uint32_t)(lq * 32) << 16;
@@ -258,6 +271,15 @@ __device__ __forceinline__ bool produce_tile(const PArgs& a, const Tile& T, int 
                     poff = 0;
                 }
                 load_half<B>(src(), ring[ui ^ 1]);
+            }
+            if (fchunk < fmax) {
+                prefetch_l2(P.pool + (size_t)P.pidx[T.first + fslot] * P.page_bytes +
+                            (size_t)foff * chunk_bytes(B) + off);
+                ++fchunk;
+                if (++foff == cpp) {
+                    ++fslot;
+                    foff = 0;
+                }
             }
             const uint32_t g = g0 + 2 * j + hp;
             const uint32_t m = g / kAStages;
@@ -277,7 +299,10 @@ __device__ __forceinline__ bool produce_tile(const PArgs& a, const Tile& T, int 
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&a_full[s]);
+            if (lane == 0) {
+                const uint32_t fm = g / kTStages;
+                mbar_arrive(&full[g - fm * kTStages]);
+            }
         }
     }
     return true;
@@ -291,8 +316,8 @@ __device__ __forceinline__ bool produce_tile(const PArgs& a, const Tile& T, int 
 // ---------------------------------------------------------------------------
 template <bool GATEUP>
 __device__ __forceinline__ bool load_tile_tokens(const PArgs& a, const CUtensorMap* map,
-                                                 const Tile& T, uint8_t* tring, uint64_t* t_full,
-                                                 uint64_t* t_empty, Ring& tr, uint32_t& issued) {
+                                                 const Tile& T, uint8_t* tring, uint64_t* full,
+                                                 uint64_t* t_empty, Ring& tr) {
     const int nts = (GATEUP ? a.P.H : a.P.F) / 64;
     for (int j = 0; j < nts; ++j) {
         const int s = tr.s;
@@ -301,9 +326,8 @@ __device__ __forceinline__ bool load_tile_tokens(const PArgs& a, const CUtensorM
             tr.phase ^= 1u << s;
         }
         tr.used |= 1u << s;
-        mbar_arrive_expect_tx(&t_full[s], (uint32_t)kTStageBytes);
-        tma_tile(smem_u32(tring + (size_t)s * kTStageBytes), map, 64 * j, T.pos0, &t_full[s]);
-        issued ^= 1u << s;  // parity of the number of fills of slot s
+        mbar_arrive_expect_tx(&full[s], (uint32_t)kTStageBytes);
+        tma_tile(smem_u32(tring + (size_t)s * kTStageBytes), map, 64 * j, T.pos0, &full[s]);
         tr.advance<kTStages>();
     }
     return true;
@@ -331,10 +355,11 @@ k_prefill(const __grid_constant__ CUtensorMap tmap, PArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* tring = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint64_t* a_full = reinterpret_cast<uint64_t*>(tring + (size_t)kTStages * kTStageBytes);
-    uint64_t* a_empty = a_full + kAStages;
-    uint64_t* t_full = a_empty + kAStages;
-    uint64_t* t_empty = t_full + kTStages;
+    // full[g % kTStages]: K-step g is ready -- its A stage written (four producer
+    // warps) and its token stage landed (the loader's arrive + the copy's bytes)
+    uint64_t* full = reinterpret_cast<uint64_t*>(tring + (size_t)kTStages * kTStageBytes);
+    uint64_t* a_empty = full + kTStages;
+    uint64_t* t_empty = a_empty + kAStages;
     uint64_t* d_full = t_empty + kTStages;
     uint64_t* d_empty = d_full + 2;
     uint64_t* drain = d_empty + 2;
@@ -353,14 +378,11 @@ k_prefill(const __grid_constant__ CUtensorMap tmap, PArgs a) {
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     if (threadIdx.x == 32) {
-        for (int i = 0; i < kAStages; ++i) {
-            mbar_init(&a_full[i], 4);  // the four warps of the half that owns the K-step
-            mbar_init(&a_empty[i], 1);
-        }
         for (int i = 0; i < kTStages; ++i) {
-            mbar_init(&t_full[i], 1);  // the loader's arrive + the copies' bytes
+            mbar_init(&full[i], 5);  // four producer warps of the step's half + the loader
             mbar_init(&t_empty[i], 1);
         }
+        for (int i = 0; i < kAStages; ++i) mbar_init(&a_empty[i], 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&d_full[i], 1);
             mbar_init(&d_empty[i], 4);
@@ -381,65 +403,72 @@ k_prefill(const __grid_constant__ CUtensorMap tmap, PArgs a) {
         for (int task = blockIdx.x; task < n_tasks && ok; task += gridDim.x, g0 += nk) {
             const Tile T = load_tile(a, task, n_nt);
             switch (T.bits) {
-                case 3: ok = produce_tile<3, GATEUP>(a, T, hp, lq, lane, tbase, a_full, a_empty, g0); break;
-                case 4: ok = produce_tile<4, GATEUP>(a, T, hp, lq, lane, tbase, a_full, a_empty, g0); break;
-                default: ok = produce_tile<8, GATEUP>(a, T, hp, lq, lane, tbase, a_full, a_empty, g0); break;
+                case 3: ok = produce_tile<3, GATEUP>(a, T, hp, lq, lane, tbase, full, a_empty, g0); break;
+                case 4: ok = produce_tile<4, GATEUP>(a, T, hp, lq, lane, tbase, full, a_empty, g0); break;
+                default: ok = produce_tile<8, GATEUP>(a, T, hp, lq, lane, tbase, full, a_empty, g0); break;
             }
         }
     } else if (warp == kLoadWarp) {
         // ---------------- token loader ----------------
         Ring tr;
-        uint32_t issued = 0;
         if (lane == 0)
             for (int task = blockIdx.x; task < n_tasks && ok; task += gridDim.x) {
                 const Tile T = load_tile(a, task, n_nt);
-                ok = load_tile_tokens<GATEUP>(a, &tmap, T, tring, t_full, t_empty, tr, issued);
+                ok = load_tile_tokens<GATEUP>(a, &tmap, T, tring, full, t_empty, tr);
             }
-        // the copies of every slot's last fill have landed before shared memory is
-        // released (already true unless a wait above gave up)
-        if (lane == 0)
-            for (int s = 0; s < kTStages; ++s)
-                if (((tr.used >> s) & 1u) && !mbar_wait_bounded(&t_full[s], ((issued >> s) & 1u) ^ 1u))
-                    ok = false;
+        // on a failed wait, give copies still in flight time to land before the
+        // CTA releases its shared memory (every copy was consumed otherwise)
+        if (!ok) {
+            const uint64_t t0 = global_ns();
+            while (global_ns() - t0 < 1000000ull) {
+            }
+        }
         __syncwarp();
     } else if (warp == kMmaWarp) {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
-            Ring tr, dr;
-            uint32_t t_ph = 0, g = 0;
-            // descriptor of token stage 0; stage ts adds ts * kTStageBytes / 16
+            // The issuing thread is on the critical path: a tcgen05.mma of this shape
+            // holds it ~120 cycles and only about one more MMA queues behind the
+            // one executing, so the bookkeeping between MMAs is kept to a few
+            // instructions (ring slots and phase bits as counters and bit masks).
+            int ts = 0, as = 0;              // full/token slot (g % kTStages), A slot (g % kAStages)
+            uint32_t fph = 0;                // phase parity to wait for, per full[] slot
+            int db = 0;                      // accumulator buffer
+            uint32_t dph = 0, dused = 0;
             const uint64_t desc0 = umma_desc(smem_u32(tring));
-            for (int task = blockIdx.x; task < n_tasks && ok; task += gridDim.x) {
-                const Tile T = load_tile(a, task, n_nt);
-                const int b = dr.s;
-                if ((dr.used >> b) & 1u) {
-                    if (!mbar_wait_bounded(&d_empty[b], (dr.phase >> b) & 1u)) { ok = false; break; }
-                    dr.phase ^= 1u << b;
+            const uint32_t acol0 = tbase + (uint32_t)kACol0;
+            int task = blockIdx.x;
+            int ntok = task < n_tasks ? load_tile(a, task, n_nt).ntok : 0;
+            for (; task < n_tasks && ok; task += gridDim.x) {
+                // the next tile's token count, fetched while this one runs
+                const int nxt = task + (int)gridDim.x;
+                const int ntok_next = nxt < n_tasks ? a.wg[3 * (nxt / n_nt) + 2] : 0;
+                if ((dused >> db) & 1u) {
+                    if (!mbar_wait_bounded(&d_empty[db], (dph >> db) & 1u)) { ok = false; break; }
+                    dph ^= 1u << db;
                 }
-                dr.used |= 1u << b;
-                tc_fence_after();
-                const uint32_t idesc = umma_idesc(128, (T.ntok + 15) & ~15);
-                const uint32_t dcol = tbase + (uint32_t)(b * kNT);
-                for (int kk = 0; kk < nk; ++kk, ++g) {
-                    const int ts = tr.s;
-                    if (!mbar_wait_bounded(&t_full[ts], (t_ph >> ts) & 1u)) { ok = false; break; }
-                    t_ph ^= 1u << ts;
-                    const uint32_t m = g / kAStages;
-                    const int s = (int)(g - m * kAStages);
-                    if (!mbar_wait_bounded(&a_full[s], m & 1u)) { ok = false; break; }
+                dused |= 1u << db;
+                const uint32_t idesc = umma_idesc(128, (ntok + 15) & ~15);
+                const uint32_t dcol = tbase + (uint32_t)(db * kNT);
+                for (int kk = 0; kk < nk; ++kk) {
+                    if (!mbar_wait_spin(&full[ts], (fph >> ts) & 1u)) { ok = false; break; }
+                    fph ^= 1u << ts;
                     tc_fence_after();
                     const uint64_t bd = desc0 + (uint64_t)(ts * (kTStageBytes >> 4));
-                    const uint32_t acol = tbase + (uint32_t)(kACol0 + s * kAStageCols);
-#pragma unroll
-                    for (int k16 = 0; k16 < 4; ++k16)
-                        umma_ts(dcol, acol + 8 * k16, bd + 2 * k16, idesc, (kk | k16) ? 1u : 0u);
-                    umma_commit(&a_empty[s]);
+                    const uint32_t acol = acol0 + (uint32_t)(as * kAStageCols);
+                    umma_ts(dcol, acol, bd, idesc, kk ? 1u : 0u);
+                    umma_ts(dcol, acol + 8, bd + 2, idesc, 1u);
+                    umma_ts(dcol, acol + 16, bd + 4, idesc, 1u);
+                    umma_ts(dcol, acol + 24, bd + 6, idesc, 1u);
+                    umma_commit(&a_empty[as]);
                     umma_commit(&t_empty[ts]);
-                    tr.advance<kTStages>();
+                    ts = (ts + 1 == kTStages) ? 0 : ts + 1;
+                    as = (as + 1 == kAStages) ? 0 : as + 1;
                 }
                 if (!ok) break;
-                umma_commit(&d_full[b]);
-                dr.advance<2>();
+                umma_commit(&d_full[db]);
+                db ^= 1;
+                ntok = ntok_next;
             }
             // every MMA issued by this thread has finished before TMEM is freed
             umma_commit(drain);
