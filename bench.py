@@ -174,10 +174,17 @@ def measured_peaks() -> tuple[dict, str]:
                  "bf16_tflops_sustained": FALLBACK_BF16_TFLOPS_SUSTAINED}, "fallback")
 
 
-def kernel_source_hash() -> str:
+# the source files each profiled kernel is built from
+KERNEL_SOURCES = {
+    "k_decode_gateup": ["decode.cu", "common.cuh", "internal.h"],
+    "k_prefill_gateup": ["prefill.cu", "common.cuh", "internal.h"],
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "mixed_precision_expert_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in KERNEL_SOURCES[kernel]:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode())
             h.update(f.read())
@@ -185,8 +192,8 @@ def kernel_source_hash() -> str:
 
 
 def recorded_traffic(kernel: str, workload: str) -> float | None:
-    """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current kernel sources."""
+    """DRAM bytes per launch from a committed ncu summary (profiles/traffic.json),
+    if it was taken on the kernel's current sources."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
@@ -194,7 +201,7 @@ def recorded_traffic(kernel: str, workload: str) -> float | None:
     except (OSError, ValueError):
         return None
     ent = rec.get(f"{kernel}:{workload}")
-    if not ent or ent.get("source_hash") != kernel_source_hash():
+    if not ent or ent.get("source_hash") != kernel_source_hash(kernel):
         return None
     return float(ent["dram_bytes_per_launch"])
 
