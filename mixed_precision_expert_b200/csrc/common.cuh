@@ -273,4 +273,46 @@ __device__ __forceinline__ uint32_t unpack_pair<3>(const uint32_t* w, int m) {
     return bf2_sub(and_or(x, 0x00070007u, kMagic), kBf2_132);  // 128 + u - 132
 }
 
+// Offset form of the unpack for b = 3, 4: the same single lop3 per field without
+// the subtraction, i.e. the exact bf16 integer k + off instead of k, with
+//   b = 4: off = 136 (128 + 8) for every code;
+//   b = 3: off = 132 (128 + 4) for the fields at bits 0-2 / 6-8 / 12-14 and the
+//          assembled 16th pair, and off = 20 (16 + 4) for the fields at bits 3-5 /
+//          9-11, which OR into bf16 16.0 (mantissa unit 1/8, so 16 + u exactly).
+// An MMA over these values gives K x + off . x; the decode kernels subtract the
+// off . x term, computed by one more MMA whose A operand is the constant offset
+// pattern, in fp32.
+constexpr uint32_t kMagic16 = 0x41804180u;  // bf16x2 (16, 16)
+
+template <int B>
+__device__ __forceinline__ uint32_t unpack_pair_off(const uint32_t* w, int m);
+
+template <>
+__device__ __forceinline__ uint32_t unpack_pair_off<4>(const uint32_t* w, int m) {
+    const uint32_t v = (m & 3) ? shr(w[m >> 2], 4 * (m & 3)) : w[m >> 2];
+    return and_or(v, 0x000F000Fu, kMagic);
+}
+
+template <>
+__device__ __forceinline__ uint32_t unpack_pair_off<3>(const uint32_t* w, int m) {
+    if (m == 15) {
+        uint32_t t = and_or(shr(w[0], 15), 0x00010001u, kMagic);
+        t = and_or(shr(w[1], 14), 0x00020002u, t);
+        return and_or(shr(w[2], 13), 0x00040004u, t);
+    }
+    const int v = m / 5, f = m % 5;
+    const int sh = f < 2 ? 0 : (f < 4 ? 6 : 12);
+    const uint32_t x = sh ? shr(w[v], sh) : w[v];
+    if (f == 1 || f == 3) return and_or(x, 0x00380038u, kMagic16);  // 16 + u
+    return and_or(x, 0x00070007u, kMagic);                            // 128 + u
+}
+
+// bf16x2 offset of pair m (both halves) in the offset form above.
+template <int B>
+__host__ __device__ constexpr uint32_t pair_offset(int m) {
+    return B == 4 ? 0x43084308u                                             // 136
+                  : ((m < 15 && (m % 5 == 1 || m % 5 == 3)) ? 0x41A041A0u   // 20
+                                                            : 0x43044304u);  // 132
+}
+
 }  // namespace mpe

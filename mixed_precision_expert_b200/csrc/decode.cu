@@ -131,25 +131,46 @@ __device__ __forceinline__ void load_act_half(const __nv_bfloat16* row, int j, i
 }
 
 // Unpack and multiply one block (128 codes of 16 rows, NM matrices) with NT
-// 8-token n-tiles of activations.
+// 8-token n-tiles of activations. Widths 3 and 4 unpack to the offset form
+// (k + off, see common.cuh) and accumulate off . x once per n-tile in accc,
+// which the caller subtracts before finishing the task; width 8 unpacks to k.
 template <int B, int NM, int NT>
 __device__ __forceinline__ void block_mma(const uint32_t (&wr)[NM][2][Geo<B, 1>::WORDS],
                                           const uint32_t (&xa)[kMaxTiles][8],
                                           const uint32_t (&xz)[kMaxTiles][8],
-                                          float (&acc)[kMaxTiles][NM][4]) {
+                                          float (&acc)[kMaxTiles][NM][4],
+                                          float (&accc)[kMaxTiles][4]) {
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
 #pragma unroll
         for (int m = 0; m < NM; ++m) {
-            const uint32_t a0 = unpack_pair<B>(wr[m][0], 2 * c);
-            const uint32_t a1 = unpack_pair<B>(wr[m][1], 2 * c);
-            const uint32_t a2 = unpack_pair<B>(wr[m][0], 2 * c + 1);
-            const uint32_t a3 = unpack_pair<B>(wr[m][1], 2 * c + 1);
+            uint32_t a0, a1, a2, a3;
+            if constexpr (B == 8) {
+                a0 = unpack_pair<B>(wr[m][0], 2 * c);
+                a1 = unpack_pair<B>(wr[m][1], 2 * c);
+                a2 = unpack_pair<B>(wr[m][0], 2 * c + 1);
+                a3 = unpack_pair<B>(wr[m][1], 2 * c + 1);
+            } else {
+                a0 = unpack_pair_off<B>(wr[m][0], 2 * c);
+                a1 = unpack_pair_off<B>(wr[m][1], 2 * c);
+                a2 = unpack_pair_off<B>(wr[m][0], 2 * c + 1);
+                a3 = unpack_pair_off<B>(wr[m][1], 2 * c + 1);
+            }
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
                 const uint32_t b0 = c < 4 ? xa[nt][2 * c] : xz[nt][2 * c - 8];
                 const uint32_t b1 = c < 4 ? xa[nt][2 * c + 1] : xz[nt][2 * c - 7];
                 mma_bf16_16816(acc[nt][m], a0, a1, a2, a3, b0, b1);
+            }
+        }
+        if constexpr (B != 8) {
+            // rows of the offset matrix are all alike: rows g and g+8 share a value
+            const uint32_t o0 = pair_offset<B>(2 * c), o1 = pair_offset<B>(2 * c + 1);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const uint32_t b0 = c < 4 ? xa[nt][2 * c] : xz[nt][2 * c - 8];
+                const uint32_t b1 = c < 4 ? xa[nt][2 * c + 1] : xz[nt][2 * c - 7];
+                mma_bf16_16816(accc[nt], o0, o0, o1, o1, b0, b1);
             }
         }
     }
@@ -329,7 +350,19 @@ __device__ __forceinline__ bool consume_class(const Args& a, const CtaSmem& sm, 
     const __nv_bfloat16* arow[kMaxTiles] = {nullptr, nullptr};
     int ntiles = 0;
     float acc[kMaxTiles][NM][4];
+    float accc[kMaxTiles][4];  // offset term (widths 3, 4), subtracted at the task's end
     uint32_t xa[kMaxTiles][8], xz[kMaxTiles][8];
+    // acc <- acc - off . x for every matrix (a no-op for width 8)
+    auto settle = [&]() {
+        if constexpr (B != 8) {
+#pragma unroll
+            for (int nt = 0; nt < kMaxTiles; ++nt)
+#pragma unroll
+                for (int m = 0; m < NM; ++m)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) acc[nt][m][q] -= accc[nt][q];
+        }
+    };
     for (int s = 0;; s = (s + 1 == S) ? 0 : s + 1) {
         const uint32_t par = (fp >> s) & 1u;
         fp ^= 1u << s;
@@ -339,13 +372,17 @@ __device__ __forceinline__ bool consume_class(const Args& a, const CtaSmem& sm, 
         }
         const SlotDesc d = sm.descs[s];
         if (d.task < 0) {  // terminator
+            settle();
             finish<GATEUP>(a, T, acc, lane);
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.empty[s]);
             return true;
         }
         if (d.task != cur) {
-            if (cur >= 0) finish<GATEUP>(a, T, acc, lane);
+            if (cur >= 0) {
+                settle();
+                finish<GATEUP>(a, T, acc, lane);
+            }
             cur = d.task;
             int tq;
             split_task(cur, n_tq, a.parts, T.gi, tq, T.p);
@@ -371,6 +408,8 @@ __device__ __forceinline__ bool consume_class(const Args& a, const CtaSmem& sm, 
                 for (int m = 0; m < NM; ++m)
 #pragma unroll
                     for (int q = 0; q < 4; ++q) acc[nt][m][q] = 0.0f;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) accc[nt][q] = 0.0f;
             }
         }
         const int j = d.j;
@@ -391,9 +430,9 @@ __device__ __forceinline__ bool consume_class(const Args& a, const CtaSmem& sm, 
         if (ntiles > 1) {
             load_act_half(arow[1], j, t, B == 8, 0, xa[1]);
             load_act_half(arow[1], j, t, B == 8, 1, xz[1]);
-            block_mma<B, NM, kMaxTiles>(wr, xa, xz, acc);
+            block_mma<B, NM, kMaxTiles>(wr, xa, xz, acc, accc);
         } else {
-            block_mma<B, NM, 1>(wr, xa, xz, acc);
+            block_mma<B, NM, 1>(wr, xa, xz, acc, accc);
         }
     }
 }
