@@ -42,11 +42,16 @@ constexpr int kRingBytes = 96 * 1024;            // shared-memory ring per CTA
 constexpr int kMaxSlots = 16;
 constexpr int kMaxTiles = kDecodeGroup / 8;
 
+// A slot holds J consecutive block columns of 8 tiles. The bulk-copy engine
+// takes ~80 cycles per copy whatever its size up to a few KB, so the chunks of
+// a tile's consecutive block columns -- adjacent in its page -- go in one copy:
+// J = 2 for 3 and 4 bits (1.5 / 2 KB copies), 1 for 8 bits (2 KB chunks).
 template <int B, int NM>
 struct Geo {
     static constexpr int CB = 256 * B;                   // chunk bytes
-    static constexpr int TILE = NM * CB;                 // one warp's share of a slot
-    static constexpr int SLOT = kConsumers * TILE;       // one block column of 8 tiles
+    static constexpr int J = (B == 8) ? 1 : 2;           // block columns per slot
+    static constexpr int TILE = NM * J * CB;             // one warp's share of a slot
+    static constexpr int SLOT = kConsumers * TILE;       // J block columns of 8 tiles
     static constexpr int S = (kRingBytes / SLOT) < kMaxSlots ? (kRingBytes / SLOT) : kMaxSlots;
     static constexpr int WORDS = (B == 8) ? 8 : B;       // raw words per row
     static_assert(S >= 3, "ring geometry");
@@ -54,7 +59,8 @@ struct Geo {
 
 struct SlotDesc {
     int task;  // -1: no more tasks of this class
-    int j;     // block column held by the slot
+    int j;     // first block column held by the slot
+    int nc;    // block columns held (1 .. J)
 };
 
 struct Args {
@@ -307,23 +313,37 @@ __device__ __forceinline__ bool produce_class(const Args& a, const CtaSmem& sm, 
                 pre_row = a.act + (size_t)(GATEUP ? (a.perm[pos] / a.k) : pos) * K;
             }
         }
+        const int jc = min(G::J, j_hi - j);  // block columns in this slot
         if (lane == 0) {
-            sm.descs[s] = SlotDesc{task, j};
-            mbar_arrive_expect_tx(&sm.full[s], (uint32_t)(active * G::TILE));
+            sm.descs[s] = SlotDesc{task, j, jc};
+            mbar_arrive_expect_tx(&sm.full[s], (uint32_t)(active * NM * jc * G::CB));
         }
         __syncwarp();
         if (my_tile) {
-            const uint8_t* src = P.pool + (size_t)P.pidx[first + pslot] * P.page_bytes +
-                                 (size_t)poff * G::CB;
-            bulk_g2s(sm.ring + (size_t)s * G::SLOT + (size_t)lane * G::CB, src, (uint32_t)G::CB,
-                     &sm.full[s]);
-            if (++poff == cpp) {
+            // jc consecutive chunks of this (tile, matrix); a page boundary splits
+            // the copy in two
+            uint8_t* dst = sm.ring + (size_t)s * G::SLOT + (size_t)lane * G::J * G::CB;
+            const int n1 = min(jc, cpp - poff);
+            bulk_g2s(dst, P.pool + (size_t)P.pidx[first + pslot] * P.page_bytes +
+                              (size_t)poff * G::CB,
+                     (uint32_t)(n1 * G::CB), &sm.full[s]);
+            poff += n1;
+            if (poff == cpp) {
                 ++pslot;
                 poff = 0;
             }
+            if (n1 < jc) {
+                bulk_g2s(dst + n1 * G::CB, P.pool + (size_t)P.pidx[first + pslot] * P.page_bytes,
+                         (uint32_t)((jc - n1) * G::CB), &sm.full[s]);
+                poff = jc - n1;
+            }
         }
-        if (pre_row) prefetch_l1(pre_row + 128 * j + 64 * pre_half);
-        ++j;
+        if (pre_row) {
+#pragma unroll
+            for (int jj = 0; jj < G::J; ++jj)
+                if (jj < jc) prefetch_l1(pre_row + 128 * (j + jj) + 64 * pre_half);
+        }
+        j += jc;
         s = (s + 1 == S) ? 0 : s + 1;
     }
 }
@@ -412,27 +432,36 @@ __device__ __forceinline__ bool consume_class(const Args& a, const CtaSmem& sm, 
                 for (int q = 0; q < 4; ++q) accc[nt][q] = 0.0f;
             }
         }
-        const int j = d.j;
-        uint32_t wr[NM][2][G::WORDS];
-        if (T.valid) {
-            const uint8_t* tile = sm.ring + (size_t)s * G::SLOT + (size_t)w * G::TILE;
+        if (!T.valid) {  // this warp has no tile in the task: release at once
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.empty[s]);
+            continue;
+        }
+        const uint8_t* tile = sm.ring + (size_t)s * G::SLOT + (size_t)w * G::TILE;
+#pragma unroll
+        for (int jj = 0; jj < G::J; ++jj) {
+            if (jj >= d.nc) break;
+            uint32_t wr[NM][2][G::WORDS];
 #pragma unroll
             for (int m = 0; m < NM; ++m) {
-                load_row_words<B>(tile + m * G::CB, g, t, g, wr[m][0]);
-                load_row_words<B>(tile + m * G::CB, g + 8, t, g, wr[m][1]);
+                const uint8_t* chunk = tile + (m * G::J + jj) * G::CB;
+                load_row_words<B>(chunk, g, t, g, wr[m][0]);
+                load_row_words<B>(chunk, g + 8, t, g, wr[m][1]);
             }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.empty[s]);  // words are in registers: release the slot
-        if (!T.valid) continue;
-        load_act_half(arow[0], j, t, B == 8, 0, xa[0]);
-        load_act_half(arow[0], j, t, B == 8, 1, xz[0]);
-        if (ntiles > 1) {
-            load_act_half(arow[1], j, t, B == 8, 0, xa[1]);
-            load_act_half(arow[1], j, t, B == 8, 1, xz[1]);
-            block_mma<B, NM, kMaxTiles>(wr, xa, xz, acc, accc);
-        } else {
-            block_mma<B, NM, 1>(wr, xa, xz, acc, accc);
+            if (jj + 1 == d.nc) {  // the slot's last words are in registers: release it
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.empty[s]);
+            }
+            const int j = d.j + jj;
+            load_act_half(arow[0], j, t, B == 8, 0, xa[0]);
+            load_act_half(arow[0], j, t, B == 8, 1, xz[0]);
+            if (ntiles > 1) {
+                load_act_half(arow[1], j, t, B == 8, 0, xa[1]);
+                load_act_half(arow[1], j, t, B == 8, 1, xz[1]);
+                block_mma<B, NM, kMaxTiles>(wr, xa, xz, acc, accc);
+            } else {
+                block_mma<B, NM, 1>(wr, xa, xz, acc, accc);
+            }
         }
     }
 }
