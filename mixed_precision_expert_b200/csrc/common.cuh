@@ -12,9 +12,11 @@
 //          c'_30 / c'_31 is bit 15 / 31 of word n (n < 3)
 // so each pair (c'_{2m}, c'_{2m+1}) sits in matching positions of the two
 // 16-bit halves of a word and unpacks to one bf16x2 register.
-// An expert stream is the chunks of W1 (gate [F x H]), W3 (up [F x H]) and W2
-// (down [H x F]); chunk c of an expert lives in page pidx[first + c / cpp] at
-// byte (c % cpp) * 256 b, cpp = page_bytes / (256 b).
+// An expert stream is the chunks of W1 (gate [F x H]) and W3 (up [F x H])
+// interleaved -- chunk 2c is W1's chunk c, 2c+1 is W3's -- then those of W2
+// (down [H x F]); a tile's gate and up chunks for consecutive block columns are
+// therefore one contiguous run. Chunk c of an expert lives in page
+// pidx[first + c / cpp] at byte (c % cpp) * 256 b, cpp = page_bytes / (256 b).
 #pragma once
 
 #include <cstdint>
@@ -59,7 +61,8 @@ __device__ __forceinline__ void set_status(uint32_t* status, uint32_t bit) {
     atomicOr(status, bit);
 }
 
-// chunk index offsets of the three matrices inside an expert stream
+// chunks of one [F x H] matrix: the stream holds 2 of these interleaved (W1, W3),
+// then W2's chunks from index 2 * chunks_w1
 __host__ __device__ inline int chunks_w1(int H, int F) { return (F / 16) * (H / 128); }
 
 // Address of chunk c of an expert.

@@ -43,18 +43,20 @@ constexpr int kMaxSlots = 16;
 constexpr int kMaxTiles = kDecodeGroup / 8;
 
 // A slot holds J consecutive block columns of 8 tiles. The bulk-copy engine
-// takes ~80 cycles per copy whatever its size up to a few KB, so the chunks of
-// a tile's consecutive block columns -- adjacent in its page -- go in one copy:
-// J = 2 for 3 and 4 bits (1.5 / 2 KB copies), 1 for 8 bits (2 KB chunks).
+// takes ~80 cycles per copy whatever its size up to a few KB, so a tile's
+// chunks for the slot -- gate and up interleaved, consecutive block columns,
+// one contiguous run of its page -- go in one copy, as many columns as keep a
+// slot within 32 KB (three slots per 96 KB ring): gate/up 2 (3, 4 bits) or 1
+// (8 bits), down 5 / 4 / 2.
 template <int B, int NM>
 struct Geo {
     static constexpr int CB = 256 * B;                   // chunk bytes
-    static constexpr int J = (B == 8) ? 1 : 2;           // block columns per slot
+    static constexpr int J = 32768 / (kConsumers * NM * CB);  // block columns per slot
     static constexpr int TILE = NM * J * CB;             // one warp's share of a slot
     static constexpr int SLOT = kConsumers * TILE;       // J block columns of 8 tiles
     static constexpr int S = (kRingBytes / SLOT) < kMaxSlots ? (kRingBytes / SLOT) : kMaxSlots;
     static constexpr int WORDS = (B == 8) ? 8 : B;       // raw words per row
-    static_assert(S >= 3, "ring geometry");
+    static_assert(S >= 3 && J >= 1, "ring geometry");
 };
 
 struct SlotDesc {
@@ -233,10 +235,10 @@ struct CtaSmem {
     SlotDesc* descs;
 };
 
-// Producer warp: all tasks of one width class. Lane l < 8*NM owns the copy
-// stream of tile l / NM, matrix l % NM (a page cursor in registers); lane 0
-// claims tasks, arms the full barriers and writes the slot descriptors; every
-// lane prefetches one activation line. `ep`/`used` track the empty barriers'
+// Producer warp: all tasks of one width class. Lane l < 8 owns the copy stream
+// of tile l (a page cursor in registers): per slot one run of NM x jc chunks
+// (gate/up: W1 and W3 alternate). Lane 0 claims tasks, arms the full barriers
+// and writes the slot descriptors; every lane prefetches one activation line. `ep`/`used` track the empty barriers'
 // phases per slot across classes.
 template <int B, bool GATEUP>
 __device__ __forceinline__ bool produce_class(const Args& a, const CtaSmem& sm, int group0,
@@ -256,8 +258,8 @@ __device__ __forceinline__ bool produce_class(const Args& a, const CtaSmem& sm, 
     const int n_tasks = n_groups * n_tq * a.parts;
     if (n_tasks == 0) return true;
     const int cpp = chunks_per_page(B, P.page_bytes);
-    const int my_w = lane / NM, my_m = lane % NM;
-    const bool copier = lane < kConsumers * NM;
+    const int my_w = lane;
+    const bool copier = lane < kConsumers;
 
     int s = 0;
     int task = -1, j = 0, j_hi = 0;
@@ -302,7 +304,7 @@ __device__ __forceinline__ bool produce_class(const Args& a, const CtaSmem& sm, 
             const int tau = tq * kConsumers + my_w;
             my_tile = copier && my_w < active;
             if (my_tile) {
-                const int c = (GATEUP ? my_m * nc1 : 2 * nc1) + tau * nj + j;
+                const int c = GATEUP ? 2 * (tau * nj + j) : 2 * nc1 + tau * nj + j;
                 pslot = c / cpp;
                 poff = c - pslot * cpp;
             }
@@ -320,10 +322,11 @@ __device__ __forceinline__ bool produce_class(const Args& a, const CtaSmem& sm, 
         }
         __syncwarp();
         if (my_tile) {
-            // jc consecutive chunks of this (tile, matrix); a page boundary splits
-            // the copy in two
-            uint8_t* dst = sm.ring + (size_t)s * G::SLOT + (size_t)lane * G::J * G::CB;
-            const int n1 = min(jc, cpp - poff);
+            // NM x jc consecutive chunks of this tile; a page boundary splits the
+            // copy in two
+            uint8_t* dst = sm.ring + (size_t)s * G::SLOT + (size_t)lane * G::TILE;
+            const int total = NM * jc;
+            const int n1 = min(total, cpp - poff);
             bulk_g2s(dst, P.pool + (size_t)P.pidx[first + pslot] * P.page_bytes +
                               (size_t)poff * G::CB,
                      (uint32_t)(n1 * G::CB), &sm.full[s]);
@@ -332,10 +335,10 @@ __device__ __forceinline__ bool produce_class(const Args& a, const CtaSmem& sm, 
                 ++pslot;
                 poff = 0;
             }
-            if (n1 < jc) {
+            if (n1 < total) {
                 bulk_g2s(dst + n1 * G::CB, P.pool + (size_t)P.pidx[first + pslot] * P.page_bytes,
-                         (uint32_t)((jc - n1) * G::CB), &sm.full[s]);
-                poff = jc - n1;
+                         (uint32_t)((total - n1) * G::CB), &sm.full[s]);
+                poff = total - n1;
             }
         }
         if (pre_row) {
@@ -444,7 +447,7 @@ __device__ __forceinline__ bool consume_class(const Args& a, const CtaSmem& sm, 
             uint32_t wr[NM][2][G::WORDS];
 #pragma unroll
             for (int m = 0; m < NM; ++m) {
-                const uint8_t* chunk = tile + (m * G::J + jj) * G::CB;
+                const uint8_t* chunk = tile + (jj * NM + m) * G::CB;
                 load_row_words<B>(chunk, g, t, g, wr[m][0]);
                 load_row_words<B>(chunk, g + 8, t, g, wr[m][1]);
             }

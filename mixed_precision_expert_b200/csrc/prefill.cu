@@ -226,11 +226,14 @@ __device__ __forceinline__ bool produce_tile(const PArgs& a, const Tile& T, int 
     const int nc1 = chunks_w1(H, F);
     const int cpp = chunks_per_page(B, P.page_bytes);
     // this thread's A row: gate/up feature nt*64 + 16 lq + lane/2 of W1 (even
-    // lanes) or W3 (odd lanes); down: output nt*128 + 32 lq + lane of W2
+    // lanes) or W3 (odd lanes); down: output nt*128 + 32 lq + lane of W2. Its
+    // chunk for block column j is c + cs * j: the stream interleaves W1 and W3
+    // chunks (cs = 2), W2's are consecutive (cs = 1).
+    constexpr int cs = GATEUP ? 2 : 1;
     int c, rr;
     if (GATEUP) {
         const int f = T.nt * 64 + lq * 16 + (lane >> 1);
-        c = (lane & 1) * nc1 + (f >> 4) * nj;
+        c = 2 * ((f >> 4) * nj) + (lane & 1);
         rr = f & 15;
     } else {
         const int o = T.nt * 128 + lq * 32 + lane;
@@ -247,12 +250,12 @@ __device__ __forceinline__ bool produce_tile(const PArgs& a, const Tile& T, int 
     // a second cursor kPrefetch block columns ahead pulls this row's packed words
     // into L2 (no registers held), so the register loads one block ahead hit L2
     constexpr int kPrefetch = 4;
-    int fslot = (c + kPrefetch) / cpp;
-    int foff = (c + kPrefetch) - fslot * cpp;
-    const int fmax = c + nj;  // the row's chunks end here
-    int fchunk = c + kPrefetch;
+    int fslot = (c + kPrefetch * cs) / cpp;
+    int foff = (c + kPrefetch * cs) - fslot * cpp;
+    const int fmax = c + nj * cs;  // the row's chunks end here
+    int fchunk = c + kPrefetch * cs;
     for (int i = 1; i < kPrefetch && i < nj; ++i) {
-        const int ci = c + i;
+        const int ci = c + i * cs;
         const int si = ci / cpp;
         prefetch_l2(P.pool + (size_t)P.pidx[T.first + si] * P.page_bytes +
                     (size_t)(ci - si * cpp) * chunk_bytes(B) + off);
@@ -266,19 +269,21 @@ __device__ __forceinline__ bool produce_tile(const PArgs& a, const Tile& T, int 
             const int j = j0 + ui;
             if (j >= nj) break;
             if (j + 1 < nj) {
-                if (++poff == cpp) {
+                poff += cs;
+                if (poff >= cpp) {
+                    poff -= cpp;
                     ++pslot;
-                    poff = 0;
                 }
                 load_half<B>(src(), ring[ui ^ 1]);
             }
             if (fchunk < fmax) {
                 prefetch_l2(P.pool + (size_t)P.pidx[T.first + fslot] * P.page_bytes +
                             (size_t)foff * chunk_bytes(B) + off);
-                ++fchunk;
-                if (++foff == cpp) {
+                fchunk += cs;
+                foff += cs;
+                if (foff >= cpp) {
+                    foff -= cpp;
                     ++fslot;
-                    foff = 0;
                 }
             }
             const uint32_t g = g0 + 2 * j + hp;

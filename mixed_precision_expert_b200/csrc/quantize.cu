@@ -170,12 +170,11 @@ k_encode(PagedExperts P, const void* const* masters, const int32_t* list) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int c = blockIdx.x * 8 + warp;
     if (c >= 3 * nc1) return;
+    // stream chunk c: W1 / W3 chunks alternate (2 cc + m), then W2's chunks
     int K, cc;
     size_t moff;
-    if (c < nc1) {
-        K = H; cc = c; moff = 0;
-    } else if (c < 2 * nc1) {
-        K = H; cc = c - nc1; moff = (size_t)F * H;
+    if (c < 2 * nc1) {
+        K = H; cc = c >> 1; moff = (c & 1) ? (size_t)F * H : 0;
     } else {
         K = F; cc = c - 2 * nc1; moff = 2 * (size_t)F * H;
     }

@@ -13,8 +13,11 @@ needs R % 16 == 0 and K % 128 == 0.
 * chunk   -- 16 blocks: rows 16*tau .. 16*tau + 15, block column j; 256*b bytes.
              Block of row 16*tau + rho sits at byte offset 16*b*rho.
              Chunks of a matrix run tau-major: chunk index c = tau*(K/128) + j.
-* expert stream -- the chunks of W1 (gate, [F x H]), then W3 (up, [F x H]),
-             then W2 (down, [H x F]).
+* expert stream -- the chunks of W1 (gate, [F x H]) and W3 (up, [F x H])
+             interleaved, chunk 2c = W1's chunk c and 2c+1 = W3's chunk c, then
+             the chunks of W2 (down, [H x F]). A gate row's block and the up
+             row's block for the same feature and K range are thus adjacent, and
+             so are a tile's consecutive block columns of both.
 
 Inside a quarter the 32 codes c'_0 .. c'_31 are b little-endian 32-bit words:
 * b = 8: word w (0..7) holds c'_{4w+i} at bit 16*(i&1) + 8*(i>>1), i = 0..3.
@@ -142,5 +145,8 @@ def n_chunks(H: int, F: int) -> int:
 
 
 def expert_stream(u1: np.ndarray, u3: np.ndarray, u2: np.ndarray, b: int) -> np.ndarray:
-    """Chunk stream of one expert: W1, then W3, then W2. uint8 [n_chunks, 256*b]."""
-    return np.concatenate([pack_matrix(u1, b), pack_matrix(u3, b), pack_matrix(u2, b)])
+    """Chunk stream of one expert: W1 and W3 chunk by chunk (W1 chunk c at 2c,
+    W3 chunk c at 2c + 1), then W2. uint8 [n_chunks, 256*b]."""
+    g1, g3 = pack_matrix(u1, b), pack_matrix(u3, b)
+    gu = np.stack([g1, g3], axis=1).reshape(2 * g1.shape[0], chunk_bytes(b))
+    return np.concatenate([gu, pack_matrix(u2, b)])

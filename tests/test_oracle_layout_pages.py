@@ -115,9 +115,19 @@ def test_expert_stream_order():
     n = L.n_chunks(H, F)
     assert s.shape[0] == n == 3 * (F // 16) * (H // 128)
     third = n // 3
-    # constant codes -> every nibble equal; W1, W3, W2 in that order
-    assert np.all(s[:third] == 0x11) and np.all(s[third:2 * third] == 0x22)
+    # constant codes -> every nibble equal; W1 and W3 chunks alternate, then W2
+    assert np.all(s[0:2 * third:2] == 0x11) and np.all(s[1:2 * third:2] == 0x22)
     assert np.all(s[2 * third:] == 0x33)
+    # distinct codes per matrix row: chunk 2c is W1's chunk c, 2c+1 is W3's
+    H, F = 256, 128
+    rng = np.random.default_rng(1)
+    u1 = rng.integers(0, 16, size=(F, H)).astype(np.uint32)
+    u3 = rng.integers(0, 16, size=(F, H)).astype(np.uint32)
+    u2 = rng.integers(0, 16, size=(H, F)).astype(np.uint32)
+    s = L.expert_stream(u1, u3, u2, b)
+    g1, g3 = L.pack_matrix(u1, b), L.pack_matrix(u3, b)
+    for c in range(g1.shape[0]):
+        assert np.array_equal(s[2 * c], g1[c]) and np.array_equal(s[2 * c + 1], g3[c])
 
 
 # ----------------------------------------------------------------------------
