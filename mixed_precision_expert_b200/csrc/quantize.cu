@@ -69,30 +69,29 @@ __global__ void k_scales(Pte* pte, const uint32_t* absmax, int E, uint32_t* stat
     pte[e].scale = (m == 0) ? 0.0f : __fdiv_rn(mf, (float)q_levels(b));
 }
 
+// Rare path of encode_one: r lies within 2^-11 of a half-integer, so the exact
+// quotient w / s decides. The sign of the single-rounded fma (k -+ 1/2) s - w is
+// exact: ties go to the even integer.
+__device__ __noinline__ float tie_fix(float w, float s, float kf) {
+    const float lo = __fmaf_rn(__fsub_rn(kf, 0.5f), s, -w);  // (k - 1/2) s - w
+    const float hi = __fmaf_rn(__fadd_rn(kf, 0.5f), s, -w);  // (k + 1/2) s - w
+    const bool odd = (((int)kf) & 1) != 0;
+    if (lo > 0.0f) return __fsub_rn(kf, 1.0f);
+    if (hi < 0.0f) return __fadd_rn(kf, 1.0f);
+    if (lo == 0.0f && odd) return __fsub_rn(kf, 1.0f);
+    if (hi == 0.0f && odd) return __fadd_rn(kf, 1.0f);
+    return kf;
+}
+
 // k = round-half-even(w / s), exactly, clamped; returns offset-binary u = k + 2^(b-1).
 // r = w * (1/s) is within ~2^-16 of the exact quotient (|w/s| < 2^8), so
-// rounding r agrees with rounding the exact quotient unless r lies within
-// that distance of a half-integer; there the sign of the single-rounded
-// fma (k -+ 1/2) s - w decides exactly.
+// rounding r (one round-to-integral, ties to even) agrees with rounding the
+// exact quotient unless r lies within that distance of a half-integer, which
+// tie_fix settles.
 __device__ __forceinline__ uint32_t encode_one(float w, float s, float inv_s, float qf, int off) {
     const float r = __fmul_rn(w, inv_s);
-    const float kr = __fsub_rn(__fadd_rn(r, 12582912.0f), 12582912.0f);  // RNE to integer
-    float kf = kr;
-    const float d = __fsub_rn(r, kr);
-    if (fabsf(d) > 0.4990234375f) {
-        const float lo = __fmaf_rn(__fsub_rn(kf, 0.5f), s, -w);  // (k - 1/2) s - w
-        const float hi = __fmaf_rn(__fadd_rn(kf, 0.5f), s, -w);  // (k + 1/2) s - w
-        const bool odd = (((int)kf) & 1) != 0;
-        if (lo > 0.0f) {
-            kf = __fsub_rn(kf, 1.0f);
-        } else if (hi < 0.0f) {
-            kf = __fadd_rn(kf, 1.0f);
-        } else if (lo == 0.0f) {
-            if (odd) kf = __fsub_rn(kf, 1.0f);
-        } else if (hi == 0.0f) {
-            if (odd) kf = __fadd_rn(kf, 1.0f);
-        }
-    }
+    float kf = rintf(r);
+    if (fabsf(__fsub_rn(r, kf)) > 0.4990234375f) kf = tie_fix(w, s, kf);
     kf = fminf(fmaxf(kf, -qf), qf);
     return (uint32_t)((int)kf + off);
 }
@@ -128,7 +127,7 @@ __device__ __forceinline__ void encode_quarter(const __half* src, float s, float
         uint32_t wv[8];
 #pragma unroll
         for (int w = 0; w < 8; ++w)
-            wv[w] = u[4 * w] | (u[4 * w + 1] << 16) | (u[4 * w + 2] << 8) | (u[4 * w + 3] << 24);
+            wv[w] = u[4 * w] + (u[4 * w + 1] << 16) + (u[4 * w + 2] << 8) + (u[4 * w + 3] << 24);
         reinterpret_cast<uint4*>(dst)[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
         reinterpret_cast<uint4*>(dst)[1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
     } else if constexpr (B == 4) {
@@ -137,7 +136,7 @@ __device__ __forceinline__ void encode_quarter(const __half* src, float s, float
         for (int w = 0; w < 4; ++w) {
             uint32_t x = 0;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) x |= u[8 * w + i] << (16 * (i & 1) + 4 * (i >> 1));
+            for (int i = 0; i < 8; ++i) x += u[8 * w + i] << (16 * (i & 1) + 4 * (i >> 1));
             wv[w] = x;
         }
         reinterpret_cast<uint4*>(dst)[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
@@ -147,9 +146,9 @@ __device__ __forceinline__ void encode_quarter(const __half* src, float s, float
         for (int v = 0; v < 3; ++v) {
             uint32_t x = 0;
 #pragma unroll
-            for (int i = 0; i < 10; ++i) x |= u[10 * v + i] << (16 * (i & 1) + 3 * (i >> 1));
-            x |= ((u[30] >> v) & 1u) << 15;
-            x |= ((u[31] >> v) & 1u) << 31;
+            for (int i = 0; i < 10; ++i) x += u[10 * v + i] << (16 * (i & 1) + 3 * (i >> 1));
+            x += ((u[30] >> v) & 1u) << 15;
+            x += ((u[31] >> v) & 1u) << 31;
             d32[v] = x;
         }
     }
