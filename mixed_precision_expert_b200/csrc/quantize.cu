@@ -84,16 +84,19 @@ __device__ __noinline__ float tie_fix(float w, float s, float kf) {
 }
 
 // k = round-half-even(w / s), exactly, clamped; returns offset-binary u = k + 2^(b-1).
-// r = w * (1/s) is within ~2^-16 of the exact quotient (|w/s| < 2^8), so
-// rounding r (one round-to-integral, ties to even) agrees with rounding the
-// exact quotient unless r lies within that distance of a half-integer, which
-// tie_fix settles.
-__device__ __forceinline__ uint32_t encode_one(float w, float s, float inv_s, float qf, int off) {
+// r = w * (1/s) is within ~2^-16 of the exact quotient (|w/s| < 2^8). Adding
+// 1.5 * 2^23 rounds r to an integer, ties to even, and leaves that integer in
+// the low mantissa bits, so k is read out with integer operations (no
+// conversion instruction). Rounding r agrees with rounding the exact quotient
+// unless r lies within 2^-11 of a half-integer, which tie_fix settles.
+__device__ __forceinline__ uint32_t encode_one(float w, float s, float inv_s, int q, int off) {
+    constexpr float kRound = 12582912.0f;  // 1.5 * 2^23, bits 0x4B400000
     const float r = __fmul_rn(w, inv_s);
-    float kf = rintf(r);
-    if (fabsf(__fsub_rn(r, kf)) > 0.4990234375f) kf = tie_fix(w, s, kf);
-    kf = fminf(fmaxf(kf, -qf), qf);
-    return (uint32_t)((int)kf + off);
+    const float rf = __fadd_rn(r, kRound);
+    int k = __float_as_int(rf) - 0x4B400000;
+    if (fabsf(__fsub_rn(r, __fsub_rn(rf, kRound))) > 0.4990234375f)
+        k = (int)tie_fix(w, s, (float)k);
+    return (uint32_t)(min(max(k, -q), q) + off);
 }
 
 __device__ __forceinline__ void load32_half(const __half* src, float (&f)[32]) {
@@ -116,13 +119,13 @@ __device__ __forceinline__ void load32_half(const __half* src, float (&f)[32]) {
 template <int B>
 __device__ __forceinline__ void encode_quarter(const __half* src, float s, float inv_s,
                                                uint8_t* dst) {
-    constexpr float qf = (float)q_levels(B);
+    constexpr int q = q_levels(B);
     constexpr int off = 1 << (B - 1);
     float f[32];
     load32_half(src, f);
     uint32_t u[32];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) u[i] = encode_one(f[i], s, inv_s, qf, off);
+    for (int i = 0; i < 32; ++i) u[i] = encode_one(f[i], s, inv_s, q, off);
     if constexpr (B == 8) {
         uint32_t wv[8];
 #pragma unroll
