@@ -30,15 +30,25 @@ __device__ uint64_t gcd_u64(uint64_t a, uint64_t b) {
 }
 
 constexpr int kThreads = 1024;
+// Dynamic shared memory for the two DP rows and the choice table (see below).
+constexpr size_t kAllocSmemMax = 200 * 1024;
 
+// Choices are 2-bit codes (0: 3 bits, 1: 4 bits, 2: 8 bits), four budget
+// states per byte, so thread i owns whole bytes and no two threads write the
+// same byte. When both DP rows and the table fit in shared memory
+// (R <= smem_R; -1 = no on-chip buffers) the whole solve stays on chip -- every expert step is a
+// shared-memory pass plus one barrier, and the serial backtrack reads shared
+// memory -- else rows and table live in the global buffers D and choice.
 __global__ void __launch_bounds__(kThreads)
 k_allocate(const double* p, const uint64_t* W, int E, uint64_t B, uint8_t* bits,
-           int32_t* status, uint8_t* choice, double* D, int state_cap) {
+           int32_t* status, uint8_t* choice, double* D, int state_cap, int64_t smem_R) {
+    extern __shared__ __align__(16) uint8_t dyn[];
     __shared__ int s_mode;      // 0 = solve, 1 = infeasible, 2 = all 8, 3 = state cap
     __shared__ uint32_t s_R;
     __shared__ uint64_t s_g;
     __shared__ uint32_t s_up4[MPE_MAX_EXPERTS];
     __shared__ uint32_t s_up8[MPE_MAX_EXPERTS];
+    __shared__ double s_p[MPE_MAX_EXPERTS];
     const int tid = threadIdx.x;
     if (tid == 0) {
         uint64_t sum_w = 0, g = 0;
@@ -73,49 +83,60 @@ k_allocate(const double* p, const uint64_t* W, int E, uint64_t B, uint8_t* bits,
     if (mode != 0) return;
     const uint32_t R = s_R;
     const uint64_t g = s_g;
+    const uint32_t nq = (R + 4) / 4;  // choice bytes per expert
     for (int e = tid; e < E; e += kThreads) {
         const uint64_t u4 = W[e] / g, u8 = 5 * (W[e] / g);
         s_up4[e] = (uint32_t)min(u4, (uint64_t)R + 1);
         s_up8[e] = (uint32_t)min(u8, (uint64_t)R + 1);
+        s_p[e] = p[e];
     }
+    const bool on_chip = (int64_t)R <= smem_R;
+    double* Dcur = on_chip ? reinterpret_cast<double*>(dyn) : D;
+    double* Dnext = Dcur + (R + 1);
+    uint8_t* chb = on_chip ? dyn + 16 * (size_t)(R + 1) : choice;
     const double L3 = __ddiv_rn(1.0, 9.0);
     const double L4 = __ddiv_rn(1.0, 49.0);
     const double L8 = __ddiv_rn(1.0, 16129.0);
-    double* Dcur = D;
-    double* Dnext = D + (R + 1);
     for (uint32_t r = tid; r <= R; r += kThreads) Dcur[r] = (r == 0) ? 0.0 : dinf();
     __syncthreads();
     for (int e = 0; e < E; ++e) {
-        const double pe = p[e];
+        const double pe = s_p[e];
         const double c3 = __dmul_rn(pe, L3);
         const double c4 = __dmul_rn(pe, L4);
         const double c8 = __dmul_rn(pe, L8);
         const uint32_t u4 = s_up4[e], u8 = s_up8[e];
-        uint8_t* ch = choice + (size_t)e * (R + 1);
-        for (uint32_t r = tid; r <= R; r += kThreads) {
-            double best = dinf();
-            uint8_t bb = 0;
-            double prev = Dcur[r];
-            if (prev != dinf()) {
-                const double cand = __dadd_rn(prev, c3);
-                if (cand < best) { best = cand; bb = 3; }
-            }
-            if (r >= u4) {
-                prev = Dcur[r - u4];
+        uint8_t* ch = chb + (size_t)e * nq;
+        for (uint32_t qd = tid; qd < nq; qd += kThreads) {
+            uint32_t byte = 0;
+#pragma unroll
+            for (uint32_t i = 0; i < 4; ++i) {
+                const uint32_t r = 4 * qd + i;
+                if (r > R) break;
+                double best = dinf();
+                uint32_t code = 0;
+                double prev = Dcur[r];
                 if (prev != dinf()) {
-                    const double cand = __dadd_rn(prev, c4);
-                    if (cand < best) { best = cand; bb = 4; }
+                    const double cand = __dadd_rn(prev, c3);
+                    if (cand < best) { best = cand; code = 0; }
                 }
-            }
-            if (r >= u8) {
-                prev = Dcur[r - u8];
-                if (prev != dinf()) {
-                    const double cand = __dadd_rn(prev, c8);
-                    if (cand < best) { best = cand; bb = 8; }
+                if (r >= u4) {
+                    prev = Dcur[r - u4];
+                    if (prev != dinf()) {
+                        const double cand = __dadd_rn(prev, c4);
+                        if (cand < best) { best = cand; code = 1; }
+                    }
                 }
+                if (r >= u8) {
+                    prev = Dcur[r - u8];
+                    if (prev != dinf()) {
+                        const double cand = __dadd_rn(prev, c8);
+                        if (cand < best) { best = cand; code = 2; }
+                    }
+                }
+                Dnext[r] = best;
+                byte |= code << (2 * i);
             }
-            Dnext[r] = best;
-            ch[r] = bb;
+            ch[qd] = (uint8_t)byte;
         }
         __syncthreads();
         double* t = Dcur;
@@ -128,19 +149,29 @@ k_allocate(const double* p, const uint64_t* W, int E, uint64_t B, uint8_t* bits,
             if (Dcur[r] < Dcur[rb]) rb = r;
         uint32_t r = rb;
         for (int e = E - 1; e >= 0; --e) {
-            const uint8_t b = choice[(size_t)e * (R + 1) + r];
-            bits[e] = b;
-            r -= (b == 3) ? 0u : (b == 4 ? s_up4[e] : s_up8[e]);
+            const uint32_t code = (chb[(size_t)e * nq + r / 4] >> (2 * (r % 4))) & 3u;
+            bits[e] = code == 0 ? 3 : (code == 1 ? 4 : 8);
+            r -= code == 0 ? 0u : (code == 1 ? s_up4[e] : s_up8[e]);
         }
     }
 }
 
 }  // namespace
 
+size_t allocate_choice_bytes(int E, uint64_t R) { return (size_t)E * (size_t)((R + 4) / 4); }
+
 void launch_allocate(cudaStream_t st, const double* p, const uint64_t* W, int E, uint64_t B,
                      uint8_t* bits_out, int32_t* status, uint8_t* choice, double* D,
-                     int state_cap) {
-    k_allocate<<<1, kThreads, 0, st>>>(p, W, E, B, bits_out, status, choice, D, state_cap);
+                     int state_cap, uint64_t R) {
+    // R is the host's count of budget units (same formula as the kernel's);
+    // it only sizes the on-chip buffers
+    const size_t smem = 16 * (size_t)(R + 1) + allocate_choice_bytes(E, R);
+    const bool on_chip = smem <= kAllocSmemMax;
+    // the attribute is per device: set it on every launch that needs it
+    if (on_chip && smem > 48 * 1024)
+        cudaFuncSetAttribute(k_allocate, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    k_allocate<<<1, kThreads, on_chip ? smem : 0, st>>>(p, W, E, B, bits_out, status, choice, D,
+                                                        state_cap, on_chip ? (int64_t)R : -1);
 }
 
 }  // namespace mpe

@@ -216,7 +216,7 @@ int run_allocate(mpe_ctx* c, const double* p, uint64_t B, std::vector<uint8_t>& 
     uint64_t R = B >= 8 * sum_w ? 0 : (B - 3 * sum_w) / g;
     R = std::min<uint64_t>(R, 5 * (sum_w / g));
     if (R + 1 > MPE_ALLOC_STATE_CAP) return fail(c, MPE_ERR_STATE_CAP, "too many states");
-    const size_t need = (size_t)E * (R + 1);
+    const size_t need = allocate_choice_bytes(E, R);
     if (need > c->choice_cap) {
         cudaFree(c->d_choice);
         CK(cudaMalloc(&c->d_choice, need));
@@ -226,7 +226,7 @@ int run_allocate(mpe_ctx* c, const double* p, uint64_t B, std::vector<uint8_t>& 
     CK(cudaMemcpyAsync(c->d_W, W.data(), sizeof(uint64_t) * E, cudaMemcpyHostToDevice,
                        c->stream));
     launch_allocate(c->stream, c->d_p, c->d_W, E, B, c->d_bits_out, c->d_alloc_status,
-                    c->d_choice, c->d_D, MPE_ALLOC_STATE_CAP);
+                    c->d_choice, c->d_D, MPE_ALLOC_STATE_CAP, R);
     c->launches++;
     CKLAUNCH();
     int32_t st = -1;
@@ -388,13 +388,13 @@ int mpe_allocate_bits(const double* p, const uint64_t* W, int32_t E, uint64_t B_
     auto ok = [](cudaError_t e) { return e == cudaSuccess; };
     if (!ok(cudaMalloc(&dp, sizeof(double) * E)) || !ok(cudaMalloc(&dW, sizeof(uint64_t) * E)) ||
         !ok(cudaMalloc(&db, E)) || !ok(cudaMalloc(&ds, sizeof(int32_t))) ||
-        !ok(cudaMalloc(&dch, (size_t)E * (R + 1))) ||
+        !ok(cudaMalloc(&dch, allocate_choice_bytes(E, R))) ||
         !ok(cudaMalloc(&dD, 2 * sizeof(double) * (R + 1))) ||
         !ok(cudaMemcpy(dp, p, sizeof(double) * E, cudaMemcpyHostToDevice)) ||
         !ok(cudaMemcpy(dW, W, sizeof(uint64_t) * E, cudaMemcpyHostToDevice))) {
         rc = fail_global(MPE_ERR_CUDA, "allocate_bits: %s", cudaGetErrorString(cudaGetLastError()));
     } else {
-        launch_allocate(nullptr, dp, dW, E, B_bits, db, ds, dch, dD, MPE_ALLOC_STATE_CAP);
+        launch_allocate(nullptr, dp, dW, E, B_bits, db, ds, dch, dD, MPE_ALLOC_STATE_CAP, R);
         if (!ok(cudaGetLastError()) || !ok(cudaMemcpy(&st, ds, sizeof(int32_t), cudaMemcpyDeviceToHost)) ||
             !ok(cudaMemcpy(bits_out, db, E, cudaMemcpyDeviceToHost)))
             rc = fail_global(MPE_ERR_CUDA, "allocate_bits kernel: %s",
@@ -560,7 +560,7 @@ static int moe_ffn_device(mpe_ctx* c, const void* x, int32_t T, const int32_t* i
         }
         {
             KernelSpan sp(c, 4);
-            launch_combine_by_position(c, w, T, k, reinterpret_cast<__nv_bfloat16*>(out));
+            launch_combine_by_position(c, w, T, k, 1, reinterpret_cast<__nv_bfloat16*>(out));
         }
         CKLAUNCH();
         return MPE_OK;
@@ -591,11 +591,11 @@ static int moe_ffn_device(mpe_ctx* c, const void* x, int32_t T, const int32_t* i
     }
     {
         KernelSpan sp(c, 3);
-        launch_decode_down(c, w, Tk, pl.p_dn, pl.kb_dn, pl.claim);
+        launch_decode_down(c, Tk, pl.p_dn, pl.kb_dn, pl.claim);
     }
     {
         KernelSpan sp(c, 4);
-        launch_combine(c, ids, T, k, pl.p_dn, reinterpret_cast<__nv_bfloat16*>(out));
+        launch_combine_by_position(c, w, T, k, pl.p_dn, reinterpret_cast<__nv_bfloat16*>(out));
     }
     CKLAUNCH();
     return MPE_OK;

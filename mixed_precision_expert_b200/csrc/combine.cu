@@ -1,7 +1,8 @@
-// Top-k weighted combine: out[t] = bf16( sum_j sum_p y[p][t*k + j] ), summed in
+// Top-k weighted combine: out[t] = bf16( sum_j w[t, j] sum_p y[p][pos_j] ) with
+// pos_j = inv[t*k + j] the route position of token t's j-th slot, summed in
 // fp32 with slots j = 0..k-1 outermost and K parts p = 0..P-1 inside (the down
-// kernel already applied w[t, j] and the scale); slots with an id outside
-// [0, E) contribute nothing. Deterministic: no atomics.
+// kernels already applied the scale); slots with an id outside [0, E)
+// contribute nothing. Deterministic: no atomics.
 //
 // SwiGLU reduce (gate/up split over K): h[pos][f] = bf16( silu(g) v ) with
 // g = sum_p gv[p][pos][0][f], v = sum_p gv[p][pos][1][f] (already scaled).
@@ -15,6 +16,9 @@ namespace {
 __global__ void __launch_bounds__(256)
 k_swiglu_reduce(const float* gv, const int32_t* offsets, int E, int F, int parts,
                 size_t part_stride, __nv_bfloat16* h) {
+    // the down kernel after this one reads only route outputs before its own wait
+    griddep_launch_dependents();
+    griddep_wait();
     const int n_pos = offsets[E];
     const size_t total = (size_t)n_pos * F;
     for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
@@ -30,41 +34,15 @@ k_swiglu_reduce(const float* gv, const int32_t* offsets, int E, int F, int parts
     }
 }
 
-// One thread per 4 columns of one token; a CTA covers 256 x 4 columns of one
-// token row (grid: tokens x column blocks).
-__global__ void __launch_bounds__(128)
-k_combine(const float* y, const int32_t* ids, int T, int k, int H, int E, int parts,
-          size_t part_stride, __nv_bfloat16* out) {
-    const int t = blockIdx.x;
-    const int i = blockIdx.y * blockDim.x + threadIdx.x;  // float4 column index
-    if (i >= H / 4) return;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j = 0; j < k; ++j) {
-        const int e = ids[t * k + j];
-        if (e < 0 || e >= E) continue;
-        for (int p = 0; p < parts; ++p) {
-            const float4 v = reinterpret_cast<const float4*>(y + (size_t)p * part_stride +
-                                                             (size_t)(t * k + j) * H)[i];
-            acc.x += v.x;
-            acc.y += v.y;
-            acc.z += v.z;
-            acc.w += v.w;
-        }
-    }
-    __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
-    __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
-    uint2 pk;
-    pk.x = *reinterpret_cast<uint32_t*>(&lo);
-    pk.y = *reinterpret_cast<uint32_t*>(&hi);
-    reinterpret_cast<uint2*>(out + (size_t)t * H)[i] = pk;
-}
-
-// Tensor-core path: y[pos] = s * (W2 h_pos) is stored by route position, so
-// out[t] = bf16( sum_j w[t, j] * y[inv[t k + j]] ) in slot order; dropped slots
-// (inv < 0) add nothing.
+// out[t] = bf16( sum_j w[t, j] * sum_p y[p][inv[t k + j]] ): y is stored by
+// route position in P K-part slices (P = 1 on the tensor-core path); slots in
+// order, parts summed first in part order; dropped slots (inv < 0) add
+// nothing. One thread per 4 columns of one token; a CTA covers 512 columns of
+// one token row (grid: tokens x column blocks).
 __global__ void __launch_bounds__(128)
 k_combine_by_position(const float* y, const int32_t* inv, const float* w, int T, int k, int H,
-                      __nv_bfloat16* out) {
+                      int parts, size_t part_stride, __nv_bfloat16* out) {
+    griddep_wait();
     const int t = blockIdx.x;
     const int i = blockIdx.y * blockDim.x + threadIdx.x;  // float4 column index
     if (i >= H / 4) return;
@@ -73,7 +51,29 @@ k_combine_by_position(const float* y, const int32_t* inv, const float* w, int T,
         const int pos = inv[t * k + j];
         if (pos < 0) continue;
         const float wj = w[t * k + j];
-        const float4 v = reinterpret_cast<const float4*>(y + (size_t)pos * H)[i];
+        const float4* src = reinterpret_cast<const float4*>(y + (size_t)pos * H) + i;
+        float4 v = src[0];
+        int p = 1;
+        // parts in order; four independent loads in flight per step
+        for (; p + 4 <= parts; p += 4) {
+            float4 u[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) u[r] = src[(p + r) * (part_stride / 4)];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                v.x += u[r].x;
+                v.y += u[r].y;
+                v.z += u[r].z;
+                v.w += u[r].w;
+            }
+        }
+        for (; p < parts; ++p) {
+            const float4 u = src[p * (part_stride / 4)];
+            v.x += u.x;
+            v.y += u.y;
+            v.z += u.z;
+            v.w += u.w;
+        }
         acc.x = fmaf(wj, v.x, acc.x);
         acc.y = fmaf(wj, v.y, acc.y);
         acc.z = fmaf(wj, v.z, acc.z);
@@ -92,24 +92,17 @@ k_combine_by_position(const float* y, const int32_t* inv, const float* w, int T,
 void launch_swiglu_reduce(mpe_ctx* c, size_t Tk, int parts) {
     const size_t total = Tk * c->F;
     const int grid = (int)std::min<size_t>((total + 255) / 256, 148 * 8);
-    k_swiglu_reduce<<<grid, 256, 0, c->stream>>>(c->s.part, c->s.offsets, c->E, c->F, parts,
-                                                 (size_t)2 * Tk * c->F, c->s.h);
+    launch_pdl(k_swiglu_reduce, dim3(grid), dim3(256), 0, c->stream, (const float*)c->s.part,
+               (const int32_t*)c->s.offsets, c->E, c->F, parts, (size_t)2 * Tk * c->F, c->s.h);
     c->launches++;
 }
 
-void launch_combine(mpe_ctx* c, const int32_t* ids, int T, int k, int parts,
-                    __nv_bfloat16* out) {
+void launch_combine_by_position(mpe_ctx* c, const float* w, int T, int k, int parts,
+                                __nv_bfloat16* out) {
     const int n4 = c->H / 4;
     dim3 grid((unsigned)T, (unsigned)((n4 + 127) / 128));
-    k_combine<<<grid, 128, 0, c->stream>>>(c->s.y, ids, T, k, c->H, c->E, parts,
-                                           (size_t)T * k * c->H, out);
-    c->launches++;
-}
-
-void launch_combine_by_position(mpe_ctx* c, const float* w, int T, int k, __nv_bfloat16* out) {
-    const int n4 = c->H / 4;
-    dim3 grid((unsigned)T, (unsigned)((n4 + 127) / 128));
-    k_combine_by_position<<<grid, 128, 0, c->stream>>>(c->s.y, c->s.inv, w, T, k, c->H, out);
+    launch_pdl(k_combine_by_position, grid, dim3(128), 0, c->stream, (const float*)c->s.y,
+               (const int32_t*)c->s.inv, w, T, k, c->H, parts, (size_t)T * k * c->H, out);
     c->launches++;
 }
 

@@ -163,6 +163,18 @@ __device__ __forceinline__ void prefetch_l2(const void* p) {
     asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
+// Programmatic dependent launch. griddep_wait blocks until the preceding
+// kernel in the stream has completed and its memory is visible (a no-op when
+// the launch was not programmatic); griddep_launch_dependents lets the next
+// kernel's CTAs start once every CTA of this grid has issued it or exited.
+__device__ __forceinline__ void griddep_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Wait for phase `parity` of an mbarrier, giving up after kWaitLimitNs.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;

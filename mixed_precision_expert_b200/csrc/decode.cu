@@ -5,23 +5,33 @@
 // (decode is memory-bound -- DecDEC summary, 2.1 -- so the packed bytes are
 // the cost). Per expert e with scale s_e and codes K1, K3, K2:
 //   gate/up:  g = s_e (K1 x), v = s_e (K3 x), h = silu(g) v   (h stored bf16)
-//   down:     y_a = w_a s_e (K2 h_a)                          (y stored fp32)
+//   down:     y_pos = s_e (K2 h_pos)                         (y stored fp32 by
+//             route position; the combine applies the top-k weights)
 //
-// Warp-specialised persistent kernel. A CTA has 8 consumer warps and 1
-// producer warp and works on one task at a time: a work group (<= 16 tokens of
-// one expert) x 8 consecutive 16-row output tiles (one per consumer warp) x a
-// K part. The producer warp claims tasks from a per-width-class counter and,
-// for each block column j of the task, fills one slot of the CTA's
-// shared-memory ring with the 8 tiles' chunks (one 1-D bulk copy per tile and
-// matrix, issued by 8-16 producer lanes in parallel, no multicast; a full
-// mbarrier counts the bytes) and prefetches the block's activation lines into
-// L1. Consumer warps wait on the slot's full barrier, copy their chunk's words
-// to registers, release the slot on its empty barrier (8 arrivals) and only
-// then unpack (common.cuh) and multiply with mma.sync m16n8k16 -- weights are
-// the 16-row A operand, one or two 8-token n-tiles of activations are B, fp32
-// accumulate, the per-expert scale applied once at the end. A task whose K
-// range is split in P parts writes a scaled partial to its own slice; a later
-// pass sums the slices in part order (deterministic, no atomics).
+// Warp-specialised persistent kernel. A CTA (one per SM) has 14 consumer
+// warps, 1 copy warp and 1 task warp and works on one task at a time: a work
+// group (<= 8 tokens of one expert) x 14 consecutive 16-row output tiles (one
+// per consumer warp) x a K part.
+//   task warp:  claims tasks from a per-width-class counter and resolves them
+//               (expert, tokens, activation rows, scale, first page entry)
+//               into a 4-entry task queue in shared memory, ahead of use, so
+//               no other warp waits on a chain of dependent global loads;
+//   copy warp:  for each queued task and each group of J block columns, fills
+//               one slot of the CTA's shared-memory ring with the 14 tiles'
+//               chunks (one 1-D bulk copy per tile, issued by 14 lanes in
+//               parallel, no multicast; a full mbarrier counts the bytes) and
+//               prefetches the block's activation lines into L1;
+//   consumers:  wait on the slot's full barrier, copy their chunk's words to
+//               registers, release the slot on its empty barrier and only then
+//               unpack (common.cuh) and multiply with mma.sync m16n8k16 --
+//               weights are the 16-row A operand, one 8-token n-tile of
+//               activations (loaded a block ahead) is B, fp32 accumulate,
+//               the per-expert scale applied once at the end.
+// A task whose K range is split in P parts writes a scaled partial to its own
+// slice; a later pass sums the slices in part order (deterministic, no
+// atomics). The forward-pass kernels chain with programmatic dependent launch:
+// a kernel starts while its predecessor drains and waits (griddepcontrol) only
+// where it reads what the predecessor wrote.
 //
 // k-permutation: inside a 128-code block, thread t (= lane & 3) owns 16 code
 // pairs; mma step c (0..7) uses its pairs 2c and 2c+1 as the logical k-pairs
@@ -36,33 +46,64 @@
 namespace mpe {
 namespace {
 
-constexpr int kConsumers = 8;                    // consumer warps per CTA (one tile each)
-constexpr int kThreads = (kConsumers + 1) * 32;  // + the producer warp
-constexpr int kRingBytes = 96 * 1024;            // shared-memory ring per CTA
+// 16 warps per SM in all: ptxas rounds a CTA's warps up to a multiple of 4
+// when it sets the register budget, and 16 warps leave 128 registers a thread
+// (17-20 warps would leave 96, too few for the gate/up consumer).
+constexpr int kConsumers = 14;                   // consumer warps per CTA (one tile each)
+constexpr int kCopyWarp = kConsumers;            // fills the ring
+constexpr int kTaskWarp = kConsumers + 1;        // claims and resolves tasks
+constexpr int kThreads = (kConsumers + 2) * 32;  // one CTA per SM
+constexpr int kRingBytes = 192 * 1024;           // shared-memory ring per CTA
+constexpr int kSlotBudget = 56 * 1024;           // at least three slots per ring
 constexpr int kMaxSlots = 16;
+constexpr int kTaskQ = 4;                        // resolved tasks queued ahead
 constexpr int kMaxTiles = kDecodeGroup / 8;
 
-// A slot holds J consecutive block columns of 8 tiles. The bulk-copy engine
+// A slot holds J consecutive block columns of 14 tiles. The bulk-copy engine
 // takes ~80 cycles per copy whatever its size up to a few KB, so a tile's
 // chunks for the slot -- gate and up interleaved, consecutive block columns,
 // one contiguous run of its page -- go in one copy, as many columns as keep a
-// slot within 32 KB (three slots per 96 KB ring): gate/up 2 (3, 4 bits) or 1
-// (8 bits), down 5 / 4 / 2.
+// slot within 56 KB (at least three slots per 192 KB ring): gate/up 2 (3, 4
+// bits) or 1 (8 bits), down 5 / 4 / 2.
 template <int B, int NM>
 struct Geo {
     static constexpr int CB = 256 * B;                   // chunk bytes
-    static constexpr int J = 32768 / (kConsumers * NM * CB);  // block columns per slot
+    static constexpr int J = kSlotBudget / (kConsumers * NM * CB);  // block columns per slot
     static constexpr int TILE = NM * J * CB;             // one warp's share of a slot
-    static constexpr int SLOT = kConsumers * TILE;       // J block columns of 8 tiles
+    static constexpr int SLOT = kConsumers * TILE;       // J block columns of all tiles
     static constexpr int S = (kRingBytes / SLOT) < kMaxSlots ? (kRingBytes / SLOT) : kMaxSlots;
     static constexpr int WORDS = (B == 8) ? 8 : B;       // raw words per row
     static_assert(S >= 3 && J >= 1, "ring geometry");
 };
+// Each width class starts its ring at slot 0; a new class's slot i must lie
+// within the previous class's slots 0..i, so slot sizes may not grow from one
+// class to the next (the classes run 8, 4, 3 bits).
+static_assert(Geo<8, 2>::SLOT >= Geo<4, 2>::SLOT && Geo<4, 2>::SLOT >= Geo<3, 2>::SLOT &&
+                  Geo<8, 1>::SLOT >= Geo<4, 1>::SLOT && Geo<4, 1>::SLOT >= Geo<3, 1>::SLOT,
+              "slot sizes per class");
+
+constexpr int kFirstSlot = 1;  // the slot opens its task
+constexpr int kLastSlot = 2;   // the slot closes its task
 
 struct SlotDesc {
-    int task;  // -1: no more tasks of this class
-    int j;     // first block column held by the slot
-    int nc;    // block columns held (1 .. J)
+    int q;      // task-queue entry of the slot's task; -1: no more tasks of this class
+    int j;      // first block column held by the slot (end of class: the queue entry)
+    int nc;     // block columns held (1 .. J)
+    int flags;  // kFirstSlot | kLastSlot
+};
+
+// One resolved task, written by the task warp, read by the copy warp and the
+// consumers when the task starts.
+struct TaskMeta {
+    int valid;   // 0: no more tasks of this width class
+    int tq;      // tile group: tiles 14 tq .. 14 tq + 13
+    int p;       // K part
+    int pos0;    // first route position of the work group
+    int ntok;    // tokens in the group (1 .. kDecodeGroup)
+    int j0, j_hi;  // block columns [j0, j_hi)
+    float scale;   // s_e
+    uint32_t first;  // the expert's first entry in the page-index array
+    int rows[kDecodeGroup];  // activation row of each token (x row, or h row = position)
 };
 
 struct Args {
@@ -73,8 +114,7 @@ struct Args {
     int k;
     const __nv_bfloat16* act;  // gate/up: x [T x H]; down: h [Tk x F] in perm order
     __nv_bfloat16* h_out;      // gate/up: h [Tk x F]
-    float* y_out;              // down: y [P][Tk][H], row a = assignment
-    const float* topk_w;       // down: [Tk]
+    float* y_out;              // down: y [P][Tk][H], row = route position
     float* part;               // gate/up split-K partials [P][Tk][2][F]
     size_t part_stride;        // floats per part slice (gate/up partials or down y)
     int32_t* task_ctr;         // claimed-task counters (one per class), zero at launch
@@ -83,8 +123,12 @@ struct Args {
     uint32_t* status;
 };
 
+constexpr size_t kBarOff = kRingBytes;
+constexpr size_t kDescOff = kBarOff + (2 * kMaxSlots + 2 * kTaskQ) * sizeof(uint64_t);
+constexpr size_t kTaskOff = kDescOff + kMaxSlots * sizeof(SlotDesc);
+
 __host__ __device__ constexpr size_t smem_bytes() {
-    return (size_t)kRingBytes + kMaxSlots * (2 * sizeof(uint64_t) + sizeof(SlotDesc));
+    return kTaskOff + kTaskQ * sizeof(TaskMeta);
 }
 
 // CTA task order: tile group fastest, then K part, then work group, so tasks
@@ -185,15 +229,15 @@ __device__ __forceinline__ void block_mma(const uint32_t (&wr)[NM][2][Geo<B, 1>:
 }
 
 struct Task {
-    int gi, tau, p, pos0, ntok, j_hi;
+    int tau, p, pos0, ntok, j_hi;
     float scale;
     bool valid;  // this warp's tile exists
 };
 
 // Finish a task. One K part (P = 1): gate/up applies SwiGLU and stores h
-// (bf16); down stores y_a = w_a s_e acc (fp32). Several parts: the task's
+// (bf16); down stores y_pos = s_e acc (fp32). Several parts: the task's
 // scaled partial goes to its own slice of the partial buffer -- gate/up
-// gv[p][pos][m][row] = s_e acc, down y[p][a][row] = w_a s_e acc -- and a later
+// gv[p][pos][m][row] = s_e acc, down y[p][pos][row] = s_e acc -- and a later
 // pass sums the slices in part order (deterministic, no atomics).
 template <bool GATEUP>
 __device__ __forceinline__ void finish(const Args& a, const Task& T,
@@ -221,56 +265,110 @@ __device__ __forceinline__ void finish(const Args& a, const Task& T,
                     dst[F] = uv;
                 }
             } else {
-                const int asg = a.perm[pos];
-                a.y_out[(size_t)T.p * a.part_stride + (size_t)asg * H + row] =
-                    a.topk_w[asg] * (T.scale * acc[nt][0][q]);
+                a.y_out[(size_t)T.p * a.part_stride + (size_t)pos * H + row] =
+                    T.scale * acc[nt][0][q];
             }
         }
 }
 
 struct CtaSmem {
     uint8_t* ring;
-    uint64_t* full;   // per slot: 1 producer arrival + transaction bytes
-    uint64_t* empty;  // per slot: one arrival per consumer warp
+    uint64_t* full;      // per slot: 1 producer arrival + transaction bytes
+    uint64_t* empty;     // per slot: one arrival per consumer warp
+    uint64_t* tq_full;   // per queue entry: the task warp's arrival
+    uint64_t* tq_empty;  // per queue entry: the copy warp + every consumer warp
     SlotDesc* descs;
+    TaskMeta* taskq;
 };
 
-// Producer warp: all tasks of one width class. Lane l < 8 owns the copy stream
-// of tile l (a page cursor in registers): per slot one run of NM x jc chunks
-// (gate/up: W1 and W3 alternate). Lane 0 claims tasks, arms the full barriers
-// and writes the slot descriptors; every lane prefetches one activation line. `ep`/`used` track the empty barriers'
-// phases per slot across classes.
+__device__ __forceinline__ uint32_t next_q(uint32_t q) { return q + 1 == kTaskQ ? 0u : q + 1; }
+
+// Task warp: claims the tasks of one width class in counter order and writes
+// each, resolved, into the next free queue entry; then one end-of-class entry.
+// `q` and the phase bits `ph` / `used` of the queue's empty barriers carry
+// over between classes.
+template <bool GATEUP>
+__device__ __forceinline__ bool resolve_class(const Args& a, const CtaSmem& sm, int group0,
+                                              int n_groups, int32_t* ctr, uint32_t& q,
+                                              uint32_t& ph, uint32_t& used) {
+    const PagedExperts& P = a.P;
+    const int K = GATEUP ? P.H : P.F;
+    const int R = GATEUP ? P.F : P.H;
+    const int nj = K / kCodesPerBlock;
+    const int n_tq = (R / 16 + kConsumers - 1) / kConsumers;
+    const int n_tasks = n_groups * n_tq * a.parts;
+    const int lane = threadIdx.x & 31;
+    for (;;) {
+        if ((used >> q) & 1u) {
+            if (!mbar_wait_bounded(&sm.tq_empty[q], (ph >> q) & 1u)) {
+                if (lane == 0) set_status(a.status, MPE_STATUS_WAIT_TIMEOUT);
+                return false;
+            }
+            ph ^= 1u << q;
+        }
+        used |= 1u << q;
+        int t = 0;
+        if (lane == 0 && n_tasks > 0) t = atomicAdd(ctr, 1);
+        t = __shfl_sync(0xffffffffu, t, 0);
+        TaskMeta* m = sm.taskq + q;
+        const bool more = t < n_tasks;
+        if (more) {
+            int gi, tq, p;
+            split_task(t, n_tq, a.parts, gi, tq, p);
+            gi += group0;
+            // route outputs are read through L2 (written by the preceding kernel)
+            const int e = __ldcg(a.wg + 3 * gi);
+            const int pos0 = __ldcg(a.wg + 3 * gi + 1);
+            const int ntok = __ldcg(a.wg + 3 * gi + 2);
+            if (lane < ntok)
+                m->rows[lane] = GATEUP ? __ldcg(a.perm + pos0 + lane) / a.k : pos0 + lane;
+            if (lane == 0) {
+                m->valid = 1;
+                m->tq = tq;
+                m->p = p;
+                m->pos0 = pos0;
+                m->ntok = ntok;
+                m->j0 = p * a.kb;
+                m->j_hi = min(nj, p * a.kb + a.kb);
+                m->scale = __ldcg(&P.pte[e].scale);
+                m->first = __ldcg(&P.pte[e].first);
+            }
+        } else if (lane == 0) {
+            m->valid = 0;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.tq_full[q]);
+        q = next_q(q);
+        if (!more) return true;
+    }
+}
+
+// Copy warp: every task of one width class, from the queue. Lane l < 14 owns
+// the copy stream of tile l (a page cursor in registers, the next page's index
+// loaded ahead): per slot one run of NM x jc chunks (gate/up: W1 and W3
+// alternate). Lane 0 arms the full barriers and writes the slot descriptors;
+// every lane prefetches one activation line. `ep` / `used` track the slots'
+// empty-barrier phases across classes, `fph` the queue's full-barrier phases.
+// In the down kernel the activations (h) come from the preceding kernel, so
+// the warp waits for it (`need_wait`) before its first prefetch.
 template <int B, bool GATEUP>
-__device__ __forceinline__ bool produce_class(const Args& a, const CtaSmem& sm, int group0,
-                                              int n_groups, int32_t* ctr, uint32_t& ep,
-                                              uint32_t& used) {
+__device__ __forceinline__ bool produce_class(const Args& a, const CtaSmem& sm, uint32_t& q,
+                                              uint32_t& fph, uint32_t& ep, uint32_t& used,
+                                              bool& need_wait) {
     constexpr int NM = GATEUP ? 2 : 1;
     using G = Geo<B, NM>;
     constexpr int S = G::S;
     const PagedExperts& P = a.P;
-    const int H = P.H, F = P.F;
-    const int K = GATEUP ? H : F;
-    const int R = GATEUP ? F : H;
+    const int K = GATEUP ? P.H : P.F;
+    const int R = GATEUP ? P.F : P.H;
     const int nj = K / kCodesPerBlock, n_tiles = R / 16;
-    const int n_tq = (n_tiles + kConsumers - 1) / kConsumers;
-    const int nc1 = chunks_w1(H, F);
-    const int lane = threadIdx.x & 31;
-    const int n_tasks = n_groups * n_tq * a.parts;
-    if (n_tasks == 0) return true;
+    const int nc1 = chunks_w1(P.H, P.F);
     const int cpp = chunks_per_page(B, P.page_bytes);
-    const int my_w = lane;
+    const int n_pages = (3 * nc1 + cpp - 1) / cpp;
+    const int lane = threadIdx.x & 31;
     const bool copier = lane < kConsumers;
 
-    int s = 0;
-    int task = -1, j = 0, j_hi = 0;
-    uint32_t first = 0;
-    int pslot = 0, poff = 0;           // this lane's page cursor
-    bool my_tile = false;
-    const __nv_bfloat16* pre_row = nullptr;  // this lane's activation row to prefetch
-    int pre_half = 0;
-    int active = 0;                    // tiles present in the current task
-    for (;;) {
-        // slot s must have been released by all consumers since its last fill
+    auto acquire = [&](int s) -> bool {
         if ((used >> s) & 1u) {
             if (!mbar_wait_bounded(&sm.empty[s], (ep >> s) & 1u)) {
                 if (lane == 0) set_status(a.status, MPE_STATUS_WAIT_TIMEOUT);
@@ -279,102 +377,135 @@ __device__ __forceinline__ bool produce_class(const Args& a, const CtaSmem& sm, 
             ep ^= 1u << s;
         }
         used |= 1u << s;
-        if (task < 0 || j >= j_hi) {
-            int nt = 0;
-            if (lane == 0) nt = atomicAdd(ctr, 1);
-            nt = __shfl_sync(0xffffffffu, nt, 0);
-            if (nt >= n_tasks) {
-                if (lane == 0) {
-                    sm.descs[s] = SlotDesc{-1, 0};
-                    mbar_arrive(&sm.full[s]);
-                }
-                __syncwarp();
-                return true;
-            }
-            int gi, tq, p;
-            split_task(nt, n_tq, a.parts, gi, tq, p);
-            task = nt;
-            gi += group0;
-            const int e = a.wg[3 * gi];
-            const int pos0 = a.wg[3 * gi + 1], ntok = a.wg[3 * gi + 2];
-            first = P.pte[e].first;
-            j = p * a.kb;
-            j_hi = min(nj, j + a.kb);
-            active = min(kConsumers, n_tiles - tq * kConsumers);
-            const int tau = tq * kConsumers + my_w;
-            my_tile = copier && my_w < active;
-            if (my_tile) {
-                const int c = GATEUP ? 2 * (tau * nj + j) : 2 * nc1 + tau * nj + j;
-                pslot = c / cpp;
-                poff = c - pslot * cpp;
-            }
-            pre_row = nullptr;
-            pre_half = lane & 1;
-            if ((lane >> 1) < ntok) {
-                const int pos = pos0 + (lane >> 1);
-                pre_row = a.act + (size_t)(GATEUP ? (a.perm[pos] / a.k) : pos) * K;
-            }
+        return true;
+    };
+
+    int s = 0;
+    for (;;) {
+        if (!mbar_wait_bounded(&sm.tq_full[q], (fph >> q) & 1u)) {
+            if (lane == 0) set_status(a.status, MPE_STATUS_WAIT_TIMEOUT);
+            return false;
         }
-        const int jc = min(G::J, j_hi - j);  // block columns in this slot
-        if (lane == 0) {
-            sm.descs[s] = SlotDesc{task, j, jc};
-            mbar_arrive_expect_tx(&sm.full[s], (uint32_t)(active * NM * jc * G::CB));
+        fph ^= 1u << q;
+        const TaskMeta* m = sm.taskq + q;
+        const int valid = m->valid;
+        int tq = 0, j = 0, j_hi = 0;
+        uint32_t first = 0;
+        const __nv_bfloat16* pre_row = nullptr;  // this lane's activation row to prefetch
+        if (valid) {
+            tq = m->tq;
+            j = m->j0;
+            j_hi = m->j_hi;
+            first = m->first;
+            if ((lane >> 1) < m->ntok) pre_row = a.act + (size_t)m->rows[lane >> 1] * K;
         }
         __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.tq_empty[q]);
+        const uint32_t mq = q;
+        q = next_q(q);
+        if (!valid) {  // end of the class: a terminator slot names the queue entry
+            if (!acquire(s)) return false;
+            if (lane == 0) {
+                sm.descs[s] = SlotDesc{-1, (int)mq, 0, 0};
+                mbar_arrive(&sm.full[s]);
+            }
+            __syncwarp();
+            return true;
+        }
+        const int active = min(kConsumers, n_tiles - tq * kConsumers);
+        const bool my_tile = copier && lane < active;
+        int pslot = 0, poff = 0;
+        uint32_t page = 0, page_next = 0;
         if (my_tile) {
-            // NM x jc consecutive chunks of this tile; a page boundary splits the
-            // copy in two
-            uint8_t* dst = sm.ring + (size_t)s * G::SLOT + (size_t)lane * G::TILE;
-            const int total = NM * jc;
-            const int n1 = min(total, cpp - poff);
-            bulk_g2s(dst, P.pool + (size_t)P.pidx[first + pslot] * P.page_bytes +
-                              (size_t)poff * G::CB,
-                     (uint32_t)(n1 * G::CB), &sm.full[s]);
-            poff += n1;
-            if (poff == cpp) {
-                ++pslot;
-                poff = 0;
-            }
-            if (n1 < total) {
-                bulk_g2s(dst + n1 * G::CB, P.pool + (size_t)P.pidx[first + pslot] * P.page_bytes,
-                         (uint32_t)((total - n1) * G::CB), &sm.full[s]);
-                poff = total - n1;
-            }
+            const int tau = tq * kConsumers + lane;
+            const int c = GATEUP ? 2 * (tau * nj + j) : 2 * nc1 + tau * nj + j;
+            pslot = c / cpp;
+            poff = c - pslot * cpp;
+            page = __ldcg(P.pidx + first + pslot);
+            if (pslot + 1 < n_pages) page_next = __ldcg(P.pidx + first + pslot + 1);
         }
-        if (pre_row) {
+        const int jstart = j;
+        const int pre_half = lane & 1;
+        while (j < j_hi) {
+            if (!acquire(s)) return false;
+            const int jc = min(G::J, j_hi - j);  // block columns in this slot
+            if (lane == 0) {
+                sm.descs[s] = SlotDesc{(int)mq, j, jc,
+                                       (j == jstart ? kFirstSlot : 0) |
+                                           (j + jc >= j_hi ? kLastSlot : 0)};
+                mbar_arrive_expect_tx(&sm.full[s], (uint32_t)(active * NM * jc * G::CB));
+            }
+            __syncwarp();
+            if (my_tile) {
+                // NM x jc consecutive chunks of this tile; a page boundary splits
+                // the copy in two
+                uint8_t* dst = sm.ring + (size_t)s * G::SLOT + (size_t)lane * G::TILE;
+                const int total = NM * jc;
+                const int n1 = min(total, cpp - poff);
+                bulk_g2s(dst, P.pool + (size_t)page * P.page_bytes + (size_t)poff * G::CB,
+                         (uint32_t)(n1 * G::CB), &sm.full[s]);
+                poff += n1;
+                if (poff == cpp) {
+                    ++pslot;
+                    poff = 0;
+                    page = page_next;
+                    if (pslot + 1 < n_pages) page_next = __ldcg(P.pidx + first + pslot + 1);
+                }
+                if (n1 < total) {
+                    bulk_g2s(dst + n1 * G::CB, P.pool + (size_t)page * P.page_bytes,
+                             (uint32_t)((total - n1) * G::CB), &sm.full[s]);
+                    poff = total - n1;
+                }
+            }
+            if (need_wait) {
+                griddep_wait();
+                need_wait = false;
+            }
+            if (pre_row) {
 #pragma unroll
-            for (int jj = 0; jj < G::J; ++jj)
-                if (jj < jc) prefetch_l1(pre_row + 128 * (j + jj) + 64 * pre_half);
+                for (int jj = 0; jj < G::J; ++jj)
+                    if (jj < jc) prefetch_l1(pre_row + 128 * (j + jj) + 64 * pre_half);
+            }
+            j += jc;
+            s = (s + 1 == S) ? 0 : s + 1;
         }
-        j += jc;
-        s = (s + 1 == S) ? 0 : s + 1;
     }
 }
 
-// Consumer warp w: all tasks of one width class, tile w of each task.
+// Consumer warp w: all tasks of one width class, tile w of each task. `fp`
+// tracks the slots' full-barrier phases across classes.
 template <int B, bool GATEUP>
-__device__ __forceinline__ bool consume_class(const Args& a, const CtaSmem& sm, int group0,
-                                              int n_groups, uint32_t& fp, int w) {
+__device__ __forceinline__ bool consume_class(const Args& a, const CtaSmem& sm, uint32_t& fp,
+                                              int w) {
     constexpr int NM = GATEUP ? 2 : 1;
     using G = Geo<B, NM>;
     constexpr int S = G::S;
     const PagedExperts& P = a.P;
-    const int H = P.H, F = P.F;
-    const int K = GATEUP ? H : F;
-    const int R = GATEUP ? F : H;
-    const int nj = K / kCodesPerBlock, n_tiles = R / 16;
-    const int n_tq = (n_tiles + kConsumers - 1) / kConsumers;
+    const int K = GATEUP ? P.H : P.F;
+    const int R = GATEUP ? P.F : P.H;
+    const int n_tiles = R / 16;
     const int lane = threadIdx.x & 31;
-    const int g = lane >> 2, t = lane & 3;
-    if (n_groups * n_tq * a.parts == 0) return true;
+    const int g = lane >> 2;
 
-    int cur = -1;
     Task T{};
-    const __nv_bfloat16* arow[kMaxTiles] = {nullptr, nullptr};
+    const __nv_bfloat16* arow[kMaxTiles] = {};
     int ntiles = 0;
     float acc[kMaxTiles][NM][4];
     float accc[kMaxTiles][4];  // offset term (widths 3, 4), subtracted at the task's end
+    // activations of the block being multiplied (xa, xz) and of the next block
+    // of the task (na, nz), loaded one block ahead so that the loads' latency
+    // hides behind a block of unpacking and MMAs
     uint32_t xa[kMaxTiles][8], xz[kMaxTiles][8];
+    uint32_t na[kMaxTiles][8], nz[kMaxTiles][8];
+    auto load_next = [&](int j) {
+#pragma unroll
+        for (int nt = 0; nt < kMaxTiles; ++nt) {
+            if (nt == 0 || nt < ntiles) {
+                load_act_half(arow[nt], j, lane & 3, B == 8, 0, na[nt]);
+                load_act_half(arow[nt], j, lane & 3, B == 8, 1, nz[nt]);
+            }
+        }
+    };
     // acc <- acc - off . x for every matrix (a no-op for width 8)
     auto settle = [&]() {
         if constexpr (B != 8) {
@@ -394,52 +525,45 @@ __device__ __forceinline__ bool consume_class(const Args& a, const CtaSmem& sm, 
             return false;
         }
         const SlotDesc d = sm.descs[s];
-        if (d.task < 0) {  // terminator
-            settle();
-            finish<GATEUP>(a, T, acc, lane);
+        if (d.q < 0) {  // end of the class
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.empty[s]);
+            if (lane == 0) {
+                mbar_arrive(&sm.tq_empty[d.j]);
+                mbar_arrive(&sm.empty[s]);
+            }
             return true;
         }
-        if (d.task != cur) {
-            if (cur >= 0) {
-                settle();
-                finish<GATEUP>(a, T, acc, lane);
-            }
-            cur = d.task;
-            int tq;
-            split_task(cur, n_tq, a.parts, T.gi, tq, T.p);
-            T.gi += group0;
-            T.tau = tq * kConsumers + w;
+        if (d.flags & kFirstSlot) {
+            const TaskMeta* m = sm.taskq + d.q;
+            T.tau = m->tq * kConsumers + w;
             T.valid = T.tau < n_tiles;
-            const int e = a.wg[3 * T.gi];
-            T.pos0 = a.wg[3 * T.gi + 1];
-            T.ntok = a.wg[3 * T.gi + 2];
-            T.scale = P.pte[e].scale;
-            T.j_hi = min(nj, T.p * a.kb + a.kb);
+            T.p = m->p;
+            T.pos0 = m->pos0;
+            T.ntok = m->ntok;
+            T.j_hi = m->j_hi;
+            T.scale = m->scale;
             ntiles = (T.ntok + 7) / 8;
 #pragma unroll
             for (int nt = 0; nt < kMaxTiles; ++nt) {
                 const int n = nt * 8 + g;
-                arow[nt] = nullptr;
-                if (n < T.ntok) {
-                    const int pos = T.pos0 + n;
-                    const int row = GATEUP ? (a.perm[pos] / a.k) : pos;
-                    arow[nt] = a.act + (size_t)row * K;
-                }
+                arow[nt] = n < T.ntok ? a.act + (size_t)m->rows[n] * K : nullptr;
 #pragma unroll
-                for (int m = 0; m < NM; ++m)
+                for (int mm = 0; mm < NM; ++mm)
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) acc[nt][m][q] = 0.0f;
+                    for (int q = 0; q < 4; ++q) acc[nt][mm][q] = 0.0f;
 #pragma unroll
                 for (int q = 0; q < 4; ++q) accc[nt][q] = 0.0f;
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.tq_empty[d.q]);
+            if (T.valid) load_next(d.j);
         }
         if (!T.valid) {  // this warp has no tile in the task: release at once
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.empty[s]);
             continue;
         }
+        const int t = lane & 3;
         const uint8_t* tile = sm.ring + (size_t)s * G::SLOT + (size_t)w * G::TILE;
 #pragma unroll
         for (int jj = 0; jj < G::J; ++jj) {
@@ -456,49 +580,79 @@ __device__ __forceinline__ bool consume_class(const Args& a, const CtaSmem& sm, 
                 if (lane == 0) mbar_arrive(&sm.empty[s]);
             }
             const int j = d.j + jj;
-            load_act_half(arow[0], j, t, B == 8, 0, xa[0]);
-            load_act_half(arow[0], j, t, B == 8, 1, xz[0]);
-            if (ntiles > 1) {
-                load_act_half(arow[1], j, t, B == 8, 0, xa[1]);
-                load_act_half(arow[1], j, t, B == 8, 1, xz[1]);
-                block_mma<B, NM, kMaxTiles>(wr, xa, xz, acc, accc);
-            } else {
-                block_mma<B, NM, 1>(wr, xa, xz, acc, accc);
+#pragma unroll
+            for (int nt = 0; nt < kMaxTiles; ++nt)
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    xa[nt][i] = na[nt][i];
+                    xz[nt][i] = nz[nt][i];
+                }
+            if (j + 1 < T.j_hi) load_next(j + 1);
+            if constexpr (kMaxTiles > 1) {
+                if (ntiles > 1) {
+                    block_mma<B, NM, kMaxTiles>(wr, xa, xz, acc, accc);
+                    continue;
+                }
             }
+            block_mma<B, NM, 1>(wr, xa, xz, acc, accc);
+        }
+        if (d.flags & kLastSlot) {
+            settle();
+            finish<GATEUP>(a, T, acc, lane);
         }
     }
 }
 
 template <bool GATEUP>
-__global__ void __launch_bounds__(kThreads, 2) k_decode(Args a) {
+__global__ void __launch_bounds__(kThreads, 1) k_decode(Args a) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     CtaSmem sm;
     sm.ring = smem;
-    sm.full = reinterpret_cast<uint64_t*>(smem + kRingBytes);
+    sm.full = reinterpret_cast<uint64_t*>(smem + kBarOff);
     sm.empty = sm.full + kMaxSlots;
-    sm.descs = reinterpret_cast<SlotDesc*>(sm.empty + kMaxSlots);
+    sm.tq_full = sm.empty + kMaxSlots;
+    sm.tq_empty = sm.tq_full + kTaskQ;
+    sm.descs = reinterpret_cast<SlotDesc*>(smem + kDescOff);
+    sm.taskq = reinterpret_cast<TaskMeta*>(smem + kTaskOff);
     if (threadIdx.x == 0) {
         for (int s = 0; s < kMaxSlots; ++s) {
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], kConsumers);
         }
+        for (int q = 0; q < kTaskQ; ++q) {
+            mbar_init(&sm.tq_full[q], 1);
+            mbar_init(&sm.tq_empty[q], kConsumers + 1);
+        }
         fence_mbar_init();
         fence_proxy_async_smem();
     }
     __syncthreads();
-    const int n8 = a.n_wg_class[0], n4 = a.n_wg_class[1], n3 = a.n_wg_class[2];
-    if (warp == kConsumers) {
-        uint32_t ep = 0, used = 0;
-        (void)lane;
-        if (!produce_class<8, GATEUP>(a, sm, 0, n8, a.task_ctr + 0, ep, used)) return;
-        if (!produce_class<4, GATEUP>(a, sm, n8, n4, a.task_ctr + 1, ep, used)) return;
-        produce_class<3, GATEUP>(a, sm, n8 + n4, n3, a.task_ctr + 2, ep, used);
+    if (warp == kTaskWarp) {
+        // gate/up: the work groups and task counters come from the route kernel
+        // just before; down: that kernel finished before the one that precedes
+        // this launch let it start
+        if (GATEUP) griddep_wait();
+        if (lane == 0) griddep_launch_dependents();
+        const int n8 = __ldcg(a.n_wg_class), n4 = __ldcg(a.n_wg_class + 1),
+                  n3 = __ldcg(a.n_wg_class + 2);
+        uint32_t q = 0, ph = 0, used = 0;
+        if (!resolve_class<GATEUP>(a, sm, 0, n8, a.task_ctr + 0, q, ph, used)) return;
+        if (!resolve_class<GATEUP>(a, sm, n8, n4, a.task_ctr + 1, q, ph, used)) return;
+        resolve_class<GATEUP>(a, sm, n8 + n4, n3, a.task_ctr + 2, q, ph, used);
+    } else if (warp == kCopyWarp) {
+        uint32_t q = 0, fph = 0, ep = 0, used = 0;
+        bool need_wait = !GATEUP;
+        if (!produce_class<8, GATEUP>(a, sm, q, fph, ep, used, need_wait)) return;
+        if (!produce_class<4, GATEUP>(a, sm, q, fph, ep, used, need_wait)) return;
+        produce_class<3, GATEUP>(a, sm, q, fph, ep, used, need_wait);
     } else {
+        // down: h is written by the preceding kernel
+        if (!GATEUP) griddep_wait();
         uint32_t fp = 0;
-        if (!consume_class<8, GATEUP>(a, sm, 0, n8, fp, warp)) return;
-        if (!consume_class<4, GATEUP>(a, sm, n8, n4, fp, warp)) return;
-        consume_class<3, GATEUP>(a, sm, n8 + n4, n3, fp, warp);
+        if (!consume_class<8, GATEUP>(a, sm, fp, warp)) return;
+        if (!consume_class<4, GATEUP>(a, sm, fp, warp)) return;
+        consume_class<3, GATEUP>(a, sm, fp, warp);
     }
 }
 
@@ -530,7 +684,7 @@ static int env_int(const char* name, int dflt) {
 
 void decode_plan(mpe_ctx* c, size_t Tk, DecodePlan& pl) {
     if (!g_num_sms) cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, c->device);
-    const int ctas = g_num_sms * 2;
+    const int ctas = g_num_sms;
     const int groups = (int)std::min<size_t>((size_t)c->E, Tk);
     const int per_cta = env_int("MPE_DECODE_TASKS_PER_CTA", 8);
     pl.claim = 1;
@@ -568,12 +722,11 @@ void launch_decode_gateup(mpe_ctx* c, const __nv_bfloat16* x, int k, size_t Tk, 
     a.kb = kb;
     a.status = c->d_status;
     const int grid = persistent_grid(c, (const void*)k_decode<true>, smem_bytes());
-    k_decode<true><<<grid, kThreads, smem_bytes(), c->stream>>>(a);
+    launch_pdl(k_decode<true>, dim3(grid), dim3(kThreads), smem_bytes(), c->stream, a);
     c->launches++;
 }
 
-void launch_decode_down(mpe_ctx* c, const float* topk_w, size_t Tk, int parts, int kb,
-                        int claim) {
+void launch_decode_down(mpe_ctx* c, size_t Tk, int parts, int kb, int claim) {
     (void)claim;
     Args a{};
     a.P = paged(c);
@@ -583,7 +736,6 @@ void launch_decode_down(mpe_ctx* c, const float* topk_w, size_t Tk, int parts, i
     a.k = 1;
     a.act = c->s.h;
     a.y_out = c->s.y;
-    a.topk_w = topk_w;
     a.part = c->s.part;
     a.part_stride = (size_t)Tk * c->H;
     a.task_ctr = c->s.task_ctr + 3;
@@ -591,7 +743,7 @@ void launch_decode_down(mpe_ctx* c, const float* topk_w, size_t Tk, int parts, i
     a.kb = kb;
     a.status = c->d_status;
     const int grid = persistent_grid(c, (const void*)k_decode<false>, smem_bytes());
-    k_decode<false><<<grid, kThreads, smem_bytes(), c->stream>>>(a);
+    launch_pdl(k_decode<false>, dim3(grid), dim3(kThreads), smem_bytes(), c->stream, a);
     c->launches++;
 }
 

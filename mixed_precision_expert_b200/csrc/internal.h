@@ -5,6 +5,7 @@
 
 #include <cstdint>
 #include <string>
+#include <utility>
 #include <vector>
 
 #include "common.cuh"
@@ -12,8 +13,10 @@
 
 namespace mpe {
 
-// Tokens per work group of the decode kernels (two 8-token mma n-tiles).
-constexpr int kDecodeGroup = 16;
+// Tokens per work group of the decode kernels (one 8-token mma n-tile): an
+// expert with more tokens is served by several groups, which read its pages
+// close together in time (mostly from L2).
+constexpr int kDecodeGroup = 8;
 
 struct Scratch {
     size_t cap_assign = 0;   // T*k capacity
@@ -108,6 +111,25 @@ namespace mpe {
 
 PagedExperts paged(const mpe_ctx* c);
 
+// Launch with programmatic stream serialization: the kernel may start while
+// the preceding kernel in the stream drains; it must call griddep_wait before
+// it reads anything that kernel writes.
+template <typename... KArgs, typename... Actual>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Actual&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Actual>(args)...);
+}
+
 // quantize.cu
 void launch_absmax(mpe_ctx* c, const int32_t* d_list, int n_list);
 void launch_scales(mpe_ctx* c);
@@ -117,7 +139,9 @@ void launch_gather_stream(mpe_ctx* c, int e, uint8_t* dst);
 // allocate.cu
 void launch_allocate(cudaStream_t st, const double* p, const uint64_t* W, int E, uint64_t B,
                      uint8_t* bits_out, int32_t* status, uint8_t* choice, double* D,
-                     int state_cap);
+                     int state_cap, uint64_t R);
+// bytes of the global choice table for E experts and R budget units
+size_t allocate_choice_bytes(int E, uint64_t R);
 
 // route.cu
 void launch_route(mpe_ctx* c, const int32_t* ids, int Tk, int k, int32_t* perm,
@@ -131,8 +155,7 @@ struct DecodePlan {
 void decode_plan(mpe_ctx* c, size_t Tk, DecodePlan& pl);
 void launch_decode_gateup(mpe_ctx* c, const __nv_bfloat16* x, int k, size_t Tk, int parts,
                           int kb, int claim);
-void launch_decode_down(mpe_ctx* c, const float* topk_w, size_t Tk, int parts, int kb,
-                        int claim);
+void launch_decode_down(mpe_ctx* c, size_t Tk, int parts, int kb, int claim);
 
 // prefill.cu (tcgen05 grouped GEMM; work groups of up to kPrefillGroup positions)
 constexpr int kPrefillGroup = 208;
@@ -144,9 +167,9 @@ int launch_prefill_down(mpe_ctx* c, size_t Tk);
 
 // combine.cu
 void launch_swiglu_reduce(mpe_ctx* c, size_t Tk, int parts);
-void launch_combine(mpe_ctx* c, const int32_t* ids, int T, int k, int parts,
-                    __nv_bfloat16* out);
-// y stored by route position (tensor-core path); weights applied here
-void launch_combine_by_position(mpe_ctx* c, const float* w, int T, int k, __nv_bfloat16* out);
+// y stored by route position in `parts` K-part slices; the top-k weights are
+// applied here
+void launch_combine_by_position(mpe_ctx* c, const float* w, int T, int k, int parts,
+                                __nv_bfloat16* out);
 
 }  // namespace mpe

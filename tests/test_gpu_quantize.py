@@ -48,6 +48,23 @@ def test_allocate_bits_workloads(cfg, avg):
     assert sum(int(b) * w for b, w in zip(got, W)) <= B
 
 
+@pytest.mark.parametrize("units", [9000, 12000])
+def test_allocate_bits_many_states(units):
+    # sizes with gcd 1 give about `units` budget states: at 9000 the DP rows and
+    # the 2-bit choice table fit in the kernel's shared memory, at 12000 they
+    # live in global memory
+    rng = np.random.default_rng(units)
+    E = 16
+    W = [int(x) for x in rng.integers(3000, 5000, size=E)]
+    W[0] = 4099  # prime: gcd(W) = 1
+    p = rng.dirichlet(np.full(E, 0.7))
+    B = 3 * sum(W) + units
+    got = mpe.allocate_bits(p, W, B)
+    ref = oa.allocate_bits(p, W, B, state_cap=mpe.ALLOC_STATE_CAP)
+    assert np.array_equal(got, ref)
+    assert sum(int(b) * w for b, w in zip(got, W)) <= B
+
+
 def test_allocate_bits_errors():
     with pytest.raises(mpe.MpeError) as ei:
         mpe.allocate_bits([1.0, 1.0], [7, 11], 3 * 18 - 1)
