@@ -10,22 +10,22 @@
 //
 // Warp-specialised persistent kernel. A CTA (one per SM) has 14 consumer
 // warps, 1 copy warp and 1 task warp and works on one task at a time: a work
-// group (<= 8 tokens of one expert) x 14 consecutive 16-row output tiles (one
-// per consumer warp) x a K part.
+// group (<= 8 tokens of one expert) x 14 (gate/up: one per consumer warp) or
+// 28 (down: two per warp) consecutive 16-row output tiles x a K part.
 //   task warp:  claims tasks from a per-width-class counter and resolves them
 //               (expert, tokens, activation rows, scale, first page entry)
 //               into a 4-entry task queue in shared memory, ahead of use, so
 //               no other warp waits on a chain of dependent global loads;
 //   copy warp:  for each queued task and each group of J block columns, fills
-//               one slot of the CTA's shared-memory ring with the 14 tiles'
-//               chunks (one 1-D bulk copy per tile, issued by 14 lanes in
+//               one slot of the CTA's shared-memory ring with the task's
+//               chunks (one 1-D bulk copy per tile, issued by 14-28 lanes in
 //               parallel, no multicast; a full mbarrier counts the bytes) and
 //               prefetches the block's activation lines into L1;
 //   consumers:  wait on the slot's full barrier, copy their chunk's words to
 //               registers, release the slot on its empty barrier and only then
 //               unpack (common.cuh) and multiply with mma.sync m16n8k16 --
 //               weights are the 16-row A operand, one 8-token n-tile of
-//               activations (loaded a block ahead) is B, fp32 accumulate,
+//               activations is B, fp32 accumulate,
 //               the per-expert scale applied once at the end.
 // A task whose K range is split in P parts writes a scaled partial to its own
 // slice; a later pass sums the slices in part order (deterministic, no
@@ -49,7 +49,7 @@ namespace {
 // 16 warps per SM in all: ptxas rounds a CTA's warps up to a multiple of 4
 // when it sets the register budget, and 16 warps leave 128 registers a thread
 // (17-20 warps would leave 96, too few for the gate/up consumer).
-constexpr int kConsumers = 14;                   // consumer warps per CTA (one tile each)
+constexpr int kConsumers = 14;                   // consumer warps per CTA
 constexpr int kCopyWarp = kConsumers;            // fills the ring
 constexpr int kTaskWarp = kConsumers + 1;        // claims and resolves tasks
 constexpr int kThreads = (kConsumers + 2) * 32;  // one CTA per SM
@@ -59,28 +59,43 @@ constexpr int kMaxSlots = 16;
 constexpr int kTaskQ = 4;                        // resolved tasks queued ahead
 constexpr int kMaxTiles = kDecodeGroup / 8;
 
-// A slot holds J consecutive block columns of 14 tiles. The bulk-copy engine
-// takes ~80 cycles per copy whatever its size up to a few KB, so a tile's
-// chunks for the slot -- gate and up interleaved, consecutive block columns,
-// one contiguous run of its page -- go in one copy, as many columns as keep a
-// slot within 56 KB (at least three slots per 192 KB ring): gate/up 2 (3, 4
-// bits) or 1 (8 bits), down 5 / 4 / 2.
-template <int B, int NM>
+// Tiles per consumer warp: the down kernel gives each warp two 16-row tiles
+// that share one activation fragment (its rows stream 1 weight byte per 2
+// activation bytes through L1 otherwise); gate/up already multiplies two
+// matrices per fragment.
+__host__ __device__ constexpr int tiles_per_warp(bool gateup) { return gateup ? 1 : 2; }
+__host__ __device__ constexpr int tiles_per_task(bool gateup) {
+    return kConsumers * tiles_per_warp(gateup);
+}
+
+// A slot holds J consecutive block columns of every tile of a task (tiles in
+// order, so a warp's tiles are adjacent). The bulk-copy engine takes ~80
+// cycles per copy whatever its size up to a few KB, so a tile's chunks for the
+// slot -- gate and up interleaved, consecutive block columns, one contiguous
+// run of its page -- go in one copy, as many columns as keep a slot within
+// 56 KB (at least three slots per 192 KB ring): gate/up 2 (3, 4 bits) or 1
+// (8 bits), down (two tiles a warp) 2 / 2 / 1.
+template <int B, int NM, int TPW>
 struct Geo {
     static constexpr int CB = 256 * B;                   // chunk bytes
-    static constexpr int J = kSlotBudget / (kConsumers * NM * CB);  // block columns per slot
-    static constexpr int TILE = NM * J * CB;             // one warp's share of a slot
-    static constexpr int SLOT = kConsumers * TILE;       // J block columns of all tiles
+    static constexpr int J = kSlotBudget / (kConsumers * TPW * NM * CB);  // columns per slot
+    static constexpr int TILEB = NM * J * CB;            // one tile's share of a slot
+    static constexpr int SLOT = kConsumers * TPW * TILEB;
     static constexpr int S = (kRingBytes / SLOT) < kMaxSlots ? (kRingBytes / SLOT) : kMaxSlots;
     static constexpr int WORDS = (B == 8) ? 8 : B;       // raw words per row
     static_assert(S >= 3 && J >= 1, "ring geometry");
 };
+template <int B>
+using GeoGU = Geo<B, 2, tiles_per_warp(true)>;
+template <int B>
+using GeoDN = Geo<B, 1, tiles_per_warp(false)>;
 // Each width class starts its ring at slot 0; a new class's slot i must lie
 // within the previous class's slots 0..i, so slot sizes may not grow from one
 // class to the next (the classes run 8, 4, 3 bits).
-static_assert(Geo<8, 2>::SLOT >= Geo<4, 2>::SLOT && Geo<4, 2>::SLOT >= Geo<3, 2>::SLOT &&
-                  Geo<8, 1>::SLOT >= Geo<4, 1>::SLOT && Geo<4, 1>::SLOT >= Geo<3, 1>::SLOT,
+static_assert(GeoGU<8>::SLOT >= GeoGU<4>::SLOT && GeoGU<4>::SLOT >= GeoGU<3>::SLOT &&
+                  GeoDN<8>::SLOT >= GeoDN<4>::SLOT && GeoDN<4>::SLOT >= GeoDN<3>::SLOT,
               "slot sizes per class");
+static_assert(tiles_per_task(true) <= 32 && tiles_per_task(false) <= 32, "one copy lane a tile");
 
 constexpr int kFirstSlot = 1;  // the slot opens its task
 constexpr int kLastSlot = 2;   // the slot closes its task
@@ -96,7 +111,7 @@ struct SlotDesc {
 // consumers when the task starts.
 struct TaskMeta {
     int valid;   // 0: no more tasks of this width class
-    int tq;      // tile group: tiles 14 tq .. 14 tq + 13
+    int tq;      // tile group: tiles n tq .. n tq + n - 1, n = tiles_per_task
     int p;       // K part
     int pos0;    // first route position of the work group
     int ntok;    // tokens in the group (1 .. kDecodeGroup)
@@ -145,7 +160,7 @@ __device__ __forceinline__ void split_task(int task, int n_tq, int parts, int& g
 // Raw words of this thread's share of one row's block (chunk row `r`).
 template <int B>
 __device__ __forceinline__ void load_row_words(const uint8_t* chunk, int r, int t, int g,
-                                               uint32_t (&w)[Geo<B, 1>::WORDS]) {
+                                               uint32_t (&w)[Geo<B, 1, 1>::WORDS]) {
     const uint8_t* blk = chunk + r * block_bytes(B);
     if constexpr (B == 4) {
         const uint4 v = *reinterpret_cast<const uint4*>(blk + 16 * t);
@@ -182,12 +197,91 @@ __device__ __forceinline__ void load_act_half(const __nv_bfloat16* row, int j, i
     xb[4] = v1.x; xb[5] = v1.y; xb[6] = v1.z; xb[7] = v1.w;
 }
 
+// The unpack's masks and magic numbers, held in registers. Each is produced by
+// an opaque move once per consumer class, so the compiler keeps it in a
+// register for the LOP3s instead of materialising the constant beside every
+// use (the register budget allows it).
+__device__ __forceinline__ uint32_t reg_const(uint32_t v) {
+    uint32_t d;
+    asm volatile("mov.b32 %0, %1;" : "=r"(d) : "r"(v));
+    return d;
+}
+
+template <int N>
+__device__ __forceinline__ uint32_t shr_imm(uint32_t a) {
+    uint32_t d;
+    asm("shr.b32 %0, %1, %2;" : "=r"(d) : "r"(a), "n"(N));
+    return d;
+}
+
+template <int B>
+struct UnpackRegs;
+
+template <>
+struct UnpackRegs<4> {
+    uint32_t mask, magic, off;
+    __device__ __forceinline__ UnpackRegs()
+        : mask(reg_const(0x000F000Fu)), magic(reg_const(kMagic)),
+          off(reg_const(pair_offset<4>(0))) {}
+    // pair m (0..15) of a quarter's 4 words, offset form: k + 136
+    __device__ __forceinline__ uint32_t pair(const uint32_t* w, int m) const {
+        const uint32_t x = w[m >> 2];
+        const uint32_t v = (m & 3) == 0 ? x
+                           : (m & 3) == 1 ? shr_imm<4>(x)
+                           : (m & 3) == 2 ? shr_imm<8>(x)
+                                          : shr_imm<12>(x);
+        return and_or(v, mask, magic);
+    }
+    __device__ __forceinline__ uint32_t offset(int) const { return off; }
+};
+
+template <>
+struct UnpackRegs<3> {
+    uint32_t m7, m38, b1, b2, b4, magic, magic16, off132, off20;
+    __device__ __forceinline__ UnpackRegs()
+        : m7(reg_const(0x00070007u)), m38(reg_const(0x00380038u)), b1(reg_const(0x00010001u)),
+          b2(reg_const(0x00020002u)), b4(reg_const(0x00040004u)), magic(reg_const(kMagic)),
+          magic16(reg_const(kMagic16)), off132(reg_const(pair_offset<3>(0))),
+          off20(reg_const(pair_offset<3>(1))) {}
+    // pair m (0..15) of a quarter's 3 words, offset form (see unpack_pair_off)
+    __device__ __forceinline__ uint32_t pair(const uint32_t* w, int m) const {
+        if (m == 15) {
+            uint32_t t = and_or(shr_imm<15>(w[0]), b1, magic);
+            t = and_or(shr_imm<14>(w[1]), b2, t);
+            return and_or(shr_imm<13>(w[2]), b4, t);
+        }
+        const int v = m / 5, f = m % 5;
+        const uint32_t x = f < 2 ? w[v] : (f < 4 ? shr_imm<6>(w[v]) : shr_imm<12>(w[v]));
+        if (f == 1 || f == 3) return and_or(x, m38, magic16);  // 16 + u
+        return and_or(x, m7, magic);                            // 128 + u
+    }
+    __device__ __forceinline__ uint32_t offset(int m) const {
+        return (m < 15 && (m % 5 == 1 || m % 5 == 3)) ? off20 : off132;
+    }
+};
+
+template <>
+struct UnpackRegs<8> {
+    uint32_t m7f, m80, magic;
+    __device__ __forceinline__ UnpackRegs()
+        : m7f(reg_const(0x007F007Fu)), m80(reg_const(0x00800080u)), magic(reg_const(kMagic)) {}
+    // pair m (0..15) of the thread's two 16-byte pieces: the signed code k
+    __device__ __forceinline__ uint32_t pair(const uint32_t* w, int m) const {
+        const uint32_t v = (m & 1) ? shr_imm<8>(w[m >> 1]) : w[m >> 1];
+        const uint32_t lo = and_or(v, m7f, magic);     // 128 + (u & 127)
+        const uint32_t hi = andnot_or(v, m80, magic);  // 256 - 128 * bit7(u)
+        return bf2_sub(lo, hi);                        // u - 128 = k
+    }
+};
+
 // Unpack and multiply one block (128 codes of 16 rows, NM matrices) with NT
 // 8-token n-tiles of activations. Widths 3 and 4 unpack to the offset form
-// (k + off, see common.cuh) and accumulate off . x once per n-tile in accc,
-// which the caller subtracts before finishing the task; width 8 unpacks to k.
-template <int B, int NM, int NT>
-__device__ __forceinline__ void block_mma(const uint32_t (&wr)[NM][2][Geo<B, 1>::WORDS],
+// (k + off, see common.cuh); with OFFSET the off . x term is accumulated in
+// accc (once per n-tile, shared by all tiles of a warp), which the caller
+// subtracts before finishing the task; width 8 unpacks to k.
+template <int B, int NM, int NT, bool OFFSET>
+__device__ __forceinline__ void block_mma(const UnpackRegs<B>& U,
+                                          const uint32_t (&wr)[NM][2][Geo<B, 1, 1>::WORDS],
                                           const uint32_t (&xa)[kMaxTiles][8],
                                           const uint32_t (&xz)[kMaxTiles][8],
                                           float (&acc)[kMaxTiles][NM][4],
@@ -196,18 +290,10 @@ __device__ __forceinline__ void block_mma(const uint32_t (&wr)[NM][2][Geo<B, 1>:
     for (int c = 0; c < 8; ++c) {
 #pragma unroll
         for (int m = 0; m < NM; ++m) {
-            uint32_t a0, a1, a2, a3;
-            if constexpr (B == 8) {
-                a0 = unpack_pair<B>(wr[m][0], 2 * c);
-                a1 = unpack_pair<B>(wr[m][1], 2 * c);
-                a2 = unpack_pair<B>(wr[m][0], 2 * c + 1);
-                a3 = unpack_pair<B>(wr[m][1], 2 * c + 1);
-            } else {
-                a0 = unpack_pair_off<B>(wr[m][0], 2 * c);
-                a1 = unpack_pair_off<B>(wr[m][1], 2 * c);
-                a2 = unpack_pair_off<B>(wr[m][0], 2 * c + 1);
-                a3 = unpack_pair_off<B>(wr[m][1], 2 * c + 1);
-            }
+            const uint32_t a0 = U.pair(wr[m][0], 2 * c);
+            const uint32_t a1 = U.pair(wr[m][1], 2 * c);
+            const uint32_t a2 = U.pair(wr[m][0], 2 * c + 1);
+            const uint32_t a3 = U.pair(wr[m][1], 2 * c + 1);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
                 const uint32_t b0 = c < 4 ? xa[nt][2 * c] : xz[nt][2 * c - 8];
@@ -215,9 +301,9 @@ __device__ __forceinline__ void block_mma(const uint32_t (&wr)[NM][2][Geo<B, 1>:
                 mma_bf16_16816(acc[nt][m], a0, a1, a2, a3, b0, b1);
             }
         }
-        if constexpr (B != 8) {
+        if constexpr (B != 8 && OFFSET) {
             // rows of the offset matrix are all alike: rows g and g+8 share a value
-            const uint32_t o0 = pair_offset<B>(2 * c), o1 = pair_offset<B>(2 * c + 1);
+            const uint32_t o0 = U.offset(2 * c), o1 = U.offset(2 * c + 1);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
                 const uint32_t b0 = c < 4 ? xa[nt][2 * c] : xz[nt][2 * c - 8];
@@ -229,9 +315,10 @@ __device__ __forceinline__ void block_mma(const uint32_t (&wr)[NM][2][Geo<B, 1>:
 }
 
 struct Task {
-    int tau, p, pos0, ntok, j_hi;
+    int tau, p, pos0, ntok, j_hi;  // tau: the warp's first tile
     float scale;
-    bool valid;  // this warp's tile exists
+    bool valid;   // the warp's first tile exists
+    bool valid1;  // its second tile exists (two tiles a warp)
 };
 
 // Finish a task. One K part (P = 1): gate/up applies SwiGLU and stores h
@@ -240,9 +327,9 @@ struct Task {
 // gv[p][pos][m][row] = s_e acc, down y[p][pos][row] = s_e acc -- and a later
 // pass sums the slices in part order (deterministic, no atomics).
 template <bool GATEUP>
-__device__ __forceinline__ void finish(const Args& a, const Task& T,
-                                       float (&acc)[kMaxTiles][GATEUP ? 2 : 1][4], int lane) {
-    if (!T.valid) return;
+__device__ __forceinline__ void finish(const Args& a, const Task& T, int tau,
+                                       const float (&acc)[kMaxTiles][GATEUP ? 2 : 1][4],
+                                       int lane) {
     const int g = lane >> 2, t = lane & 3;
     const int F = a.P.F, H = a.P.H;
 #pragma unroll
@@ -251,7 +338,7 @@ __device__ __forceinline__ void finish(const Args& a, const Task& T,
         for (int q = 0; q < 4; ++q) {
             const int n = nt * 8 + 2 * t + (q & 1);
             if (n >= T.ntok) continue;
-            const int row = T.tau * 16 + g + 8 * (q >> 1);
+            const int row = tau * 16 + g + 8 * (q >> 1);
             const int pos = T.pos0 + n;
             if (GATEUP) {
                 const float gv = T.scale * acc[nt][0][q];
@@ -295,7 +382,8 @@ __device__ __forceinline__ bool resolve_class(const Args& a, const CtaSmem& sm, 
     const int K = GATEUP ? P.H : P.F;
     const int R = GATEUP ? P.F : P.H;
     const int nj = K / kCodesPerBlock;
-    const int n_tq = (R / 16 + kConsumers - 1) / kConsumers;
+    constexpr int TT = tiles_per_task(GATEUP);
+    const int n_tq = (R / 16 + TT - 1) / TT;
     const int n_tasks = n_groups * n_tq * a.parts;
     const int lane = threadIdx.x & 31;
     for (;;) {
@@ -343,8 +431,8 @@ __device__ __forceinline__ bool resolve_class(const Args& a, const CtaSmem& sm, 
     }
 }
 
-// Copy warp: every task of one width class, from the queue. Lane l < 14 owns
-// the copy stream of tile l (a page cursor in registers, the next page's index
+// Copy warp: every task of one width class, from the queue. Lane l owns the
+// copy stream of the task's tile l (a page cursor in registers, the next page's index
 // loaded ahead): per slot one run of NM x jc chunks (gate/up: W1 and W3
 // alternate). Lane 0 arms the full barriers and writes the slot descriptors;
 // every lane prefetches one activation line. `ep` / `used` track the slots'
@@ -356,7 +444,8 @@ __device__ __forceinline__ bool produce_class(const Args& a, const CtaSmem& sm, 
                                               uint32_t& fph, uint32_t& ep, uint32_t& used,
                                               bool& need_wait) {
     constexpr int NM = GATEUP ? 2 : 1;
-    using G = Geo<B, NM>;
+    constexpr int TT = tiles_per_task(GATEUP);
+    using G = Geo<B, NM, tiles_per_warp(GATEUP)>;
     constexpr int S = G::S;
     const PagedExperts& P = a.P;
     const int K = GATEUP ? P.H : P.F;
@@ -366,7 +455,7 @@ __device__ __forceinline__ bool produce_class(const Args& a, const CtaSmem& sm, 
     const int cpp = chunks_per_page(B, P.page_bytes);
     const int n_pages = (3 * nc1 + cpp - 1) / cpp;
     const int lane = threadIdx.x & 31;
-    const bool copier = lane < kConsumers;
+    const bool copier = lane < TT;
 
     auto acquire = [&](int s) -> bool {
         if ((used >> s) & 1u) {
@@ -412,12 +501,12 @@ __device__ __forceinline__ bool produce_class(const Args& a, const CtaSmem& sm, 
             __syncwarp();
             return true;
         }
-        const int active = min(kConsumers, n_tiles - tq * kConsumers);
+        const int active = min(TT, n_tiles - tq * TT);
         const bool my_tile = copier && lane < active;
         int pslot = 0, poff = 0;
         uint32_t page = 0, page_next = 0;
         if (my_tile) {
-            const int tau = tq * kConsumers + lane;
+            const int tau = tq * TT + lane;
             const int c = GATEUP ? 2 * (tau * nj + j) : 2 * nc1 + tau * nj + j;
             pslot = c / cpp;
             poff = c - pslot * cpp;
@@ -439,7 +528,7 @@ __device__ __forceinline__ bool produce_class(const Args& a, const CtaSmem& sm, 
             if (my_tile) {
                 // NM x jc consecutive chunks of this tile; a page boundary splits
                 // the copy in two
-                uint8_t* dst = sm.ring + (size_t)s * G::SLOT + (size_t)lane * G::TILE;
+                uint8_t* dst = sm.ring + (size_t)s * G::SLOT + (size_t)lane * G::TILEB;
                 const int total = NM * jc;
                 const int n1 = min(total, cpp - poff);
                 bulk_g2s(dst, P.pool + (size_t)page * P.page_bytes + (size_t)poff * G::CB,
@@ -472,13 +561,14 @@ __device__ __forceinline__ bool produce_class(const Args& a, const CtaSmem& sm, 
     }
 }
 
-// Consumer warp w: all tasks of one width class, tile w of each task. `fp`
-// tracks the slots' full-barrier phases across classes.
+// Consumer warp w: all tasks of one width class, tiles w * TPW .. of each
+// task. `fp` tracks the slots' full-barrier phases across classes.
 template <int B, bool GATEUP>
 __device__ __forceinline__ bool consume_class(const Args& a, const CtaSmem& sm, uint32_t& fp,
                                               int w) {
     constexpr int NM = GATEUP ? 2 : 1;
-    using G = Geo<B, NM>;
+    constexpr int TPW = tiles_per_warp(GATEUP);
+    using G = Geo<B, NM, TPW>;
     constexpr int S = G::S;
     const PagedExperts& P = a.P;
     const int K = GATEUP ? P.H : P.F;
@@ -490,31 +580,21 @@ __device__ __forceinline__ bool consume_class(const Args& a, const CtaSmem& sm, 
     Task T{};
     const __nv_bfloat16* arow[kMaxTiles] = {};
     int ntiles = 0;
-    float acc[kMaxTiles][NM][4];
+    float acc[TPW][kMaxTiles][NM][4];
     float accc[kMaxTiles][4];  // offset term (widths 3, 4), subtracted at the task's end
-    // activations of the block being multiplied (xa, xz) and of the next block
-    // of the task (na, nz), loaded one block ahead so that the loads' latency
-    // hides behind a block of unpacking and MMAs
-    uint32_t xa[kMaxTiles][8], xz[kMaxTiles][8];
-    uint32_t na[kMaxTiles][8], nz[kMaxTiles][8];
-    auto load_next = [&](int j) {
-#pragma unroll
-        for (int nt = 0; nt < kMaxTiles; ++nt) {
-            if (nt == 0 || nt < ntiles) {
-                load_act_half(arow[nt], j, lane & 3, B == 8, 0, na[nt]);
-                load_act_half(arow[nt], j, lane & 3, B == 8, 1, nz[nt]);
-            }
-        }
-    };
-    // acc <- acc - off . x for every matrix (a no-op for width 8)
+    uint32_t xa[kMaxTiles][8], xz[kMaxTiles][8];  // activations of the block
+    const UnpackRegs<B> U;
+    // acc <- acc - off . x for every tile and matrix (a no-op for width 8)
     auto settle = [&]() {
         if constexpr (B != 8) {
 #pragma unroll
-            for (int nt = 0; nt < kMaxTiles; ++nt)
+            for (int i = 0; i < TPW; ++i)
 #pragma unroll
-                for (int m = 0; m < NM; ++m)
+                for (int nt = 0; nt < kMaxTiles; ++nt)
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) acc[nt][m][q] -= accc[nt][q];
+                    for (int m = 0; m < NM; ++m)
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) acc[i][nt][m][q] -= accc[nt][q];
         }
     };
     for (int s = 0;; s = (s + 1 == S) ? 0 : s + 1) {
@@ -535,8 +615,9 @@ __device__ __forceinline__ bool consume_class(const Args& a, const CtaSmem& sm, 
         }
         if (d.flags & kFirstSlot) {
             const TaskMeta* m = sm.taskq + d.q;
-            T.tau = m->tq * kConsumers + w;
+            T.tau = m->tq * tiles_per_task(GATEUP) + w * TPW;
             T.valid = T.tau < n_tiles;
+            T.valid1 = TPW > 1 && T.tau + 1 < n_tiles;
             T.p = m->p;
             T.pos0 = m->pos0;
             T.ntok = m->ntok;
@@ -548,15 +629,16 @@ __device__ __forceinline__ bool consume_class(const Args& a, const CtaSmem& sm, 
                 const int n = nt * 8 + g;
                 arow[nt] = n < T.ntok ? a.act + (size_t)m->rows[n] * K : nullptr;
 #pragma unroll
-                for (int mm = 0; mm < NM; ++mm)
+                for (int i = 0; i < TPW; ++i)
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) acc[nt][mm][q] = 0.0f;
+                    for (int mm = 0; mm < NM; ++mm)
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) acc[i][nt][mm][q] = 0.0f;
 #pragma unroll
                 for (int q = 0; q < 4; ++q) accc[nt][q] = 0.0f;
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.tq_empty[d.q]);
-            if (T.valid) load_next(d.j);
         }
         if (!T.valid) {  // this warp has no tile in the task: release at once
             __syncwarp();
@@ -564,16 +646,20 @@ __device__ __forceinline__ bool consume_class(const Args& a, const CtaSmem& sm, 
             continue;
         }
         const int t = lane & 3;
-        const uint8_t* tile = sm.ring + (size_t)s * G::SLOT + (size_t)w * G::TILE;
+        const uint8_t* tiles = sm.ring + (size_t)s * G::SLOT + (size_t)w * TPW * G::TILEB;
 #pragma unroll
         for (int jj = 0; jj < G::J; ++jj) {
             if (jj >= d.nc) break;
-            uint32_t wr[NM][2][G::WORDS];
+            uint32_t wr[TPW][NM][2][G::WORDS];
 #pragma unroll
-            for (int m = 0; m < NM; ++m) {
-                const uint8_t* chunk = tile + (jj * NM + m) * G::CB;
-                load_row_words<B>(chunk, g, t, g, wr[m][0]);
-                load_row_words<B>(chunk, g + 8, t, g, wr[m][1]);
+            for (int i = 0; i < TPW; ++i) {
+                if (i > 0 && !T.valid1) break;
+#pragma unroll
+                for (int m = 0; m < NM; ++m) {
+                    const uint8_t* chunk = tiles + i * G::TILEB + (jj * NM + m) * G::CB;
+                    load_row_words<B>(chunk, g, t, g, wr[i][m][0]);
+                    load_row_words<B>(chunk, g + 8, t, g, wr[i][m][1]);
+                }
             }
             if (jj + 1 == d.nc) {  // the slot's last words are in registers: release it
                 __syncwarp();
@@ -581,24 +667,23 @@ __device__ __forceinline__ bool consume_class(const Args& a, const CtaSmem& sm, 
             }
             const int j = d.j + jj;
 #pragma unroll
-            for (int nt = 0; nt < kMaxTiles; ++nt)
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    xa[nt][i] = na[nt][i];
-                    xz[nt][i] = nz[nt][i];
-                }
-            if (j + 1 < T.j_hi) load_next(j + 1);
-            if constexpr (kMaxTiles > 1) {
-                if (ntiles > 1) {
-                    block_mma<B, NM, kMaxTiles>(wr, xa, xz, acc, accc);
-                    continue;
+            for (int nt = 0; nt < kMaxTiles; ++nt) {
+                if (nt == 0 || nt < ntiles) {
+                    load_act_half(arow[nt], j, t, B == 8, 0, xa[nt]);
+                    load_act_half(arow[nt], j, t, B == 8, 1, xz[nt]);
                 }
             }
-            block_mma<B, NM, 1>(wr, xa, xz, acc, accc);
+            block_mma<B, NM, kMaxTiles, true>(U, wr[0], xa, xz, acc[0], accc);
+            if constexpr (TPW > 1) {
+                if (T.valid1) block_mma<B, NM, kMaxTiles, false>(U, wr[1], xa, xz, acc[1], accc);
+            }
         }
         if (d.flags & kLastSlot) {
             settle();
-            finish<GATEUP>(a, T, acc, lane);
+            finish<GATEUP>(a, T, T.tau, acc[0], lane);
+            if constexpr (TPW > 1) {
+                if (T.valid1) finish<GATEUP>(a, T, T.tau + 1, acc[1], lane);
+            }
         }
     }
 }
@@ -689,10 +774,11 @@ void decode_plan(mpe_ctx* c, size_t Tk, DecodePlan& pl) {
     const int per_cta = env_int("MPE_DECODE_TASKS_PER_CTA", 8);
     pl.claim = 1;
     const int nj_gu = c->H / kCodesPerBlock, nj_dn = c->F / kCodesPerBlock;
-    int p = decode_parts(groups, (c->F / 16 + kConsumers - 1) / kConsumers, nj_gu, ctas, per_cta);
+    const int tt_gu = tiles_per_task(true), tt_dn = tiles_per_task(false);
+    int p = decode_parts(groups, (c->F / 16 + tt_gu - 1) / tt_gu, nj_gu, ctas, per_cta);
     pl.kb_gu = (nj_gu + p - 1) / p;
     pl.p_gu = (nj_gu + pl.kb_gu - 1) / pl.kb_gu;
-    p = decode_parts(groups, (c->H / 16 + kConsumers - 1) / kConsumers, nj_dn, ctas, per_cta);
+    p = decode_parts(groups, (c->H / 16 + tt_dn - 1) / tt_dn, nj_dn, ctas, per_cta);
     pl.kb_dn = (nj_dn + p - 1) / p;
     pl.p_dn = (nj_dn + pl.kb_dn - 1) / pl.kb_dn;
 }
