@@ -119,6 +119,10 @@ struct TaskMeta {
     float scale;   // s_e
     uint32_t first;  // the expert's first entry in the page-index array
     int rows[kDecodeGroup];  // activation row of each token (x row, or h row = position)
+    // widths 3 and 4: off . x of each token over the task's K range, the term
+    // the offset-form unpack adds to every row (written after the rest, see
+    // tq_sum)
+    float offsum[kDecodeGroup];
 };
 
 struct Args {
@@ -139,7 +143,7 @@ struct Args {
 };
 
 constexpr size_t kBarOff = kRingBytes;
-constexpr size_t kDescOff = kBarOff + (2 * kMaxSlots + 2 * kTaskQ) * sizeof(uint64_t);
+constexpr size_t kDescOff = kBarOff + (2 * kMaxSlots + 3 * kTaskQ) * sizeof(uint64_t);
 constexpr size_t kTaskOff = kDescOff + kMaxSlots * sizeof(SlotDesc);
 
 __host__ __device__ constexpr size_t smem_bytes() {
@@ -219,10 +223,8 @@ struct UnpackRegs;
 
 template <>
 struct UnpackRegs<4> {
-    uint32_t mask, magic, off;
-    __device__ __forceinline__ UnpackRegs()
-        : mask(reg_const(0x000F000Fu)), magic(reg_const(kMagic)),
-          off(reg_const(pair_offset<4>(0))) {}
+    uint32_t mask, magic;
+    __device__ __forceinline__ UnpackRegs() : mask(reg_const(0x000F000Fu)), magic(reg_const(kMagic)) {}
     // pair m (0..15) of a quarter's 4 words, offset form: k + 136
     __device__ __forceinline__ uint32_t pair(const uint32_t* w, int m) const {
         const uint32_t x = w[m >> 2];
@@ -232,17 +234,15 @@ struct UnpackRegs<4> {
                                           : shr_imm<12>(x);
         return and_or(v, mask, magic);
     }
-    __device__ __forceinline__ uint32_t offset(int) const { return off; }
 };
 
 template <>
 struct UnpackRegs<3> {
-    uint32_t m7, m38, b1, b2, b4, magic, magic16, off132, off20;
+    uint32_t m7, m38, b1, b2, b4, magic, magic16;
     __device__ __forceinline__ UnpackRegs()
         : m7(reg_const(0x00070007u)), m38(reg_const(0x00380038u)), b1(reg_const(0x00010001u)),
           b2(reg_const(0x00020002u)), b4(reg_const(0x00040004u)), magic(reg_const(kMagic)),
-          magic16(reg_const(kMagic16)), off132(reg_const(pair_offset<3>(0))),
-          off20(reg_const(pair_offset<3>(1))) {}
+          magic16(reg_const(kMagic16)) {}
     // pair m (0..15) of a quarter's 3 words, offset form (see unpack_pair_off)
     __device__ __forceinline__ uint32_t pair(const uint32_t* w, int m) const {
         if (m == 15) {
@@ -254,9 +254,6 @@ struct UnpackRegs<3> {
         const uint32_t x = f < 2 ? w[v] : (f < 4 ? shr_imm<6>(w[v]) : shr_imm<12>(w[v]));
         if (f == 1 || f == 3) return and_or(x, m38, magic16);  // 16 + u
         return and_or(x, m7, magic);                            // 128 + u
-    }
-    __device__ __forceinline__ uint32_t offset(int m) const {
-        return (m < 15 && (m % 5 == 1 || m % 5 == 3)) ? off20 : off132;
     }
 };
 
@@ -276,16 +273,14 @@ struct UnpackRegs<8> {
 
 // Unpack and multiply one block (128 codes of 16 rows, NM matrices) with NT
 // 8-token n-tiles of activations. Widths 3 and 4 unpack to the offset form
-// (k + off, see common.cuh); with OFFSET the off . x term is accumulated in
-// accc (once per n-tile, shared by all tiles of a warp), which the caller
-// subtracts before finishing the task; width 8 unpacks to k.
-template <int B, int NM, int NT, bool OFFSET>
+// (k + off, see common.cuh), whose off . x term the task's offset sums remove;
+// width 8 unpacks to k.
+template <int B, int NM, int NT>
 __device__ __forceinline__ void block_mma(const UnpackRegs<B>& U,
                                           const uint32_t (&wr)[NM][2][Geo<B, 1, 1>::WORDS],
                                           const uint32_t (&xa)[kMaxTiles][8],
                                           const uint32_t (&xz)[kMaxTiles][8],
-                                          float (&acc)[kMaxTiles][NM][4],
-                                          float (&accc)[kMaxTiles][4]) {
+                                          float (&acc)[kMaxTiles][NM][4]) {
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
 #pragma unroll
@@ -299,16 +294,6 @@ __device__ __forceinline__ void block_mma(const UnpackRegs<B>& U,
                 const uint32_t b0 = c < 4 ? xa[nt][2 * c] : xz[nt][2 * c - 8];
                 const uint32_t b1 = c < 4 ? xa[nt][2 * c + 1] : xz[nt][2 * c - 7];
                 mma_bf16_16816(acc[nt][m], a0, a1, a2, a3, b0, b1);
-            }
-        }
-        if constexpr (B != 8 && OFFSET) {
-            // rows of the offset matrix are all alike: rows g and g+8 share a value
-            const uint32_t o0 = U.offset(2 * c), o1 = U.offset(2 * c + 1);
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                const uint32_t b0 = c < 4 ? xa[nt][2 * c] : xz[nt][2 * c - 8];
-                const uint32_t b1 = c < 4 ? xa[nt][2 * c + 1] : xz[nt][2 * c - 7];
-                mma_bf16_16816(accc[nt], o0, o0, o1, o1, b0, b1);
             }
         }
     }
@@ -362,7 +347,8 @@ struct CtaSmem {
     uint8_t* ring;
     uint64_t* full;      // per slot: 1 producer arrival + transaction bytes
     uint64_t* empty;     // per slot: one arrival per consumer warp
-    uint64_t* tq_full;   // per queue entry: the task warp's arrival
+    uint64_t* tq_full;   // per queue entry: the task warp's arrival (task resolved)
+    uint64_t* tq_sum;    // per queue entry: the task warp's arrival (offset sums written)
     uint64_t* tq_empty;  // per queue entry: the copy warp + every consumer warp
     SlotDesc* descs;
     TaskMeta* taskq;
@@ -370,14 +356,27 @@ struct CtaSmem {
 
 __device__ __forceinline__ uint32_t next_q(uint32_t q) { return q + 1 == kTaskQ ? 0u : q + 1; }
 
+// Offset of code position c (0..31) of a quarter in the offset-form unpack
+// (common.cuh): 136 for width 4; 132 or 20 by pair for width 3.
+template <int B>
+__device__ __forceinline__ float code_offset(int c) {
+    if constexpr (B == 4) return 136.0f;
+    const int m = c >> 1;
+    return (m < 15 && (m % 5 == 1 || m % 5 == 3)) ? 20.0f : 132.0f;
+}
+
 // Task warp: claims the tasks of one width class in counter order and writes
 // each, resolved, into the next free queue entry; then one end-of-class entry.
-// `q` and the phase bits `ph` / `used` of the queue's empty barriers carry
-// over between classes.
-template <bool GATEUP>
+// For widths 3 and 4 it then adds up, per token, off(k) x[k] over the task's K
+// range in fp32 (the offset-form unpack adds off(k) to every code; the
+// consumers subtract this sum once per task) and signals tq_sum. In the down
+// kernel the activations come from the preceding kernel, so the first sum
+// waits for it (`need_wait`). `q` and the phase bits `ph` / `used` of the
+// queue's empty barriers carry over between classes.
+template <int B, bool GATEUP>
 __device__ __forceinline__ bool resolve_class(const Args& a, const CtaSmem& sm, int group0,
                                               int n_groups, int32_t* ctr, uint32_t& q,
-                                              uint32_t& ph, uint32_t& used) {
+                                              uint32_t& ph, uint32_t& used, bool& need_wait) {
     const PagedExperts& P = a.P;
     const int K = GATEUP ? P.H : P.F;
     const int R = GATEUP ? P.F : P.H;
@@ -426,6 +425,40 @@ __device__ __forceinline__ bool resolve_class(const Args& a, const CtaSmem& sm, 
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.tq_full[q]);
+        if (more) {
+            if constexpr (B != 8) {
+                if (need_wait) {
+                    griddep_wait();
+                    need_wait = false;
+                }
+                // lane l adds 8 consecutive codes per 256: positions 8 (l % 4) .. + 7
+                // of a quarter
+                float off[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) off[e] = code_offset<B>(8 * (lane & 3) + e);
+                const int k_lo = 128 * m->j0, k_hi = 128 * m->j_hi, ntok = m->ntok;
+                for (int i = 0; i < ntok; ++i) {
+                    const __nv_bfloat16* row = a.act + (size_t)m->rows[i] * K;
+                    float sum = 0.0f;
+                    for (int k = k_lo + 8 * lane; k < k_hi; k += 256) {
+                        const uint4 v = __ldg(reinterpret_cast<const uint4*>(row + k));
+                        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float lo = __uint_as_float(wv[e] << 16);
+                            const float hi = __uint_as_float(wv[e] & 0xFFFF0000u);
+                            sum = fmaf(off[2 * e], lo, sum);
+                            sum = fmaf(off[2 * e + 1], hi, sum);
+                        }
+                    }
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+                    if (lane == 0) m->offsum[i] = sum;
+                }
+                __syncwarp();
+            }
+            if (lane == 0) mbar_arrive(&sm.tq_sum[q]);
+        }
         q = next_q(q);
         if (!more) return true;
     }
@@ -562,10 +595,12 @@ __device__ __forceinline__ bool produce_class(const Args& a, const CtaSmem& sm, 
 }
 
 // Consumer warp w: all tasks of one width class, tiles w * TPW .. of each
-// task. `fp` tracks the slots' full-barrier phases across classes.
+// task. `fp` tracks the slots' full-barrier phases across classes, `sph` the
+// queue's offset-sum barrier phases. A warp holds its task's queue entry until
+// the task's last slot, where it reads the offset sums.
 template <int B, bool GATEUP>
 __device__ __forceinline__ bool consume_class(const Args& a, const CtaSmem& sm, uint32_t& fp,
-                                              int w) {
+                                              uint32_t& sph, int w) {
     constexpr int NM = GATEUP ? 2 : 1;
     constexpr int TPW = tiles_per_warp(GATEUP);
     using G = Geo<B, NM, TPW>;
@@ -581,20 +616,27 @@ __device__ __forceinline__ bool consume_class(const Args& a, const CtaSmem& sm, 
     const __nv_bfloat16* arow[kMaxTiles] = {};
     int ntiles = 0;
     float acc[TPW][kMaxTiles][NM][4];
-    float accc[kMaxTiles][4];  // offset term (widths 3, 4), subtracted at the task's end
     uint32_t xa[kMaxTiles][8], xz[kMaxTiles][8];  // activations of the block
     const UnpackRegs<B> U;
-    // acc <- acc - off . x for every tile and matrix (a no-op for width 8)
-    auto settle = [&]() {
+    // widths 3, 4: acc <- acc - off . x for every tile and matrix, with the
+    // task warp's per-token sums (accumulator column n = token n)
+    auto settle = [&](const TaskMeta* m) {
         if constexpr (B != 8) {
+            const int t = lane & 3;
 #pragma unroll
-            for (int i = 0; i < TPW; ++i)
+            for (int nt = 0; nt < kMaxTiles; ++nt)
 #pragma unroll
-                for (int nt = 0; nt < kMaxTiles; ++nt)
+                for (int h = 0; h < 2; ++h) {
+                    const int n = nt * 8 + 2 * t + h;
+                    const float o = n < T.ntok ? m->offsum[n] : 0.0f;
 #pragma unroll
-                    for (int m = 0; m < NM; ++m)
+                    for (int i = 0; i < TPW; ++i)
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) acc[i][nt][m][q] -= accc[nt][q];
+                        for (int mm = 0; mm < NM; ++mm) {
+                            acc[i][nt][mm][h] -= o;
+                            acc[i][nt][mm][h + 2] -= o;
+                        }
+                }
         }
     };
     for (int s = 0;; s = (s + 1 == S) ? 0 : s + 1) {
@@ -613,6 +655,28 @@ __device__ __forceinline__ bool consume_class(const Args& a, const CtaSmem& sm, 
             }
             return true;
         }
+        // the task's last slot: offset sums, finish, release the queue entry
+        auto close_task = [&]() -> bool {
+            const uint32_t sp = (sph >> d.q) & 1u;
+            sph ^= 1u << d.q;
+            const TaskMeta* m = sm.taskq + d.q;
+            if (T.valid) {
+                if constexpr (B != 8) {
+                    if (!mbar_wait_bounded(&sm.tq_sum[d.q], sp)) {
+                        if (lane == 0) set_status(a.status, MPE_STATUS_WAIT_TIMEOUT);
+                        return false;
+                    }
+                    settle(m);
+                }
+                finish<GATEUP>(a, T, T.tau, acc[0], lane);
+                if constexpr (TPW > 1) {
+                    if (T.valid1) finish<GATEUP>(a, T, T.tau + 1, acc[1], lane);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.tq_empty[d.q]);
+            return true;
+        };
         if (d.flags & kFirstSlot) {
             const TaskMeta* m = sm.taskq + d.q;
             T.tau = m->tq * tiles_per_task(GATEUP) + w * TPW;
@@ -634,15 +698,12 @@ __device__ __forceinline__ bool consume_class(const Args& a, const CtaSmem& sm, 
                     for (int mm = 0; mm < NM; ++mm)
 #pragma unroll
                         for (int q = 0; q < 4; ++q) acc[i][nt][mm][q] = 0.0f;
-#pragma unroll
-                for (int q = 0; q < 4; ++q) accc[nt][q] = 0.0f;
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.tq_empty[d.q]);
         }
         if (!T.valid) {  // this warp has no tile in the task: release at once
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.empty[s]);
+            if ((d.flags & kLastSlot) && !close_task()) return false;
             continue;
         }
         const int t = lane & 3;
@@ -673,18 +734,12 @@ __device__ __forceinline__ bool consume_class(const Args& a, const CtaSmem& sm, 
                     load_act_half(arow[nt], j, t, B == 8, 1, xz[nt]);
                 }
             }
-            block_mma<B, NM, kMaxTiles, true>(U, wr[0], xa, xz, acc[0], accc);
+            block_mma<B, NM, kMaxTiles>(U, wr[0], xa, xz, acc[0]);
             if constexpr (TPW > 1) {
-                if (T.valid1) block_mma<B, NM, kMaxTiles, false>(U, wr[1], xa, xz, acc[1], accc);
+                if (T.valid1) block_mma<B, NM, kMaxTiles>(U, wr[1], xa, xz, acc[1]);
             }
         }
-        if (d.flags & kLastSlot) {
-            settle();
-            finish<GATEUP>(a, T, T.tau, acc[0], lane);
-            if constexpr (TPW > 1) {
-                if (T.valid1) finish<GATEUP>(a, T, T.tau + 1, acc[1], lane);
-            }
-        }
+        if ((d.flags & kLastSlot) && !close_task()) return false;
     }
 }
 
@@ -697,7 +752,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(Args a) {
     sm.full = reinterpret_cast<uint64_t*>(smem + kBarOff);
     sm.empty = sm.full + kMaxSlots;
     sm.tq_full = sm.empty + kMaxSlots;
-    sm.tq_empty = sm.tq_full + kTaskQ;
+    sm.tq_sum = sm.tq_full + kTaskQ;
+    sm.tq_empty = sm.tq_sum + kTaskQ;
     sm.descs = reinterpret_cast<SlotDesc*>(smem + kDescOff);
     sm.taskq = reinterpret_cast<TaskMeta*>(smem + kTaskOff);
     if (threadIdx.x == 0) {
@@ -707,6 +763,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(Args a) {
         }
         for (int q = 0; q < kTaskQ; ++q) {
             mbar_init(&sm.tq_full[q], 1);
+            mbar_init(&sm.tq_sum[q], 1);
             mbar_init(&sm.tq_empty[q], kConsumers + 1);
         }
         fence_mbar_init();
@@ -716,15 +773,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(Args a) {
     if (warp == kTaskWarp) {
         // gate/up: the work groups and task counters come from the route kernel
         // just before; down: that kernel finished before the one that precedes
-        // this launch let it start
+        // this launch let it start (the offset sums over h wait for it)
         if (GATEUP) griddep_wait();
         if (lane == 0) griddep_launch_dependents();
         const int n8 = __ldcg(a.n_wg_class), n4 = __ldcg(a.n_wg_class + 1),
                   n3 = __ldcg(a.n_wg_class + 2);
         uint32_t q = 0, ph = 0, used = 0;
-        if (!resolve_class<GATEUP>(a, sm, 0, n8, a.task_ctr + 0, q, ph, used)) return;
-        if (!resolve_class<GATEUP>(a, sm, n8, n4, a.task_ctr + 1, q, ph, used)) return;
-        resolve_class<GATEUP>(a, sm, n8 + n4, n3, a.task_ctr + 2, q, ph, used);
+        bool need_wait = !GATEUP;
+        if (!resolve_class<8, GATEUP>(a, sm, 0, n8, a.task_ctr + 0, q, ph, used, need_wait)) return;
+        if (!resolve_class<4, GATEUP>(a, sm, n8, n4, a.task_ctr + 1, q, ph, used, need_wait)) return;
+        resolve_class<3, GATEUP>(a, sm, n8 + n4, n3, a.task_ctr + 2, q, ph, used, need_wait);
     } else if (warp == kCopyWarp) {
         uint32_t q = 0, fph = 0, ep = 0, used = 0;
         bool need_wait = !GATEUP;
@@ -734,10 +792,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(Args a) {
     } else {
         // down: h is written by the preceding kernel
         if (!GATEUP) griddep_wait();
-        uint32_t fp = 0;
-        if (!consume_class<8, GATEUP>(a, sm, fp, warp)) return;
-        if (!consume_class<4, GATEUP>(a, sm, fp, warp)) return;
-        consume_class<3, GATEUP>(a, sm, fp, warp);
+        uint32_t fp = 0, sph = 0;
+        if (!consume_class<8, GATEUP>(a, sm, fp, sph, warp)) return;
+        if (!consume_class<4, GATEUP>(a, sm, fp, sph, warp)) return;
+        consume_class<3, GATEUP>(a, sm, fp, sph, warp);
     }
 }
 
