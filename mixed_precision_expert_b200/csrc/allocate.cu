@@ -34,8 +34,8 @@ constexpr int kThreads = 1024;
 constexpr size_t kAllocSmemMax = 200 * 1024;
 
 // Choices are 2-bit codes (0: 3 bits, 1: 4 bits, 2: 8 bits), four budget
-// states per byte, so thread i owns whole bytes and no two threads write the
-// same byte. When both DP rows and the table fit in shared memory
+// states per byte; each thread evaluates one state per pass and the first
+// lane of every four writes their byte. When both DP rows and the table fit in shared memory
 // (R <= smem_R; -1 = no on-chip buffers) the whole solve stays on chip -- every expert step is a
 // shared-memory pass plus one barrier, and the serial backtrack reads shared
 // memory -- else rows and table live in the global buffers D and choice.
@@ -106,37 +106,27 @@ k_allocate(const double* p, const uint64_t* W, int E, uint64_t B, uint8_t* bits,
         const double c8 = __dmul_rn(pe, L8);
         const uint32_t u4 = s_up4[e], u8 = s_up8[e];
         uint8_t* ch = chb + (size_t)e * nq;
-        for (uint32_t qd = tid; qd < nq; qd += kThreads) {
-            uint32_t byte = 0;
-#pragma unroll
-            for (uint32_t i = 0; i < 4; ++i) {
-                const uint32_t r = 4 * qd + i;
-                if (r > R) break;
+        // one state a thread; the loop bound is the same for every thread (the
+        // code packing below shuffles across the warp)
+        for (uint32_t base = 0; base <= R; base += kThreads) {
+            const uint32_t r = base + tid;
+            uint32_t code = 0;
+            if (r <= R) {
+                // an unreachable predecessor is +inf and its candidate stays +inf
+                const double x3 = __dadd_rn(Dcur[r], c3);
+                const double x4 = r >= u4 ? __dadd_rn(Dcur[r - u4], c4) : dinf();
+                const double x8 = r >= u8 ? __dadd_rn(Dcur[r - u8], c8) : dinf();
                 double best = dinf();
-                uint32_t code = 0;
-                double prev = Dcur[r];
-                if (prev != dinf()) {
-                    const double cand = __dadd_rn(prev, c3);
-                    if (cand < best) { best = cand; code = 0; }
-                }
-                if (r >= u4) {
-                    prev = Dcur[r - u4];
-                    if (prev != dinf()) {
-                        const double cand = __dadd_rn(prev, c4);
-                        if (cand < best) { best = cand; code = 1; }
-                    }
-                }
-                if (r >= u8) {
-                    prev = Dcur[r - u8];
-                    if (prev != dinf()) {
-                        const double cand = __dadd_rn(prev, c8);
-                        if (cand < best) { best = cand; code = 2; }
-                    }
-                }
+                if (x3 < best) best = x3;
+                if (x4 < best) { best = x4; code = 1; }
+                if (x8 < best) { best = x8; code = 2; }
                 Dnext[r] = best;
-                byte |= code << (2 * i);
             }
-            ch[qd] = (uint8_t)byte;
+            // lanes 4m .. 4m+3 hold states 4m' .. 4m'+3: one byte of codes
+            const uint32_t k1 = __shfl_down_sync(0xffffffffu, code, 1);
+            const uint32_t k2 = __shfl_down_sync(0xffffffffu, code, 2);
+            const uint32_t k3 = __shfl_down_sync(0xffffffffu, code, 3);
+            if ((tid & 3) == 0 && r <= R) ch[r >> 2] = (uint8_t)(code | k1 << 2 | k2 << 4 | k3 << 6);
         }
         __syncthreads();
         double* t = Dcur;

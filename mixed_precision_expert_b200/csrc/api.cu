@@ -77,51 +77,68 @@ int pages_needed(int b, int H, int F, uint32_t page_bytes) {
 
 bool valid_bits(int b) { return b == 3 || b == 4 || b == 8; }
 
-// Lowest-index-first page moves for the experts whose width changes.
-// Transactional: on shortage, returns false and leaves `a` untouched.
-bool plan_pages(const mpe_ctx* c, const std::vector<uint8_t>& new_bits, HostAllocator& a,
+// Lowest-index-first page moves for the experts whose width changes: their
+// pages are released (ascending e), then allocated (ascending e) from the
+// lowest free pages. Transactional: the plan is built beside the allocator
+// (a copy of the free bitmap and new page lists for the changed experts only)
+// and applied by commit_pages; on shortage it returns false and nothing changes.
+struct PagePlan {
+    std::vector<uint8_t> free;
+    std::vector<std::pair<int, std::vector<uint32_t>>> moved;
+};
+
+bool plan_pages(const mpe_ctx* c, const std::vector<uint8_t>& new_bits, PagePlan& plan,
                 std::vector<int>& changed) {
-    HostAllocator n = c->alloc;
     changed.clear();
     for (int e = 0; e < c->E; ++e)
         if (new_bits[e] != c->bits[e]) changed.push_back(e);
-    for (int e : changed) {
-        for (uint32_t p : n.pages[e]) n.free[p] = 1;
-        n.pages[e].clear();
-    }
+    plan.free = c->alloc.free;
+    plan.moved.clear();
+    for (int e : changed)
+        for (uint32_t p : c->alloc.pages[e]) plan.free[p] = 1;
     uint32_t cursor = 0;
     for (int e : changed) {
         const int need = pages_needed(new_bits[e], c->H, c->F, c->page_bytes);
+        std::vector<uint32_t> pg;
+        pg.reserve(need);
         for (int i = 0; i < need; ++i) {
-            while (cursor < c->pool_pages && !n.free[cursor]) ++cursor;
+            while (cursor < c->pool_pages && !plan.free[cursor]) ++cursor;
             if (cursor >= c->pool_pages) return false;
-            n.free[cursor] = 0;
-            n.pages[e].push_back(cursor);
+            plan.free[cursor] = 0;
+            pg.push_back(cursor);
         }
+        plan.moved.emplace_back(e, std::move(pg));
     }
-    a = std::move(n);
     return true;
 }
 
-// Rebuild the host page table from the allocator and upload it (async, from
-// pinned staging that is reused only after the previous upload finished).
+void commit_pages(mpe_ctx* c, PagePlan& plan, const std::vector<uint8_t>& new_bits) {
+    c->alloc.free.swap(plan.free);
+    for (auto& m : plan.moved) c->alloc.pages[m.first] = std::move(m.second);
+    c->bits = new_bits;
+}
+
+// Rebuild the page table (compact page-index array, experts in order) in the
+// pinned staging and upload it (async; the staging is reused only after the
+// previous upload finished).
 int upload_table(mpe_ctx* c) {
-    c->pidx.clear();
+    CK(cudaEventSynchronize(c->upload_done));
+    uint32_t n = 0;
     for (int e = 0; e < c->E; ++e) {
         Pte& p = c->pte[e];
+        const std::vector<uint32_t>& pg = c->alloc.pages[e];
         p.bits = c->bits[e];
-        p.first = (uint32_t)c->pidx.size();
-        p.n_pages = (uint32_t)c->alloc.pages[e].size();
-        c->pidx.insert(c->pidx.end(), c->alloc.pages[e].begin(), c->alloc.pages[e].end());
+        p.first = n;
+        p.n_pages = (uint32_t)pg.size();
+        if (!pg.empty()) std::memcpy(c->h_pidx_pinned + n, pg.data(), sizeof(uint32_t) * pg.size());
+        n += (uint32_t)pg.size();
     }
-    CK(cudaEventSynchronize(c->upload_done));
+    c->pidx_count = n;
     std::memcpy(c->h_pte_pinned, c->pte.data(), sizeof(Pte) * c->E);
-    if (!c->pidx.empty())
-        std::memcpy(c->h_pidx_pinned, c->pidx.data(), sizeof(uint32_t) * c->pidx.size());
     CK(cudaMemcpyAsync(c->d_pte, c->h_pte_pinned, sizeof(Pte) * c->E, cudaMemcpyHostToDevice,
                        c->stream));
-    if (!c->pidx.empty())
-        CK(cudaMemcpyAsync(c->d_pidx, c->h_pidx_pinned, sizeof(uint32_t) * c->pidx.size(),
+    if (n)
+        CK(cudaMemcpyAsync(c->d_pidx, c->h_pidx_pinned, sizeof(uint32_t) * n,
                            cudaMemcpyHostToDevice, c->stream));
     CK(cudaEventRecord(c->upload_done, c->stream));
     return MPE_OK;
@@ -129,11 +146,11 @@ int upload_table(mpe_ctx* c) {
 
 int upload_list(mpe_ctx* c, const std::vector<int>& list) {
     // the list staging is shared with the previous call: wait for its upload
-    CK(cudaEventSynchronize(c->upload_done));
+    CK(cudaEventSynchronize(c->list_done));
     for (size_t i = 0; i < list.size(); ++i) c->h_list_pinned[i] = list[i];
     CK(cudaMemcpyAsync(c->d_list, c->h_list_pinned, sizeof(int32_t) * list.size(),
                        cudaMemcpyHostToDevice, c->stream));
-    CK(cudaEventRecord(c->upload_done, c->stream));
+    CK(cudaEventRecord(c->list_done, c->stream));
     return MPE_OK;
 }
 
@@ -202,17 +219,18 @@ int ensure_stage(mpe_ctx* c, int T, int k) {
     return MPE_OK;
 }
 
-// Run the allocator kernel on the context's stream and fetch the widths.
+// Run the allocator kernel on the context's stream and fetch the widths
+// (pinned staging; the expert sizes are uploaded once).
 int run_allocate(mpe_ctx* c, const double* p, uint64_t B, std::vector<uint8_t>& out) {
     const int E = c->E;
     for (int e = 0; e < E; ++e)
         if (!(p[e] >= 0.0) || !std::isfinite(p[e]))
             return fail(c, MPE_ERR_INVALID, "importance p[%d] must be finite and >= 0", e);
-    std::vector<uint64_t> W(E, (uint64_t)3 * c->H * c->F);
-    const uint64_t sum_w = W[0] * E;
+    const uint64_t w_e = (uint64_t)3 * c->H * c->F;
+    const uint64_t sum_w = w_e * E;
     if (B < 3 * sum_w) return fail(c, MPE_ERR_INFEASIBLE, "budget %llu < 3 * sum W = %llu",
                                    (unsigned long long)B, (unsigned long long)(3 * sum_w));
-    const uint64_t g = W[0];
+    const uint64_t g = w_e;
     uint64_t R = B >= 8 * sum_w ? 0 : (B - 3 * sum_w) / g;
     R = std::min<uint64_t>(R, 5 * (sum_w / g));
     if (R + 1 > MPE_ALLOC_STATE_CAP) return fail(c, MPE_ERR_STATE_CAP, "too many states");
@@ -222,21 +240,30 @@ int run_allocate(mpe_ctx* c, const double* p, uint64_t B, std::vector<uint8_t>& 
         CK(cudaMalloc(&c->d_choice, need));
         c->choice_cap = need;
     }
-    CK(cudaMemcpyAsync(c->d_p, p, sizeof(double) * E, cudaMemcpyHostToDevice, c->stream));
-    CK(cudaMemcpyAsync(c->d_W, W.data(), sizeof(uint64_t) * E, cudaMemcpyHostToDevice,
+    if (!c->w_uploaded) {
+        for (int e = 0; e < E; ++e) c->h_w_pinned[e] = w_e;
+        CK(cudaMemcpyAsync(c->d_W, c->h_w_pinned, sizeof(uint64_t) * E, cudaMemcpyHostToDevice,
+                           c->stream));
+        c->w_uploaded = true;
+    }
+    // the staging is free: the previous call ended with a synchronize
+    std::memcpy(c->h_p_pinned, p, sizeof(double) * E);
+    CK(cudaMemcpyAsync(c->d_p, c->h_p_pinned, sizeof(double) * E, cudaMemcpyHostToDevice,
                        c->stream));
     launch_allocate(c->stream, c->d_p, c->d_W, E, B, c->d_bits_out, c->d_alloc_status,
                     c->d_choice, c->d_D, MPE_ALLOC_STATE_CAP, R);
     c->launches++;
     CKLAUNCH();
-    int32_t st = -1;
-    out.assign(E, 0);
-    CK(cudaMemcpyAsync(&st, c->d_alloc_status, sizeof(int32_t), cudaMemcpyDeviceToHost,
+    CK(cudaMemcpyAsync(c->h_alloc_pinned, c->d_alloc_status, sizeof(int32_t),
+                       cudaMemcpyDeviceToHost, c->stream));
+    CK(cudaMemcpyAsync(c->h_alloc_pinned + 1, c->d_bits_out, E, cudaMemcpyDeviceToHost,
                        c->stream));
-    CK(cudaMemcpyAsync(out.data(), c->d_bits_out, E, cudaMemcpyDeviceToHost, c->stream));
     CK(cudaStreamSynchronize(c->stream));
+    const int32_t st = c->h_alloc_pinned[0];
     if (st == 1) return fail(c, MPE_ERR_INFEASIBLE, "budget below 3 bits per weight");
     if (st == 3) return fail(c, MPE_ERR_STATE_CAP, "too many allocation states");
+    const uint8_t* bits = reinterpret_cast<const uint8_t*>(c->h_alloc_pinned + 1);
+    out.assign(bits, bits + E);
     return MPE_OK;
 }
 
@@ -309,11 +336,16 @@ int mpe_create(mpe_ctx** out, const mpe_config* cfg) {
         cudaMallocHost(&c->h_pidx_pinned, sizeof(uint32_t) * c->pool_pages) != cudaSuccess ||
         cudaMallocHost(&c->h_list_pinned, sizeof(int32_t) * c->E) != cudaSuccess ||
         cudaMallocHost(&c->h_masters_pinned, sizeof(void*) * c->E) != cudaSuccess ||
-        cudaEventCreateWithFlags(&c->upload_done, cudaEventDisableTiming) != cudaSuccess)
+        cudaMallocHost(&c->h_p_pinned, sizeof(double) * c->E) != cudaSuccess ||
+        cudaMallocHost(&c->h_w_pinned, sizeof(uint64_t) * c->E) != cudaSuccess ||
+        cudaMallocHost(&c->h_alloc_pinned, sizeof(int32_t) * (1 + (c->E + 3) / 4)) != cudaSuccess ||
+        cudaEventCreateWithFlags(&c->upload_done, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&c->list_done, cudaEventDisableTiming) != cudaSuccess)
         return bail(fail_global(MPE_ERR_CUDA, "host staging allocation failed"));
     if (cudaMemset(c->d_pte, 0, sizeof(Pte) * c->E) != cudaSuccess ||
         cudaMemset(c->d_status, 0, sizeof(uint32_t)) != cudaSuccess ||
-        cudaEventRecord(c->upload_done, c->stream) != cudaSuccess)
+        cudaEventRecord(c->upload_done, c->stream) != cudaSuccess ||
+        cudaEventRecord(c->list_done, c->stream) != cudaSuccess)
         return bail(fail_global(MPE_ERR_CUDA, "initialisation failed"));
     c->bits.assign(c->E, 0);
     c->pte.assign(c->E, Pte{});
@@ -341,7 +373,9 @@ void mpe_destroy(mpe_ctx* c) {
         cudaFree(c->d_choice); cudaFree(c->d_D); cudaFree(c->d_gather);
         cudaFreeHost(c->h_pte_pinned); cudaFreeHost(c->h_pidx_pinned);
         cudaFreeHost(c->h_list_pinned); cudaFreeHost(c->h_masters_pinned);
+        cudaFreeHost(c->h_p_pinned); cudaFreeHost(c->h_w_pinned); cudaFreeHost(c->h_alloc_pinned);
         if (c->upload_done) cudaEventDestroy(c->upload_done);
+        if (c->list_done) cudaEventDestroy(c->list_done);
         for (const ProfileRecord& r : c->prof) {
             cudaEventDestroy(r.start);
             cudaEventDestroy(r.stop);
@@ -418,11 +452,10 @@ int mpe_quantize_experts(mpe_ctx* c, const void* const* master_f16, const uint8_
     }
     DeviceGuard guard(c->device);
     std::vector<uint8_t> nb(bits, bits + c->E);
-    HostAllocator na;
+    PagePlan plan;
     std::vector<int> changed;
-    if (!plan_pages(c, nb, na, changed)) return fail(c, MPE_ERR_POOL, "page pool exhausted");
-    c->alloc = std::move(na);
-    c->bits = nb;
+    if (!plan_pages(c, nb, plan, changed)) return fail(c, MPE_ERR_POOL, "page pool exhausted");
+    commit_pages(c, plan, nb);
     int r;
     if ((r = upload_table(c))) return r;
     // master pointers and the all-experts list
@@ -453,11 +486,10 @@ int mpe_repage(mpe_ctx* c, uint64_t B_bits, const double* p, int32_t* n_changed_
     std::vector<uint8_t> nb;
     int r;
     if ((r = run_allocate(c, p, B_bits, nb))) return r;
-    HostAllocator na;
+    PagePlan plan;
     std::vector<int> changed;
-    if (!plan_pages(c, nb, na, changed)) return fail(c, MPE_ERR_POOL, "page pool exhausted");
-    c->alloc = std::move(na);
-    c->bits = nb;
+    if (!plan_pages(c, nb, plan, changed)) return fail(c, MPE_ERR_POOL, "page pool exhausted");
+    commit_pages(c, plan, nb);
     if ((r = upload_table(c))) return r;
     launch_scales(c);
     if (!changed.empty()) {
@@ -660,9 +692,10 @@ int mpe_get_page_table(mpe_ctx* c, mpe_pte* pte_host, uint32_t* page_idx_host, s
     CK(cudaStreamSynchronize(c->stream));
     if (pte_host) CK(cudaMemcpy(pte_host, c->d_pte, sizeof(Pte) * c->E, cudaMemcpyDeviceToHost));
     if (page_idx_host) {
-        if (cap < c->pidx.size()) return fail(c, MPE_ERR_INVALID, "cap %zu < %zu", cap, c->pidx.size());
-        if (!c->pidx.empty())
-            CK(cudaMemcpy(page_idx_host, c->d_pidx, sizeof(uint32_t) * c->pidx.size(),
+        if (cap < c->pidx_count)
+            return fail(c, MPE_ERR_INVALID, "cap %zu < %u", cap, (unsigned)c->pidx_count);
+        if (c->pidx_count)
+            CK(cudaMemcpy(page_idx_host, c->d_pidx, sizeof(uint32_t) * c->pidx_count,
                           cudaMemcpyDeviceToHost));
     }
     return MPE_OK;

@@ -47,37 +47,51 @@ k_combine_by_position(const float* y, const int32_t* inv, const float* w, int T,
     const int i = blockIdx.y * blockDim.x + threadIdx.x;  // float4 column index
     if (i >= H / 4) return;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j = 0; j < k; ++j) {
-        const int pos = inv[t * k + j];
-        if (pos < 0) continue;
-        const float wj = w[t * k + j];
-        const float4* src = reinterpret_cast<const float4*>(y + (size_t)pos * H) + i;
-        float4 v = src[0];
-        int p = 1;
-        // parts in order; four independent loads in flight per step
-        for (; p + 4 <= parts; p += 4) {
-            float4 u[4];
+    if (parts == 1) {
+        // a plain loop: the slots' loads are independent and issue together
+        for (int j = 0; j < k; ++j) {
+            const int pos = inv[t * k + j];
+            if (pos < 0) continue;
+            const float wj = w[t * k + j];
+            const float4 v = reinterpret_cast<const float4*>(y + (size_t)pos * H)[i];
+            acc.x = fmaf(wj, v.x, acc.x);
+            acc.y = fmaf(wj, v.y, acc.y);
+            acc.z = fmaf(wj, v.z, acc.z);
+            acc.w = fmaf(wj, v.w, acc.w);
+        }
+    } else {
+        for (int j = 0; j < k; ++j) {
+            const int pos = inv[t * k + j];
+            if (pos < 0) continue;
+            const float wj = w[t * k + j];
+            const float4* src = reinterpret_cast<const float4*>(y + (size_t)pos * H) + i;
+            float4 v = src[0];
+            int p = 1;
+            // parts in order; four independent loads in flight per step
+            for (; p + 4 <= parts; p += 4) {
+                float4 u[4];
 #pragma unroll
-            for (int r = 0; r < 4; ++r) u[r] = src[(p + r) * (part_stride / 4)];
+                for (int r = 0; r < 4; ++r) u[r] = src[(p + r) * (part_stride / 4)];
 #pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                v.x += u[r].x;
-                v.y += u[r].y;
-                v.z += u[r].z;
-                v.w += u[r].w;
+                for (int r = 0; r < 4; ++r) {
+                    v.x += u[r].x;
+                    v.y += u[r].y;
+                    v.z += u[r].z;
+                    v.w += u[r].w;
+                }
             }
+            for (; p < parts; ++p) {
+                const float4 u = src[p * (part_stride / 4)];
+                v.x += u.x;
+                v.y += u.y;
+                v.z += u.z;
+                v.w += u.w;
+            }
+            acc.x = fmaf(wj, v.x, acc.x);
+            acc.y = fmaf(wj, v.y, acc.y);
+            acc.z = fmaf(wj, v.z, acc.z);
+            acc.w = fmaf(wj, v.w, acc.w);
         }
-        for (; p < parts; ++p) {
-            const float4 u = src[p * (part_stride / 4)];
-            v.x += u.x;
-            v.y += u.y;
-            v.z += u.z;
-            v.w += u.w;
-        }
-        acc.x = fmaf(wj, v.x, acc.x);
-        acc.y = fmaf(wj, v.y, acc.y);
-        acc.z = fmaf(wj, v.z, acc.z);
-        acc.w = fmaf(wj, v.w, acc.w);
     }
     __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
     __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);

@@ -91,12 +91,17 @@ struct mpe_ctx {
     std::vector<const void*> masters;
     std::vector<uint8_t> bits;
     std::vector<mpe::Pte> pte;
-    std::vector<uint32_t> pidx;
+    uint32_t pidx_count = 0;                // entries of the page-index array in use
     mpe::Pte* h_pte_pinned = nullptr;       // upload staging (pinned)
     uint32_t* h_pidx_pinned = nullptr;
     int32_t* h_list_pinned = nullptr;
     const void** h_masters_pinned = nullptr;
-    cudaEvent_t upload_done = nullptr;
+    double* h_p_pinned = nullptr;           // allocator staging: importances in,
+    uint64_t* h_w_pinned = nullptr;         // expert sizes (uploaded once),
+    int32_t* h_alloc_pinned = nullptr;      // status word + widths out
+    bool w_uploaded = false;
+    cudaEvent_t upload_done = nullptr;      // page-table staging free again
+    cudaEvent_t list_done = nullptr;        // expert-list staging free again
     bool absmax_valid = false;
     mpe::HostAllocator alloc;
     mpe::Scratch s;

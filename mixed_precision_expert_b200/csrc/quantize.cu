@@ -4,8 +4,9 @@
 //   Q(w) = round(w / s) * s,  s = max|w| / (2^(b-1) - 1),  one s per expert.
 // Here: m_e = max |w| over the expert's fp16 master (exact integer max of the
 // magnitude bits), s_e = RN_f32(m_e / q_b), k = round-half-even of the exact
-// quotient w / s_e, clamped to [-q_b, q_b], stored offset-binary in the packed
-// chunk format (common.cuh) inside the expert's pages.
+// quotient w / s_e (it lies in [-q_b, q_b], so the clamp is a no-op; see
+// round_bits), stored offset-binary in the packed chunk format (common.cuh)
+// inside the expert's pages.
 #include "internal.h"
 
 namespace mpe {
@@ -69,7 +70,7 @@ __global__ void k_scales(Pte* pte, const uint32_t* absmax, int E, uint32_t* stat
     pte[e].scale = (m == 0) ? 0.0f : __fdiv_rn(mf, (float)q_levels(b));
 }
 
-// Rare path of encode_one: r lies within 2^-11 of a half-integer, so the exact
+// Rare path of round_bits: r lies within 2^-11 of a half-integer, so the exact
 // quotient w / s decides. The sign of the single-rounded fma (k -+ 1/2) s - w is
 // exact: ties go to the even integer.
 __device__ __noinline__ float tie_fix(float w, float s, float kf) {
@@ -83,20 +84,27 @@ __device__ __noinline__ float tie_fix(float w, float s, float kf) {
     return kf;
 }
 
-// k = round-half-even(w / s), exactly, clamped; returns offset-binary u = k + 2^(b-1).
-// r = w * (1/s) is within ~2^-16 of the exact quotient (|w/s| < 2^8). Adding
-// 1.5 * 2^23 rounds r to an integer, ties to even, and leaves that integer in
-// the low mantissa bits, so k is read out with integer operations (no
-// conversion instruction). Rounding r agrees with rounding the exact quotient
-// unless r lies within 2^-11 of a half-integer, which tie_fix settles.
-__device__ __forceinline__ uint32_t encode_one(float w, float s, float inv_s, int q, int off) {
+// Rounding of one weight. r = w * (1/s) is within ~2^-16 of the exact
+// quotient (|w/s| < 2^8). Adding 1.5 * 2^23 rounds r to an integer, ties to
+// even, and leaves that integer k in the low mantissa bits: the returned bit
+// pattern is 0x4B400000 + k, which the packing below turns into k + 2^(b-1)
+// without extracting k first. Rounding r agrees with rounding the exact
+// quotient unless r lies within 2^-11 of a half-integer; then tie_fix settles
+// the exact code and the pattern moves by its difference from k.
+//
+// No clamp is needed: |w| <= max|w| = m and s = RN(m / q) give
+// |r| <= q (1 + 3 * 2^-24) < q + 1/2, so k lies in [-q, q] (the exact tie
+// repair never leaves that range either). This holds because the master is
+// immutable after quantize_experts (its absmax is cached).
+__device__ __forceinline__ uint32_t round_bits(float w, float s, float inv_s) {
     constexpr float kRound = 12582912.0f;  // 1.5 * 2^23, bits 0x4B400000
     const float r = __fmul_rn(w, inv_s);
     const float rf = __fadd_rn(r, kRound);
-    int k = __float_as_int(rf) - 0x4B400000;
-    if (fabsf(__fsub_rn(r, __fsub_rn(rf, kRound))) > 0.4990234375f)
-        k = (int)tie_fix(w, s, (float)k);
-    return (uint32_t)(min(max(k, -q), q) + off);
+    const float kf = __fsub_rn(rf, kRound);
+    uint32_t bits = __float_as_uint(rf);
+    if (fabsf(__fsub_rn(r, kf)) > 0.4990234375f)
+        bits += (uint32_t)((int)tie_fix(w, s, kf) - (int)kf);
+    return bits;
 }
 
 __device__ __forceinline__ void load32_half(const __half* src, float (&f)[32]) {
@@ -115,43 +123,55 @@ __device__ __forceinline__ void load32_half(const __half* src, float (&f)[32]) {
     }
 }
 
+// Bit position of code c'_i of a quarter inside its word (widths 4 and 8;
+// width 3 below): fields pair up in the two 16-bit halves.
+template <int B>
+__host__ __device__ constexpr int field_shift(int i) {
+    return B == 8 ? 16 * (i & 1) + 8 * ((i & 3) >> 1) : 16 * (i & 1) + 4 * ((i & 7) >> 1);
+}
+
 // Encode one quarter (32 consecutive weights of a row) and store its b words.
+// A word is sum_i (k_i + 2^(b-1)) << sh_i over its fields, i.e. (mod 2^32)
+// sum_i bits_i << sh_i plus the constant sum_i (2^(b-1) - 0x4B400000) << sh_i,
+// with bits_i = 0x4B400000 + k_i from round_bits: one multiply-add a code.
 template <int B>
 __device__ __forceinline__ void encode_quarter(const __half* src, float s, float inv_s,
                                                uint8_t* dst) {
-    constexpr int q = q_levels(B);
-    constexpr int off = 1 << (B - 1);
+    constexpr uint32_t off = 1u << (B - 1);
+    constexpr uint32_t bias = off - 0x4B400000u;  // mod 2^32
     float f[32];
     load32_half(src, f);
-    uint32_t u[32];
+    if constexpr (B == 8 || B == 4) {
+        constexpr int PER = 32 / B;  // codes per word
+        uint32_t wv[B];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) u[i] = encode_one(f[i], s, inv_s, q, off);
-    if constexpr (B == 8) {
-        uint32_t wv[8];
-#pragma unroll
-        for (int w = 0; w < 8; ++w)
-            wv[w] = u[4 * w] + (u[4 * w + 1] << 16) + (u[4 * w + 2] << 8) + (u[4 * w + 3] << 24);
-        reinterpret_cast<uint4*>(dst)[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-        reinterpret_cast<uint4*>(dst)[1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
-    } else if constexpr (B == 4) {
-        uint32_t wv[4];
-#pragma unroll
-        for (int w = 0; w < 4; ++w) {
+        for (int w = 0; w < B; ++w) {
             uint32_t x = 0;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) x += u[8 * w + i] << (16 * (i & 1) + 4 * (i >> 1));
+            for (int i = 0; i < PER; ++i) x += bias << field_shift<B>(i);
+#pragma unroll
+            for (int i = 0; i < PER; ++i) x += round_bits(f[PER * w + i], s, inv_s) << field_shift<B>(i);
             wv[w] = x;
         }
         reinterpret_cast<uint4*>(dst)[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+        if constexpr (B == 8)
+            reinterpret_cast<uint4*>(dst)[1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
     } else {
+        // word v holds c'_{10v+i} at bit 16(i&1) + 3(i>>1) (i < 10); bit v of
+        // c'_30 / c'_31 is bit 15 / 31 of word v
+        const uint32_t u30 = round_bits(f[30], s, inv_s) + bias;  // k_30 + 4
+        const uint32_t u31 = round_bits(f[31], s, inv_s) + bias;
         uint32_t* d32 = reinterpret_cast<uint32_t*>(dst);
 #pragma unroll
         for (int v = 0; v < 3; ++v) {
             uint32_t x = 0;
 #pragma unroll
-            for (int i = 0; i < 10; ++i) x += u[10 * v + i] << (16 * (i & 1) + 3 * (i >> 1));
-            x += ((u[30] >> v) & 1u) << 15;
-            x += ((u[31] >> v) & 1u) << 31;
+            for (int i = 0; i < 10; ++i) x += bias << (16 * (i & 1) + 3 * (i >> 1));
+#pragma unroll
+            for (int i = 0; i < 10; ++i)
+                x += round_bits(f[10 * v + i], s, inv_s) << (16 * (i & 1) + 3 * (i >> 1));
+            x += ((u30 >> v) & 1u) << 15;
+            x += ((u31 >> v) & 1u) << 31;
             d32[v] = x;
         }
     }
