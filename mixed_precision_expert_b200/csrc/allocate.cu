@@ -20,69 +20,47 @@ namespace {
 
 __device__ __forceinline__ double dinf() { return __longlong_as_double(0x7FF0000000000000ll); }
 
-__device__ uint64_t gcd_u64(uint64_t a, uint64_t b) {
-    while (b) {
-        const uint64_t t = a % b;
-        a = b;
-        b = t;
-    }
-    return a;
-}
-
-constexpr int kThreads = 1024;
+constexpr int kThreads = 256;
 // Dynamic shared memory for the two DP rows and the choice table (see below).
 constexpr size_t kAllocSmemMax = 200 * 1024;
 
 // Choices are 2-bit codes (0: 3 bits, 1: 4 bits, 2: 8 bits), four budget
-// states per byte; each thread evaluates one state per pass and the first
-// lane of every four writes their byte. When both DP rows and the table fit in shared memory
-// (R <= smem_R; -1 = no on-chip buffers) the whole solve stays on chip -- every expert step is a
-// shared-memory pass plus one barrier, and the serial backtrack reads shared
-// memory -- else rows and table live in the global buffers D and choice.
+// states per byte; a thread evaluates the four states of one byte per pass
+// (independent chains) and writes the byte. ON_CHIP: both DP rows and the
+// table live in shared memory, so every expert step is a shared-memory pass
+// plus one barrier and the serial backtrack reads shared memory; otherwise
+// they live in the global buffers D and choice. The host supplies sum W and
+// g = gcd(W) (no serial 64-bit arithmetic on the device).
+template <bool ON_CHIP>
 __global__ void __launch_bounds__(kThreads)
-k_allocate(const double* p, const uint64_t* W, int E, uint64_t B, uint8_t* bits,
-           int32_t* status, uint8_t* choice, double* D, int state_cap, int64_t smem_R) {
+k_allocate(const double* p, const uint64_t* W, int E, uint64_t B, uint64_t sum_w, uint64_t g,
+           uint8_t* bits, int32_t* status, uint8_t* choice, double* D, int state_cap) {
     extern __shared__ __align__(16) uint8_t dyn[];
-    __shared__ int s_mode;      // 0 = solve, 1 = infeasible, 2 = all 8, 3 = state cap
-    __shared__ uint32_t s_R;
-    __shared__ uint64_t s_g;
     __shared__ uint32_t s_up4[MPE_MAX_EXPERTS];
     __shared__ uint32_t s_up8[MPE_MAX_EXPERTS];
     __shared__ double s_p[MPE_MAX_EXPERTS];
+    __shared__ double s_rv[kThreads / 32];
+    __shared__ uint32_t s_ri[kThreads / 32];
     const int tid = threadIdx.x;
-    if (tid == 0) {
-        uint64_t sum_w = 0, g = 0;
-        for (int e = 0; e < E; ++e) {
-            sum_w += W[e];
-            g = gcd_u64(g, W[e]);
-        }
-        s_g = g;
-        if (B < 3 * sum_w) {
-            s_mode = 1;
-        } else if (B >= 8 * sum_w) {
-            s_mode = 2;
-        } else {
-            uint64_t R = (B - 3 * sum_w) / g;
-            const uint64_t rmax = 5 * (sum_w / g);
-            if (R > rmax) R = rmax;
-            if (R + 1 > (uint64_t)state_cap) {
-                s_mode = 3;
-            } else {
-                s_mode = 0;
-                s_R = (uint32_t)R;
-            }
-        }
-        *status = s_mode;
+    int mode;  // 0 = solve, 1 = infeasible, 2 = all 8, 3 = state cap
+    uint64_t R64 = 0;
+    if (B < 3 * sum_w) {
+        mode = 1;
+    } else if (B >= 8 * sum_w) {
+        mode = 2;
+    } else {
+        R64 = (B - 3 * sum_w) / g;
+        const uint64_t rmax = 5 * (sum_w / g);
+        if (R64 > rmax) R64 = rmax;
+        mode = (R64 + 1 > (uint64_t)state_cap) ? 3 : 0;
     }
-    __syncthreads();
-    const int mode = s_mode;
+    if (tid == 0) *status = mode;
     if (mode == 2) {
         for (int e = tid; e < E; e += kThreads) bits[e] = 8;
         return;
     }
     if (mode != 0) return;
-    const uint32_t R = s_R;
-    const uint64_t g = s_g;
+    const uint32_t R = (uint32_t)R64;
     const uint32_t nq = (R + 4) / 4;  // choice bytes per expert
     for (int e = tid; e < E; e += kThreads) {
         const uint64_t u4 = W[e] / g, u8 = 5 * (W[e] / g);
@@ -90,10 +68,9 @@ k_allocate(const double* p, const uint64_t* W, int E, uint64_t B, uint8_t* bits,
         s_up8[e] = (uint32_t)min(u8, (uint64_t)R + 1);
         s_p[e] = p[e];
     }
-    const bool on_chip = (int64_t)R <= smem_R;
-    double* Dcur = on_chip ? reinterpret_cast<double*>(dyn) : D;
+    double* Dcur = ON_CHIP ? reinterpret_cast<double*>(dyn) : D;
     double* Dnext = Dcur + (R + 1);
-    uint8_t* chb = on_chip ? dyn + 16 * (size_t)(R + 1) : choice;
+    uint8_t* chb = ON_CHIP ? dyn + 16 * (size_t)(R + 1) : choice;
     const double L3 = __ddiv_rn(1.0, 9.0);
     const double L4 = __ddiv_rn(1.0, 49.0);
     const double L8 = __ddiv_rn(1.0, 16129.0);
@@ -106,38 +83,52 @@ k_allocate(const double* p, const uint64_t* W, int E, uint64_t B, uint8_t* bits,
         const double c8 = __dmul_rn(pe, L8);
         const uint32_t u4 = s_up4[e], u8 = s_up8[e];
         uint8_t* ch = chb + (size_t)e * nq;
-        // one state a thread; the loop bound is the same for every thread (the
-        // code packing below shuffles across the warp)
-        for (uint32_t base = 0; base <= R; base += kThreads) {
-            const uint32_t r = base + tid;
-            uint32_t code = 0;
-            if (r <= R) {
+        for (uint32_t qd = tid; qd < nq; qd += kThreads) {
+            uint32_t byte = 0;
+#pragma unroll
+            for (uint32_t i = 0; i < 4; ++i) {
+                const uint32_t r = 4 * qd + i;
                 // an unreachable predecessor is +inf and its candidate stays +inf
-                const double x3 = __dadd_rn(Dcur[r], c3);
-                const double x4 = r >= u4 ? __dadd_rn(Dcur[r - u4], c4) : dinf();
-                const double x8 = r >= u8 ? __dadd_rn(Dcur[r - u8], c8) : dinf();
+                const double x3 = r <= R ? __dadd_rn(Dcur[r], c3) : dinf();
+                const double x4 = (r <= R && r >= u4) ? __dadd_rn(Dcur[r - u4], c4) : dinf();
+                const double x8 = (r <= R && r >= u8) ? __dadd_rn(Dcur[r - u8], c8) : dinf();
                 double best = dinf();
+                uint32_t code = 0;
                 if (x3 < best) best = x3;
                 if (x4 < best) { best = x4; code = 1; }
                 if (x8 < best) { best = x8; code = 2; }
-                Dnext[r] = best;
+                if (r <= R) Dnext[r] = best;
+                byte |= code << (2 * i);
             }
-            // lanes 4m .. 4m+3 hold states 4m' .. 4m'+3: one byte of codes
-            const uint32_t k1 = __shfl_down_sync(0xffffffffu, code, 1);
-            const uint32_t k2 = __shfl_down_sync(0xffffffffu, code, 2);
-            const uint32_t k3 = __shfl_down_sync(0xffffffffu, code, 3);
-            if ((tid & 3) == 0 && r <= R) ch[r >> 2] = (uint8_t)(code | k1 << 2 | k2 << 4 | k3 << 6);
+            ch[qd] = (uint8_t)byte;
         }
         __syncthreads();
         double* t = Dcur;
         Dcur = Dnext;
         Dnext = t;
     }
+    // argmin over the budget states, ties to the smallest state
+    double bv = dinf();
+    uint32_t bi = 0xFFFFFFFFu;
+    for (uint32_t r = tid; r <= R; r += kThreads)
+        if (Dcur[r] < bv) { bv = Dcur[r]; bi = r; }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const double ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const uint32_t oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (ov < bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+    }
+    if ((tid & 31) == 0) {
+        s_rv[tid >> 5] = bv;
+        s_ri[tid >> 5] = bi;
+    }
+    __syncthreads();
     if (tid == 0) {
-        uint32_t rb = 0;
-        for (uint32_t r = 1; r <= R; ++r)
-            if (Dcur[r] < Dcur[rb]) rb = r;
-        uint32_t r = rb;
+        bv = s_rv[0];
+        bi = s_ri[0];
+        for (int w = 1; w < kThreads / 32; ++w)
+            if (s_rv[w] < bv || (s_rv[w] == bv && s_ri[w] < bi)) { bv = s_rv[w]; bi = s_ri[w]; }
+        uint32_t r = bi;
         for (int e = E - 1; e >= 0; --e) {
             const uint32_t code = (chb[(size_t)e * nq + r / 4] >> (2 * (r % 4))) & 3u;
             bits[e] = code == 0 ? 3 : (code == 1 ? 4 : 8);
@@ -151,17 +142,22 @@ k_allocate(const double* p, const uint64_t* W, int E, uint64_t B, uint8_t* bits,
 size_t allocate_choice_bytes(int E, uint64_t R) { return (size_t)E * (size_t)((R + 4) / 4); }
 
 void launch_allocate(cudaStream_t st, const double* p, const uint64_t* W, int E, uint64_t B,
-                     uint8_t* bits_out, int32_t* status, uint8_t* choice, double* D,
-                     int state_cap, uint64_t R) {
+                     uint64_t sum_w, uint64_t g, uint8_t* bits_out, int32_t* status,
+                     uint8_t* choice, double* D, int state_cap, uint64_t R) {
     // R is the host's count of budget units (same formula as the kernel's);
     // it only sizes the on-chip buffers
     const size_t smem = 16 * (size_t)(R + 1) + allocate_choice_bytes(E, R);
-    const bool on_chip = smem <= kAllocSmemMax;
-    // the attribute is per device: set it on every launch that needs it
-    if (on_chip && smem > 48 * 1024)
-        cudaFuncSetAttribute(k_allocate, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    k_allocate<<<1, kThreads, on_chip ? smem : 0, st>>>(p, W, E, B, bits_out, status, choice, D,
-                                                        state_cap, on_chip ? (int64_t)R : -1);
+    if (smem <= kAllocSmemMax) {
+        // the attribute is per device: set it on every launch that needs it
+        if (smem > 48 * 1024)
+            cudaFuncSetAttribute(k_allocate<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem);
+        k_allocate<true><<<1, kThreads, smem, st>>>(p, W, E, B, sum_w, g, bits_out, status, choice,
+                                                    D, state_cap);
+    } else {
+        k_allocate<false><<<1, kThreads, 0, st>>>(p, W, E, B, sum_w, g, bits_out, status, choice,
+                                                  D, state_cap);
+    }
 }
 
 }  // namespace mpe

@@ -250,8 +250,8 @@ int run_allocate(mpe_ctx* c, const double* p, uint64_t B, std::vector<uint8_t>& 
     std::memcpy(c->h_p_pinned, p, sizeof(double) * E);
     CK(cudaMemcpyAsync(c->d_p, c->h_p_pinned, sizeof(double) * E, cudaMemcpyHostToDevice,
                        c->stream));
-    launch_allocate(c->stream, c->d_p, c->d_W, E, B, c->d_bits_out, c->d_alloc_status,
-                    c->d_choice, c->d_D, MPE_ALLOC_STATE_CAP, R);
+    launch_allocate(c->stream, c->d_p, c->d_W, E, B, sum_w, g, c->d_bits_out,
+                    c->d_alloc_status, c->d_choice, c->d_D, MPE_ALLOC_STATE_CAP, R);
     c->launches++;
     CKLAUNCH();
     CK(cudaMemcpyAsync(c->h_alloc_pinned, c->d_alloc_status, sizeof(int32_t),
@@ -428,7 +428,8 @@ int mpe_allocate_bits(const double* p, const uint64_t* W, int32_t E, uint64_t B_
         !ok(cudaMemcpy(dW, W, sizeof(uint64_t) * E, cudaMemcpyHostToDevice))) {
         rc = fail_global(MPE_ERR_CUDA, "allocate_bits: %s", cudaGetErrorString(cudaGetLastError()));
     } else {
-        launch_allocate(nullptr, dp, dW, E, B_bits, db, ds, dch, dD, MPE_ALLOC_STATE_CAP, R);
+        launch_allocate(nullptr, dp, dW, E, B_bits, sum_w, g, db, ds, dch, dD, MPE_ALLOC_STATE_CAP,
+                        R);
         if (!ok(cudaGetLastError()) || !ok(cudaMemcpy(&st, ds, sizeof(int32_t), cudaMemcpyDeviceToHost)) ||
             !ok(cudaMemcpy(bits_out, db, E, cudaMemcpyDeviceToHost)))
             rc = fail_global(MPE_ERR_CUDA, "allocate_bits kernel: %s",

@@ -142,9 +142,11 @@ void launch_encode(mpe_ctx* c, const int32_t* d_list, int n_list);
 void launch_gather_stream(mpe_ctx* c, int e, uint8_t* dst);
 
 // allocate.cu
+// sum_w = sum of W, g = gcd(W) (host-computed); R = budget units (sizes the
+// on-chip buffers)
 void launch_allocate(cudaStream_t st, const double* p, const uint64_t* W, int E, uint64_t B,
-                     uint8_t* bits_out, int32_t* status, uint8_t* choice, double* D,
-                     int state_cap, uint64_t R);
+                     uint64_t sum_w, uint64_t g, uint8_t* bits_out, int32_t* status,
+                     uint8_t* choice, double* D, int state_cap, uint64_t R);
 // bytes of the global choice table for E experts and R budget units
 size_t allocate_choice_bytes(int E, uint64_t R);
 
