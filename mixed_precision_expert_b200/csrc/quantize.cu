@@ -107,20 +107,16 @@ __device__ __forceinline__ uint32_t round_bits(float w, float s, float inv_s) {
     return bits;
 }
 
-__device__ __forceinline__ void load32_half(const __half* src, float (&f)[32]) {
-    const uint4* p = reinterpret_cast<const uint4*>(src);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const uint4 v = __ldcs(p + i);
-        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const __half2 h2 = *reinterpret_cast<const __half2*>(&wv[j]);
-            const float2 ff = __half22float2(h2);
-            f[8 * i + 2 * j] = ff.x;
-            f[8 * i + 2 * j + 1] = ff.y;
-        }
-    }
+// Weights 2i, 2i+1 of a quarter's raw fp16 data (four 16-byte vectors).
+__device__ __forceinline__ float2 raw_pair(const uint4 (&raw)[4], int i) {
+    const uint4 v = raw[i >> 2];
+    const uint32_t x = (i & 3) == 0 ? v.x : (i & 3) == 1 ? v.y : (i & 3) == 2 ? v.z : v.w;
+    return __half22float2(*reinterpret_cast<const __half2*>(&x));
+}
+
+__device__ __forceinline__ float raw_weight(const uint4 (&raw)[4], int c) {
+    const float2 f = raw_pair(raw, c >> 1);
+    return (c & 1) ? f.y : f.x;
 }
 
 // Bit position of code c'_i of a quarter inside its word (widths 4 and 8;
@@ -130,46 +126,62 @@ __host__ __device__ constexpr int field_shift(int i) {
     return B == 8 ? 16 * (i & 1) + 8 * ((i & 3) >> 1) : 16 * (i & 1) + 4 * ((i & 7) >> 1);
 }
 
-// Encode one quarter (32 consecutive weights of a row) and store its b words.
-// A word is sum_i (k_i + 2^(b-1)) << sh_i over its fields, i.e. (mod 2^32)
-// sum_i bits_i << sh_i plus the constant sum_i (2^(b-1) - 0x4B400000) << sh_i,
-// with bits_i = 0x4B400000 + k_i from round_bits: one multiply-add a code.
+// One packed word: codes c0 .. c0+n-1 of the quarter at bit positions sh(i),
+// as sum_i (k_i + 2^(b-1)) << sh(i) = const + sum_i bits_i << sh(i) (mod 2^32),
+// bits_i = 0x4B400000 + k_i the pattern of r_i + 1.5 * 2^23: one multiply-add a
+// code. If any code of the word lies within 2^-11 of a half-integer, the word
+// is recomputed with the exact rounding (round_bits): one branch a word.
+template <int B, int N, typename Shift>
+__device__ __forceinline__ uint32_t encode_word(const uint4 (&raw)[4], int c0, float s,
+                                                float inv_s, Shift sh) {
+    constexpr float kRound = 12582912.0f;  // 1.5 * 2^23, bits 0x4B400000
+    constexpr uint32_t bias = (1u << (B - 1)) - 0x4B400000u;  // mod 2^32
+    uint32_t x = 0;
+#pragma unroll
+    for (int i = 0; i < N; ++i) x += bias << sh(i);
+    const uint32_t x0 = x;
+    bool near = false;
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+        const float r = __fmul_rn(raw_weight(raw, c0 + i), inv_s);
+        const float rf = __fadd_rn(r, kRound);
+        near |= fabsf(__fsub_rn(r, __fsub_rn(rf, kRound))) > 0.4990234375f;
+        x += __float_as_uint(rf) << sh(i);
+    }
+    if (near) {
+        x = x0;
+#pragma unroll
+        for (int i = 0; i < N; ++i) x += round_bits(raw_weight(raw, c0 + i), s, inv_s) << sh(i);
+    }
+    return x;
+}
+
+// Encode one quarter (32 consecutive weights of a row, raw fp16 in registers)
+// and store its b words.
 template <int B>
-__device__ __forceinline__ void encode_quarter(const __half* src, float s, float inv_s,
+__device__ __forceinline__ void encode_quarter(const uint4 (&raw)[4], float s, float inv_s,
                                                uint8_t* dst) {
-    constexpr uint32_t off = 1u << (B - 1);
-    constexpr uint32_t bias = off - 0x4B400000u;  // mod 2^32
-    float f[32];
-    load32_half(src, f);
     if constexpr (B == 8 || B == 4) {
         constexpr int PER = 32 / B;  // codes per word
         uint32_t wv[B];
 #pragma unroll
-        for (int w = 0; w < B; ++w) {
-            uint32_t x = 0;
-#pragma unroll
-            for (int i = 0; i < PER; ++i) x += bias << field_shift<B>(i);
-#pragma unroll
-            for (int i = 0; i < PER; ++i) x += round_bits(f[PER * w + i], s, inv_s) << field_shift<B>(i);
-            wv[w] = x;
-        }
+        for (int w = 0; w < B; ++w)
+            wv[w] = encode_word<B, PER>(raw, PER * w, s, inv_s,
+                                        [](int i) { return field_shift<B>(i); });
         reinterpret_cast<uint4*>(dst)[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
         if constexpr (B == 8)
             reinterpret_cast<uint4*>(dst)[1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
     } else {
         // word v holds c'_{10v+i} at bit 16(i&1) + 3(i>>1) (i < 10); bit v of
         // c'_30 / c'_31 is bit 15 / 31 of word v
-        const uint32_t u30 = round_bits(f[30], s, inv_s) + bias;  // k_30 + 4
-        const uint32_t u31 = round_bits(f[31], s, inv_s) + bias;
+        constexpr uint32_t bias = 4u - 0x4B400000u;
+        const uint32_t u30 = round_bits(raw_weight(raw, 30), s, inv_s) + bias;  // k_30 + 4
+        const uint32_t u31 = round_bits(raw_weight(raw, 31), s, inv_s) + bias;
         uint32_t* d32 = reinterpret_cast<uint32_t*>(dst);
 #pragma unroll
         for (int v = 0; v < 3; ++v) {
-            uint32_t x = 0;
-#pragma unroll
-            for (int i = 0; i < 10; ++i) x += bias << (16 * (i & 1) + 3 * (i >> 1));
-#pragma unroll
-            for (int i = 0; i < 10; ++i)
-                x += round_bits(f[10 * v + i], s, inv_s) << (16 * (i & 1) + 3 * (i >> 1));
+            uint32_t x = encode_word<3, 10>(raw, 10 * v, s, inv_s,
+                                            [](int i) { return 16 * (i & 1) + 3 * (i >> 1); });
             x += ((u30 >> v) & 1u) << 15;
             x += ((u31 >> v) & 1u) << 31;
             d32[v] = x;
@@ -180,7 +192,9 @@ __device__ __forceinline__ void encode_quarter(const __half* src, float s, float
 // One warp per chunk (16 rows x 128 codes). Lane l encodes quarter (l & 3) of
 // rows (l >> 2) and (l >> 2) + 8; quarter index in the chunk is l and l + 32,
 // so the lanes' stores cover the chunk contiguously.
-__global__ void __launch_bounds__(256)
+// 4 CTAs per SM (64 registers): more warps hide the loads better than more
+// registers would
+__global__ void __launch_bounds__(256, 4)
 k_encode(PagedExperts P, const void* const* masters, const int32_t* list) {
     const int e = list[blockIdx.y];
     const Pte pte = P.pte[e];
@@ -208,18 +222,25 @@ k_encode(PagedExperts P, const void* const* masters, const int32_t* list) {
     const __half* r8 = r0 + (size_t)8 * K;
     uint8_t* dst = const_cast<uint8_t*>(chunk_addr(P, pte, b, c));
     const float inv_s = s > 0.0f ? __frcp_rn(s) : 0.0f;
+    // both quarters' weights in flight before any arithmetic
+    uint4 q0[4], q8[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        q0[i] = __ldcs(reinterpret_cast<const uint4*>(r0) + i);
+        q8[i] = __ldcs(reinterpret_cast<const uint4*>(r8) + i);
+    }
     switch (b) {
         case 3:
-            encode_quarter<3>(r0, s, inv_s, dst + 12 * lane);
-            encode_quarter<3>(r8, s, inv_s, dst + 12 * (lane + 32));
+            encode_quarter<3>(q0, s, inv_s, dst + 12 * lane);
+            encode_quarter<3>(q8, s, inv_s, dst + 12 * (lane + 32));
             break;
         case 4:
-            encode_quarter<4>(r0, s, inv_s, dst + 16 * lane);
-            encode_quarter<4>(r8, s, inv_s, dst + 16 * (lane + 32));
+            encode_quarter<4>(q0, s, inv_s, dst + 16 * lane);
+            encode_quarter<4>(q8, s, inv_s, dst + 16 * (lane + 32));
             break;
         case 8:
-            encode_quarter<8>(r0, s, inv_s, dst + 32 * lane);
-            encode_quarter<8>(r8, s, inv_s, dst + 32 * (lane + 32));
+            encode_quarter<8>(q0, s, inv_s, dst + 32 * lane);
+            encode_quarter<8>(q8, s, inv_s, dst + 32 * (lane + 32));
             break;
         default:
             break;
