@@ -43,6 +43,7 @@ __global__ void __launch_bounds__(128)
 k_combine_by_position(const float* y, const int32_t* inv, const float* w, int T, int k, int H,
                       int parts, size_t part_stride, __nv_bfloat16* out) {
     griddep_wait();
+    griddep_launch_dependents();
     const int t = blockIdx.x;
     const int i = blockIdx.y * blockDim.x + threadIdx.x;  // float4 column index
     if (i >= H / 4) return;

@@ -829,14 +829,16 @@ void decode_plan(mpe_ctx* c, size_t Tk, DecodePlan& pl) {
     if (!g_num_sms) cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, c->device);
     const int ctas = g_num_sms;
     const int groups = (int)std::min<size_t>((size_t)c->E, Tk);
-    const int per_cta = env_int("MPE_DECODE_TASKS_PER_CTA", 8);
+    // tasks per CTA (measured best: gate/up 6, down 8; one override for both)
+    const int pc_env = env_int("MPE_DECODE_TASKS_PER_CTA", 0);
+    const int pc_gu = pc_env > 0 ? pc_env : 6, pc_dn = pc_env > 0 ? pc_env : 8;
     pl.claim = 1;
     const int nj_gu = c->H / kCodesPerBlock, nj_dn = c->F / kCodesPerBlock;
     const int tt_gu = tiles_per_task(true), tt_dn = tiles_per_task(false);
-    int p = decode_parts(groups, (c->F / 16 + tt_gu - 1) / tt_gu, nj_gu, ctas, per_cta);
+    int p = decode_parts(groups, (c->F / 16 + tt_gu - 1) / tt_gu, nj_gu, ctas, pc_gu);
     pl.kb_gu = (nj_gu + p - 1) / p;
     pl.p_gu = (nj_gu + pl.kb_gu - 1) / pl.kb_gu;
-    p = decode_parts(groups, (c->H / 16 + tt_dn - 1) / tt_dn, nj_dn, ctas, per_cta);
+    p = decode_parts(groups, (c->H / 16 + tt_dn - 1) / tt_dn, nj_dn, ctas, pc_dn);
     pl.kb_dn = (nj_dn + p - 1) / p;
     pl.p_dn = (nj_dn + pl.kb_dn - 1) / pl.kb_dn;
 }

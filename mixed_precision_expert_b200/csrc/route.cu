@@ -129,6 +129,10 @@ __global__ void __launch_bounds__(kChunk)
 k_route_small(const int32_t* ids, int Tk, int E, int group, const Pte* pte, int32_t* perm,
               int32_t* offsets, int32_t* inv, int32_t* wg, int32_t* n_wg, uint32_t* status,
               int32_t* zero6) {
+    // launched programmatically: the previous pass's kernels still read these
+    // buffers until they finish
+    griddep_wait();
+    griddep_launch_dependents();
     if (threadIdx.x < 6 && zero6) zero6[threadIdx.x] = 0;
     extern __shared__ __align__(16) uint8_t sm[];
     int32_t* s_cnt = reinterpret_cast<int32_t*>(sm);       // [E]
@@ -151,6 +155,8 @@ k_route_small(const int32_t* ids, int Tk, int E, int group, const Pte* pte, int3
 // T*k > 1024, step 1: per-chunk histograms hist[c][e].
 __global__ void __launch_bounds__(kChunk)
 k_route_hist(const int32_t* ids, int Tk, int E, int32_t* hist) {
+    griddep_wait();
+    griddep_launch_dependents();
     __shared__ int32_t s_cnt[MPE_MAX_EXPERTS];
     for (int i = threadIdx.x; i < E; i += kChunk) s_cnt[i] = 0;
     __syncthreads();
@@ -167,6 +173,8 @@ k_route_hist(const int32_t* ids, int Tk, int E, int32_t* hist) {
 __global__ void __launch_bounds__(kChunk)
 k_route_scan(int32_t* hist, int n_chunks, int E, int group, const Pte* pte, int32_t* offsets,
              int32_t* wg, int32_t* n_wg, int32_t* zero6) {
+    griddep_wait();
+    griddep_launch_dependents();
     if (threadIdx.x < 6 && zero6) zero6[threadIdx.x] = 0;
     __shared__ int32_t s_off[MPE_MAX_EXPERTS];
     const int e = threadIdx.x;
@@ -190,6 +198,8 @@ k_route_scan(int32_t* hist, int n_chunks, int E, int group, const Pte* pte, int3
 __global__ void __launch_bounds__(kChunk)
 k_route_scatter(const int32_t* ids, int Tk, int E, const int32_t* hist, int32_t* perm,
                 int32_t* inv, uint32_t* status) {
+    griddep_wait();
+    griddep_launch_dependents();
     extern __shared__ __align__(16) uint8_t sm[];
     uint16_t* wcnt = reinterpret_cast<uint16_t*>(sm);  // [32][E]
     for (int i = threadIdx.x; i < 32 * E; i += kChunk) wcnt[i] = 0;
@@ -207,19 +217,19 @@ void launch_route(mpe_ctx* c, const int32_t* ids, int Tk, int k, int32_t* perm,
     const int E = c->E;
     if (Tk <= kChunk) {
         const size_t sm = 2 * MPE_MAX_EXPERTS * sizeof(int32_t) + 32 * E * sizeof(uint16_t);
-        k_route_small<<<1, kChunk, sm, c->stream>>>(ids, Tk, E, group, c->d_pte, perm, offsets,
-                                                    inv, c->s.wg, c->s.n_wg, c->d_status,
-                                                    c->s.task_ctr);
+        launch_pdl(k_route_small, dim3(1), dim3(kChunk), sm, c->stream, ids, Tk, E, group,
+                   (const Pte*)c->d_pte, perm, offsets, inv, c->s.wg, c->s.n_wg, c->d_status,
+                   c->s.task_ctr);
         c->launches++;
         return;
     }
     const int nch = (Tk + kChunk - 1) / kChunk;
-    k_route_hist<<<nch, kChunk, 0, c->stream>>>(ids, Tk, E, c->s.hist);
-    k_route_scan<<<1, kChunk, 0, c->stream>>>(c->s.hist, nch, E, group, c->d_pte, offsets,
-                                              c->s.wg, c->s.n_wg, c->s.task_ctr);
+    launch_pdl(k_route_hist, dim3(nch), dim3(kChunk), 0, c->stream, ids, Tk, E, c->s.hist);
+    launch_pdl(k_route_scan, dim3(1), dim3(kChunk), 0, c->stream, c->s.hist, nch, E, group,
+               (const Pte*)c->d_pte, offsets, c->s.wg, c->s.n_wg, c->s.task_ctr);
     const size_t sm = 32 * E * sizeof(uint16_t);
-    k_route_scatter<<<nch, kChunk, sm, c->stream>>>(ids, Tk, E, c->s.hist, perm, inv,
-                                                    c->d_status);
+    launch_pdl(k_route_scatter, dim3(nch), dim3(kChunk), sm, c->stream, ids, Tk, E,
+               (const int32_t*)c->s.hist, perm, inv, c->d_status);
     c->launches += 3;
 }
 
