@@ -241,8 +241,10 @@ int mpe_get_page_table(mpe_ctx* ctx, mpe_pte* pte_host, uint32_t* page_idx_host,
 size_t mpe_expert_stream_bytes(mpe_ctx* ctx, int32_t e);
 
 /*
- * mpe_read_expert_packed -- gather expert e's chunk stream (W1, W3, W2 chunks
- * in stream order) out of its pages into host_dst (bytes >= the stream size).
+ * mpe_read_expert_packed -- gather expert e's chunk stream out of its pages
+ * into host_dst (bytes >= the stream size), in stream order: W1 and W3 chunks
+ * alternating (chunk 2c is W1's chunk c, 2c+1 W3's), then W2's chunks with
+ * row tiles 2v and 2v+1 alternating by block column.
  * Synchronous.
  */
 int mpe_read_expert_packed(mpe_ctx* ctx, int32_t e, void* host_dst, size_t bytes);

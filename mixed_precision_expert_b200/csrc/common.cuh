@@ -14,8 +14,10 @@
 // 16-bit halves of a word and unpacks to one bf16x2 register.
 // An expert stream is the chunks of W1 (gate [F x H]) and W3 (up [F x H])
 // interleaved -- chunk 2c is W1's chunk c, 2c+1 is W3's -- then those of W2
-// (down [H x F]); a tile's gate and up chunks for consecutive block columns are
-// therefore one contiguous run. Chunk c of an expert lives in page
+// (down [H x F]) with each pair of row tiles interleaved -- tile 2v's chunk j at
+// 2 (v nj + j), tile 2v+1's at 2 (v nj + j) + 1 (nj = F / 128). A tile's gate
+// and up chunks, or a tile pair's down chunks, for consecutive block columns
+// are therefore one contiguous run. Chunk c of an expert lives in page
 // pidx[first + c / cpp] at byte (c % cpp) * 256 b, cpp = page_bytes / (256 b).
 #pragma once
 
@@ -62,7 +64,7 @@ __device__ __forceinline__ void set_status(uint32_t* status, uint32_t bit) {
 }
 
 // chunks of one [F x H] matrix: the stream holds 2 of these interleaved (W1, W3),
-// then W2's chunks from index 2 * chunks_w1
+// then W2's chunks (tile pairs interleaved) from index 2 * chunks_w1
 __host__ __device__ inline int chunks_w1(int H, int F) { return (F / 16) * (H / 128); }
 
 // Address of chunk c of an expert.

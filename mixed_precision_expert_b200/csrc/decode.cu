@@ -68,13 +68,13 @@ __host__ __device__ constexpr int tiles_per_task(bool gateup) {
     return kConsumers * tiles_per_warp(gateup);
 }
 
-// A slot holds J consecutive block columns of every tile of a task (tiles in
-// order, so a warp's tiles are adjacent). The bulk-copy engine takes ~80
-// cycles per copy whatever its size up to a few KB, so a tile's chunks for the
-// slot -- gate and up interleaved, consecutive block columns, one contiguous
-// run of its page -- go in one copy, as many columns as keep a slot within
-// 56 KB (at least three slots per 192 KB ring): gate/up 2 (3, 4 bits) or 1
-// (8 bits), down (two tiles a warp) 2 / 2 / 1.
+// A slot holds J consecutive block columns of every tile of a task, one share
+// per consumer warp. The bulk-copy engine takes ~80 cycles per copy whatever
+// its size up to a few KB, so a share's chunks for the slot -- gate and up of
+// its tile interleaved, or its two down tiles interleaved, for consecutive
+// block columns: one contiguous run of the page -- go in one copy, as many
+// columns as keep a slot within 56 KB (at least three slots per 192 KB ring):
+// gate/up 2 (3, 4 bits) or 1 (8 bits), down (two tiles a warp) 2 / 2 / 1.
 template <int B, int NM, int TPW>
 struct Geo {
     static constexpr int CB = 256 * B;                   // chunk bytes
@@ -464,10 +464,11 @@ __device__ __forceinline__ bool resolve_class(const Args& a, const CtaSmem& sm, 
     }
 }
 
-// Copy warp: every task of one width class, from the queue. Lane l owns the
-// copy stream of the task's tile l (a page cursor in registers, the next page's index
-// loaded ahead): per slot one run of NM x jc chunks (gate/up: W1 and W3
-// alternate). Lane 0 arms the full barriers and writes the slot descriptors;
+// Copy warp: every task of one width class, from the queue. Lane w owns the
+// copy stream of consumer w's share of the task (a page cursor in registers,
+// the next page's index loaded ahead): per slot one run of NM x TPW x jc
+// chunks (gate/up: W1 and W3 of the tile alternate; down: the share's two
+// tiles alternate). Lane 0 arms the full barriers and writes the slot descriptors;
 // every lane prefetches one activation line. `ep` / `used` track the slots'
 // empty-barrier phases across classes, `fph` the queue's full-barrier phases.
 // In the down kernel the activations (h) come from the preceding kernel, so
@@ -487,8 +488,9 @@ __device__ __forceinline__ bool produce_class(const Args& a, const CtaSmem& sm, 
     const int nc1 = chunks_w1(P.H, P.F);
     const int cpp = chunks_per_page(B, P.page_bytes);
     const int n_pages = (3 * nc1 + cpp - 1) / cpp;
+    constexpr int TPW = tiles_per_warp(GATEUP);
     const int lane = threadIdx.x & 31;
-    const bool copier = lane < TT;
+    const bool copier = lane < kConsumers;  // lane w copies consumer w's share
 
     auto acquire = [&](int s) -> bool {
         if ((used >> s) & 1u) {
@@ -534,13 +536,15 @@ __device__ __forceinline__ bool produce_class(const Args& a, const CtaSmem& sm, 
             __syncwarp();
             return true;
         }
-        const int active = min(TT, n_tiles - tq * TT);
-        const bool my_tile = copier && lane < active;
+        const int active = min(TT, n_tiles - tq * TT);  // tiles (a multiple of TPW)
+        const bool my_tile = copier && lane * TPW < active;
         int pslot = 0, poff = 0;
         uint32_t page = 0, page_next = 0;
         if (my_tile) {
-            const int tau = tq * TT + lane;
-            const int c = GATEUP ? 2 * (tau * nj + j) : 2 * nc1 + tau * nj + j;
+            // the share's first chunk: gate/up interleaves W1 and W3 of a tile,
+            // down the two tiles (2v, 2v+1) of the share: two chunks a column
+            const int tau = tq * TT + lane * TPW;
+            const int c = GATEUP ? 2 * (tau * nj + j) : 2 * nc1 + 2 * ((tau >> 1) * nj + j);
             pslot = c / cpp;
             poff = c - pslot * cpp;
             page = __ldcg(P.pidx + first + pslot);
@@ -559,10 +563,10 @@ __device__ __forceinline__ bool produce_class(const Args& a, const CtaSmem& sm, 
             }
             __syncwarp();
             if (my_tile) {
-                // NM x jc consecutive chunks of this tile; a page boundary splits
-                // the copy in two
-                uint8_t* dst = sm.ring + (size_t)s * G::SLOT + (size_t)lane * G::TILEB;
-                const int total = NM * jc;
+                // the share's NM x TPW x jc consecutive chunks (two a block
+                // column); a page boundary splits the copy in two
+                uint8_t* dst = sm.ring + (size_t)s * G::SLOT + (size_t)lane * TPW * G::TILEB;
+                const int total = NM * TPW * jc;
                 const int n1 = min(total, cpp - poff);
                 bulk_g2s(dst, P.pool + (size_t)page * P.page_bytes + (size_t)poff * G::CB,
                          (uint32_t)(n1 * G::CB), &sm.full[s]);
@@ -717,7 +721,7 @@ __device__ __forceinline__ bool consume_class(const Args& a, const CtaSmem& sm, 
                 if (i > 0 && !T.valid1) break;
 #pragma unroll
                 for (int m = 0; m < NM; ++m) {
-                    const uint8_t* chunk = tiles + i * G::TILEB + (jj * NM + m) * G::CB;
+                    const uint8_t* chunk = tiles + ((jj * TPW + i) * NM + m) * G::CB;
                     load_row_words<B>(chunk, g, t, g, wr[i][m][0]);
                     load_row_words<B>(chunk, g + 8, t, g, wr[i][m][1]);
                 }

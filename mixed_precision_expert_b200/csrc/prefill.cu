@@ -227,9 +227,9 @@ __device__ __forceinline__ bool produce_tile(const PArgs& a, const Tile& T, int 
     const int cpp = chunks_per_page(B, P.page_bytes);
     // this thread's A row: gate/up feature nt*64 + 16 lq + lane/2 of W1 (even
     // lanes) or W3 (odd lanes); down: output nt*128 + 32 lq + lane of W2. Its
-    // chunk for block column j is c + cs * j: the stream interleaves W1 and W3
-    // chunks (cs = 2), W2's are consecutive (cs = 1).
-    constexpr int cs = GATEUP ? 2 : 1;
+    // chunk for block column j is c + 2 j: the stream interleaves W1 and W3
+    // chunks, and W2's tile pairs.
+    constexpr int cs = 2;
     int c, rr;
     if (GATEUP) {
         const int f = T.nt * 64 + lq * 16 + (lane >> 1);
@@ -237,7 +237,7 @@ __device__ __forceinline__ bool produce_tile(const PArgs& a, const Tile& T, int 
         rr = f & 15;
     } else {
         const int o = T.nt * 128 + lq * 32 + lane;
-        c = 2 * nc1 + (o >> 4) * nj;
+        c = 2 * nc1 + 2 * ((o >> 5) * nj) + ((o >> 4) & 1);
         rr = o & 15;
     }
     int pslot = c / cpp;

@@ -206,16 +206,24 @@ k_encode(PagedExperts P, const void* const* masters, const int32_t* list) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int c = blockIdx.x * 8 + warp;
     if (c >= 3 * nc1) return;
-    // stream chunk c: W1 / W3 chunks alternate (2 cc + m), then W2's chunks
-    int K, cc;
+    // stream chunk c: W1 / W3 chunks alternate (2 cc + m); W2's tiles 2v and
+    // 2v+1 alternate by block column (2 (v nj + j) + i)
+    int K, tau, j;
     size_t moff;
     if (c < 2 * nc1) {
-        K = H; cc = c >> 1; moff = (c & 1) ? (size_t)F * H : 0;
+        K = H;
+        const int cc = c >> 1, nj = K / kCodesPerBlock;
+        moff = (c & 1) ? (size_t)F * H : 0;
+        tau = cc / nj;
+        j = cc - tau * nj;
     } else {
-        K = F; cc = c - 2 * nc1; moff = 2 * (size_t)F * H;
+        K = F;
+        const int cc = c - 2 * nc1, nj = K / kCodesPerBlock;
+        moff = 2 * (size_t)F * H;
+        const int pr = cc >> 1, v = pr / nj;
+        j = pr - v * nj;
+        tau = 2 * v + (cc & 1);
     }
-    const int nj = K / kCodesPerBlock;
-    const int tau = cc / nj, j = cc - tau * nj;
     const int rho = lane >> 2, q = lane & 3;
     const __half* base = reinterpret_cast<const __half*>(masters[e]) + moff;
     const __half* r0 = base + (size_t)(tau * 16 + rho) * K + 128 * j + 32 * q;

@@ -146,7 +146,15 @@ def n_chunks(H: int, F: int) -> int:
 
 def expert_stream(u1: np.ndarray, u3: np.ndarray, u2: np.ndarray, b: int) -> np.ndarray:
     """Chunk stream of one expert: W1 and W3 chunk by chunk (W1 chunk c at 2c,
-    W3 chunk c at 2c + 1), then W2. uint8 [n_chunks, 256*b]."""
+    W3 chunk c at 2c + 1), then W2 with each pair of row tiles interleaved by
+    block column (tile 2v's chunk j at 2(v nj + j), tile 2v+1's at
+    2(v nj + j) + 1 after the gate/up chunks). uint8 [n_chunks, 256*b]."""
     g1, g3 = pack_matrix(u1, b), pack_matrix(u3, b)
     gu = np.stack([g1, g3], axis=1).reshape(2 * g1.shape[0], chunk_bytes(b))
-    return np.concatenate([gu, pack_matrix(u2, b)])
+    R2, K2 = np.asarray(u2).shape
+    nt2, nj2 = R2 // ROWS_PER_CHUNK, K2 // CODES_PER_BLOCK
+    if nt2 % 2:
+        raise ValueError("W2 needs an even number of 16-row tiles (H % 32 == 0)")
+    g2 = pack_matrix(u2, b).reshape(nt2 // 2, 2, nj2, chunk_bytes(b))
+    g2 = g2.transpose(0, 2, 1, 3).reshape(nt2 * nj2, chunk_bytes(b))
+    return np.concatenate([gu, g2])

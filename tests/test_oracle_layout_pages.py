@@ -128,6 +128,15 @@ def test_expert_stream_order():
     g1, g3 = L.pack_matrix(u1, b), L.pack_matrix(u3, b)
     for c in range(g1.shape[0]):
         assert np.array_equal(s[2 * c], g1[c]) and np.array_equal(s[2 * c + 1], g3[c])
+    # W2: tiles 2v and 2v+1 alternate by block column
+    g2 = L.pack_matrix(u2, b)
+    nc1, nt2, nj2 = g1.shape[0], H // 16, F // 128
+    for tau in range(nt2):
+        for j in range(nj2):
+            pos = 2 * nc1 + 2 * ((tau // 2) * nj2 + j) + (tau % 2)
+            assert np.array_equal(s[pos], g2[tau * nj2 + j])
+    # and the stream still carries every code exactly once
+    assert sorted(map(bytes, s[2 * nc1:])) == sorted(map(bytes, g2))
 
 
 # ----------------------------------------------------------------------------
