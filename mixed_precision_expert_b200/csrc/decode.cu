@@ -24,8 +24,9 @@
 //   consumers:  wait on the slot's full barrier, copy their chunk's words to
 //               registers, release the slot on its empty barrier and only then
 //               unpack (common.cuh) and multiply with mma.sync m16n8k16 --
-//               weights are the 16-row A operand, one 8-token n-tile of
-//               activations is B, fp32 accumulate,
+//               weights are the 16-row A operand, the 8-token n-tile of
+//               activations is B (a down warp's two tiles interleave
+//               step by step), fp32 accumulate,
 //               the per-expert scale applied once at the end.
 // A task whose K range is split in P parts writes a scaled partial to its own
 // slice; a later pass sums the slices in part order (deterministic, no
@@ -271,30 +272,56 @@ struct UnpackRegs<8> {
     }
 };
 
-// Unpack and multiply one block (128 codes of 16 rows, NM matrices) with NT
-// 8-token n-tiles of activations. Widths 3 and 4 unpack to the offset form
+// Unpack and multiply one block (128 codes of 16 rows, NM matrices, NTILE
+// tiles) with NT 8-token n-tiles of activations: every unpacked weight
+// fragment serves all n-tiles. Widths 3 and 4 unpack to the offset form
 // (k + off, see common.cuh), whose off . x term the task's offset sums remove;
-// width 8 unpacks to k.
-template <int B, int NM, int NT>
+// width 8 unpacks to k. One n-tile loads the block's activations up front;
+// two load them half a block at a time (the same 16 registers).
+template <int B, int NM, int NT, int NTILE, int TPW>
 __device__ __forceinline__ void block_mma(const UnpackRegs<B>& U,
-                                          const uint32_t (&wr)[NM][2][Geo<B, 1, 1>::WORDS],
-                                          const uint32_t (&xa)[kMaxTiles][8],
-                                          const uint32_t (&xz)[kMaxTiles][8],
-                                          float (&acc)[kMaxTiles][NM][4]) {
+                                          const uint32_t (&wr)[TPW][NM][2][Geo<B, 1, 1>::WORDS],
+                                          const __nv_bfloat16* const (&arow)[kMaxTiles], int j,
+                                          int t, float (&acc)[TPW][kMaxTiles][NM][4]) {
+    constexpr int HALVES = NT == 1 ? 1 : 2;  // activation loads per block
+    constexpr int CH = 8 / HALVES;           // mma steps per load
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
+    for (int h = 0; h < HALVES; ++h) {
+        uint32_t x[NT][16 / HALVES];
 #pragma unroll
-        for (int m = 0; m < NM; ++m) {
-            const uint32_t a0 = U.pair(wr[m][0], 2 * c);
-            const uint32_t a1 = U.pair(wr[m][1], 2 * c);
-            const uint32_t a2 = U.pair(wr[m][0], 2 * c + 1);
-            const uint32_t a3 = U.pair(wr[m][1], 2 * c + 1);
+        for (int nt = 0; nt < NT; ++nt) {
+            if constexpr (HALVES == 1) {
+                uint32_t xa[8], xz[8];
+                load_act_half(arow[nt], j, t, B == 8, 0, xa);
+                load_act_half(arow[nt], j, t, B == 8, 1, xz);
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                const uint32_t b0 = c < 4 ? xa[nt][2 * c] : xz[nt][2 * c - 8];
-                const uint32_t b1 = c < 4 ? xa[nt][2 * c + 1] : xz[nt][2 * c - 7];
-                mma_bf16_16816(acc[nt][m], a0, a1, a2, a3, b0, b1);
+                for (int i = 0; i < 8; ++i) {
+                    x[nt][i] = xa[i];
+                    x[nt][8 + i] = xz[i];
+                }
+            } else {
+                uint32_t xh[8];
+                load_act_half(arow[nt], j, t, B == 8, h, xh);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) x[nt][i] = xh[i];
             }
+        }
+#pragma unroll
+        for (int cc = 0; cc < CH; ++cc) {
+            const int c = h * CH + cc;
+#pragma unroll
+            for (int i = 0; i < NTILE; ++i)
+#pragma unroll
+                for (int m = 0; m < NM; ++m) {
+                    const uint32_t a0 = U.pair(wr[i][m][0], 2 * c);
+                    const uint32_t a1 = U.pair(wr[i][m][1], 2 * c);
+                    const uint32_t a2 = U.pair(wr[i][m][0], 2 * c + 1);
+                    const uint32_t a3 = U.pair(wr[i][m][1], 2 * c + 1);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+                        mma_bf16_16816(acc[i][nt][m], a0, a1, a2, a3, x[nt][2 * cc],
+                                       x[nt][2 * cc + 1]);
+                }
         }
     }
 }
@@ -302,8 +329,7 @@ __device__ __forceinline__ void block_mma(const UnpackRegs<B>& U,
 struct Task {
     int tau, p, pos0, ntok, j_hi;  // tau: the warp's first tile
     float scale;
-    bool valid;   // the warp's first tile exists
-    bool valid1;  // its second tile exists (two tiles a warp)
+    bool valid;   // the warp's tiles exist
 };
 
 // Finish a task. One K part (P = 1): gate/up applies SwiGLU and stores h
@@ -620,7 +646,6 @@ __device__ __forceinline__ bool consume_class(const Args& a, const CtaSmem& sm, 
     const __nv_bfloat16* arow[kMaxTiles] = {};
     int ntiles = 0;
     float acc[TPW][kMaxTiles][NM][4];
-    uint32_t xa[kMaxTiles][8], xz[kMaxTiles][8];  // activations of the block
     const UnpackRegs<B> U;
     // widths 3, 4: acc <- acc - off . x for every tile and matrix, with the
     // task warp's per-token sums (accumulator column n = token n)
@@ -673,9 +698,7 @@ __device__ __forceinline__ bool consume_class(const Args& a, const CtaSmem& sm, 
                     settle(m);
                 }
                 finish<GATEUP>(a, T, T.tau, acc[0], lane);
-                if constexpr (TPW > 1) {
-                    if (T.valid1) finish<GATEUP>(a, T, T.tau + 1, acc[1], lane);
-                }
+                if constexpr (TPW > 1) finish<GATEUP>(a, T, T.tau + 1, acc[1], lane);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.tq_empty[d.q]);
@@ -684,8 +707,9 @@ __device__ __forceinline__ bool consume_class(const Args& a, const CtaSmem& sm, 
         if (d.flags & kFirstSlot) {
             const TaskMeta* m = sm.taskq + d.q;
             T.tau = m->tq * tiles_per_task(GATEUP) + w * TPW;
+            // a task's tile count is even (H and F are multiples of 128), so a
+            // down warp with a first tile also has its second
             T.valid = T.tau < n_tiles;
-            T.valid1 = TPW > 1 && T.tau + 1 < n_tiles;
             T.p = m->p;
             T.pos0 = m->pos0;
             T.ntok = m->ntok;
@@ -718,7 +742,6 @@ __device__ __forceinline__ bool consume_class(const Args& a, const CtaSmem& sm, 
             uint32_t wr[TPW][NM][2][G::WORDS];
 #pragma unroll
             for (int i = 0; i < TPW; ++i) {
-                if (i > 0 && !T.valid1) break;
 #pragma unroll
                 for (int m = 0; m < NM; ++m) {
                     const uint8_t* chunk = tiles + ((jj * TPW + i) * NM + m) * G::CB;
@@ -731,17 +754,15 @@ __device__ __forceinline__ bool consume_class(const Args& a, const CtaSmem& sm, 
                 if (lane == 0) mbar_arrive(&sm.empty[s]);
             }
             const int j = d.j + jj;
-#pragma unroll
-            for (int nt = 0; nt < kMaxTiles; ++nt) {
-                if (nt == 0 || nt < ntiles) {
-                    load_act_half(arow[nt], j, t, B == 8, 0, xa[nt]);
-                    load_act_half(arow[nt], j, t, B == 8, 1, xz[nt]);
+            // one instantiation per n-tile count that can occur: the unrolled
+            // block is large, and duplicates cost instruction fetch
+            if constexpr (kMaxTiles > 1) {
+                if (ntiles > 1) {
+                    block_mma<B, NM, kMaxTiles, TPW, TPW>(U, wr, arow, j, t, acc);
+                    continue;
                 }
             }
-            block_mma<B, NM, kMaxTiles>(U, wr[0], xa, xz, acc[0]);
-            if constexpr (TPW > 1) {
-                if (T.valid1) block_mma<B, NM, kMaxTiles>(U, wr[1], xa, xz, acc[1]);
-            }
+            block_mma<B, NM, 1, TPW, TPW>(U, wr, arow, j, t, acc);
         }
         if ((d.flags & kLastSlot) && !close_task()) return false;
     }
