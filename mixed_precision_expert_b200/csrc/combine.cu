@@ -66,27 +66,23 @@ k_combine_by_position(const float* y, const int32_t* inv, const float* w, int T,
             if (pos < 0) continue;
             const float wj = w[t * k + j];
             const float4* src = reinterpret_cast<const float4*>(y + (size_t)pos * H) + i;
-            float4 v = src[0];
-            int p = 1;
-            // parts in order; four independent loads in flight per step
-            for (; p + 4 <= parts; p += 4) {
-                float4 u[4];
+            const size_t stride = part_stride / 4;
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            // parts summed in order; up to 16 independent loads in flight
+            for (int p0 = 0; p0 < parts; p0 += 16) {
+                float4 u[16];
 #pragma unroll
-                for (int r = 0; r < 4; ++r) u[r] = src[(p + r) * (part_stride / 4)];
+                for (int r = 0; r < 16; ++r)
+                    if (p0 + r < parts) u[r] = src[(size_t)(p0 + r) * stride];
 #pragma unroll
-                for (int r = 0; r < 4; ++r) {
-                    v.x += u[r].x;
-                    v.y += u[r].y;
-                    v.z += u[r].z;
-                    v.w += u[r].w;
+                for (int r = 0; r < 16; ++r) {
+                    if (p0 + r < parts) {
+                        v.x += u[r].x;
+                        v.y += u[r].y;
+                        v.z += u[r].z;
+                        v.w += u[r].w;
+                    }
                 }
-            }
-            for (; p < parts; ++p) {
-                const float4 u = src[p * (part_stride / 4)];
-                v.x += u.x;
-                v.y += u.y;
-                v.z += u.z;
-                v.w += u.w;
             }
             acc.x = fmaf(wj, v.x, acc.x);
             acc.y = fmaf(wj, v.y, acc.y);

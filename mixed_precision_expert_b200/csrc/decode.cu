@@ -10,7 +10,7 @@
 //
 // Warp-specialised persistent kernel. A CTA (one per SM) has 14 consumer
 // warps, 1 copy warp and 1 task warp and works on one task at a time: a work
-// group (<= 8 tokens of one expert) x 14 (gate/up: one per consumer warp) or
+// group (<= 16 tokens of one expert) x 14 (gate/up: one per consumer warp) or
 // 28 (down: two per warp) consecutive 16-row output tiles x a K part.
 //   task warp:  claims tasks from a per-width-class counter and resolves them
 //               (expert, tokens, activation rows, scale, first page entry)
@@ -18,15 +18,16 @@
 //               no other warp waits on a chain of dependent global loads;
 //   copy warp:  for each queued task and each group of J block columns, fills
 //               one slot of the CTA's shared-memory ring with the task's
-//               chunks (one 1-D bulk copy per tile, issued by 14-28 lanes in
-//               parallel, no multicast; a full mbarrier counts the bytes) and
-//               prefetches the block's activation lines into L1;
+//               chunks (one 1-D bulk copy per consumer share, issued by 14
+//               lanes in parallel, no multicast; a full mbarrier counts the
+//               bytes) and prefetches the block's activation lines into L1;
 //   consumers:  wait on the slot's full barrier, copy their chunk's words to
 //               registers, release the slot on its empty barrier and only then
 //               unpack (common.cuh) and multiply with mma.sync m16n8k16 --
-//               weights are the 16-row A operand, the 8-token n-tile of
-//               activations is B (a down warp's two tiles interleave
-//               step by step), fp32 accumulate,
+//               weights are the 16-row A operand, one or two 8-token
+//               n-tiles of activations are B (they share every unpacked
+//               weight fragment; a down warp's two tiles interleave step
+//               by step), fp32 accumulate,
 //               the per-expert scale applied once at the end.
 // A task whose K range is split in P parts writes a scaled partial to its own
 // slice; a later pass sums the slices in part order (deterministic, no
@@ -736,7 +737,11 @@ __device__ __forceinline__ bool consume_class(const Args& a, const CtaSmem& sm, 
         }
         const int t = lane & 3;
         const uint8_t* tiles = sm.ring + (size_t)s * G::SLOT + (size_t)w * TPW * G::TILEB;
-#pragma unroll
+        // the block columns of a slot stay a loop: each block is a large
+        // unrolled body, and the code for one width class has to stay in the
+        // instruction cache (with this loop unrolled, 16-token groups cost the
+        // Mixtral-shaped layer 5 %; rolled, they cost nothing)
+#pragma unroll 1
         for (int jj = 0; jj < G::J; ++jj) {
             if (jj >= d.nc) break;
             uint32_t wr[TPW][NM][2][G::WORDS];
@@ -854,9 +859,12 @@ void decode_plan(mpe_ctx* c, size_t Tk, DecodePlan& pl) {
     if (!g_num_sms) cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, c->device);
     const int ctas = g_num_sms;
     const int groups = (int)std::min<size_t>((size_t)c->E, Tk);
-    // tasks per CTA (measured best: gate/up 6, down 8; one override for both)
+    // tasks per CTA (measured best: gate/up 6, down 8); tuning overrides
     const int pc_env = env_int("MPE_DECODE_TASKS_PER_CTA", 0);
-    const int pc_gu = pc_env > 0 ? pc_env : 6, pc_dn = pc_env > 0 ? pc_env : 8;
+    const int pc_gu_env = env_int("MPE_DECODE_TASKS_PER_CTA_GATEUP", 0);
+    const int pc_dn_env = env_int("MPE_DECODE_TASKS_PER_CTA_DOWN", 0);
+    const int pc_gu = pc_gu_env > 0 ? pc_gu_env : (pc_env > 0 ? pc_env : 6);
+    const int pc_dn = pc_dn_env > 0 ? pc_dn_env : (pc_env > 0 ? pc_env : 8);
     pl.claim = 1;
     const int nj_gu = c->H / kCodesPerBlock, nj_dn = c->F / kCodesPerBlock;
     const int tt_gu = tiles_per_task(true), tt_dn = tiles_per_task(false);

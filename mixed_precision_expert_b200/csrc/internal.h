@@ -13,13 +13,12 @@
 
 namespace mpe {
 
-// Tokens per work group of the decode kernels (one 8-token mma n-tile): an
-// expert with more tokens is served by several groups, which read its pages
-// close together in time (mostly from L2). The decode kernels also build with
-// 16 (two n-tiles sharing every unpacked weight fragment), which unpacks the
-// pages of heavily routed experts half as often but doubles the unrolled code
-// and the accumulators; with 8 the Mixtral-shaped layer runs 5 % faster.
-constexpr int kDecodeGroup = 8;
+// Tokens per work group of the decode kernels (up to two 8-token mma n-tiles,
+// which share every unpacked weight fragment, so a heavily routed expert's
+// pages are unpacked once per 16 tokens): an expert with more tokens is
+// served by several groups, which read its pages close together in time
+// (mostly from L2).
+constexpr int kDecodeGroup = 16;
 
 struct Scratch {
     size_t cap_assign = 0;   // T*k capacity
