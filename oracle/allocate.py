@@ -128,3 +128,59 @@ def objective(p, bits) -> float:
 
 def budget_used(W, bits) -> int:
     return sum(int(w) * int(b) for w, b in zip(W, bits))
+
+
+def proportional_widths(p, W, B: int) -> np.ndarray:
+    """The page's simplified allocator ("Code Illustration",
+    compute_budgeted_precision), read for what it computes: expert e gets the
+    budget share B p_e / sum p, i.e. share / W_e bits per weight, rounded UP to
+    the next available width (3 if at most 3, 4 if in (3, 4], 8 above 4 -- the
+    illustration's bucketize over (3, 4, 8) with the index clamped to the last
+    width). The result can exceed the budget.
+
+    Float64, in this order: total = p_0 + p_1 + ... (ascending e); share =
+    (B * p_e) / total; bits = share / W_e. B counts bits (the illustration's
+    "budget_bytes" divided by element counts is read as bits per element, as in
+    the exact allocator); all-zero importances give every expert 3 bits.
+    """
+    p = np.asarray(p, dtype=np.float64)
+    W = [int(w) for w in W]
+    E = len(W)
+    if E == 0 or len(p) != E or any(w <= 0 for w in W):
+        raise ValueError("need E > 0 experts with W_e > 0 and one p_e each")
+    total = 0.0
+    for pe in p:
+        total = total + float(pe)
+    bits = np.empty(E, dtype=np.uint8)
+    for e in range(E):
+        share = (float(int(B)) * float(p[e])) / total if total > 0.0 else 0.0
+        per_weight = share / float(W[e])
+        bits[e] = 3 if per_weight <= 3.0 else (4 if per_weight <= 4.0 else 8)
+    return bits
+
+
+def allocate_bits_proportional(p, W, B: int) -> np.ndarray:
+    """proportional_widths followed by a budget repair -- a reading of this
+    build (the illustration has no such step): experts are walked in ascending
+    (p_e, e) and each is downgraded one width at a time (8 -> 4 -> 3) until
+    sum b_e W_e <= B. Raises Infeasible if B < 3 sum W."""
+    W = [int(w) for w in W]
+    B = int(B)
+    if B < 3 * sum(W):
+        raise Infeasible(f"B={B} < 3*sum(W)={3 * sum(W)}")
+    p = np.asarray(p, dtype=np.float64)
+    bits = proportional_widths(p, W, B)
+    used = budget_used(W, bits)
+    for e in sorted(range(len(W)), key=lambda i: (float(p[i]), i)):
+        if used <= B:
+            break
+        if bits[e] == 8:
+            bits[e] = 4
+            used -= 4 * W[e]
+        if used <= B:
+            break
+        if bits[e] == 4:
+            bits[e] = 3
+            used -= W[e]
+    assert used <= B
+    return bits

@@ -129,3 +129,50 @@ def test_exchange_property_equal_W(seed):
 def test_state_cap():
     with pytest.raises(A.StateCapExceeded):
         A.allocate_bits([0.5, 0.5], [1, 2], 3 * 3 + 10, state_cap=4)
+
+
+# ----------------------------------------------------------------------------
+# the page's proportional illustration (+ budget repair), a selectable variant
+# ----------------------------------------------------------------------------
+def test_proportional_rounds_up_like_the_illustration():
+    # one expert, so its share is the whole budget: B / W bits a weight, rounded
+    # up to the next width (3.0 -> 3, 3.001 -> 4, 4.0 -> 4, 4.001 -> 8, > 8 -> 8)
+    # (p = 0.5 keeps B p / p exact in float64; p = 0.7 would give 4000.0000000000005)
+    W = [1000]
+    cases = {1000: 3, 3000: 3, 3001: 4, 3010: 4, 4000: 4, 4001: 8, 4500: 8, 8000: 8, 9000: 8}
+    for B, want in cases.items():
+        assert list(A.proportional_widths([0.5], W, B)) == [want], B
+    # the repair then brings a width that exceeds the budget down
+    assert list(A.allocate_bits_proportional([0.5], W, 3001)) == [3]
+    assert list(A.allocate_bits_proportional([0.5], W, 4500)) == [4]
+    assert list(A.allocate_bits_proportional([0.5], W, 9000)) == [8]
+    # all-zero importances: no share, 3 bits
+    assert list(A.proportional_widths([0.0, 0.0], [10, 10], 100)) == [3, 3]
+
+
+def test_proportional_hand_example():
+    # shares 160/320/480/640 bits for W = 100: 1.6, 3.2, 4.8, 6.4 bits a weight
+    # -> (3, 4, 8, 8) using 2300 > 1600; repair in ascending p: expert 1 4->3
+    # (2200), expert 2 8->4 (1800) and 4->3 (1700), expert 3 8->4 (1300)
+    p = [0.1, 0.2, 0.3, 0.4]
+    bits = A.allocate_bits_proportional(p, [100] * 4, 1600)
+    assert list(bits) == [3, 3, 3, 4]
+    # a budget that fits the rounded-up widths is left alone
+    assert list(A.allocate_bits_proportional(p, [100] * 4, 2300)) == [3, 4, 8, 8]
+
+
+def test_proportional_budget_and_errors():
+    rng = np.random.default_rng(5)
+    for _ in range(200):
+        E = int(rng.integers(1, 12))
+        p = rng.dirichlet(np.full(E, 0.5))
+        W = [int(x) for x in rng.integers(1, 60, size=E)]
+        B = int(rng.integers(3 * sum(W), 9 * sum(W)))
+        bits = A.allocate_bits_proportional(p, W, B)
+        assert set(bits.tolist()) <= {3, 4, 8}
+        assert A.budget_used(W, bits) <= B
+        # the exact allocator is never worse on the page's objective
+        exact = A.allocate_bits(p, W, B)
+        assert A.objective(p, exact) <= A.objective(p, bits) * (1 + 1e-12)
+    with pytest.raises(A.Infeasible):
+        A.allocate_bits_proportional([1.0, 1.0], [5, 5], 29)
