@@ -128,6 +128,27 @@ int mpe_allocate_bits(const double* p, const uint64_t* W, int32_t E, uint64_t B_
                       uint8_t* bits_out);
 
 /*
+ * mpe_allocate_bits_proportional -- the page's simplified allocator
+ * ("Code Illustration", compute_budgeted_precision): expert e's share of the
+ * budget, B_bits p_e / sum p, in bits per weight (share / W_e) rounded up to
+ * the next width (3 if <= 3, 4 if <= 4, else 8); then, since rounding up can
+ * exceed the budget, experts in ascending (p_e, e) are downgraded one width at
+ * a time (8 -> 4 -> 3) until sum b_e W_e <= B_bits (the repair is this
+ * library's addition). float64 throughout, sum p in ascending e; one device
+ * kernel on the current device. Same arguments as mpe_allocate_bits.
+ * Synchronous. MPE_ERR_INFEASIBLE if B_bits < 3 sum W.
+ */
+int mpe_allocate_bits_proportional(const double* p, const uint64_t* W, int32_t E,
+                                   uint64_t B_bits, uint8_t* bits_out);
+
+/* width rules mpe_repage can use (mpe_set_allocator) */
+#define MPE_ALLOCATOR_EXACT        0  /* mpe_allocate_bits (default)            */
+#define MPE_ALLOCATOR_PROPORTIONAL 1  /* mpe_allocate_bits_proportional         */
+
+/* mpe_set_allocator -- choose the width rule of later mpe_repage calls. */
+int mpe_set_allocator(mpe_ctx* ctx, int32_t allocator);
+
+/*
  * mpe_quantize_experts -- quantize every expert at the given widths
  * ("Implementation Details", quantization scheme): per-expert absmax m_e
  * (cached: the master must not change while the context lives), scale
@@ -149,8 +170,10 @@ int mpe_quantize_experts(mpe_ctx* ctx, const void* const* master_f16, const uint
 /*
  * mpe_repage -- budget change with KV-cache occupancy ("Implementation
  * Details"; 0to1log digest: lower precision as the KV cache grows, raise it
- * as it shrinks): re-run mpe_allocate_bits with B_bits and importances p
- * (host float64[E]), release the pages of experts whose width changed, give
+ * as it shrinks): re-run the context's width rule (mpe_allocate_bits, or
+ * mpe_allocate_bits_proportional after mpe_set_allocator) with B_bits and
+ * importances p (host float64[E]), release the pages of experts whose width
+ * changed, give
  * them new pages and re-encode only those experts from the fp16 master with
  * the cached absmax. *n_changed_out (host, may be NULL) receives the count.
  * Synchronises once (the new widths decide the page moves); the encode is

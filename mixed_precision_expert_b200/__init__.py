@@ -30,12 +30,14 @@ STATUS_BAD_EXPERT_ID = 0x1
 STATUS_NONFINITE = 0x2
 STATUS_WAIT_TIMEOUT = 0x4
 PATH_AUTO, PATH_DECODE, PATH_PREFILL = 0, 1, 2
+ALLOCATOR_EXACT, ALLOCATOR_PROPORTIONAL = 0, 1
 ALLOC_STATE_CAP = 65536
 MAX_EXPERTS = 1024
 
 # every symbol include/mpe.h declares
 EXPORTS = [
     "mpe_create", "mpe_destroy", "mpe_set_stream", "mpe_set_path", "mpe_allocate_bits",
+    "mpe_allocate_bits_proportional", "mpe_set_allocator",
     "mpe_quantize_experts", "mpe_repage", "mpe_moe_ffn", "mpe_moe_ffn_host", "mpe_route",
     "mpe_get_page_table", "mpe_expert_stream_bytes", "mpe_read_expert_packed",
     "mpe_get_scales", "mpe_get_bits", "mpe_get_status", "mpe_last_error",
@@ -88,6 +90,8 @@ def lib() -> ctypes.CDLL:
         "mpe_set_stream": (i32, [vp, vp]),
         "mpe_set_path": (i32, [vp, i32]),
         "mpe_allocate_bits": (i32, [vp, vp, i32, u64, vp]),
+        "mpe_allocate_bits_proportional": (i32, [vp, vp, i32, u64, vp]),
+        "mpe_set_allocator": (i32, [vp, i32]),
         "mpe_quantize_experts": (i32, [vp, vp, vp]),
         "mpe_repage": (i32, [vp, u64, vp, vp]),
         "mpe_moe_ffn": (i32, [vp, vp, i32, vp, vp, i32, vp]),
@@ -146,6 +150,16 @@ def allocate_bits(p, W, B: int) -> np.ndarray:
     return out
 
 
+def allocate_bits_proportional(p, W, B: int) -> np.ndarray:
+    """The page's proportional rule (budget share by importance, rounded up to
+    3/4/8 bits) with the library's budget repair (device kernel)."""
+    p = np.ascontiguousarray(p, dtype=np.float64)
+    W = np.ascontiguousarray(W, dtype=np.uint64)
+    out = np.zeros(len(p), dtype=np.uint8)
+    _check(lib().mpe_allocate_bits_proportional(_ptr(p), _ptr(W), len(p), int(B), _ptr(out)))
+    return out
+
+
 def route_noalloc(ids, E: int, perm, offsets, inv):
     """Bucketing into caller-provided device buffers without any device
     allocation (mpe_route_noalloc); runs on the current stream."""
@@ -185,6 +199,10 @@ class Context:
 
     def set_path(self, path: int):
         _check(lib().mpe_set_path(self._h, path), self._h)
+
+    def set_allocator(self, allocator: int):
+        """ALLOCATOR_EXACT (default) or ALLOCATOR_PROPORTIONAL for later repages."""
+        _check(lib().mpe_set_allocator(self._h, allocator), self._h)
 
     def quantize_experts(self, masters, bits):
         """masters: E flat fp16 CUDA tensors (W1 | W3 | W2); bits: uint8[E]."""

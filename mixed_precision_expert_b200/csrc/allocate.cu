@@ -137,6 +137,92 @@ k_allocate(const double* p, const uint64_t* W, int E, uint64_t B, uint64_t sum_w
     }
 }
 
+// The page's simplified allocator ("Code Illustration",
+// compute_budgeted_precision) with a budget repair, one CTA: each expert's
+// budget share B p_e / sum p in bits per weight, rounded up to 3 / 4 / 8 (3 if
+// at most 3, 4 if at most 4, else 8); then, in ascending (p_e, e), each expert
+// is downgraded one width at a time until sum b_e W_e <= B. The sum of p runs
+// in ascending e (one thread) and every operation is one correctly rounded
+// float64 step, so the widths are reproducible bit for bit. status: 0 solved,
+// 1 infeasible (B < 3 sum W).
+constexpr int kPropThreads = 256;
+constexpr int kPropSort = MPE_MAX_EXPERTS;  // sort capacity (a power of two)
+
+__global__ void __launch_bounds__(kPropThreads)
+k_allocate_proportional(const double* p, const uint64_t* W, int E, uint64_t B, uint64_t sum_w,
+                        uint8_t* bits_out, int32_t* status) {
+    __shared__ double s_key[kPropSort];
+    __shared__ int32_t s_idx[kPropSort];
+    __shared__ uint8_t s_bits[MPE_MAX_EXPERTS];
+    __shared__ double s_total;
+    const int tid = threadIdx.x;
+    if (B < 3 * sum_w) {
+        if (tid == 0) *status = 1;
+        return;
+    }
+    if (tid == 0) {
+        double t = 0.0;
+        for (int e = 0; e < E; ++e) t = __dadd_rn(t, p[e]);
+        s_total = t;
+        *status = 0;
+    }
+    __syncthreads();
+    const double total = s_total;
+    const double Bd = __ull2double_rn(B);
+    for (int e = tid; e < E; e += kPropThreads) {
+        const double pe = p[e];
+        const double share = total > 0.0 ? __ddiv_rn(__dmul_rn(Bd, pe), total) : 0.0;
+        const double pw = __ddiv_rn(share, __ull2double_rn(W[e]));
+        s_bits[e] = pw <= 3.0 ? 3 : (pw <= 4.0 ? 4 : 8);
+    }
+    // bitonic sort of (p_e, e) ascending; padding sorts last
+    int n = 1;
+    while (n < E) n <<= 1;
+    for (int i = tid; i < n; i += kPropThreads) {
+        s_key[i] = i < E ? p[i] : __longlong_as_double(0x7FF0000000000000ll);
+        s_idx[i] = i < E ? i : 0x7FFFFFFF;
+    }
+    __syncthreads();
+    for (int k = 2; k <= n; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            for (int i = tid; i < n; i += kPropThreads) {
+                const int l = i ^ j;
+                if (l > i) {
+                    const bool up = (i & k) == 0;
+                    const bool gt = s_key[i] > s_key[l] || (s_key[i] == s_key[l] && s_idx[i] > s_idx[l]);
+                    if (gt == up) {
+                        const double tk = s_key[i];
+                        s_key[i] = s_key[l];
+                        s_key[l] = tk;
+                        const int ti = s_idx[i];
+                        s_idx[i] = s_idx[l];
+                        s_idx[l] = ti;
+                    }
+                }
+            }
+            __syncthreads();
+        }
+    }
+    if (tid == 0) {
+        uint64_t used = 0;
+        for (int e = 0; e < E; ++e) used += (uint64_t)s_bits[e] * W[e];
+        for (int r = 0; r < E && used > B; ++r) {
+            const int e = s_idx[r];
+            if (s_bits[e] == 8) {
+                s_bits[e] = 4;
+                used -= 4 * W[e];
+            }
+            if (used <= B) break;
+            if (s_bits[e] == 4) {
+                s_bits[e] = 3;
+                used -= W[e];
+            }
+        }
+    }
+    __syncthreads();
+    for (int e = tid; e < E; e += kPropThreads) bits_out[e] = s_bits[e];
+}
+
 }  // namespace
 
 size_t allocate_choice_bytes(int E, uint64_t R) { return (size_t)E * (size_t)((R + 4) / 4); }
@@ -158,6 +244,11 @@ void launch_allocate(cudaStream_t st, const double* p, const uint64_t* W, int E,
         k_allocate<false><<<1, kThreads, 0, st>>>(p, W, E, B, sum_w, g, bits_out, status, choice,
                                                   D, state_cap);
     }
+}
+
+void launch_allocate_proportional(cudaStream_t st, const double* p, const uint64_t* W, int E,
+                                  uint64_t B, uint64_t sum_w, uint8_t* bits_out, int32_t* status) {
+    k_allocate_proportional<<<1, kPropThreads, 0, st>>>(p, W, E, B, sum_w, bits_out, status);
 }
 
 }  // namespace mpe

@@ -231,10 +231,11 @@ int run_allocate(mpe_ctx* c, const double* p, uint64_t B, std::vector<uint8_t>& 
     if (B < 3 * sum_w) return fail(c, MPE_ERR_INFEASIBLE, "budget %llu < 3 * sum W = %llu",
                                    (unsigned long long)B, (unsigned long long)(3 * sum_w));
     const uint64_t g = w_e;
+    const bool exact = c->allocator == MPE_ALLOCATOR_EXACT;
     uint64_t R = B >= 8 * sum_w ? 0 : (B - 3 * sum_w) / g;
     R = std::min<uint64_t>(R, 5 * (sum_w / g));
-    if (R + 1 > MPE_ALLOC_STATE_CAP) return fail(c, MPE_ERR_STATE_CAP, "too many states");
-    const size_t need = allocate_choice_bytes(E, R);
+    if (exact && R + 1 > MPE_ALLOC_STATE_CAP) return fail(c, MPE_ERR_STATE_CAP, "too many states");
+    const size_t need = exact ? allocate_choice_bytes(E, R) : 0;
     if (need > c->choice_cap) {
         cudaFree(c->d_choice);
         CK(cudaMalloc(&c->d_choice, need));
@@ -250,8 +251,12 @@ int run_allocate(mpe_ctx* c, const double* p, uint64_t B, std::vector<uint8_t>& 
     std::memcpy(c->h_p_pinned, p, sizeof(double) * E);
     CK(cudaMemcpyAsync(c->d_p, c->h_p_pinned, sizeof(double) * E, cudaMemcpyHostToDevice,
                        c->stream));
-    launch_allocate(c->stream, c->d_p, c->d_W, E, B, sum_w, g, c->d_bits_out,
-                    c->d_alloc_status, c->d_choice, c->d_D, MPE_ALLOC_STATE_CAP, R);
+    if (exact)
+        launch_allocate(c->stream, c->d_p, c->d_W, E, B, sum_w, g, c->d_bits_out,
+                        c->d_alloc_status, c->d_choice, c->d_D, MPE_ALLOC_STATE_CAP, R);
+    else
+        launch_allocate_proportional(c->stream, c->d_p, c->d_W, E, B, sum_w, c->d_bits_out,
+                                     c->d_alloc_status);
     c->launches++;
     CKLAUNCH();
     CK(cudaMemcpyAsync(c->h_alloc_pinned, c->d_alloc_status, sizeof(int32_t),
@@ -441,6 +446,49 @@ int mpe_allocate_bits(const double* p, const uint64_t* W, int32_t E, uint64_t B_
     }
     cudaFree(dp); cudaFree(dW); cudaFree(db); cudaFree(ds); cudaFree(dch); cudaFree(dD);
     return rc;
+}
+
+int mpe_allocate_bits_proportional(const double* p, const uint64_t* W, int32_t E,
+                                   uint64_t B_bits, uint8_t* bits_out) {
+    if (!p || !W || !bits_out) return fail_global(MPE_ERR_INVALID, "null argument");
+    if (E < 1 || E > MPE_MAX_EXPERTS) return fail_global(MPE_ERR_INVALID, "E out of range");
+    uint64_t sum_w = 0;
+    for (int e = 0; e < E; ++e) {
+        if (W[e] == 0) return fail_global(MPE_ERR_INVALID, "W[%d] = 0", e);
+        if (!(p[e] >= 0.0) || !std::isfinite(p[e]))
+            return fail_global(MPE_ERR_INVALID, "p[%d] must be finite and >= 0", e);
+        sum_w += W[e];
+    }
+    if (B_bits < 3 * sum_w) return fail_global(MPE_ERR_INFEASIBLE, "budget below 3 bits per weight");
+    double* dp = nullptr; uint64_t* dW = nullptr; uint8_t* db = nullptr; int32_t* ds = nullptr;
+    int rc = MPE_OK;
+    int32_t st = -1;
+    auto ok = [](cudaError_t e) { return e == cudaSuccess; };
+    if (!ok(cudaMalloc(&dp, sizeof(double) * E)) || !ok(cudaMalloc(&dW, sizeof(uint64_t) * E)) ||
+        !ok(cudaMalloc(&db, E)) || !ok(cudaMalloc(&ds, sizeof(int32_t))) ||
+        !ok(cudaMemcpy(dp, p, sizeof(double) * E, cudaMemcpyHostToDevice)) ||
+        !ok(cudaMemcpy(dW, W, sizeof(uint64_t) * E, cudaMemcpyHostToDevice))) {
+        rc = fail_global(MPE_ERR_CUDA, "allocate_bits_proportional: %s",
+                         cudaGetErrorString(cudaGetLastError()));
+    } else {
+        launch_allocate_proportional(nullptr, dp, dW, E, B_bits, sum_w, db, ds);
+        if (!ok(cudaGetLastError()) || !ok(cudaMemcpy(&st, ds, sizeof(int32_t), cudaMemcpyDeviceToHost)) ||
+            !ok(cudaMemcpy(bits_out, db, E, cudaMemcpyDeviceToHost)))
+            rc = fail_global(MPE_ERR_CUDA, "allocate_bits_proportional kernel: %s",
+                             cudaGetErrorString(cudaGetLastError()));
+        else if (st == 1)
+            rc = fail_global(MPE_ERR_INFEASIBLE, "budget below 3 bits per weight");
+    }
+    cudaFree(dp); cudaFree(dW); cudaFree(db); cudaFree(ds);
+    return rc;
+}
+
+int mpe_set_allocator(mpe_ctx* c, int32_t allocator) {
+    if (!c) return fail_global(MPE_ERR_INVALID, "null context");
+    if (allocator != MPE_ALLOCATOR_EXACT && allocator != MPE_ALLOCATOR_PROPORTIONAL)
+        return fail(c, MPE_ERR_INVALID, "bad allocator %d", allocator);
+    c->allocator = allocator;
+    return MPE_OK;
 }
 
 int mpe_quantize_experts(mpe_ctx* c, const void* const* master_f16, const uint8_t* bits) {

@@ -67,6 +67,7 @@ struct mpe_ctx {
     uint32_t page_bytes = MPE_DEFAULT_PAGE_BYTES;
     uint32_t pool_pages = 0;
     int path = MPE_PATH_AUTO;
+    int allocator = MPE_ALLOCATOR_EXACT;   // the width rule repage uses
     cudaStream_t stream = nullptr;
     std::string err;
     uint64_t launches = 0;
@@ -151,6 +152,9 @@ void launch_allocate(cudaStream_t st, const double* p, const uint64_t* W, int E,
                      uint8_t* choice, double* D, int state_cap, uint64_t R);
 // bytes of the global choice table for E experts and R budget units
 size_t allocate_choice_bytes(int E, uint64_t R);
+// the page's proportional rule with a budget repair (status 1: infeasible)
+void launch_allocate_proportional(cudaStream_t st, const double* p, const uint64_t* W, int E,
+                                  uint64_t B, uint64_t sum_w, uint8_t* bits_out, int32_t* status);
 
 // route.cu
 void launch_route(mpe_ctx* c, const int32_t* ids, int Tk, int k, int32_t* perm,

@@ -187,3 +187,60 @@ def test_pool_exhaustion_is_transactional():
     assert np.array_equal(pte0, pte1) and np.array_equal(pidx0, pidx1)
     assert all(np.array_equal(a, ctx.expert_stream(e)) for e, a in enumerate(s0))
     assert list(ctx.bits()) == [3, 3, 3, 3]
+
+
+# ----------------------------------------------------------------------------
+# the page's proportional allocator (+ budget repair): a selectable width rule
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("seed", range(8))
+def test_allocate_bits_proportional_small(seed):
+    rng = np.random.default_rng(100 + seed)
+    E = int(rng.integers(1, 40))
+    p = rng.dirichlet(np.full(E, 0.5))
+    W = [int(x) * 128 for x in rng.integers(1, 50, size=E)]
+    B = int(rng.integers(3 * sum(W), 9 * sum(W)))
+    got = mpe.allocate_bits_proportional(p, W, B)
+    assert np.array_equal(got, oa.allocate_bits_proportional(p, W, B))
+
+
+@pytest.mark.parametrize("cfg,avg", [(1, 4.5), (2, 4.5), (3, 3.5), (5, 8.0), (5, 6.0), (5, 3.0)])
+def test_allocate_bits_proportional_workloads(cfg, avg):
+    wl = synth.WORKLOADS[cfg]
+    p = synth.importance(wl)
+    W = [wl.W_e] * wl.E
+    B = synth.budget_for(wl, avg)
+    got = mpe.allocate_bits_proportional(p, W, B)
+    assert np.array_equal(got, oa.allocate_bits_proportional(p, W, B))
+    assert sum(int(b) * w for b, w in zip(got, W)) <= B
+
+
+def test_allocate_bits_proportional_errors():
+    with pytest.raises(mpe.MpeError) as ei:
+        mpe.allocate_bits_proportional([1.0, 1.0], [7, 11], 3 * 18 - 1)
+    assert ei.value.code == -2
+    # all-zero importances: every expert at 3 bits
+    assert list(mpe.allocate_bits_proportional([0.0, 0.0, 0.0], [5, 5, 5], 100)) == [3, 3, 3]
+
+
+def test_repage_with_proportional_allocator():
+    wl = synth.scaled(synth.WORKLOADS[1], E=8, H=256, F=256)
+    p = synth.importance(wl)
+    W = [wl.W_e] * wl.E
+    masters = [synth.expert_weights(wl, e, device="cuda") for e in range(wl.E)]
+    cpu = [m.cpu().numpy() for m in masters]
+    pool = wl.E * op.pages_needed(8, wl.H, wl.F)
+    ctx = mpe.Context(wl.E, wl.H, wl.F, pool_pages=pool)
+    ctx.set_allocator(mpe.ALLOCATOR_PROPORTIONAL)
+    alloc = op.PageAllocator(pool, wl.E, wl.H, wl.F)
+    bits0 = oa.allocate_bits_proportional(p, W, synth.budget_for(wl, 8.0))
+    ctx.quantize_experts(masters, bits0)
+    alloc.place(bits0)
+    for avg in [6.0, 4.0, 3.0, 5.0]:
+        B = synth.budget_for(wl, avg)
+        n = ctx.repage(B, p)
+        nb = oa.allocate_bits_proportional(p, W, B)
+        assert n == len(alloc.repage(nb))
+        assert np.array_equal(ctx.bits(), nb)
+        _check_expert_state(ctx, wl, nb, cpu, alloc)
+    with pytest.raises(mpe.MpeError):
+        ctx.set_allocator(7)
