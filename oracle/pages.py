@@ -21,6 +21,11 @@ Readings taken (listed in the design doc):
 * Page table: per expert (bits, first, n_pages); first indexes one compact
   page-index array that lists each expert's pages in stream order, experts
   in ascending order.
+* Overlapped repage (the scheduler changes precision while decode goes on):
+  the changed experts keep their old pages readable until a commit, so their
+  new pages come from the pages free at the call (lowest index first,
+  ascending e); the old pages return to the pool at the commit. Transactional
+  as well; one overlapped repage at a time.
 """
 from __future__ import annotations
 
@@ -65,6 +70,7 @@ class PageAllocator:
         self.free = np.ones(pool_pages, dtype=bool)
         self.pages: list[list[int]] = [[] for _ in range(E)]
         self.bits = np.zeros(E, dtype=np.uint8)
+        self.pending_release: list[int] | None = None
 
     def _take(self, free: np.ndarray, n: int) -> list[int]:
         idx = np.flatnonzero(free)[:n]
@@ -92,6 +98,34 @@ class PageAllocator:
         self.pages = pages
         self.bits = new_bits.copy()
         return changed
+
+    def repage_overlapped(self, new_bits) -> list[int]:
+        """Repage while the old pages stay in use: new pages for the changed
+        experts from the currently free pages; the old ones are released by
+        commit(). Returns the changed experts (the table shows the new pages)."""
+        if self.pending_release is not None:
+            raise RuntimeError("an overlapped repage is pending: commit it first")
+        new_bits = np.asarray(new_bits, dtype=np.uint8)
+        changed = [e for e in range(self.E) if int(new_bits[e]) != int(self.bits[e])]
+        free = self.free.copy()
+        pages = [list(p) for p in self.pages]
+        released: list[int] = []
+        for e in changed:
+            n = pages_needed(int(new_bits[e]), self.H, self.F, self.page_bytes)
+            new_pages = self._take(free, n)
+            released.extend(pages[e])
+            pages[e] = new_pages
+        self.free = free
+        self.pages = pages
+        self.bits = new_bits.copy()
+        self.pending_release = released
+        return changed
+
+    def commit(self) -> None:
+        """Release the old pages of the last overlapped repage."""
+        if self.pending_release:
+            self.free[self.pending_release] = True
+        self.pending_release = None
 
     def table(self) -> PageTable:
         first = np.zeros(self.E, dtype=np.uint32)

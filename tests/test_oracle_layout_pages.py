@@ -209,3 +209,46 @@ def test_place_and_gather_stream():
     P.place_stream(pool, [2], stream, b)
     assert np.array_equal(P.gather_stream(pool, [2], nch, b), stream)
     assert np.all(pool[:2 * 65536] == 0)
+
+
+def test_overlapped_repage_keeps_old_pages_until_commit():
+    H, F = 256, 256
+    E = 4
+    need8 = P.pages_needed(8, H, F)
+    need3 = P.pages_needed(3, H, F)
+    A = P.PageAllocator(E * need8 + 2 * need3, E, H, F)
+    A.place(np.array([8, 8, 8, 8], np.uint8))
+    old = [list(x) for x in A.pages]
+    changed = A.repage_overlapped(np.array([3, 8, 3, 8], np.uint8))
+    assert changed == [0, 2]
+    # unchanged experts keep their pages; new pages avoid every old page
+    assert A.pages[1] == old[1] and A.pages[3] == old[3]
+    in_use_before = set(p for x in old for p in x)
+    assert not (set(A.pages[0]) | set(A.pages[2])) & in_use_before
+    # lowest free pages first, ascending e: right after the 8-bit experts
+    assert A.pages[0] == list(range(E * need8, E * need8 + need3))
+    assert A.pages[2] == list(range(E * need8 + need3, E * need8 + 2 * need3))
+    # old pages stay allocated until the commit
+    assert A.used() == E * need8 + 2 * need3
+    with pytest.raises(RuntimeError):
+        A.repage_overlapped(np.array([3, 3, 3, 3], np.uint8))
+    A.commit()
+    assert A.used() == 2 * need8 + 2 * need3
+    assert all(A.free[p] for p in old[0] + old[2])
+    # after the commit the freed pages are reused, lowest first
+    A.repage_overlapped(np.array([3, 3, 3, 8], np.uint8))
+    assert A.pages[1] == list(range(need3))
+    A.commit()
+
+
+def test_overlapped_repage_is_transactional():
+    H, F = 256, 256
+    need8 = P.pages_needed(8, H, F)
+    A = P.PageAllocator(2 * need8, 2, H, F)
+    A.place(np.array([8, 8], np.uint8))
+    t0 = A.table()
+    with pytest.raises(P.PoolExhausted):
+        A.repage_overlapped(np.array([4, 8], np.uint8))  # no free page for the new ones
+    t1 = A.table()
+    assert np.array_equal(t0.page_idx, t1.page_idx) and list(A.bits) == [8, 8]
+    assert A.pending_release is None
