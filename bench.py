@@ -521,7 +521,10 @@ def run_repage_schedule(args, dist: Dist):
         masters.append(t)
     p = synth.importance(wl)
     W = [wl.W_e] * E
-    ctx = mpe.Context(E, H, F)
+    # a quarter of headroom beside the all-8-bit pages: the overlapped repage
+    # keeps the changed experts' old pages until its commit
+    pages8 = -(-3 * (F // 16) * (H // 128) // (65536 // (256 * 8)))
+    ctx = mpe.Context(E, H, F, pool_pages=(5 * E * pages8) // 4)
     peaks, peak_kind = measured_peaks()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
 
@@ -582,6 +585,43 @@ def run_repage_schedule(args, dist: Dist):
     rp_bytes = sum(r["GB/s"] * r["ms"] / 1e3 * 1e9 for r in moved)
     rp_ms = sum(r["ms"] for r in moved)
 
+    # a budget change while decode batches are served: synchronous repage then
+    # the batches, against the overlapped repage (forward passes keep the old
+    # pages until the commit); device time from the first call to the commit
+    overlap = None
+    x_l, ids_l, w_l = last
+    idt_l, wt_l = torch.from_numpy(ids_l).cuda(), torch.from_numpy(w_l).cuda()
+    n_dec = 5
+    ev_first = torch.cuda.Event(enable_timing=True)
+    try:
+        res = {"sequential": [], "overlapped": []}
+        first = {"sequential": [], "overlapped": []}
+        for mode in ("sequential", "overlapped", "sequential", "overlapped"):
+            for avg in (4.5, 6.0):
+                torch.cuda.synchronize()
+                ev0.record()
+                if mode == "sequential":
+                    ctx.repage(synth.budget_for(wl, avg), p)
+                else:
+                    ctx.repage_async(synth.budget_for(wl, avg), p)
+                for i in range(n_dec):
+                    ctx.moe_ffn(x_l, idt_l, wt_l, out)
+                    if i == 0:
+                        ev_first.record()
+                if mode == "overlapped":
+                    ctx.repage_commit(wait=True)
+                ev1.record()
+                torch.cuda.synchronize()
+                res[mode].append(ev0.elapsed_time(ev1))
+                first[mode].append(ev0.elapsed_time(ev_first))
+        overlap = {"decode_batches": n_dec, "budget_changes": "6 -> 4.5 -> 6 avg bits, twice",
+                   "sequential_ms": float(np.median(res["sequential"])),
+                   "overlapped_ms": float(np.median(res["overlapped"])),
+                   "first_batch_sequential_ms": float(np.median(first["sequential"])),
+                   "first_batch_overlapped_ms": float(np.median(first["overlapped"]))}
+    except mpe.MpeError as err:
+        overlap = {"unavailable": str(err)}
+
     # end to end: the last decode batch through the host-buffer entry point
     x, ids, w = last
     xh, ih = x.cpu().pin_memory(), torch.from_numpy(ids).pin_memory()
@@ -625,6 +665,7 @@ def run_repage_schedule(args, dist: Dist):
         "repage_total": {"ms": rp_ms, "GB/s": rp_bytes / (rp_ms / 1e3) / 1e9 if rp_ms else None,
                          "frac": rp_bytes / (rp_ms / 1e3) / 1e9 / peaks["hbm_gbs"] if rp_ms else None},
         "repage": repages,
+        "repage_overlap": overlap,
         "decode": decode,
         "gpu_launches": launches,
         "clocks": clk,

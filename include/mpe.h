@@ -182,6 +182,34 @@ int mpe_quantize_experts(mpe_ctx* ctx, const void* const* master_f16, const uint
 int mpe_repage(mpe_ctx* ctx, uint64_t B_bits, const double* p, int32_t* n_changed_out);
 
 /*
+ * mpe_repage_async -- the same budget change overlapped with serving: the new
+ * widths come from the context's width rule as in mpe_repage, but the changed
+ * experts' old pages stay in use -- mpe_moe_ffn keeps reading the current page
+ * table -- while the new page table is prepared and the changed experts are
+ * re-encoded into pages that are free now (lowest first, ascending e) on an
+ * internal stream of the context. The switch happens at mpe_repage_commit,
+ * which also returns the old pages to the pool.
+ *   B_bits, p, n_changed_out   as for mpe_repage
+ * Synchronises the internal stream once (the widths); the encode is
+ * asynchronous. The pool needs free pages for the changed experts' new pages
+ * beside the old ones: MPE_ERR_POOL (nothing changed) otherwise.
+ * MPE_ERR_ORDER if a previous overlapped repage is not committed. Until the
+ * commit, mpe_get_bits reports the new widths; mpe_quantize_experts,
+ * mpe_repage, mpe_get_page_table, mpe_get_scales and mpe_read_expert_packed
+ * commit first (waiting on the device, not the host).
+ */
+int mpe_repage_async(mpe_ctx* ctx, uint64_t B_bits, const double* p, int32_t* n_changed_out);
+
+/*
+ * mpe_repage_commit -- switch later work to the page table of the pending
+ * overlapped repage. wait = 0: only if its device work has finished
+ * (*committed = 0 otherwise, nothing changes); wait != 0: always -- later work
+ * on the context stream is ordered after that device work (the host does not
+ * block). *committed (host, may be NULL) = 1 when no repage is pending.
+ */
+int mpe_repage_commit(mpe_ctx* ctx, int32_t wait, int32_t* committed);
+
+/*
  * mpe_moe_ffn -- the routed expert SwiGLU FFN run from the pages ("Dynamic
  * Paging"): bucket the T*k (token, slot) assignments by expert, then for each
  * expert with tokens, stream its pages through the page table, unpack and

@@ -37,7 +37,8 @@ MAX_EXPERTS = 1024
 # every symbol include/mpe.h declares
 EXPORTS = [
     "mpe_create", "mpe_destroy", "mpe_set_stream", "mpe_set_path", "mpe_allocate_bits",
-    "mpe_allocate_bits_proportional", "mpe_set_allocator",
+    "mpe_allocate_bits_proportional", "mpe_set_allocator", "mpe_repage_async",
+    "mpe_repage_commit",
     "mpe_quantize_experts", "mpe_repage", "mpe_moe_ffn", "mpe_moe_ffn_host", "mpe_route",
     "mpe_get_page_table", "mpe_expert_stream_bytes", "mpe_read_expert_packed",
     "mpe_get_scales", "mpe_get_bits", "mpe_get_status", "mpe_last_error",
@@ -92,6 +93,8 @@ def lib() -> ctypes.CDLL:
         "mpe_allocate_bits": (i32, [vp, vp, i32, u64, vp]),
         "mpe_allocate_bits_proportional": (i32, [vp, vp, i32, u64, vp]),
         "mpe_set_allocator": (i32, [vp, i32]),
+        "mpe_repage_async": (i32, [vp, u64, vp, vp]),
+        "mpe_repage_commit": (i32, [vp, i32, vp]),
         "mpe_quantize_experts": (i32, [vp, vp, vp]),
         "mpe_repage": (i32, [vp, u64, vp, vp]),
         "mpe_moe_ffn": (i32, [vp, vp, i32, vp, vp, i32, vp]),
@@ -219,6 +222,22 @@ class Context:
         n = ctypes.c_int32(0)
         _check(lib().mpe_repage(self._h, int(B), _ptr(p), ctypes.byref(n)), self._h)
         return n.value
+
+    def repage_async(self, B: int, p) -> int:
+        """Start an overlapped repage (forward passes keep the current pages
+        until repage_commit); returns the number of experts changed."""
+        self._sync_stream()
+        p = np.ascontiguousarray(p, dtype=np.float64)
+        n = ctypes.c_int32(0)
+        _check(lib().mpe_repage_async(self._h, int(B), _ptr(p), ctypes.byref(n)), self._h)
+        return n.value
+
+    def repage_commit(self, wait: bool = True) -> bool:
+        """Switch to the pending repage's pages (wait=False: only if ready)."""
+        self._sync_stream()
+        done = ctypes.c_int32(0)
+        _check(lib().mpe_repage_commit(self._h, 1 if wait else 0, ctypes.byref(done)), self._h)
+        return bool(done.value)
 
     def moe_ffn(self, x, ids, w, out=None):
         import torch

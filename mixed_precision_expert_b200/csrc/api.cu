@@ -118,11 +118,75 @@ void commit_pages(mpe_ctx* c, PagePlan& plan, const std::vector<uint8_t>& new_bi
     c->bits = new_bits;
 }
 
+// Overlapped repage plan: the changed experts' old pages stay allocated (work
+// on the current page table still reads them), their new pages come from the
+// pages free now (lowest first, ascending e); `release` lists the old pages,
+// returned to the pool at the commit. Transactional like plan_pages.
+bool plan_pages_overlapped(const mpe_ctx* c, const std::vector<uint8_t>& new_bits,
+                           PagePlan& plan, std::vector<int>& changed,
+                           std::vector<uint32_t>& release) {
+    changed.clear();
+    release.clear();
+    for (int e = 0; e < c->E; ++e)
+        if (new_bits[e] != c->bits[e]) changed.push_back(e);
+    plan.free = c->alloc.free;
+    plan.moved.clear();
+    uint32_t cursor = 0;
+    for (int e : changed) {
+        const int need = pages_needed(new_bits[e], c->H, c->F, c->page_bytes);
+        std::vector<uint32_t> pg;
+        pg.reserve(need);
+        for (int i = 0; i < need; ++i) {
+            while (cursor < c->pool_pages && !plan.free[cursor]) ++cursor;
+            if (cursor >= c->pool_pages) return false;
+            plan.free[cursor] = 0;
+            pg.push_back(cursor);
+        }
+        release.insert(release.end(), c->alloc.pages[e].begin(), c->alloc.pages[e].end());
+        plan.moved.emplace_back(e, std::move(pg));
+    }
+    return true;
+}
+
+// Side stream, events and the second page table, made on the first
+// overlapped repage.
+int ensure_side(mpe_ctx* c) {
+    if (c->side) return MPE_OK;
+    CK(cudaStreamCreateWithFlags(&c->side, cudaStreamNonBlocking));
+    CK(cudaEventCreateWithFlags(&c->side_done, cudaEventDisableTiming));
+    CK(cudaEventCreateWithFlags(&c->old_table_free, cudaEventDisableTiming));
+    CK(cudaEventRecord(c->old_table_free, c->stream));
+    CK(cudaMalloc(&c->d_pte_next, sizeof(Pte) * c->E));
+    CK(cudaMalloc(&c->d_pidx_next, sizeof(uint32_t) * c->pool_pages));
+    CK(cudaMalloc(&c->d_list_next, sizeof(int32_t) * c->E));
+    CK(cudaMallocHost(&c->h_pte_next_pinned, sizeof(Pte) * c->E));
+    CK(cudaMallocHost(&c->h_pidx_next_pinned, sizeof(uint32_t) * c->pool_pages));
+    CK(cudaMallocHost(&c->h_list_next_pinned, sizeof(int32_t) * c->E));
+    return MPE_OK;
+}
+
+// Switch to the prepared page table: later work on the context stream waits
+// for the side stream's encode; the old pages return to the pool, and the
+// next overlapped repage will not write them before the work launched so far
+// (which may read them) has finished.
+int commit_pending(mpe_ctx* c) {
+    if (!c->pending) return MPE_OK;
+    CK(cudaStreamWaitEvent(c->stream, c->side_done, 0));
+    std::swap(c->d_pte, c->d_pte_next);
+    std::swap(c->d_pidx, c->d_pidx_next);
+    c->pidx_count = c->pidx_count_next;
+    for (uint32_t pg : c->pending_release) c->alloc.free[pg] = 1;
+    c->pending_release.clear();
+    CK(cudaEventRecord(c->old_table_free, c->stream));
+    c->pending = false;
+    return MPE_OK;
+}
+
 // Rebuild the page table (compact page-index array, experts in order) in the
 // pinned staging and upload it (async; the staging is reused only after the
 // previous upload finished).
-int upload_table(mpe_ctx* c) {
-    CK(cudaEventSynchronize(c->upload_done));
+// The page table of the allocator's current state into host staging.
+uint32_t fill_table(mpe_ctx* c, Pte* h_pte, uint32_t* h_pidx) {
     uint32_t n = 0;
     for (int e = 0; e < c->E; ++e) {
         Pte& p = c->pte[e];
@@ -130,11 +194,17 @@ int upload_table(mpe_ctx* c) {
         p.bits = c->bits[e];
         p.first = n;
         p.n_pages = (uint32_t)pg.size();
-        if (!pg.empty()) std::memcpy(c->h_pidx_pinned + n, pg.data(), sizeof(uint32_t) * pg.size());
+        if (!pg.empty()) std::memcpy(h_pidx + n, pg.data(), sizeof(uint32_t) * pg.size());
         n += (uint32_t)pg.size();
     }
+    std::memcpy(h_pte, c->pte.data(), sizeof(Pte) * c->E);
+    return n;
+}
+
+int upload_table(mpe_ctx* c) {
+    CK(cudaEventSynchronize(c->upload_done));
+    const uint32_t n = fill_table(c, c->h_pte_pinned, c->h_pidx_pinned);
     c->pidx_count = n;
-    std::memcpy(c->h_pte_pinned, c->pte.data(), sizeof(Pte) * c->E);
     CK(cudaMemcpyAsync(c->d_pte, c->h_pte_pinned, sizeof(Pte) * c->E, cudaMemcpyHostToDevice,
                        c->stream));
     if (n)
@@ -221,7 +291,8 @@ int ensure_stage(mpe_ctx* c, int T, int k) {
 
 // Run the allocator kernel on the context's stream and fetch the widths
 // (pinned staging; the expert sizes are uploaded once).
-int run_allocate(mpe_ctx* c, const double* p, uint64_t B, std::vector<uint8_t>& out) {
+int run_allocate(mpe_ctx* c, const double* p, uint64_t B, std::vector<uint8_t>& out,
+                 cudaStream_t st) {
     const int E = c->E;
     for (int e = 0; e < E; ++e)
         if (!(p[e] >= 0.0) || !std::isfinite(p[e]))
@@ -244,29 +315,29 @@ int run_allocate(mpe_ctx* c, const double* p, uint64_t B, std::vector<uint8_t>& 
     if (!c->w_uploaded) {
         for (int e = 0; e < E; ++e) c->h_w_pinned[e] = w_e;
         CK(cudaMemcpyAsync(c->d_W, c->h_w_pinned, sizeof(uint64_t) * E, cudaMemcpyHostToDevice,
-                           c->stream));
+                           st));
         c->w_uploaded = true;
     }
     // the staging is free: the previous call ended with a synchronize
     std::memcpy(c->h_p_pinned, p, sizeof(double) * E);
     CK(cudaMemcpyAsync(c->d_p, c->h_p_pinned, sizeof(double) * E, cudaMemcpyHostToDevice,
-                       c->stream));
+                       st));
     if (exact)
-        launch_allocate(c->stream, c->d_p, c->d_W, E, B, sum_w, g, c->d_bits_out,
+        launch_allocate(st, c->d_p, c->d_W, E, B, sum_w, g, c->d_bits_out,
                         c->d_alloc_status, c->d_choice, c->d_D, MPE_ALLOC_STATE_CAP, R);
     else
-        launch_allocate_proportional(c->stream, c->d_p, c->d_W, E, B, sum_w, c->d_bits_out,
+        launch_allocate_proportional(st, c->d_p, c->d_W, E, B, sum_w, c->d_bits_out,
                                      c->d_alloc_status);
     c->launches++;
     CKLAUNCH();
     CK(cudaMemcpyAsync(c->h_alloc_pinned, c->d_alloc_status, sizeof(int32_t),
-                       cudaMemcpyDeviceToHost, c->stream));
+                       cudaMemcpyDeviceToHost, st));
     CK(cudaMemcpyAsync(c->h_alloc_pinned + 1, c->d_bits_out, E, cudaMemcpyDeviceToHost,
-                       c->stream));
-    CK(cudaStreamSynchronize(c->stream));
-    const int32_t st = c->h_alloc_pinned[0];
-    if (st == 1) return fail(c, MPE_ERR_INFEASIBLE, "budget below 3 bits per weight");
-    if (st == 3) return fail(c, MPE_ERR_STATE_CAP, "too many allocation states");
+                       st));
+    CK(cudaStreamSynchronize(st));
+    const int32_t status = c->h_alloc_pinned[0];
+    if (status == 1) return fail(c, MPE_ERR_INFEASIBLE, "budget below 3 bits per weight");
+    if (status == 3) return fail(c, MPE_ERR_STATE_CAP, "too many allocation states");
     const uint8_t* bits = reinterpret_cast<const uint8_t*>(c->h_alloc_pinned + 1);
     out.assign(bits, bits + E);
     return MPE_OK;
@@ -371,6 +442,15 @@ void mpe_destroy(mpe_ctx* c) {
     {
         DeviceGuard guard(c->device);
         cudaStreamSynchronize(c->stream);
+        if (c->side) {
+            cudaStreamSynchronize(c->side);
+            cudaStreamDestroy(c->side);
+            cudaEventDestroy(c->side_done);
+            cudaEventDestroy(c->old_table_free);
+            cudaFree(c->d_pte_next); cudaFree(c->d_pidx_next); cudaFree(c->d_list_next);
+            cudaFreeHost(c->h_pte_next_pinned); cudaFreeHost(c->h_pidx_next_pinned);
+            cudaFreeHost(c->h_list_next_pinned);
+        }
         free_scratch(c->s);
         cudaFree(c->pool); cudaFree(c->d_pte); cudaFree(c->d_pidx); cudaFree(c->d_absmax);
         cudaFree(c->d_status); cudaFree(c->d_masters); cudaFree(c->d_list); cudaFree(c->d_p);
@@ -500,6 +580,8 @@ int mpe_quantize_experts(mpe_ctx* c, const void* const* master_f16, const uint8_
             return fail(c, MPE_ERR_INVALID, "master[%d] null or not 16-byte aligned", e);
     }
     DeviceGuard guard(c->device);
+    int r0;
+    if ((r0 = commit_pending(c))) return r0;
     std::vector<uint8_t> nb(bits, bits + c->E);
     PagePlan plan;
     std::vector<int> changed;
@@ -534,7 +616,8 @@ int mpe_repage(mpe_ctx* c, uint64_t B_bits, const double* p, int32_t* n_changed_
     DeviceGuard guard(c->device);
     std::vector<uint8_t> nb;
     int r;
-    if ((r = run_allocate(c, p, B_bits, nb))) return r;
+    if ((r = commit_pending(c))) return r;
+    if ((r = run_allocate(c, p, B_bits, nb, c->stream))) return r;
     PagePlan plan;
     std::vector<int> changed;
     if (!plan_pages(c, nb, plan, changed)) return fail(c, MPE_ERR_POOL, "page pool exhausted");
@@ -547,6 +630,69 @@ int mpe_repage(mpe_ctx* c, uint64_t B_bits, const double* p, int32_t* n_changed_
     }
     CKLAUNCH();
     if (n_changed_out) *n_changed_out = (int32_t)changed.size();
+    return MPE_OK;
+}
+
+int mpe_repage_async(mpe_ctx* c, uint64_t B_bits, const double* p, int32_t* n_changed_out) {
+    if (!c) return fail_global(MPE_ERR_INVALID, "null context");
+    if (!p) return fail(c, MPE_ERR_INVALID, "null importances");
+    if (!c->absmax_valid) return fail(c, MPE_ERR_ORDER, "repage before quantize_experts");
+    if (c->pending) return fail(c, MPE_ERR_ORDER, "an overlapped repage is pending: commit it");
+    DeviceGuard guard(c->device);
+    int r;
+    if ((r = ensure_side(c))) return r;
+    std::vector<uint8_t> nb;
+    if ((r = run_allocate(c, p, B_bits, nb, c->side))) return r;
+    PagePlan plan;
+    std::vector<int> changed;
+    std::vector<uint32_t> release;
+    if (!plan_pages_overlapped(c, nb, plan, changed, release))
+        return fail(c, MPE_ERR_POOL, "page pool exhausted (an overlapped repage needs free "
+                                     "pages for the changed experts' new pages)");
+    commit_pages(c, plan, nb);
+    // the next table (run_allocate synchronised the side stream, so its
+    // staging is free)
+    c->pidx_count_next = fill_table(c, c->h_pte_next_pinned, c->h_pidx_next_pinned);
+    CK(cudaMemcpyAsync(c->d_pte_next, c->h_pte_next_pinned, sizeof(Pte) * c->E,
+                       cudaMemcpyHostToDevice, c->side));
+    if (c->pidx_count_next)
+        CK(cudaMemcpyAsync(c->d_pidx_next, c->h_pidx_next_pinned,
+                           sizeof(uint32_t) * c->pidx_count_next, cudaMemcpyHostToDevice,
+                           c->side));
+    // pages freed by the last commit may still be read by work launched before it
+    CK(cudaStreamWaitEvent(c->side, c->old_table_free, 0));
+    launch_scales_on(c, c->d_pte_next, c->side);
+    if (!changed.empty()) {
+        for (size_t i = 0; i < changed.size(); ++i) c->h_list_next_pinned[i] = changed[i];
+        CK(cudaMemcpyAsync(c->d_list_next, c->h_list_next_pinned, sizeof(int32_t) * changed.size(),
+                           cudaMemcpyHostToDevice, c->side));
+        PagedExperts P = paged(c);
+        P.pte = c->d_pte_next;
+        P.pidx = c->d_pidx_next;
+        launch_encode_on(c, P, c->d_list_next, (int)changed.size(), c->side);
+    }
+    CKLAUNCH();
+    CK(cudaEventRecord(c->side_done, c->side));
+    c->pending_release = std::move(release);
+    c->pending = true;
+    if (n_changed_out) *n_changed_out = (int32_t)changed.size();
+    return MPE_OK;
+}
+
+int mpe_repage_commit(mpe_ctx* c, int32_t wait, int32_t* committed) {
+    if (!c) return fail_global(MPE_ERR_INVALID, "null context");
+    DeviceGuard guard(c->device);
+    if (c->pending && !wait) {
+        const cudaError_t q = cudaEventQuery(c->side_done);
+        if (q == cudaErrorNotReady) {
+            if (committed) *committed = 0;
+            return MPE_OK;
+        }
+        if (q != cudaSuccess) return fail(c, MPE_ERR_CUDA, "%s", cudaGetErrorString(q));
+    }
+    int r;
+    if ((r = commit_pending(c))) return r;
+    if (committed) *committed = 1;
     return MPE_OK;
 }
 
@@ -738,6 +884,8 @@ int mpe_route(mpe_ctx* c, const int32_t* ids, int32_t T, int32_t k, int32_t* per
 int mpe_get_page_table(mpe_ctx* c, mpe_pte* pte_host, uint32_t* page_idx_host, size_t cap) {
     if (!c) return fail_global(MPE_ERR_INVALID, "null context");
     DeviceGuard guard(c->device);
+    int rc;
+    if ((rc = commit_pending(c))) return rc;
     CK(cudaStreamSynchronize(c->stream));
     if (pte_host) CK(cudaMemcpy(pte_host, c->d_pte, sizeof(Pte) * c->E, cudaMemcpyDeviceToHost));
     if (page_idx_host) {
@@ -762,6 +910,10 @@ int mpe_read_expert_packed(mpe_ctx* c, int32_t e, void* host_dst, size_t bytes) 
     if (n == 0) return fail(c, MPE_ERR_ORDER, "expert %d not quantized", e);
     if (bytes < n) return fail(c, MPE_ERR_INVALID, "buffer %zu < stream %zu", bytes, n);
     DeviceGuard guard(c->device);
+    {
+        const int rc = commit_pending(c);
+        if (rc) return rc;
+    }
     if (n > c->gather_cap) {
         CK(cudaStreamSynchronize(c->stream));
         cudaFree(c->d_gather);
@@ -779,6 +931,10 @@ int mpe_read_expert_packed(mpe_ctx* c, int32_t e, void* host_dst, size_t bytes) 
 int mpe_get_scales(mpe_ctx* c, float* scale_host, float* absmax_host) {
     if (!c) return fail_global(MPE_ERR_INVALID, "null context");
     DeviceGuard guard(c->device);
+    {
+        const int rc = commit_pending(c);
+        if (rc) return rc;
+    }
     CK(cudaStreamSynchronize(c->stream));
     if (scale_host) {
         std::vector<Pte> p(c->E);

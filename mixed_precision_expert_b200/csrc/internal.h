@@ -109,6 +109,22 @@ struct mpe_ctx {
     mpe::HostAllocator alloc;
     mpe::Scratch s;
 
+    // overlapped repage (mpe_repage_async / mpe_repage_commit): the next page
+    // table is prepared and the changed experts encoded on `side` while work
+    // on `stream` keeps reading the current table
+    cudaStream_t side = nullptr;
+    mpe::Pte* d_pte_next = nullptr;
+    uint32_t* d_pidx_next = nullptr;
+    int32_t* d_list_next = nullptr;
+    mpe::Pte* h_pte_next_pinned = nullptr;
+    uint32_t* h_pidx_next_pinned = nullptr;
+    int32_t* h_list_next_pinned = nullptr;
+    uint32_t pidx_count_next = 0;
+    cudaEvent_t side_done = nullptr;        // the pending repage's device work finished
+    cudaEvent_t old_table_free = nullptr;   // work launched before the last commit finished
+    bool pending = false;
+    std::vector<uint32_t> pending_release;  // old pages of the changed experts
+
     // tracing
     bool profiling = false;
     std::vector<mpe::ProfileRecord> prof;
@@ -142,6 +158,10 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 void launch_absmax(mpe_ctx* c, const int32_t* d_list, int n_list);
 void launch_scales(mpe_ctx* c);
 void launch_encode(mpe_ctx* c, const int32_t* d_list, int n_list);
+// the same on an explicit page table / stream (overlapped repage)
+void launch_scales_on(mpe_ctx* c, Pte* pte, cudaStream_t st);
+void launch_encode_on(mpe_ctx* c, const PagedExperts& P, const int32_t* d_list, int n_list,
+                      cudaStream_t st);
 void launch_gather_stream(mpe_ctx* c, int e, uint8_t* dst);
 
 // allocate.cu

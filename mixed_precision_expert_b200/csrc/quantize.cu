@@ -290,16 +290,23 @@ void launch_absmax(mpe_ctx* c, const int32_t* d_list, int n_list) {
     c->launches++;
 }
 
-void launch_scales(mpe_ctx* c) {
-    k_scales<<<(c->E + 127) / 128, 128, 0, c->stream>>>(c->d_pte, c->d_absmax, c->E, c->d_status);
+void launch_scales_on(mpe_ctx* c, Pte* pte, cudaStream_t st) {
+    k_scales<<<(c->E + 127) / 128, 128, 0, st>>>(pte, c->d_absmax, c->E, c->d_status);
+    c->launches++;
+}
+
+void launch_scales(mpe_ctx* c) { launch_scales_on(c, c->d_pte, c->stream); }
+
+void launch_encode_on(mpe_ctx* c, const PagedExperts& P, const int32_t* d_list, int n_list,
+                      cudaStream_t st) {
+    const int nc = 3 * chunks_w1(c->H, c->F);
+    dim3 grid((unsigned)((nc + 7) / 8), (unsigned)n_list);
+    k_encode<<<grid, 256, 0, st>>>(P, c->d_masters, d_list);
     c->launches++;
 }
 
 void launch_encode(mpe_ctx* c, const int32_t* d_list, int n_list) {
-    const int nc = 3 * chunks_w1(c->H, c->F);
-    dim3 grid((unsigned)((nc + 7) / 8), (unsigned)n_list);
-    k_encode<<<grid, 256, 0, c->stream>>>(paged(c), c->d_masters, d_list);
-    c->launches++;
+    launch_encode_on(c, paged(c), d_list, n_list, c->stream);
 }
 
 void launch_gather_stream(mpe_ctx* c, int e, uint8_t* dst) {
