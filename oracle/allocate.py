@@ -58,17 +58,36 @@ def allocate_bits(p, W, B: int, state_cap: int = 1 << 22) -> np.ndarray:
     p: float64[E] importances; W: int[E] weight elements (> 0); B: budget in bits.
     Returns uint8[E]. Raises Infeasible or StateCapExceeded.
     """
+    E = len(W)
+    if E > 0 and len(p) == E and all(int(w) > 0 for w in W) and int(B) >= 8 * sum(int(w) for w in W):
+        return np.full(E, 8, dtype=np.uint8)
+    table = np.tile(np.array([loss(b) for b in BIT_OPTIONS], dtype=np.float64), (E, 1))
+    return allocate_bits_table(p, table, W, B, state_cap)
+
+
+def allocate_bits_table(p, L, W, B: int, state_cap: int = 1 << 22) -> np.ndarray:
+    """The same program with a loss per expert and width: minimise
+    sum_e p_e L[e, b_e] under sum b_e W_e <= B, L float64[E, 3] with columns
+    for 3, 4 and 8 bits. With every row (1/9, 1/49, 1/16129) this is
+    allocate_bits; with L[e] the measured quantization error of expert e
+    (quantize.quantization_mse) it is the page's "sensitivity" reading of
+    L_e(b). Each cost p_e * L[e, b] is one float64 multiply.
+    """
     p = np.asarray(p, dtype=np.float64)
+    L = np.asarray(L, dtype=np.float64)
     W = [int(w) for w in W]
     E = len(W)
     if E == 0 or len(p) != E or any(w <= 0 for w in W):
         raise ValueError("need E > 0 experts with W_e > 0 and one p_e each")
+    if L.shape != (E, len(BIT_OPTIONS)):
+        raise ValueError("need one loss row (3, 4, 8 bits) per expert")
     B = int(B)
     sum_w = sum(W)
     if B < 3 * sum_w:
         raise Infeasible(f"B={B} < 3*sum(W)={3 * sum_w}")
-    if B >= 8 * sum_w:
-        return np.full(E, 8, dtype=np.uint8)
+    # a budget of 8 sum W or more caps R at every expert's 3 -> 8 upgrade; the
+    # program then picks each expert's least p_e L[e, b] (all 8 for allocate_bits,
+    # which returns that case before coming here)
     g = 0
     for w in W:
         g = math.gcd(g, w)
@@ -78,7 +97,6 @@ def allocate_bits(p, W, B: int, state_cap: int = 1 << 22) -> np.ndarray:
     if R + 1 > state_cap:
         raise StateCapExceeded(f"{R + 1} states > cap {state_cap}")
 
-    L = {b: loss(b) for b in BIT_OPTIONS}
     inf = math.inf
     D = [0.0] + [inf] * R
     choice = np.zeros((E, R + 1), dtype=np.uint8)
@@ -87,14 +105,14 @@ def allocate_bits(p, W, B: int, state_cap: int = 1 << 22) -> np.ndarray:
         for r in range(R + 1):
             best = inf
             best_b = 0
-            for b in BIT_OPTIONS:
+            for i, b in enumerate(BIT_OPTIONS):
                 rp = r - up[e][b]
                 if rp < 0:
                     continue
                 prev = D[rp]
                 if prev == inf:
                     continue
-                cost = p[e] * L[b]          # float64 multiply
+                cost = p[e] * L[e, i]       # float64 multiply
                 cand = prev + cost          # float64 add
                 if cand < best:
                     best = cand
@@ -123,6 +141,15 @@ def objective(p, bits) -> float:
     total = 0.0
     for pe, b in zip(np.asarray(p, dtype=np.float64), bits):
         total = total + pe * loss(int(b))
+    return total
+
+
+def objective_table(p, L, bits) -> float:
+    """sum_e p_e L[e, b_e], ascending e, float64 multiply then add."""
+    L = np.asarray(L, dtype=np.float64)
+    total = 0.0
+    for e, (pe, b) in enumerate(zip(np.asarray(p, dtype=np.float64), bits)):
+        total = total + pe * L[e, BIT_OPTIONS.index(int(b))]
     return total
 
 

@@ -19,6 +19,8 @@ Codes are stored as offset binary u = k + 2^(b-1).
 """
 from __future__ import annotations
 
+import math
+
 import numpy as np
 
 from .allocate import q_levels
@@ -77,3 +79,35 @@ def quantize_expert(master_fp16, b: int):
     m = absmax(master_fp16)
     s = scale(m, b)
     return m, s, encode(master_fp16, s, b)
+
+
+def quantization_mse(master_fp16, b: int) -> float:
+    """Mean squared quantization error of one expert at b bits,
+    (1/n) sum_i (w_i - Q(w_i))^2 over the expert's n fp16 weights, with the
+    expert's own s and codes (quantize_expert). PagedWeight, "Quality-Aware
+    Quantization", names the mean squared error as its example loss L(b) and
+    ties it to the expert's sensitivity; this is that loss measured on the
+    expert.
+
+    Value: the exact sum of squares rounded once to float64, then divided by
+    n in float64 (a second rounding). Exactness of the sum: w is fp16 and
+    k * s is exact in float64 (8-bit k times 24-bit s), so each error
+    w - k * s is an exact float64 whose bits lie at or above 2^-60 (fp16's
+    smallest step is 2^-24 and s >= 2^-24 / 127 has its last bit at or above
+    2^-55); scaled by 2^60 it is an integer, and the squares are summed as
+    Python integers.
+    """
+    w = np.asarray(master_fp16)
+    assert w.dtype == np.float16
+    n = w.size
+    if n == 0:
+        return 0.0
+    m, s, k = quantize_expert(w, b)
+    err = w.astype(np.float64) - dequantize(k, s)
+    total = 0
+    for e in err.tolist():
+        i = int(math.ldexp(e, 60))
+        assert math.ldexp(float(i), -60) == e  # the scaled error is an integer
+        total += i * i
+    sum_sq = math.ldexp(float(total), -120)  # float(int) rounds to nearest, ties to even
+    return float(np.float64(sum_sq) / np.float64(n))
