@@ -141,11 +141,30 @@ int mpe_allocate_bits(const double* p, const uint64_t* W, int32_t E, uint64_t B_
 int mpe_allocate_bits_proportional(const double* p, const uint64_t* W, int32_t E,
                                    uint64_t B_bits, uint8_t* bits_out);
 
+/*
+ * mpe_allocate_bits_table -- the same exact program with a loss per expert
+ * and width: minimise sum_e p_e loss[e][b_e] subject to sum_e b_e W_e <= B_bits
+ * (PagedWeight, "Quality-Aware Quantization": L(b) is a loss such as the mean
+ * squared error, and experts differ in sensitivity). Each cost is one float64
+ * multiply p_e * loss[e][b]; ties keep the lower width and the lower budget.
+ * Unlike mpe_allocate_bits, a budget of 8 sum W or more is solved too (each
+ * expert then takes its least cost, which need not be 8 bits).
+ *   loss     host, float64[E][3], row e = (loss at 3, 4, 8 bits), finite, >= 0;
+ *            e.g. the output of mpe_measure_loss
+ *   other arguments as for mpe_allocate_bits
+ * Synchronous. Same errors as mpe_allocate_bits.
+ */
+int mpe_allocate_bits_table(const double* p, const double* loss, const uint64_t* W, int32_t E,
+                            uint64_t B_bits, uint8_t* bits_out);
+
 /* width rules mpe_repage can use (mpe_set_allocator) */
 #define MPE_ALLOCATOR_EXACT        0  /* mpe_allocate_bits (default)            */
 #define MPE_ALLOCATOR_PROPORTIONAL 1  /* mpe_allocate_bits_proportional         */
+#define MPE_ALLOCATOR_MEASURED     2  /* mpe_allocate_bits_table with the
+                                         context's mpe_measure_loss values      */
 
-/* mpe_set_allocator -- choose the width rule of later mpe_repage calls. */
+/* mpe_set_allocator -- choose the width rule of later mpe_repage calls
+ * (MPE_ALLOCATOR_MEASURED measures the losses on first use). */
 int mpe_set_allocator(mpe_ctx* ctx, int32_t allocator);
 
 /*
@@ -168,10 +187,25 @@ int mpe_set_allocator(mpe_ctx* ctx, int32_t allocator);
 int mpe_quantize_experts(mpe_ctx* ctx, const void* const* master_f16, const uint8_t* bits);
 
 /*
+ * mpe_measure_loss -- the measured quantization error of every expert at
+ * every width: loss[e][i] = (1/n) sum (w - k s_b)^2 over expert e's n = 3 H F
+ * fp16 master weights, with that width's own scale s_b = RN_f32(m_e / q_b)
+ * and codes k = round-half-even(w / s_b), for b = 3, 4, 8 (i = 0, 1, 2). The
+ * sum of squares is exact (integer arithmetic on the device), rounded once to
+ * float64, then divided by n in float64. A zero expert gives 0, a non-finite
+ * master NaN. Measured once per context (the master is immutable) and kept
+ * for MPE_ALLOCATOR_MEASURED.
+ *   loss_host  host, float64[E][3]
+ * Synchronous. MPE_ERR_ORDER before mpe_quantize_experts.
+ */
+int mpe_measure_loss(mpe_ctx* ctx, double* loss_host);
+
+/*
  * mpe_repage -- budget change with KV-cache occupancy ("Implementation
  * Details"; 0to1log digest: lower precision as the KV cache grows, raise it
  * as it shrinks): re-run the context's width rule (mpe_allocate_bits, or
- * mpe_allocate_bits_proportional after mpe_set_allocator) with B_bits and
+ * mpe_allocate_bits_proportional / the measured-loss program after
+ * mpe_set_allocator) with B_bits and
  * importances p (host float64[E]), release the pages of experts whose width
  * changed, give
  * them new pages and re-encode only those experts from the fp16 master with

@@ -30,15 +30,15 @@ STATUS_BAD_EXPERT_ID = 0x1
 STATUS_NONFINITE = 0x2
 STATUS_WAIT_TIMEOUT = 0x4
 PATH_AUTO, PATH_DECODE, PATH_PREFILL = 0, 1, 2
-ALLOCATOR_EXACT, ALLOCATOR_PROPORTIONAL = 0, 1
+ALLOCATOR_EXACT, ALLOCATOR_PROPORTIONAL, ALLOCATOR_MEASURED = 0, 1, 2
 ALLOC_STATE_CAP = 65536
 MAX_EXPERTS = 1024
 
 # every symbol include/mpe.h declares
 EXPORTS = [
     "mpe_create", "mpe_destroy", "mpe_set_stream", "mpe_set_path", "mpe_allocate_bits",
-    "mpe_allocate_bits_proportional", "mpe_set_allocator", "mpe_repage_async",
-    "mpe_repage_commit",
+    "mpe_allocate_bits_proportional", "mpe_allocate_bits_table", "mpe_set_allocator",
+    "mpe_measure_loss", "mpe_repage_async", "mpe_repage_commit",
     "mpe_quantize_experts", "mpe_repage", "mpe_moe_ffn", "mpe_moe_ffn_host", "mpe_route",
     "mpe_get_page_table", "mpe_expert_stream_bytes", "mpe_read_expert_packed",
     "mpe_get_scales", "mpe_get_bits", "mpe_get_status", "mpe_last_error",
@@ -92,6 +92,8 @@ def lib() -> ctypes.CDLL:
         "mpe_set_path": (i32, [vp, i32]),
         "mpe_allocate_bits": (i32, [vp, vp, i32, u64, vp]),
         "mpe_allocate_bits_proportional": (i32, [vp, vp, i32, u64, vp]),
+        "mpe_allocate_bits_table": (i32, [vp, vp, vp, i32, u64, vp]),
+        "mpe_measure_loss": (i32, [vp, vp]),
         "mpe_set_allocator": (i32, [vp, i32]),
         "mpe_repage_async": (i32, [vp, u64, vp, vp]),
         "mpe_repage_commit": (i32, [vp, i32, vp]),
@@ -163,6 +165,20 @@ def allocate_bits_proportional(p, W, B: int) -> np.ndarray:
     return out
 
 
+def allocate_bits_table(p, loss, W, B: int) -> np.ndarray:
+    """The exact program with a loss per expert and width (float64[E, 3],
+    columns 3, 4, 8 bits), e.g. Context.measure_loss() (device DP)."""
+    p = np.ascontiguousarray(p, dtype=np.float64)
+    loss = np.ascontiguousarray(loss, dtype=np.float64)
+    W = np.ascontiguousarray(W, dtype=np.uint64)
+    if loss.shape != (len(p), 3):
+        raise ValueError("loss must be float64[E, 3]")
+    out = np.zeros(len(p), dtype=np.uint8)
+    _check(lib().mpe_allocate_bits_table(_ptr(p), _ptr(loss), _ptr(W), len(p), int(B),
+                                         _ptr(out)))
+    return out
+
+
 def route_noalloc(ids, E: int, perm, offsets, inv):
     """Bucketing into caller-provided device buffers without any device
     allocation (mpe_route_noalloc); runs on the current stream."""
@@ -204,8 +220,16 @@ class Context:
         _check(lib().mpe_set_path(self._h, path), self._h)
 
     def set_allocator(self, allocator: int):
-        """ALLOCATOR_EXACT (default) or ALLOCATOR_PROPORTIONAL for later repages."""
+        """ALLOCATOR_EXACT (default), ALLOCATOR_PROPORTIONAL or ALLOCATOR_MEASURED
+        for later repages."""
         _check(lib().mpe_set_allocator(self._h, allocator), self._h)
+
+    def measure_loss(self) -> np.ndarray:
+        """float64[E, 3]: each expert's measured quantization MSE at 3, 4, 8 bits."""
+        self._sync_stream()
+        out = np.zeros((self.E, 3), dtype=np.float64)
+        _check(lib().mpe_measure_loss(self._h, _ptr(out)), self._h)
+        return out
 
     def quantize_experts(self, masters, bits):
         """masters: E flat fp16 CUDA tensors (W1 | W3 | W2); bits: uint8[E]."""

@@ -13,6 +13,11 @@
 // minimum; a backtrack recovers the widths. Every product and sum is one
 // correctly rounded float64 operation (no fused multiply-add), so the result
 // is reproducible bit for bit.
+//
+// With a loss table (float64[E][3], widths 3, 4, 8) the cost of expert e at
+// width b is p_e * loss[e][b] instead of p_e * L(b), e.g. the measured mean
+// squared error of each expert's own quantization; the all-8 shortcut for a
+// budget of 8 sum W or more is then not taken (the program itself decides).
 #include "internal.h"
 
 namespace mpe {
@@ -33,8 +38,9 @@ constexpr size_t kAllocSmemMax = 200 * 1024;
 // g = gcd(W) (no serial 64-bit arithmetic on the device).
 template <bool ON_CHIP>
 __global__ void __launch_bounds__(kThreads)
-k_allocate(const double* p, const uint64_t* W, int E, uint64_t B, uint64_t sum_w, uint64_t g,
-           uint8_t* bits, int32_t* status, uint8_t* choice, double* D, int state_cap) {
+k_allocate(const double* p, const double* loss, const uint64_t* W, int E, uint64_t B,
+           uint64_t sum_w, uint64_t g, uint8_t* bits, int32_t* status, uint8_t* choice, double* D,
+           int state_cap) {
     extern __shared__ __align__(16) uint8_t dyn[];
     __shared__ uint32_t s_up4[MPE_MAX_EXPERTS];
     __shared__ uint32_t s_up8[MPE_MAX_EXPERTS];
@@ -46,7 +52,7 @@ k_allocate(const double* p, const uint64_t* W, int E, uint64_t B, uint64_t sum_w
     uint64_t R64 = 0;
     if (B < 3 * sum_w) {
         mode = 1;
-    } else if (B >= 8 * sum_w) {
+    } else if (B >= 8 * sum_w && !loss) {
         mode = 2;
     } else {
         R64 = (B - 3 * sum_w) / g;
@@ -78,9 +84,9 @@ k_allocate(const double* p, const uint64_t* W, int E, uint64_t B, uint64_t sum_w
     __syncthreads();
     for (int e = 0; e < E; ++e) {
         const double pe = s_p[e];
-        const double c3 = __dmul_rn(pe, L3);
-        const double c4 = __dmul_rn(pe, L4);
-        const double c8 = __dmul_rn(pe, L8);
+        const double c3 = __dmul_rn(pe, loss ? loss[3 * e] : L3);
+        const double c4 = __dmul_rn(pe, loss ? loss[3 * e + 1] : L4);
+        const double c8 = __dmul_rn(pe, loss ? loss[3 * e + 2] : L8);
         const uint32_t u4 = s_up4[e], u8 = s_up8[e];
         uint8_t* ch = chb + (size_t)e * nq;
         for (uint32_t qd = tid; qd < nq; qd += kThreads) {
@@ -227,9 +233,9 @@ k_allocate_proportional(const double* p, const uint64_t* W, int E, uint64_t B, u
 
 size_t allocate_choice_bytes(int E, uint64_t R) { return (size_t)E * (size_t)((R + 4) / 4); }
 
-void launch_allocate(cudaStream_t st, const double* p, const uint64_t* W, int E, uint64_t B,
-                     uint64_t sum_w, uint64_t g, uint8_t* bits_out, int32_t* status,
-                     uint8_t* choice, double* D, int state_cap, uint64_t R) {
+void launch_allocate(cudaStream_t st, const double* p, const double* loss, const uint64_t* W,
+                     int E, uint64_t B, uint64_t sum_w, uint64_t g, uint8_t* bits_out,
+                     int32_t* status, uint8_t* choice, double* D, int state_cap, uint64_t R) {
     // R is the host's count of budget units (same formula as the kernel's);
     // it only sizes the on-chip buffers
     const size_t smem = 16 * (size_t)(R + 1) + allocate_choice_bytes(E, R);
@@ -238,11 +244,11 @@ void launch_allocate(cudaStream_t st, const double* p, const uint64_t* W, int E,
         if (smem > 48 * 1024)
             cudaFuncSetAttribute(k_allocate<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)smem);
-        k_allocate<true><<<1, kThreads, smem, st>>>(p, W, E, B, sum_w, g, bits_out, status, choice,
-                                                    D, state_cap);
+        k_allocate<true><<<1, kThreads, smem, st>>>(p, loss, W, E, B, sum_w, g, bits_out, status,
+                                                    choice, D, state_cap);
     } else {
-        k_allocate<false><<<1, kThreads, 0, st>>>(p, W, E, B, sum_w, g, bits_out, status, choice,
-                                                  D, state_cap);
+        k_allocate<false><<<1, kThreads, 0, st>>>(p, loss, W, E, B, sum_w, g, bits_out, status,
+                                                  choice, D, state_cap);
     }
 }
 

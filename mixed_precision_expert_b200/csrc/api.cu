@@ -302,8 +302,17 @@ int run_allocate(mpe_ctx* c, const double* p, uint64_t B, std::vector<uint8_t>& 
     if (B < 3 * sum_w) return fail(c, MPE_ERR_INFEASIBLE, "budget %llu < 3 * sum W = %llu",
                                    (unsigned long long)B, (unsigned long long)(3 * sum_w));
     const uint64_t g = w_e;
-    const bool exact = c->allocator == MPE_ALLOCATOR_EXACT;
-    uint64_t R = B >= 8 * sum_w ? 0 : (B - 3 * sum_w) / g;
+    const bool measured = c->allocator == MPE_ALLOCATOR_MEASURED;
+    const bool exact = c->allocator == MPE_ALLOCATOR_EXACT || measured;
+    if (measured && !c->loss_valid) {
+        // the master never changes while the context lives: measure once
+        if (!c->absmax_valid) return fail(c, MPE_ERR_ORDER, "measured loss before quantize_experts");
+        launch_measure_mse(c, c->d_mse_acc, c->d_loss);
+        CKLAUNCH();
+        if (st != c->stream) CK(cudaStreamSynchronize(c->stream));  // once per context
+        c->loss_valid = true;
+    }
+    uint64_t R = (B >= 8 * sum_w && !measured) ? 0 : (B - 3 * sum_w) / g;
     R = std::min<uint64_t>(R, 5 * (sum_w / g));
     if (exact && R + 1 > MPE_ALLOC_STATE_CAP) return fail(c, MPE_ERR_STATE_CAP, "too many states");
     const size_t need = exact ? allocate_choice_bytes(E, R) : 0;
@@ -323,8 +332,9 @@ int run_allocate(mpe_ctx* c, const double* p, uint64_t B, std::vector<uint8_t>& 
     CK(cudaMemcpyAsync(c->d_p, c->h_p_pinned, sizeof(double) * E, cudaMemcpyHostToDevice,
                        st));
     if (exact)
-        launch_allocate(st, c->d_p, c->d_W, E, B, sum_w, g, c->d_bits_out,
-                        c->d_alloc_status, c->d_choice, c->d_D, MPE_ALLOC_STATE_CAP, R);
+        launch_allocate(st, c->d_p, measured ? c->d_loss : nullptr, c->d_W, E, B, sum_w, g,
+                        c->d_bits_out, c->d_alloc_status, c->d_choice, c->d_D,
+                        MPE_ALLOC_STATE_CAP, R);
     else
         launch_allocate_proportional(st, c->d_p, c->d_W, E, B, sum_w, c->d_bits_out,
                                      c->d_alloc_status);
@@ -408,6 +418,8 @@ int mpe_create(mpe_ctx** out, const mpe_config* cfg) {
     if ((r = dev_alloc(c, &c->d_bits_out, c->E))) return bail(r);
     if ((r = dev_alloc(c, &c->d_alloc_status, 1))) return bail(r);
     if ((r = dev_alloc(c, &c->d_D, 2 * (size_t)MPE_ALLOC_STATE_CAP))) return bail(r);
+    if ((r = dev_alloc(c, &c->d_loss, 3 * (size_t)c->E))) return bail(r);
+    if ((r = dev_alloc(c, &c->d_mse_acc, 6 * (size_t)c->E))) return bail(r);
     if (cudaMallocHost(&c->h_pte_pinned, sizeof(Pte) * c->E) != cudaSuccess ||
         cudaMallocHost(&c->h_pidx_pinned, sizeof(uint32_t) * c->pool_pages) != cudaSuccess ||
         cudaMallocHost(&c->h_list_pinned, sizeof(int32_t) * c->E) != cudaSuccess ||
@@ -456,6 +468,7 @@ void mpe_destroy(mpe_ctx* c) {
         cudaFree(c->d_status); cudaFree(c->d_masters); cudaFree(c->d_list); cudaFree(c->d_p);
         cudaFree(c->d_W); cudaFree(c->d_bits_out); cudaFree(c->d_alloc_status);
         cudaFree(c->d_choice); cudaFree(c->d_D); cudaFree(c->d_gather);
+        cudaFree(c->d_loss); cudaFree(c->d_mse_acc);
         cudaFreeHost(c->h_pte_pinned); cudaFreeHost(c->h_pidx_pinned);
         cudaFreeHost(c->h_list_pinned); cudaFreeHost(c->h_masters_pinned);
         cudaFreeHost(c->h_p_pinned); cudaFreeHost(c->h_w_pinned); cudaFreeHost(c->h_alloc_pinned);
@@ -484,8 +497,12 @@ int mpe_set_path(mpe_ctx* c, int32_t path) {
     return MPE_OK;
 }
 
-int mpe_allocate_bits(const double* p, const uint64_t* W, int32_t E, uint64_t B_bits,
-                      uint8_t* bits_out) {
+namespace {
+
+// The exact program on a temporary device copy of its inputs; loss (host
+// float64[E][3]) may be null for the fixed L(b).
+int allocate_exact(const double* p, const double* loss, const uint64_t* W, int32_t E,
+                   uint64_t B_bits, uint8_t* bits_out) {
     if (!p || !W || !bits_out) return fail_global(MPE_ERR_INVALID, "null argument");
     if (E < 1 || E > MPE_MAX_EXPERTS) return fail_global(MPE_ERR_INVALID, "E out of range");
     uint64_t sum_w = 0, g = 0;
@@ -493,15 +510,19 @@ int mpe_allocate_bits(const double* p, const uint64_t* W, int32_t E, uint64_t B_
         if (W[e] == 0) return fail_global(MPE_ERR_INVALID, "W[%d] = 0", e);
         if (!(p[e] >= 0.0) || !std::isfinite(p[e]))
             return fail_global(MPE_ERR_INVALID, "p[%d] must be finite and >= 0", e);
+        if (loss)
+            for (int i = 0; i < 3; ++i)
+                if (!(loss[3 * e + i] >= 0.0) || !std::isfinite(loss[3 * e + i]))
+                    return fail_global(MPE_ERR_INVALID, "loss[%d][%d] must be finite and >= 0", e, i);
         sum_w += W[e];
         g = std::gcd(g, W[e]);
     }
     if (B_bits < 3 * sum_w) return fail_global(MPE_ERR_INFEASIBLE, "budget below 3 bits per weight");
-    uint64_t R = B_bits >= 8 * sum_w ? 0 : (B_bits - 3 * sum_w) / g;
+    uint64_t R = (B_bits >= 8 * sum_w && !loss) ? 0 : (B_bits - 3 * sum_w) / g;
     R = std::min<uint64_t>(R, 5 * (sum_w / g));
     if (R + 1 > MPE_ALLOC_STATE_CAP) return fail_global(MPE_ERR_STATE_CAP, "too many states");
     double* dp = nullptr; uint64_t* dW = nullptr; uint8_t* db = nullptr; int32_t* ds = nullptr;
-    uint8_t* dch = nullptr; double* dD = nullptr;
+    uint8_t* dch = nullptr; double* dD = nullptr; double* dl = nullptr;
     int rc = MPE_OK;
     int32_t st = -1;
     auto ok = [](cudaError_t e) { return e == cudaSuccess; };
@@ -509,12 +530,14 @@ int mpe_allocate_bits(const double* p, const uint64_t* W, int32_t E, uint64_t B_
         !ok(cudaMalloc(&db, E)) || !ok(cudaMalloc(&ds, sizeof(int32_t))) ||
         !ok(cudaMalloc(&dch, allocate_choice_bytes(E, R))) ||
         !ok(cudaMalloc(&dD, 2 * sizeof(double) * (R + 1))) ||
+        (loss && !ok(cudaMalloc(&dl, 3 * sizeof(double) * E))) ||
         !ok(cudaMemcpy(dp, p, sizeof(double) * E, cudaMemcpyHostToDevice)) ||
+        (loss && !ok(cudaMemcpy(dl, loss, 3 * sizeof(double) * E, cudaMemcpyHostToDevice))) ||
         !ok(cudaMemcpy(dW, W, sizeof(uint64_t) * E, cudaMemcpyHostToDevice))) {
         rc = fail_global(MPE_ERR_CUDA, "allocate_bits: %s", cudaGetErrorString(cudaGetLastError()));
     } else {
-        launch_allocate(nullptr, dp, dW, E, B_bits, sum_w, g, db, ds, dch, dD, MPE_ALLOC_STATE_CAP,
-                        R);
+        launch_allocate(nullptr, dp, dl, dW, E, B_bits, sum_w, g, db, ds, dch, dD,
+                        MPE_ALLOC_STATE_CAP, R);
         if (!ok(cudaGetLastError()) || !ok(cudaMemcpy(&st, ds, sizeof(int32_t), cudaMemcpyDeviceToHost)) ||
             !ok(cudaMemcpy(bits_out, db, E, cudaMemcpyDeviceToHost)))
             rc = fail_global(MPE_ERR_CUDA, "allocate_bits kernel: %s",
@@ -525,7 +548,36 @@ int mpe_allocate_bits(const double* p, const uint64_t* W, int32_t E, uint64_t B_
             rc = fail_global(MPE_ERR_STATE_CAP, "too many allocation states");
     }
     cudaFree(dp); cudaFree(dW); cudaFree(db); cudaFree(ds); cudaFree(dch); cudaFree(dD);
+    cudaFree(dl);
     return rc;
+}
+
+}  // namespace
+
+int mpe_allocate_bits(const double* p, const uint64_t* W, int32_t E, uint64_t B_bits,
+                      uint8_t* bits_out) {
+    return allocate_exact(p, nullptr, W, E, B_bits, bits_out);
+}
+
+int mpe_allocate_bits_table(const double* p, const double* loss, const uint64_t* W, int32_t E,
+                            uint64_t B_bits, uint8_t* bits_out) {
+    if (!loss) return fail_global(MPE_ERR_INVALID, "null argument");
+    return allocate_exact(p, loss, W, E, B_bits, bits_out);
+}
+
+int mpe_measure_loss(mpe_ctx* c, double* loss_host) {
+    if (!c) return fail_global(MPE_ERR_INVALID, "null context");
+    if (!loss_host) return fail(c, MPE_ERR_INVALID, "null argument");
+    if (!c->absmax_valid) return fail(c, MPE_ERR_ORDER, "measure_loss before quantize_experts");
+    if (!c->loss_valid) {
+        launch_measure_mse(c, c->d_mse_acc, c->d_loss);
+        CKLAUNCH();
+        c->loss_valid = true;
+    }
+    CK(cudaMemcpyAsync(loss_host, c->d_loss, 3 * sizeof(double) * c->E, cudaMemcpyDeviceToHost,
+                       c->stream));
+    CK(cudaStreamSynchronize(c->stream));
+    return MPE_OK;
 }
 
 int mpe_allocate_bits_proportional(const double* p, const uint64_t* W, int32_t E,
@@ -565,7 +617,8 @@ int mpe_allocate_bits_proportional(const double* p, const uint64_t* W, int32_t E
 
 int mpe_set_allocator(mpe_ctx* c, int32_t allocator) {
     if (!c) return fail_global(MPE_ERR_INVALID, "null context");
-    if (allocator != MPE_ALLOCATOR_EXACT && allocator != MPE_ALLOCATOR_PROPORTIONAL)
+    if (allocator != MPE_ALLOCATOR_EXACT && allocator != MPE_ALLOCATOR_PROPORTIONAL &&
+        allocator != MPE_ALLOCATOR_MEASURED)
         return fail(c, MPE_ERR_INVALID, "bad allocator %d", allocator);
     c->allocator = allocator;
     return MPE_OK;
@@ -606,6 +659,7 @@ int mpe_quantize_experts(mpe_ctx* c, const void* const* master_f16, const uint8_
     launch_encode(c, c->d_list, c->E);
     CKLAUNCH();
     c->absmax_valid = true;
+    c->loss_valid = false;
     return MPE_OK;
 }
 

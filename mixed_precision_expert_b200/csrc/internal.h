@@ -87,6 +87,9 @@ struct mpe_ctx {
     uint8_t* d_choice = nullptr;
     size_t choice_cap = 0;
     double* d_D = nullptr;            // two DP rows
+    double* d_loss = nullptr;         // measured MSE per expert and width [E][3]
+    unsigned long long* d_mse_acc = nullptr;  // its exact sums [E][3][2]
+    bool loss_valid = false;          // d_loss holds the current master's values
     uint8_t* d_gather = nullptr;      // expert stream gather buffer
     size_t gather_cap = 0;
 
@@ -163,13 +166,16 @@ void launch_scales_on(mpe_ctx* c, Pte* pte, cudaStream_t st);
 void launch_encode_on(mpe_ctx* c, const PagedExperts& P, const int32_t* d_list, int n_list,
                       cudaStream_t st);
 void launch_gather_stream(mpe_ctx* c, int e, uint8_t* dst);
+// mse[e][0..2] = measured quantization MSE of expert e at 3 / 4 / 8 bits (uses
+// the cached absmax); acc: [E][3][2] 64-bit words of scratch
+void launch_measure_mse(mpe_ctx* c, unsigned long long* d_acc, double* d_mse);
 
 // allocate.cu
 // sum_w = sum of W, g = gcd(W) (host-computed); R = budget units (sizes the
-// on-chip buffers)
-void launch_allocate(cudaStream_t st, const double* p, const uint64_t* W, int E, uint64_t B,
-                     uint64_t sum_w, uint64_t g, uint8_t* bits_out, int32_t* status,
-                     uint8_t* choice, double* D, int state_cap, uint64_t R);
+// on-chip buffers); loss = float64[E][3] per-expert losses or null for L(b)
+void launch_allocate(cudaStream_t st, const double* p, const double* loss, const uint64_t* W,
+                     int E, uint64_t B, uint64_t sum_w, uint64_t g, uint8_t* bits_out,
+                     int32_t* status, uint8_t* choice, double* D, int state_cap, uint64_t R);
 // bytes of the global choice table for E experts and R budget units
 size_t allocate_choice_bytes(int E, uint64_t R);
 // the page's proportional rule with a budget repair (status 1: infeasible)

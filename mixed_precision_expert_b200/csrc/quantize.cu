@@ -255,6 +255,179 @@ k_encode(PagedExperts P, const void* const* masters, const int32_t* list) {
     }
 }
 
+// Measured quantization error of every expert at every width (PagedWeight,
+// "Quality-Aware Quantization": the mean squared error is the page's example
+// loss, and experts differ in sensitivity). For width b the expert's own
+// s_b = RN_f32(m / q_b) and codes k = round-half-even(w / s_b) give the error
+// w - k s_b, which is exact in float32: |w - k s_b| <= s_b / 2, and when k != 0
+// |w| >= s_b / 2 puts w's last bit at or above s_b's, so the error is a
+// multiple of s_b's last bit below 2^24 of them (k = 0 leaves w itself). Each
+// error, scaled to an integer in units of Q_b = 2^min(e_b - 23, -24) (e_b the
+// exponent of s_b), is squared and summed exactly in integers: the sum does
+// not depend on the order, so the result is reproducible bit for bit.
+//
+// Fast form (s_3 < 1, every width's Q_b = 2^(e_b - 23)): scaled errors are
+// below 2^23, squares below 2^46; a thread sums at most 2^7 of them per width
+// in 64 bits and a block's sum stays below 2^62. Wide form (s_3 >= 1): scaled
+// errors up to 2^39, squares and sums in 128 bits. Either form ends in a
+// 128-bit total per (expert, width) kept as two 64-bit words, added with
+// atomics and an explicit carry.
+constexpr int kMseThreads = 256;
+constexpr int64_t kMseSegVec = 4096;  // 16-byte vectors (32768 weights) per CTA
+static_assert(kMseSegVec * 8 / kMseThreads <= 128, "fast-form per-thread bound");
+
+struct MseWidth {
+    float s, inv_s, sc;  // scale, its reciprocal, 1 / Q_b
+};
+
+__device__ __forceinline__ MseWidth mse_width(float mf, int q) {
+    MseWidth w;
+    w.s = __fdiv_rn(mf, (float)q);
+    w.inv_s = __frcp_rn(w.s);
+    const int eb = (int)((__float_as_uint(w.s) >> 23) & 0xFF) - 127;  // s is normal
+    const int shift = max(23 - eb, 24);                                // -log2 Q_b
+    w.sc = __uint_as_float((uint32_t)(127 + shift) << 23);
+    return w;
+}
+
+// k = round-half-even(w / s) exactly (same rounding as the encoder), then the
+// scaled error (w - k s) / Q as an exactly integer-valued float.
+__device__ __forceinline__ float mse_scaled_error(float w, const MseWidth& m) {
+    constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+    const float r = __fmul_rn(w, m.inv_s);
+    float kf = __fsub_rn(__fadd_rn(r, kRound), kRound);
+    if (fabsf(__fsub_rn(r, kf)) > 0.4990234375f) kf = tie_fix(w, m.s, kf);
+    return __fmul_rn(__fmaf_rn(-kf, m.s, w), m.sc);  // exact error, exact scaling
+}
+
+__device__ __forceinline__ void add128(unsigned long long& lo, unsigned long long& hi,
+                                       unsigned long long alo, unsigned long long ahi) {
+    const unsigned long long t = lo + alo;
+    hi += ahi + (t < lo ? 1ull : 0ull);
+    lo = t;
+}
+
+template <bool WIDE>
+__device__ __forceinline__ void mse_accumulate(float w, const MseWidth (&mw)[3],
+                                               unsigned long long (&lo)[3],
+                                               unsigned long long (&hi)[3]) {
+#pragma unroll
+    for (int i = 0; i < 3; ++i) {
+        const float v = mse_scaled_error(w, mw[i]);
+        if constexpr (WIDE) {
+            const unsigned long long a = (unsigned long long)llabs(__float2ll_rn(v));
+            add128(lo[i], hi[i], a * a, __umul64hi(a, a));
+        } else {
+            const int a = __float2int_rn(v);
+            lo[i] += (unsigned long long)((long long)a * a);
+        }
+    }
+}
+
+// acc: [E][3][2] (low word, high word), zeroed by the caller.
+__global__ void __launch_bounds__(kMseThreads)
+k_mse_sum(const void* const* masters, int64_t n_vec, const uint32_t* absmax,
+          unsigned long long* acc) {
+    const int e = blockIdx.y;
+    const uint32_t m = absmax[e];
+    if (m == 0 || m >= 0x7C00u) return;  // zero expert: no error; non-finite: reported by the finisher
+    const float mf = __half2float(__ushort_as_half((unsigned short)m));
+    MseWidth mw[3];
+    mw[0] = mse_width(mf, 3);
+    mw[1] = mse_width(mf, 7);
+    mw[2] = mse_width(mf, 127);
+    const bool wide = mw[0].s >= 1.0f;  // s_3 is the largest scale
+    const uint4* src = reinterpret_cast<const uint4*>(masters[e]);
+    const int64_t beg = (int64_t)blockIdx.x * kMseSegVec;
+    const int64_t end = min(beg + kMseSegVec, n_vec);
+    unsigned long long lo[3] = {0, 0, 0}, hi[3] = {0, 0, 0};
+    constexpr int kUnroll = 4;  // 16-byte loads in flight per thread
+    for (int64_t i0 = beg + threadIdx.x; i0 < end; i0 += kMseThreads * kUnroll) {
+        uint4 v[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int64_t i = i0 + (int64_t)u * kMseThreads;
+            v[u] = i < end ? __ldcs(src + i) : make_uint4(0, 0, 0, 0);  // zeros add no error
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const uint32_t wv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&wv[h]));
+                if (wide) {
+                    mse_accumulate<true>(f.x, mw, lo, hi);
+                    mse_accumulate<true>(f.y, mw, lo, hi);
+                } else {
+                    mse_accumulate<false>(f.x, mw, lo, hi);
+                    mse_accumulate<false>(f.y, mw, lo, hi);
+                }
+            }
+        }
+    }
+    __shared__ unsigned long long red_lo[kMseThreads / 32][3], red_hi[kMseThreads / 32][3];
+#pragma unroll
+    for (int i = 0; i < 3; ++i) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            add128(lo[i], hi[i], __shfl_xor_sync(0xffffffffu, lo[i], o),
+                   __shfl_xor_sync(0xffffffffu, hi[i], o));
+    }
+    const int warp = threadIdx.x >> 5;
+    if ((threadIdx.x & 31) == 0) {
+#pragma unroll
+        for (int i = 0; i < 3; ++i) {
+            red_lo[warp][i] = lo[i];
+            red_hi[warp][i] = hi[i];
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x < 3) {
+        const int i = threadIdx.x;
+        unsigned long long l = 0, h = 0;
+        for (int w = 0; w < kMseThreads / 32; ++w) add128(l, h, red_lo[w][i], red_hi[w][i]);
+        unsigned long long* a = acc + ((size_t)e * 3 + i) * 2;
+        const unsigned long long old = atomicAdd(a, l);
+        const unsigned long long carry = (old + l < old) ? 1ull : 0ull;
+        if (h + carry) atomicAdd(a + 1, h + carry);
+    }
+}
+
+// Round a 128-bit integer to the nearest float64 (ties to even): the top 64
+// bits with the rest folded into their last bit (a sticky bit far below the
+// rounding position), converted once, then scaled by a power of two.
+__device__ __forceinline__ double u128_to_double(unsigned long long lo, unsigned long long hi) {
+    if (hi == 0) return __ull2double_rn(lo);
+    const int lz = __clzll((long long)hi);
+    const int sh = 64 - lz;  // 1 .. 64
+    const unsigned long long top = lz == 0 ? hi : (hi << lz) | (lo >> sh);
+    const unsigned long long rest = lz == 0 ? lo : (lo << lz);
+    return ldexp(__ull2double_rn(top | (rest != 0 ? 1ull : 0ull)), sh);
+}
+
+// mse[e][i] = RN(RN(sum of squared errors) / n): the 128-bit total rounded to
+// float64 and scaled by Q_b^2 (exact), then one float64 division by n.
+__global__ void k_mse_finish(const unsigned long long* acc, const uint32_t* absmax, int E,
+                             double n, double* mse) {
+    const int t = blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= 3 * E) return;
+    const int e = t / 3, i = t - 3 * e;
+    const uint32_t m = absmax[e];
+    if (m >= 0x7C00u) {
+        mse[t] = __longlong_as_double(0x7FF8000000000000ll);
+        return;
+    }
+    if (m == 0) {
+        mse[t] = 0.0;
+        return;
+    }
+    const float mf = __half2float(__ushort_as_half((unsigned short)m));
+    const MseWidth mw = mse_width(mf, i == 0 ? 3 : (i == 1 ? 7 : 127));
+    const int shift = (int)((__float_as_uint(mw.sc) >> 23) & 0xFF) - 127;
+    const double sum_sq = ldexp(u128_to_double(acc[2 * t], acc[2 * t + 1]), -2 * shift);
+    mse[t] = __ddiv_rn(sum_sq, n);
+}
+
 // Copy expert e's chunk stream out of its pages, in stream order.
 __global__ void k_gather_stream(PagedExperts P, int e, uint8_t* dst) {
     const Pte pte = P.pte[e];
@@ -307,6 +480,16 @@ void launch_encode_on(mpe_ctx* c, const PagedExperts& P, const int32_t* d_list, 
 
 void launch_encode(mpe_ctx* c, const int32_t* d_list, int n_list) {
     launch_encode_on(c, paged(c), d_list, n_list, c->stream);
+}
+
+void launch_measure_mse(mpe_ctx* c, unsigned long long* d_acc, double* d_mse) {
+    const int64_t n_vec = (int64_t)3 * c->H * c->F / 8;
+    cudaMemsetAsync(d_acc, 0, sizeof(unsigned long long) * 6 * c->E, c->stream);
+    dim3 grid((unsigned)((n_vec + kMseSegVec - 1) / kMseSegVec), (unsigned)c->E);
+    k_mse_sum<<<grid, kMseThreads, 0, c->stream>>>(c->d_masters, n_vec, c->d_absmax, d_acc);
+    k_mse_finish<<<(3 * c->E + 127) / 128, 128, 0, c->stream>>>(
+        d_acc, c->d_absmax, c->E, (double)(n_vec * 8), d_mse);
+    c->launches += 2;
 }
 
 void launch_gather_stream(mpe_ctx* c, int e, uint8_t* dst) {

@@ -104,10 +104,8 @@ def quantization_mse(master_fp16, b: int) -> float:
         return 0.0
     m, s, k = quantize_expert(w, b)
     err = w.astype(np.float64) - dequantize(k, s)
-    total = 0
-    for e in err.tolist():
-        i = int(math.ldexp(e, 60))
-        assert math.ldexp(float(i), -60) == e  # the scaled error is an integer
-        total += i * i
+    scaled = np.ldexp(err, 60)
+    assert np.array_equal(scaled, np.trunc(scaled))  # every scaled error is an integer
+    total = sum(i * i for i in map(int, scaled.tolist()))
     sum_sq = math.ldexp(float(total), -120)  # float(int) rounds to nearest, ties to even
     return float(np.float64(sum_sq) / np.float64(n))
