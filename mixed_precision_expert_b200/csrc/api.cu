@@ -152,7 +152,11 @@ bool plan_pages_overlapped(const mpe_ctx* c, const std::vector<uint8_t>& new_bit
 // overlapped repage.
 int ensure_side(mpe_ctx* c) {
     if (c->side) return MPE_OK;
-    CK(cudaStreamCreateWithFlags(&c->side, cudaStreamNonBlocking));
+    // the lowest priority: when the forward calls run on a stream of higher
+    // priority, the block scheduler starts their CTAs before the encode's
+    int least = 0, greatest = 0;
+    CK(cudaDeviceGetStreamPriorityRange(&least, &greatest));
+    CK(cudaStreamCreateWithPriority(&c->side, cudaStreamNonBlocking, least));
     CK(cudaEventCreateWithFlags(&c->side_done, cudaEventDisableTiming));
     CK(cudaEventCreateWithFlags(&c->old_table_free, cudaEventDisableTiming));
     CK(cudaEventRecord(c->old_table_free, c->stream));
