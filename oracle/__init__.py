@@ -24,6 +24,9 @@ Quantization", llmdb.app summary page):
   to physical pages).
 * ``route``     -- token-to-expert bucketing for the forward pass (PagedWeight,
   "Dynamic Paging": the router decides which experts a pass needs).
+* ``compensate`` -- dynamic error compensation of salient input channels
+  (DecDEC summary, 3.1-3.2 and Figure 4): (W^ + R (.) M) x with R = W - W^
+  and M keeping the channels of largest |x|.
 * ``ffn``       -- dequantize-then-multiply expert FFN (PagedWeight, "Dynamic
   Paging": fetch pages, dequantize on the fly; DecDEC summary, 2.2: weight-only
   quantization dequantizes before multiplying with full-precision
