@@ -459,29 +459,73 @@ __device__ __forceinline__ bool resolve_class(const Args& a, const CtaSmem& sm, 
                     need_wait = false;
                 }
                 // lane l adds 8 consecutive codes per 256: positions 8 (l % 4) .. + 7
-                // of a quarter
+                // of a quarter. All tokens at once (loads of 8 rows in flight per
+                // step), then one transposing reduction of the 16 sums.
+                static_assert(kDecodeGroup == 16, "the reduction below folds 16 sums");
                 float off[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) off[e] = code_offset<B>(8 * (lane & 3) + e);
                 const int k_lo = 128 * m->j0, k_hi = 128 * m->j_hi, ntok = m->ntok;
-                for (int i = 0; i < ntok; ++i) {
-                    const __nv_bfloat16* row = a.act + (size_t)m->rows[i] * K;
-                    float sum = 0.0f;
-                    for (int k = k_lo + 8 * lane; k < k_hi; k += 256) {
-                        const uint4 v = __ldg(reinterpret_cast<const uint4*>(row + k));
-                        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+                float sum[kDecodeGroup];
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float lo = __uint_as_float(wv[e] << 16);
-                            const float hi = __uint_as_float(wv[e] & 0xFFFF0000u);
-                            sum = fmaf(off[2 * e], lo, sum);
-                            sum = fmaf(off[2 * e + 1], hi, sum);
+                for (int i = 0; i < kDecodeGroup; ++i) sum[i] = 0.0f;
+                for (int k = k_lo + 8 * lane; k < k_hi; k += 256) {
+#pragma unroll
+                    for (int h8 = 0; h8 < kDecodeGroup; h8 += 8) {
+                        if (h8 >= ntok) break;
+                        uint4 v[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            v[i] = h8 + i < ntok
+                                       ? __ldg(reinterpret_cast<const uint4*>(
+                                             a.act + (size_t)m->rows[h8 + i] * K + k))
+                                       : make_uint4(0, 0, 0, 0);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const uint32_t wv[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float lo = __uint_as_float(wv[e] << 16);
+                                const float hi = __uint_as_float(wv[e] & 0xFFFF0000u);
+                                sum[h8 + i] = fmaf(off[2 * e], lo, sum[h8 + i]);
+                                sum[h8 + i] = fmaf(off[2 * e + 1], hi, sum[h8 + i]);
+                            }
                         }
                     }
-#pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-                    if (lane == 0) m->offsum[i] = sum;
                 }
+                // fold: at offset 16 a lane keeps the half of the sums its lane bit
+                // 4 selects and adds its partner's copy of that half; then 8, 4, 2
+                // (halving again), and 1. Lane l ends with token (l >> 1) & 15.
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const bool up = (lane & 16) != 0;
+                    const float send = up ? sum[i] : sum[i + 8];
+                    const float keep = up ? sum[i + 8] : sum[i];
+                    sum[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const bool up = (lane & 8) != 0;
+                    const float send = up ? sum[i] : sum[i + 4];
+                    const float keep = up ? sum[i + 4] : sum[i];
+                    sum[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+                }
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const bool up = (lane & 4) != 0;
+                    const float send = up ? sum[i] : sum[i + 2];
+                    const float keep = up ? sum[i + 2] : sum[i];
+                    sum[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+                }
+                {
+                    const bool up = (lane & 2) != 0;
+                    const float send = up ? sum[0] : sum[1];
+                    const float keep = up ? sum[1] : sum[0];
+                    sum[0] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+                }
+                sum[0] += __shfl_xor_sync(0xffffffffu, sum[0], 1);
+                const int tok = (lane >> 1) & 15;
+                if ((lane & 1) == 0 && tok < ntok) m->offsum[tok] = sum[0];
                 __syncwarp();
             }
             if (lane == 0) mbar_arrive(&sm.tq_sum[q]);
@@ -842,10 +886,10 @@ void decode_set_smem_limits() {
 
 // K parts per task: enough CTA tasks that every CTA of the persistent grid gets
 // about `per_cta` of them, at least 4 blocks per part.
-int decode_parts(int est_groups, int n_tq, int nj, int total_ctas, int per_cta) {
+int decode_parts(int est_groups, int n_tq, int nj, int total_ctas, int per_cta, int min_kb) {
     const long target = (long)per_cta * total_ctas;
     int P = 1;
-    const int pmax = max(1, nj / 4);
+    const int pmax = max(1, nj / min_kb);
     while (P < pmax && (long)est_groups * n_tq * P < target) ++P;
     return P;
 }
@@ -865,13 +909,16 @@ void decode_plan(mpe_ctx* c, size_t Tk, DecodePlan& pl) {
     const int pc_dn_env = env_int("MPE_DECODE_TASKS_PER_CTA_DOWN", 0);
     const int pc_gu = pc_gu_env > 0 ? pc_gu_env : (pc_env > 0 ? pc_env : 6);
     const int pc_dn = pc_dn_env > 0 ? pc_dn_env : (pc_env > 0 ? pc_env : 8);
+    // at least this many block columns per K part (a part's fixed costs)
+    const int min_kb_gu = std::max(1, env_int("MPE_DECODE_MIN_KB_GATEUP", 4));
+    const int min_kb_dn = std::max(1, env_int("MPE_DECODE_MIN_KB_DOWN", 4));
     pl.claim = 1;
     const int nj_gu = c->H / kCodesPerBlock, nj_dn = c->F / kCodesPerBlock;
     const int tt_gu = tiles_per_task(true), tt_dn = tiles_per_task(false);
-    int p = decode_parts(groups, (c->F / 16 + tt_gu - 1) / tt_gu, nj_gu, ctas, pc_gu);
+    int p = decode_parts(groups, (c->F / 16 + tt_gu - 1) / tt_gu, nj_gu, ctas, pc_gu, min_kb_gu);
     pl.kb_gu = (nj_gu + p - 1) / p;
     pl.p_gu = (nj_gu + pl.kb_gu - 1) / pl.kb_gu;
-    p = decode_parts(groups, (c->H / 16 + tt_dn - 1) / tt_dn, nj_dn, ctas, pc_dn);
+    p = decode_parts(groups, (c->H / 16 + tt_dn - 1) / tt_dn, nj_dn, ctas, pc_dn, min_kb_dn);
     pl.kb_dn = (nj_dn + p - 1) / p;
     pl.p_dn = (nj_dn + pl.kb_dn - 1) / pl.kb_dn;
 }
