@@ -471,6 +471,38 @@ def run_mpe(args, dist: Dist):
     e2e = {"value": T * n_e2e * dist.world / e2e_s, "unit": "tokens/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e}
 
+    # salient-channel compensation on the streaming path (timed apart from the
+    # headline value): step time with n channels kept per row, store in device
+    # or mapped host memory
+    comp = None
+    if not prof["tc_gate_up"][1]:
+        comp = {"n_channels": [], "store": [], "step_us": []}
+        ev_a, ev_b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_comp = max(20, min(args.steps, 200))
+        try:
+            for n_ch, store in ((16, mpe.STORE_DEVICE), (64, mpe.STORE_DEVICE),
+                                (16, mpe.STORE_HOST)):
+                ctx.set_compensation(n_ch, store)
+                for i in range(3):
+                    x, idt, wt, _ = batches[i % nb]
+                    ctx.moe_ffn(x, idt, wt, out)
+                dist.barrier()
+                torch.cuda.synchronize()
+                ev_a.record()
+                for i in range(n_comp):
+                    x, idt, wt, _ = batches[i % nb]
+                    ctx.moe_ffn(x, idt, wt, out)
+                ev_b.record()
+                torch.cuda.synchronize()
+                comp["n_channels"].append(n_ch)
+                comp["store"].append("host" if store == mpe.STORE_HOST else "device")
+                comp["step_us"].append(dist.max(ev_a.elapsed_time(ev_b) / n_comp * 1e3))
+            ctx.set_compensation(0)
+            comp["plain_step_us"] = ms / args.steps * 1e3
+        except mpe.MpeError as err:
+            comp = {"unavailable": str(err)}
+            ctx.set_compensation(0)
+
     cpu = None
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         slice_rows = 128
@@ -504,6 +536,7 @@ def run_mpe(args, dist: Dist):
                          "bytes": ml_bytes,
                          "note": "exact MSE of every expert at 3, 4 and 8 bits; one read "
                                  "of the fp16 masters; integer-ALU bound"},
+        "compensation": comp,
         "gpu_launches": launches,
         "clocks": clk,
         "e2e": e2e,

@@ -60,6 +60,7 @@ extern "C" {
 #define MPE_MAX_EXPERTS        1024  /* E                                               */
 #define MPE_ALLOC_STATE_CAP    65536 /* allocator DP states (budget units + 1)          */
 #define MPE_DEFAULT_PAGE_BYTES 65536
+#define MPE_MAX_COMP_CHANNELS  256   /* salient channels compensated per input row    */
 
 /* ---- forward-pass path selection --------------------------------------- */
 #define MPE_PATH_AUTO    0   /* decode kernels for small token counts, prefill above */
@@ -199,6 +200,59 @@ int mpe_quantize_experts(mpe_ctx* ctx, const void* const* master_f16, const uint
  * Synchronous. MPE_ERR_ORDER before mpe_quantize_experts.
  */
 int mpe_measure_loss(mpe_ctx* ctx, double* loss_host);
+
+/* where mpe_set_compensation keeps its residual store */
+#define MPE_STORE_DEVICE 0  /* device memory                                        */
+#define MPE_STORE_HOST   1  /* mapped pinned host memory, read by the kernels over
+                               the bus (the CPU-side residuals of the paper)        */
+
+/*
+ * mpe_set_compensation -- dynamic error compensation of salient input
+ * channels on the streaming path (DecDEC summary, 3.1-3.2: each quantized
+ * linear W^ x becomes (W^ + R (.) M) x with R = W - W^ and M keeping the input
+ * channels of largest |x|). With n_channels > 0 every later mpe_moe_ffn keeps,
+ * per input row (a token's x for gate and up, a routed position's h for
+ * down), its n_channels channels of largest |x| (ties to the lower index; all
+ * of them when the row is shorter) and adds R[:, c] x_c for those channels,
+ * so their weights are exactly the fp16 master values. R is recomputed from a
+ * transposed copy of the masters (the residual store, 2 bytes per weight)
+ * and each expert's current scale.
+ *   n_channels  0 (off: the store is released) .. MPE_MAX_COMP_CHANNELS
+ *   store       MPE_STORE_DEVICE or MPE_STORE_HOST
+ * Synchronous (builds the store from the borrowed masters; mpe_quantize_experts
+ * rebuilds it). While on, MPE_PATH_AUTO takes the streaming path and
+ * mpe_moe_ffn fails with MPE_ERR_INVALID under MPE_PATH_PREFILL.
+ * MPE_ERR_ORDER before mpe_quantize_experts; MPE_ERR_CUDA if the store cannot
+ * be allocated (compensation stays off).
+ */
+int mpe_set_compensation(mpe_ctx* ctx, int32_t n_channels, int32_t store);
+
+/*
+ * mpe_get_kept_channels -- the channels the last compensated mpe_moe_ffn kept:
+ * which = 0: per token, x's channels (gate and up), int32 [T][n];
+ * which = 1: per route position, h's channels (down), int32 [T k][n]
+ * (route positions: the experts' buckets in expert order, the slots of an
+ * expert in assignment order t k + j). A row holds min(n, row length)
+ * ascending entries; n is the compensation's n_channels.
+ *   idx_host  host, int32, at least cap entries
+ * Synchronous. MPE_ERR_ORDER if compensation is off or nothing ran yet;
+ * MPE_ERR_INVALID if cap is too small.
+ */
+int mpe_get_kept_channels(mpe_ctx* ctx, int32_t which, int32_t* idx_host, size_t cap);
+
+/*
+ * mpe_select_salient -- the channel choice of the compensation on its own:
+ * for each of n_rows rows of n_cols bf16 values, the n channels of largest
+ * magnitude (ties to the lower index), ascending; every channel when
+ * n >= n_cols. Allocates nothing; asynchronous on `stream`.
+ *   rows_bf16  device, bf16 [n_rows][n_cols], row-major
+ *   idx_out    device, int32 [n_rows][n]; row r's first min(n, n_cols)
+ *              entries are written
+ *   n          1 .. MPE_MAX_COMP_CHANNELS
+ *   stream     cudaStream_t (NULL: the default stream)
+ */
+int mpe_select_salient(const void* rows_bf16, int32_t n_rows, int32_t n_cols, int32_t n,
+                       int32_t* idx_out, void* stream);
 
 /*
  * mpe_repage -- budget change with KV-cache occupancy ("Implementation
@@ -368,7 +422,8 @@ int mpe_profile_enable(mpe_ctx* ctx, int32_t enable);
  * mpe_profile_read -- synchronise and sum the recorded kernel times per slot
  * (0 route, 1 gate/up, 2 SwiGLU reduce, 3 down, 4 combine -- the streaming
  * path; 5 gate/up, 6 down, 7 token permute -- the tensor-core path; route
- * and combine are shared): ms_host
+ * and combine are shared; 8 salient-channel selection, 9 compensation --
+ * with mpe_set_compensation): ms_host
  * double[n_slots] milliseconds, launches_host int64[n_slots] counts (either
  * may be NULL). reset != 0 clears the records.
  */

@@ -31,6 +31,8 @@ STATUS_NONFINITE = 0x2
 STATUS_WAIT_TIMEOUT = 0x4
 PATH_AUTO, PATH_DECODE, PATH_PREFILL = 0, 1, 2
 ALLOCATOR_EXACT, ALLOCATOR_PROPORTIONAL, ALLOCATOR_MEASURED = 0, 1, 2
+STORE_DEVICE, STORE_HOST = 0, 1
+MAX_COMP_CHANNELS = 256
 ALLOC_STATE_CAP = 65536
 MAX_EXPERTS = 1024
 
@@ -38,7 +40,8 @@ MAX_EXPERTS = 1024
 EXPORTS = [
     "mpe_create", "mpe_destroy", "mpe_set_stream", "mpe_set_path", "mpe_allocate_bits",
     "mpe_allocate_bits_proportional", "mpe_allocate_bits_table", "mpe_set_allocator",
-    "mpe_measure_loss", "mpe_repage_async", "mpe_repage_commit",
+    "mpe_measure_loss", "mpe_repage_async", "mpe_repage_commit", "mpe_set_compensation",
+    "mpe_select_salient", "mpe_get_kept_channels",
     "mpe_quantize_experts", "mpe_repage", "mpe_moe_ffn", "mpe_moe_ffn_host", "mpe_route",
     "mpe_get_page_table", "mpe_expert_stream_bytes", "mpe_read_expert_packed",
     "mpe_get_scales", "mpe_get_bits", "mpe_get_status", "mpe_last_error",
@@ -46,7 +49,7 @@ EXPORTS = [
     "mpe_profile_read", "mpe_route_noalloc",
 ]
 PROFILE_SLOTS = ["route", "gate_up", "swiglu_reduce", "down", "combine", "tc_gate_up",
-                 "tc_down", "tc_permute"]
+                 "tc_down", "tc_permute", "select", "compensate"]
 
 
 class MpeError(RuntimeError):
@@ -94,6 +97,9 @@ def lib() -> ctypes.CDLL:
         "mpe_allocate_bits_proportional": (i32, [vp, vp, i32, u64, vp]),
         "mpe_allocate_bits_table": (i32, [vp, vp, vp, i32, u64, vp]),
         "mpe_measure_loss": (i32, [vp, vp]),
+        "mpe_set_compensation": (i32, [vp, i32, i32]),
+        "mpe_select_salient": (i32, [vp, i32, i32, i32, vp, vp]),
+        "mpe_get_kept_channels": (i32, [vp, i32, vp, sz]),
         "mpe_set_allocator": (i32, [vp, i32]),
         "mpe_repage_async": (i32, [vp, u64, vp, vp]),
         "mpe_repage_commit": (i32, [vp, i32, vp]),
@@ -179,6 +185,18 @@ def allocate_bits_table(p, loss, W, B: int) -> np.ndarray:
     return out
 
 
+def select_salient(rows, n: int, out=None):
+    """Per row of a bf16 CUDA matrix [rows, cols]: the n channels of largest
+    magnitude (ties to the lower index), ascending; int32 [rows, n] (a row's
+    first min(n, cols) entries). Current stream."""
+    import torch
+    R, C = rows.shape
+    if out is None:
+        out = torch.full((R, n), -1, dtype=torch.int32, device=rows.device)
+    _check(lib().mpe_select_salient(_ptr(rows), R, C, n, _ptr(out), _stream()))
+    return out
+
+
 def route_noalloc(ids, E: int, perm, offsets, inv):
     """Bucketing into caller-provided device buffers without any device
     allocation (mpe_route_noalloc); runs on the current stream."""
@@ -223,6 +241,20 @@ class Context:
         """ALLOCATOR_EXACT (default), ALLOCATOR_PROPORTIONAL or ALLOCATOR_MEASURED
         for later repages."""
         _check(lib().mpe_set_allocator(self._h, allocator), self._h)
+
+    def set_compensation(self, n_channels: int, store: int = STORE_DEVICE):
+        """Compensate the n_channels salient input channels of every projection
+        on the streaming path (0: off); the residual store in device memory
+        (STORE_DEVICE) or mapped host memory (STORE_HOST)."""
+        self._sync_stream()
+        _check(lib().mpe_set_compensation(self._h, int(n_channels), int(store)), self._h)
+
+    def kept_channels(self, which: int, rows: int, n: int) -> np.ndarray:
+        """int32 [rows, n]: the last compensated forward's kept channels of x
+        (which 0, rows = T) or of h (which 1, rows = T k, by route position)."""
+        out = np.zeros((rows, n), dtype=np.int32)
+        _check(lib().mpe_get_kept_channels(self._h, which, _ptr(out), out.size), self._h)
+        return out
 
     def measure_loss(self) -> np.ndarray:
         """float64[E, 3]: each expert's measured quantization MSE at 3, 4, 8 bits."""

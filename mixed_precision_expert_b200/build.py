@@ -19,7 +19,8 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libmpe.so")
 
-SOURCES = ["api.cu", "quantize.cu", "allocate.cu", "route.cu", "decode.cu", "combine.cu", "prefill.cu"]
+SOURCES = ["api.cu", "quantize.cu", "allocate.cu", "route.cu", "decode.cu", "combine.cu", "prefill.cu",
+           "compensate.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-std=c++17", "-O3", "-lineinfo", "-Xcompiler", "-fPIC", "-DNDEBUG"]
 

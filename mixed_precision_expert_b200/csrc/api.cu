@@ -473,6 +473,8 @@ void mpe_destroy(mpe_ctx* c) {
         cudaFree(c->d_W); cudaFree(c->d_bits_out); cudaFree(c->d_alloc_status);
         cudaFree(c->d_choice); cudaFree(c->d_D); cudaFree(c->d_gather);
         cudaFree(c->d_loss); cudaFree(c->d_mse_acc);
+        cudaFree(c->comp_dev); cudaFree(c->sel_x); cudaFree(c->sel_h);
+        if (c->comp_host) cudaFreeHost(c->comp_host);
         cudaFreeHost(c->h_pte_pinned); cudaFreeHost(c->h_pidx_pinned);
         cudaFreeHost(c->h_list_pinned); cudaFreeHost(c->h_masters_pinned);
         cudaFreeHost(c->h_p_pinned); cudaFreeHost(c->h_w_pinned); cudaFreeHost(c->h_alloc_pinned);
@@ -619,6 +621,84 @@ int mpe_allocate_bits_proportional(const double* p, const uint64_t* W, int32_t E
     return rc;
 }
 
+int mpe_set_compensation(mpe_ctx* c, int32_t n_channels, int32_t store) {
+    if (!c) return fail_global(MPE_ERR_INVALID, "null context");
+    if (n_channels < 0 || n_channels > MPE_MAX_COMP_CHANNELS)
+        return fail(c, MPE_ERR_INVALID, "n_channels %d outside 0 .. %d", n_channels,
+                    MPE_MAX_COMP_CHANNELS);
+    if (store != MPE_STORE_DEVICE && store != MPE_STORE_HOST)
+        return fail(c, MPE_ERR_INVALID, "bad store %d", store);
+    DeviceGuard guard(c->device);
+    CK(cudaStreamSynchronize(c->stream));
+    const bool keep = n_channels > 0 && c->comp_store && c->comp_store_kind == store;
+    if (!keep) {
+        cudaFree(c->comp_dev);
+        if (c->comp_host) cudaFreeHost(c->comp_host);
+        c->comp_dev = nullptr;
+        c->comp_host = nullptr;
+        c->comp_store = nullptr;
+        c->comp_n = 0;
+    }
+    if (n_channels == 0) return MPE_OK;
+    if (!c->absmax_valid) return fail(c, MPE_ERR_ORDER, "compensation before quantize_experts");
+    if (!keep) {
+        const size_t bytes = (size_t)3 * c->H * c->F * c->E * sizeof(__half);
+        if (store == MPE_STORE_DEVICE) {
+            if (cudaMalloc(&c->comp_dev, bytes) != cudaSuccess) {
+                cudaGetLastError();
+                return fail(c, MPE_ERR_CUDA, "residual store: %zu bytes of device memory", bytes);
+            }
+            c->comp_store = c->comp_dev;
+        } else {
+            void* dev = nullptr;
+            if (cudaHostAlloc(&c->comp_host, bytes, cudaHostAllocMapped | cudaHostAllocPortable) !=
+                    cudaSuccess ||
+                cudaHostGetDevicePointer(&dev, c->comp_host, 0) != cudaSuccess) {
+                cudaGetLastError();
+                if (c->comp_host) cudaFreeHost(c->comp_host);
+                c->comp_host = nullptr;
+                return fail(c, MPE_ERR_CUDA, "residual store: %zu bytes of mapped host memory",
+                            bytes);
+            }
+            c->comp_store = reinterpret_cast<const __half*>(dev);
+        }
+        c->comp_store_kind = store;
+        launch_transpose_masters(c, const_cast<__half*>(c->comp_store));
+        CKLAUNCH();
+        CK(cudaStreamSynchronize(c->stream));
+    }
+    c->comp_n = n_channels;
+    return MPE_OK;
+}
+
+int mpe_get_kept_channels(mpe_ctx* c, int32_t which, int32_t* idx_host, size_t cap) {
+    if (!c) return fail_global(MPE_ERR_INVALID, "null context");
+    if (!idx_host || (which != 0 && which != 1)) return fail(c, MPE_ERR_INVALID, "bad argument");
+    if (c->comp_n == 0 || c->last_T == 0) return fail(c, MPE_ERR_ORDER, "no compensated forward yet");
+    const size_t rows = which == 0 ? (size_t)c->last_T : (size_t)c->last_T * c->last_k;
+    const size_t need = rows * (size_t)c->comp_n;
+    if (cap < need) return fail(c, MPE_ERR_INVALID, "cap %zu < %zu entries", cap, need);
+    DeviceGuard guard(c->device);
+    CK(cudaMemcpyAsync(idx_host, which == 0 ? c->sel_x : c->sel_h, need * sizeof(int32_t),
+                       cudaMemcpyDeviceToHost, c->stream));
+    CK(cudaStreamSynchronize(c->stream));
+    return MPE_OK;
+}
+
+int mpe_select_salient(const void* rows_bf16, int32_t n_rows, int32_t n_cols, int32_t n,
+                       int32_t* idx_out, void* stream) {
+    if (n_rows < 0 || n_cols < 1 || n < 1 || n > MPE_MAX_COMP_CHANNELS)
+        return fail_global(MPE_ERR_INVALID, "bad n_rows %d, n_cols %d or n %d", n_rows, n_cols, n);
+    if (n_rows == 0) return MPE_OK;
+    if (!rows_bf16 || !idx_out) return fail_global(MPE_ERR_INVALID, "null argument");
+    launch_select_channels(nullptr, reinterpret_cast<const __nv_bfloat16*>(rows_bf16),
+                           (size_t)n_cols, n_rows, n_cols, nullptr, n, idx_out,
+                           reinterpret_cast<cudaStream_t>(stream));
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail_global(MPE_ERR_CUDA, "select_salient: %s", cudaGetErrorString(e));
+    return MPE_OK;
+}
+
 int mpe_set_allocator(mpe_ctx* c, int32_t allocator) {
     if (!c) return fail_global(MPE_ERR_INVALID, "null context");
     if (allocator != MPE_ALLOCATOR_EXACT && allocator != MPE_ALLOCATOR_PROPORTIONAL &&
@@ -661,6 +741,7 @@ int mpe_quantize_experts(mpe_ctx* c, const void* const* master_f16, const uint8_
     launch_absmax(c, c->d_list, c->E);
     launch_scales(c);
     launch_encode(c, c->d_list, c->E);
+    if (c->comp_n > 0) launch_transpose_masters(c, const_cast<__half*>(c->comp_store));
     CKLAUNCH();
     c->absmax_valid = true;
     c->loss_valid = false;
@@ -789,6 +870,7 @@ struct KernelSpan {
 constexpr size_t kPrefillMinAvg = 32;
 
 static bool use_prefill(const mpe_ctx* c, size_t Tk) {
+    if (c->comp_n > 0) return false;  // compensation runs on the streaming path
     if (c->path == MPE_PATH_PREFILL) return true;
     if (c->path == MPE_PATH_DECODE) return false;
     return Tk >= kPrefillMinAvg * (size_t)c->E;
@@ -815,6 +897,22 @@ static int grow_xp(mpe_ctx* c, size_t need) {
     int r;
     if ((r = dev_alloc(c, &c->s.xp, need))) return r;
     c->s.xp_cap = need;
+    return MPE_OK;
+}
+
+// kept-channel lists for Tk rows (x uses the first T of them)
+static int grow_sel(mpe_ctx* c, size_t Tk) {
+    const size_t need = Tk * (size_t)c->comp_n;
+    if (need <= c->sel_cap) return MPE_OK;
+    CK(cudaStreamSynchronize(c->stream));
+    cudaFree(c->sel_x);
+    cudaFree(c->sel_h);
+    c->sel_x = c->sel_h = nullptr;
+    c->sel_cap = 0;
+    int r;
+    if ((r = dev_alloc(c, &c->sel_x, need))) return r;
+    if ((r = dev_alloc(c, &c->sel_h, need))) return r;
+    c->sel_cap = need;
     return MPE_OK;
 }
 
@@ -856,7 +954,11 @@ static int moe_ffn_device(mpe_ctx* c, const void* x, int32_t T, const int32_t* i
     }
     DecodePlan pl;
     decode_plan(c, Tk, pl);
-    const size_t need_part = pl.p_gu > 1 ? (size_t)pl.p_gu * 2 * Tk * c->F : 0;
+    // compensation adds one slice after the gate/up partials and one after the
+    // down partials, so the gate/up kernel always writes partials then
+    const int ec = c->comp_n > 0 ? 1 : 0;
+    const int p_gu = pl.p_gu + ec, p_dn = pl.p_dn + ec;
+    const size_t need_part = p_gu > 1 ? (size_t)p_gu * 2 * Tk * c->F : 0;
     if (need_part > c->s.part_cap) {
         CK(cudaStreamSynchronize(c->stream));
         cudaFree(c->s.part);
@@ -865,22 +967,44 @@ static int moe_ffn_device(mpe_ctx* c, const void* x, int32_t T, const int32_t* i
         if ((r = dev_alloc(c, &c->s.part, need_part))) return r;
         c->s.part_cap = need_part;
     }
-    if ((r = grow_y(c, (size_t)pl.p_dn * Tk * c->H))) return r;
+    if ((r = grow_y(c, (size_t)p_dn * Tk * c->H))) return r;
+    if (ec) {
+        if ((r = grow_sel(c, Tk))) return r;
+        c->last_T = T;
+        c->last_k = k;
+        KernelSpan sp(c, 8);
+        launch_select_channels(c, xb, c->H, T, c->H, nullptr, c->comp_n, c->sel_x, c->stream);
+    }
     {
         KernelSpan sp(c, 1);
-        launch_decode_gateup(c, xb, k, Tk, pl.p_gu, pl.kb_gu, pl.claim);
+        launch_decode_gateup(c, xb, k, Tk, pl.p_gu, pl.kb_gu, pl.claim, ec != 0);
     }
-    if (pl.p_gu > 1) {
+    if (ec) {
+        KernelSpan sp(c, 9);
+        launch_comp_gateup(c, xb, k, Tk, c->sel_x, c->comp_n, c->comp_store,
+                           c->s.part + (size_t)pl.p_gu * 2 * Tk * c->F);
+    }
+    if (p_gu > 1) {
         KernelSpan sp(c, 2);
-        launch_swiglu_reduce(c, Tk, pl.p_gu);
+        launch_swiglu_reduce(c, Tk, p_gu);
+    }
+    if (ec) {
+        KernelSpan sp(c, 8);
+        launch_select_channels(c, c->s.h, c->F, (int)Tk, c->F, c->s.offsets + c->E, c->comp_n,
+                               c->sel_h, c->stream);
     }
     {
         KernelSpan sp(c, 3);
         launch_decode_down(c, Tk, pl.p_dn, pl.kb_dn, pl.claim);
     }
+    if (ec) {
+        KernelSpan sp(c, 9);
+        launch_comp_down(c, Tk, c->sel_h, c->comp_n, c->comp_store,
+                         c->s.y + (size_t)pl.p_dn * Tk * c->H);
+    }
     {
         KernelSpan sp(c, 4);
-        launch_combine_by_position(c, w, T, k, pl.p_dn, reinterpret_cast<__nv_bfloat16*>(out));
+        launch_combine_by_position(c, w, T, k, p_dn, reinterpret_cast<__nv_bfloat16*>(out));
     }
     CKLAUNCH();
     return MPE_OK;
@@ -895,6 +1019,8 @@ int mpe_moe_ffn(mpe_ctx* c, const void* x, int32_t T, const int32_t* ids, const 
     if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(out)) & 15)
         return fail(c, MPE_ERR_INVALID, "x and out must be 16-byte aligned");
     if (!c->absmax_valid) return fail(c, MPE_ERR_ORDER, "moe_ffn before quantize_experts");
+    if (c->comp_n > 0 && c->path == MPE_PATH_PREFILL)
+        return fail(c, MPE_ERR_INVALID, "compensation runs on the streaming path only");
     DeviceGuard guard(c->device);
     return moe_ffn_device(c, x, T, ids, w, k, out);
 }

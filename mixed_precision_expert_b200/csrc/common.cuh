@@ -76,6 +76,34 @@ __device__ __forceinline__ const uint8_t* chunk_addr(const PagedExperts& P, cons
 }
 
 // ---------------------------------------------------------------------------
+// the quantizer's rounding: k = round-half-even(w / s), exactly
+// ---------------------------------------------------------------------------
+// Rare path: r = w (1/s) lies within 2^-11 of a half-integer, so the exact
+// quotient w / s decides. The sign of the single-rounded fma (k -+ 1/2) s - w is
+// exact: ties go to the even integer.
+static __device__ __noinline__ float tie_fix(float w, float s, float kf) {
+    const float lo = __fmaf_rn(__fsub_rn(kf, 0.5f), s, -w);  // (k - 1/2) s - w
+    const float hi = __fmaf_rn(__fadd_rn(kf, 0.5f), s, -w);  // (k + 1/2) s - w
+    const bool odd = (((int)kf) & 1) != 0;
+    if (lo > 0.0f) return __fsub_rn(kf, 1.0f);
+    if (hi < 0.0f) return __fadd_rn(kf, 1.0f);
+    if (lo == 0.0f && odd) return __fsub_rn(kf, 1.0f);
+    if (hi == 0.0f && odd) return __fadd_rn(kf, 1.0f);
+    return kf;
+}
+
+// k as a float for |w / s| < 2^8, s > 0, inv_s = RN(1 / s): r = w inv_s is
+// within ~2^-16 of the exact quotient; adding 1.5 * 2^23 rounds it to an
+// integer (ties to even), which agrees with rounding the exact quotient unless
+// r lies within 2^-11 of a half-integer, where tie_fix decides.
+__device__ __forceinline__ float exact_code(float w, float s, float inv_s) {
+    constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+    const float r = __fmul_rn(w, inv_s);
+    const float kf = __fsub_rn(__fadd_rn(r, kRound), kRound);
+    return fabsf(__fsub_rn(r, kf)) > 0.4990234375f ? tie_fix(w, s, kf) : kf;
+}
+
+// ---------------------------------------------------------------------------
 // timers and bounded waits
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint64_t global_ns() {

@@ -140,6 +140,7 @@ struct Args {
     size_t part_stride;        // floats per part slice (gate/up partials or down y)
     int32_t* task_ctr;         // claimed-task counters (one per class), zero at launch
     int parts;                 // P
+    int direct_h;              // gate/up with P = 1: write h itself (else the partial)
     int kb;                    // blocks per part
     uint32_t* status;
 };
@@ -355,7 +356,7 @@ __device__ __forceinline__ void finish(const Args& a, const Task& T, int tau,
             if (GATEUP) {
                 const float gv = T.scale * acc[nt][0][q];
                 const float uv = T.scale * acc[nt][GATEUP ? 1 : 0][q];
-                if (a.parts == 1) {
+                if (a.direct_h) {
                     const float hv = gv / (1.0f + __expf(-gv)) * uv;
                     a.h_out[(size_t)pos * F + row] = __float2bfloat16_rn(hv);
                 } else {
@@ -931,7 +932,7 @@ static int persistent_grid(mpe_ctx* c, const void* fn, size_t smem) {
 }
 
 void launch_decode_gateup(mpe_ctx* c, const __nv_bfloat16* x, int k, size_t Tk, int parts,
-                          int kb, int claim) {
+                          int kb, int claim, bool partials) {
     (void)claim;
     Args a{};
     a.P = paged(c);
@@ -945,6 +946,7 @@ void launch_decode_gateup(mpe_ctx* c, const __nv_bfloat16* x, int k, size_t Tk, 
     a.part_stride = (size_t)2 * Tk * c->F;
     a.task_ctr = c->s.task_ctr;
     a.parts = parts;
+    a.direct_h = (parts == 1 && !partials) ? 1 : 0;
     a.kb = kb;
     a.status = c->d_status;
     const int grid = persistent_grid(c, (const void*)k_decode<true>, smem_bytes());

@@ -1,6 +1,7 @@
 // Host-side context of libmpe and the launch wrappers each kernel file exports.
 #pragma once
 
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -47,8 +48,9 @@ struct Scratch {
 
 // CUDA-event records around the forward-pass kernels (optional tracing).
 // route, gate/up, swiglu reduce, down, combine, tensor-core gate/up, tensor-core
-// down, token permute (tensor-core path)
-constexpr int kProfileSlots = 8;
+// down, token permute (tensor-core path), salient-channel selection,
+// compensation
+constexpr int kProfileSlots = 10;
 struct ProfileRecord {
     int slot;
     cudaEvent_t start, stop;
@@ -88,6 +90,17 @@ struct mpe_ctx {
     size_t choice_cap = 0;
     double* d_D = nullptr;            // two DP rows
     double* d_loss = nullptr;         // measured MSE per expert and width [E][3]
+    // salient-channel compensation: channels kept per row (0: off), the
+    // residual store (device or mapped host memory) and the kept-channel lists
+    int comp_n = 0;
+    int comp_store_kind = MPE_STORE_DEVICE;
+    const __half* comp_store = nullptr;  // device-visible address of the store
+    __half* comp_dev = nullptr;          // the store when in device memory
+    void* comp_host = nullptr;           // the store when in mapped host memory
+    int32_t* sel_x = nullptr;            // [T][comp_n] kept channels of x
+    int32_t* sel_h = nullptr;            // [T k][comp_n] kept channels of h
+    size_t sel_cap = 0;                  // entries of each
+    int last_T = 0, last_k = 0;          // shape of the last compensated forward
     unsigned long long* d_mse_acc = nullptr;  // its exact sums [E][3][2]
     bool loss_valid = false;          // d_loss holds the current master's values
     uint8_t* d_gather = nullptr;      // expert stream gather buffer
@@ -182,6 +195,20 @@ size_t allocate_choice_bytes(int E, uint64_t R);
 void launch_allocate_proportional(cudaStream_t st, const double* p, const uint64_t* W, int E,
                                   uint64_t B, uint64_t sum_w, uint8_t* bits_out, int32_t* status);
 
+// compensate.cu (salient-channel error compensation, streaming path)
+// the residual store: every expert's master transposed per matrix
+void launch_transpose_masters(mpe_ctx* c, __half* store);
+// kept channels of rows [n_rows][ld] (first n_cols used), out [n_rows][n];
+// rows at or beyond *n_rows_dev skipped when it is given; c may be null
+void launch_select_channels(mpe_ctx* c, const __nv_bfloat16* rows, size_t ld, int n_rows,
+                            int n_cols, const int32_t* n_rows_dev, int n, int32_t* out,
+                            cudaStream_t st);
+// compensation slices: gate/up out [Tk][2F], down out [Tk][H]
+void launch_comp_gateup(mpe_ctx* c, const __nv_bfloat16* x, int k, size_t Tk, const int32_t* sel,
+                        int n, const __half* store, float* out);
+void launch_comp_down(mpe_ctx* c, size_t Tk, const int32_t* sel, int n, const __half* store,
+                      float* out);
+
 // route.cu
 void launch_route(mpe_ctx* c, const int32_t* ids, int Tk, int k, int32_t* perm,
                   int32_t* offsets, int32_t* inv, int group);
@@ -192,8 +219,10 @@ struct DecodePlan {
     int p_gu = 1, kb_gu = 1, p_dn = 1, kb_dn = 1, claim = 1;
 };
 void decode_plan(mpe_ctx* c, size_t Tk, DecodePlan& pl);
+// partials: write the gate/up partial slice even when parts == 1 (a later
+// pass adds more slices before the SwiGLU)
 void launch_decode_gateup(mpe_ctx* c, const __nv_bfloat16* x, int k, size_t Tk, int parts,
-                          int kb, int claim);
+                          int kb, int claim, bool partials);
 void launch_decode_down(mpe_ctx* c, size_t Tk, int parts, int kb, int claim);
 
 // prefill.cu (tcgen05 grouped GEMM; work groups of up to kPrefillGroup positions)

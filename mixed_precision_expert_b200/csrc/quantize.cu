@@ -70,20 +70,6 @@ __global__ void k_scales(Pte* pte, const uint32_t* absmax, int E, uint32_t* stat
     pte[e].scale = (m == 0) ? 0.0f : __fdiv_rn(mf, (float)q_levels(b));
 }
 
-// Rare path of round_bits: r lies within 2^-11 of a half-integer, so the exact
-// quotient w / s decides. The sign of the single-rounded fma (k -+ 1/2) s - w is
-// exact: ties go to the even integer.
-__device__ __noinline__ float tie_fix(float w, float s, float kf) {
-    const float lo = __fmaf_rn(__fsub_rn(kf, 0.5f), s, -w);  // (k - 1/2) s - w
-    const float hi = __fmaf_rn(__fadd_rn(kf, 0.5f), s, -w);  // (k + 1/2) s - w
-    const bool odd = (((int)kf) & 1) != 0;
-    if (lo > 0.0f) return __fsub_rn(kf, 1.0f);
-    if (hi < 0.0f) return __fadd_rn(kf, 1.0f);
-    if (lo == 0.0f && odd) return __fsub_rn(kf, 1.0f);
-    if (hi == 0.0f && odd) return __fadd_rn(kf, 1.0f);
-    return kf;
-}
-
 // Rounding of one weight. r = w * (1/s) is within ~2^-16 of the exact
 // quotient (|w/s| < 2^8). Adding 1.5 * 2^23 rounds r to an integer, ties to
 // even, and leaves that integer k in the low mantissa bits: the returned bit
@@ -293,10 +279,7 @@ __device__ __forceinline__ MseWidth mse_width(float mf, int q) {
 // k = round-half-even(w / s) exactly (same rounding as the encoder), then the
 // scaled error (w - k s) / Q as an exactly integer-valued float.
 __device__ __forceinline__ float mse_scaled_error(float w, const MseWidth& m) {
-    constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-    const float r = __fmul_rn(w, m.inv_s);
-    float kf = __fsub_rn(__fadd_rn(r, kRound), kRound);
-    if (fabsf(__fsub_rn(r, kf)) > 0.4990234375f) kf = tie_fix(w, m.s, kf);
+    const float kf = exact_code(w, m.s, m.inv_s);
     return __fmul_rn(__fmaf_rn(-kf, m.s, w), m.sc);  // exact error, exact scaling
 }
 

@@ -53,24 +53,33 @@ def compensated_linear(w_hat: np.ndarray, w: np.ndarray, x: np.ndarray, n: int) 
     return w_hat @ x + (w[:, sel] - w_hat[:, sel]) @ x[sel]
 
 
-def expert_ffn_compensated(x_rows, hat, master, n: int) -> np.ndarray:
+def expert_ffn_compensated(x_rows, hat, master, n: int, down_masks=None) -> np.ndarray:
     """y [rows, H] for input rows x [rows, H]; hat = (W1^, W3^, W2^), master =
-    (W1, W3, W2) in float64 (the fp16 values)."""
+    (W1, W3, W2) in float64 (the fp16 values). down_masks: optional kept
+    channels of each row's h (a list of index arrays) to use instead of
+    choosing them here -- several choices are correct where |h| values tie or
+    nearly tie at the cut, so a parity check takes the device's choice, after
+    checking it is one of them."""
     w1h, w3h, w2h = hat
     w1, w3, w2 = master
     out = []
-    for x in np.asarray(x_rows, dtype=np.float64):
+    for r, x in enumerate(np.asarray(x_rows, dtype=np.float64)):
         g = compensated_linear(w1h, w1, x, n)
         v = compensated_linear(w3h, w3, x, n)
         h = silu(g) * v
-        out.append(compensated_linear(w2h, w2, h, n))
+        if down_masks is None:
+            out.append(compensated_linear(w2h, w2, h, n))
+        else:
+            sel = np.asarray(down_masks[r])
+            out.append(w2h @ h + (w2[:, sel] - w2h[:, sel]) @ h[sel])
     return np.stack(out) if out else np.zeros((0, w2h.shape[0]))
 
 
 def moe_ffn_compensated(x, ids, w, expert_weights: Callable, expert_masters: Callable, E: int,
-                        n: int, tokens=None) -> np.ndarray:
+                        n: int, tokens=None, down_masks=None) -> np.ndarray:
     """The routed layer of ffn.moe_ffn with every projection compensated.
-    expert_weights(e) -> (W1^, W3^, W2^); expert_masters(e) -> (W1, W3, W2)."""
+    expert_weights(e) -> (W1^, W3^, W2^); expert_masters(e) -> (W1, W3, W2);
+    down_masks: optional {(t, j): kept channels of that slot's h}."""
     x = np.asarray(x, dtype=np.float64)
     ids = np.asarray(ids)
     w = np.asarray(w, dtype=np.float64)
@@ -82,11 +91,27 @@ def moe_ffn_compensated(x, ids, w, expert_weights: Callable, expert_masters: Cal
                 if ids[t, j] == e]
         if not rows:
             continue
+        masks = None if down_masks is None else [down_masks[(t, j)] for _, t, j in rows]
         y = expert_ffn_compensated(np.stack([x[t] for _, t, _ in rows]), expert_weights(e),
-                                   expert_masters(e), n)
+                                   expert_masters(e), n, masks)
         for r, (oi, t, j) in enumerate(rows):
             out[oi] += w[t, j] * y[r]
     return out
+
+
+def is_valid_choice(row, kept, n: int, tol: float) -> bool:
+    """True when `kept` (n distinct indices, or every index when n >= len(row))
+    is a largest-|row| choice up to `tol`: no left-out entry exceeds a kept one
+    by more than tol. For checking a choice made on rounded values."""
+    row = np.abs(np.asarray(row, dtype=np.float64))
+    L = row.shape[0]
+    kept = np.asarray(kept)
+    if n >= L:
+        return np.array_equal(np.sort(kept), np.arange(L))
+    if len(kept) != n or len(set(kept.tolist())) != n:
+        return False
+    rest = np.setdiff1d(np.arange(L), kept)
+    return row[rest].max() <= row[kept].min() + tol
 
 
 def error_curve(w_hat: np.ndarray, w: np.ndarray, x: np.ndarray, order) -> np.ndarray:

@@ -105,3 +105,36 @@ def test_figure4_sorted_beats_random():
     for i in (1, 5, 20):
         got = np.mean((C.compensated_linear(w_hat, w, x, i) - w @ x) ** 2)
         assert got == pytest.approx(es[i], rel=1e-9)
+
+
+def test_valid_choice_check():
+    row = np.array([0.1, -3.0, 2.0, 2.001, 0.5])
+    assert C.is_valid_choice(row, C.salient_channels(row, 2), 2, 0.0)  # {1, 3}
+    assert not C.is_valid_choice(row, [1, 2], 2, 0.0)      # 2.001 left out
+    assert C.is_valid_choice(row, [1, 2], 2, 0.01)         # within the tolerance
+    assert not C.is_valid_choice(row, [1, 1], 2, 1.0)      # not distinct
+    assert C.is_valid_choice(row, [0, 1, 2, 3, 4], 9, 0.0)  # n >= len: everything
+    rng = np.random.default_rng(9)
+    for _ in range(50):
+        r = rng.standard_normal(30)
+        n = int(rng.integers(1, 30))
+        assert C.is_valid_choice(r, C.salient_channels(r, n), n, 0.0)
+
+
+def test_down_masks_reproduce_own_choice():
+    masters, hats, x, ids, w, E, H, F = _tiny_layer(seed=6)
+    n = 5
+    # the masks the oracle would choose itself, passed back in: same output
+    masks = {}
+    for t in range(ids.shape[0]):
+        for j in range(ids.shape[1]):
+            e = ids[t, j]
+            w1h, w3h, _ = hats[e]
+            w1, w3, _ = masters[e]
+            g = C.compensated_linear(w1h, w1, x[t], n)
+            v = C.compensated_linear(w3h, w3, x[t], n)
+            masks[(t, j)] = C.salient_channels(of.silu(g) * v, n)
+    a = C.moe_ffn_compensated(x, ids, w, lambda e: hats[e], lambda e: masters[e], E, n)
+    b = C.moe_ffn_compensated(x, ids, w, lambda e: hats[e], lambda e: masters[e], E, n,
+                              down_masks=masks)
+    np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-15)
