@@ -31,11 +31,12 @@
 namespace mpe {
 namespace {
 
-constexpr int kSelThreads = 256;
+constexpr int kHistCopies = 8;     // histogram copies, one per group of warps
 constexpr int kCompThreads = 256;
 
-// Exclusive prefix sum of one int per thread over the CTA; *total gets the
-// sum. Ends with a barrier, so the scratch can be reused at once.
+// Exclusive prefix sum of one int per thread over a CTA of TH threads; *total
+// gets the sum. Ends with a barrier, so the scratch can be reused at once.
+template <int TH>
 __device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp, int* total) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     int inc = v;
@@ -47,7 +48,7 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp, int* tot
     if (lane == 31) s_warp[warp] = inc;
     __syncthreads();
     int before = 0, all = 0;
-    for (int w = 0; w < kSelThreads / 32; ++w) {
+    for (int w = 0; w < TH / 32; ++w) {
         const int t = s_warp[w];
         if (w < warp) before += t;
         all += t;
@@ -58,8 +59,10 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp, int* tot
 }
 
 // Kept channels of row r: out[r][0 .. min(n, n_cols)), ascending. Rows at or
-// beyond *n_rows_dev (when given) are skipped. One CTA a row.
-__global__ void __launch_bounds__(kSelThreads)
+// beyond *n_rows_dev (when given) are skipped. One CTA of TH threads a row
+// (1024 for long rows: short per-thread loops; 256 for short ones).
+template <int TH>
+__global__ void __launch_bounds__(TH)
 k_select_channels(const __nv_bfloat16* rows, size_t ld, int n_cols, const int32_t* n_rows_dev,
                   int n, int32_t* out) {
     const int row = blockIdx.x;
@@ -68,54 +71,55 @@ k_select_channels(const __nv_bfloat16* rows, size_t ld, int n_cols, const int32_
     int32_t* o = out + (size_t)row * n;
     const int tid = threadIdx.x;
     if (n >= n_cols) {
-        for (int c = tid; c < n_cols; c += kSelThreads) o[c] = c;
+        for (int c = tid; c < n_cols; c += TH) o[c] = c;
         return;
     }
     // the row's magnitude keys, read once (all loads in flight) into shared memory
     extern __shared__ uint16_t r[];
 #pragma unroll 8
-    for (int c = tid; c < n_cols; c += kSelThreads) r[c] = src[c] & 0x7FFF;
+    for (int c = tid; c < n_cols; c += TH) r[c] = src[c] & 0x7FFF;
     __syncthreads();
     // per-warp histograms; lanes that hit the same bin add once (match_any), so
     // the common case -- most magnitudes in a few exponent bins -- costs a few
     // shared atomics per warp instruction instead of 32 on one address
-    __shared__ int hist[kSelThreads / 32][256];
-    __shared__ int s_warp[kSelThreads / 32];
+    __shared__ int hist[kHistCopies][256];
+    __shared__ int s_warp[TH / 32];
     __shared__ int s_b1, s_above, s_thr, s_take;
     const int lane = tid & 31, warp = tid >> 5;
     auto count = [&](int bin, bool valid) {
         const unsigned active = __ballot_sync(0xffffffffu, valid);
         if (!valid) return;
         const unsigned peers = __match_any_sync(active, bin);
-        if (lane == __ffs(peers) - 1) atomicAdd(&hist[warp][bin], __popc(peers));
+        if (lane == __ffs(peers) - 1) atomicAdd(&hist[warp % kHistCopies][bin], __popc(peers));
     };
     auto zero = [&]() {
-        for (int i = tid; i < (kSelThreads / 32) * 256; i += kSelThreads) (&hist[0][0])[i] = 0;
+        for (int i = tid; i < kHistCopies * 256; i += TH) (&hist[0][0])[i] = 0;
     };
     auto merged = [&](int bin) {
         int t = 0;
 #pragma unroll
-        for (int w = 0; w < kSelThreads / 32; ++w) t += hist[w][bin];
+        for (int w = 0; w < kHistCopies; ++w) t += hist[w][bin];
         return t;
     };
-    const int n_iter = (n_cols + kSelThreads - 1) / kSelThreads;  // whole warps iterate together
+    const int n_iter = (n_cols + TH - 1) / TH;  // whole warps iterate together
     // pass 1: the high byte of the 15 magnitude bits
     zero();
     __syncthreads();
     for (int it = 0; it < n_iter; ++it) {
-        const int c = it * kSelThreads + tid;
+        const int c = it * TH + tid;
         const bool v = c < n_cols;
         count(v ? r[c] >> 8 : 0, v);
     }
     __syncthreads();
-    // the bin where the count from the top first reaches n: thread t holds bin
-    // 255 - t, so an exclusive scan gives the keys in the bins above it
-    static_assert(kSelThreads == 256, "one thread per bin");
+    // the bin where the count from the top first reaches n: thread t < 256
+    // holds bin 255 - t (the others 0), so an exclusive scan gives the keys in
+    // the bins above it
+    static_assert(TH >= 256, "one thread per bin");
     {
         int all;
-        const int h = merged(255 - tid);
-        const int above = block_exclusive_scan(h, s_warp, &all);
-        if (above < n && above + h >= n) {
+        const int h = tid < 256 ? merged(255 - tid) : 0;
+        const int above = block_exclusive_scan<TH>(h, s_warp, &all);
+        if (tid < 256 && above < n && above + h >= n) {
             s_b1 = 255 - tid;
             s_above = above;  // keys whose high byte exceeds the bin
         }
@@ -126,7 +130,7 @@ k_select_channels(const __nv_bfloat16* rows, size_t ld, int n_cols, const int32_
     zero();
     __syncthreads();
     for (int it = 0; it < n_iter; ++it) {
-        const int c = it * kSelThreads + tid;
+        const int c = it * TH + tid;
         const int key = c < n_cols ? r[c] : -1;
         const bool v = key >= 0 && (key >> 8) == b1;
         count(v ? key & 255 : 0, v);
@@ -134,9 +138,9 @@ k_select_channels(const __nv_bfloat16* rows, size_t ld, int n_cols, const int32_
     __syncthreads();
     {
         int all;
-        const int h = merged(255 - tid);
-        const int above = s_above + block_exclusive_scan(h, s_warp, &all);
-        if (above < n && above + h >= n) {
+        const int h = tid < 256 ? merged(255 - tid) : 0;
+        const int above = s_above + block_exclusive_scan<TH>(h, s_warp, &all);
+        if (tid < 256 && above < n && above + h >= n) {
             s_thr = (b1 << 8) | (255 - tid);  // the n-th largest key
             s_take = n - above;               // keys equal to it that are kept (lowest indices)
         }
@@ -147,7 +151,7 @@ k_select_channels(const __nv_bfloat16* rows, size_t ld, int n_cols, const int32_
     // `take` keys equal to it. Thread t walks its own contiguous segment, so
     // index order is thread order: one scan places each thread's equal keys,
     // a second its kept ones.
-    const int seg = (n_cols + kSelThreads - 1) / kSelThreads;
+    const int seg = (n_cols + TH - 1) / TH;
     const int c_lo = min(n_cols, tid * seg), c_hi = min(n_cols, c_lo + seg);
     int n_gt = 0, n_eq = 0;
     for (int c = c_lo; c < c_hi; ++c) {
@@ -156,9 +160,9 @@ k_select_channels(const __nv_bfloat16* rows, size_t ld, int n_cols, const int32_
         n_eq += key == thr;
     }
     int total;
-    const int eq_before = block_exclusive_scan(n_eq, s_warp, &total);
+    const int eq_before = block_exclusive_scan<TH>(n_eq, s_warp, &total);
     const int eq_keep = max(0, min(n_eq, take - eq_before));
-    int at = block_exclusive_scan(n_gt + eq_keep, s_warp, &total);
+    int at = block_exclusive_scan<TH>(n_gt + eq_keep, s_warp, &total);
     int eq_seen = 0;
     for (int c = c_lo; c < c_hi; ++c) {
         const int key = r[c];
@@ -333,11 +337,15 @@ void launch_select_channels(mpe_ctx* c, const __nv_bfloat16* rows, size_t ld, in
     // the staged row: 2 bytes a column (rows longer than ~110K columns would
     // exceed a CTA's shared memory; the widths of this path are far below)
     const size_t smem = (size_t)n_cols * sizeof(uint16_t);
-    if (smem > 48 * 1024)
-        cudaFuncSetAttribute(k_select_channels, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
-    k_select_channels<<<(unsigned)n_rows, kSelThreads, smem, st>>>(rows, ld, n_cols, n_rows_dev,
-                                                                   n, out);
+    auto launch = [&](auto kernel, int th) {
+        if (smem > 48 * 1024)
+            cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        kernel<<<(unsigned)n_rows, th, smem, st>>>(rows, ld, n_cols, n_rows_dev, n, out);
+    };
+    if (n_cols >= 8192)
+        launch(k_select_channels<1024>, 1024);
+    else
+        launch(k_select_channels<256>, 256);
     if (c) c->launches++;
 }
 
