@@ -181,7 +181,8 @@ def measured_peaks() -> tuple[dict, str]:
                  "bf16_tflops_sustained": FALLBACK_BF16_TFLOPS_SUSTAINED}, "fallback")
 
 
-# the source files each profiled kernel is built from
+# the source files each profiled kernel is built from: its device code and the
+# types and constants it uses (context.h, the host-side context, is not one)
 KERNEL_SOURCES = {
     "k_decode_gateup": ["decode.cu", "common.cuh", "internal.h"],
     "k_prefill_gateup": ["prefill.cu", "common.cuh", "internal.h"],

@@ -63,89 +63,7 @@ struct HostAllocator {
 
 }  // namespace mpe
 
-struct mpe_ctx {
-    int device = 0;
-    int E = 0, H = 0, F = 0;
-    uint32_t page_bytes = MPE_DEFAULT_PAGE_BYTES;
-    uint32_t pool_pages = 0;
-    int path = MPE_PATH_AUTO;
-    int allocator = MPE_ALLOCATOR_EXACT;   // the width rule repage uses
-    cudaStream_t stream = nullptr;
-    std::string err;
-    uint64_t launches = 0;
-
-    // device state
-    uint8_t* pool = nullptr;
-    mpe::Pte* d_pte = nullptr;
-    uint32_t* d_pidx = nullptr;
-    uint32_t* d_absmax = nullptr;     // fp16 bits of max|w| per expert
-    uint32_t* d_status = nullptr;
-    const void** d_masters = nullptr; // E device pointers
-    int32_t* d_list = nullptr;        // expert list for encode
-    double* d_p = nullptr;            // allocator inputs
-    uint64_t* d_W = nullptr;
-    uint8_t* d_bits_out = nullptr;
-    int32_t* d_alloc_status = nullptr;
-    uint8_t* d_choice = nullptr;
-    size_t choice_cap = 0;
-    double* d_D = nullptr;            // two DP rows
-    double* d_loss = nullptr;         // measured MSE per expert and width [E][3]
-    // salient-channel compensation: channels kept per row (0: off), the
-    // residual store (device or mapped host memory) and the kept-channel lists
-    int comp_n = 0;
-    int comp_store_kind = MPE_STORE_DEVICE;
-    const __half* comp_store = nullptr;  // device-visible address of the store
-    __half* comp_dev = nullptr;          // the store when in device memory
-    void* comp_host = nullptr;           // the store when in mapped host memory
-    int32_t* sel_x = nullptr;            // [T][comp_n] kept channels of x
-    int32_t* sel_h = nullptr;            // [T k][comp_n] kept channels of h
-    size_t sel_cap = 0;                  // entries of each
-    int last_T = 0, last_k = 0;          // shape of the last compensated forward
-    unsigned long long* d_mse_acc = nullptr;  // its exact sums [E][3][2]
-    bool loss_valid = false;          // d_loss holds the current master's values
-    uint8_t* d_gather = nullptr;      // expert stream gather buffer
-    size_t gather_cap = 0;
-
-    // host mirrors
-    std::vector<const void*> masters;
-    std::vector<uint8_t> bits;
-    std::vector<mpe::Pte> pte;
-    uint32_t pidx_count = 0;                // entries of the page-index array in use
-    mpe::Pte* h_pte_pinned = nullptr;       // upload staging (pinned)
-    uint32_t* h_pidx_pinned = nullptr;
-    int32_t* h_list_pinned = nullptr;
-    const void** h_masters_pinned = nullptr;
-    double* h_p_pinned = nullptr;           // allocator staging: importances in,
-    uint64_t* h_w_pinned = nullptr;         // expert sizes (uploaded once),
-    int32_t* h_alloc_pinned = nullptr;      // status word + widths out
-    bool w_uploaded = false;
-    cudaEvent_t upload_done = nullptr;      // page-table staging free again
-    cudaEvent_t list_done = nullptr;        // expert-list staging free again
-    bool absmax_valid = false;
-    mpe::HostAllocator alloc;
-    mpe::Scratch s;
-
-    // overlapped repage (mpe_repage_async / mpe_repage_commit): the next page
-    // table is prepared and the changed experts encoded on `side` while work
-    // on `stream` keeps reading the current table
-    cudaStream_t side = nullptr;
-    mpe::Pte* d_pte_next = nullptr;
-    uint32_t* d_pidx_next = nullptr;
-    int32_t* d_list_next = nullptr;
-    mpe::Pte* h_pte_next_pinned = nullptr;
-    uint32_t* h_pidx_next_pinned = nullptr;
-    int32_t* h_list_next_pinned = nullptr;
-    uint32_t pidx_count_next = 0;
-    cudaEvent_t side_done = nullptr;        // the pending repage's device work finished
-    cudaEvent_t old_table_free = nullptr;   // work launched before the last commit finished
-    bool pending = false;
-    std::vector<uint32_t> pending_release;  // old pages of the changed experts
-
-    // tracing
-    bool profiling = false;
-    std::vector<mpe::ProfileRecord> prof;
-    std::vector<cudaEvent_t> event_pool;
-};
+#include "context.h"
 
 namespace mpe {
 
