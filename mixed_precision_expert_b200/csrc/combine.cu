@@ -38,33 +38,52 @@ k_swiglu_reduce(const float* gv, const int32_t* offsets, int E, int F, int parts
 // route position in P K-part slices (P = 1 on the tensor-core path); slots in
 // order, parts summed first in part order; dropped slots (inv < 0) add
 // nothing. One thread per 4 columns of one token; a CTA covers 512 columns of
-// one token row (grid: tokens x column blocks).
+// one token row (grid: tokens x column blocks). The token's positions and
+// weights are read once into shared memory, so every thread can issue all its
+// slots' loads before the first sum.
+constexpr int kCombineSlots = 8;  // slots whose loads are in flight together
+
+template <bool SINGLE>  // one part (no K split): fewer registers, more CTAs
 __global__ void __launch_bounds__(128)
 k_combine_by_position(const float* y, const int32_t* inv, const float* w, int T, int k, int H,
                       int parts, size_t part_stride, __nv_bfloat16* out) {
+    __shared__ int s_pos[32];
+    __shared__ float s_w[32];
     griddep_wait();
     griddep_launch_dependents();
     const int t = blockIdx.x;
+    if (threadIdx.x < k) {
+        s_pos[threadIdx.x] = inv[t * k + threadIdx.x];
+        s_w[threadIdx.x] = w[t * k + threadIdx.x];
+    }
+    __syncthreads();
     const int i = blockIdx.y * blockDim.x + threadIdx.x;  // float4 column index
     if (i >= H / 4) return;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (parts == 1) {
-        // a plain loop: the slots' loads are independent and issue together
-        for (int j = 0; j < k; ++j) {
-            const int pos = inv[t * k + j];
-            if (pos < 0) continue;
-            const float wj = w[t * k + j];
-            const float4 v = reinterpret_cast<const float4*>(y + (size_t)pos * H)[i];
-            acc.x = fmaf(wj, v.x, acc.x);
-            acc.y = fmaf(wj, v.y, acc.y);
-            acc.z = fmaf(wj, v.z, acc.z);
-            acc.w = fmaf(wj, v.w, acc.w);
+    if constexpr (SINGLE) {
+        for (int j0 = 0; j0 < k; j0 += kCombineSlots) {
+            float4 v[kCombineSlots];
+#pragma unroll
+            for (int r = 0; r < kCombineSlots; ++r) {
+                const int pos = j0 + r < k ? s_pos[j0 + r] : -1;
+                v[r] = pos >= 0 ? reinterpret_cast<const float4*>(y + (size_t)pos * H)[i]
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int r = 0; r < kCombineSlots; ++r) {
+                if (j0 + r >= k || s_pos[j0 + r] < 0) continue;
+                const float wj = s_w[j0 + r];
+                acc.x = fmaf(wj, v[r].x, acc.x);
+                acc.y = fmaf(wj, v[r].y, acc.y);
+                acc.z = fmaf(wj, v[r].z, acc.z);
+                acc.w = fmaf(wj, v[r].w, acc.w);
+            }
         }
     } else {
         for (int j = 0; j < k; ++j) {
-            const int pos = inv[t * k + j];
+            const int pos = s_pos[j];
             if (pos < 0) continue;
-            const float wj = w[t * k + j];
+            const float wj = s_w[j];
             const float4* src = reinterpret_cast<const float4*>(y + (size_t)pos * H) + i;
             const size_t stride = part_stride / 4;
             float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -112,8 +131,14 @@ void launch_combine_by_position(mpe_ctx* c, const float* w, int T, int k, int pa
                                 __nv_bfloat16* out) {
     const int n4 = c->H / 4;
     dim3 grid((unsigned)T, (unsigned)((n4 + 127) / 128));
-    launch_pdl(k_combine_by_position, grid, dim3(128), 0, c->stream, (const float*)c->s.y,
-               (const int32_t*)c->s.inv, w, T, k, c->H, parts, (size_t)T * k * c->H, out);
+    if (parts == 1)
+        launch_pdl(k_combine_by_position<true>, grid, dim3(128), 0, c->stream,
+                   (const float*)c->s.y, (const int32_t*)c->s.inv, w, T, k, c->H, parts,
+                   (size_t)T * k * c->H, out);
+    else
+        launch_pdl(k_combine_by_position<false>, grid, dim3(128), 0, c->stream,
+                   (const float*)c->s.y, (const int32_t*)c->s.inv, w, T, k, c->H, parts,
+                   (size_t)T * k * c->H, out);
     c->launches++;
 }
 
