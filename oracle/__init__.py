@@ -27,6 +27,9 @@ Quantization", llmdb.app summary page):
 * ``compensate`` -- dynamic error compensation of salient input channels
   (DecDEC summary, 3.1-3.2 and Figure 4): (W^ + R (.) M) x with R = W - W^
   and M keeping the channels of largest |x|.
+* ``prefix``    -- the prefix-compatible variant: a nested grid (the b-bit
+  code is the top b bits of the 8-bit one) stored in layers, so a width
+  change drops or adds layers instead of re-encoding.
 * ``ffn``       -- dequantize-then-multiply expert FFN (PagedWeight, "Dynamic
   Paging": fetch pages, dequantize on the fly; DecDEC summary, 2.2: weight-only
   quantization dequantizes before multiplying with full-precision
