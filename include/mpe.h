@@ -436,6 +436,62 @@ uint64_t mpe_kernel_launches(mpe_ctx* ctx);
 /* mpe_version -- library version, e.g. 100 for 0.1.0. */
 int32_t mpe_version(void);
 
+/* ------------------------------------------------------------------------
+ * Prefix-compatible variant (a separate store). A nested grid -- 2^b uniform
+ * bins over [-m, m], m = max |w| of the expert, values at the bin centres --
+ * makes every width's code the top bits of the 8-bit code:
+ *   u8 = clamp(floor(128 w / m) + 128, 0, 255), u_b = u8 >> (8 - b),
+ *   w^_b = (m / 2^b)(2 u_b + 1 - 2^b).
+ * The codes are stored in layers, each in its own pages: A = u8 >> 5
+ * (3 bits), B = bit 4 of u8, C = u8 & 15; a b-bit expert holds A, A B or
+ * A B C. Layer streams: the rows of W1 | W3 | W2 in order, each in groups of
+ * 32 codes of 3 / 1 / 4 words (code i at bits (3|1|4) i of the group's
+ * little-endian string); a page holds whole groups. Lowering a width frees
+ * the dropped layers' pages and encodes nothing; raising it adds pages for
+ * the new layers and encodes only those (one read of the master). Placement
+ * takes the lowest free pages, experts ascending, layers A, B, C; a repage
+ * frees first (ascending e) and allocates after (ascending e).
+ * ------------------------------------------------------------------------ */
+typedef struct mpe_prefix mpe_prefix;
+
+/* mpe_prefix_create -- a store for cfg->E experts of cfg->H x cfg->F (path is
+ * ignored; pool_pages 0 = every expert at 8 bits). *out is owned by the
+ * caller (mpe_prefix_destroy). MPE_ERR_INVALID / MPE_ERR_CUDA. */
+int mpe_prefix_create(mpe_prefix** out, const mpe_config* cfg);
+void mpe_prefix_destroy(mpe_prefix* store);
+const char* mpe_prefix_last_error(mpe_prefix* store);
+
+/* mpe_prefix_quantize -- m_e and all stored layers of every expert at the
+ * given widths. master_f16: host array of E device pointers as for
+ * mpe_quantize_experts (borrowed; repage re-reads it); bits: host uint8[E],
+ * each 3, 4 or 8. Synchronous. MPE_ERR_POOL if the pool is too small. */
+int mpe_prefix_quantize(mpe_prefix* store, const void* const* master_f16, const uint8_t* bits);
+
+/* mpe_prefix_repage -- new widths (host uint8[E]); *bytes_moved_out (may be
+ * NULL) receives the bytes the change moved: per expert that gains layers,
+ * one read of its master (2 bytes a weight) plus the added layers written;
+ * experts that only lose layers move nothing. Synchronous; waits for work
+ * already queued (it may read the dropped pages). MPE_ERR_POOL leaves
+ * everything unchanged. */
+int mpe_prefix_repage(mpe_prefix* store, const uint8_t* new_bits, uint64_t* bytes_moved_out);
+
+/* mpe_prefix_moe_ffn -- the routed SwiGLU layer from the layered store, same
+ * arguments and result layout as mpe_moe_ffn (x, ids, w, out device, x
+ * 16-byte aligned, k <= 32; ids outside [0, E) contribute nothing). The
+ * expert is dequantized as w^_b above. Asynchronous on the store's stream. */
+int mpe_prefix_moe_ffn(mpe_prefix* store, const void* x_bf16, int32_t T, const int32_t* ids,
+                       const float* w, int32_t k, void* out_bf16);
+
+/* mpe_prefix_read_layer -- layer (0 A, 1 B, 2 C) of expert e in stream order
+ * into host_dst (uint32 words; 3 H F / 32 groups of 3 / 1 / 4 words), read
+ * through the device page table. Synchronous. MPE_ERR_INVALID if the layer
+ * is not stored or the buffer is short. */
+int mpe_prefix_read_layer(mpe_prefix* store, int32_t e, int32_t layer, void* host_dst,
+                          size_t bytes);
+
+/* mpe_prefix_get_absmax -- m_e of every expert (host float[E]). */
+int mpe_prefix_get_absmax(mpe_prefix* store, float* m_host);
+
 #ifdef __cplusplus
 }
 #endif

@@ -41,7 +41,9 @@ EXPORTS = [
     "mpe_create", "mpe_destroy", "mpe_set_stream", "mpe_set_path", "mpe_allocate_bits",
     "mpe_allocate_bits_proportional", "mpe_allocate_bits_table", "mpe_set_allocator",
     "mpe_measure_loss", "mpe_repage_async", "mpe_repage_commit", "mpe_set_compensation",
-    "mpe_select_salient", "mpe_get_kept_channels",
+    "mpe_select_salient", "mpe_get_kept_channels", "mpe_prefix_create", "mpe_prefix_destroy",
+    "mpe_prefix_last_error", "mpe_prefix_quantize", "mpe_prefix_repage", "mpe_prefix_moe_ffn",
+    "mpe_prefix_read_layer", "mpe_prefix_get_absmax",
     "mpe_quantize_experts", "mpe_repage", "mpe_moe_ffn", "mpe_moe_ffn_host", "mpe_route",
     "mpe_get_page_table", "mpe_expert_stream_bytes", "mpe_read_expert_packed",
     "mpe_get_scales", "mpe_get_bits", "mpe_get_status", "mpe_last_error",
@@ -100,6 +102,14 @@ def lib() -> ctypes.CDLL:
         "mpe_set_compensation": (i32, [vp, i32, i32]),
         "mpe_select_salient": (i32, [vp, i32, i32, i32, vp, vp]),
         "mpe_get_kept_channels": (i32, [vp, i32, vp, sz]),
+        "mpe_prefix_create": (i32, [ctypes.POINTER(vp), ctypes.POINTER(Config)]),
+        "mpe_prefix_destroy": (None, [vp]),
+        "mpe_prefix_last_error": (ctypes.c_char_p, [vp]),
+        "mpe_prefix_quantize": (i32, [vp, vp, vp]),
+        "mpe_prefix_repage": (i32, [vp, vp, ctypes.POINTER(u64)]),
+        "mpe_prefix_moe_ffn": (i32, [vp, vp, i32, vp, vp, i32, vp]),
+        "mpe_prefix_read_layer": (i32, [vp, i32, i32, vp, sz]),
+        "mpe_prefix_get_absmax": (i32, [vp, vp]),
         "mpe_set_allocator": (i32, [vp, i32]),
         "mpe_repage_async": (i32, [vp, u64, vp, vp]),
         "mpe_repage_commit": (i32, [vp, i32, vp]),
@@ -370,3 +380,73 @@ class Context:
         _check(lib().mpe_profile_read(self._h, _ptr(ms), _ptr(cnt), n, 1 if reset else 0),
                self._h)
         return {name: (float(ms[i]), int(cnt[i])) for i, name in enumerate(PROFILE_SLOTS)}
+
+
+class PrefixStore:
+    """The prefix-compatible variant (mpe_prefix_*): nested-grid codes stored in
+    layers A (3 bits), B (1 bit), C (4 bits); a width change drops or adds
+    layers."""
+
+    LAYER_WORDS = (3, 1, 4)
+
+    def __init__(self, E: int, H: int, F: int, page_bytes: int = 0, pool_pages: int = 0,
+                 device: int | None = None):
+        import torch
+        L = lib()
+        dev = torch.cuda.current_device() if device is None else device
+        cfg = Config(E, H, F, page_bytes, pool_pages, dev, 0, 0,
+                     torch.cuda.current_stream().cuda_stream)
+        h = ctypes.c_void_p()
+        _check(L.mpe_prefix_create(ctypes.byref(h), ctypes.byref(cfg)))
+        self._h = h
+        self.E, self.H, self.F = E, H, F
+        self._masters = None
+
+    def _check(self, rc):
+        if rc != 0:
+            msg = lib().mpe_prefix_last_error(self._h)
+            raise MpeError(rc, msg.decode() if msg else "")
+
+    def close(self):
+        if getattr(self, "_h", None):
+            lib().mpe_prefix_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def quantize(self, masters, bits):
+        arr = (ctypes.c_void_p * self.E)(*[m.data_ptr() for m in masters])
+        b = np.ascontiguousarray(bits, dtype=np.uint8)
+        self._masters = list(masters)
+        self._check(lib().mpe_prefix_quantize(self._h, arr, _ptr(b)))
+
+    def repage(self, bits) -> int:
+        """New widths; returns the bytes the change moved."""
+        b = np.ascontiguousarray(bits, dtype=np.uint8)
+        moved = ctypes.c_uint64(0)
+        self._check(lib().mpe_prefix_repage(self._h, _ptr(b), ctypes.byref(moved)))
+        return int(moved.value)
+
+    def moe_ffn(self, x, ids, w, out=None):
+        import torch
+        T, k = ids.shape
+        if out is None:
+            out = torch.empty((T, self.H), dtype=torch.bfloat16, device=x.device)
+        self._check(lib().mpe_prefix_moe_ffn(self._h, _ptr(x), T, _ptr(ids), _ptr(w), k,
+                                             _ptr(out)))
+        return out
+
+    def read_layer(self, e: int, layer: int) -> np.ndarray:
+        n = 3 * self.H * self.F // 32 * self.LAYER_WORDS[layer]
+        out = np.zeros(n, dtype=np.uint32)
+        self._check(lib().mpe_prefix_read_layer(self._h, e, layer, _ptr(out), out.nbytes))
+        return out
+
+    def absmax(self) -> np.ndarray:
+        out = np.zeros(self.E, dtype=np.float32)
+        self._check(lib().mpe_prefix_get_absmax(self._h, _ptr(out)))
+        return out
