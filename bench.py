@@ -596,7 +596,7 @@ def run_repage_schedule(args, dist: Dist):
     q_bytes = 4 * wl.sum_W + sum(int(b) * wl.W_e // 8 for b in bits)
     reps = max(1, args.steps // 10)
     out = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
-    decode, repages = [], []
+    decode, repages, widths = [], [], []
     dec_tokens, dec_ms = 0, 0.0
     last = None
     for kind, arg in synth.schedule(wl):
@@ -624,7 +624,9 @@ def run_repage_schedule(args, dist: Dist):
             nbytes = sum(2 * wl.W_e + int(after[e]) * wl.W_e // 8 for e in changed)
             repages.append({"avg_bits": arg, "changed": int(n), "ms": ms,
                             "GB/s": nbytes / (ms / 1e3) / 1e9 if n else None,
-                            "frac": nbytes / (ms / 1e3) / 1e9 / peaks["hbm_gbs"] if n else None})
+                            "frac": nbytes / (ms / 1e3) / 1e9 / peaks["hbm_gbs"] if n else None,
+                            "bytes": nbytes})
+            widths.append(after)
     launches = ctx.kernel_launches() - launches0
     clk = clocks.stop()
     if ctx.status() != 0:
@@ -679,6 +681,36 @@ def run_repage_schedule(args, dist: Dist):
     except mpe.MpeError as err:
         overlap = {"unavailable": str(err)}
 
+    # the prefix-compatible variant on the same width sequence: a layered store
+    # quantized at the initial widths, then the schedule's widths; a change
+    # that only lowers widths drops layers and moves nothing
+    prefix = None
+    try:
+        store = mpe.PrefixStore(E, H, F)
+        _, pq_ms = timed(lambda: store.quantize(masters, bits))
+        steps = []
+        for wbits, r in zip(widths, repages):
+            moved_b, pr_ms = timed(lambda: store.repage(wbits))
+            steps.append({"avg_bits": r["avg_bits"], "ms": pr_ms, "bytes": moved_b,
+                          "packed_ms": r["ms"], "packed_bytes": r["bytes"]})
+        x_l2, ids_l2, w_l2 = last
+        idt2, wt2 = torch.from_numpy(ids_l2).cuda(), torch.from_numpy(w_l2).cuda()
+        for _ in range(3):
+            store.moe_ffn(x_l2, idt2, wt2, out)
+        _, pd_ms = timed(lambda: [store.moe_ffn(x_l2, idt2, wt2, out) for _ in range(5)])
+        prefix = {"quantize_ms": pq_ms, "repage": steps,
+                  "repage_total_ms": sum(st["ms"] for st in steps),
+                  "repage_total_bytes": sum(st["bytes"] for st in steps),
+                  "packed_repage_total_ms": sum(st["packed_ms"] for st in steps),
+                  "packed_repage_total_bytes": sum(st["packed_bytes"] for st in steps),
+                  "decode_us_final_widths": pd_ms / 5 * 1e3,
+                  "note": "forward pass of the variant: plain CUDA-core grouped GEMV from "
+                          "the layers (not the main format's tensor-core pipeline)"}
+        store.close()
+        del store
+    except mpe.MpeError as err:
+        prefix = {"unavailable": str(err)}
+
     # end to end: the last decode batch through the host-buffer entry point
     x, ids, w = last
     xh, ih = x.cpu().pin_memory(), torch.from_numpy(ids).pin_memory()
@@ -719,6 +751,7 @@ def run_repage_schedule(args, dist: Dist):
                      "unit": "GB/s", "frac": q_gbs / peaks["hbm_gbs"], "peak_source": peak_kind,
                      "traffic": None, "algorithmic_bytes_per_launch": q_bytes},
         "quantize": {"ms": q_ms, "GB/s": q_gbs, "frac": q_gbs / peaks["hbm_gbs"], "bytes": q_bytes},
+        "prefix_variant": prefix,
         "repage_total": {"ms": rp_ms, "GB/s": rp_bytes / (rp_ms / 1e3) / 1e9 if rp_ms else None,
                          "frac": rp_bytes / (rp_ms / 1e3) / 1e9 / peaks["hbm_gbs"] if rp_ms else None},
         "repage": repages,

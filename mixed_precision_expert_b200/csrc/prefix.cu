@@ -105,10 +105,10 @@ __device__ __forceinline__ const uint32_t* group_addr(const PxPaged& P, const Px
 // u8 = clamp(floor(128 w / m) + 128, 0, 255) exactly: the rounded quotient's
 // floor is off by at most one, and the sign of the single-rounded fma
 // 128 w - k m is the sign of the exact difference.
-__device__ __forceinline__ int prefix_code(float w, float m) {
+__device__ __forceinline__ int prefix_code(float w, float m, float inv_m) {
     if (!(m > 0.0f)) return 128;
     const float w128 = 128.0f * w;  // exact
-    float k = floorf(__fdiv_rn(w128, m));
+    float k = floorf(__fmul_rn(w128, inv_m));  // within one of the exact floor
     if (__fmaf_rn(-k, m, w128) < 0.0f) k -= 1.0f;
     else if (__fmaf_rn(-(k + 1.0f), m, w128) >= 0.0f) k += 1.0f;
     return min(255, max(0, (int)k + 128));
@@ -147,19 +147,20 @@ __global__ void k_px_scales(PxExpert* ex, const uint32_t* absmax, int E, uint32_
     ex[e].m = __half2float(__ushort_as_half((unsigned short)m));
 }
 
-// One thread per 32-code group of one (expert, layer) job: the group's 32
-// master weights -> u8 -> the layer's bits -> its words in the layer's page.
+// One thread per 32-code group of one expert's job: the group's 32 master
+// weights -> u8 (once) -> the bits of every layer in the job's mask -> each
+// layer's words in its page. jobs: (expert, layer mask) pairs.
 __global__ void __launch_bounds__(256)
 k_px_encode(PxPaged P, uint8_t* pool, const void* const* masters, const int32_t* jobs,
             uint32_t n_groups) {
-    const int e = jobs[2 * blockIdx.y], L = jobs[2 * blockIdx.y + 1];
+    const int e = jobs[2 * blockIdx.y], mask = jobs[2 * blockIdx.y + 1];
     const uint32_t g = blockIdx.x * blockDim.x + threadIdx.x;
     if (g >= n_groups) return;
     const PxExpert x = P.ex[e];
     if (!(x.m >= 0.0f)) return;  // non-finite master
+    const float inv_m = x.m > 0.0f ? __frcp_rn(x.m) : 0.0f;
     const uint4* src = reinterpret_cast<const uint4*>(masters[e]) + (size_t)g * 4;
-    uint32_t words[4] = {0, 0, 0, 0};
-    const int bits = layer_bits(L);
+    uint32_t wa[3] = {0, 0, 0}, wb = 0, wc[4] = {0, 0, 0, 0};
 #pragma unroll
     for (int v = 0; v < 4; ++v) {
         const uint4 q = __ldcs(src + v);
@@ -170,20 +171,26 @@ k_px_encode(PxPaged P, uint8_t* pool, const void* const* masters, const int32_t*
 #pragma unroll
             for (int hlf = 0; hlf < 2; ++hlf) {
                 const int i = 8 * v + 2 * j + hlf;  // code index in the group
-                const int u8 = prefix_code(hlf ? f.y : f.x, x.m);
-                const uint32_t val = L == 0 ? (uint32_t)(u8 >> 5)
-                                            : (L == 1 ? (uint32_t)((u8 >> 4) & 1) : (uint32_t)(u8 & 15));
-                const int pos = bits * i, wi = pos >> 5, sh = pos & 31;
-                words[wi] |= val << sh;
-                if (sh + bits > 32) words[wi + 1] |= val >> (32 - sh);
+                const uint32_t u8 = (uint32_t)prefix_code(hlf ? f.y : f.x, x.m, inv_m);
+                const int pos = 3 * i, wi = pos >> 5, sh = pos & 31;  // layer A
+                wa[wi] |= (u8 >> 5) << sh;
+                if (sh > 29) wa[wi + 1] |= (u8 >> 5) >> (32 - sh);
+                wb |= ((u8 >> 4) & 1u) << i;                          // layer B
+                wc[i >> 3] |= (u8 & 15u) << (4 * (i & 7));            // layer C
             }
         }
     }
-    const uint32_t gpp = groups_per_page(L, P.page_bytes);
-    const uint32_t page = P.pidx[x.first[L] + g / gpp];
-    uint32_t* dst = reinterpret_cast<uint32_t*>(pool + (size_t)page * P.page_bytes +
-                                                (size_t)(g % gpp) * 4 * group_words(L));
-    for (int w = 0; w < group_words(L); ++w) dst[w] = words[w];
+#pragma unroll
+    for (int L = 0; L < kLayers; ++L) {
+        if (!((mask >> L) & 1)) continue;
+        const uint32_t gpp = groups_per_page(L, P.page_bytes);
+        const uint32_t page = P.pidx[x.first[L] + g / gpp];
+        uint32_t* dst = reinterpret_cast<uint32_t*>(pool + (size_t)page * P.page_bytes +
+                                                    (size_t)(g % gpp) * 4 * group_words(L));
+        if (L == 0) { dst[0] = wa[0]; dst[1] = wa[1]; dst[2] = wa[2]; }
+        else if (L == 1) { dst[0] = wb; }
+        else { dst[0] = wc[0]; dst[1] = wc[1]; dst[2] = wc[2]; dst[3] = wc[3]; }
+    }
 }
 
 // Layer L of expert e in stream order (introspection).
@@ -545,14 +552,14 @@ int mpe_prefix_quantize(mpe_prefix* p, const void* const* master_f16, const uint
     // placement: lowest free pages, experts ascending, layers A, B, C
     std::vector<uint8_t> free(p->pool_pages, 1);
     std::vector<std::vector<uint32_t>> pages((size_t)p->E * kLayers);
-    std::vector<int32_t> jobs;
-    for (int e = 0; e < p->E; ++e)
-        for (int L = 0; L < layer_count(bits[e]); ++L) {
+    std::vector<int32_t> jobs;  // (expert, mask of the layers to encode)
+    for (int e = 0; e < p->E; ++e) {
+        for (int L = 0; L < layer_count(bits[e]); ++L)
             if (!take_pages(free, layer_pages(L, p), pages[(size_t)e * kLayers + L]))
                 return px_fail(p, MPE_ERR_POOL, "page pool exhausted");
-            jobs.push_back(e);
-            jobs.push_back(L);
-        }
+        jobs.push_back(e);
+        jobs.push_back((1 << layer_count(bits[e])) - 1);
+    }
     p->free = std::move(free);
     p->pages = std::move(pages);
     p->bits.assign(bits, bits + p->E);
@@ -593,16 +600,18 @@ int mpe_prefix_repage(mpe_prefix* p, const uint8_t* new_bits, uint64_t* bytes_mo
     uint64_t moved = 0;
     const uint64_t W = (uint64_t)3 * p->H * p->F;
     for (int e : changed) {  // then the added layers, ascending e
-        bool any = false;
+        int mask = 0;
         for (int L = layer_count(p->bits[e]); L < layer_count(new_bits[e]); ++L) {
             if (!take_pages(free, layer_pages(L, p), pages[(size_t)e * kLayers + L]))
                 return px_fail(p, MPE_ERR_POOL, "page pool exhausted");  // nothing changed
-            jobs.push_back(e);
-            jobs.push_back(L);
             moved += W * layer_bits(L) / 8;
-            any = true;
+            mask |= 1 << L;
         }
-        if (any) moved += 2 * W;  // the master is read once
+        if (mask) {
+            jobs.push_back(e);
+            jobs.push_back(mask);
+            moved += 2 * W;  // the master is read once
+        }
     }
     // the forward passes launched so far may still read the dropped pages
     PCK(cudaStreamSynchronize(p->stream));
