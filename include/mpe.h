@@ -324,7 +324,10 @@ int mpe_moe_ffn(mpe_ctx* ctx, const void* x, int32_t T, const int32_t* ids, cons
 /*
  * mpe_moe_ffn_host -- mpe_moe_ffn with HOST buffers (preferably pinned):
  * copies x, ids and w to context-owned device staging, runs the layer and
- * copies out back, then synchronises. Same shapes as mpe_moe_ffn.
+ * copies out back, then synchronises. Same shapes as mpe_moe_ffn. It runs on
+ * a context-internal stream ordered after the work queued on the context
+ * stream; when the same (T, k) repeats with no reallocation, path or
+ * compensation change in between, its kernels replay as one CUDA graph.
  */
 int mpe_moe_ffn_host(mpe_ctx* ctx, const void* x_host, int32_t T, const int32_t* ids_host,
                      const float* w_host, int32_t k, void* out_host);

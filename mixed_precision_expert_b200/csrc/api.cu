@@ -176,6 +176,7 @@ int ensure_side(mpe_ctx* c) {
 int commit_pending(mpe_ctx* c) {
     if (!c->pending) return MPE_OK;
     CK(cudaStreamWaitEvent(c->stream, c->side_done, 0));
+    c->epoch++;  // the table pointers swap
     std::swap(c->d_pte, c->d_pte_next);
     std::swap(c->d_pidx, c->d_pidx_next);
     c->pidx_count = c->pidx_count_next;
@@ -233,6 +234,7 @@ int dev_alloc(mpe_ctx* c, T** p, size_t n) {
     *p = nullptr;
     if (n == 0) n = 1;
     CK(cudaMalloc(reinterpret_cast<void**>(p), n * sizeof(T)));
+    c->epoch++;  // a captured forward may hold the old pointer
     return MPE_OK;
 }
 
@@ -474,6 +476,12 @@ void mpe_destroy(mpe_ctx* c) {
         cudaFree(c->d_choice); cudaFree(c->d_D); cudaFree(c->d_gather);
         cudaFree(c->d_loss); cudaFree(c->d_mse_acc);
         cudaFree(c->comp_dev); cudaFree(c->sel_x); cudaFree(c->sel_h);
+        if (c->fwd_exec) cudaGraphExecDestroy(c->fwd_exec);
+        if (c->host_stream) {
+            cudaStreamSynchronize(c->host_stream);
+            cudaStreamDestroy(c->host_stream);
+        }
+        if (c->host_ready) cudaEventDestroy(c->host_ready);
         if (c->comp_host) cudaFreeHost(c->comp_host);
         cudaFreeHost(c->h_pte_pinned); cudaFreeHost(c->h_pidx_pinned);
         cudaFreeHost(c->h_list_pinned); cudaFreeHost(c->h_masters_pinned);
@@ -493,6 +501,7 @@ void mpe_destroy(mpe_ctx* c) {
 int mpe_set_stream(mpe_ctx* c, void* stream) {
     if (!c) return fail_global(MPE_ERR_INVALID, "null context");
     c->stream = reinterpret_cast<cudaStream_t>(stream);
+    c->epoch++;
     return MPE_OK;
 }
 
@@ -500,6 +509,7 @@ int mpe_set_path(mpe_ctx* c, int32_t path) {
     if (!c) return fail_global(MPE_ERR_INVALID, "null context");
     if (path < MPE_PATH_AUTO || path > MPE_PATH_PREFILL) return fail(c, MPE_ERR_INVALID, "bad path");
     c->path = path;
+    c->epoch++;
     return MPE_OK;
 }
 
@@ -639,6 +649,7 @@ int mpe_set_compensation(mpe_ctx* c, int32_t n_channels, int32_t store) {
         c->comp_store = nullptr;
         c->comp_n = 0;
     }
+    c->epoch++;
     if (n_channels == 0) return MPE_OK;
     if (!c->absmax_valid) return fail(c, MPE_ERR_ORDER, "compensation before quantize_experts");
     if (!keep) {
@@ -668,6 +679,7 @@ int mpe_set_compensation(mpe_ctx* c, int32_t n_channels, int32_t store) {
         CK(cudaStreamSynchronize(c->stream));
     }
     c->comp_n = n_channels;
+    c->epoch++;
     return MPE_OK;
 }
 
@@ -1025,6 +1037,60 @@ int mpe_moe_ffn(mpe_ctx* c, const void* x, int32_t T, const int32_t* ids, const 
     return moe_ffn_device(c, x, T, ids, w, k, out);
 }
 
+// The host-buffer forward on c->stream (the internal stream): copies in, the
+// forward's kernels, the copy out, a synchronize. The kernels run as a CUDA
+// graph once the same (T, k) comes twice with nothing reallocated or
+// switched in between (the first call sizes every buffer, the second
+// captures, later ones replay): one launch instead of one per kernel.
+static int host_forward(mpe_ctx* c, const void* x_host, int32_t T, const int32_t* ids_host,
+                        const float* w_host, int32_t k, void* out_host) {
+    Scratch& s = c->s;
+    const size_t xb = (size_t)T * c->H * 2;
+    CK(cudaMemcpyAsync(s.x_stage, x_host, xb, cudaMemcpyHostToDevice, c->stream));
+    CK(cudaMemcpyAsync(s.ids_stage, ids_host, (size_t)T * k * 4, cudaMemcpyHostToDevice, c->stream));
+    CK(cudaMemcpyAsync(s.w_stage, w_host, (size_t)T * k * 4, cudaMemcpyHostToDevice, c->stream));
+    const bool same = c->fwd_T == T && c->fwd_k == k && c->fwd_epoch == c->epoch;
+    int r = MPE_OK;
+    if (same && c->fwd_exec && !c->profiling) {
+        CK(cudaGraphLaunch(c->fwd_exec, c->stream));
+        c->launches += c->fwd_launches;
+    } else if (same && !c->profiling) {
+        cudaGraph_t g = nullptr;
+        CK(cudaStreamBeginCapture(c->stream, cudaStreamCaptureModeThreadLocal));
+        const uint64_t l0 = c->launches;
+        r = moe_ffn_device(c, s.x_stage, T, s.ids_stage, s.w_stage, k, s.out_stage);
+        const cudaError_t ce = cudaStreamEndCapture(c->stream, &g);
+        if (r == MPE_OK && ce == cudaSuccess && c->epoch == c->fwd_epoch) {
+            cudaGraphExec_t exec = nullptr;
+            const cudaError_t ie = cudaGraphInstantiate(&exec, g, 0);
+            cudaGraphDestroy(g);
+            if (ie != cudaSuccess) return fail(c, MPE_ERR_CUDA, "graph instantiate: %s", cudaGetErrorString(ie));
+            c->fwd_exec = exec;
+            c->fwd_launches = c->launches - l0;
+            CK(cudaGraphLaunch(c->fwd_exec, c->stream));
+        } else {
+            if (g) cudaGraphDestroy(g);
+            cudaGetLastError();
+            if (r) return r;
+            if (ce != cudaSuccess) return fail(c, MPE_ERR_CUDA, "graph capture: %s", cudaGetErrorString(ce));
+            // something was reallocated while capturing: run it plainly
+            if ((r = moe_ffn_device(c, s.x_stage, T, s.ids_stage, s.w_stage, k, s.out_stage))) return r;
+        }
+    } else {
+        if (c->fwd_exec) {
+            cudaGraphExecDestroy(c->fwd_exec);
+            c->fwd_exec = nullptr;
+        }
+        if ((r = moe_ffn_device(c, s.x_stage, T, s.ids_stage, s.w_stage, k, s.out_stage))) return r;
+        c->fwd_T = T;
+        c->fwd_k = k;
+        c->fwd_epoch = c->epoch;
+    }
+    CK(cudaMemcpyAsync(out_host, s.out_stage, xb, cudaMemcpyDeviceToHost, c->stream));
+    CK(cudaStreamSynchronize(c->stream));
+    return MPE_OK;
+}
+
 int mpe_moe_ffn_host(mpe_ctx* c, const void* x_host, int32_t T, const int32_t* ids_host,
                      const float* w_host, int32_t k, void* out_host) {
     if (!c) return fail_global(MPE_ERR_INVALID, "null context");
@@ -1033,18 +1099,25 @@ int mpe_moe_ffn_host(mpe_ctx* c, const void* x_host, int32_t T, const int32_t* i
     if (!x_host || !ids_host || !w_host || !out_host) return fail(c, MPE_ERR_INVALID, "null argument");
     if (!c->absmax_valid) return fail(c, MPE_ERR_ORDER, "moe_ffn before quantize_experts");
     DeviceGuard guard(c->device);
+    if (c->comp_n > 0 && c->path == MPE_PATH_PREFILL)
+        return fail(c, MPE_ERR_INVALID, "compensation runs on the streaming path only");
     int r;
     if ((r = ensure_scratch(c, (size_t)T * k))) return r;
     if ((r = ensure_stage(c, T, k))) return r;
-    Scratch& s = c->s;
-    const size_t xb = (size_t)T * c->H * 2;
-    CK(cudaMemcpyAsync(s.x_stage, x_host, xb, cudaMemcpyHostToDevice, c->stream));
-    CK(cudaMemcpyAsync(s.ids_stage, ids_host, (size_t)T * k * 4, cudaMemcpyHostToDevice, c->stream));
-    CK(cudaMemcpyAsync(s.w_stage, w_host, (size_t)T * k * 4, cudaMemcpyHostToDevice, c->stream));
-    if ((r = moe_ffn_device(c, s.x_stage, T, s.ids_stage, s.w_stage, k, s.out_stage))) return r;
-    CK(cudaMemcpyAsync(out_host, s.out_stage, xb, cudaMemcpyDeviceToHost, c->stream));
-    CK(cudaStreamSynchronize(c->stream));
-    return MPE_OK;
+    if (!c->host_stream) {
+        CK(cudaStreamCreateWithFlags(&c->host_stream, cudaStreamNonBlocking));
+        CK(cudaEventCreateWithFlags(&c->host_ready, cudaEventDisableTiming));
+    }
+    // the call is synchronous: it runs on the internal stream (which can be
+    // captured, unlike the legacy default stream) after the work queued on
+    // the context stream, and is finished when it returns
+    CK(cudaEventRecord(c->host_ready, c->stream));
+    CK(cudaStreamWaitEvent(c->host_stream, c->host_ready, 0));
+    const cudaStream_t user = c->stream;
+    c->stream = c->host_stream;
+    r = host_forward(c, x_host, T, ids_host, w_host, k, out_host);
+    c->stream = user;
+    return r;
 }
 
 int mpe_route(mpe_ctx* c, const int32_t* ids, int32_t T, int32_t k, int32_t* perm,

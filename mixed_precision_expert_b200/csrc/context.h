@@ -81,6 +81,18 @@ struct mpe_ctx {
     bool pending = false;
     std::vector<uint32_t> pending_release;  // old pages of the changed experts
 
+    // the host-buffer forward replays a CUDA graph of its kernels on an
+    // internal stream once the same (T, k) repeats; `epoch` counts changes
+    // that invalidate a captured graph (any device reallocation, a table
+    // swap, a new path or compensation setting)
+    uint64_t epoch = 0;
+    cudaStream_t host_stream = nullptr;
+    cudaEvent_t host_ready = nullptr;
+    cudaGraphExec_t fwd_exec = nullptr;
+    int fwd_T = 0, fwd_k = 0;
+    uint64_t fwd_epoch = ~0ull;
+    uint64_t fwd_launches = 0;
+
     // tracing
     bool profiling = false;
     std::vector<mpe::ProfileRecord> prof;

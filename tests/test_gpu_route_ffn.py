@@ -140,6 +140,36 @@ def test_ffn_host_buffers_match_device_call():
     assert np.array_equal(oh.double().numpy(), dev)
 
 
+def _host_call(ctx, x, ids, w):
+    xh = x.pin_memory()
+    idh = torch.from_numpy(ids).pin_memory()
+    wh = torch.from_numpy(w).pin_memory()
+    oh = torch.empty(x.shape, dtype=torch.bfloat16).pin_memory()
+    ctx.moe_ffn_host(xh, idh, wh, oh)
+    return oh.double().numpy()
+
+
+@pytest.mark.parametrize("path", [1, 2])
+def test_ffn_host_graph_replay_matches_device_call(path):
+    # the host-buffer call sizes its buffers on the first call with a shape,
+    # captures its kernels as a CUDA graph on the second and replays it on
+    # later ones: every call must equal the device-pointer call bit for bit,
+    # also across a repage (new widths, same buffers) and a compensation switch
+    wl = synth.scaled(synth.WORKLOADS[3], E=16, T=48, k=4)
+    ctx, masters, _ = _layer(wl, path=path)
+    p = synth.importance(wl)
+    for step in range(7):
+        if step == 3:
+            ctx.repage(synth.budget_for(wl, 3.2), p)
+        if step == 5 and path == 1:
+            ctx.set_compensation(8)
+        ids, w = synth.routing(wl, seed=50 + step)
+        x = synth.activations(wl, seed=50 + step)
+        got = _host_call(ctx, x, ids, w)
+        assert np.array_equal(got, _run(ctx, x, ids, w)), step
+    assert ctx.status() == 0
+
+
 def test_ffn_finegrained_decode_full_size():
     # 128 experts, hidden 2048, ffn 768, 64 tokens top-8 (Zipf-skewed), 3.5 bits average
     wl = synth.WORKLOADS[3]
