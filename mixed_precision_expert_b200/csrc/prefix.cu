@@ -298,11 +298,26 @@ k_px_gemv(PxPaged P, const int32_t* off, const int32_t* list, int k, const __nv_
         __syncthreads();  // the previous pass is done with s_act
         // staged code-position major, [i][t][g] for element k = 32 g + i of
         // token t, so the lanes (one group each) read consecutive words
-        for (int t = 0; t < nt; ++t) {
+        // a thread takes one (token, group): 64 contiguous bytes in, 32 stores
+        // whose addresses run along g across the warp (no bank conflicts)
+        for (int idx = threadIdx.x; idx < nt * ng; idx += blockDim.x) {
+            const int t = idx / ng, g = idx - t * ng;
             const int a = list[a0 + t0 + t];
-            const __nv_bfloat16* src = GATEUP ? act + (size_t)(a / k) * H : act + (size_t)a * F;
-            for (int kk = threadIdx.x; kk < K; kk += blockDim.x)
-                s_act[((size_t)(kk & 31) * kPxTok + t) * ng + (kk >> 5)] = src[kk];
+            const __nv_bfloat16* src =
+                (GATEUP ? act + (size_t)(a / k) * H : act + (size_t)a * F) + g * kGroupCodes;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const uint4 v = reinterpret_cast<const uint4*>(src)[q];
+                const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int i = 8 * q + 2 * j;  // elements i and i + 1
+                    s_act[((size_t)i * kPxTok + t) * ng + g] =
+                        __ushort_as_bfloat16((unsigned short)(wd[j] & 0xFFFFu));
+                    s_act[((size_t)(i + 1) * kPxTok + t) * ng + g] =
+                        __ushort_as_bfloat16((unsigned short)(wd[j] >> 16));
+                }
+            }
         }
         __syncthreads();
         // GATEUP: the two features r0, r0 + 1, each a W1 and a W3 row
