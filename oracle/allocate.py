@@ -5,7 +5,7 @@ sum_e p_e * L(b_e) subject to sum_e b_e * W_e <= B, where p_e is the expert's
 average routing probability and W_e its number of weight elements. The bit
 widths available are {3, 4, 8} (PagedWeight, "Code Illustration", bit_options).
 
-Readings taken where the page is open (each listed in the design doc):
+Readings taken where the page is open:
 * L(b) is the mean squared error of a uniform symmetric quantizer whose step
   is proportional to 1/q_b, q_b = 2^(b-1) - 1, so L(b) = 1 / q_b^2 (the page
   says "e.g., mean squared error"; the allocator receives no weights, so the

@@ -11,7 +11,7 @@ Figure 4: replacing the channels of W^ by their FP16 values in descending
 order of |x| lowers the error of W^ x against W x much faster than in random
 order.
 
-Readings taken (listed in the design doc):
+Readings taken where the pages leave the step open:
 * M is chosen per input row: per token for the gate and up projections
   (they share x, so they share the mask), per routed position for the down
   projection (its input is that position's h). A row keeps its n channels of

@@ -6,7 +6,7 @@ management: a page table maps expert IDs to physical page addresses, and the
 scheduler re-sizes experts' pages as KV-cache occupancy changes; "Code
 Illustration": an expert's page_size is set by the allocator.
 
-Readings taken (listed in the design doc):
+Readings taken where the pages leave the step open:
 * Physical pages have one fixed size P (default 64 KiB). A page holds whole
   chunks (16 rows x 128 codes) of one expert at one bit width:
   chunks_per_page(b) = floor(P / (256 b)) = 85 / 64 / 32 at b = 3 / 4 / 8.

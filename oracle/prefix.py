@@ -9,7 +9,7 @@ scheduler lowers or raises their precision as KV-cache occupancy changes.
 The main format's symmetric grid (s = m / (2^(b-1) - 1)) is not nested
 across widths, so this variant uses a nested grid.
 
-Readings taken (listed in the design doc):
+Readings taken where the pages leave the step open:
 * Grid: 2^b uniform bins over [-m, m] (m = max |w| of the expert), the value
   of a bin its centre. The 8-bit code is u8 = clamp(floor(128 w / m) + 128,
   0, 255), taken exactly; the b-bit code is its top b bits, u_b = u8 >> (8 - b);

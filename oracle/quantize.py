@@ -4,7 +4,7 @@ PagedWeight, "Implementation Details", quantization scheme: for bit width b,
 Q(w) = round(w / s) * s with s = max(|w|) / (2^(b-1) - 1), one scaling factor
 per expert ("per-expert scaling factors").
 
-Readings taken (listed in the design doc):
+Readings taken where the pages leave the step open:
 * max |w| runs over the whole expert (gate, up and down matrices together):
   one s per expert.
 * The page calls the scheme "uniform affine" but its formula has no zero
