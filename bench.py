@@ -60,6 +60,8 @@ def parse_args():
     ap.add_argument("--impl", choices=["mpe", "reference"], default="mpe")
     ap.add_argument("--workload", type=int, default=2, choices=[1, 2, 3, 4, 5])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--variant", choices=["packed", "prefix"], default="packed",
+                    help="prefix: the layered prefix-compatible store on a decode workload")
     args = ap.parse_args()
     if args.steps is None:
         args.steps = {4: 400, 5: 200}.get(args.workload, 2000)
@@ -767,6 +769,91 @@ def run_repage_schedule(args, dist: Dist):
     ctx.close()
 
 
+def run_prefix_variant(args, dist: Dist):
+    """The prefix-compatible layered store on a decode workload: forward
+    tokens/s at the workload's widths, plus one lowering and one raising width
+    change (time and bytes moved). Inputs as for the packed format."""
+    import torch
+
+    from mixed_precision_expert_b200.build import build
+    if dist.rank == 0:
+        build()
+    dist.barrier()
+    import mixed_precision_expert_b200 as mpe
+    import synth
+
+    dev = dist.local_rank
+    torch.cuda.set_device(dev)
+    wl = synth.WORKLOADS[args.workload]
+    if args.workload in (4, 5):
+        raise SystemExit("the prefix variant runs on the decode workloads 1-3")
+    E, H, F, T, k = wl.E, wl.H, wl.F, wl.T, wl.k
+    masters = []
+    for e in range(E):
+        t = torch.empty(wl.W_e, dtype=torch.float16, device="cuda")
+        synth.fill_expert_weights(wl, e, t)
+        masters.append(t)
+    bits = mpe.allocate_bits(synth.importance(wl), [wl.W_e] * E, wl.budget_bits)
+    store = mpe.PrefixStore(E, H, F)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def timed(fn):
+        torch.cuda.synchronize()
+        ev0.record()
+        r = fn()
+        ev1.record()
+        torch.cuda.synchronize()
+        return r, ev0.elapsed_time(ev1)
+
+    _, q_ms = timed(lambda: store.quantize(masters, np.full(E, 8, np.uint8)))
+    low, low_ms = timed(lambda: store.repage(np.full(E, 3, np.uint8)))
+    up, up_ms = timed(lambda: store.repage(bits))
+    nb = min(16, args.steps + args.warmup)
+    batches = []
+    for i in range(nb):
+        seed = 7_000_000 + 1000 * dist.rank + i
+        ids, w = synth.routing(wl, seed=seed)
+        x = synth.activations(wl, seed=seed, device="cuda")
+        batches.append((x, torch.from_numpy(ids).cuda(), torch.from_numpy(w).cuda()))
+    out = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
+    for i in range(args.warmup):
+        x, idt, wt = batches[i % nb]
+        store.moe_ffn(x, idt, wt, out)
+    dist.barrier()
+    clocks = ClockSampler(dev)
+    clocks.start()
+    time.sleep(0.2)
+    torch.cuda.synchronize()
+    ev0.record()
+    for i in range(args.steps):
+        x, idt, wt = batches[i % nb]
+        store.moe_ffn(x, idt, wt, out)
+    ev1.record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = dist.max(ev0.elapsed_time(ev1))
+    stored = sum(int(b) * wl.W_e // 8 for b in bits)
+    line = {
+        "metric": METRIC, "value": T * args.steps * dist.world / (ms / 1e3), "unit": "tokens/s",
+        "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {**workload_config(wl, bits), "variant": "prefix-compatible layered store",
+                   "l2": "no flush", "parallelism": "replicas"},
+        "roofline": None,
+        "stored_bytes": stored,
+        "quantize_8bit_ms": q_ms,
+        "repage_lower_to_3bit": {"ms": low_ms, "bytes_moved": low},
+        "repage_raise_to_widths": {"ms": up_ms, "bytes_moved": up,
+                                   "GB/s": up / (up_ms / 1e3) / 1e9 if up else None},
+        "clocks": clk,
+        "note": "forward pass of the variant: CUDA-core grouped GEMV from the layers",
+    }
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+    store.close()
+
+
 def main():
     args = parse_args()
     dist = Dist()
@@ -777,7 +864,9 @@ def main():
     torch.cuda.set_device(dist.local_rank)
     dist.init("nccl")
     try:
-        if args.workload == 5:
+        if args.variant == "prefix":
+            run_prefix_variant(args, dist)
+        elif args.workload == 5:
             run_repage_schedule(args, dist)
         else:
             run_mpe(args, dist)
