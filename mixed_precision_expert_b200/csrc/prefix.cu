@@ -250,29 +250,37 @@ k_px_bucket(const int32_t* ids, int Tk, int E, int32_t* off, int32_t* list, uint
 constexpr int kPxWarps = 8;   // a CTA: 8 warps x 2 rows = one 16-row tile
 constexpr int kPxTok = 8;     // tokens multiplied per pass over the tile
 
-// The 32 codes of group g of an expert as c = 2 u_b + 1 - 2^b (odd integers).
-__device__ __forceinline__ void group_codes(const PxPaged& P, const PxExpert& x, uint32_t g,
-                                            float (&c)[kGroupCodes]) {
-    const int b = x.bits;
+// The stored words of group g of an expert (layers A, B, C as its width has).
+struct GroupWords {
+    uint32_t a0, a1, a2, b, c[4];
+};
+
+__device__ __forceinline__ GroupWords group_words_of(const PxPaged& P, const PxExpert& x,
+                                                     uint32_t g) {
+    GroupWords w{};
     const uint32_t* a = group_addr(P, x, 0, g);
-    const uint32_t a0 = a[0], a1 = a[1], a2 = a[2];
-    uint32_t bb = 0, c4[4] = {0, 0, 0, 0};
-    if (b >= 4) bb = *group_addr(P, x, 1, g);
-    if (b == 8) {
+    w.a0 = a[0];
+    w.a1 = a[1];
+    w.a2 = a[2];
+    if (x.bits >= 4) w.b = *group_addr(P, x, 1, g);
+    if (x.bits == 8) {
         const uint32_t* cc = group_addr(P, x, 2, g);
-        c4[0] = cc[0]; c4[1] = cc[1]; c4[2] = cc[2]; c4[3] = cc[3];
+        w.c[0] = cc[0]; w.c[1] = cc[1]; w.c[2] = cc[2]; w.c[3] = cc[3];
     }
-    const uint64_t lo = ((uint64_t)a1 << 32) | a0;
-#pragma unroll
-    for (int i = 0; i < kGroupCodes; ++i) {
-        const int pos = 3 * i;
-        uint32_t u = pos < 64 ? (uint32_t)(lo >> pos) : (a2 >> (pos - 64));
-        if (pos < 64 && pos + 3 > 64) u |= a2 << (64 - pos);
-        u &= 7u;
-        if (b >= 4) u = (u << 1) | ((bb >> i) & 1u);
-        if (b == 8) u = (u << 4) | ((c4[i >> 3] >> (4 * (i & 7))) & 15u);
-        c[i] = (float)(2 * (int)u + 1 - (1 << b));
-    }
+    return w;
+}
+
+// Code i of the group as c = 2 u_b + 1 - 2^b (an odd integer); i is a
+// compile-time constant after unrolling.
+__device__ __forceinline__ float code_at(const GroupWords& w, int i, int b) {
+    const int pos = 3 * i;
+    uint32_t u = pos < 32 ? (w.a0 >> pos) : (pos < 64 ? (w.a1 >> (pos - 32)) : (w.a2 >> (pos - 64)));
+    if (pos < 32 && pos + 3 > 32) u |= w.a1 << (32 - pos);
+    if (pos >= 32 && pos < 64 && pos + 3 > 64) u |= w.a2 << (64 - pos);
+    u &= 7u;
+    if (b >= 4) u = (u << 1) | ((w.b >> i) & 1u);
+    if (b == 8) u = (u << 4) | ((w.c[i >> 3] >> (4 * (i & 7))) & 15u);
+    return (float)(2 * (int)u + 1 - (1 << b));
 }
 
 // GATEUP: CTA (e, tile) computes h[a][r] = silu(s g) (s v) for the tile's 16
@@ -322,44 +330,50 @@ k_px_gemv(PxPaged P, const int32_t* off, const int32_t* list, int k, const __nv_
         __syncthreads();
         // GATEUP: the two features r0, r0 + 1, each a W1 and a W3 row
         // (accumulators [feature][matrix][token]); down: two W2 rows. Lane l
-        // takes groups l, l + 32, ...: each group's 32 codes unpacked once,
-        // then multiplied with every token of the pass.
-        float acc[2][2][kPxTok];
+        // takes groups l, l + 32, ...: a group's words are read once and its
+        // codes, eight at a time, multiplied with every token of the pass.
+        constexpr int NM = GATEUP ? 2 : 1;
+        float acc[2][NM][kPxTok];
 #pragma unroll
         for (int f = 0; f < 2; ++f)
 #pragma unroll
-            for (int m = 0; m < 2; ++m)
+            for (int m = 0; m < NM; ++m)
 #pragma unroll
                 for (int t = 0; t < kPxTok; ++t) acc[f][m][t] = 0.0f;
         for (int g = lane; g < ng; g += 32) {
 #pragma unroll
             for (int f = 0; f < 2; ++f)
 #pragma unroll
-                for (int m = 0; m < (GATEUP ? 2 : 1); ++m) {
+                for (int m = 0; m < NM; ++m) {
                     // group index in the expert's stream: W1 rows, then W3 rows
                     // (H / 32 groups each), then W2 rows (F / 32 groups each)
                     const uint32_t gi =
                         GATEUP ? (uint32_t)(m * F + r0 + f) * (uint32_t)ng + g
                                : (uint32_t)(2 * F) * (uint32_t)(H / kGroupCodes) +
                                      (uint32_t)(r0 + f) * (uint32_t)ng + g;
-                    float c[kGroupCodes];
-                    group_codes(P, x, gi, c);
+                    const GroupWords gw = group_words_of(P, x, gi);
 #pragma unroll
-                    for (int t = 0; t < kPxTok; ++t) {
-                        if (t >= nt) break;
-                        const __nv_bfloat16* xg = s_act + (size_t)t * ng + g;
-                        float sum = acc[f][m][t];
+                    for (int i0 = 0; i0 < kGroupCodes; i0 += 8) {
+                        float c[8];
 #pragma unroll
-                        for (int i = 0; i < kGroupCodes; ++i)
-                            sum = fmaf(c[i], __bfloat162float(xg[(size_t)i * kPxTok * ng]), sum);
-                        acc[f][m][t] = sum;
+                        for (int i = 0; i < 8; ++i) c[i] = code_at(gw, i0 + i, x.bits);
+#pragma unroll
+                        for (int t = 0; t < kPxTok; ++t) {
+                            if (t >= nt) break;
+                            const __nv_bfloat16* xg = s_act + (size_t)t * ng + g;
+                            float sum = acc[f][m][t];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i)
+                                sum = fmaf(c[i], __bfloat162float(xg[(size_t)(i0 + i) * kPxTok * ng]), sum);
+                            acc[f][m][t] = sum;
+                        }
                     }
                 }
         }
 #pragma unroll
         for (int f = 0; f < 2; ++f)
 #pragma unroll
-            for (int m = 0; m < 2; ++m)
+            for (int m = 0; m < NM; ++m)
 #pragma unroll
                 for (int t = 0; t < kPxTok; ++t)
 #pragma unroll
@@ -370,8 +384,8 @@ k_px_gemv(PxPaged P, const int32_t* off, const int32_t* list, int k, const __nv_
                 const int a = list[a0 + t0 + t];
 #pragma unroll
                 for (int f = 0; f < 2; ++f) {
-                    if (GATEUP) {
-                        const float gv = s * acc[f][0][t], uv = s * acc[f][1][t];
+                    if constexpr (GATEUP) {
+                        const float gv = s * acc[f][0][t], uv = s * acc[f][NM - 1][t];
                         h_out[(size_t)a * F + r0 + f] =
                             __float2bfloat16_rn(gv / (1.0f + __expf(-gv)) * uv);
                     } else {
