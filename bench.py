@@ -77,6 +77,7 @@ class Dist:
         self.rank = int(os.environ.get("RANK", "0"))
         self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
         self.pg = None
+        self.device = "cuda"
 
     def init(self, backend: str):
         if self.world > 1:
@@ -85,6 +86,7 @@ class Dist:
             import torch.distributed as dist
             dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
             self.pg = dist
+            self.device = "cpu" if backend == "gloo" else "cuda"
 
     def barrier(self):
         if self.pg:
@@ -94,7 +96,7 @@ class Dist:
         if not self.pg:
             return v
         import torch
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        t = torch.tensor([v], dtype=torch.float64, device=self.device)
         self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
         return float(t.item())
 
