@@ -433,6 +433,15 @@ int mpe_profile_enable(mpe_ctx* ctx, int32_t enable);
 int mpe_profile_read(mpe_ctx* ctx, double* ms_host, int64_t* launches_host, int32_t n_slots,
                      int32_t reset);
 
+/*
+ * mpe_selftest_wait -- exercises the failure path of the bounded device
+ * waits without a fault: a kernel waits on a shared-memory barrier that
+ * nothing completes, gives up after limit_ns (1 .. 1e9) and sets
+ * MPE_STATUS_WAIT_TIMEOUT in the status word (read it with mpe_get_status);
+ * nothing is left in flight and the context stays usable. Synchronous.
+ */
+int mpe_selftest_wait(mpe_ctx* ctx, uint64_t limit_ns);
+
 /* mpe_kernel_launches -- how many kernels this context has launched so far. */
 uint64_t mpe_kernel_launches(mpe_ctx* ctx);
 

@@ -43,7 +43,7 @@ EXPORTS = [
     "mpe_measure_loss", "mpe_repage_async", "mpe_repage_commit", "mpe_set_compensation",
     "mpe_select_salient", "mpe_get_kept_channels", "mpe_prefix_create", "mpe_prefix_destroy",
     "mpe_prefix_last_error", "mpe_prefix_quantize", "mpe_prefix_repage", "mpe_prefix_moe_ffn",
-    "mpe_prefix_read_layer", "mpe_prefix_get_absmax",
+    "mpe_prefix_read_layer", "mpe_prefix_get_absmax", "mpe_selftest_wait",
     "mpe_quantize_experts", "mpe_repage", "mpe_moe_ffn", "mpe_moe_ffn_host", "mpe_route",
     "mpe_get_page_table", "mpe_expert_stream_bytes", "mpe_read_expert_packed",
     "mpe_get_scales", "mpe_get_bits", "mpe_get_status", "mpe_last_error",
@@ -110,6 +110,7 @@ def lib() -> ctypes.CDLL:
         "mpe_prefix_moe_ffn": (i32, [vp, vp, i32, vp, vp, i32, vp]),
         "mpe_prefix_read_layer": (i32, [vp, i32, i32, vp, sz]),
         "mpe_prefix_get_absmax": (i32, [vp, vp]),
+        "mpe_selftest_wait": (i32, [vp, u64]),
         "mpe_set_allocator": (i32, [vp, i32]),
         "mpe_repage_async": (i32, [vp, u64, vp, vp]),
         "mpe_repage_commit": (i32, [vp, i32, vp]),
@@ -265,6 +266,12 @@ class Context:
         out = np.zeros((rows, n), dtype=np.int32)
         _check(lib().mpe_get_kept_channels(self._h, which, _ptr(out), out.size), self._h)
         return out
+
+    def selftest_wait(self, limit_ns: int):
+        """A device wait that nothing completes gives up after limit_ns and sets
+        STATUS_WAIT_TIMEOUT (the failure path of every bounded wait)."""
+        self._sync_stream()
+        _check(lib().mpe_selftest_wait(self._h, int(limit_ns)), self._h)
 
     def measure_loss(self) -> np.ndarray:
         """float64[E, 3]: each expert's measured quantization MSE at 3, 4, 8 bits."""

@@ -20,7 +20,7 @@ BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libmpe.so")
 
 SOURCES = ["api.cu", "quantize.cu", "allocate.cu", "route.cu", "decode.cu", "combine.cu", "prefill.cu",
-           "compensate.cu", "prefix.cu"]
+           "compensate.cu", "prefix.cu", "selftest.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-std=c++17", "-O3", "-lineinfo", "-Xcompiler", "-fPIC", "-DNDEBUG"]
 

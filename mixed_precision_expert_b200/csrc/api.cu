@@ -10,6 +10,8 @@
 #include "internal.h"
 
 namespace mpe {
+// selftest.cu: a bounded wait that runs out (status MPE_STATUS_WAIT_TIMEOUT)
+void launch_wait_selftest(mpe_ctx* c, uint64_t limit_ns);
 void route_set_smem_limits();
 void decode_set_smem_limits();
 }  // namespace mpe
@@ -693,6 +695,17 @@ int mpe_get_kept_channels(mpe_ctx* c, int32_t which, int32_t* idx_host, size_t c
     DeviceGuard guard(c->device);
     CK(cudaMemcpyAsync(idx_host, which == 0 ? c->sel_x : c->sel_h, need * sizeof(int32_t),
                        cudaMemcpyDeviceToHost, c->stream));
+    CK(cudaStreamSynchronize(c->stream));
+    return MPE_OK;
+}
+
+int mpe_selftest_wait(mpe_ctx* c, uint64_t limit_ns) {
+    if (!c) return fail_global(MPE_ERR_INVALID, "null context");
+    if (limit_ns == 0 || limit_ns > 1000000000ull)
+        return fail(c, MPE_ERR_INVALID, "limit_ns must be in 1 .. 1e9");
+    DeviceGuard guard(c->device);
+    launch_wait_selftest(c, limit_ns);
+    CKLAUNCH();
     CK(cudaStreamSynchronize(c->stream));
     return MPE_OK;
 }

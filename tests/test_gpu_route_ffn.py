@@ -179,3 +179,19 @@ def test_ffn_finegrained_decode_full_size():
     got = _run(ctx, x, ids, w)
     toks = np.arange(0, wl.T, 4)
     check_ffn(got[toks], oracle_moe(x, ids, w, mats_of, wl.E, tokens=toks))
+
+
+def test_bounded_wait_gives_up_and_context_stays_usable():
+    # a device wait that nothing completes gives up after its limit and
+    # reports STATUS_WAIT_TIMEOUT; the context then serves a forward pass
+    wl = synth.scaled(synth.WORKLOADS[1], E=4, H=256, F=256, T=8, k=2)
+    ctx, _, mats_of = _layer(wl, np.array([3, 4, 8, 4], np.uint8))
+    assert ctx.status() == 0
+    ctx.selftest_wait(5_000_000)  # 5 ms
+    assert ctx.status(clear=True) & mpe.STATUS_WAIT_TIMEOUT
+    assert ctx.status() == 0
+    ids, w = synth.routing(wl)
+    x = synth.activations(wl)
+    check_ffn(_run(ctx, x, ids, w), oracle_moe(x, ids, w, mats_of, wl.E))
+    with pytest.raises(mpe.MpeError):
+        ctx.selftest_wait(0)
