@@ -409,11 +409,11 @@ int mpe_create(mpe_ctx** out, const mpe_config* cfg) {
         return r;
     };
     int r;
-    if (cudaMalloc(&c->pool, (size_t)c->pool_pages * pb) != cudaSuccess) {
+    const size_t pool_bytes = (size_t)c->pool_pages * pb;
+    if (cudaMalloc(&c->pool, pool_bytes) != cudaSuccess) {
         cudaGetLastError();
         delete c;
-        return fail_global(MPE_ERR_CUDA, "pool allocation of %zu bytes failed",
-                           (size_t)c->pool_pages * pb);
+        return fail_global(MPE_ERR_CUDA, "pool allocation of %zu bytes failed", pool_bytes);
     }
     if ((r = dev_alloc(c, &c->d_pte, c->E))) return bail(r);
     if ((r = dev_alloc(c, &c->d_pidx, c->pool_pages))) return bail(r);
