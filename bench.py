@@ -275,6 +275,26 @@ class OracleSample:
         return time.perf_counter() - t0, n_slices * slice_rows / F / self.wl.k
 
 
+def oracle_quantize_rate(wl, n_weights: int = 1 << 21) -> dict:
+    """The oracle's quantizer on a bounded sample (the first n_weights fp16
+    weights of expert 0 at its allocated width): absmax, scale, codes, offset
+    codes. Rate in the quantize pass's bytes: 4 per weight (two reads of the
+    master) + b / 8 written."""
+    import synth
+    from oracle import allocate as oa
+    from oracle import quantize as oq
+    bits = oa.allocate_bits(synth.importance(wl), [wl.W_e] * wl.E, wl.budget_bits)
+    b = int(bits[0])
+    n = min(n_weights, wl.W_e)
+    master = synth.expert_weights(wl, 0, count=n).numpy()
+    t0 = time.perf_counter()
+    m, s, k = oq.quantize_expert(master, b)
+    oq.offset_codes(k, b)
+    dt = time.perf_counter() - t0
+    nbytes = 4 * n + b * n // 8
+    return {"GB/s": nbytes / dt / 1e9, "sample": f"{n} weights of expert 0 at {b} bits"}
+
+
 # ---------------------------------------------------------------------------
 # reference arm: the float64 oracle on the host cores
 # ---------------------------------------------------------------------------
@@ -299,7 +319,8 @@ def run_reference(args, dist: Dist):
                          "kind": "oracle",
                          "sample": f"each step: one {slice_rows}-row slice of ffn for one token "
                                    f"through one expert (dequantize + SwiGLU, float64); "
-                                   f"{args.steps} steps = {frac:.4f} tokens of layer work"},
+                                   f"{args.steps} steps = {frac:.4f} tokens of layer work",
+                         "quantize": oracle_quantize_rate(wl)},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -516,7 +537,8 @@ def run_mpe(args, dist: Dist):
         dt, frac = OracleSample(wl).run(n_slices, slice_rows)
         cpu = {"value": frac / dt, "unit": "tokens/s", "cores": cores_used(), "kind": "oracle",
                "sample": f"one token through one expert (all {F} ffn rows in {n_slices} slices; "
-                         f"dequantize + SwiGLU in float64) = {frac:.3f} tokens of layer work"}
+                         f"dequantize + SwiGLU in float64) = {frac:.3f} tokens of layer work",
+               "quantize": oracle_quantize_rate(wl)}
 
     qms = float(np.median(q_ms))
     line = {

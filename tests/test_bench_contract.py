@@ -24,4 +24,5 @@ def test_reference_arm_json_line():
     assert d["config"]["workload"].startswith("tiny")
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"]
+    assert cb["quantize"]["GB/s"] > 0  # the oracle's quantizer on a bounded sample
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
