@@ -4,12 +4,17 @@ widths follow the budget as KV-cache occupancy changes): 256 experts, hidden
 seeded schedule of 10 decode batches (128 tokens, top-8) alternating with 10
 budget changes (average bits 7, 6, 5, 4, 3, 3.75, 4.5, 5.25, 6, 6).
 
-Against the oracle at every step: the bit widths (exact DP) and the whole page
-table (lowest-free-first allocator). On samples, because the float64 oracle
-takes seconds per expert at this size: the packed codes of seeded experts after
-the initial quantize and after repages (every changed expert's width is then
-pinned by the page-table check), and the FFN output of one seeded token on
-three decode steps, including the all-3-bit state."""
+Against the oracle:
+* every step: the bit widths (exact program) and the whole page table
+  (lowest-free-first allocator);
+* the packed codes, absmax and scale of EVERY expert after the initial
+  quantize and after the 8 -> 3 sweep ends (the repage to 3 bits average,
+  where most experts change), and of 16 seeded changed experts (all of them
+  when fewer changed) after every other repage;
+* the FFN output of every token on the first decode batch (8 bits) and on the
+  batch after the 3-bit repage, and of 16 seeded tokens on every other batch.
+The oracle evaluates each expert by value (tests/_helpers.py), which the CPU
+tests prove identical to its direct evaluation."""
 import numpy as np
 import pytest
 import torch
@@ -18,7 +23,8 @@ import synth
 from oracle import allocate as oa
 from oracle import pages as op
 
-from _helpers import OracleExpert, check_ffn, oracle_moe
+from _helpers import (OracleExpertByValue, check_experts_in_full, check_ffn, check_page_table,
+                      oracle_moe_parallel, workload_masters_gpu)
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
@@ -32,36 +38,12 @@ def _built():
     assert torch.cuda.is_available()
 
 
-def _master_cpu(wl, e):
-    return synth.expert_weights(wl, e).numpy()
-
-
-def _check_table(ctx, alloc, bits):
-    pte, pidx = ctx.page_table()
-    table = alloc.table()
-    assert np.array_equal(pte["bits"], np.asarray(bits, np.uint8))
-    assert np.array_equal(pte["first"], table.first)
-    assert np.array_equal(pte["n_pages"], table.n_pages)
-    assert np.array_equal(pidx, table.page_idx)
-
-
-def _check_codes(ctx, wl, e, b):
-    ref = OracleExpert(_master_cpu(wl, e), wl.H, wl.F, int(b))
-    assert np.array_equal(ctx.expert_stream(e), ref.stream()), f"expert {e} at {b} bits"
-    s, m = ctx.scales()
-    assert s[e] == ref.s and m[e] == np.float32(ref.m)
-
-
 def test_repage_schedule_full_size():
     wl = synth.WORKLOADS[5]
     E, H, F = wl.E, wl.H, wl.F
     W = [wl.W_e] * E
     p = synth.importance(wl)
-    masters = []
-    for e in range(E):
-        t = torch.empty(wl.W_e, dtype=torch.float16, device="cuda")
-        synth.fill_expert_weights(wl, e, t)
-        masters.append(t)
+    masters = workload_masters_gpu(wl)
     pool = E * op.pages_needed(8, H, F)
     ctx = mpe.Context(E, H, F, pool_pages=pool)
     alloc = op.PageAllocator(pool, E, H, F)
@@ -71,12 +53,12 @@ def test_repage_schedule_full_size():
     assert np.array_equal(mpe.allocate_bits(p, W, synth.budget_for(wl, wl.avg_bits)), bits)
     ctx.quantize_experts(masters, bits)
     alloc.place(bits)
-    _check_table(ctx, alloc, bits)
-    for e in rng.choice(E, 2, replace=False):
-        _check_codes(ctx, wl, int(e), bits[e])
+    check_page_table(ctx, alloc, bits)
+    assert check_experts_in_full(ctx, masters, bits, H, F) == E
     assert ctx.status() == 0
 
-    checked_ffn = 0
+    full_ffn_steps, sampled_ffn_steps, full_code_checks = 0, 0, 1
+    after_3bit = False
     for i, (kind, arg) in enumerate(synth.schedule(wl)):
         if kind == "decode":
             ids, w = synth.routing(wl, seed=arg)
@@ -84,18 +66,20 @@ def test_repage_schedule_full_size():
             out = ctx.moe_ffn(x.cuda(), torch.from_numpy(ids).cuda(), torch.from_numpy(w).cuda())
             torch.cuda.synchronize()
             assert not (ctx.status() & mpe.STATUS_WAIT_TIMEOUT)
-            # the first batch (8 bits), the batch after the 8 -> 3 sweep ends
-            # (all 3-bit) and the last batch
-            if i in (0, 10, 18):
-                tok = np.array([int(rng.integers(0, wl.T))])
-                cur = ctx.bits()
+            cur = ctx.bits()
 
-                def mats_of(e, cur=cur):
-                    return OracleExpert(_master_cpu(wl, e), H, F, int(cur[e])).mats()
+            def mats_of(e, cur=cur):
+                return OracleExpertByValue(masters[e].cpu().numpy(), H, F, int(cur[e])).mats()
 
-                got = out.double().cpu().numpy()[tok]
-                check_ffn(got, oracle_moe(x, ids, w, mats_of, E, tokens=tok))
-                checked_ffn += 1
+            got = out.double().cpu().numpy()
+            if i == 0 or after_3bit:
+                check_ffn(got, oracle_moe_parallel(x, ids, w, mats_of, E))
+                full_ffn_steps += 1
+                after_3bit = False
+            else:
+                tok = np.sort(rng.choice(wl.T, 16, replace=False))
+                check_ffn(got[tok], oracle_moe_parallel(x, ids, w, mats_of, E, tokens=tok))
+                sampled_ffn_steps += 1
         else:
             B = synth.budget_for(wl, arg)
             before = alloc.bits.copy()
@@ -104,11 +88,18 @@ def test_repage_schedule_full_size():
             changed = alloc.repage(nb)
             assert n == len(changed)
             assert np.array_equal(ctx.bits(), nb)
-            _check_table(ctx, alloc, nb)
-            if changed:
-                e = int(rng.choice(changed))
-                assert nb[e] != before[e]
-                _check_codes(ctx, wl, e, nb[e])
+            check_page_table(ctx, alloc, nb)
+            assert all(nb[e] != before[e] for e in changed)
+            if arg == 3.0 and not after_3bit and full_code_checks == 1:
+                # the end of the 8 -> 3 sweep: every expert, changed or not
+                assert check_experts_in_full(ctx, masters, nb, H, F) == E
+                full_code_checks += 1
+                after_3bit = True
+            elif changed:
+                pick = changed if len(changed) <= 16 else \
+                    sorted(rng.choice(changed, 16, replace=False).tolist())
+                assert check_experts_in_full(ctx, masters, nb, H, F, experts=pick) == len(pick)
             assert ctx.status() == 0
-    assert checked_ffn == 3
+    assert full_code_checks == 2
+    assert full_ffn_steps == 2 and sampled_ffn_steps == 8
     ctx.close()
