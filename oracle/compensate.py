@@ -99,10 +99,15 @@ def moe_ffn_compensated(x, ids, w, expert_weights: Callable, expert_masters: Cal
     return out
 
 
-def is_valid_choice(row, kept, n: int, tol: float) -> bool:
+def is_valid_choice(row, kept, n: int, tol: float, rel: float = 0.0) -> bool:
     """True when `kept` (n distinct indices, or every index when n >= len(row))
-    is a largest-|row| choice up to `tol`: no left-out entry exceeds a kept one
-    by more than tol. For checking a choice made on rounded values."""
+    is a largest-|row| choice up to rounding: no left-out entry a exceeds a
+    kept one c by more than tol + rel * (|a| + |c|). For checking a choice made
+    on rounded values: if each compared value may be off by a relative rel
+    (its rounding) plus tol / 2 (the error before it), two values whose
+    rounded forms are ordered one way may truly differ the other way by at
+    most that much. The extreme pair (largest left out, smallest kept) decides
+    it, since the bound grows with both values."""
     row = np.abs(np.asarray(row, dtype=np.float64))
     L = row.shape[0]
     kept = np.asarray(kept)
@@ -111,7 +116,8 @@ def is_valid_choice(row, kept, n: int, tol: float) -> bool:
     if len(kept) != n or len(set(kept.tolist())) != n:
         return False
     rest = np.setdiff1d(np.arange(L), kept)
-    return row[rest].max() <= row[kept].min() + tol
+    a, c = row[rest].max(), row[kept].min()
+    return a - c <= tol + rel * (a + c)
 
 
 def error_curve(w_hat: np.ndarray, w: np.ndarray, x: np.ndarray, order) -> np.ndarray:

@@ -114,6 +114,11 @@ def test_valid_choice_check():
     assert C.is_valid_choice(row, [1, 2], 2, 0.01)         # within the tolerance
     assert not C.is_valid_choice(row, [1, 1], 2, 1.0)      # not distinct
     assert C.is_valid_choice(row, [0, 1, 2, 3, 4], 9, 0.0)  # n >= len: everything
+    # relative part: 2.001 - 2.0 = 1e-3 against rel * (2.001 + 2.0)
+    assert C.is_valid_choice(row, [1, 2], 2, 0.0, rel=2.0 ** -8)     # 1e-3 <= 0.0156
+    assert not C.is_valid_choice(row, [1, 2], 2, 0.0, rel=1e-4)      # 1e-3 > 4e-4
+    assert C.is_valid_choice(row, [1, 2], 2, 6e-4, rel=1e-4)         # 1e-3 <= 6e-4 + 4e-4
+    assert not C.is_valid_choice(row, [1, 4], 2, 0.0, rel=2.0 ** -8)  # 2.001 vs 0.5: far apart
     rng = np.random.default_rng(9)
     for _ in range(50):
         r = rng.standard_normal(30)
