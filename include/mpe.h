@@ -61,6 +61,7 @@ extern "C" {
 #define MPE_ALLOC_STATE_CAP    65536 /* allocator DP states (budget units + 1)          */
 #define MPE_DEFAULT_PAGE_BYTES 65536
 #define MPE_MAX_COMP_CHANNELS  256   /* salient channels compensated per input row    */
+#define MPE_MAX_ASSIGNMENTS    (1 << 24) /* T*k per forward / route call               */
 
 /* ---- forward-pass path selection --------------------------------------- */
 #define MPE_PATH_AUTO    0   /* decode kernels for small token counts, prefill above */
@@ -312,9 +313,12 @@ int mpe_repage_commit(mpe_ctx* ctx, int32_t wait, int32_t* committed);
  *   k    1 .. 32
  *   out  device, bf16 [T x H]
  * Two contraction paths compute the same values: a streaming one (packed
- * pages read once per 16-token work group, warp-level MMA) and a tensor-core
- * one (tcgen05 MMA over 128-token groups, weights dequantized into shared
- * memory). MPE_PATH_AUTO takes the tensor-core path when T*k >= 32 E.
+ * pages read once per work group of up to 16 tokens, warp-level MMA) and a
+ * tensor-core one (tcgen05 MMA over work groups of up to 208 tokens, the
+ * weights dequantized to bf16 straight into tensor memory as the MMA's A
+ * operand, the tokens brought into shared memory by TMA). MPE_PATH_AUTO takes
+ * the tensor-core path when T*k >= 32 E.
+ * T*k above MPE_MAX_ASSIGNMENTS: MPE_ERR_INVALID.
  * Asynchronous on the context stream; scratch grows on demand (that call
  * synchronises).
  */
@@ -337,7 +341,8 @@ int mpe_moe_ffn_host(mpe_ctx* ctx, const void* x_host, int32_t T, const int32_t*
  * assignments a = t*k + j sorted stably by expert id, offsets[E+1] = exclusive
  * prefix sums of the per-expert counts, inv[a] = position of a in perm (-1 for
  * dropped ids). Device pointers: ids int32 [T*k], perm int32 [T*k],
- * offsets int32 [E+1], inv int32 [T*k]. Asynchronous.
+ * offsets int32 [E+1], inv int32 [T*k]. Asynchronous. T*k above
+ * MPE_MAX_ASSIGNMENTS: MPE_ERR_INVALID.
  */
 int mpe_route(mpe_ctx* ctx, const int32_t* ids, int32_t T, int32_t k, int32_t* perm,
               int32_t* offsets, int32_t* inv);
@@ -357,13 +362,19 @@ int mpe_route(mpe_ctx* ctx, const int32_t* ids, int32_t T, int32_t k, int32_t* p
  *   perm     device, int32 [T*k]; offsets device, int32 [E+1];
  *   inv      device, int32 [T*k]
  *   stream   cudaStream_t (NULL = the legacy default stream)
- * The first call on a device looks up the array's device address (once per
- * device, with that device current); make that first call before any stream
- * capture. All calls on a device share the array: calls that overlap on the
- * GPU (different streams, no ordering between them) race and must not be
- * issued. Asynchronous. With T*k = 0 only offsets is written (all zero) and
- * ids, perm, inv may be NULL. MPE_ERR_INVALID (message in
- * mpe_last_error_global) for a null pointer, a bad E/T/k or T*k above 65536.
+ * Each call looks up the array's device address on the current device
+ * (cudaGetSymbolAddress, which allocates nothing) and sets the kernels'
+ * shared-memory limit there, so a device reset between calls is harmless; the
+ * first call on a device also loads the library's kernels onto it, so make
+ * that first call before any stream capture. All calls on a device share the
+ * array: calls that overlap on the GPU (different streams, no ordering
+ * between them) race and must not be issued. Asynchronous. With T*k = 0 only
+ * offsets is written (all zero) and ids, perm, inv may be NULL.
+ * MPE_ERR_INVALID (message in mpe_last_error_global) for a null pointer, a
+ * bad E/T/k or T*k above 65536. MPE_ERR_CUDA if a CUDA error from earlier
+ * work is pending on the calling thread when the call starts (it is left
+ * pending, and the message says it came from earlier work), or if one of the
+ * call's own launches fails (the message names the kernel).
  */
 int mpe_route_noalloc(const int32_t* ids, int32_t T, int32_t k, int32_t E, int32_t* perm,
                       int32_t* offsets, int32_t* inv, void* stream);

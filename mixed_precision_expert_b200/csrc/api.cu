@@ -1040,6 +1040,9 @@ int mpe_moe_ffn(mpe_ctx* c, const void* x, int32_t T, const int32_t* ids, const 
     if (!c) return fail_global(MPE_ERR_INVALID, "null context");
     if (T < 0 || k < 1 || k > 32) return fail(c, MPE_ERR_INVALID, "bad T=%d or k=%d", T, k);
     if (T == 0) return MPE_OK;
+    if ((long long)T * k > MPE_MAX_ASSIGNMENTS)
+        return fail(c, MPE_ERR_INVALID, "T*k = %lld exceeds %d", (long long)T * k,
+                    MPE_MAX_ASSIGNMENTS);
     if (!x || !ids || !w || !out) return fail(c, MPE_ERR_INVALID, "null argument");
     if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(out)) & 15)
         return fail(c, MPE_ERR_INVALID, "x and out must be 16-byte aligned");
@@ -1109,6 +1112,9 @@ int mpe_moe_ffn_host(mpe_ctx* c, const void* x_host, int32_t T, const int32_t* i
     if (!c) return fail_global(MPE_ERR_INVALID, "null context");
     if (T < 0 || k < 1 || k > 32) return fail(c, MPE_ERR_INVALID, "bad T=%d or k=%d", T, k);
     if (T == 0) return MPE_OK;
+    if ((long long)T * k > MPE_MAX_ASSIGNMENTS)
+        return fail(c, MPE_ERR_INVALID, "T*k = %lld exceeds %d", (long long)T * k,
+                    MPE_MAX_ASSIGNMENTS);
     if (!x_host || !ids_host || !w_host || !out_host) return fail(c, MPE_ERR_INVALID, "null argument");
     if (!c->absmax_valid) return fail(c, MPE_ERR_ORDER, "moe_ffn before quantize_experts");
     DeviceGuard guard(c->device);
@@ -1137,6 +1143,9 @@ int mpe_route(mpe_ctx* c, const int32_t* ids, int32_t T, int32_t k, int32_t* per
               int32_t* offsets, int32_t* inv) {
     if (!c) return fail_global(MPE_ERR_INVALID, "null context");
     if (T < 0 || k < 1 || k > 32) return fail(c, MPE_ERR_INVALID, "bad T or k");
+    if ((long long)T * k > MPE_MAX_ASSIGNMENTS)
+        return fail(c, MPE_ERR_INVALID, "T*k = %lld exceeds %d", (long long)T * k,
+                    MPE_MAX_ASSIGNMENTS);
     if (!ids || !perm || !offsets || !inv) return fail(c, MPE_ERR_INVALID, "null argument");
     DeviceGuard guard(c->device);
     const size_t Tk = (size_t)T * k;

@@ -14,7 +14,6 @@
 // id rank by lane; across warps, by the per-warp counts of earlier warps;
 // across 1024-assignment chunks, by the per-chunk histograms.
 #include <cstdio>
-#include <mutex>
 
 #include "internal.h"
 
@@ -22,6 +21,13 @@ namespace mpe {
 namespace {
 
 constexpr int kChunk = 1024;
+
+// offsets_and_groups packs the work-group counts of the three width classes
+// into 21-bit fields of one 64-bit scan: a class holds at most
+// MPE_MAX_ASSIGNMENTS / group + E groups (group >= kDecodeGroup), which must
+// stay below 2^21. The entry points reject T*k above MPE_MAX_ASSIGNMENTS.
+static_assert((long long)MPE_MAX_ASSIGNMENTS / kDecodeGroup + MPE_MAX_EXPERTS < (1ll << 21),
+              "work-group counts overflow their 21-bit scan fields");
 
 // Exclusive block scan of one uint64 per thread over 1024 threads.
 __device__ uint64_t block_exclusive_scan(uint64_t v, uint64_t* s_warp, uint64_t* total) {
@@ -272,32 +278,24 @@ constexpr size_t kNaBytes = kNaHistBytes + kNaWgBytes + kNaSmallBytes + kNaPteBy
 // widths 0, so no decode work groups are formed).
 static __device__ __align__(256) unsigned char g_route_scratch[kNaBytes];
 
-std::mutex g_noalloc_mu;
-constexpr int kMaxDevices = 64;
-void* g_noalloc_addr[kMaxDevices] = {};
+int noalloc_cuda_error(const char* what, cudaError_t e) {
+    char buf[256];
+    snprintf(buf, sizeof(buf), "mpe_route_noalloc: %s: %s", what, cudaGetErrorString(e));
+    return report_global_error(MPE_ERR_CUDA, buf);
+}
 
-// Device address of the array on the current device (host code may only use
-// the symbol through cudaGetSymbolAddress); set up once per device.
+// Device address of the array on the current device. Host code may use the
+// symbol only through cudaGetSymbolAddress; it is looked up on every call
+// (it allocates nothing), so nothing cached can outlive a device reset. The
+// kernels' shared-memory limit is set on every call for the same reason.
 int noalloc_scratch(unsigned char** out) {
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
-        return report_global_error(MPE_ERR_CUDA, "mpe_route_noalloc: no usable device");
-    std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (!g_noalloc_addr[dev]) {
-        void* p = nullptr;
-        const cudaError_t e = cudaGetSymbolAddress(&p, g_route_scratch);
-        if (e != cudaSuccess) {
-            char buf[256];
-            snprintf(buf, sizeof(buf), "mpe_route_noalloc: cudaGetSymbolAddress failed: %s",
-                     cudaGetErrorString(e));
-            return report_global_error(MPE_ERR_CUDA, buf);
-        }
-        route_set_smem_limits();
-        if (cudaGetLastError() != cudaSuccess)
-            return report_global_error(MPE_ERR_CUDA, "mpe_route_noalloc: kernel setup failed");
-        g_noalloc_addr[dev] = p;
-    }
-    *out = static_cast<unsigned char*>(g_noalloc_addr[dev]);
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_route_scratch);
+    if (e != cudaSuccess) return noalloc_cuda_error("cudaGetSymbolAddress failed", e);
+    route_set_smem_limits();
+    if ((e = cudaGetLastError()) != cudaSuccess)
+        return noalloc_cuda_error("setting the shared-memory limit failed", e);
+    *out = static_cast<unsigned char*>(p);
     return MPE_OK;
 }
 
@@ -319,6 +317,11 @@ extern "C" int mpe_route_noalloc(const int32_t* ids, int32_t T, int32_t k, int32
                  Tk, kNoAllocMaxAssign);
         return report_global_error(MPE_ERR_INVALID, buf);
     }
+    // an error left by earlier work on this thread is reported as such (and
+    // left pending), not taken for a failure of this call's launches
+    const cudaError_t before = cudaPeekAtLastError();
+    if (before != cudaSuccess)
+        return noalloc_cuda_error("a CUDA error from earlier work is pending", before);
     unsigned char* base = nullptr;
     int rc = noalloc_scratch(&base);
     if (rc != MPE_OK) return rc;
@@ -334,23 +337,26 @@ extern "C" int mpe_route_noalloc(const int32_t* ids, int32_t T, int32_t k, int32
             return report_global_error(MPE_ERR_CUDA, "mpe_route_noalloc: memset failed");
         return MPE_OK;
     }
+    cudaError_t e;
     if (n <= kChunk) {
         const size_t sm = 2 * MPE_MAX_EXPERTS * sizeof(int32_t) + 32 * E * sizeof(uint16_t);
         k_route_small<<<1, kChunk, sm, st>>>(ids, n, E, kDecodeGroup, pte, perm, offsets, inv, wg,
                                              n_wg, status, nullptr);
+        if ((e = cudaGetLastError()) != cudaSuccess)
+            return noalloc_cuda_error("launch of k_route_small failed", e);
     } else {
         const int nch = (n + kChunk - 1) / kChunk;
         k_route_hist<<<nch, kChunk, 0, st>>>(ids, n, E, hist);
+        if ((e = cudaGetLastError()) != cudaSuccess)
+            return noalloc_cuda_error("launch of k_route_hist failed", e);
         k_route_scan<<<1, kChunk, 0, st>>>(hist, nch, E, kDecodeGroup, pte, offsets, wg, n_wg,
                                            nullptr);
+        if ((e = cudaGetLastError()) != cudaSuccess)
+            return noalloc_cuda_error("launch of k_route_scan failed", e);
         k_route_scatter<<<nch, kChunk, 32 * E * sizeof(uint16_t), st>>>(ids, n, E, hist, perm,
                                                                          inv, status);
-    }
-    const cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) {
-        char buf[200];
-        snprintf(buf, sizeof(buf), "mpe_route_noalloc: launch failed: %s", cudaGetErrorString(e));
-        return report_global_error(MPE_ERR_CUDA, buf);
+        if ((e = cudaGetLastError()) != cudaSuccess)
+            return noalloc_cuda_error("launch of k_route_scatter failed", e);
     }
     return MPE_OK;
 }

@@ -42,6 +42,21 @@ def test_route_parity(T, k, E, seed):
     assert bool(ctx.status(clear=True) & mpe.STATUS_BAD_EXPERT_ID) == bad
 
 
+def test_route_and_forward_reject_too_many_assignments():
+    # T*k above MPE_MAX_ASSIGNMENTS (2^24) is refused before any device work
+    # (the work-group counts of the bucketing live in 21-bit scan fields)
+    L = mpe.lib()
+    ctx = mpe.Context(8, 128, 128)
+    buf = torch.zeros(16, dtype=torch.int32, device="cuda")
+    rc = L.mpe_route(ctx._h, buf.data_ptr(), (1 << 20) + 1, 16, buf.data_ptr(), buf.data_ptr(),
+                     buf.data_ptr())
+    assert rc == -1 and b"exceeds" in L.mpe_last_error(ctx._h)
+    rc = L.mpe_moe_ffn(ctx._h, buf.data_ptr(), (1 << 20) + 1, buf.data_ptr(), buf.data_ptr(), 16,
+                       buf.data_ptr())
+    assert rc == -1
+    ctx.close()
+
+
 def _layer(wl, bits=None, device="cuda", path=0):
     if bits is None:
         bits = mpe.allocate_bits(synth.importance(wl), [wl.W_e] * wl.E, wl.budget_bits)
