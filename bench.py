@@ -1,19 +1,19 @@
 """Benchmark: MoE-layer tokens/s and packed-weight HBM GB/s against the roofline.
 
-Default workload: the Mixtral-shaped decode layer (8 experts, hidden 4096, SwiGLU
-ffn 14336, fp16 master ~N(0, 0.02) with 0.1% outliers at 10 sigma, 4.5 bits per
-weight on average, 16 bf16 tokens per step, top-2). One step = one pass of the
-forward path over one fresh batch (route, page-table gather + unpack/dequant
-fused into the gate/up and down contractions, SwiGLU, top-k combine) with the
-quantized pages resident; the quantize pass that produced them is timed
-separately and reported under "quantize".
+Default workload (--workload 5): dynamic repaging at full size, the largest
+single-GPU configuration -- 256 experts, hidden 7168, SwiGLU ffn 2048, 22.5 GB
+of fp16 masters ~N(0, 0.02), top-8 routing. Quantize at 8 bits average, then 10
+phases, each a run of decode steps (one forward pass of a 128-token batch:
+route, page-table gather + unpack/dequant fused into the gate/up and down
+contractions, SwiGLU, top-k combine) followed by a budget change (average bits
+7, 6, 5, 4, 3, 3.75, 4.5, 5.25, 6, 6) whose repage re-quantizes only the
+experts whose width changed. Exactly K decode steps are timed, spread over the
+phases; value = decode tokens/s; the quantize and repage rates are reported
+beside it against the HBM roofline.
 
---workload 5 runs the dynamic-repaging schedule at full size (256 experts,
-hidden 7168, ffn 2048, 22.5 GB of fp16 masters): quantize at 8 bits, then 10
-decode batches of 128 tokens alternating with 10 budget changes (average bits
-7, 6, 5, 4, 3, 3.75, 4.5, 5.25, 6, 6), each repage re-quantizing only the
-experts whose width changed; it reports decode tokens/s and quantize / repage
-GB/s.
+--workload 2 / 3: one decode layer (Mixtral-shaped 8 x 4096 x 14336 with 16
+tokens top-2; fine-grained 128 x 2048 x 768 with 64 tokens top-8); a step is
+one forward pass over a fresh batch with the pages resident.
 
 --workload 4 times the fine-grained prefill layer (128 experts, hidden 2048,
 ffn 768, 8192 tokens top-8, 3.5 bits average), which runs on the tensor-core
@@ -23,7 +23,7 @@ The value comes from a timed region without per-kernel events; the kernel
 durations behind the roofline come from a second pass over the same batches
 with CUDA events around each kernel on the context stream.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 2]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 5]
     python bench.py --impl reference ...   # the float64 CPU oracle arm
 
 With N > 1 (torchrun), every rank runs an independent replica of the layer on
@@ -58,13 +58,16 @@ def parse_args():
                     help="timed steps (default: 2000 decode, 400 prefill)")
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["mpe", "reference"], default="mpe")
-    ap.add_argument("--workload", type=int, default=2, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--workload", type=int, default=5, choices=[1, 2, 3, 4, 5])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--variant", choices=["packed", "prefix"], default="packed",
                     help="prefix: the layered prefix-compatible store on a decode workload")
     args = ap.parse_args()
     if args.steps is None:
         args.steps = {4: 400, 5: 200}.get(args.workload, 2000)
+    # at least 3 untimed warm-up steps whatever is asked (the JSON line
+    # reports the number run)
+    args.warmup = max(3, args.warmup)
     return args
 
 
@@ -203,6 +206,24 @@ def kernel_source_hash(kernel: str) -> str:
     return h.hexdigest()[:16]
 
 
+def recorded_traffic_ratio(kernel: str, workload: str) -> float | None:
+    """DRAM bytes over algorithmic bytes per launch from a committed ncu
+    summary (profiles/traffic.json), if it was taken on the kernel's current
+    sources: for a workload too large to capture whole, the capture runs a
+    smaller case of the same kernel and the ratio scales it."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    ent = rec.get(f"{kernel}:{workload}")
+    if not ent or ent.get("source_hash") != kernel_source_hash(kernel) or \
+            "traffic_over_algorithmic" not in ent:
+        return None
+    return float(ent["traffic_over_algorithmic"])
+
+
 def recorded_traffic(kernel: str, workload: str) -> float | None:
     """DRAM bytes per launch from a committed ncu summary (profiles/traffic.json),
     if it was taken on the kernel's current sources."""
@@ -218,13 +239,34 @@ def recorded_traffic(kernel: str, workload: str) -> float | None:
     return float(ent["dram_bytes_per_launch"])
 
 
-def workload_config(wl, bits=None):
+PREFILL_MIN_AVG = 32  # the library's automatic path rule: tensor cores when T*k >= 32 E
+
+
+def bench_config(wl) -> dict:
+    """The workload as both arms print it: static, so the two lines carry the
+    same dict (measured values go in keys of their own)."""
+    path = "tensor-core" if wl.T * wl.k >= PREFILL_MIN_AVG * wl.E else "streaming"
     cfg = {"workload": wl.name, "E": wl.E, "H": wl.H, "F": wl.F, "tokens_per_step": wl.T,
            "top_k": wl.k, "avg_bits_budget": wl.avg_bits, "page_bytes": 65536,
-           "parallelism": "replicas"}
-    if bits is not None:
-        cfg["bits_hist"] = {str(b): int((np.asarray(bits) == b).sum()) for b in (3, 4, 8)}
+           "parallelism": "replicas", "path": path}
+    if wl.cfg == 5:
+        cfg["schedule"] = ("quantize at 8 bits average, then 10 phases: decode steps of 128 "
+                           "tokens, then a budget change (repage) to 7, 6, 5, 4, 3, 3.75, 4.5, "
+                           "5.25, 6, 6 bits average")
+        cfg["l2"] = ("no flush: each decode step reads the active experts' pages (4-11 GB) "
+                     "and each repage the changed experts' masters, far above the 126 MB L2")
+    elif wl.cfg == 1:
+        cfg["l2"] = "no flush: a correctness-size layer (1.8 MB of pages) that fits in L2"
+    elif path == "tensor-core":
+        cfg["l2"] = ("no flush: each step reads the packed pages of every expert (264 MB) and "
+                     "the routed tokens (256 MB), above the 126 MB L2")
+    else:
+        cfg["l2"] = "no flush: the active experts' packed pages read per step exceed the 126 MB L2"
     return cfg
+
+
+def bits_hist(bits) -> dict:
+    return {str(b): int((np.asarray(bits) == b).sum()) for b in (3, 4, 8)}
 
 
 def cores_used() -> int:
@@ -314,7 +356,7 @@ def run_reference(args, dist: Dist):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(wl),
+        "config": bench_config(wl),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores_used(),
                          "kind": "oracle",
                          "sample": f"each step: one {slice_rows}-row slice of ffn for one token "
@@ -546,10 +588,10 @@ def run_mpe(args, dist: Dist):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {**workload_config(wl, bits),
-                   "l2": f"no flush: packed weights of the active experts "
-                         f"({alg_layer / 1e6:.0f} MB per step) exceed the 126 MB L2",
-                   "path": "tensor-core" if prof["tc_gate_up"][1] else "streaming"},
+        "config": bench_config(wl),
+        "bits_hist": bits_hist(bits),
+        "path_taken": "tensor-core" if prof["tc_gate_up"][1] else "streaming",
+        "packed_bytes_per_step": alg_layer,
         "packed_weight_gbs": layer_gbs,
         "packed_weight_frac_of_peak": layer_gbs / peaks["hbm_gbs"],
         "layer_tflops": layer_tflops,
@@ -578,7 +620,22 @@ def run_mpe(args, dist: Dist):
 # ---------------------------------------------------------------------------
 # the dynamic-repaging schedule (workload 5)
 # ---------------------------------------------------------------------------
+def phase_steps(K: int, phases: int) -> list[int]:
+    """K timed decode steps spread over the schedule's phases (earlier phases
+    take the remainder)."""
+    return [K // phases + (1 if i < K % phases else 0) for i in range(phases)]
+
+
 def run_repage_schedule(args, dist: Dist):
+    """The dynamic-repaging workload (the largest single-GPU configuration):
+    256 experts, hidden 7168, ffn 2048, 22.5 GB of fp16 masters. After the
+    initial quantize at 8 bits average, 10 phases: decode steps (one forward
+    pass of 128 tokens, top-8, each), then a budget change whose repage
+    re-quantizes only the experts whose width changed. Exactly K decode steps
+    are timed, spread over the phases, inside one region that also holds the
+    repages (each timed on its own); value = decode tokens / decode device
+    time. The roofline is the decode gate/up kernel's, over every launch of
+    the schedule (a second pass with per-kernel events)."""
     import torch
 
     from mixed_precision_expert_b200.build import build
@@ -614,63 +671,137 @@ def run_repage_schedule(args, dist: Dist):
         torch.cuda.synchronize()
         return r, ev0.elapsed_time(ev1)
 
-    bits = mpe.allocate_bits(p, W, synth.budget_for(wl, wl.avg_bits))
+    sched = synth.schedule(wl)
+    phases = [(sched[2 * i][1], sched[2 * i + 1][1]) for i in range(len(sched) // 2)]
+    # every phase's batch resident in HBM before the timed region
+    batches = []
+    for seed, _ in phases:
+        ids, w = synth.routing(wl, seed=seed + 1000 * dist.rank)
+        x = synth.activations(wl, seed=seed + 1000 * dist.rank, device="cuda")
+        batches.append((x, torch.from_numpy(ids).cuda(), torch.from_numpy(w).cuda(), ids))
+    out = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
+    steps = phase_steps(args.steps, len(phases))
+    B0 = synth.budget_for(wl, wl.avg_bits)
+    bits0 = mpe.allocate_bits(p, W, B0)
+
+    # initial quantize (timed), then W untimed warm-up steps on the first batch
+    _, q_ms = timed(lambda: ctx.quantize_experts(masters, bits0))
+    q_bytes = 4 * wl.sum_W + sum(int(b) * wl.W_e // 8 for b in bits0)
+    if ctx.status() != 0:
+        raise RuntimeError(f"device status {ctx.status():#x} after quantize")
+    for _ in range(args.warmup):
+        ctx.moe_ffn(batches[0][0], batches[0][1], batches[0][2], out)
+    torch.cuda.synchronize()
+
+    def pages_read(ids_np, cur):
+        return sum(int(cur[e]) * wl.W_e // 8 for e in np.unique(ids_np))
+
+    def gateup_bytes(ids_np, cur):
+        act = np.unique(ids_np[(ids_np >= 0) & (ids_np < E)])
+        return sum(int(cur[e]) * 2 * F * H // 8 for e in act) + T * H * 2 + T * k * F * 2
+
+    # the timed region: K decode steps over the 10 phases, the repages between
     clocks = ClockSampler(dev)
     clocks.start()
     time.sleep(0.3)
     launches0 = ctx.kernel_launches()
-    _, q_ms = timed(lambda: ctx.quantize_experts(masters, bits))
-    q_bytes = 4 * wl.sum_W + sum(int(b) * wl.W_e // 8 for b in bits)
-    reps = max(1, args.steps // 10)
-    out = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
-    decode, repages, widths = [], [], []
-    dec_tokens, dec_ms = 0, 0.0
-    last = None
-    for kind, arg in synth.schedule(wl):
-        if kind == "decode":
-            ids, w = synth.routing(wl, seed=arg + 1000 * dist.rank)
-            x = synth.activations(wl, seed=arg + 1000 * dist.rank, device="cuda")
-            idt, wt = torch.from_numpy(ids).cuda(), torch.from_numpy(w).cuda()
-            for _ in range(max(1, args.warmup)):
-                ctx.moe_ffn(x, idt, wt, out)
-            _, ms = timed(lambda: [ctx.moe_ffn(x, idt, wt, out) for _ in range(reps)])
-            ms /= reps
-            act = np.unique(ids)
-            cur = ctx.bits()
-            pbytes = sum(int(cur[e]) * wl.W_e // 8 for e in act)
-            decode.append({"avg_bits": float(cur.mean()), "us": ms * 1e3,
-                           "tokens_per_s": T / (ms / 1e3), "packed_GB/s": pbytes / (ms / 1e3) / 1e9})
-            dec_tokens += T
-            dec_ms += ms
-            last = (x, ids, w)
-        else:
-            before = ctx.bits()
-            n, ms = timed(lambda: ctx.repage(synth.budget_for(wl, arg), p))
-            after = ctx.bits()
-            changed = np.nonzero(after != before)[0]
-            nbytes = sum(2 * wl.W_e + int(after[e]) * wl.W_e // 8 for e in changed)
-            repages.append({"avg_bits": arg, "changed": int(n), "ms": ms,
-                            "GB/s": nbytes / (ms / 1e3) / 1e9 if n else None,
-                            "frac": nbytes / (ms / 1e3) / 1e9 / peaks["hbm_gbs"] if n else None,
-                            "bytes": nbytes})
-            widths.append(after)
+    ev_d = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in phases]
+    ev_r = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in phases]
+    n_changed, widths = [], []
+    dist.barrier()
+    torch.cuda.synchronize()
+    ev0.record()
+    for i, (_, avg) in enumerate(phases):
+        x, idt, wt, _ = batches[i]
+        ev_d[i][0].record()
+        for _ in range(steps[i]):
+            ctx.moe_ffn(x, idt, wt, out)
+        ev_d[i][1].record()
+        widths.append(ctx.bits())
+        ev_r[i][0].record()
+        n_changed.append(ctx.repage(synth.budget_for(wl, avg), p))
+        ev_r[i][1].record()
+    ev1.record()
+    torch.cuda.synchronize()
+    dist.barrier()
     launches = ctx.kernel_launches() - launches0
     clk = clocks.stop()
+    final_bits = ctx.bits()
     if ctx.status() != 0:
         raise RuntimeError(f"device status {ctx.status():#x} after the schedule")
-    dec_ms_max = dist.max(dec_ms)
-    value = dec_tokens * dist.world / (dec_ms_max / 1e3)
+    dec_ms_ph = [a.elapsed_time(b_) for a, b_ in ev_d]
+    rep_ms_ph = [a.elapsed_time(b_) for a, b_ in ev_r]
+    dec_ms_local = sum(dec_ms_ph)
+    dec_ms = dist.max(dec_ms_local)
+    region_ms = dist.max(ev0.elapsed_time(ev1))
+    value = T * args.steps * dist.world / (dec_ms / 1e3)
     q_gbs = q_bytes / (q_ms / 1e3) / 1e9
+
+    decode, repages = [], []
+    for i, (_, avg) in enumerate(phases):
+        cur = widths[i]
+        pb = pages_read(batches[i][3], cur)
+        ms = dec_ms_ph[i] / max(steps[i], 1)
+        decode.append({"avg_bits": float(cur.mean()), "steps": steps[i],
+                       "us_per_step": ms * 1e3 if steps[i] else None,
+                       "packed_GB/s": pb / (ms / 1e3) / 1e9 if steps[i] else None})
+        after = widths[i + 1] if i + 1 < len(widths) else final_bits
+        changed = np.nonzero(after != cur)[0]
+        nbytes = sum(2 * wl.W_e + int(after[e]) * wl.W_e // 8 for e in changed)
+        rms = rep_ms_ph[i]
+        repages.append({"avg_bits": avg, "changed": int(n_changed[i]), "ms": rms,
+                        "bytes": nbytes,
+                        "GB/s": nbytes / (rms / 1e3) / 1e9 if n_changed[i] else None,
+                        "frac": nbytes / (rms / 1e3) / 1e9 / peaks["hbm_gbs"]
+                        if n_changed[i] else None})
     moved = [r for r in repages if r["changed"]]
-    rp_bytes = sum(r["GB/s"] * r["ms"] / 1e3 * 1e9 for r in moved)
+    rp_bytes = sum(r["bytes"] for r in moved)
     rp_ms = sum(r["ms"] for r in moved)
+    dec_pages = sum(pages_read(batches[i][3], widths[i]) * steps[i] for i in range(len(phases)))
+
+    # kernel durations: the same schedule again from the initial widths, with
+    # CUDA events around each forward kernel on the context stream
+    ctx.repage(B0, p)
+    ctx.profile(True)
+    gu_ms, gu_n, gu_bytes = 0.0, 0, 0.0
+    tot = {}
+    for i, (_, avg) in enumerate(phases):
+        x, idt, wt, ids_np = batches[i]
+        cur = ctx.bits()
+        for _ in range(steps[i]):
+            ctx.moe_ffn(x, idt, wt, out)
+        prof = ctx.profile_read(reset=True)
+        gu_ms += prof["gate_up"][0]
+        gu_n += prof["gate_up"][1]
+        gu_bytes += gateup_bytes(ids_np, cur) * prof["gate_up"][1]
+        for kname, v in prof.items():
+            a = tot.setdefault(kname, [0.0, 0])
+            a[0] += v[0]
+            a[1] += v[1]
+        ctx.repage(synth.budget_for(wl, avg), p)
+    ctx.profile(False)
+    achieved = (gu_bytes / gu_n) / (gu_ms / gu_n / 1e3) / 1e9 if gu_n else None
+    traffic_ratio = recorded_traffic_ratio("k_decode_gateup", wl.name)
+    roofline = {"bound": "hbm", "kernel": "decode gate/up (k_decode<true>), every launch of "
+                "the schedule (3-, 4- and 8-bit pages)",
+                "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"] if achieved else None,
+                "peak_source": peak_kind,
+                "traffic": traffic_ratio * gu_bytes / gu_n if (traffic_ratio and gu_n) else None,
+                "algorithmic_bytes_per_launch": gu_bytes / gu_n if gu_n else None,
+                "avg_launch_us": gu_ms / gu_n * 1e3 if gu_n else None}
+    total_prof = max(sum(v[0] for v in tot.values()), 1e-9)
+    kernel_us = {kn: round(v[0] / v[1] * 1e3, 2) for kn, v in tot.items() if v[1]}
+    kernel_share = {kn: round(v[0] / total_prof, 4) for kn, v in tot.items() if v[1]}
 
     # a budget change while decode batches are served: synchronous repage then
     # the batches, against the overlapped repage (forward passes keep the old
     # pages until the commit); device time from the first call to the commit
     overlap = None
-    x_l, ids_l, w_l = last
-    idt_l, wt_l = torch.from_numpy(ids_l).cuda(), torch.from_numpy(w_l).cuda()
+    x_l, idt_l, wt_l, ids_l = batches[-1]
+    w_l = wt_l.cpu().numpy()
     n_dec = 5
     ev_first = torch.cuda.Event(enable_timing=True)
     # forwards on a high-priority stream: the library's side stream has the
@@ -714,44 +845,41 @@ def run_repage_schedule(args, dist: Dist):
     prefix = None
     try:
         store = mpe.PrefixStore(E, H, F)
-        _, pq_ms = timed(lambda: store.quantize(masters, bits))
-        steps = []
-        for wbits, r in zip(widths, repages):
+        _, pq_ms = timed(lambda: store.quantize(masters, bits0))
+        psteps = []
+        for wbits, r in zip(widths[1:] + [final_bits], repages):
             moved_b, pr_ms = timed(lambda: store.repage(wbits))
-            steps.append({"avg_bits": r["avg_bits"], "ms": pr_ms, "bytes": moved_b,
-                          "packed_ms": r["ms"], "packed_bytes": r["bytes"]})
-        x_l2, ids_l2, w_l2 = last
-        idt2, wt2 = torch.from_numpy(ids_l2).cuda(), torch.from_numpy(w_l2).cuda()
+            psteps.append({"avg_bits": r["avg_bits"], "ms": pr_ms, "bytes": moved_b,
+                           "packed_ms": r["ms"], "packed_bytes": r["bytes"]})
         for _ in range(3):
-            store.moe_ffn(x_l2, idt2, wt2, out)
-        _, pd_ms = timed(lambda: [store.moe_ffn(x_l2, idt2, wt2, out) for _ in range(5)])
-        prefix = {"quantize_ms": pq_ms, "repage": steps,
-                  "repage_total_ms": sum(st["ms"] for st in steps),
-                  "repage_total_bytes": sum(st["bytes"] for st in steps),
-                  "packed_repage_total_ms": sum(st["packed_ms"] for st in steps),
-                  "packed_repage_total_bytes": sum(st["packed_bytes"] for st in steps),
-                  "decode_us_final_widths": pd_ms / 5 * 1e3,
-                  "note": "forward pass of the variant: plain CUDA-core grouped GEMV from "
-                          "the layers (not the main format's tensor-core pipeline)"}
+            store.moe_ffn(x_l, idt_l, wt_l, out)
+        _, pd_ms = timed(lambda: [store.moe_ffn(x_l, idt_l, wt_l, out) for _ in range(5)])
+        prefix = {"quantize_ms": pq_ms, "repage": psteps,
+                  "repage_total_ms": sum(st["ms"] for st in psteps),
+                  "repage_total_bytes": sum(st["bytes"] for st in psteps),
+                  "packed_repage_total_ms": sum(st["packed_ms"] for st in psteps),
+                  "packed_repage_total_bytes": sum(st["packed_bytes"] for st in psteps),
+                  "decode_us_final_widths": pd_ms / 5 * 1e3}
         store.close()
         del store
     except mpe.MpeError as err:
         prefix = {"unavailable": str(err)}
 
-    # end to end: the last decode batch through the host-buffer entry point
-    x, ids, w = last
-    xh, ih = x.cpu().pin_memory(), torch.from_numpy(ids).pin_memory()
-    wh, oh = torch.from_numpy(w).pin_memory(), torch.empty(T, H, dtype=torch.bfloat16).pin_memory()
-    n_e2e = max(10, reps)
+    # end to end: the last phase's batch through the host-buffer entry point
+    # (pinned host x, ids, w in; out back; copies inside the timed loop)
+    xh, ih = x_l.cpu().pin_memory(), torch.from_numpy(ids_l).pin_memory()
+    wh, oh = torch.from_numpy(w_l).pin_memory(), torch.empty(T, H, dtype=torch.bfloat16).pin_memory()
+    n_e2e = max(10, min(args.steps, 200))
     for _ in range(3):
         ctx.moe_ffn_host(xh, ih, wh, oh)
+    dist.barrier()
     t0 = time.perf_counter()
     for _ in range(n_e2e):
         ctx.moe_ffn_host(xh, ih, wh, oh)
     e2e_s = dist.max(time.perf_counter() - t0)
     e2e = {"value": T * n_e2e * dist.world / e2e_s, "unit": "tokens/s",
            "h2d_bytes_per_step": T * H * 2 + 2 * T * k * 4, "d2h_bytes_per_step": T * H * 2,
-           "steps": n_e2e}
+           "steps": n_e2e, "widths": "the schedule's final widths (6 bits average)"}
 
     cpu = None
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
@@ -761,29 +889,33 @@ def run_repage_schedule(args, dist: Dist):
         cpu = {"value": frac / dt, "unit": "tokens/s", "cores": cores_used(), "kind": "oracle",
                "sample": f"one token through one expert at 8 bits (all {F} ffn rows in "
                          f"{n_slices} slices; dequantize + SwiGLU in float64) = {frac:.4f} "
-                         f"tokens of layer work"}
+                         f"tokens of layer work",
+               "quantize": oracle_quantize_rate(wl)}
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": dist.world,
-        "steps": reps * len(decode), "warmup": args.warmup,
-        "ms_per_step": dec_ms / len(decode), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {**workload_config(wl, bits),
-                   "schedule": "quantize at 8 bits; 10 x (decode 128 tokens, repage)",
-                   "decode_reps_per_batch": reps,
-                   "l2": "no flush: the active experts' pages (1.4-2.9 GB per batch) and the "
-                         "22.5 GB master exceed the 126 MB L2"},
-        "roofline": {"bound": "hbm", "kernel": "quantize pass (k_absmax + k_encode) over the "
-                     "22.5 GB master", "achieved": q_gbs, "peak": peaks["hbm_gbs"],
-                     "unit": "GB/s", "frac": q_gbs / peaks["hbm_gbs"], "peak_source": peak_kind,
-                     "traffic": None, "algorithmic_bytes_per_launch": q_bytes},
-        "quantize": {"ms": q_ms, "GB/s": q_gbs, "frac": q_gbs / peaks["hbm_gbs"], "bytes": q_bytes},
-        "prefix_variant": prefix,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dec_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": bench_config(wl),
+        "bits_hist": bits_hist(bits0),
+        "packed_weight_gbs": dec_pages / (dec_ms_local / 1e3) / 1e9,
+        "packed_weight_frac_of_peak": dec_pages / (dec_ms_local / 1e3) / 1e9 / peaks["hbm_gbs"],
+        "roofline": roofline,
+        "kernel_us": kernel_us,
+        "kernel_time_share": kernel_share,
+        "schedule": {"region_ms": region_ms, "decode_ms": dec_ms,
+                     "repage_ms": sum(rep_ms_ph),
+                     "tokens_per_s_with_repages": T * args.steps * dist.world / (region_ms / 1e3)},
+        "quantize": {"ms": q_ms, "GB/s": q_gbs, "frac": q_gbs / peaks["hbm_gbs"], "bytes": q_bytes,
+                     "passes": "absmax read + encode read/write of the 22.5 GB master"},
         "repage_total": {"ms": rp_ms, "GB/s": rp_bytes / (rp_ms / 1e3) / 1e9 if rp_ms else None,
-                         "frac": rp_bytes / (rp_ms / 1e3) / 1e9 / peaks["hbm_gbs"] if rp_ms else None},
+                         "frac": rp_bytes / (rp_ms / 1e3) / 1e9 / peaks["hbm_gbs"] if rp_ms else None,
+                         "bytes": rp_bytes},
         "repage": repages,
-        "repage_overlap": overlap,
         "decode": decode,
+        "repage_overlap": overlap,
+        "prefix_variant": prefix,
         "gpu_launches": launches,
         "clocks": clk,
         "e2e": e2e,
@@ -863,8 +995,8 @@ def run_prefix_variant(args, dist: Dist):
         "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {**workload_config(wl, bits), "variant": "prefix-compatible layered store",
-                   "l2": "no flush", "parallelism": "replicas"},
+        "config": {**bench_config(wl), "variant": "prefix-compatible layered store"},
+        "bits_hist": bits_hist(bits),
         "roofline": None,
         "stored_bytes": stored,
         "quantize_8bit_ms": q_ms,

@@ -10,7 +10,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 def test_reference_arm_json_line():
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
-                        "--workload", "1", "--steps", "2", "--warmup", "1"],
+                        "--workload", "1", "--steps", "2", "--warmup", "3"],
                        capture_output=True, text=True, timeout=300, cwd=ROOT)
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
@@ -22,6 +22,11 @@ def test_reference_arm_json_line():
         assert key in d, key
     assert d["impl"] == "reference" and d["value"] > 0 and d["steps"] == 2
     assert d["config"]["workload"].startswith("tiny")
+    # the library arm prints the same static dict (bench_config) for its config
+    sys.path.insert(0, ROOT)
+    import bench
+    import synth
+    assert d["config"] == bench.bench_config(synth.WORKLOADS[1])
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"]
     assert cb["quantize"]["GB/s"] > 0  # the oracle's quantizer on a bounded sample
