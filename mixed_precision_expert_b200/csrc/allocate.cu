@@ -25,29 +25,32 @@ namespace {
 
 __device__ __forceinline__ double dinf() { return __longlong_as_double(0x7FF0000000000000ll); }
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 1024;
 // Dynamic shared memory for the two DP rows and the choice table (see below).
 constexpr size_t kAllocSmemMax = 200 * 1024;
 
-// Choices are 2-bit codes (0: 3 bits, 1: 4 bits, 2: 8 bits), four budget
-// states per byte; a thread evaluates the four states of one byte per pass
-// (independent chains) and writes the byte. ON_CHIP: both DP rows and the
-// table live in shared memory, so every expert step is a shared-memory pass
-// plus one barrier and the serial backtrack reads shared memory; otherwise
-// they live in the global buffers D and choice. The host supplies sum W and
-// g = gcd(W) (no serial 64-bit arithmetic on the device).
+// Budget states r = 0 .. R. Thread t evaluates states t, t + 1024, ...: the 32
+// lanes of a warp hold 32 consecutive states, so each expert step is one
+// pass (one state per thread up to 1,024 states) and one barrier. A choice is
+// a 2-bit code (0: 3 bits, 1: 4 bits, 2: 8 bits); a warp's 32 codes are two
+// ballot words (low and high code bits), word w of an expert row covering
+// states 32 w .. 32 w + 31. ON_CHIP: both DP rows and the table live in
+// shared memory; otherwise in the global buffers D and choice. The host
+// supplies sum W and g = gcd(W) (no serial 64-bit arithmetic on the device).
+__host__ __device__ constexpr uint32_t choice_words(uint64_t R) { return (uint32_t)(R / 32 + 1); }
+
 template <bool ON_CHIP>
 __global__ void __launch_bounds__(kThreads)
 k_allocate(const double* p, const double* loss, const uint64_t* W, int E, uint64_t B,
-           uint64_t sum_w, uint64_t g, uint8_t* bits, int32_t* status, uint8_t* choice, double* D,
-           int state_cap) {
+           uint64_t sum_w, uint64_t g, uint8_t* bits, int32_t* status, uint32_t* choice,
+           double* D, int state_cap) {
     extern __shared__ __align__(16) uint8_t dyn[];
     __shared__ uint32_t s_up4[MPE_MAX_EXPERTS];
     __shared__ uint32_t s_up8[MPE_MAX_EXPERTS];
     __shared__ double s_p[MPE_MAX_EXPERTS];
     __shared__ double s_rv[kThreads / 32];
     __shared__ uint32_t s_ri[kThreads / 32];
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31;
     int mode;  // 0 = solve, 1 = infeasible, 2 = all 8, 3 = state cap
     uint64_t R64 = 0;
     if (B < 3 * sum_w) {
@@ -67,7 +70,7 @@ k_allocate(const double* p, const double* loss, const uint64_t* W, int E, uint64
     }
     if (mode != 0) return;
     const uint32_t R = (uint32_t)R64;
-    const uint32_t nq = (R + 4) / 4;  // choice bytes per expert
+    const uint32_t nw = choice_words(R);  // ballot-word pairs per expert row
     for (int e = tid; e < E; e += kThreads) {
         const uint64_t u4 = W[e] / g, u8 = 5 * (W[e] / g);
         s_up4[e] = (uint32_t)min(u4, (uint64_t)R + 1);
@@ -76,7 +79,7 @@ k_allocate(const double* p, const double* loss, const uint64_t* W, int E, uint64
     }
     double* Dcur = ON_CHIP ? reinterpret_cast<double*>(dyn) : D;
     double* Dnext = Dcur + (R + 1);
-    uint8_t* chb = ON_CHIP ? dyn + 16 * (size_t)(R + 1) : choice;
+    uint32_t* chw = ON_CHIP ? reinterpret_cast<uint32_t*>(dyn + 16 * (size_t)(R + 1)) : choice;
     const double L3 = __ddiv_rn(1.0, 9.0);
     const double L4 = __ddiv_rn(1.0, 49.0);
     const double L8 = __ddiv_rn(1.0, 16129.0);
@@ -88,25 +91,26 @@ k_allocate(const double* p, const double* loss, const uint64_t* W, int E, uint64
         const double c4 = __dmul_rn(pe, loss ? loss[3 * e + 1] : L4);
         const double c8 = __dmul_rn(pe, loss ? loss[3 * e + 2] : L8);
         const uint32_t u4 = s_up4[e], u8 = s_up8[e];
-        uint8_t* ch = chb + (size_t)e * nq;
-        for (uint32_t qd = tid; qd < nq; qd += kThreads) {
-            uint32_t byte = 0;
-#pragma unroll
-            for (uint32_t i = 0; i < 4; ++i) {
-                const uint32_t r = 4 * qd + i;
-                // an unreachable predecessor is +inf and its candidate stays +inf
-                const double x3 = r <= R ? __dadd_rn(Dcur[r], c3) : dinf();
-                const double x4 = (r <= R && r >= u4) ? __dadd_rn(Dcur[r - u4], c4) : dinf();
-                const double x8 = (r <= R && r >= u8) ? __dadd_rn(Dcur[r - u8], c8) : dinf();
-                double best = dinf();
-                uint32_t code = 0;
-                if (x3 < best) best = x3;
-                if (x4 < best) { best = x4; code = 1; }
-                if (x8 < best) { best = x8; code = 2; }
-                if (r <= R) Dnext[r] = best;
-                byte |= code << (2 * i);
+        uint32_t* ch = chw + (size_t)e * 2 * nw;
+        // warp-uniform trip count: every lane takes part in the ballots
+        for (uint32_t r0 = tid - lane; r0 <= R; r0 += kThreads) {
+            const uint32_t r = r0 + lane;
+            // an unreachable predecessor is +inf and its candidate stays +inf
+            const double x3 = r <= R ? __dadd_rn(Dcur[r], c3) : dinf();
+            const double x4 = (r <= R && r >= u4) ? __dadd_rn(Dcur[r - u4], c4) : dinf();
+            const double x8 = (r <= R && r >= u8) ? __dadd_rn(Dcur[r - u8], c8) : dinf();
+            double best = dinf();
+            uint32_t code = 0;
+            if (x3 < best) best = x3;
+            if (x4 < best) { best = x4; code = 1; }
+            if (x8 < best) { best = x8; code = 2; }
+            if (r <= R) Dnext[r] = best;
+            const uint32_t lo = __ballot_sync(0xffffffffu, code & 1u);
+            const uint32_t hi = __ballot_sync(0xffffffffu, code >> 1);
+            if (lane == 0) {
+                ch[2 * (r0 / 32)] = lo;
+                ch[2 * (r0 / 32) + 1] = hi;
             }
-            ch[qd] = (uint8_t)byte;
         }
         __syncthreads();
         double* t = Dcur;
@@ -124,7 +128,7 @@ k_allocate(const double* p, const double* loss, const uint64_t* W, int E, uint64
         const uint32_t oi = __shfl_xor_sync(0xffffffffu, bi, o);
         if (ov < bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
     }
-    if ((tid & 31) == 0) {
+    if (lane == 0) {
         s_rv[tid >> 5] = bv;
         s_ri[tid >> 5] = bi;
     }
@@ -136,7 +140,8 @@ k_allocate(const double* p, const double* loss, const uint64_t* W, int E, uint64
             if (s_rv[w] < bv || (s_rv[w] == bv && s_ri[w] < bi)) { bv = s_rv[w]; bi = s_ri[w]; }
         uint32_t r = bi;
         for (int e = E - 1; e >= 0; --e) {
-            const uint32_t code = (chb[(size_t)e * nq + r / 4] >> (2 * (r % 4))) & 3u;
+            const uint32_t* ch = chw + (size_t)e * 2 * nw + 2 * (r / 32);
+            const uint32_t code = ((ch[0] >> (r % 32)) & 1u) | (((ch[1] >> (r % 32)) & 1u) << 1);
             bits[e] = code == 0 ? 3 : (code == 1 ? 4 : 8);
             r -= code == 0 ? 0u : (code == 1 ? s_up4[e] : s_up8[e]);
         }
@@ -231,11 +236,14 @@ k_allocate_proportional(const double* p, const uint64_t* W, int E, uint64_t B, u
 
 }  // namespace
 
-size_t allocate_choice_bytes(int E, uint64_t R) { return (size_t)E * (size_t)((R + 4) / 4); }
+size_t allocate_choice_bytes(int E, uint64_t R) {
+    return (size_t)E * 2 * choice_words(R) * sizeof(uint32_t);
+}
 
 void launch_allocate(cudaStream_t st, const double* p, const double* loss, const uint64_t* W,
                      int E, uint64_t B, uint64_t sum_w, uint64_t g, uint8_t* bits_out,
                      int32_t* status, uint8_t* choice, double* D, int state_cap, uint64_t R) {
+    uint32_t* chw = reinterpret_cast<uint32_t*>(choice);
     // R is the host's count of budget units (same formula as the kernel's);
     // it only sizes the on-chip buffers
     const size_t smem = 16 * (size_t)(R + 1) + allocate_choice_bytes(E, R);
@@ -245,10 +253,10 @@ void launch_allocate(cudaStream_t st, const double* p, const double* loss, const
             cudaFuncSetAttribute(k_allocate<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)smem);
         k_allocate<true><<<1, kThreads, smem, st>>>(p, loss, W, E, B, sum_w, g, bits_out, status,
-                                                    choice, D, state_cap);
+                                                    chw, D, state_cap);
     } else {
         k_allocate<false><<<1, kThreads, 0, st>>>(p, loss, W, E, B, sum_w, g, bits_out, status,
-                                                  choice, D, state_cap);
+                                                  chw, D, state_cap);
     }
 }
 

@@ -320,6 +320,11 @@ int run_allocate(mpe_ctx* c, const double* p, uint64_t B, std::vector<uint8_t>& 
         if (st != c->stream) CK(cudaStreamSynchronize(c->stream));  // once per context
         c->loss_valid = true;
     }
+    if (c->memo_valid && c->memo_allocator == c->allocator && c->memo_B == B &&
+        std::memcmp(c->memo_p.data(), p, sizeof(double) * E) == 0) {
+        out = c->memo_bits;
+        return MPE_OK;
+    }
     uint64_t R = (B >= 8 * sum_w && !measured) ? 0 : (B - 3 * sum_w) / g;
     R = std::min<uint64_t>(R, 5 * (sum_w / g));
     if (exact && R + 1 > MPE_ALLOC_STATE_CAP) return fail(c, MPE_ERR_STATE_CAP, "too many states");
@@ -358,6 +363,11 @@ int run_allocate(mpe_ctx* c, const double* p, uint64_t B, std::vector<uint8_t>& 
     if (status == 3) return fail(c, MPE_ERR_STATE_CAP, "too many allocation states");
     const uint8_t* bits = reinterpret_cast<const uint8_t*>(c->h_alloc_pinned + 1);
     out.assign(bits, bits + E);
+    c->memo_p.assign(p, p + E);
+    c->memo_B = B;
+    c->memo_allocator = c->allocator;
+    c->memo_bits = out;
+    c->memo_valid = true;
     return MPE_OK;
 }
 
@@ -770,6 +780,7 @@ int mpe_quantize_experts(mpe_ctx* c, const void* const* master_f16, const uint8_
     CKLAUNCH();
     c->absmax_valid = true;
     c->loss_valid = false;
+    c->memo_valid = false;  // a measured-loss allocation depends on the master
     return MPE_OK;
 }
 
@@ -782,6 +793,10 @@ int mpe_repage(mpe_ctx* c, uint64_t B_bits, const double* p, int32_t* n_changed_
     int r;
     if ((r = commit_pending(c))) return r;
     if ((r = run_allocate(c, p, B_bits, nb, c->stream))) return r;
+    if (nb == c->bits) {  // no width changes: the pages, table and scales stand
+        if (n_changed_out) *n_changed_out = 0;
+        return MPE_OK;
+    }
     PagePlan plan;
     std::vector<int> changed;
     if (!plan_pages(c, nb, plan, changed)) return fail(c, MPE_ERR_POOL, "page pool exhausted");

@@ -78,7 +78,7 @@ __device__ __forceinline__ const uint8_t* chunk_addr(const PagedExperts& P, cons
 // ---------------------------------------------------------------------------
 // the quantizer's rounding: k = round-half-even(w / s), exactly
 // ---------------------------------------------------------------------------
-// Rare path: r = w (1/s) lies within 2^-11 of a half-integer, so the exact
+// Rare path: r = w (1/s) lies within 2^-14 of a half-integer, so the exact
 // quotient w / s decides. The sign of the single-rounded fma (k -+ 1/2) s - w is
 // exact: ties go to the even integer.
 static __device__ __noinline__ float tie_fix(float w, float s, float kf) {
@@ -92,15 +92,23 @@ static __device__ __noinline__ float tie_fix(float w, float s, float kf) {
     return kf;
 }
 
-// k as a float for |w / s| < 2^8, s > 0, inv_s = RN(1 / s): r = w inv_s is
-// within ~2^-16 of the exact quotient; adding 1.5 * 2^23 rounds it to an
-// integer (ties to even), which agrees with rounding the exact quotient unless
-// r lies within 2^-11 of a half-integer, where tie_fix decides.
+// Window of the exact repair. For |w / s| <= 127.00003 (|w| <= max|w|, s =
+// RN(max|w| / q)) and inv_s = RN(1 / s), r = RN(w inv_s) has a relative error
+// below 2^-23, so |r - w/s| < 127.00003 * 2^-23 < 2^-16. When |r - k| <= 1/2 -
+// 2^-14 for the integer k nearest r, the exact quotient is within 1/2 - 2^-14 +
+// 2^-16 < 1/2 of k, so k is its rounding; only codes closer than 2^-14 to a
+// half-integer go to tie_fix (the window keeps a factor 4 over the bound).
+constexpr float kNearTie = 0.49993896484375f;  // 1/2 - 2^-14
+
+// k as a float for |w / s| < 2^8, s > 0, inv_s = RN(1 / s): adding 1.5 * 2^23
+// rounds r = w inv_s to an integer (ties to even), which agrees with rounding
+// the exact quotient unless r lies within 2^-14 of a half-integer, where
+// tie_fix decides.
 __device__ __forceinline__ float exact_code(float w, float s, float inv_s) {
     constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
     const float r = __fmul_rn(w, inv_s);
     const float kf = __fsub_rn(__fadd_rn(r, kRound), kRound);
-    return fabsf(__fsub_rn(r, kf)) > 0.4990234375f ? tie_fix(w, s, kf) : kf;
+    return fabsf(__fsub_rn(r, kf)) > kNearTie ? tie_fix(w, s, kf) : kf;
 }
 
 // ---------------------------------------------------------------------------

@@ -173,7 +173,7 @@ k_select_channels(const __nv_bfloat16* rows, size_t ld, int n_cols, const int32_
 }
 
 // Codes k = round(w / s) of a batch of weights by the quantizer's fast rule
-// (w (1/s) rounded by the 1.5 * 2^23 add); if any lies within 2^-11 of a
+// (w (1/s) rounded by the 1.5 * 2^23 add); if any lies within 2^-14 of a
 // half-integer the batch is redone with the exact rule, so the codes are the
 // encoder's. s = 0 (an all-zero expert: inv_s = 0) gives k = 0, and a
 // non-finite master's NaN scale gives NaN, which propagates.
@@ -186,7 +186,7 @@ __device__ __forceinline__ void batch_codes(const float (&w)[NW], float s, float
     for (int i = 0; i < NW; ++i) {
         const float r = __fmul_rn(w[i], inv_s);
         kf[i] = __fsub_rn(__fadd_rn(r, kRound), kRound);
-        near |= fabsf(__fsub_rn(r, kf[i])) > 0.4990234375f;
+        near |= fabsf(__fsub_rn(r, kf[i])) > kNearTie;
     }
     if (near) {
 #pragma unroll

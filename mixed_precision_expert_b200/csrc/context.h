@@ -43,6 +43,13 @@ struct mpe_ctx {
     int last_T = 0, last_k = 0;          // shape of the last compensated forward
     unsigned long long* d_mse_acc = nullptr;  // its exact sums [E][3][2]
     bool loss_valid = false;          // d_loss holds the current master's values
+    // the last allocation's inputs and widths: the same (B, p, width rule,
+    // losses) give the same widths, so a repeat skips the allocator kernel
+    bool memo_valid = false;
+    int memo_allocator = -1;
+    uint64_t memo_B = 0;
+    std::vector<double> memo_p;
+    std::vector<uint8_t> memo_bits;
     uint8_t* d_gather = nullptr;      // expert stream gather buffer
     size_t gather_cap = 0;
 
