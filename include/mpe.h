@@ -314,10 +314,10 @@ int mpe_repage_commit(mpe_ctx* ctx, int32_t wait, int32_t* committed);
  *   out  device, bf16 [T x H]
  * Two contraction paths compute the same values: a streaming one (packed
  * pages read once per work group of up to 16 tokens, warp-level MMA) and a
- * tensor-core one (tcgen05 MMA over work groups of up to 208 tokens, the
+ * tensor-core one (tcgen05 MMA over work groups of up to 192 tokens, the
  * weights dequantized to bf16 straight into tensor memory as the MMA's A
- * operand, the tokens brought into shared memory by TMA). MPE_PATH_AUTO takes
- * the tensor-core path when T*k >= 32 E.
+ * operand, the tokens brought into shared memory by TMA and shared by two
+ * weight tiles). MPE_PATH_AUTO takes the tensor-core path when T*k >= 32 E.
  * T*k above MPE_MAX_ASSIGNMENTS: MPE_ERR_INVALID.
  * Asynchronous on the context stream; scratch grows on demand (that call
  * synchronises).

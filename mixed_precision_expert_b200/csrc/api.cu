@@ -963,7 +963,7 @@ static int moe_ffn_device(mpe_ctx* c, const void* x, int32_t T, const int32_t* i
     if ((r = ensure_scratch(c, Tk))) return r;
     const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
     if (use_prefill(c, Tk)) {
-        if ((r = grow_y(c, Tk * c->H))) return r;
+        if ((r = grow_y(c, (Tk * c->H + 1) / 2))) return r;  // bf16 y (capacity in floats)
         if ((r = grow_xp(c, Tk * c->H))) return r;
         {
             KernelSpan sp(c, 0);
@@ -983,7 +983,7 @@ static int moe_ffn_device(mpe_ctx* c, const void* x, int32_t T, const int32_t* i
         }
         {
             KernelSpan sp(c, 4);
-            launch_combine_by_position(c, w, T, k, 1, reinterpret_cast<__nv_bfloat16*>(out));
+            launch_combine_by_position(c, w, T, k, 1, reinterpret_cast<__nv_bfloat16*>(out), true);
         }
         CKLAUNCH();
         return MPE_OK;
@@ -1044,7 +1044,7 @@ static int moe_ffn_device(mpe_ctx* c, const void* x, int32_t T, const int32_t* i
     }
     {
         KernelSpan sp(c, 4);
-        launch_combine_by_position(c, w, T, k, p_dn, reinterpret_cast<__nv_bfloat16*>(out));
+        launch_combine_by_position(c, w, T, k, p_dn, reinterpret_cast<__nv_bfloat16*>(out), false);
     }
     CKLAUNCH();
     return MPE_OK;

@@ -35,7 +35,8 @@ k_swiglu_reduce(const float* gv, const int32_t* offsets, int E, int F, int parts
 }
 
 // out[t] = bf16( sum_j w[t, j] * sum_p y[p][inv[t k + j]] ): y is stored by
-// route position in P K-part slices (P = 1 on the tensor-core path); slots in
+// route position in P K-part slices (fp32), or as one bf16 slice on the
+// tensor-core path; slots in
 // order, parts summed first in part order; dropped slots (inv < 0) add
 // nothing. One thread per 4 columns of one token; a CTA covers 512 columns of
 // one token row (grid: tokens x column blocks). The token's positions and
@@ -117,6 +118,57 @@ k_combine_by_position(const float* y, const int32_t* inv, const float* w, int T,
     reinterpret_cast<uint2*>(out + (size_t)t * H)[i] = pk;
 }
 
+// The tensor-core path's combine: y holds bf16(s acc) by route position (one
+// part). One CTA per token, a thread 8 columns (one 16-byte load a slot, the
+// token's slots all in flight), the same slot-order fp32 sum.
+constexpr int kCombBf16Threads = 256;
+
+__global__ void __launch_bounds__(kCombBf16Threads)
+k_combine_bf16y(const __nv_bfloat16* y, const int32_t* inv, const float* w, int k, int H,
+                __nv_bfloat16* out) {
+    __shared__ int s_pos[32];
+    __shared__ float s_w[32];
+    griddep_wait();
+    griddep_launch_dependents();
+    const int t = blockIdx.x;
+    if (threadIdx.x < k) {
+        s_pos[threadIdx.x] = inv[t * k + threadIdx.x];
+        s_w[threadIdx.x] = w[t * k + threadIdx.x];
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < H / 8; i += kCombBf16Threads) {
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int j0 = 0; j0 < k; j0 += kCombineSlots) {
+            uint4 v[kCombineSlots];
+#pragma unroll
+            for (int r = 0; r < kCombineSlots; ++r) {
+                const int pos = j0 + r < k ? s_pos[j0 + r] : -1;
+                v[r] = pos >= 0 ? reinterpret_cast<const uint4*>(y + (size_t)pos * H)[i]
+                                : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int r = 0; r < kCombineSlots; ++r) {
+                if (j0 + r >= k || s_pos[j0 + r] < 0) continue;
+                const float wj = s_w[j0 + r];
+                const uint32_t u[4] = {v[r].x, v[r].y, v[r].z, v[r].w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    acc[2 * q] = fmaf(wj, __uint_as_float(u[q] << 16), acc[2 * q]);
+                    acc[2 * q + 1] = fmaf(wj, __uint_as_float(u[q] & 0xFFFF0000u), acc[2 * q + 1]);
+                }
+            }
+        }
+        uint4 pk;
+        uint32_t* pw = reinterpret_cast<uint32_t*>(&pk);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[2 * q], acc[2 * q + 1]);
+            pw[q] = *reinterpret_cast<uint32_t*>(&b2);
+        }
+        reinterpret_cast<uint4*>(out + (size_t)t * H)[i] = pk;
+    }
+}
+
 }  // namespace
 
 void launch_swiglu_reduce(mpe_ctx* c, size_t Tk, int parts) {
@@ -128,10 +180,13 @@ void launch_swiglu_reduce(mpe_ctx* c, size_t Tk, int parts) {
 }
 
 void launch_combine_by_position(mpe_ctx* c, const float* w, int T, int k, int parts,
-                                __nv_bfloat16* out) {
+                                __nv_bfloat16* out, bool y_bf16) {
     const int n4 = c->H / 4;
     dim3 grid((unsigned)T, (unsigned)((n4 + 127) / 128));
-    if (parts == 1)
+    if (y_bf16)
+        launch_pdl(k_combine_bf16y, dim3((unsigned)T), dim3(kCombBf16Threads), 0, c->stream,
+                   (const __nv_bfloat16*)c->s.y, (const int32_t*)c->s.inv, w, k, c->H, out);
+    else if (parts == 1)
         launch_pdl(k_combine_by_position<true>, grid, dim3(128), 0, c->stream,
                    (const float*)c->s.y, (const int32_t*)c->s.inv, w, T, k, c->H, parts,
                    (size_t)T * k * c->H, out);

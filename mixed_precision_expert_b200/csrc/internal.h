@@ -144,7 +144,7 @@ void launch_decode_gateup(mpe_ctx* c, const __nv_bfloat16* x, int k, size_t Tk, 
 void launch_decode_down(mpe_ctx* c, size_t Tk, int parts, int kb, int claim);
 
 // prefill.cu (tcgen05 grouped GEMM; work groups of up to kPrefillGroup positions)
-constexpr int kPrefillGroup = 208;
+constexpr int kPrefillGroup = 192;
 void prefill_set_smem_limits();
 // xp[pos] = x[perm[pos] / k] for the routed positions
 void launch_permute_tokens(mpe_ctx* c, const __nv_bfloat16* x, int k);
@@ -156,6 +156,6 @@ void launch_swiglu_reduce(mpe_ctx* c, size_t Tk, int parts);
 // y stored by route position in `parts` K-part slices; the top-k weights are
 // applied here
 void launch_combine_by_position(mpe_ctx* c, const float* w, int T, int k, int parts,
-                                __nv_bfloat16* out);
+                                __nv_bfloat16* out, bool y_bf16);
 
 }  // namespace mpe

@@ -186,16 +186,23 @@ k_route_scan(int32_t* hist, int n_chunks, int E, int group, const Pte* pte, int3
     const int e = threadIdx.x;
     int run = 0;
     if (e < E) {
-        for (int c = 0; c < n_chunks; ++c) {
-            const int h = hist[(size_t)c * E + e];
-            hist[(size_t)c * E + e] = run;
-            run += h;
+        // eight chunks' counts loaded before their exclusive sums are written
+        for (int c0 = 0; c0 < n_chunks; c0 += 8) {
+            int h[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) h[u] = c0 + u < n_chunks ? hist[(size_t)(c0 + u) * E + e] : 0;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                if (c0 + u < n_chunks) hist[(size_t)(c0 + u) * E + e] = run;
+                run += h[u];
+            }
         }
     }
     offsets_and_groups(E, run, group, pte, offsets, wg, n_wg, s_off);
     __syncthreads();
     if (e < E) {
         const int off = s_off[e];
+#pragma unroll 8
         for (int c = 0; c < n_chunks; ++c) hist[(size_t)c * E + e] += off;
     }
 }

@@ -3,7 +3,7 @@ dequantize-then-multiply oracle (PagedWeight, "Dynamic Paging"; tolerance
 rel-Frobenius <= 5e-3, max-abs <= 2e-2 * max|oracle|).
 
 The path is forced with MPE_PATH_PREFILL so that small layers, single tokens and
-ragged 128-token work groups all run through it; the full-size case is the
+ragged 192-token work groups all run through it; the full-size case is the
 fine-grained layer (128 experts, hidden 2048, ffn 768) with 8192 tokens top-8,
 checked on every token."""
 import numpy as np
@@ -27,9 +27,22 @@ def _built():
     assert torch.cuda.is_available()
 
 
+def test_prefill_odd_tile_count_and_group_boundaries():
+    # hidden 384: the down projection has 3 output tiles of 128, so its last
+    # tile pair has one tile; ~330 assignments per expert split into a full
+    # 192-token group and a ragged one
+    wl = synth.scaled(synth.WORKLOADS[1], E=3, H=384, F=256, T=500, k=2)
+    ctx, _, mats_of = _layer(wl, np.array([3, 8, 4], np.uint8), path=mpe.PATH_PREFILL)
+    ids, w = synth.routing(wl)
+    assert np.bincount(ids.ravel(), minlength=3).max() > 192
+    x = synth.activations(wl)
+    check_ffn(_run(ctx, x, ids, w), oracle_moe(x, ids, w, mats_of, wl.E))
+    assert ctx.status() == 0
+
+
 @pytest.mark.parametrize("bits", [(3,) * 4, (4,) * 4, (8,) * 4, (3, 4, 8, 3)])
 def test_prefill_each_width(bits):
-    # ~150 assignments per expert: one full and one ragged 128-token group each;
+    # ~150 assignments per expert: one ragged group of up to 192 tokens each;
     # 4 K-steps per tile and 2 feature tiles in both contractions
     wl = synth.scaled(synth.WORKLOADS[1], E=4, H=256, F=256, T=300, k=2)
     ctx, _, mats_of = _layer(wl, np.array(bits, np.uint8), path=mpe.PATH_PREFILL)
@@ -120,7 +133,7 @@ def test_prefill_finegrained_full_size():
     ctx.profile(False)
     assert prof["tc_gate_up"][1] == 1 and prof["tc_down"][1] == 1
     assert prof["gate_up"][1] == 0 and prof["down"][1] == 0
-    # every token: each heavy expert's 208-token work groups, ragged tails and
+    # every token: each heavy expert's 192-token work groups, ragged tails and
     # the experts with a handful of tokens
     check_ffn(got, oracle_moe_parallel(x, ids, w, mats_of, wl.E))
     assert ctx.status() == 0
