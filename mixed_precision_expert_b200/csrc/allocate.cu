@@ -39,6 +39,23 @@ constexpr size_t kAllocSmemMax = 200 * 1024;
 // supplies sum W and g = gcd(W) (no serial 64-bit arithmetic on the device).
 __host__ __device__ constexpr uint32_t choice_words(uint64_t R) { return (uint32_t)(R / 32 + 1); }
 
+// One cell of the program: the least objective over experts 0..e spending
+// exactly q units, from row Dp of experts 0..e-1; code = the width taken (0:
+// 3 bits, 1: 4, 2: 8). Widths are tried 3, 4, 8 and replace only on a strictly
+// smaller value; an unreachable predecessor is +inf and stays +inf.
+__device__ __forceinline__ double dp_cell(const double* Dp, uint32_t q, uint32_t u4, uint32_t u8,
+                                          double c3, double c4, double c8, uint32_t& code) {
+    const double x3 = __dadd_rn(Dp[q], c3);
+    const double x4 = q >= u4 ? __dadd_rn(Dp[q - u4], c4) : dinf();
+    const double x8 = q >= u8 ? __dadd_rn(Dp[q - u8], c8) : dinf();
+    double best = dinf();
+    code = 0;
+    if (x3 < best) best = x3;
+    if (x4 < best) { best = x4; code = 1; }
+    if (x8 < best) { best = x8; code = 2; }
+    return best;
+}
+
 template <bool ON_CHIP>
 __global__ void __launch_bounds__(kThreads)
 k_allocate(const double* p, const double* loss, const uint64_t* W, int E, uint64_t B,
@@ -85,32 +102,71 @@ k_allocate(const double* p, const double* loss, const uint64_t* W, int E, uint64
     const double L8 = __ddiv_rn(1.0, 16129.0);
     for (uint32_t r = tid; r <= R; r += kThreads) Dcur[r] = (r == 0) ? 0.0 : dinf();
     __syncthreads();
-    for (int e = 0; e < E; ++e) {
+    // Two experts per barrier: the thread that owns state r of expert e + 1
+    // also evaluates expert e at r, r - u4' and r - u8' (u' of expert e + 1)
+    // from the row of expert e - 1 -- the same operations in the same order as
+    // the owners of those states, so every value is the one a one-expert step
+    // would store -- and then expert e + 1 at r. An odd last expert takes a
+    // step of its own.
+    auto costs = [&](int e, double& c3, double& c4, double& c8) {
         const double pe = s_p[e];
-        const double c3 = __dmul_rn(pe, loss ? loss[3 * e] : L3);
-        const double c4 = __dmul_rn(pe, loss ? loss[3 * e + 1] : L4);
-        const double c8 = __dmul_rn(pe, loss ? loss[3 * e + 2] : L8);
-        const uint32_t u4 = s_up4[e], u8 = s_up8[e];
-        uint32_t* ch = chw + (size_t)e * 2 * nw;
+        c3 = __dmul_rn(pe, loss ? loss[3 * e] : L3);
+        c4 = __dmul_rn(pe, loss ? loss[3 * e + 1] : L4);
+        c8 = __dmul_rn(pe, loss ? loss[3 * e + 2] : L8);
+    };
+    auto store_codes = [&](int e, uint32_t r0, uint32_t code) {
+        const uint32_t lo = __ballot_sync(0xffffffffu, code & 1u);
+        const uint32_t hi = __ballot_sync(0xffffffffu, code >> 1);
+        if (lane == 0) {
+            uint32_t* ch = chw + (size_t)e * 2 * nw + 2 * (r0 / 32);
+            ch[0] = lo;
+            ch[1] = hi;
+        }
+    };
+    int e = 0;
+    for (; e + 1 < E; e += 2) {
+        double a3, a4, a8, b3, b4, b8;
+        costs(e, a3, a4, a8);
+        costs(e + 1, b3, b4, b8);
+        const uint32_t ua4 = s_up4[e], ua8 = s_up8[e];
+        const uint32_t ub4 = s_up4[e + 1], ub8 = s_up8[e + 1];
         // warp-uniform trip count: every lane takes part in the ballots
         for (uint32_t r0 = tid - lane; r0 <= R; r0 += kThreads) {
             const uint32_t r = r0 + lane;
-            // an unreachable predecessor is +inf and its candidate stays +inf
-            const double x3 = r <= R ? __dadd_rn(Dcur[r], c3) : dinf();
-            const double x4 = (r <= R && r >= u4) ? __dadd_rn(Dcur[r - u4], c4) : dinf();
-            const double x8 = (r <= R && r >= u8) ? __dadd_rn(Dcur[r - u8], c8) : dinf();
-            double best = dinf();
-            uint32_t code = 0;
-            if (x3 < best) best = x3;
-            if (x4 < best) { best = x4; code = 1; }
-            if (x8 < best) { best = x8; code = 2; }
-            if (r <= R) Dnext[r] = best;
-            const uint32_t lo = __ballot_sync(0xffffffffu, code & 1u);
-            const uint32_t hi = __ballot_sync(0xffffffffu, code >> 1);
-            if (lane == 0) {
-                ch[2 * (r0 / 32)] = lo;
-                ch[2 * (r0 / 32) + 1] = hi;
+            uint32_t ca = 0, cb = 0;
+            if (r <= R) {
+                uint32_t unused;
+                const double d0 = dp_cell(Dcur, r, ua4, ua8, a3, a4, a8, ca);
+                const double d4 = r >= ub4 ? dp_cell(Dcur, r - ub4, ua4, ua8, a3, a4, a8, unused)
+                                           : dinf();
+                const double d8 = r >= ub8 ? dp_cell(Dcur, r - ub8, ua4, ua8, a3, a4, a8, unused)
+                                           : dinf();
+                const double x3 = __dadd_rn(d0, b3);
+                const double x4 = r >= ub4 ? __dadd_rn(d4, b4) : dinf();
+                const double x8 = r >= ub8 ? __dadd_rn(d8, b8) : dinf();
+                double best = dinf();
+                if (x3 < best) best = x3;
+                if (x4 < best) { best = x4; cb = 1; }
+                if (x8 < best) { best = x8; cb = 2; }
+                Dnext[r] = best;
             }
+            store_codes(e, r0, ca);
+            store_codes(e + 1, r0, cb);
+        }
+        __syncthreads();
+        double* t = Dcur;
+        Dcur = Dnext;
+        Dnext = t;
+    }
+    if (e < E) {
+        double c3, c4, c8;
+        costs(e, c3, c4, c8);
+        const uint32_t u4 = s_up4[e], u8 = s_up8[e];
+        for (uint32_t r0 = tid - lane; r0 <= R; r0 += kThreads) {
+            const uint32_t r = r0 + lane;
+            uint32_t code = 0;
+            if (r <= R) Dnext[r] = dp_cell(Dcur, r, u4, u8, c3, c4, c8, code);
+            store_codes(e, r0, code);
         }
         __syncthreads();
         double* t = Dcur;

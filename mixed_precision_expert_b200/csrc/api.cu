@@ -89,6 +89,14 @@ struct PagePlan {
     std::vector<std::pair<int, std::vector<uint32_t>>> moved;
 };
 
+// The lowest free page at or after `from` (pool_pages if none): memchr scans
+// the byte map many pages at a time.
+uint32_t next_free(const std::vector<uint8_t>& free, uint32_t from, uint32_t pool_pages) {
+    if (from >= pool_pages) return pool_pages;
+    const void* hit = std::memchr(free.data() + from, 1, pool_pages - from);
+    return hit ? (uint32_t)(static_cast<const uint8_t*>(hit) - free.data()) : pool_pages;
+}
+
 bool plan_pages(const mpe_ctx* c, const std::vector<uint8_t>& new_bits, PagePlan& plan,
                 std::vector<int>& changed) {
     changed.clear();
@@ -104,7 +112,7 @@ bool plan_pages(const mpe_ctx* c, const std::vector<uint8_t>& new_bits, PagePlan
         std::vector<uint32_t> pg;
         pg.reserve(need);
         for (int i = 0; i < need; ++i) {
-            while (cursor < c->pool_pages && !plan.free[cursor]) ++cursor;
+            cursor = next_free(plan.free, cursor, c->pool_pages);
             if (cursor >= c->pool_pages) return false;
             plan.free[cursor] = 0;
             pg.push_back(cursor);
@@ -139,7 +147,7 @@ bool plan_pages_overlapped(const mpe_ctx* c, const std::vector<uint8_t>& new_bit
         std::vector<uint32_t> pg;
         pg.reserve(need);
         for (int i = 0; i < need; ++i) {
-            while (cursor < c->pool_pages && !plan.free[cursor]) ++cursor;
+            cursor = next_free(plan.free, cursor, c->pool_pages);
             if (cursor >= c->pool_pages) return false;
             plan.free[cursor] = 0;
             pg.push_back(cursor);
