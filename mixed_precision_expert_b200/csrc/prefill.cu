@@ -642,10 +642,16 @@ k_prefill(const __grid_constant__ CUtensorMap tmap, PArgs a) {
 #pragma unroll
                         for (int u = 0; u < kEpiBatch; ++u)
 #pragma unroll
-                            for (int i = 0; i < 16; ++i)
-                                if (c0 + 16 * u + i < T.ntok)
-                                    st[(c0 + 16 * u + i) * kOStageCols + ol] =
-                                        __float2bfloat16_rn(T.scale * __uint_as_float(y[u][i]));
+                            for (int i = 0; i < 16; i += 2) {
+                                // two tokens' values in one packed conversion
+                                const int t = c0 + 16 * u + i;
+                                const __nv_bfloat162 two = __floats2bfloat162_rn(
+                                    T.scale * __uint_as_float(y[u][i]),
+                                    T.scale * __uint_as_float(y[u][i + 1]));
+                                if (t < T.ntok) st[t * kOStageCols + ol] = __low2bfloat16(two);
+                                if (t + 1 < T.ntok)
+                                    st[(t + 1) * kOStageCols + ol] = __high2bfloat16(two);
+                            }
                     }
                 }
                 tc_fence_before();

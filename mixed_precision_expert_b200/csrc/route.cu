@@ -183,9 +183,24 @@ k_route_scan(int32_t* hist, int n_chunks, int E, int group, const Pte* pte, int3
     griddep_launch_dependents();
     if (threadIdx.x < 6 && zero6) zero6[threadIdx.x] = 0;
     __shared__ int32_t s_off[MPE_MAX_EXPERTS];
+    // small tables (chunks x experts <= kScanSmem) go through shared memory:
+    // one coalesced read, the per-expert sums on chip, one coalesced write
+    constexpr int kScanSmem = 10240;
+    __shared__ int32_t s_h[kScanSmem];
     const int e = threadIdx.x;
+    const int n_h = n_chunks * E;
+    const bool on_chip = n_h <= kScanSmem;
     int run = 0;
-    if (e < E) {
+    if (on_chip) {
+        for (int i = threadIdx.x; i < n_h; i += kChunk) s_h[i] = hist[i];
+        __syncthreads();
+        if (e < E)
+            for (int c = 0; c < n_chunks; ++c) {
+                const int h = s_h[c * E + e];
+                s_h[c * E + e] = run;
+                run += h;
+            }
+    } else if (e < E) {
         // eight chunks' counts loaded before their exclusive sums are written
         for (int c0 = 0; c0 < n_chunks; c0 += 8) {
             int h[8];
@@ -200,7 +215,9 @@ k_route_scan(int32_t* hist, int n_chunks, int E, int group, const Pte* pte, int3
     }
     offsets_and_groups(E, run, group, pte, offsets, wg, n_wg, s_off);
     __syncthreads();
-    if (e < E) {
+    if (on_chip) {
+        for (int i = threadIdx.x; i < n_h; i += kChunk) hist[i] = s_h[i] + s_off[i % E];
+    } else if (e < E) {
         const int off = s_off[e];
 #pragma unroll 8
         for (int c = 0; c < n_chunks; ++c) hist[(size_t)c * E + e] += off;
