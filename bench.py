@@ -989,6 +989,21 @@ def run_prefix_variant(args, dist: Dist):
     torch.cuda.synchronize()
     clk = clocks.stop()
     ms = dist.max(ev0.elapsed_time(ev1))
+    # the packed format on the same masters, widths and batches, for comparison
+    ctx = mpe.Context(E, H, F, path=mpe.PATH_DECODE)
+    ctx.quantize_experts(masters, bits)
+    for i in range(args.warmup):
+        x, idt, wt = batches[i % nb]
+        ctx.moe_ffn(x, idt, wt, out)
+    torch.cuda.synchronize()
+    ev0.record()
+    for i in range(args.steps):
+        x, idt, wt = batches[i % nb]
+        ctx.moe_ffn(x, idt, wt, out)
+    ev1.record()
+    torch.cuda.synchronize()
+    packed_ms = dist.max(ev0.elapsed_time(ev1))
+    ctx.close()
     stored = sum(int(b) * wl.W_e // 8 for b in bits)
     line = {
         "metric": METRIC, "value": T * args.steps * dist.world / (ms / 1e3), "unit": "tokens/s",
@@ -1004,7 +1019,11 @@ def run_prefix_variant(args, dist: Dist):
         "repage_raise_to_widths": {"ms": up_ms, "bytes_moved": up,
                                    "GB/s": up / (up_ms / 1e3) / 1e9 if up else None},
         "clocks": clk,
-        "note": "forward pass of the variant: CUDA-core grouped GEMV from the layers",
+        "packed_ms_per_step": packed_ms / args.steps,
+        "vs_packed_step": ms / packed_ms,
+        "note": "forward pass of the variant: the streaming kernels (bulk copies into a "
+                "shared-memory ring, mma.sync) reading each chunk's stored layers, merged in "
+                "registers",
     }
     if dist.rank == 0:
         print(json.dumps(line), flush=True)

@@ -467,9 +467,12 @@ int32_t mpe_version(void);
  *   w^_b = (m / 2^b)(2 u_b + 1 - 2^b).
  * The codes are stored in layers, each in its own pages: A = u8 >> 5
  * (3 bits), B = bit 4 of u8, C = u8 & 15; a b-bit expert holds A, A B or
- * A B C. Layer streams: the rows of W1 | W3 | W2 in order, each in groups of
- * 32 codes of 3 / 1 / 4 words (code i at bits (3|1|4) i of the group's
- * little-endian string); a page holds whole groups. Lowering a width frees
+ * A B C. A layer is a chunk stream in the main format's layout at the layer's
+ * width: chunks of 16 rows x 128 codes in the expert stream's order (W1 and
+ * W3 alternating, then W2 by tile pairs), a row's codes as four quarters of
+ * 32 -- A in the 3-bit quarter layout, C in the 4-bit one, B in a 1-bit
+ * quarter (code c'_i at bit 16 (i & 1) + (i >> 1) of one word); a page holds
+ * whole chunks (256 x layer bits bytes each). Lowering a width frees
  * the dropped layers' pages and encodes nothing; raising it adds pages for
  * the new layers and encodes only those (one read of the master). Placement
  * takes the lowest free pages, experts ascending, layers A, B, C; a repage
@@ -499,14 +502,16 @@ int mpe_prefix_quantize(mpe_prefix* store, const void* const* master_f16, const 
 int mpe_prefix_repage(mpe_prefix* store, const uint8_t* new_bits, uint64_t* bytes_moved_out);
 
 /* mpe_prefix_moe_ffn -- the routed SwiGLU layer from the layered store, same
- * arguments and result layout as mpe_moe_ffn (x, ids, w, out device, x
- * 16-byte aligned, k <= 32; ids outside [0, E) contribute nothing). The
- * expert is dequantized as w^_b above. Asynchronous on the store's stream. */
+ * arguments, checks and result layout as mpe_moe_ffn (x, ids, w, out device,
+ * x and out 16-byte aligned, k <= 32, T k <= MPE_MAX_ASSIGNMENTS; ids outside
+ * [0, E) contribute nothing). The expert is dequantized as w^_b above, in
+ * registers inside the streaming path's kernels, which read the stored
+ * layers of each chunk side by side. Asynchronous on the store's stream. */
 int mpe_prefix_moe_ffn(mpe_prefix* store, const void* x_bf16, int32_t T, const int32_t* ids,
                        const float* w, int32_t k, void* out_bf16);
 
 /* mpe_prefix_read_layer -- layer (0 A, 1 B, 2 C) of expert e in stream order
- * into host_dst (uint32 words; 3 H F / 32 groups of 3 / 1 / 4 words), read
+ * into host_dst (3 H F / 2048 chunks of 768 / 256 / 1024 bytes), read
  * through the device page table. Synchronous. MPE_ERR_INVALID if the layer
  * is not stored or the buffer is short. */
 int mpe_prefix_read_layer(mpe_prefix* store, int32_t e, int32_t layer, void* host_dst,

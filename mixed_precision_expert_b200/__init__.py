@@ -394,7 +394,7 @@ class PrefixStore:
     layers A (3 bits), B (1 bit), C (4 bits); a width change drops or adds
     layers."""
 
-    LAYER_WORDS = (3, 1, 4)
+    LAYER_BITS = (3, 1, 4)
 
     def __init__(self, E: int, H: int, F: int, page_bytes: int = 0, pool_pages: int = 0,
                  device: int | None = None):
@@ -448,8 +448,9 @@ class PrefixStore:
         return out
 
     def read_layer(self, e: int, layer: int) -> np.ndarray:
-        n = 3 * self.H * self.F // 32 * self.LAYER_WORDS[layer]
-        out = np.zeros(n, dtype=np.uint32)
+        """Layer `layer` (0 A, 1 B, 2 C) of expert e: its chunk stream, uint8."""
+        n = 3 * self.H * self.F * self.LAYER_BITS[layer] // 8
+        out = np.zeros(n, dtype=np.uint8)
         self._check(lib().mpe_prefix_read_layer(self._h, e, layer, _ptr(out), out.nbytes))
         return out
 

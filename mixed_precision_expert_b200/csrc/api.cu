@@ -384,6 +384,38 @@ int run_allocate(mpe_ctx* c, const double* p, uint64_t B, std::vector<uint8_t>& 
 namespace mpe {
 // Records a message for mpe_last_error_global (context-free calls in other files).
 int report_global_error(int code, const char* msg) { return fail_global(code, "%s", msg); }
+
+int create_view(mpe_ctx** out, int device, int E, int H, int F, uint32_t page_bytes,
+                cudaStream_t stream, uint8_t* pool, Pte* d_pte, uint32_t* d_pidx,
+                uint32_t pool_pages, const uint32_t* lfirst) {
+    *out = nullptr;
+    auto* c = new mpe_ctx();
+    c->view = true;
+    c->device = device;
+    DeviceGuard guard(device);
+    c->E = E;
+    c->H = H;
+    c->F = F;
+    c->page_bytes = page_bytes;
+    c->path = MPE_PATH_DECODE;
+    c->stream = stream;
+    c->pool_pages = pool_pages;
+    c->pool = pool;
+    c->d_pte = d_pte;
+    c->d_pidx = d_pidx;
+    c->px_lfirst = lfirst;
+    c->absmax_valid = true;  // the viewed store checks its own state
+    if (cudaMalloc(&c->d_status, sizeof(uint32_t)) != cudaSuccess ||
+        cudaMemset(c->d_status, 0, sizeof(uint32_t)) != cudaSuccess) {
+        cudaGetLastError();
+        mpe_destroy(c);
+        return fail_global(MPE_ERR_CUDA, "view: device allocation failed");
+    }
+    route_set_smem_limits();
+    decode_set_smem_limits();
+    *out = c;
+    return MPE_OK;
+}
 }  // namespace mpe
 
 extern "C" {
@@ -490,6 +522,11 @@ void mpe_destroy(mpe_ctx* c) {
             cudaFreeHost(c->h_list_next_pinned);
         }
         free_scratch(c->s);
+        if (c->view) {  // the viewed store owns these
+            c->pool = nullptr;
+            c->d_pte = nullptr;
+            c->d_pidx = nullptr;
+        }
         cudaFree(c->pool); cudaFree(c->d_pte); cudaFree(c->d_pidx); cudaFree(c->d_absmax);
         cudaFree(c->d_status); cudaFree(c->d_masters); cudaFree(c->d_list); cudaFree(c->d_p);
         cudaFree(c->d_W); cudaFree(c->d_bits_out); cudaFree(c->d_alloc_status);

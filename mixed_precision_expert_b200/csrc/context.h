@@ -100,6 +100,13 @@ struct mpe_ctx {
     uint64_t fwd_epoch = ~0ull;
     uint64_t fwd_launches = 0;
 
+    // a view over another store's pages (the prefix-compatible layered store
+    // runs its forward pass through one): pool, page table and page-index
+    // array belong to that store; px_lfirst holds, per expert, the first
+    // page-index entries of its layers B and C
+    bool view = false;
+    const uint32_t* px_lfirst = nullptr;
+
     // tracing
     bool profiling = false;
     std::vector<mpe::ProfileRecord> prof;

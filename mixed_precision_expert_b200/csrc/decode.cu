@@ -120,6 +120,7 @@ struct TaskMeta {
     int j0, j_hi;  // block columns [j0, j_hi)
     float scale;   // s_e
     uint32_t first;  // the expert's first entry in the page-index array
+    uint32_t lfirst[2];  // layered store: first entries of layers B and C
     int rows[kDecodeGroup];  // activation row of each token (x row, or h row = position)
     // widths 3 and 4: off . x of each token over the task's K range, the term
     // the offset-form unpack adds to every row (written after the rest, see
@@ -143,6 +144,10 @@ struct Args {
     int direct_h;              // gate/up with P = 1: write h itself (else the partial)
     int kb;                    // blocks per part
     uint32_t* status;
+    // layered (prefix-compatible) store: per expert the first page-index
+    // entries of layers B and C (layer A's is the page table's `first`);
+    // null for the main format
+    const uint32_t* lfirst;
 };
 
 constexpr size_t kBarOff = kRingBytes;
@@ -274,17 +279,125 @@ struct UnpackRegs<8> {
     }
 };
 
+// Layered (prefix-compatible) store. Its layers are chunk streams in the
+// main format's layout: A (u8 >> 5) in the 3-bit quarter layout, B (bit 4 of
+// u8) in the 1-bit one (code pair m at bits m and 16 + m of the quarter's
+// word), C (u8 & 15) in the 4-bit one; a b-bit expert keeps A (b = 3), A B
+// (b = 4) or A B C (b = 8). The consumer's words of one row: A in w[0..2],
+// B in w[3], C in w[4..7]. A 3-bit expert is the main 3-bit format with
+// u = A (UnpackRegs<3>).
+// a >> s for s > 0, a << -s for s < 0 (s is a constant once the block loop
+// is unrolled)
+__device__ __forceinline__ uint32_t shift_by(uint32_t a, int s) {
+    return s > 0 ? (a >> s) : (s < 0 ? (a << (-s)) : a);
+}
+
+// 4 bits, u4 = 2 A + B: pair m's A field moves next to its B bit. Fields
+// 0, 2, 4 of an A word (and the spare pair) give 128 + u4 (u4 at mantissa
+// bits 0-3); fields 1 and 3 stay in place and give 32 + u4 (u4 at bits 2-5
+// under the exponent of 32).
+struct UnpackPx4 {
+    uint32_t mA1, mB0, mA3, mB2, magic, magic32;
+    __device__ __forceinline__ UnpackPx4()
+        : mA1(reg_const(0x000E000Eu)), mB0(reg_const(0x00010001u)), mA3(reg_const(0x00380038u)),
+          mB2(reg_const(0x00040004u)), magic(reg_const(kMagic)), magic32(reg_const(0x42004200u)) {}
+    __device__ __forceinline__ uint32_t pair(const uint32_t* w, int m) const {
+        const uint32_t b = w[3];
+        if (m == 15) {
+            uint32_t t = and_or(shr_imm<15>(b), mB0, magic);
+            t = and_or(shr_imm<14>(w[0]), 0x00020002u, t);
+            t = and_or(shr_imm<13>(w[1]), mB2, t);
+            return and_or(shr_imm<12>(w[2]), 0x00080008u, t);
+        }
+        const int v = m / 5, f = m % 5;
+        const uint32_t a = w[v];
+        if (f == 1) return and_or(shift_by(b, m - 2), mB2, and_or(a, mA3, magic32));
+        if (f == 3) return and_or(shift_by(b, m - 2), mB2, and_or(shr_imm<6>(a), mA3, magic32));
+        const uint32_t af = f == 0 ? (a << 1) : (f == 2 ? shr_imm<5>(a) : shr_imm<11>(a));
+        return and_or(shift_by(b, m), mB0, and_or(af, mA1, magic));
+    }
+};
+
+// 8 bits: the main 8-bit form u8 - 128 = (128 + (u8 & 127)) - (256 - 128 bit7),
+// with C at bits 0-3, B at bit 4 and A at bits 5-7 gathered from the layers.
+struct UnpackPx8 {
+    uint32_t mC, mB4, mA56, mA7, magic;
+    __device__ __forceinline__ UnpackPx8()
+        : mC(reg_const(0x000F000Fu)), mB4(reg_const(0x00100010u)), mA56(reg_const(0x00600060u)),
+          mA7(reg_const(0x00800080u)), magic(reg_const(kMagic)) {}
+    __device__ __forceinline__ uint32_t pair(const uint32_t* w, int m) const {
+        uint32_t lo = and_or(shift_by(w[4 + (m >> 2)], 4 * (m & 3)), mC, magic);
+        lo = and_or(shift_by(w[3], m - 4), mB4, lo);
+        if (m == 15) {
+            lo = and_or(shr_imm<10>(w[0]), 0x00200020u, lo);
+            lo = and_or(shr_imm<9>(w[1]), 0x00400040u, lo);
+            return bf2_sub(lo, andnot_or(shr_imm<8>(w[2]), mA7, magic));
+        }
+        const int v = m / 5, f = m % 5;
+        const uint32_t a = shift_by(w[v], 3 * f - 5);  // A at bits 5-7
+        lo = and_or(a, mA56, lo);
+        return bf2_sub(lo, andnot_or(a, mA7, magic));
+    }
+};
+
+// The unpacker of a width class.
+template <int B, bool PX>
+struct Unpacker : UnpackRegs<B> {};
+template <>
+struct Unpacker<4, true> : UnpackPx4 {};
+template <>
+struct Unpacker<8, true> : UnpackPx8 {};
+
+// Offset the unpack adds to code position c (0..31) of a quarter, which the
+// task warp's offset sums remove: main format 136 (b = 4) or 132 / 20 by pair
+// (b = 3); layered store 131.5 / 19.5 (b = 3), 135.5 / 39.5 (b = 4) by pair,
+// -0.5 (b = 8), where its value is (m / 2^b)(2 u + 1 - 2^b) = s (unpacked -
+// offset) with s = m / 4, m / 8, m / 128.
+template <int B, bool PX>
+__device__ __forceinline__ float code_offset(int c) {
+    const int m = c >> 1;
+    const bool mid = m < 15 && (m % 5 == 1 || m % 5 == 3);
+    if constexpr (!PX) {
+        if constexpr (B == 4) return 136.0f;
+        return mid ? 20.0f : 132.0f;
+    } else {
+        if constexpr (B == 8) return -0.5f;
+        if constexpr (B == 4) return mid ? 39.5f : 135.5f;
+        return mid ? 19.5f : 131.5f;
+    }
+}
+
+// Layered store: a row's words of one chunk of a consumer share. The share
+// holds each layer's chunks as one run (A, then B, then C), each run sized
+// for the slot's J block columns; `ci` is the chunk's index in its run.
+template <int B, int RUN>  // RUN: chunks per layer run of a share
+__device__ __forceinline__ void load_row_words_px(const uint8_t* share, int ci, int r, int t,
+                                                  uint32_t (&w)[Geo<B, 1, 1>::WORDS]) {
+    const uint32_t* a = reinterpret_cast<const uint32_t*>(share + ci * 768 + r * 48 + 12 * t);
+    w[0] = a[0];
+    w[1] = a[1];
+    w[2] = a[2];
+    if constexpr (B >= 4)
+        w[3] = *reinterpret_cast<const uint32_t*>(share + RUN * 768 + ci * 256 + r * 16 + 4 * t);
+    if constexpr (B == 8) {
+        const uint4 c =
+            *reinterpret_cast<const uint4*>(share + RUN * 1024 + ci * 1024 + r * 64 + 16 * t);
+        w[4] = c.x; w[5] = c.y; w[6] = c.z; w[7] = c.w;
+    }
+}
+
 // Unpack and multiply one block (128 codes of 16 rows, NM matrices, NTILE
 // tiles) with NT 8-token n-tiles of activations: every unpacked weight
 // fragment serves all n-tiles. Widths 3 and 4 unpack to the offset form
 // (k + off, see common.cuh), whose off . x term the task's offset sums remove;
 // width 8 unpacks to k. One n-tile loads the block's activations up front;
 // two load them half a block at a time (the same 16 registers).
-template <int B, int NM, int NT, int NTILE, int TPW>
-__device__ __forceinline__ void block_mma(const UnpackRegs<B>& U,
+template <int B, bool PX, int NM, int NT, int NTILE, int TPW>
+__device__ __forceinline__ void block_mma(const Unpacker<B, PX>& U,
                                           const uint32_t (&wr)[TPW][NM][2][Geo<B, 1, 1>::WORDS],
                                           const __nv_bfloat16* const (&arow)[kMaxTiles], int j,
                                           int t, float (&acc)[TPW][kMaxTiles][NM][4]) {
+    constexpr bool b8 = B == 8 && !PX;  // the main 8-bit k permutation
     constexpr int HALVES = NT == 1 ? 1 : 2;  // activation loads per block
     constexpr int CH = 8 / HALVES;           // mma steps per load
 #pragma unroll
@@ -294,8 +407,8 @@ __device__ __forceinline__ void block_mma(const UnpackRegs<B>& U,
         for (int nt = 0; nt < NT; ++nt) {
             if constexpr (HALVES == 1) {
                 uint32_t xa[8], xz[8];
-                load_act_half(arow[nt], j, t, B == 8, 0, xa);
-                load_act_half(arow[nt], j, t, B == 8, 1, xz);
+                load_act_half(arow[nt], j, t, b8, 0, xa);
+                load_act_half(arow[nt], j, t, b8, 1, xz);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     x[nt][i] = xa[i];
@@ -303,7 +416,7 @@ __device__ __forceinline__ void block_mma(const UnpackRegs<B>& U,
                 }
             } else {
                 uint32_t xh[8];
-                load_act_half(arow[nt], j, t, B == 8, h, xh);
+                load_act_half(arow[nt], j, t, b8, h, xh);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) x[nt][i] = xh[i];
             }
@@ -384,24 +497,16 @@ struct CtaSmem {
 
 __device__ __forceinline__ uint32_t next_q(uint32_t q) { return q + 1 == kTaskQ ? 0u : q + 1; }
 
-// Offset of code position c (0..31) of a quarter in the offset-form unpack
-// (common.cuh): 136 for width 4; 132 or 20 by pair for width 3.
-template <int B>
-__device__ __forceinline__ float code_offset(int c) {
-    if constexpr (B == 4) return 136.0f;
-    const int m = c >> 1;
-    return (m < 15 && (m % 5 == 1 || m % 5 == 3)) ? 20.0f : 132.0f;
-}
-
 // Task warp: claims the tasks of one width class in counter order and writes
 // each, resolved, into the next free queue entry; then one end-of-class entry.
-// For widths 3 and 4 it then adds up, per token, off(k) x[k] over the task's K
-// range in fp32 (the offset-form unpack adds off(k) to every code; the
-// consumers subtract this sum once per task) and signals tq_sum. In the down
+// For widths 3 and 4 (every width of the layered store) it then adds up, per
+// token, off(k) x[k] over the task's K range in fp32 (the offset-form unpack
+// adds off(k) to every code; the consumers subtract this sum once per task)
+// and signals tq_sum. In the down
 // kernel the activations come from the preceding kernel, so the first sum
 // waits for it (`need_wait`). `q` and the phase bits `ph` / `used` of the
 // queue's empty barriers carry over between classes.
-template <int B, bool GATEUP>
+template <int B, bool GATEUP, bool PX>
 __device__ __forceinline__ bool resolve_class(const Args& a, const CtaSmem& sm, int group0,
                                               int n_groups, int32_t* ctr, uint32_t& q,
                                               uint32_t& ph, uint32_t& used, bool& need_wait) {
@@ -447,6 +552,10 @@ __device__ __forceinline__ bool resolve_class(const Args& a, const CtaSmem& sm, 
                 m->j_hi = min(nj, p * a.kb + a.kb);
                 m->scale = __ldcg(&P.pte[e].scale);
                 m->first = __ldcg(&P.pte[e].first);
+                if constexpr (PX) {
+                    m->lfirst[0] = __ldg(a.lfirst + 2 * e);
+                    m->lfirst[1] = __ldg(a.lfirst + 2 * e + 1);
+                }
             }
         } else if (lane == 0) {
             m->valid = 0;
@@ -454,7 +563,7 @@ __device__ __forceinline__ bool resolve_class(const Args& a, const CtaSmem& sm, 
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.tq_full[q]);
         if (more) {
-            if constexpr (B != 8) {
+            if constexpr (B != 8 || PX) {
                 if (need_wait) {
                     griddep_wait();
                     need_wait = false;
@@ -465,7 +574,7 @@ __device__ __forceinline__ bool resolve_class(const Args& a, const CtaSmem& sm, 
                 static_assert(kDecodeGroup == 16, "the reduction below folds 16 sums");
                 float off[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) off[e] = code_offset<B>(8 * (lane & 3) + e);
+                for (int e = 0; e < 8; ++e) off[e] = code_offset<B, PX>(8 * (lane & 3) + e);
                 const int k_lo = 128 * m->j0, k_hi = 128 * m->j_hi, ntok = m->ntok;
                 float sum[kDecodeGroup];
 #pragma unroll
@@ -544,8 +653,10 @@ __device__ __forceinline__ bool resolve_class(const Args& a, const CtaSmem& sm, 
 // every lane prefetches one activation line. `ep` / `used` track the slots'
 // empty-barrier phases across classes, `fph` the queue's full-barrier phases.
 // In the down kernel the activations (h) come from the preceding kernel, so
-// the warp waits for it (`need_wait`) before its first prefetch.
-template <int B, bool GATEUP>
+// the warp waits for it (`need_wait`) before its first prefetch. The layered
+// store copies each layer's run of the share from that layer's pages (the
+// runs sit one after another in the share: A, B, C).
+template <int B, bool GATEUP, bool PX>
 __device__ __forceinline__ bool produce_class(const Args& a, const CtaSmem& sm, uint32_t& q,
                                               uint32_t& fph, uint32_t& ep, uint32_t& used,
                                               bool& need_wait) {
@@ -558,9 +669,19 @@ __device__ __forceinline__ bool produce_class(const Args& a, const CtaSmem& sm, 
     const int R = GATEUP ? P.F : P.H;
     const int nj = K / kCodesPerBlock, n_tiles = R / 16;
     const int nc1 = chunks_w1(P.H, P.F);
-    const int cpp = chunks_per_page(B, P.page_bytes);
-    const int n_pages = (3 * nc1 + cpp - 1) / cpp;
     constexpr int TPW = tiles_per_warp(GATEUP);
+    // layers of the class (one for the main format) and their geometry
+    constexpr int NL = PX ? (B == 3 ? 1 : (B == 4 ? 2 : 3)) : 1;
+    int lcb[NL], lcpp[NL], lnp[NL], lrun[NL];
+#pragma unroll
+    for (int L = 0; L < NL; ++L) {
+        const int lb = PX ? (L == 0 ? 3 : (L == 1 ? 1 : 4)) : B;
+        lcb[L] = 256 * lb;
+        lcpp[L] = chunks_per_page(lb, P.page_bytes);
+        lnp[L] = (3 * nc1 + lcpp[L] - 1) / lcpp[L];
+        // the run's offset in a share: the runs before it, J columns each
+        lrun[L] = L == 0 ? 0 : (L == 1 ? TPW * NM * G::J * 768 : TPW * NM * G::J * 1024);
+    }
     const int lane = threadIdx.x & 31;
     const bool copier = lane < kConsumers;  // lane w copies consumer w's share
 
@@ -586,13 +707,15 @@ __device__ __forceinline__ bool produce_class(const Args& a, const CtaSmem& sm, 
         const TaskMeta* m = sm.taskq + q;
         const int valid = m->valid;
         int tq = 0, j = 0, j_hi = 0;
-        uint32_t first = 0;
+        uint32_t first[NL];
         const __nv_bfloat16* pre_row = nullptr;  // this lane's activation row to prefetch
         if (valid) {
             tq = m->tq;
             j = m->j0;
             j_hi = m->j_hi;
-            first = m->first;
+            first[0] = m->first;
+#pragma unroll
+            for (int L = 1; L < NL; ++L) first[L] = m->lfirst[L - 1];
             if ((lane >> 1) < m->ntok) pre_row = a.act + (size_t)m->rows[lane >> 1] * K;
         }
         __syncwarp();
@@ -610,17 +733,26 @@ __device__ __forceinline__ bool produce_class(const Args& a, const CtaSmem& sm, 
         }
         const int active = min(TT, n_tiles - tq * TT);  // tiles (a multiple of TPW)
         const bool my_tile = copier && lane * TPW < active;
-        int pslot = 0, poff = 0;
-        uint32_t page = 0, page_next = 0;
+        int pslot[NL], poff[NL];
+        uint32_t page[NL], page_next[NL];
+#pragma unroll
+        for (int L = 0; L < NL; ++L) {
+            pslot[L] = poff[L] = 0;
+            page[L] = page_next[L] = 0;
+        }
         if (my_tile) {
             // the share's first chunk: gate/up interleaves W1 and W3 of a tile,
             // down the two tiles (2v, 2v+1) of the share: two chunks a column
+            // (the same index in every layer)
             const int tau = tq * TT + lane * TPW;
             const int c = GATEUP ? 2 * (tau * nj + j) : 2 * nc1 + 2 * ((tau >> 1) * nj + j);
-            pslot = c / cpp;
-            poff = c - pslot * cpp;
-            page = __ldcg(P.pidx + first + pslot);
-            if (pslot + 1 < n_pages) page_next = __ldcg(P.pidx + first + pslot + 1);
+#pragma unroll
+            for (int L = 0; L < NL; ++L) {
+                pslot[L] = c / lcpp[L];
+                poff[L] = c - pslot[L] * lcpp[L];
+                page[L] = __ldcg(P.pidx + first[L] + pslot[L]);
+                if (pslot[L] + 1 < lnp[L]) page_next[L] = __ldcg(P.pidx + first[L] + pslot[L] + 1);
+            }
         }
         const int jstart = j;
         const int pre_half = lane & 1;
@@ -636,23 +768,28 @@ __device__ __forceinline__ bool produce_class(const Args& a, const CtaSmem& sm, 
             __syncwarp();
             if (my_tile) {
                 // the share's NM x TPW x jc consecutive chunks (two a block
-                // column); a page boundary splits the copy in two
-                uint8_t* dst = sm.ring + (size_t)s * G::SLOT + (size_t)lane * TPW * G::TILEB;
+                // column) of each layer; a page boundary splits a copy in two
+                uint8_t* share = sm.ring + (size_t)s * G::SLOT + (size_t)lane * TPW * G::TILEB;
                 const int total = NM * TPW * jc;
-                const int n1 = min(total, cpp - poff);
-                bulk_g2s(dst, P.pool + (size_t)page * P.page_bytes + (size_t)poff * G::CB,
-                         (uint32_t)(n1 * G::CB), &sm.full[s]);
-                poff += n1;
-                if (poff == cpp) {
-                    ++pslot;
-                    poff = 0;
-                    page = page_next;
-                    if (pslot + 1 < n_pages) page_next = __ldcg(P.pidx + first + pslot + 1);
-                }
-                if (n1 < total) {
-                    bulk_g2s(dst + n1 * G::CB, P.pool + (size_t)page * P.page_bytes,
-                             (uint32_t)((total - n1) * G::CB), &sm.full[s]);
-                    poff = total - n1;
+#pragma unroll
+                for (int L = 0; L < NL; ++L) {
+                    uint8_t* dst = share + lrun[L];
+                    const int n1 = min(total, lcpp[L] - poff[L]);
+                    bulk_g2s(dst, P.pool + (size_t)page[L] * P.page_bytes + (size_t)poff[L] * lcb[L],
+                             (uint32_t)(n1 * lcb[L]), &sm.full[s]);
+                    poff[L] += n1;
+                    if (poff[L] == lcpp[L]) {
+                        ++pslot[L];
+                        poff[L] = 0;
+                        page[L] = page_next[L];
+                        if (pslot[L] + 1 < lnp[L])
+                            page_next[L] = __ldcg(P.pidx + first[L] + pslot[L] + 1);
+                    }
+                    if (n1 < total) {
+                        bulk_g2s(dst + n1 * lcb[L], P.pool + (size_t)page[L] * P.page_bytes,
+                                 (uint32_t)((total - n1) * lcb[L]), &sm.full[s]);
+                        poff[L] = total - n1;
+                    }
                 }
             }
             if (need_wait) {
@@ -674,7 +811,7 @@ __device__ __forceinline__ bool produce_class(const Args& a, const CtaSmem& sm, 
 // task. `fp` tracks the slots' full-barrier phases across classes, `sph` the
 // queue's offset-sum barrier phases. A warp holds its task's queue entry until
 // the task's last slot, where it reads the offset sums.
-template <int B, bool GATEUP>
+template <int B, bool GATEUP, bool PX>
 __device__ __forceinline__ bool consume_class(const Args& a, const CtaSmem& sm, uint32_t& fp,
                                               uint32_t& sph, int w) {
     constexpr int NM = GATEUP ? 2 : 1;
@@ -692,11 +829,11 @@ __device__ __forceinline__ bool consume_class(const Args& a, const CtaSmem& sm, 
     const __nv_bfloat16* arow[kMaxTiles] = {};
     int ntiles = 0;
     float acc[TPW][kMaxTiles][NM][4];
-    const UnpackRegs<B> U;
+    const Unpacker<B, PX> U;
     // widths 3, 4: acc <- acc - off . x for every tile and matrix, with the
     // task warp's per-token sums (accumulator column n = token n)
     auto settle = [&](const TaskMeta* m) {
-        if constexpr (B != 8) {
+        if constexpr (B != 8 || PX) {
             const int t = lane & 3;
 #pragma unroll
             for (int nt = 0; nt < kMaxTiles; ++nt)
@@ -736,7 +873,7 @@ __device__ __forceinline__ bool consume_class(const Args& a, const CtaSmem& sm, 
             sph ^= 1u << d.q;
             const TaskMeta* m = sm.taskq + d.q;
             if (T.valid) {
-                if constexpr (B != 8) {
+                if constexpr (B != 8 || PX) {
                     if (!mbar_wait_bounded(&sm.tq_sum[d.q], sp)) {
                         if (lane == 0) set_status(a.status, MPE_STATUS_WAIT_TIMEOUT);
                         return false;
@@ -794,9 +931,16 @@ __device__ __forceinline__ bool consume_class(const Args& a, const CtaSmem& sm, 
             for (int i = 0; i < TPW; ++i) {
 #pragma unroll
                 for (int m = 0; m < NM; ++m) {
-                    const uint8_t* chunk = tiles + ((jj * TPW + i) * NM + m) * G::CB;
-                    load_row_words<B>(chunk, g, t, g, wr[i][m][0]);
-                    load_row_words<B>(chunk, g + 8, t, g, wr[i][m][1]);
+                    const int ci = (jj * TPW + i) * NM + m;  // chunk of the share
+                    if constexpr (PX) {
+                        constexpr int RUN = TPW * NM * G::J;
+                        load_row_words_px<B, RUN>(tiles, ci, g, t, wr[i][m][0]);
+                        load_row_words_px<B, RUN>(tiles, ci, g + 8, t, wr[i][m][1]);
+                    } else {
+                        const uint8_t* chunk = tiles + ci * G::CB;
+                        load_row_words<B>(chunk, g, t, g, wr[i][m][0]);
+                        load_row_words<B>(chunk, g + 8, t, g, wr[i][m][1]);
+                    }
                 }
             }
             if (jj + 1 == d.nc) {  // the slot's last words are in registers: release it
@@ -808,17 +952,17 @@ __device__ __forceinline__ bool consume_class(const Args& a, const CtaSmem& sm, 
             // block is large, and duplicates cost instruction fetch
             if constexpr (kMaxTiles > 1) {
                 if (ntiles > 1) {
-                    block_mma<B, NM, kMaxTiles, TPW, TPW>(U, wr, arow, j, t, acc);
+                    block_mma<B, PX, NM, kMaxTiles, TPW, TPW>(U, wr, arow, j, t, acc);
                     continue;
                 }
             }
-            block_mma<B, NM, 1, TPW, TPW>(U, wr, arow, j, t, acc);
+            block_mma<B, PX, NM, 1, TPW, TPW>(U, wr, arow, j, t, acc);
         }
         if ((d.flags & kLastSlot) && !close_task()) return false;
     }
 }
 
-template <bool GATEUP>
+template <bool GATEUP, bool PX>
 __global__ void __launch_bounds__(kThreads, 1) k_decode(Args a) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -855,22 +999,22 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(Args a) {
                   n3 = __ldcg(a.n_wg_class + 2);
         uint32_t q = 0, ph = 0, used = 0;
         bool need_wait = !GATEUP;
-        if (!resolve_class<8, GATEUP>(a, sm, 0, n8, a.task_ctr + 0, q, ph, used, need_wait)) return;
-        if (!resolve_class<4, GATEUP>(a, sm, n8, n4, a.task_ctr + 1, q, ph, used, need_wait)) return;
-        resolve_class<3, GATEUP>(a, sm, n8 + n4, n3, a.task_ctr + 2, q, ph, used, need_wait);
+        if (!resolve_class<8, GATEUP, PX>(a, sm, 0, n8, a.task_ctr + 0, q, ph, used, need_wait)) return;
+        if (!resolve_class<4, GATEUP, PX>(a, sm, n8, n4, a.task_ctr + 1, q, ph, used, need_wait)) return;
+        resolve_class<3, GATEUP, PX>(a, sm, n8 + n4, n3, a.task_ctr + 2, q, ph, used, need_wait);
     } else if (warp == kCopyWarp) {
         uint32_t q = 0, fph = 0, ep = 0, used = 0;
         bool need_wait = !GATEUP;
-        if (!produce_class<8, GATEUP>(a, sm, q, fph, ep, used, need_wait)) return;
-        if (!produce_class<4, GATEUP>(a, sm, q, fph, ep, used, need_wait)) return;
-        produce_class<3, GATEUP>(a, sm, q, fph, ep, used, need_wait);
+        if (!produce_class<8, GATEUP, PX>(a, sm, q, fph, ep, used, need_wait)) return;
+        if (!produce_class<4, GATEUP, PX>(a, sm, q, fph, ep, used, need_wait)) return;
+        produce_class<3, GATEUP, PX>(a, sm, q, fph, ep, used, need_wait);
     } else {
         // down: h is written by the preceding kernel
         if (!GATEUP) griddep_wait();
         uint32_t fp = 0, sph = 0;
-        if (!consume_class<8, GATEUP>(a, sm, fp, sph, warp)) return;
-        if (!consume_class<4, GATEUP>(a, sm, fp, sph, warp)) return;
-        consume_class<3, GATEUP>(a, sm, fp, sph, warp);
+        if (!consume_class<8, GATEUP, PX>(a, sm, fp, sph, warp)) return;
+        if (!consume_class<4, GATEUP, PX>(a, sm, fp, sph, warp)) return;
+        consume_class<3, GATEUP, PX>(a, sm, fp, sph, warp);
     }
 }
 
@@ -879,9 +1023,13 @@ int g_num_sms = 0;
 }  // namespace
 
 void decode_set_smem_limits() {
-    cudaFuncSetAttribute(k_decode<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(k_decode<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)smem_bytes());
-    cudaFuncSetAttribute(k_decode<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(k_decode<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem_bytes());
+    cudaFuncSetAttribute(k_decode<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem_bytes());
+    cudaFuncSetAttribute(k_decode<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)smem_bytes());
 }
 
@@ -949,8 +1097,10 @@ void launch_decode_gateup(mpe_ctx* c, const __nv_bfloat16* x, int k, size_t Tk, 
     a.direct_h = (parts == 1 && !partials) ? 1 : 0;
     a.kb = kb;
     a.status = c->d_status;
-    const int grid = persistent_grid(c, (const void*)k_decode<true>, smem_bytes());
-    launch_pdl(k_decode<true>, dim3(grid), dim3(kThreads), smem_bytes(), c->stream, a);
+    a.lfirst = c->px_lfirst;
+    auto* fn = c->px_lfirst ? k_decode<true, true> : k_decode<true, false>;
+    const int grid = persistent_grid(c, (const void*)fn, smem_bytes());
+    launch_pdl(fn, dim3(grid), dim3(kThreads), smem_bytes(), c->stream, a);
     c->launches++;
 }
 
@@ -970,8 +1120,10 @@ void launch_decode_down(mpe_ctx* c, size_t Tk, int parts, int kb, int claim) {
     a.parts = parts;
     a.kb = kb;
     a.status = c->d_status;
-    const int grid = persistent_grid(c, (const void*)k_decode<false>, smem_bytes());
-    launch_pdl(k_decode<false>, dim3(grid), dim3(kThreads), smem_bytes(), c->stream, a);
+    a.lfirst = c->px_lfirst;
+    auto* fn = c->px_lfirst ? k_decode<false, true> : k_decode<false, false>;
+    const int grid = persistent_grid(c, (const void*)fn, smem_bytes());
+    launch_pdl(fn, dim3(grid), dim3(kThreads), smem_bytes(), c->stream, a);
     c->launches++;
 }
 

@@ -69,6 +69,14 @@ namespace mpe {
 
 PagedExperts paged(const mpe_ctx* c);
 
+// api.cu: a context over another store's pages and page table, for the
+// forward pass only (streaming path); the store keeps ownership of pool,
+// d_pte and d_pidx. lfirst: per expert the first page-index entries of the
+// layered store's layers B and C.
+int create_view(mpe_ctx** out, int device, int E, int H, int F, uint32_t page_bytes,
+                cudaStream_t stream, uint8_t* pool, Pte* d_pte, uint32_t* d_pidx,
+                uint32_t pool_pages, const uint32_t* lfirst);
+
 // Launch with programmatic stream serialization: the kernel may start while
 // the preceding kernel in the stream drains; it must call griddep_wait before
 // it reads anything that kernel writes.

@@ -25,6 +25,9 @@ Inside a quarter the 32 codes c'_0 .. c'_31 are b little-endian 32-bit words:
 * b = 3: word v (0..2) holds c'_{10v+i} at bit 16*(i&1) + 3*(i>>1), i = 0..9;
          bit n (n = 0,1,2) of c'_30 is bit 15 of word n and bit n of c'_31 is
          bit 31 of word n.
+* b = 1: word 0 holds c'_i at bit 16*(i&1) + (i>>1), i = 0..31 (not a width
+         of the main format: the one-bit layer of the prefix-compatible store,
+         oracle/prefix.py, uses it).
 In every width the pair (c'_{2m}, c'_{2m+1}) sits at the same position of the
 low and the high 16-bit half of one word (the spare pair of b = 3 excepted).
 
@@ -48,13 +51,15 @@ def chunk_bytes(b: int) -> int:
 
 
 def _shifts(b: int) -> np.ndarray:
+    if b == 1:
+        return np.array([16 * (i & 1) + (i >> 1) for i in range(32)], dtype=np.uint32)
     if b == 8:
         return np.array([16 * (i & 1) + 8 * (i >> 1) for i in range(4)], dtype=np.uint32)
     if b == 4:
         return np.array([16 * (i & 1) + 4 * (i >> 1) for i in range(8)], dtype=np.uint32)
     if b == 3:
         return np.array([16 * (i & 1) + 3 * (i >> 1) for i in range(10)], dtype=np.uint32)
-    raise ValueError(f"bit width {b} not in (3, 4, 8)")
+    raise ValueError(f"bit width {b} not in (1, 3, 4, 8)")
 
 
 def pack_quarters(u: np.ndarray, b: int) -> np.ndarray:
@@ -66,7 +71,7 @@ def pack_quarters(u: np.ndarray, b: int) -> np.ndarray:
     if np.any(u > mask):
         raise ValueError("code out of range for bit width")
     sh = _shifts(b)
-    if b in (4, 8):
+    if b in (1, 4, 8):
         per = 32 // b
         g = u.reshape(lead + (b, per))
         words = np.zeros(lead + (b,), dtype=np.uint32)
@@ -92,7 +97,7 @@ def unpack_quarters(words: np.ndarray, b: int) -> np.ndarray:
     mask = np.uint32((1 << b) - 1)
     sh = _shifts(b)
     u = np.zeros(lead + (CODES_PER_QUARTER,), dtype=np.uint32)
-    if b in (4, 8):
+    if b in (1, 4, 8):
         per = 32 // b
         for w in range(b):
             for i in range(per):

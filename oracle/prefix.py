@@ -18,18 +18,20 @@ Readings taken where the pages leave the step open:
 * Layers: A = u8 >> 5 (3 bits), B = bit 4 of u8, C = u8 & 15. A 3-bit expert
   stores A, a 4-bit one A and B, an 8-bit one A, B and C:
   u_4 = 2 u_3 + B, u_8 = 16 u_4 + C.
-* Layer streams: the expert's rows in order (W1 [F x H], W3 [F x H], W2
-  [H x F]), each row in groups of 32 codes along K; a group is 3 words (A:
-  code i at bits 3i .. 3i+2 of the 96-bit little-endian string), 1 word (B:
-  code i at bit i) or 4 words (C: code i at bits 4i .. 4i+3 of the 128-bit
-  string).
-* Pages: every layer of every expert has its own pages holding whole groups
-  (floor(P / group bytes) a page). Placement takes the lowest free pages,
-  experts ascending, layers A, B, C. A width change drops the removed layers'
-  pages (no encode at all) or adds pages for the new layers and encodes only
-  those; the changed experts release first (ascending e), then allocate
-  (ascending e); unchanged layers keep their pages; on shortage nothing
-  changes.
+* Layer streams: each layer of an expert is a chunk stream in the main
+  format's layout (oracle/layout.py) at the layer's width (A 3 bits, B 1
+  bit, C 4 bits): the layer's codes of W1, W3 [F x H] and W2 [H x F] packed
+  as layout.expert_stream packs an expert's codes, so that chunk n of every
+  layer covers the same 16 rows x 128 codes (H and F multiples of 128). The
+  pages fix no byte format; this one lets a forward pass read the layers of
+  a chunk side by side, with the main format's in-register unpack.
+* Pages: every layer of every expert has its own pages holding whole chunks
+  (floor(P / chunk bytes) a page, 256 * layer bits bytes a chunk).
+  Placement takes the lowest free pages, experts ascending, layers A, B, C.
+  A width change drops the removed layers' pages (no encode at all) or adds
+  pages for the new layers and encodes only those; the changed experts
+  release first (ascending e), then allocate (ascending e); unchanged
+  layers keep their pages; on shortage nothing changes.
 """
 from __future__ import annotations
 
@@ -38,9 +40,9 @@ import math
 
 import numpy as np
 
+from oracle import layout
+
 LAYER_BITS = {"A": 3, "B": 1, "C": 4}
-GROUP_WORDS = {"A": 3, "B": 1, "C": 4}
-GROUP_CODES = 32
 
 
 def layers_of(b: int) -> tuple[str, ...]:
@@ -79,52 +81,44 @@ def layer_values(u8: np.ndarray, layer: str) -> np.ndarray:
     return {"A": u8 >> 5, "B": (u8 >> 4) & 1, "C": u8 & 15}[layer]
 
 
-def pack_layer(vals: np.ndarray, layer: str) -> np.ndarray:
-    """Codes (one row after another, each row a multiple of 32 long) -> uint32
-    words, GROUP_WORDS[layer] per group of 32 codes."""
-    bits = LAYER_BITS[layer]
-    v = np.asarray(vals, dtype=np.uint64).reshape(-1, GROUP_CODES)
-    words = np.zeros((v.shape[0], GROUP_WORDS[layer]), dtype=np.uint64)
-    for i in range(GROUP_CODES):
-        pos = bits * i
-        wi, sh = pos // 32, pos % 32
-        words[:, wi] |= (v[:, i] << np.uint64(sh)) & np.uint64(0xFFFFFFFF)
-        if sh + bits > 32:  # the code runs into the next word
-            words[:, wi + 1] |= v[:, i] >> np.uint64(32 - sh)
-    return words.astype(np.uint32).reshape(-1)
+def _mats(flat: np.ndarray, H: int, F: int):
+    flat = np.asarray(flat)
+    return (flat[:F * H].reshape(F, H), flat[F * H:2 * F * H].reshape(F, H),
+            flat[2 * F * H:].reshape(H, F))
 
 
-def unpack_layer(words: np.ndarray, layer: str) -> np.ndarray:
-    bits = LAYER_BITS[layer]
-    w = np.asarray(words, dtype=np.uint64).reshape(-1, GROUP_WORDS[layer])
-    out = np.zeros((w.shape[0], GROUP_CODES), dtype=np.int64)
-    mask = np.uint64((1 << bits) - 1)
-    for i in range(GROUP_CODES):
-        pos = bits * i
-        wi, sh = pos // 32, pos % 32
-        v = w[:, wi] >> np.uint64(sh)
-        if sh + bits > 32:
-            v |= w[:, wi + 1] << np.uint64(32 - sh)
-        out[:, i] = (v & mask).astype(np.int64)
-    return out.reshape(-1)
+def layer_stream(u8_flat: np.ndarray, layer: str, H: int, F: int) -> np.ndarray:
+    """Layer `layer` of one expert (u8_flat: W1 | W3 | W2 row-major) as its
+    chunk stream, uint8 [n_chunks, 256 * bits]."""
+    v1, v3, v2 = _mats(layer_values(u8_flat, layer).astype(np.uint32), H, F)
+    return layout.expert_stream(v1, v3, v2, LAYER_BITS[layer])
 
 
-def layer_stream(u8_flat: np.ndarray, layer: str) -> np.ndarray:
-    """The expert's layer as uint32 words; u8_flat is W1 | W3 | W2 row-major,
-    so the rows already run in stream order."""
-    return pack_layer(layer_values(u8_flat, layer), layer)
+def layer_codes(stream: np.ndarray, layer: str, H: int, F: int) -> np.ndarray:
+    """Inverse of layer_stream: the layer's codes, W1 | W3 | W2 row-major."""
+    b = LAYER_BITS[layer]
+    cb = layout.chunk_bytes(b)
+    s = np.asarray(stream, dtype=np.uint8).reshape(-1, cb)
+    nc1 = (F // 16) * (H // 128)
+    gu = s[:2 * nc1].reshape(nc1, 2, cb)
+    u1 = layout.unpack_matrix(gu[:, 0], F, H, b)
+    u3 = layout.unpack_matrix(gu[:, 1], F, H, b)
+    nt2, nj2 = H // 16, F // 128
+    g2 = s[2 * nc1:].reshape(nt2 // 2, nj2, 2, cb).transpose(0, 2, 1, 3).reshape(-1, cb)
+    u2 = layout.unpack_matrix(g2, H, F, b)
+    return np.concatenate([u1.reshape(-1), u3.reshape(-1), u2.reshape(-1)]).astype(np.int64)
 
 
-def group_bytes(layer: str) -> int:
-    return 4 * GROUP_WORDS[layer]
+def chunk_bytes(layer: str) -> int:
+    return layout.chunk_bytes(LAYER_BITS[layer])
 
 
-def groups_per_page(layer: str, page_bytes: int) -> int:
-    return page_bytes // group_bytes(layer)
+def chunks_per_page(layer: str, page_bytes: int) -> int:
+    return page_bytes // chunk_bytes(layer)
 
 
-def layer_pages(layer: str, W_e: int, page_bytes: int) -> int:
-    return math.ceil((W_e // GROUP_CODES) / groups_per_page(layer, page_bytes))
+def layer_pages(layer: str, H: int, F: int, page_bytes: int) -> int:
+    return math.ceil(layout.n_chunks(H, F) / chunks_per_page(layer, page_bytes))
 
 
 class PoolExhausted(RuntimeError):
@@ -136,7 +130,8 @@ class LayeredPages:
     """Page bookkeeping of the layered store: pages[e][layer] lists pages."""
     n_pages: int
     E: int
-    W_e: int
+    H: int
+    F: int
     page_bytes: int
 
     def __post_init__(self):
@@ -157,7 +152,7 @@ class LayeredPages:
         pages = [dict() for _ in range(self.E)]
         for e in range(self.E):
             for L in layers_of(int(bits[e])):
-                pages[e][L] = self._take(free, layer_pages(L, self.W_e, self.page_bytes))
+                pages[e][L] = self._take(free, layer_pages(L, self.H, self.F, self.page_bytes))
         self.free, self.pages = free, pages
         self.bits = np.asarray(bits, dtype=np.uint8).copy()
         return {e: list(layers_of(int(bits[e]))) for e in range(self.E)}
@@ -178,7 +173,7 @@ class LayeredPages:
         for e in changed:  # allocate added layers, ascending e, layers in order
             added = [L for L in layers_of(int(new_bits[e])) if L not in pages[e]]
             for L in added:
-                pages[e][L] = self._take(free, layer_pages(L, self.W_e, self.page_bytes))
+                pages[e][L] = self._take(free, layer_pages(L, self.H, self.F, self.page_bytes))
             if added:
                 encode[e] = added
         self.free, self.pages = free, pages

@@ -9,7 +9,7 @@ import synth
 from oracle import ffn as of
 from oracle import prefix as ox
 
-from _helpers import check_ffn
+from _helpers import check_ffn, oracle_moe_parallel
 
 pytestmark = pytest.mark.gpu
 
@@ -26,7 +26,7 @@ def _built():
 LAYERS = ("A", "B", "C")
 
 
-def _check_layers(store, cpu, bits):
+def _check_layers(store, cpu, bits, H, F):
     m = store.absmax()
     for e, w in enumerate(cpu):
         mo, u8 = ox.prefix_codes(w)
@@ -34,7 +34,8 @@ def _check_layers(store, cpu, bits):
         n = len(ox.layers_of(int(bits[e])))
         for L in range(3):
             if L < n:
-                assert np.array_equal(store.read_layer(e, L), ox.layer_stream(u8, LAYERS[L])), (e, L)
+                want = ox.layer_stream(u8, LAYERS[L], H, F).reshape(-1)
+                assert np.array_equal(store.read_layer(e, L), want), (e, L)
             else:
                 with pytest.raises(mpe.MpeError):
                     store.read_layer(e, L)
@@ -52,19 +53,19 @@ def test_quantize_and_repage_schedule():
     E, H, F, P = 4, 256, 384, 4096
     wl, masters, cpu = _masters(E, H, F)
     W_e = 3 * H * F
-    n8 = sum(ox.layer_pages(L, W_e, P) for L in LAYERS)
+    n8 = sum(ox.layer_pages(L, H, F, P) for L in LAYERS)
     store = mpe.PrefixStore(E, H, F, page_bytes=P, pool_pages=E * n8)
-    pages = ox.LayeredPages(E * n8, E, W_e, P)
+    pages = ox.LayeredPages(E * n8, E, H, F, P)
     bits = np.array([3, 4, 8, 3], np.uint8)
     store.quantize(masters, bits)
     pages.place(bits)
-    _check_layers(store, cpu, bits)
+    _check_layers(store, cpu, bits, H, F)
     for nb in ([8, 8, 8, 8], [3, 4, 8, 3], [4, 3, 3, 8], [3, 3, 3, 3], [8, 4, 3, 4], [8, 4, 3, 4]):
         nb = np.array(nb, np.uint8)
         moved = store.repage(nb)
         enc = pages.repage(nb)
         assert moved == ox.repage_bytes(enc, W_e)
-        _check_layers(store, cpu, nb)
+        _check_layers(store, cpu, nb, H, F)
     # lowering widths only moves nothing
     assert store.repage(np.array([3, 4, 3, 3], np.uint8)) == 0
 
@@ -81,22 +82,24 @@ def test_edge_masters_and_pool():
     store = mpe.PrefixStore(E, H, F, page_bytes=4096)
     bits = np.array([8, 8, 8], np.uint8)
     store.quantize(masters, bits)
-    _check_layers(store, cpu, bits)
+    _check_layers(store, cpu, bits, H, F)
     # a pool too small for a raise leaves everything unchanged
-    W_e = 3 * H * F
-    nA = ox.layer_pages("A", W_e, 4096)
+    nA = ox.layer_pages("A", H, F, 4096)
     small = mpe.PrefixStore(E, H, F, page_bytes=4096, pool_pages=3 * nA + 1)
     small.quantize(masters, np.array([3, 3, 3], np.uint8))
     with pytest.raises(mpe.MpeError):
         small.repage(np.array([8, 3, 3], np.uint8))
-    _check_layers(small, cpu, np.array([3, 3, 3], np.uint8))
+    _check_layers(small, cpu, np.array([3, 3, 3], np.uint8), H, F)
 
 
-@pytest.mark.parametrize("bits", [(3, 3, 3, 3), (4, 4, 4, 4), (8, 8, 8, 8), (3, 4, 8, 4)])
-def test_ffn_matches_oracle(bits):
+@pytest.mark.parametrize("bits,page_bytes", [((3, 3, 3, 3), 0), ((4, 4, 4, 4), 0),
+                                             ((8, 8, 8, 8), 0), ((3, 4, 8, 4), 0),
+                                             ((8, 4, 3, 8), 4096)])
+def test_ffn_matches_oracle(bits, page_bytes):
+    # 4 KiB pages split a share's run of every layer at page boundaries
     E, H, F = 4, 256, 384
     wl, masters, cpu = _masters(E, H, F, seed=1)
-    store = mpe.PrefixStore(E, H, F)
+    store = mpe.PrefixStore(E, H, F, page_bytes=page_bytes)
     store.quantize(masters, np.array(bits, np.uint8))
     wl = synth.scaled(synth.WORKLOADS[1], E=E, H=H, F=F, T=40, k=2)
     ids, w = synth.routing(wl, seed=21)
@@ -109,8 +112,9 @@ def test_ffn_matches_oracle(bits):
     check_ffn(got.double().cpu().numpy(), ref)
 
 
-def test_ffn_full_size_sampled():
-    # the fine-grained layer at full size and its widths; 16 sampled tokens
+def test_ffn_full_size_every_token():
+    # the fine-grained layer at full size and its widths, every token; then
+    # after a width change that adds and drops layers
     wl = synth.WORKLOADS[3]
     masters = [synth.expert_weights(wl, e, device="cuda") for e in range(wl.E)]
     bits = mpe.allocate_bits(synth.importance(wl), [wl.W_e] * wl.E, wl.budget_bits)
@@ -118,15 +122,25 @@ def test_ffn_full_size_sampled():
     store.quantize(masters, bits)
     ids, w = synth.routing(wl, seed=5)
     x = synth.activations(wl, seed=5)
-    got = store.moe_ffn(x.cuda(), torch.from_numpy(ids).cuda(), torch.from_numpy(w).cuda())
-    torch.cuda.synchronize()
-    tokens = np.random.default_rng(5).choice(wl.T, 16, replace=False)
-    mats = {}
+    # device reads here, in the main thread; the oracle threads use host copies
+    cpu = {int(e): masters[int(e)].cpu().numpy() for e in np.unique(ids) if 0 <= e < wl.E}
 
-    def mats_of(e):
-        if e not in mats:
-            mats[e] = ox.expert_mats(masters[e].cpu().numpy(), wl.H, wl.F, int(bits[e]))
-        return mats[e]
+    def check(b):
+        got = store.moe_ffn(x.cuda(), torch.from_numpy(ids).cuda(), torch.from_numpy(w).cuda())
+        torch.cuda.synchronize()
+        mats = {}
 
-    ref = of.moe_ffn(x.double().numpy(), ids, w, mats_of, wl.E, tokens=tokens)
-    check_ffn(got.double().cpu().numpy()[tokens], ref)
+        def mats_of(e):
+            if e not in mats:
+                mats[e] = ox.expert_mats(cpu[e], wl.H, wl.F, int(b[e]))
+            return mats[e]
+
+        ref = oracle_moe_parallel(x, ids, w, mats_of, wl.E)
+        check_ffn(got.double().cpu().numpy(), ref)
+
+    check(bits)
+    nb = bits.copy()
+    nb[::3] = 8
+    nb[1::3] = 3
+    store.repage(nb)
+    check(nb)

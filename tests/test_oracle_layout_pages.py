@@ -49,7 +49,7 @@ def test_hand_words_b3():
     assert np.all(w.reshape(4, 3) == w[:3])
 
 
-@pytest.mark.parametrize("b", [3, 4, 8])
+@pytest.mark.parametrize("b", [1, 3, 4, 8])
 def test_quarter_roundtrip_and_size(b):
     rng = np.random.default_rng(b)
     u = rng.integers(0, 1 << b, size=(50, 32)).astype(np.uint32)

@@ -3,8 +3,9 @@ its layered page store.
 
 The grid is checked by exact rational arithmetic over every finite fp16
 weight for several absmax values (each code's bin holds its weight), by a
-hand-worked example and by its bounds; the layers by a bit-string packing
-written a different way and by round trips; the page rules by their
+hand-worked example and by its bounds; the layers by the location of every
+bit of sampled codes, recomputed with scalar index arithmetic, a hand-worked
+word and round trips; the page rules by their
 invariants (disjoint pages, dropped layers freed without encoding, unchanged
 layers kept, all-or-nothing on shortage).
 """
@@ -76,28 +77,75 @@ def test_layers_compose_the_codes():
     assert np.array_equal(2 * A + B, X.code_of_width(u8, 4))
 
 
+def _code_bits(layer, mat, r, k, H, F):
+    """(byte offset of the word, bit in the word, bit of the code) for every
+    bit of code (r, k) of matrix mat (0 = W1, 1 = W3, 2 = W2) in a layer's
+    chunk stream, by scalar index arithmetic: chunks of 16 rows x 128 codes,
+    W1 / W3 chunks alternating, then W2 with tile pairs alternating by block
+    column; a row's 128 codes as four quarters of 32."""
+    b = X.LAYER_BITS[layer]
+    K = H if mat < 2 else F
+    tau, rho = divmod(r, 16)
+    j, i = divmod(k, 128)
+    q, ip = divmod(i, 32)
+    nc1 = (F // 16) * (H // 128)
+    if mat < 2:
+        chunk = 2 * (tau * (K // 128) + j) + mat
+    else:
+        chunk = 2 * nc1 + 2 * ((tau // 2) * (K // 128) + j) + (tau % 2)
+    base = chunk * 256 * b + rho * 16 * b + q * 4 * b
+    if b == 3 and ip >= 30:
+        top = 15 if ip == 30 else 31
+        return [(base + 4 * n, top, n) for n in range(3)]
+    per = 10 if b == 3 else 32 // b
+    w, ii = divmod(ip, per)
+    pos = 16 * (ii & 1) + b * (ii >> 1)
+    return [(base + 4 * w, pos + n, n) for n in range(b)]
+
+
 @pytest.mark.parametrize("layer", ["A", "B", "C"])
-def test_layer_packing_against_bit_strings(layer):
+def test_layer_stream_element_locations(layer):
+    H, F = 256, 128
     rng = np.random.default_rng(1)
-    bits = X.LAYER_BITS[layer]
-    vals = rng.integers(0, 1 << bits, size=32 * 7)
-    words = X.pack_layer(vals, layer)
-    assert words.size == 7 * X.GROUP_WORDS[layer]
-    for g in range(7):
-        s = 0  # the group as one little-endian integer: code i at bit bits * i
-        for i in range(32):
-            s |= int(vals[32 * g + i]) << (bits * i)
-        want = [(s >> (32 * j)) & 0xFFFFFFFF for j in range(X.GROUP_WORDS[layer])]
-        assert words[g * X.GROUP_WORDS[layer]:(g + 1) * X.GROUP_WORDS[layer]].tolist() == want
-    assert np.array_equal(X.unpack_layer(words, layer), vals)
+    u8 = rng.integers(0, 256, size=3 * H * F)
+    s = X.layer_stream(u8, layer, H, F)
+    b = X.LAYER_BITS[layer]
+    assert s.shape == (3 * (F // 16) * (H // 128), 256 * b)
+    assert s.size * 8 == 3 * H * F * b
+    flat = s.reshape(-1)
+    vals = X.layer_values(u8, layer)
+    mats = [(0, F, H, 0), (1, F, H, F * H), (2, H, F, 2 * F * H)]
+    for mat, R, K, off in mats:
+        rows = rng.choice(R, size=12, replace=False)
+        for r in rows:
+            for k in range(K):
+                got = 0
+                for byte, bit, n in _code_bits(layer, mat, int(r), k, H, F):
+                    word = int.from_bytes(flat[byte:byte + 4].tobytes(), "little")
+                    got |= ((word >> bit) & 1) << n
+                assert got == vals[off + r * K + k], (layer, mat, r, k)
+    assert np.array_equal(X.layer_codes(s, layer, H, F), vals)
+
+
+def test_layer_b_hand_word():
+    # the one-bit quarter: c'_i at bit 16 (i & 1) + (i >> 1). Codes 1 at
+    # i = 0, 1, 30, 31 give bits 0, 16, 15, 31 -> 0x80018001.
+    H, F = 128, 128
+    u8 = np.zeros(3 * H * F, dtype=np.int64)
+    for i in (0, 1, 30, 31):
+        u8[i] = 16  # B = bit 4 of u8
+    s = X.layer_stream(u8, "B", H, F)
+    assert int.from_bytes(s.reshape(-1)[:4].tobytes(), "little") == 0x80018001
+    assert int(s.reshape(-1)[4:].astype(np.int64).sum()) == 0
 
 
 def test_page_rules():
-    W_e, P = 3 * 128 * 256, 4096
-    n = {L: X.layer_pages(L, W_e, P) for L in "ABC"}
-    assert n == {"A": 10, "B": 3, "C": 12}  # 3072 groups at 341 / 1024 / 256 per page
+    H, F, P = 256, 128, 4096
+    W_e = 3 * H * F
+    n = {L: X.layer_pages(L, H, F, P) for L in "ABC"}
+    assert n == {"A": 10, "B": 3, "C": 12}  # 48 chunks at 5 / 16 / 4 per page
     pool = 4 * (n["A"] + n["B"] + n["C"])
-    lp = X.LayeredPages(pool, 4, W_e, P)
+    lp = X.LayeredPages(pool, 4, H, F, P)
     enc = lp.place([8, 3, 4, 8])
     assert enc == {0: ["A", "B", "C"], 1: ["A"], 2: ["A", "B"], 3: ["A", "B", "C"]}
     before = {e: dict(lp.pages[e]) for e in range(4)}
@@ -117,7 +165,7 @@ def test_page_rules():
     assert npg.tolist() == [10, 10, 25, 13]
     # shortage: nothing changes
     snap = ([dict(p) for p in lp.pages], lp.free.copy(), lp.bits.copy())
-    lp2 = X.LayeredPages(n["A"] * 4 + n["B"], 4, W_e, P)
+    lp2 = X.LayeredPages(n["A"] * 4 + n["B"], 4, H, F, P)
     lp2.place([3, 3, 3, 3])
     with pytest.raises(X.PoolExhausted):
         lp2.repage([8, 3, 3, 3])
