@@ -292,29 +292,25 @@ __device__ __forceinline__ uint32_t shift_by(uint32_t a, int s) {
     return s > 0 ? (a >> s) : (s < 0 ? (a << (-s)) : a);
 }
 
-// 4 bits, u4 = 2 A + B: pair m's A field moves next to its B bit. Fields
-// 0, 2, 4 of an A word (and the spare pair) give 128 + u4 (u4 at mantissa
-// bits 0-3); fields 1 and 3 stay in place and give 32 + u4 (u4 at bits 2-5
-// under the exponent of 32).
+// 4 bits, u4 = 2 A + B, with half the work on the FMA pipe: A through the
+// main 3-bit unpack (128 + A, or 16 + A for fields 1 and 3), B from the
+// shifted B word at bit p = m & 3 (one shift serves four pairs) under the
+// negative magic -2^(7-p) with the bit inverted: -(2^(7-p) + 1) + B. Then
+// 2 (A value) + (B value) = const + u4 in one bf16x2 fma, exact: every const
+// + u4 here is an integer of at most 8 significant bits (127 .. 254 for the
+// 128 + A pairs, -97 .. 30 for the 16 + A ones).
 struct UnpackPx4 {
-    uint32_t mA1, mB0, mA3, mB2, magic, magic32;
+    UnpackRegs<3> a;
+    uint32_t two, n128, n64, n32, n16;
     __device__ __forceinline__ UnpackPx4()
-        : mA1(reg_const(0x000E000Eu)), mB0(reg_const(0x00010001u)), mA3(reg_const(0x00380038u)),
-          mB2(reg_const(0x00040004u)), magic(reg_const(kMagic)), magic32(reg_const(0x42004200u)) {}
+        : two(reg_const(0x40004000u)), n128(reg_const(0xC300C300u)), n64(reg_const(0xC280C280u)),
+          n32(reg_const(0xC200C200u)), n16(reg_const(0xC180C180u)) {}
     __device__ __forceinline__ uint32_t pair(const uint32_t* w, int m) const {
-        const uint32_t b = w[3];
-        if (m == 15) {
-            uint32_t t = and_or(shr_imm<15>(b), mB0, magic);
-            t = and_or(shr_imm<14>(w[0]), 0x00020002u, t);
-            t = and_or(shr_imm<13>(w[1]), mB2, t);
-            return and_or(shr_imm<12>(w[2]), 0x00080008u, t);
-        }
-        const int v = m / 5, f = m % 5;
-        const uint32_t a = w[v];
-        if (f == 1) return and_or(shift_by(b, m - 2), mB2, and_or(a, mA3, magic32));
-        if (f == 3) return and_or(shift_by(b, m - 2), mB2, and_or(shr_imm<6>(a), mA3, magic32));
-        const uint32_t af = f == 0 ? (a << 1) : (f == 2 ? shr_imm<5>(a) : shr_imm<11>(a));
-        return and_or(shift_by(b, m), mB0, and_or(af, mA1, magic));
+        const uint32_t va = a.pair(w, m);
+        const int p = m & 3;
+        const uint32_t bw = shift_by(w[3], 4 * (m >> 2));
+        const uint32_t nm = p == 0 ? n128 : (p == 1 ? n64 : (p == 2 ? n32 : n16));
+        return bf2_fma(va, two, andnot_or(bw, 0x00010001u << p, nm));
     }
 };
 
@@ -350,9 +346,10 @@ struct Unpacker<8, true> : UnpackPx8 {};
 
 // Offset the unpack adds to code position c (0..31) of a quarter, which the
 // task warp's offset sums remove: main format 136 (b = 4) or 132 / 20 by pair
-// (b = 3); layered store 131.5 / 19.5 (b = 3), 135.5 / 39.5 (b = 4) by pair,
-// -0.5 (b = 8), where its value is (m / 2^b)(2 u + 1 - 2^b) = s (unpacked -
-// offset) with s = m / 4, m / 8, m / 128.
+// (b = 3); layered store, where a weight is (m / 2^b)(2 u + 1 - 2^b) =
+// s (unpacked - offset) with s = m / 4, m / 8, m / 128: 131.5 / 19.5 by pair
+// (b = 3), const + 7.5 (b = 4; const = 2 c_A - 2^(7-p) - 1 with c_A = 128 or
+// 16 and p = pair & 3, as UnpackPx4 builds it), -0.5 (b = 8).
 template <int B, bool PX>
 __device__ __forceinline__ float code_offset(int c) {
     const int m = c >> 1;
@@ -362,7 +359,8 @@ __device__ __forceinline__ float code_offset(int c) {
         return mid ? 20.0f : 132.0f;
     } else {
         if constexpr (B == 8) return -0.5f;
-        if constexpr (B == 4) return mid ? 39.5f : 135.5f;
+        if constexpr (B == 4)
+            return 2.0f * (mid ? 16.0f : 128.0f) - (float)(128 >> (m & 3)) - 1.0f + 7.5f;
         return mid ? 19.5f : 131.5f;
     }
 }
