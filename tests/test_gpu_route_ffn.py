@@ -185,6 +185,26 @@ def test_ffn_host_graph_replay_matches_device_call(path):
     assert ctx.status() == 0
 
 
+def test_split_k_forward_is_deterministic_across_forwards():
+    # gate/up of this shape runs in two K parts (8 block columns, 3 tile
+    # groups per work group) whose partials are summed in part order:
+    # repeated forwards must give the same bits, other batches in between
+    # included, and match the oracle
+    wl = synth.scaled(synth.WORKLOADS[1], E=8, H=1024, F=512, T=16, k=2)
+    ctx, _, mats_of = _layer(wl)
+    ids, w = synth.routing(wl, seed=3)
+    x = synth.activations(wl, seed=3)
+    first = _run(ctx, x, ids, w)
+    check_ffn(first, oracle_moe(x, ids, w, mats_of, wl.E))
+    for _ in range(3):
+        assert np.array_equal(_run(ctx, x, ids, w), first)
+    ids2, w2 = synth.routing(wl, seed=4)
+    x2 = synth.activations(wl, seed=4)
+    check_ffn(_run(ctx, x2, ids2, w2), oracle_moe(x2, ids2, w2, mats_of, wl.E))
+    assert np.array_equal(_run(ctx, x, ids, w), first)
+    assert ctx.status() == 0
+
+
 def test_ffn_finegrained_decode_full_size():
     # 128 experts, hidden 2048, ffn 768, 64 tokens top-8 (Zipf-skewed), 3.5 bits average
     wl = synth.WORKLOADS[3]
