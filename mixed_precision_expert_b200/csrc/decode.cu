@@ -314,25 +314,36 @@ struct UnpackPx4 {
     }
 };
 
-// 8 bits: the main 8-bit form u8 - 128 = (128 + (u8 & 127)) - (256 - 128 bit7),
-// with C at bits 0-3, B at bit 4 and A at bits 5-7 gathered from the layers.
+// 8 bits, as two mma operands into one accumulator: hi = 16 (const + u4) from
+// layers A and B (the 4-bit form above with every magic scaled by 16, so A
+// gives 2048 + 16 A or 256 + 16 A, B gives -(2^(11-p) + 16) + 16 B, and one
+// bf16x2 fma 2 hi_A + hi_B, exact), lo = 128 + C (the main 4-bit unpack of
+// layer C). Their products summed in the accumulator are (16 const + 128 +
+// u8) x, u8 = 16 u4 + C.
 struct UnpackPx8 {
-    uint32_t mC, mB4, mA56, mA7, magic;
+    uint32_t m2048, m256, two, n2048, n1024, n512, n256, magic;
     __device__ __forceinline__ UnpackPx8()
-        : mC(reg_const(0x000F000Fu)), mB4(reg_const(0x00100010u)), mA56(reg_const(0x00600060u)),
-          mA7(reg_const(0x00800080u)), magic(reg_const(kMagic)) {}
-    __device__ __forceinline__ uint32_t pair(const uint32_t* w, int m) const {
-        uint32_t lo = and_or(shift_by(w[4 + (m >> 2)], 4 * (m & 3)), mC, magic);
-        lo = and_or(shift_by(w[3], m - 4), mB4, lo);
+        : m2048(reg_const(0x45004500u)), m256(reg_const(0x43804380u)), two(reg_const(0x40004000u)),
+          n2048(reg_const(0xC500C500u)), n1024(reg_const(0xC480C480u)),
+          n512(reg_const(0xC400C400u)), n256(reg_const(0xC380C380u)), magic(reg_const(kMagic)) {}
+    __device__ __forceinline__ uint32_t hi(const uint32_t* w, int m) const {
+        uint32_t va;
         if (m == 15) {
-            lo = and_or(shr_imm<10>(w[0]), 0x00200020u, lo);
-            lo = and_or(shr_imm<9>(w[1]), 0x00400040u, lo);
-            return bf2_sub(lo, andnot_or(shr_imm<8>(w[2]), mA7, magic));
+            va = and_or(shr_imm<15>(w[0]), 0x00010001u, m2048);
+            va = and_or(shr_imm<14>(w[1]), 0x00020002u, va);
+            va = and_or(shr_imm<13>(w[2]), 0x00040004u, va);
+        } else {
+            const int v = m / 5, f = m % 5;
+            const uint32_t x = f < 2 ? w[v] : (f < 4 ? shr_imm<6>(w[v]) : shr_imm<12>(w[v]));
+            va = (f == 1 || f == 3) ? and_or(x, 0x00380038u, m256) : and_or(x, 0x00070007u, m2048);
         }
-        const int v = m / 5, f = m % 5;
-        const uint32_t a = shift_by(w[v], 3 * f - 5);  // A at bits 5-7
-        lo = and_or(a, mA56, lo);
-        return bf2_sub(lo, andnot_or(a, mA7, magic));
+        const int p = m & 3;
+        const uint32_t nm = p == 0 ? n2048 : (p == 1 ? n1024 : (p == 2 ? n512 : n256));
+        const uint32_t vb = andnot_or(shift_by(w[3], 4 * (m >> 2)), 0x00010001u << p, nm);
+        return bf2_fma(va, two, vb);
+    }
+    __device__ __forceinline__ uint32_t lo(const uint32_t* w, int m) const {
+        return and_or(shift_by(w[4 + (m >> 2)], 4 * (m & 3)), 0x000F000Fu, magic);
     }
 };
 
@@ -349,7 +360,8 @@ struct Unpacker<8, true> : UnpackPx8 {};
 // (b = 3); layered store, where a weight is (m / 2^b)(2 u + 1 - 2^b) =
 // s (unpacked - offset) with s = m / 4, m / 8, m / 128: 131.5 / 19.5 by pair
 // (b = 3), const + 7.5 (b = 4; const = 2 c_A - 2^(7-p) - 1 with c_A = 128 or
-// 16 and p = pair & 3, as UnpackPx4 builds it), -0.5 (b = 8).
+// 16 and p = pair & 3, as UnpackPx4 builds it), 16 const + 255.5 (b = 8,
+// the same const, as UnpackPx8's two operands add up).
 template <int B, bool PX>
 __device__ __forceinline__ float code_offset(int c) {
     const int m = c >> 1;
@@ -358,9 +370,9 @@ __device__ __forceinline__ float code_offset(int c) {
         if constexpr (B == 4) return 136.0f;
         return mid ? 20.0f : 132.0f;
     } else {
-        if constexpr (B == 8) return -0.5f;
-        if constexpr (B == 4)
-            return 2.0f * (mid ? 16.0f : 128.0f) - (float)(128 >> (m & 3)) - 1.0f + 7.5f;
+        const float cst = 2.0f * (mid ? 16.0f : 128.0f) - (float)(128 >> (m & 3)) - 1.0f;
+        if constexpr (B == 8) return 16.0f * cst + 255.5f;
+        if constexpr (B == 4) return cst + 7.5f;
         return mid ? 19.5f : 131.5f;
     }
 }
@@ -426,14 +438,32 @@ __device__ __forceinline__ void block_mma(const Unpacker<B, PX>& U,
             for (int i = 0; i < NTILE; ++i)
 #pragma unroll
                 for (int m = 0; m < NM; ++m) {
-                    const uint32_t a0 = U.pair(wr[i][m][0], 2 * c);
-                    const uint32_t a1 = U.pair(wr[i][m][1], 2 * c);
-                    const uint32_t a2 = U.pair(wr[i][m][0], 2 * c + 1);
-                    const uint32_t a3 = U.pair(wr[i][m][1], 2 * c + 1);
+                    if constexpr (PX && B == 8) {  // two operands, one accumulator
+                        const uint32_t a0 = U.hi(wr[i][m][0], 2 * c);
+                        const uint32_t a1 = U.hi(wr[i][m][1], 2 * c);
+                        const uint32_t a2 = U.hi(wr[i][m][0], 2 * c + 1);
+                        const uint32_t a3 = U.hi(wr[i][m][1], 2 * c + 1);
+                        const uint32_t c0 = U.lo(wr[i][m][0], 2 * c);
+                        const uint32_t c1 = U.lo(wr[i][m][1], 2 * c);
+                        const uint32_t c2 = U.lo(wr[i][m][0], 2 * c + 1);
+                        const uint32_t c3 = U.lo(wr[i][m][1], 2 * c + 1);
 #pragma unroll
-                    for (int nt = 0; nt < NT; ++nt)
-                        mma_bf16_16816(acc[i][nt][m], a0, a1, a2, a3, x[nt][2 * cc],
-                                       x[nt][2 * cc + 1]);
+                        for (int nt = 0; nt < NT; ++nt) {
+                            mma_bf16_16816(acc[i][nt][m], a0, a1, a2, a3, x[nt][2 * cc],
+                                           x[nt][2 * cc + 1]);
+                            mma_bf16_16816(acc[i][nt][m], c0, c1, c2, c3, x[nt][2 * cc],
+                                           x[nt][2 * cc + 1]);
+                        }
+                    } else {
+                        const uint32_t a0 = U.pair(wr[i][m][0], 2 * c);
+                        const uint32_t a1 = U.pair(wr[i][m][1], 2 * c);
+                        const uint32_t a2 = U.pair(wr[i][m][0], 2 * c + 1);
+                        const uint32_t a3 = U.pair(wr[i][m][1], 2 * c + 1);
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt)
+                            mma_bf16_16816(acc[i][nt][m], a0, a1, a2, a3, x[nt][2 * cc],
+                                           x[nt][2 * cc + 1]);
+                    }
                 }
         }
     }
