@@ -41,6 +41,14 @@
 //   b = 3, 4: 32 t + 2m                      (quarter t)
 //   b = 8:    16 t + 2m (m < 8), 64 + 16 t + 2(m - 8) (m >= 8)
 // and the activation registers are loaded with the same permutation.
+//
+// The same kernels serve the prefix-compatible layered store (template flag
+// PX, prefix.cu): its layers A, B, C are chunk streams in this format's
+// layout, so the copy warp fetches one run per stored layer for each share
+// (from that layer's pages) and the consumers merge the layers' words in
+// registers (UnpackRegs<3>, UnpackPx4, UnpackPx8 below; quarter permutation
+// at every width); the per-width scale and offsets come in through the page
+// table mirror and the offset sums.
 #include <cstdlib>
 
 #include "internal.h"
