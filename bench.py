@@ -196,6 +196,26 @@ KERNEL_SOURCES = {
 }
 
 
+E2E_API = ("mpe_moe_ffn_host_async + mpe_host_wait: pinned host x, ids, w in and out back "
+           "every step, step i's result waited for after step i+1 is queued (two host buffer "
+           "sets), the last one waited for inside the timed region")
+
+
+def e2e_pipeline(ctx, hb, n: int) -> None:
+    """n host-buffer steps through the library's asynchronous entry point:
+    step i is queued, then step i-1's result is waited for (its output is in
+    host memory when the wait returns); the buffer sets hb are used in turn,
+    so a set is reused only after its previous step was waited for."""
+    prev = None
+    for i in range(n):
+        xh, ih, wh, oh = hb[i % len(hb)]
+        t = ctx.moe_ffn_host_async(xh, ih, wh, oh)
+        if prev is not None:
+            ctx.wait_host(prev)
+        prev = t
+    ctx.wait_host(prev)
+
+
 def kernel_source_hash(kernel: str) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "mixed_precision_expert_b200", "csrc")
@@ -489,7 +509,7 @@ def run_mpe(args, dist: Dist):
         # burst peak: the clocks stay at their maximum through these runs (see
         # "clocks"); the power-capped sustained figure is given for context
         peak = peaks["bf16_tflops"]
-        roofline = {"bound": "tensor", "kernel": "tensor-core gate/up (k_prefill<true>)",
+        roofline = {"bound": "tensor", "kernel": "tensor-core gate/up (k_prefill<1>)",
                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                     "frac": achieved / peak,
                     "peak_source": f"{peak_kind} bf16 dense, burst; frac of the sustained "
@@ -503,7 +523,7 @@ def run_mpe(args, dist: Dist):
         alg_gu = np.mean([gateup_bytes(batches[i % nb][3]) for i in range(args.steps)])
         achieved = alg_gu / (gu_ms / gu_n / 1e3) / 1e9
         peak = peaks["hbm_gbs"]
-        roofline = {"bound": "hbm", "kernel": "decode gate/up (k_decode<true>)",
+        roofline = {"bound": "hbm", "kernel": "decode gate/up (k_decode<1, 0>)",
                     "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                     "peak_source": peak_kind,
                     "traffic": recorded_traffic("k_decode_gateup", wl.name),
@@ -530,14 +550,13 @@ def run_mpe(args, dist: Dist):
     dist.barrier()
     torch.cuda.synchronize()
     t0 = time.perf_counter()
-    for i in range(n_e2e):
-        xh, ih, wh, oh = hb[i % len(hb)]
-        ctx.moe_ffn_host(xh, ih, wh, oh)
+    e2e_pipeline(ctx, hb, n_e2e)
     e2e_s = dist.max(time.perf_counter() - t0)
     h2d = T * H * 2 + T * k * 4 + T * k * 4
     d2h = T * H * 2
     e2e = {"value": T * n_e2e * dist.world / e2e_s, "unit": "tokens/s",
-           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e}
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e,
+           "api": E2E_API}
 
     # salient-channel compensation on the streaming path (timed apart from the
     # headline value): step time with n channels kept per row, store in device
@@ -784,7 +803,7 @@ def run_repage_schedule(args, dist: Dist):
     ctx.profile(False)
     achieved = (gu_bytes / gu_n) / (gu_ms / gu_n / 1e3) / 1e9 if gu_n else None
     traffic_ratio = recorded_traffic_ratio("k_decode_gateup", wl.name)
-    roofline = {"bound": "hbm", "kernel": "decode gate/up (k_decode<true>), every launch of "
+    roofline = {"bound": "hbm", "kernel": "decode gate/up (k_decode<1, 0>), every launch of "
                 "the schedule (3-, 4- and 8-bit pages)",
                 "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"] if achieved else None,
@@ -867,19 +886,20 @@ def run_repage_schedule(args, dist: Dist):
 
     # end to end: the last phase's batch through the host-buffer entry point
     # (pinned host x, ids, w in; out back; copies inside the timed loop)
-    xh, ih = x_l.cpu().pin_memory(), torch.from_numpy(ids_l).pin_memory()
-    wh, oh = torch.from_numpy(w_l).pin_memory(), torch.empty(T, H, dtype=torch.bfloat16).pin_memory()
+    hb = [(x_l.cpu().pin_memory(), torch.from_numpy(ids_l).pin_memory(),
+           torch.from_numpy(w_l).pin_memory(), torch.empty(T, H, dtype=torch.bfloat16).pin_memory())
+          for _ in range(2)]
     n_e2e = max(10, min(args.steps, 200))
-    for _ in range(3):
-        ctx.moe_ffn_host(xh, ih, wh, oh)
+    for i in range(3):
+        ctx.moe_ffn_host(*hb[i % 2])
     dist.barrier()
     t0 = time.perf_counter()
-    for _ in range(n_e2e):
-        ctx.moe_ffn_host(xh, ih, wh, oh)
+    e2e_pipeline(ctx, hb, n_e2e)
     e2e_s = dist.max(time.perf_counter() - t0)
     e2e = {"value": T * n_e2e * dist.world / e2e_s, "unit": "tokens/s",
            "h2d_bytes_per_step": T * H * 2 + 2 * T * k * 4, "d2h_bytes_per_step": T * H * 2,
-           "steps": n_e2e, "widths": "the schedule's final widths (6 bits average)"}
+           "steps": n_e2e, "widths": "the schedule's final widths (6 bits average)",
+           "api": E2E_API}
 
     cpu = None
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:

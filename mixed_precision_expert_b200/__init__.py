@@ -48,7 +48,7 @@ EXPORTS = [
     "mpe_get_page_table", "mpe_expert_stream_bytes", "mpe_read_expert_packed",
     "mpe_get_scales", "mpe_get_bits", "mpe_get_status", "mpe_last_error",
     "mpe_last_error_global", "mpe_kernel_launches", "mpe_version", "mpe_profile_enable",
-    "mpe_profile_read", "mpe_route_noalloc",
+    "mpe_profile_read", "mpe_route_noalloc", "mpe_moe_ffn_host_async", "mpe_host_wait",
 ]
 PROFILE_SLOTS = ["route", "gate_up", "swiglu_reduce", "down", "combine", "tc_gate_up",
                  "tc_down", "tc_permute", "select", "compensate"]
@@ -118,6 +118,8 @@ def lib() -> ctypes.CDLL:
         "mpe_repage": (i32, [vp, u64, vp, vp]),
         "mpe_moe_ffn": (i32, [vp, vp, i32, vp, vp, i32, vp]),
         "mpe_moe_ffn_host": (i32, [vp, vp, i32, vp, vp, i32, vp]),
+        "mpe_moe_ffn_host_async": (i32, [vp, vp, i32, vp, vp, i32, vp, vp]),
+        "mpe_host_wait": (i32, [vp, u64]),
         "mpe_route": (i32, [vp, vp, i32, i32, vp, vp, vp]),
         "mpe_get_page_table": (i32, [vp, vp, vp, sz]),
         "mpe_expert_stream_bytes": (sz, [vp, i32]),
@@ -329,6 +331,19 @@ class Context:
         _check(lib().mpe_moe_ffn_host(self._h, _ptr(x), T, _ptr(ids), _ptr(w), k, _ptr(out)),
                self._h)
         return out
+
+    def moe_ffn_host_async(self, x, ids, w, out) -> int:
+        """Host (pinned) buffers in, host buffer out; queued, returns a ticket.
+        The buffers belong to the library until wait_host(ticket) returns."""
+        self._sync_stream()
+        T, k = ids.shape
+        t = ctypes.c_uint64(0)
+        _check(lib().mpe_moe_ffn_host_async(self._h, _ptr(x), T, _ptr(ids), _ptr(w), k,
+                                             _ptr(out), ctypes.byref(t)), self._h)
+        return t.value
+
+    def wait_host(self, ticket: int):
+        _check(lib().mpe_host_wait(self._h, ctypes.c_uint64(ticket)), self._h)
 
     def route(self, ids):
         import torch

@@ -252,7 +252,10 @@ void free_scratch(Scratch& s) {
     cudaFree(s.perm); cudaFree(s.inv); cudaFree(s.offsets); cudaFree(s.wg); cudaFree(s.n_wg);
     cudaFree(s.hist); cudaFree(s.h); cudaFree(s.y); cudaFree(s.part); cudaFree(s.task_ctr);
     cudaFree(s.xp);
-    cudaFree(s.x_stage); cudaFree(s.ids_stage); cudaFree(s.w_stage); cudaFree(s.out_stage);
+    for (int i = 0; i < 2; ++i) {
+        cudaFree(s.x_stage[i]); cudaFree(s.ids_stage[i]); cudaFree(s.w_stage[i]);
+        cudaFree(s.out_stage[i]);
+    }
     s = Scratch{};
 }
 
@@ -264,11 +267,21 @@ int ensure_scratch(mpe_ctx* c, size_t Tk) {
     Scratch& s = c->s;
     if (Tk <= s.cap_assign && s.perm) return MPE_OK;
     CK(cudaStreamSynchronize(c->stream));
-    const size_t stage_tokens = s.stage_tokens;
-    void* xs = s.x_stage; int32_t* is = s.ids_stage; float* ws = s.w_stage; void* os = s.out_stage;
-    s.x_stage = nullptr; s.ids_stage = nullptr; s.w_stage = nullptr; s.out_stage = nullptr;
+    // the host staging survives (it is sized by ensure_stage)
+    Scratch keep;
+    keep.stage_tokens = s.stage_tokens;
+    for (int i = 0; i < 2; ++i) {
+        keep.x_stage[i] = s.x_stage[i]; keep.ids_stage[i] = s.ids_stage[i];
+        keep.w_stage[i] = s.w_stage[i]; keep.out_stage[i] = s.out_stage[i];
+        s.x_stage[i] = nullptr; s.ids_stage[i] = nullptr; s.w_stage[i] = nullptr;
+        s.out_stage[i] = nullptr;
+    }
     free_scratch(s);
-    s.stage_tokens = stage_tokens; s.x_stage = xs; s.ids_stage = is; s.w_stage = ws; s.out_stage = os;
+    s.stage_tokens = keep.stage_tokens;
+    for (int i = 0; i < 2; ++i) {
+        s.x_stage[i] = keep.x_stage[i]; s.ids_stage[i] = keep.ids_stage[i];
+        s.w_stage[i] = keep.w_stage[i]; s.out_stage[i] = keep.out_stage[i];
+    }
     size_t cap = 1024;
     while (cap < Tk) cap *= 2;
     const int E = c->E;
@@ -291,16 +304,30 @@ int ensure_scratch(mpe_ctx* c, size_t Tk) {
 
 int ensure_stage(mpe_ctx* c, int T, int k) {
     Scratch& s = c->s;
-    if ((size_t)T <= s.stage_tokens && s.x_stage && (size_t)T * k <= s.cap_assign) return MPE_OK;
+    if ((size_t)T <= s.stage_tokens && s.x_stage[0] && (size_t)T * k <= s.cap_assign) return MPE_OK;
+    // host-buffer calls still in flight use the staging
+    if (c->host_stream) CK(cudaStreamSynchronize(c->host_stream));
+    if (c->in_stream) CK(cudaStreamSynchronize(c->in_stream));
+    if (c->out_stream) CK(cudaStreamSynchronize(c->out_stream));
     CK(cudaStreamSynchronize(c->stream));
-    cudaFree(s.x_stage); cudaFree(s.ids_stage); cudaFree(s.w_stage); cudaFree(s.out_stage);
     size_t cap = 64;
     while (cap < (size_t)T) cap *= 2;
     int r;
-    if ((r = dev_alloc(c, reinterpret_cast<__nv_bfloat16**>(&s.x_stage), cap * c->H))) return r;
-    if ((r = dev_alloc(c, reinterpret_cast<__nv_bfloat16**>(&s.out_stage), cap * c->H))) return r;
-    if ((r = dev_alloc(c, &s.ids_stage, cap * 32))) return r;
-    if ((r = dev_alloc(c, &s.w_stage, cap * 32))) return r;
+    for (int i = 0; i < 2; ++i) {
+        cudaFree(s.x_stage[i]); cudaFree(s.ids_stage[i]); cudaFree(s.w_stage[i]);
+        cudaFree(s.out_stage[i]);
+        s.x_stage[i] = s.out_stage[i] = nullptr;
+        s.ids_stage[i] = nullptr;
+        s.w_stage[i] = nullptr;
+    }
+    s.stage_tokens = 0;
+    for (int i = 0; i < 2; ++i) {
+        if ((r = dev_alloc(c, reinterpret_cast<__nv_bfloat16**>(&s.x_stage[i]), cap * c->H))) return r;
+        if ((r = dev_alloc(c, reinterpret_cast<__nv_bfloat16**>(&s.out_stage[i]), cap * c->H)))
+            return r;
+        if ((r = dev_alloc(c, &s.ids_stage[i], cap * 32))) return r;
+        if ((r = dev_alloc(c, &s.w_stage[i], cap * 32))) return r;
+    }
     s.stage_tokens = cap;
     return MPE_OK;
 }
@@ -533,12 +560,23 @@ void mpe_destroy(mpe_ctx* c) {
         cudaFree(c->d_choice); cudaFree(c->d_D); cudaFree(c->d_gather);
         cudaFree(c->d_loss); cudaFree(c->d_mse_acc);
         cudaFree(c->comp_dev); cudaFree(c->sel_x); cudaFree(c->sel_h);
-        if (c->fwd_exec) cudaGraphExecDestroy(c->fwd_exec);
+        for (int i = 0; i < 2; ++i)
+            if (c->fwd_exec[i]) cudaGraphExecDestroy(c->fwd_exec[i]);
         if (c->host_stream) {
             cudaStreamSynchronize(c->host_stream);
             cudaStreamDestroy(c->host_stream);
         }
+        for (cudaStream_t st : {c->in_stream, c->out_stream})
+            if (st) {
+                cudaStreamSynchronize(st);
+                cudaStreamDestroy(st);
+            }
         if (c->host_ready) cudaEventDestroy(c->host_ready);
+        for (int i = 0; i < 2; ++i) {
+            if (c->in_done[i]) cudaEventDestroy(c->in_done[i]);
+            if (c->fwd_done[i]) cudaEventDestroy(c->fwd_done[i]);
+            if (c->out_done[i]) cudaEventDestroy(c->out_done[i]);
+        }
         if (c->comp_host) cudaFreeHost(c->comp_host);
         cudaFreeHost(c->h_pte_pinned); cudaFreeHost(c->h_pidx_pinned);
         cudaFreeHost(c->h_list_pinned); cudaFreeHost(c->h_masters_pinned);
@@ -1113,90 +1151,171 @@ int mpe_moe_ffn(mpe_ctx* c, const void* x, int32_t T, const int32_t* ids, const 
     return moe_ffn_device(c, x, T, ids, w, k, out);
 }
 
-// The host-buffer forward on c->stream (the internal stream): copies in, the
-// forward's kernels, the copy out, a synchronize. The kernels run as a CUDA
-// graph once the same (T, k) comes twice with nothing reallocated or
-// switched in between (the first call sizes every buffer, the second
-// captures, later ones replay): one launch instead of one per kernel.
-static int host_forward(mpe_ctx* c, const void* x_host, int32_t T, const int32_t* ids_host,
-                        const float* w_host, int32_t k, void* out_host) {
+// The forward's kernels of a host-buffer call on c->stream (the internal
+// stream), reading staging slot `slot`. They run as a CUDA graph (one per
+// slot) once the same (T, k) comes again with nothing reallocated or switched
+// in between (the first call of a shape sizes every buffer, the next call of
+// each slot captures, later ones replay): one launch instead of one per kernel.
+static int host_kernels(mpe_ctx* c, int slot, int32_t T, int32_t k) {
     Scratch& s = c->s;
-    const size_t xb = (size_t)T * c->H * 2;
-    CK(cudaMemcpyAsync(s.x_stage, x_host, xb, cudaMemcpyHostToDevice, c->stream));
-    CK(cudaMemcpyAsync(s.ids_stage, ids_host, (size_t)T * k * 4, cudaMemcpyHostToDevice, c->stream));
-    CK(cudaMemcpyAsync(s.w_stage, w_host, (size_t)T * k * 4, cudaMemcpyHostToDevice, c->stream));
     const bool same = c->fwd_T == T && c->fwd_k == k && c->fwd_epoch == c->epoch;
     int r = MPE_OK;
-    if (same && c->fwd_exec && !c->profiling) {
-        CK(cudaGraphLaunch(c->fwd_exec, c->stream));
+    auto plain = [&]() {
+        return moe_ffn_device(c, s.x_stage[slot], T, s.ids_stage[slot], s.w_stage[slot], k,
+                              s.out_stage[slot]);
+    };
+    if (same && c->fwd_exec[slot] && !c->profiling) {
+        CK(cudaGraphLaunch(c->fwd_exec[slot], c->stream));
         c->launches += c->fwd_launches;
     } else if (same && !c->profiling) {
         cudaGraph_t g = nullptr;
         CK(cudaStreamBeginCapture(c->stream, cudaStreamCaptureModeThreadLocal));
         const uint64_t l0 = c->launches;
-        r = moe_ffn_device(c, s.x_stage, T, s.ids_stage, s.w_stage, k, s.out_stage);
+        r = plain();
         const cudaError_t ce = cudaStreamEndCapture(c->stream, &g);
         if (r == MPE_OK && ce == cudaSuccess && c->epoch == c->fwd_epoch) {
             cudaGraphExec_t exec = nullptr;
             const cudaError_t ie = cudaGraphInstantiate(&exec, g, 0);
             cudaGraphDestroy(g);
             if (ie != cudaSuccess) return fail(c, MPE_ERR_CUDA, "graph instantiate: %s", cudaGetErrorString(ie));
-            c->fwd_exec = exec;
+            c->fwd_exec[slot] = exec;
             c->fwd_launches = c->launches - l0;
-            CK(cudaGraphLaunch(c->fwd_exec, c->stream));
+            CK(cudaGraphLaunch(c->fwd_exec[slot], c->stream));
         } else {
             if (g) cudaGraphDestroy(g);
             cudaGetLastError();
             if (r) return r;
             if (ce != cudaSuccess) return fail(c, MPE_ERR_CUDA, "graph capture: %s", cudaGetErrorString(ce));
             // something was reallocated while capturing: run it plainly
-            if ((r = moe_ffn_device(c, s.x_stage, T, s.ids_stage, s.w_stage, k, s.out_stage))) return r;
+            if ((r = plain())) return r;
         }
     } else {
-        if (c->fwd_exec) {
-            cudaGraphExecDestroy(c->fwd_exec);
-            c->fwd_exec = nullptr;
-        }
-        if ((r = moe_ffn_device(c, s.x_stage, T, s.ids_stage, s.w_stage, k, s.out_stage))) return r;
+        for (int i = 0; i < 2; ++i)
+            if (c->fwd_exec[i]) {
+                cudaGraphExecDestroy(c->fwd_exec[i]);
+                c->fwd_exec[i] = nullptr;
+            }
+        if ((r = plain())) return r;
         c->fwd_T = T;
         c->fwd_k = k;
         c->fwd_epoch = c->epoch;
     }
-    CK(cudaMemcpyAsync(out_host, s.out_stage, xb, cudaMemcpyDeviceToHost, c->stream));
-    CK(cudaStreamSynchronize(c->stream));
+    return MPE_OK;
+}
+
+// Queue one host-buffer call: inputs in on in_stream, the forward on the
+// internal stream, the output out on out_stream; returns its ticket. Three
+// streams, so that a call's inputs land while the previous call computes and
+// its output leaves while the next one does. Ordering, per staging slot: the
+// inputs land after the slot's previous forward has read them, the forward
+// waits for its inputs, for the slot's previous output copy and for the work
+// already queued on the context stream, the output copy waits for the
+// forward, and the context stream's later work waits for the forward.
+static int host_submit(mpe_ctx* c, const void* x_host, int32_t T, const int32_t* ids_host,
+                       const float* w_host, int32_t k, void* out_host, uint64_t* ticket) {
+    Scratch& s = c->s;
+    const int slot = (int)(c->host_seq & 1u);
+    const size_t xb = (size_t)T * c->H * 2;
+    CK(cudaStreamWaitEvent(c->in_stream, c->fwd_done[slot], 0));
+    CK(cudaMemcpyAsync(s.x_stage[slot], x_host, xb, cudaMemcpyHostToDevice, c->in_stream));
+    CK(cudaMemcpyAsync(s.ids_stage[slot], ids_host, (size_t)T * k * 4, cudaMemcpyHostToDevice,
+                       c->in_stream));
+    CK(cudaMemcpyAsync(s.w_stage[slot], w_host, (size_t)T * k * 4, cudaMemcpyHostToDevice,
+                       c->in_stream));
+    CK(cudaEventRecord(c->in_done[slot], c->in_stream));
+    CK(cudaEventRecord(c->host_ready, c->stream));
+    CK(cudaStreamWaitEvent(c->host_stream, c->host_ready, 0));
+    CK(cudaStreamWaitEvent(c->host_stream, c->in_done[slot], 0));
+    CK(cudaStreamWaitEvent(c->host_stream, c->out_done[slot], 0));
+    const cudaStream_t user = c->stream;
+    c->stream = c->host_stream;
+    const int r = host_kernels(c, slot, T, k);
+    c->stream = user;
+    if (r) return r;
+    CK(cudaEventRecord(c->fwd_done[slot], c->host_stream));
+    CK(cudaStreamWaitEvent(c->stream, c->fwd_done[slot], 0));
+    CK(cudaStreamWaitEvent(c->out_stream, c->fwd_done[slot], 0));
+    CK(cudaMemcpyAsync(out_host, s.out_stage[slot], xb, cudaMemcpyDeviceToHost, c->out_stream));
+    CK(cudaEventRecord(c->out_done[slot], c->out_stream));
+    *ticket = c->host_seq++;
+    return MPE_OK;
+}
+
+static int host_call_checks(mpe_ctx* c, int32_t T, int32_t k, const void* x_host,
+                            const int32_t* ids_host, const float* w_host, void* out_host) {
+    if (T < 0 || k < 1 || k > 32) return fail(c, MPE_ERR_INVALID, "bad T=%d or k=%d", T, k);
+    if ((long long)T * k > MPE_MAX_ASSIGNMENTS)
+        return fail(c, MPE_ERR_INVALID, "T*k = %lld exceeds %d", (long long)T * k,
+                    MPE_MAX_ASSIGNMENTS);
+    if (T > 0 && (!x_host || !ids_host || !w_host || !out_host))
+        return fail(c, MPE_ERR_INVALID, "null argument");
+    if (!c->absmax_valid) return fail(c, MPE_ERR_ORDER, "moe_ffn before quantize_experts");
+    if (c->comp_n > 0 && c->path == MPE_PATH_PREFILL)
+        return fail(c, MPE_ERR_INVALID, "compensation runs on the streaming path only");
+    return MPE_OK;
+}
+
+static int host_setup(mpe_ctx* c, int32_t T, int32_t k) {
+    int r;
+    if ((r = ensure_scratch(c, (size_t)T * k))) return r;
+    if ((r = ensure_stage(c, T, k))) return r;
+    if (!c->host_stream) {
+        CK(cudaStreamCreateWithFlags(&c->host_stream, cudaStreamNonBlocking));
+        CK(cudaStreamCreateWithFlags(&c->in_stream, cudaStreamNonBlocking));
+        CK(cudaStreamCreateWithFlags(&c->out_stream, cudaStreamNonBlocking));
+        CK(cudaEventCreateWithFlags(&c->host_ready, cudaEventDisableTiming));
+        for (int i = 0; i < 2; ++i) {
+            CK(cudaEventCreateWithFlags(&c->in_done[i], cudaEventDisableTiming));
+            CK(cudaEventCreateWithFlags(&c->fwd_done[i], cudaEventDisableTiming));
+            CK(cudaEventCreateWithFlags(&c->out_done[i], cudaEventDisableTiming));
+        }
+    }
+    return MPE_OK;
+}
+
+static int host_wait(mpe_ctx* c, uint64_t ticket) {
+    if (ticket >= c->host_seq) return fail(c, MPE_ERR_INVALID, "ticket %llu not issued",
+                                           (unsigned long long)ticket);
+    // the slot's latest output copy is this call's or a later one's (the
+    // output stream runs them in order)
+    CK(cudaEventSynchronize(c->out_done[ticket & 1u]));
     return MPE_OK;
 }
 
 int mpe_moe_ffn_host(mpe_ctx* c, const void* x_host, int32_t T, const int32_t* ids_host,
                      const float* w_host, int32_t k, void* out_host) {
     if (!c) return fail_global(MPE_ERR_INVALID, "null context");
-    if (T < 0 || k < 1 || k > 32) return fail(c, MPE_ERR_INVALID, "bad T=%d or k=%d", T, k);
-    if (T == 0) return MPE_OK;
-    if ((long long)T * k > MPE_MAX_ASSIGNMENTS)
-        return fail(c, MPE_ERR_INVALID, "T*k = %lld exceeds %d", (long long)T * k,
-                    MPE_MAX_ASSIGNMENTS);
-    if (!x_host || !ids_host || !w_host || !out_host) return fail(c, MPE_ERR_INVALID, "null argument");
-    if (!c->absmax_valid) return fail(c, MPE_ERR_ORDER, "moe_ffn before quantize_experts");
-    DeviceGuard guard(c->device);
-    if (c->comp_n > 0 && c->path == MPE_PATH_PREFILL)
-        return fail(c, MPE_ERR_INVALID, "compensation runs on the streaming path only");
     int r;
-    if ((r = ensure_scratch(c, (size_t)T * k))) return r;
-    if ((r = ensure_stage(c, T, k))) return r;
-    if (!c->host_stream) {
-        CK(cudaStreamCreateWithFlags(&c->host_stream, cudaStreamNonBlocking));
-        CK(cudaEventCreateWithFlags(&c->host_ready, cudaEventDisableTiming));
+    if ((r = host_call_checks(c, T, k, x_host, ids_host, w_host, out_host))) return r;
+    if (T == 0) return MPE_OK;
+    DeviceGuard guard(c->device);
+    if ((r = host_setup(c, T, k))) return r;
+    // the call is synchronous: queued like an asynchronous one, then waited for
+    uint64_t t = 0;
+    if ((r = host_submit(c, x_host, T, ids_host, w_host, k, out_host, &t))) return r;
+    return host_wait(c, t);
+}
+
+int mpe_moe_ffn_host_async(mpe_ctx* c, const void* x_host, int32_t T, const int32_t* ids_host,
+                           const float* w_host, int32_t k, void* out_host, uint64_t* ticket) {
+    if (!c) return fail_global(MPE_ERR_INVALID, "null context");
+    if (!ticket) return fail(c, MPE_ERR_INVALID, "null ticket");
+    int r;
+    if ((r = host_call_checks(c, T, k, x_host, ids_host, w_host, out_host))) return r;
+    DeviceGuard guard(c->device);
+    if (T == 0) {  // nothing to queue, nothing to wait for
+        *ticket = UINT64_MAX;
+        return MPE_OK;
     }
-    // the call is synchronous: it runs on the internal stream (which can be
-    // captured, unlike the legacy default stream) after the work queued on
-    // the context stream, and is finished when it returns
-    CK(cudaEventRecord(c->host_ready, c->stream));
-    CK(cudaStreamWaitEvent(c->host_stream, c->host_ready, 0));
-    const cudaStream_t user = c->stream;
-    c->stream = c->host_stream;
-    r = host_forward(c, x_host, T, ids_host, w_host, k, out_host);
-    c->stream = user;
-    return r;
+    if ((r = host_setup(c, T, k))) return r;
+    return host_submit(c, x_host, T, ids_host, w_host, k, out_host, ticket);
+}
+
+int mpe_host_wait(mpe_ctx* c, uint64_t ticket) {
+    if (!c) return fail_global(MPE_ERR_INVALID, "null context");
+    if (ticket == UINT64_MAX) return MPE_OK;
+    DeviceGuard guard(c->device);
+    return host_wait(c, ticket);
 }
 
 int mpe_route(mpe_ctx* c, const int32_t* ids, int32_t T, int32_t k, int32_t* perm,

@@ -88,14 +88,24 @@ struct mpe_ctx {
     bool pending = false;
     std::vector<uint32_t> pending_release;  // old pages of the changed experts
 
-    // the host-buffer forward replays a CUDA graph of its kernels on an
-    // internal stream once the same (T, k) repeats; `epoch` counts changes
-    // that invalidate a captured graph (any device reallocation, a table
-    // swap, a new path or compensation setting)
+    // the host-buffer forward replays a CUDA graph of its kernels (one per
+    // staging slot) on an internal stream once the same (T, k) repeats;
+    // `epoch` counts changes that invalidate a captured graph (any device
+    // reallocation, a table swap, a new path or compensation setting). The
+    // copies in run on in_stream, the copies out on out_stream; per slot,
+    // in_done / fwd_done / out_done mark the last call's inputs landed,
+    // forward finished and output copied; host_seq counts the calls
+    // submitted (tickets).
     uint64_t epoch = 0;
     cudaStream_t host_stream = nullptr;
+    cudaStream_t in_stream = nullptr;
+    cudaStream_t out_stream = nullptr;
     cudaEvent_t host_ready = nullptr;
-    cudaGraphExec_t fwd_exec = nullptr;
+    cudaEvent_t in_done[2] = {nullptr, nullptr};
+    cudaEvent_t fwd_done[2] = {nullptr, nullptr};
+    cudaEvent_t out_done[2] = {nullptr, nullptr};
+    uint64_t host_seq = 0;
+    cudaGraphExec_t fwd_exec[2] = {nullptr, nullptr};
     int fwd_T = 0, fwd_k = 0;
     uint64_t fwd_epoch = ~0ull;
     uint64_t fwd_launches = 0;

@@ -38,12 +38,13 @@ struct Scratch {
     int32_t* task_ctr = nullptr; // 6 task counters (3 classes x 2 kernels), zeroed by route
     __nv_bfloat16* xp = nullptr; // routed tokens in route-position order [xp_cap x H] (tensor-core path)
     size_t xp_cap = 0;           // elements
-    // staging for the host-buffer entry point
+    // staging for the host-buffer entry points: two slots, so that one
+    // call's copies overlap the neighbouring call's forward pass
     size_t stage_tokens = 0;
-    void* x_stage = nullptr;
-    int32_t* ids_stage = nullptr;
-    float* w_stage = nullptr;
-    void* out_stage = nullptr;
+    void* x_stage[2] = {nullptr, nullptr};
+    int32_t* ids_stage[2] = {nullptr, nullptr};
+    float* w_stage[2] = {nullptr, nullptr};
+    void* out_stage[2] = {nullptr, nullptr};
 };
 
 // CUDA-event records around the forward-pass kernels (optional tracing).

@@ -205,6 +205,70 @@ def test_split_k_forward_is_deterministic_across_forwards():
     assert ctx.status() == 0
 
 
+@pytest.mark.parametrize("path", [1, 2])
+def test_ffn_host_async_pipeline_matches_device_call(path):
+    # queued host-buffer calls (two staging slots taken in turn, copies on
+    # their own stream) give, call by call, the device-pointer call's bits:
+    # five calls in flight before the first wait, a shape change, and a
+    # repage queued on the context stream between two queued calls
+    wl = synth.scaled(synth.WORKLOADS[3], E=16, T=48, k=4)
+    ctx, _, _ = _layer(wl, path=path)
+    p = synth.importance(wl)
+    calls = []
+    for step in range(9):
+        T = wl.T if step != 6 else 20
+        w2 = synth.scaled(wl, T=T)
+        ids, w = synth.routing(w2, seed=80 + step)
+        x = synth.activations(w2, seed=80 + step)
+        calls.append((x, ids, w))
+    hostbuf = []
+    for x, ids, w in calls:
+        hostbuf.append((x.pin_memory(), torch.from_numpy(ids).pin_memory(),
+                        torch.from_numpy(w).pin_memory(),
+                        torch.empty(x.shape, dtype=torch.bfloat16).pin_memory()))
+    tickets = []
+    for i in range(5):
+        xh, ih, wh, oh = hostbuf[i]
+        tickets.append(ctx.moe_ffn_host_async(xh, ih, wh, oh))
+    assert tickets == sorted(tickets) and len(set(tickets)) == 5
+    for t in tickets:
+        ctx.wait_host(t)
+    want = [_run(ctx, *c) for c in calls[:5]]
+    for i in range(5):
+        assert np.array_equal(hostbuf[i][3].double().numpy(), want[i]), i
+    # a repage between queued calls: the call queued after it sees the new widths
+    t5 = ctx.moe_ffn_host_async(*hostbuf[5])
+    ctx.repage(synth.budget_for(wl, 3.2), p)
+    t6 = ctx.moe_ffn_host_async(*hostbuf[6])
+    t7 = ctx.moe_ffn_host_async(*hostbuf[7])
+    t8 = ctx.moe_ffn_host_async(*hostbuf[8])
+    for t in (t5, t6, t7, t8):
+        ctx.wait_host(t)
+    for i in (6, 7, 8):
+        assert np.array_equal(hostbuf[i][3].double().numpy(), _run(ctx, *calls[i])), i
+    assert ctx.status() == 0
+
+
+def test_ffn_host_async_tickets():
+    wl = synth.scaled(synth.WORKLOADS[1], E=4, H=256, F=256, T=8, k=2)
+    ctx, _, _ = _layer(wl)
+    ids, w = synth.routing(wl)
+    x = synth.activations(wl)
+    with pytest.raises(mpe.MpeError):
+        ctx.wait_host(0)  # nothing issued yet
+    buf = (x.pin_memory(), torch.from_numpy(ids).pin_memory(), torch.from_numpy(w).pin_memory(),
+           torch.empty(x.shape, dtype=torch.bfloat16).pin_memory())
+    t = ctx.moe_ffn_host_async(*buf)
+    with pytest.raises(mpe.MpeError):
+        ctx.wait_host(t + 1)
+    ctx.wait_host(t)
+    ctx.wait_host(t)  # waiting again is harmless
+    empty = (buf[0][:0], buf[1][:0], buf[2][:0], buf[3][:0])
+    assert ctx.moe_ffn_host_async(*empty) == 2**64 - 1
+    ctx.wait_host(2**64 - 1)
+    assert np.array_equal(buf[3].double().numpy(), _run(ctx, x, ids, w))
+
+
 def test_ffn_finegrained_decode_full_size():
     # 128 experts, hidden 2048, ffn 768, 64 tokens top-8 (Zipf-skewed), 3.5 bits average
     wl = synth.WORKLOADS[3]
