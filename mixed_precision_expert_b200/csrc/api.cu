@@ -97,6 +97,26 @@ uint32_t next_free(const std::vector<uint8_t>& free, uint32_t from, uint32_t poo
     return hit ? (uint32_t)(static_cast<const uint8_t*>(hit) - free.data()) : pool_pages;
 }
 
+// `need` lowest free pages from `cursor` on, taken in runs (freed pages come
+// back as long runs): marks them used, writes them to `out` and advances the
+// cursor; false if the pool runs out (the map is a plan's copy: nothing is
+// committed then).
+bool take_lowest(std::vector<uint8_t>& free, uint32_t& cursor, uint32_t pool_pages, int need,
+                 std::vector<uint32_t>& out) {
+    out.resize((size_t)need);
+    uint8_t* f = free.data();
+    int got = 0;
+    while (got < need) {
+        cursor = next_free(free, cursor, pool_pages);
+        if (cursor >= pool_pages) return false;
+        while (got < need && cursor < pool_pages && f[cursor]) {
+            f[cursor] = 0;
+            out[(size_t)got++] = cursor++;
+        }
+    }
+    return true;
+}
+
 bool plan_pages(const mpe_ctx* c, const std::vector<uint8_t>& new_bits, PagePlan& plan,
                 std::vector<int>& changed) {
     changed.clear();
@@ -110,13 +130,7 @@ bool plan_pages(const mpe_ctx* c, const std::vector<uint8_t>& new_bits, PagePlan
     for (int e : changed) {
         const int need = pages_needed(new_bits[e], c->H, c->F, c->page_bytes);
         std::vector<uint32_t> pg;
-        pg.reserve(need);
-        for (int i = 0; i < need; ++i) {
-            cursor = next_free(plan.free, cursor, c->pool_pages);
-            if (cursor >= c->pool_pages) return false;
-            plan.free[cursor] = 0;
-            pg.push_back(cursor);
-        }
+        if (!take_lowest(plan.free, cursor, c->pool_pages, need, pg)) return false;
         plan.moved.emplace_back(e, std::move(pg));
     }
     return true;
@@ -145,13 +159,7 @@ bool plan_pages_overlapped(const mpe_ctx* c, const std::vector<uint8_t>& new_bit
     for (int e : changed) {
         const int need = pages_needed(new_bits[e], c->H, c->F, c->page_bytes);
         std::vector<uint32_t> pg;
-        pg.reserve(need);
-        for (int i = 0; i < need; ++i) {
-            cursor = next_free(plan.free, cursor, c->pool_pages);
-            if (cursor >= c->pool_pages) return false;
-            plan.free[cursor] = 0;
-            pg.push_back(cursor);
-        }
+        if (!take_lowest(plan.free, cursor, c->pool_pages, need, pg)) return false;
         release.insert(release.end(), c->alloc.pages[e].begin(), c->alloc.pages[e].end());
         plan.moved.emplace_back(e, std::move(pg));
     }
