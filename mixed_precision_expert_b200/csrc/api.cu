@@ -547,6 +547,9 @@ void mpe_destroy(mpe_ctx* c) {
     {
         DeviceGuard guard(c->device);
         cudaStreamSynchronize(c->stream);
+        // host-buffer calls still queued read and write the staging
+        for (cudaStream_t st : {c->host_stream, c->in_stream, c->out_stream})
+            if (st) cudaStreamSynchronize(st);
         if (c->side) {
             cudaStreamSynchronize(c->side);
             cudaStreamDestroy(c->side);
@@ -1198,11 +1201,15 @@ static int host_kernels(mpe_ctx* c, int slot, int32_t T, int32_t k) {
             if ((r = plain())) return r;
         }
     } else {
-        for (int i = 0; i < 2; ++i)
-            if (c->fwd_exec[i]) {
-                cudaGraphExecDestroy(c->fwd_exec[i]);
-                c->fwd_exec[i] = nullptr;
-            }
+        if (c->fwd_exec[0] || c->fwd_exec[1]) {
+            // a queued call may still be running one of them
+            CK(cudaStreamSynchronize(c->host_stream));
+            for (int i = 0; i < 2; ++i)
+                if (c->fwd_exec[i]) {
+                    cudaGraphExecDestroy(c->fwd_exec[i]);
+                    c->fwd_exec[i] = nullptr;
+                }
+        }
         if ((r = plain())) return r;
         c->fwd_T = T;
         c->fwd_k = k;
