@@ -265,8 +265,13 @@ int mpe_select_salient(const void* rows_bf16, int32_t n_rows, int32_t n_cols, in
  * changed, give
  * them new pages and re-encode only those experts from the fp16 master with
  * the cached absmax. *n_changed_out (host, may be NULL) receives the count.
- * Synchronises once (the new widths decide the page moves); the encode is
- * asynchronous. MPE_ERR_POOL leaves widths, pages and codes unchanged.
+ * The width rule runs on a context-internal stream of the highest priority,
+ * beside the work already queued on the context stream (it reads only p and
+ * the expert sizes), and the call waits for it (the new widths decide the
+ * page moves); the page-table upload, the scales and the encode are queued
+ * on the context stream after the work already there, and the call returns
+ * without waiting for them. MPE_ERR_POOL leaves widths, pages and codes
+ * unchanged.
  */
 int mpe_repage(mpe_ctx* ctx, uint64_t B_bits, const double* p, int32_t* n_changed_out);
 

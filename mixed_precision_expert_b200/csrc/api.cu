@@ -577,7 +577,7 @@ void mpe_destroy(mpe_ctx* c) {
             cudaStreamSynchronize(c->host_stream);
             cudaStreamDestroy(c->host_stream);
         }
-        for (cudaStream_t st : {c->in_stream, c->out_stream})
+        for (cudaStream_t st : {c->in_stream, c->out_stream, c->alloc_stream})
             if (st) {
                 cudaStreamSynchronize(st);
                 cudaStreamDestroy(st);
@@ -886,7 +886,16 @@ int mpe_repage(mpe_ctx* c, uint64_t B_bits, const double* p, int32_t* n_changed_
     std::vector<uint8_t> nb;
     int r;
     if ((r = commit_pending(c))) return r;
-    if ((r = run_allocate(c, p, B_bits, nb, c->stream))) return r;
+    if (!c->alloc_stream) {
+        int least = 0, greatest = 0;
+        CK(cudaDeviceGetStreamPriorityRange(&least, &greatest));
+        CK(cudaStreamCreateWithPriority(&c->alloc_stream, cudaStreamNonBlocking, greatest));
+    }
+    // the widths: solved beside the work already queued on the context stream
+    // (the solve reads only the importances and sizes), so the host plans the
+    // page moves while that work runs; the moves and the encode are queued on
+    // the context stream behind it
+    if ((r = run_allocate(c, p, B_bits, nb, c->alloc_stream))) return r;
     if (nb == c->bits) {  // no width changes: the pages, table and scales stand
         if (n_changed_out) *n_changed_out = 0;
         return MPE_OK;

@@ -72,6 +72,11 @@ struct mpe_ctx {
     mpe::HostAllocator alloc;
     mpe::Scratch s;
 
+    // the width rule of a synchronous repage runs here, at the highest
+    // priority, beside the work already queued on `stream` (it reads only the
+    // importances and sizes); the page moves and the encode stay on `stream`
+    cudaStream_t alloc_stream = nullptr;
+
     // overlapped repage (mpe_repage_async / mpe_repage_commit): the next page
     // table is prepared and the changed experts encoded on `side` while work
     // on `stream` keeps reading the current table
