@@ -931,7 +931,12 @@ def run_repage_schedule(args, dist: Dist):
                      "passes": "absmax read + encode read/write of the 22.5 GB master"},
         "repage_total": {"ms": rp_ms, "GB/s": rp_bytes / (rp_ms / 1e3) / 1e9 if rp_ms else None,
                          "frac": rp_bytes / (rp_ms / 1e3) / 1e9 / peaks["hbm_gbs"] if rp_ms else None,
-                         "bytes": rp_bytes},
+                         "bytes": rp_bytes,
+                         "timing": "CUDA events on the context stream around each mpe_repage call: "
+                                   "the page-table upload, scales and encode of the changed experts; "
+                                   "the width solve runs beside the decode steps queued before it "
+                                   "(high-priority internal stream), its cost lands in the decode "
+                                   "and schedule figures"},
         "repage": repages,
         "decode": decode,
         "repage_overlap": overlap,
