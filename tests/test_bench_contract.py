@@ -31,3 +31,47 @@ def test_reference_arm_json_line():
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"]
     assert cb["quantize"]["GB/s"] > 0  # the oracle's quantizer on a bounded sample
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
+
+
+class _RecordingContext:
+    """Stands in for mpe.Context: records the order of queued calls and waits
+    and checks that a buffer set is never queued again before its previous
+    call was waited for."""
+
+    def __init__(self):
+        self.log = []
+        self.pending = {}   # buffer set id -> ticket not yet waited for
+        self.next = 0
+
+    def moe_ffn_host_async(self, xh, ih, wh, oh):
+        key = id(oh)
+        assert key not in self.pending, "buffer set reused while its call is in flight"
+        t = self.next
+        self.next += 1
+        self.pending[key] = t
+        self.log.append(("queue", t, key))
+        return t
+
+    def wait_host(self, t):
+        self.log.append(("wait", t))
+        for k, v in list(self.pending.items()):
+            if v <= t:
+                del self.pending[k]
+
+
+def test_e2e_pipeline_queues_ahead_and_waits_every_step():
+    sys.path.insert(0, ROOT)
+    import bench
+    ctx = _RecordingContext()
+    sets = [tuple(object() for _ in range(4)) for _ in range(2)]
+    bench.e2e_pipeline(ctx, sets, 7)
+    queues = [e for e in ctx.log if e[0] == "queue"]
+    waits = [e[1] for e in ctx.log if e[0] == "wait"]
+    assert [q[1] for q in queues] == list(range(7))
+    assert waits == list(range(7))  # every step's result is read back, in order
+    # step i is queued before step i - 1 is waited for (one call in flight ahead)
+    for i in range(1, 7):
+        assert ctx.log.index(("queue", i, queues[i][2])) < ctx.log.index(("wait", i - 1))
+    # the two buffer sets alternate
+    assert [q[2] for q in queues] == [id(sets[i % 2][3]) for i in range(7)]
+    assert not ctx.pending
