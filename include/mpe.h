@@ -347,14 +347,13 @@ int mpe_moe_ffn_host(mpe_ctx* ctx, const void* x_host, int32_t T, const int32_t*
  * The copies in and the copies out run on two context-internal streams and
  * the layer on the internal compute stream, through two device staging slots
  * taken in turn, so one call's copies overlap the neighbouring calls' layers.
- * Any number of
- * calls may be queued; each waits on the device for whatever it must not
- * overtake (its slot's previous call, the work already queued on the context
- * stream), and later work on the context stream waits for it. The call's host
- * buffers are the library's until mpe_host_wait(ticket) returns: x_host,
- * ids_host and w_host must stay unchanged and out_host unread until then
- * (pinned memory, or the copies are synchronous). T = 0 queues nothing and
- * returns the ticket UINT64_MAX. Errors as for mpe_moe_ffn_host.
+ * Any number of calls may be queued; each waits on the device for whatever it
+ * must not overtake (its slot's previous call, the work already queued on the
+ * context stream), and later work on the context stream waits for it. The
+ * call's host buffers are the library's until mpe_host_wait(ticket) returns:
+ * x_host, ids_host and w_host must stay unchanged and out_host unread until
+ * then (pinned memory, or the copies are synchronous). T = 0 queues nothing
+ * and returns the ticket UINT64_MAX. Errors as for mpe_moe_ffn_host.
  */
 int mpe_moe_ffn_host_async(mpe_ctx* ctx, const void* x_host, int32_t T, const int32_t* ids_host,
                            const float* w_host, int32_t k, void* out_host, uint64_t* ticket);
