@@ -19,6 +19,12 @@ one forward pass over a fresh batch with the pages resident.
 ffn 768, 8192 tokens top-8, 3.5 bits average), which runs on the tensor-core
 path; its roofline is the gate/up kernel's bf16 FLOP rate.
 
+--width B / --experts E / --tokens T / --topk k time one layer of the
+workload's shape instead (with --workload 5: one decode layer, not the
+schedule): every expert at B bits rather than the allocator's widths, and/or
+another expert count, batch or top-k -- the decode rate by width, or a case
+small enough for a multi-pass profiler capture. The line names the layer.
+
 The value comes from a timed region without per-kernel events; the kernel
 durations behind the roofline come from a second pass over the same batches
 with CUDA events around each kernel on the context stream.
@@ -62,7 +68,22 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--variant", choices=["packed", "prefix"], default="packed",
                     help="prefix: the layered prefix-compatible store on a decode workload")
+    ap.add_argument("--width", type=int, choices=[3, 4, 8], default=None,
+                    help="every expert at this width instead of the allocator's widths: one "
+                         "layer of the workload's shape (with --workload 5, one decode layer "
+                         "instead of the repaging schedule)")
+    ap.add_argument("--experts", type=int, default=None,
+                    help="one layer with this many experts (a smaller case of the same shape)")
+    ap.add_argument("--tokens", type=int, default=None, help="one layer, tokens per step")
+    ap.add_argument("--topk", type=int, default=None, help="one layer, experts per token")
     args = ap.parse_args()
+    layer_flags = (args.width, args.experts, args.tokens, args.topk)
+    if args.variant == "prefix" and any(v is not None for v in layer_flags):
+        ap.error("--width/--experts/--tokens/--topk time the packed format's layer")
+    E = args.experts
+    if (E is not None and E < 1) or (args.tokens is not None and args.tokens < 1) or \
+            (args.topk is not None and not 1 <= args.topk <= 32):
+        ap.error("need --experts >= 1, --tokens >= 1 and --topk in 1..32")
     if args.steps is None:
         args.steps = {4: 400, 5: 200}.get(args.workload, 2000)
     # at least 3 untimed warm-up steps whatever is asked (the JSON line
@@ -262,14 +283,47 @@ def recorded_traffic(kernel: str, workload: str) -> float | None:
 PREFILL_MIN_AVG = 32  # the library's automatic path rule: tensor cores when T*k >= 32 E
 
 
-def bench_config(wl) -> dict:
+def bench_workload(workload: int, experts=None, tokens=None, topk=None, width=None):
+    """The workload the flags name: one of the five, or one layer of its shape
+    with another expert count, batch or top-k, or with every expert at one
+    width (named after the workload it comes from, its sizes and the width)."""
+    import synth
+    wl = synth.WORKLOADS[workload]
+    ch = {n: v for n, v in (("E", experts), ("T", tokens), ("k", topk)) if v is not None}
+    if not ch and width is None:
+        return wl
+    E, T, k = ch.get("E", wl.E), ch.get("T", wl.T), ch.get("k", wl.k)
+    if k > E:
+        raise ValueError(f"top-{k} routing over {E} experts")
+    name = f"{wl.name.split('-')[0]}-layer-e{E}-h{wl.H}-f{wl.F}-t{T}-top{k}"
+    if width is not None:
+        name += f"-w{width}"
+    return synth.scaled(wl, name=name, **ch)
+
+
+def args_workload(args):
+    return bench_workload(args.workload, args.experts, args.tokens, args.topk, args.width)
+
+
+def is_schedule(wl) -> bool:
+    """The repaging schedule itself (not one layer of its shape)."""
+    return wl.cfg == 5 and wl.name.startswith("repage-e")
+
+
+def bench_config(wl, width=None) -> dict:
     """The workload as both arms print it: static, so the two lines carry the
     same dict (measured values go in keys of their own)."""
     path = "tensor-core" if wl.T * wl.k >= PREFILL_MIN_AVG * wl.E else "streaming"
     cfg = {"workload": wl.name, "E": wl.E, "H": wl.H, "F": wl.F, "tokens_per_step": wl.T,
-           "top_k": wl.k, "avg_bits_budget": wl.avg_bits, "page_bytes": 65536,
-           "parallelism": "replicas", "path": path}
-    if wl.cfg == 5:
+           "top_k": wl.k, "avg_bits_budget": None if width else wl.avg_bits,
+           "page_bytes": 65536, "parallelism": "replicas", "path": path}
+    if width:
+        cfg["width"] = width
+    if "-layer-" in wl.name:
+        pages_mb = wl.sum_W * (width or wl.avg_bits) / 8 / 1e6
+        cfg["l2"] = (f"no flush: the layer's packed pages total {pages_mb:.0f} MB (a step "
+                     f"reads those of its active experts; L2 holds 126 MB)")
+    elif is_schedule(wl):
         cfg["schedule"] = ("quantize at 8 bits average, then 10 phases: decode steps of 128 "
                            "tokens, then a budget change (repage) to 7, 6, 5, 4, 3, 3.75, 4.5, "
                            "5.25, 6, 6 bits average")
@@ -300,6 +354,15 @@ def cores_used() -> int:
     return len(os.sched_getaffinity(0))
 
 
+def oracle_widths(wl, width=None) -> np.ndarray:
+    """The oracle's widths for the workload: its allocator's, or one width for all."""
+    import synth
+    from oracle import allocate as oa
+    if width:
+        return np.full(wl.E, width, dtype=np.uint8)
+    return oa.allocate_bits(synth.importance(wl), [wl.W_e] * wl.E, wl.budget_bits)
+
+
 class OracleSample:
     """Bounded sample of the oracle's forward work: one token through one expert,
     in slices of rows of F (SwiGLU separates over F, so the slices of all F rows
@@ -307,12 +370,11 @@ class OracleSample:
     of the expert (the resident pages) happen once, untimed; each slice
     dequantizes its rows and runs the float64 SwiGLU."""
 
-    def __init__(self, wl, e: int = 0, token: int = 0):
+    def __init__(self, wl, e: int = 0, token: int = 0, width=None):
         import synth
-        from oracle import allocate as oa
         from oracle import quantize as oq
         self.wl = wl
-        bits = oa.allocate_bits(synth.importance(wl), [wl.W_e] * wl.E, wl.budget_bits)
+        bits = oracle_widths(wl, width)
         master = synth.expert_weights(wl, e).numpy()
         self.m, self.s, k = oq.quantize_expert(master, int(bits[e]))
         H, F = wl.H, wl.F
@@ -337,16 +399,14 @@ class OracleSample:
         return time.perf_counter() - t0, n_slices * slice_rows / F / self.wl.k
 
 
-def oracle_quantize_rate(wl, n_weights: int = 1 << 21) -> dict:
+def oracle_quantize_rate(wl, n_weights: int = 1 << 21, width=None) -> dict:
     """The oracle's quantizer on a bounded sample (the first n_weights fp16
-    weights of expert 0 at its allocated width): absmax, scale, codes, offset
-    codes. Rate in the quantize pass's bytes: 4 per weight (two reads of the
-    master) + b / 8 written."""
+    weights of expert 0 at its width): absmax, scale, codes, offset codes.
+    Rate in the quantize pass's bytes: 4 per weight (two reads of the master)
+    + b / 8 written."""
     import synth
-    from oracle import allocate as oa
     from oracle import quantize as oq
-    bits = oa.allocate_bits(synth.importance(wl), [wl.W_e] * wl.E, wl.budget_bits)
-    b = int(bits[0])
+    b = int(oracle_widths(wl, width)[0])
     n = min(n_weights, wl.W_e)
     master = synth.expert_weights(wl, 0, count=n).numpy()
     t0 = time.perf_counter()
@@ -364,9 +424,9 @@ def run_reference(args, dist: Dist):
     import synth
     if dist.rank != 0:
         return
-    wl = synth.WORKLOADS[args.workload]
+    wl = args_workload(args)
     slice_rows = 128
-    sample = OracleSample(wl)
+    sample = OracleSample(wl, width=args.width)
     # warm-up and timed steps: each step = one 128-row F-slice of one token-slot
     sample.run(max(1, args.warmup), slice_rows)
     dt, frac = sample.run(args.steps, slice_rows)
@@ -376,13 +436,13 @@ def run_reference(args, dist: Dist):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": bench_config(wl),
+        "config": bench_config(wl, args.width),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores_used(),
                          "kind": "oracle",
                          "sample": f"each step: one {slice_rows}-row slice of ffn for one token "
                                    f"through one expert (dequantize + SwiGLU, float64); "
                                    f"{args.steps} steps = {frac:.4f} tokens of layer work",
-                         "quantize": oracle_quantize_rate(wl)},
+                         "quantize": oracle_quantize_rate(wl, width=args.width)},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -404,7 +464,7 @@ def run_mpe(args, dist: Dist):
 
     dev = dist.local_rank
     torch.cuda.set_device(dev)
-    wl = synth.WORKLOADS[args.workload]
+    wl = args_workload(args)
     E, H, F, T, k = wl.E, wl.H, wl.F, wl.T, wl.k
 
     # resident state: fp16 masters -> bit allocation -> quantized pages
@@ -413,8 +473,10 @@ def run_mpe(args, dist: Dist):
         t = torch.empty(wl.W_e, dtype=torch.float16, device="cuda")
         synth.fill_expert_weights(wl, e, t)
         masters.append(t)
-    p = synth.importance(wl)
-    bits = mpe.allocate_bits(p, [wl.W_e] * E, wl.budget_bits)
+    if args.width:
+        bits = np.full(E, args.width, dtype=np.uint8)
+    else:
+        bits = mpe.allocate_bits(synth.importance(wl), [wl.W_e] * E, wl.budget_bits)
     ctx = mpe.Context(E, H, F)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     q_ms = []
@@ -595,11 +657,11 @@ def run_mpe(args, dist: Dist):
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         slice_rows = 128
         n_slices = max(1, F // slice_rows)
-        dt, frac = OracleSample(wl).run(n_slices, slice_rows)
+        dt, frac = OracleSample(wl, width=args.width).run(n_slices, slice_rows)
         cpu = {"value": frac / dt, "unit": "tokens/s", "cores": cores_used(), "kind": "oracle",
                "sample": f"one token through one expert (all {F} ffn rows in {n_slices} slices; "
                          f"dequantize + SwiGLU in float64) = {frac:.3f} tokens of layer work",
-               "quantize": oracle_quantize_rate(wl)}
+               "quantize": oracle_quantize_rate(wl, width=args.width)}
 
     qms = float(np.median(q_ms))
     line = {
@@ -607,7 +669,7 @@ def run_mpe(args, dist: Dist):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": bench_config(wl),
+        "config": bench_config(wl, args.width),
         "bits_hist": bits_hist(bits),
         "path_taken": "tensor-core" if prof["tc_gate_up"][1] else "streaming",
         "packed_bytes_per_step": alg_layer,
@@ -1067,7 +1129,7 @@ def main():
     try:
         if args.variant == "prefix":
             run_prefix_variant(args, dist)
-        elif args.workload == 5:
+        elif is_schedule(args_workload(args)):
             run_repage_schedule(args, dist)
         else:
             run_mpe(args, dist)

@@ -75,3 +75,32 @@ def test_e2e_pipeline_queues_ahead_and_waits_every_step():
     # the two buffer sets alternate
     assert [q[2] for q in queues] == [id(sets[i % 2][3]) for i in range(7)]
     assert not ctx.pending
+
+
+def test_reference_arm_one_layer_at_one_width():
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--workload", "1", "--width", "8", "--experts", "4", "--tokens", "8",
+                        "--topk", "2", "--steps", "1", "--warmup", "3"],
+                       capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    d = json.loads([l for l in r.stdout.splitlines() if l.startswith("{")][0])
+    sys.path.insert(0, ROOT)
+    import bench
+    wl = bench.bench_workload(1, experts=4, tokens=8, topk=2, width=8)
+    assert (wl.E, wl.T, wl.k, wl.H, wl.F) == (4, 8, 2, 256, 512)
+    assert d["config"] == bench.bench_config(wl, 8)
+    assert d["config"]["workload"] == "tiny-layer-e4-h256-f512-t8-top2-w8"
+    assert d["config"]["width"] == 8 and d["config"]["avg_bits_budget"] is None
+    assert d["cpu_baseline"]["quantize"]["sample"].endswith("at 8 bits")
+    # a layer of the repaging workload's shape is not the schedule
+    assert not bench.is_schedule(bench.bench_workload(5, width=3))
+    assert bench.is_schedule(bench.bench_workload(5))
+    assert bench.bench_workload(2) is bench.bench_workload(2, None, None, None, None)
+
+
+def test_layer_flags_are_checked():
+    for extra in (["--variant", "prefix", "--width", "3"], ["--topk", "0"], ["--experts", "0"]):
+        r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl",
+                            "reference", "--workload", "1", "--steps", "1"] + extra,
+                           capture_output=True, text=True, timeout=120, cwd=ROOT)
+        assert r.returncode == 2 and "error" in r.stderr, extra
