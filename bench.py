@@ -24,6 +24,7 @@ workload's shape instead (with --workload 5: one decode layer, not the
 schedule): every expert at B bits rather than the allocator's widths, and/or
 another expert count, batch or top-k -- the decode rate by width, or a case
 small enough for a multi-pass profiler capture. The line names the layer.
+--path decode|prefill forces one contraction path on a one-layer run.
 
 The value comes from a timed region without per-kernel events; the kernel
 durations behind the roofline come from a second pass over the same batches
@@ -76,10 +77,15 @@ def parse_args():
                     help="one layer with this many experts (a smaller case of the same shape)")
     ap.add_argument("--tokens", type=int, default=None, help="one layer, tokens per step")
     ap.add_argument("--topk", type=int, default=None, help="one layer, experts per token")
+    ap.add_argument("--path", choices=["auto", "decode", "prefill"], default="auto",
+                    help="contraction path of a one-layer run (auto: the library's rule)")
     args = ap.parse_args()
     layer_flags = (args.width, args.experts, args.tokens, args.topk)
     if args.variant == "prefix" and any(v is not None for v in layer_flags):
         ap.error("--width/--experts/--tokens/--topk time the packed format's layer")
+    if args.path != "auto" and (args.variant == "prefix" or (
+            args.workload == 5 and all(v is None for v in layer_flags))):
+        ap.error("--path applies to one layer (not the schedule or the prefix variant)")
     E = args.experts
     if (E is not None and E < 1) or (args.tokens is not None and args.tokens < 1) or \
             (args.topk is not None and not 1 <= args.topk <= 32):
@@ -310,10 +316,12 @@ def is_schedule(wl) -> bool:
     return wl.cfg == 5 and wl.name.startswith("repage-e")
 
 
-def bench_config(wl, width=None) -> dict:
+def bench_config(wl, width=None, path_flag: str = "auto") -> dict:
     """The workload as both arms print it: static, so the two lines carry the
     same dict (measured values go in keys of their own)."""
     path = "tensor-core" if wl.T * wl.k >= PREFILL_MIN_AVG * wl.E else "streaming"
+    if path_flag != "auto":
+        path = {"decode": "streaming", "prefill": "tensor-core"}[path_flag]
     cfg = {"workload": wl.name, "E": wl.E, "H": wl.H, "F": wl.F, "tokens_per_step": wl.T,
            "top_k": wl.k, "avg_bits_budget": None if width else wl.avg_bits,
            "page_bytes": 65536, "parallelism": "replicas", "path": path}
@@ -331,7 +339,7 @@ def bench_config(wl, width=None) -> dict:
                      "and each repage the changed experts' masters, far above the 126 MB L2")
     elif wl.cfg == 1:
         cfg["l2"] = "no flush: a correctness-size layer (1.8 MB of pages) that fits in L2"
-    elif path == "tensor-core":
+    elif wl.cfg == 4:
         cfg["l2"] = ("no flush: each step reads the packed pages of every expert (264 MB) and "
                      "the routed tokens (256 MB), above the 126 MB L2")
     else:
@@ -436,7 +444,7 @@ def run_reference(args, dist: Dist):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": bench_config(wl, args.width),
+        "config": bench_config(wl, args.width, args.path),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores_used(),
                          "kind": "oracle",
                          "sample": f"each step: one {slice_rows}-row slice of ffn for one token "
@@ -477,7 +485,8 @@ def run_mpe(args, dist: Dist):
         bits = np.full(E, args.width, dtype=np.uint8)
     else:
         bits = mpe.allocate_bits(synth.importance(wl), [wl.W_e] * E, wl.budget_bits)
-    ctx = mpe.Context(E, H, F)
+    ctx = mpe.Context(E, H, F, path={"auto": mpe.PATH_AUTO, "decode": mpe.PATH_DECODE,
+                                     "prefill": mpe.PATH_PREFILL}[args.path])
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     q_ms = []
     for _ in range(3):
@@ -669,7 +678,7 @@ def run_mpe(args, dist: Dist):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": bench_config(wl, args.width),
+        "config": bench_config(wl, args.width, args.path),
         "bits_hist": bits_hist(bits),
         "path_taken": "tensor-core" if prof["tc_gate_up"][1] else "streaming",
         "packed_bytes_per_step": alg_layer,

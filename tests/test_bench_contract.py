@@ -104,3 +104,19 @@ def test_layer_flags_are_checked():
                             "reference", "--workload", "1", "--steps", "1"] + extra,
                            capture_output=True, text=True, timeout=120, cwd=ROOT)
         assert r.returncode == 2 and "error" in r.stderr, extra
+
+
+def test_forced_path_is_in_the_config_and_limited_to_one_layer():
+    sys.path.insert(0, ROOT)
+    import bench
+    import synth
+    wl = synth.WORKLOADS[3]
+    assert bench.bench_config(wl)["path"] == "streaming"
+    assert bench.bench_config(wl, path_flag="prefill")["path"] == "tensor-core"
+    assert bench.bench_config(synth.WORKLOADS[4], path_flag="decode")["path"] == "streaming"
+    # the L2 note follows the workload, not the forced path
+    assert "264 MB" not in bench.bench_config(wl, path_flag="prefill")["l2"]
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--workload", "5", "--path", "prefill", "--steps", "1"],
+                       capture_output=True, text=True, timeout=120, cwd=ROOT)
+    assert r.returncode == 2 and "--path applies to one layer" in r.stderr
