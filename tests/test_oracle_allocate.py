@@ -109,6 +109,19 @@ def test_zero_importance_gets_lowest_width():
     assert list(bits) == [3, 8]
 
 
+def test_equal_experts_tie_in_expert_order():
+    # Two experts with equal p and W: giving the upgrade to either costs the
+    # same (p L(4) + p L(3) = p L(3) + p L(4) exactly, the sum commutes). The
+    # program tries 3, 4, 8 in that order and replaces its best only on a
+    # strictly smaller cost, so the later expert keeps the lower width and the
+    # earlier one takes the upgrade. Budget units of W = 10 bits: one unit
+    # buys 3 -> 4, five buy 3 -> 8.
+    W = [10, 10]
+    assert list(A.allocate_bits([0.5, 0.5], W, 3 * 20 + 10)) == [4, 3]
+    # six units: 8 + 4 either way (L(8) + L(4) beats 4 + 4 and 8 + 3)
+    assert list(A.allocate_bits([0.5, 0.5], W, 3 * 20 + 60)) == [8, 4]
+
+
 @pytest.mark.parametrize("seed", range(6))
 def test_exchange_property_equal_W(seed):
     # for equal W_e, swapping widths between i and j keeps the budget; an optimum

@@ -119,7 +119,8 @@ def test_expert_stream_order():
     assert np.all(s[0:2 * third:2] == 0x11) and np.all(s[1:2 * third:2] == 0x22)
     assert np.all(s[2 * third:] == 0x33)
     # distinct codes per matrix row: chunk 2c is W1's chunk c, 2c+1 is W3's
-    H, F = 256, 128
+    # (F = 256: W2 has two block columns, so its column interleave shows)
+    H, F = 256, 256
     rng = np.random.default_rng(1)
     u1 = rng.integers(0, 16, size=(F, H)).astype(np.uint32)
     u3 = rng.integers(0, 16, size=(F, H)).astype(np.uint32)

@@ -105,7 +105,7 @@ def _code_bits(layer, mat, r, k, H, F):
 
 @pytest.mark.parametrize("layer", ["A", "B", "C"])
 def test_layer_stream_element_locations(layer):
-    H, F = 256, 128
+    H, F = 256, 256  # W2 with two block columns
     rng = np.random.default_rng(1)
     u8 = rng.integers(0, 256, size=3 * H * F)
     s = X.layer_stream(u8, layer, H, F)
