@@ -35,6 +35,23 @@ def test_allocate_bits_small(seed):
     assert np.array_equal(got, ref)
 
 
+@pytest.mark.parametrize("E,units", [(2, 1), (2, 6), (5, 3), (8, 13)])
+def test_allocate_bits_ties_follow_expert_order(E, units):
+    # equal importances and sizes: an upgrade costs the same whichever expert
+    # takes it, up to the rounding of the running sums, so the tie rule
+    # (widths tried 3, 4, 8, replaced only on a strictly smaller cost; the
+    # budget argmin ties to the smallest state) and the order of the float64
+    # additions decide; `units` of 128 bits buy 3 -> 4 (one) or 3 -> 8 (five)
+    W = [128] * E
+    p = np.full(E, 1.0 / E)
+    B = 3 * sum(W) + units * 128
+    got = mpe.allocate_bits(p, W, B)
+    ref = oa.allocate_bits(p, W, B, state_cap=mpe.ALLOC_STATE_CAP)
+    assert np.array_equal(got, ref)
+    if (E, units) == (2, 1):
+        assert list(got) == [4, 3]
+
+
 @pytest.mark.parametrize("cfg,avg", [(1, 4.5), (2, 4.5), (3, 3.5), (5, 8.0), (5, 6.0), (5, 3.0),
                                      (5, 3.75), (5, 5.25), (3, 3.0), (3, 7.99)])
 def test_allocate_bits_workloads(cfg, avg):
